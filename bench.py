@@ -1,0 +1,419 @@
+#!/usr/bin/env python
+"""Benchmark of the routed NVFP4 MoE site on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode_t1]
+
+One step = one routed MoE site forward (router logits, sigmoid top-k, routing
+plan, expert gate/up + clamped SwiGLU, expert down x routing weight, BF16
+shared expert, combine) over one batch of synthetic inputs already resident in
+HBM, replayed from a CUDA graph of the public moe_forward call. L2 is flushed
+(a 2x-L2 buffer is rewritten) before every timed step; each step is timed
+with CUDA events on the launching stream; the reported time is the max over
+ranks. The expert-GEMV roofline comes from stage events recorded by the
+library inside the same graph.
+
+`e2e` measures the same metric through moe_forward with host buffers: pinned
+host->device copy of x, the forward, device->host copy of y, all inside the
+events.
+
+Multi-GPU: the site does not shard here (replicas only): every rank runs its
+own independent replica, value = all ranks' tokens / max-over-ranks time.
+
+--impl reference times the CPU oracle (the deliberately plain fp64 restatement)
+on the host cores for the same workload and prints the same JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s (decode) with expert-GEMV HBM GB/s vs roofline"
+PER_EXPERT_NOTE = "gate+up+down codes, E4M3 scales and tensor scales of each touched expert"
+
+
+def nvfp4_bank_bytes(rows: int, cols: int) -> int:
+    return rows * cols // 2 + rows * cols // 16 + 4
+
+
+def expert_bytes(wl) -> int:
+    return 2 * nvfp4_bank_bytes(wl.I, wl.H) + nvfp4_bank_bytes(wl.H, wl.I)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm_gbs=d["hbm_gbs"], bf16_tflops=d["bf16_tflops"],
+                    bf16_tflops_sustained=d.get("bf16_tflops_sustained"), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-lms", "100", "-i", str(self.idx)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [v.strip() for v in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ ours
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    from routed_nvfp4_expert_b200 import capi
+    from routed_nvfp4_expert_b200 import synthetic as syn
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = syn.WORKLOADS[args.workload]
+    inp = syn.make_site(wl, seed=0)
+    site = capi.site_to_device(inp, dev)
+    cfg = capi.config_for(wl)
+    path = capi.PATH_DECODE if wl.kind == "decode" else capi.PATH_PREFILL
+    T, H = wl.T, wl.H
+
+    # rotating activations: a different routing every step (seeded per rank)
+    n_x = 16
+    x_pool = torch.stack([capi.bf16_tensor(syn.random_x(wl, T, seed=1000 * rank + i), dev) for i in range(n_x)])
+    x = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    ws = capi.alloc_workspace(cfg, T, path, dev)
+    views = capi.moe_workspace_views(cfg, T, path, ws)
+    ids_view = capi.view_tensor(views.ids, (T, wl.k), torch.int32, dev)
+
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2 + (64 << 20), dtype=torch.uint8, device=dev)
+
+    stream = torch.cuda.Stream(dev)
+    nst = len(capi.STAGES) + 1
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(nst)]
+    outer = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    with torch.cuda.stream(stream):
+        for e in ev + outer:
+            e.record(stream)               # creates the CUDA events
+    stream.synchronize()
+    w_c = site.c()
+    i_gu, i_sh = capi.STAGES.index("expert_gate_up"), capi.STAGES.index("shared")
+
+    # warm the kernels once outside capture, then capture the forward into graphs:
+    #   timed: stage events only around the expert GEMVs (2 event nodes)
+    #   plain: no stage events;  stages: every stage boundary (diagnostic)
+    x.copy_(x_pool[0])
+    with torch.cuda.stream(stream):
+        capi.moe_forward(cfg, site, x, path, y, ws, stream=stream, w_c=w_c)
+    stream.synchronize()
+    capi.moe_read_device_status(ws, stream)
+
+    def capture(events):
+        g = torch.cuda.CUDAGraph()
+        capi.moe_set_stage_events(events)
+        try:
+            with torch.cuda.graph(g, stream=stream):
+                capi.moe_forward(cfg, site, x, path, y, ws, stream=stream, w_c=w_c)
+        finally:
+            capi.moe_set_stage_events(None)
+        return g
+
+    sparse = [None] * nst
+    sparse[i_gu], sparse[i_sh] = ev[i_gu], ev[i_sh]
+    g_timed = capture(sparse)
+    g_plain = capture(None)
+    g_stages = capture(ev)
+
+    def one_step(g, i, with_stages=False):
+        with torch.cuda.stream(stream):
+            flush.fill_(i & 0xFF)
+            x.copy_(x_pool[i % n_x])
+            outer[0].record(stream)
+            g.replay()
+            outer[1].record(stream)
+        stream.synchronize()
+        step = outer[0].elapsed_time(outer[1])
+        if with_stages == "all":
+            return step, [ev[s].elapsed_time(ev[s + 1]) for s in range(nst - 1)]
+        if with_stages:
+            return step, ev[i_gu].elapsed_time(ev[i_sh])
+        return step, None
+
+    for i in range(args.warmup):
+        one_step(g_timed, i, True)
+    capi.moe_read_device_status(ws, stream)
+
+    dist_barrier(world)
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    step_ms, gemv_ms_l, uniq = [], [], []
+    for i in range(args.steps):
+        ms, gm = one_step(g_timed, args.warmup + i, True)
+        step_ms.append(ms)
+        gemv_ms_l.append(gm)
+        uniq.append(int(torch.unique(ids_view).numel()))
+    torch.cuda.synchronize(dev)
+    dist_barrier(world)
+    clk = clocks.stop()
+    capi.moe_read_device_status(ws, stream)
+
+    # diagnostics (outside the timed region): no stage events; every stage
+    plain_ms = float(np.mean([one_step(g_plain, i)[0] for i in range(args.steps)]))
+    stage_ms = [one_step(g_stages, i, "all")[1] for i in range(args.steps)]
+
+    # e2e: the public call with host buffers (pinned), copies inside the events
+    xh = torch.empty((T, H), dtype=torch.bfloat16, pin_memory=True)
+    yh = torch.empty((T, H), dtype=torch.bfloat16, pin_memory=True)
+    xh_pool = [x_pool[i].cpu() for i in range(n_x)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_ms = []
+    for i in range(args.warmup + args.steps):
+        xh.copy_(xh_pool[i % n_x])
+        with torch.cuda.stream(stream):
+            flush.fill_(i & 0xFF)
+            e0.record(stream)
+            x.copy_(xh, non_blocking=True)
+            capi.moe_forward(cfg, site, x, path, y, ws, stream=stream, w_c=w_c)
+            yh.copy_(y, non_blocking=True)
+            e1.record(stream)
+        stream.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(e0.elapsed_time(e1))
+
+    ms = float(np.mean(step_ms))
+    stage_avg = np.mean(np.array(stage_ms), axis=0)
+    gemv_ms = float(np.mean(gemv_ms_l))
+    e2e = float(np.mean(e2e_ms))
+    ms_max = dist_max(world, ms, dev)
+    e2e_max = dist_max(world, e2e, dev)
+    gemv_ms = dist_max(world, gemv_ms, dev)
+    if rank != 0:
+        return None
+
+    pk = peaks()
+    U = float(np.mean(uniq))
+    algo_bytes = U * expert_bytes(wl)
+    achieved = algo_bytes / (gemv_ms * 1e-3) / 1e9
+    launches_per_step = 8 if T * wl.k <= 1024 else 10
+    traffic = read_traffic_profile()
+    out = {
+        "metric": METRIC,
+        "value": round(world * T / (ms_max * 1e-3), 2),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_max, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "nvfp4 weights x bf16 activations, fp32 accumulate",
+        "data": "synthetic (seeded; NVFP4 experts drawn in the code domain)",
+        "config": {"workload": wl.name, "T": T, "hidden": H, "experts": wl.E, "intermediate": wl.I, "top_k": wl.k,
+                   "shared_intermediate": wl.Is, "path": "decode GEMV (W4A16)", "parallelism": f"replicas x{world}",
+                   "l2": "flushed before every timed step (2x L2 rewrite)", "graph": "CUDA graph of moe_forward"},
+        "diagnostics": {
+            "ms_per_step_without_stage_events": round(plain_ms, 5),
+            "stages_ms_all_events": {n: round(float(v), 5) for n, v in zip(capi.STAGES, stage_avg)},
+            "note": "timed graph holds 2 stage-event nodes (around the expert GEMVs); stages_ms_all_events "
+                    "comes from a graph with an event node at every stage boundary"},
+        "roofline": {"bound": "hbm", "kernel": "nvfp4_expert_gemv (gate/up + down launches, timed together)",
+                     "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(achieved / pk["hbm_gbs"], 4), "peak_source": pk["source"],
+                     "algorithmic_bytes_per_step": int(algo_bytes), "unique_experts_per_step": U,
+                     "bytes_per_expert": expert_bytes(wl), "traffic": traffic},
+        "e2e": {"value": round(world * T / (e2e_max * 1e-3), 2), "unit": "tokens/s",
+                "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2,
+                "ms_per_step": round(e2e_max, 5)},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    if not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(wl, inp, budget_s=args.cpu_seconds)
+    return out
+
+
+def read_traffic_profile():
+    """DRAM bytes per launch of the expert GEMV from the committed ncu summary,
+    if one exists for the current kernels (else null)."""
+    p = os.path.join(ROOT, "profiles", "nvfp4_expert_gemv_decode_t1.traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        return json.load(open(p)).get("dram_bytes_per_step")
+    except (ValueError, OSError):
+        return None
+
+
+# ------------------------------------------------------------------ oracle timing
+
+def cpu_baseline(wl, inp, budget_s=15.0, steps=None):
+    """The CPU oracle, as it stands, on this host's cores: whole site forwards
+    of single tokens (fresh dequantisation cache per token, as a decode step
+    would), repeated for about budget_s seconds."""
+    from oracle import site as OS
+    ocfg = OS.SiteConfig(wl.H, wl.I, wl.Is, wl.E, 0, wl.E, wl.k, wl.rsf, wl.limit)
+    mode = "decode" if wl.kind == "decode" else "prefill"
+    cores = len(os.sched_getaffinity(0))
+    n = 0
+    t0 = time.perf_counter()
+    times = []
+    while True:
+        ts = time.perf_counter()
+        OS.site_forward(inp, ocfg, mode, tokens=np.array([n % wl.T]), cache=OS.ExpertCache(inp))
+        times.append(time.perf_counter() - ts)
+        n += 1
+        if (steps is not None and n >= steps) or (steps is None and time.perf_counter() - t0 > budget_s):
+            break
+    el = time.perf_counter() - t0
+    return {"value": round(n / el, 4), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} single-token site forwards of {wl.name} (fp64 numpy, fresh expert dequant per token)",
+            "seconds": round(el, 2)}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    from routed_nvfp4_expert_b200 import synthetic as syn
+    wl = syn.WORKLOADS[args.workload]
+    inp = syn.make_site(wl, seed=0)
+    cb = cpu_baseline(wl, inp, steps=args.warmup)      # warm-up
+    cb = cpu_baseline(wl, inp, steps=args.steps)
+    ms = 1e3 / cb["value"]
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": cb["value"],
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded)",
+        "config": {"workload": wl.name, "T": wl.T, "hidden": wl.H, "experts": wl.E, "intermediate": wl.I,
+                   "top_k": wl.k, "shared_intermediate": wl.Is, "path": "CPU oracle"},
+        "cpu_baseline": cb,
+        "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ------------------------------------------------------------------ dist
+
+_PG = None
+
+
+def dist_init():
+    global _PG
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
+        _PG = dist
+    return rank, world, local
+
+
+def dist_barrier(world):
+    if world > 1 and _PG is not None:
+        _PG.barrier()
+
+
+def dist_max(world, v, dev=None):
+    if world > 1 and _PG is not None:
+        import torch
+        t = torch.tensor([v], dtype=torch.float64)
+        _PG.all_reduce(t, op=_PG.ReduceOp.MAX)
+        return float(t.item())
+    return v
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode_t1")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank, world, local = dist_init()
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+    else:
+        out = run_ours(args, rank, world, local)
+    if out is not None:
+        print(json.dumps(out), flush=True)
+    if world > 1 and _PG is not None:
+        _PG.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

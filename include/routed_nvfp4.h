@@ -1,0 +1,313 @@
+/*
+ * routed_nvfp4.h -- C ABI of the B200 (sm_100a) routed NVFP4 MoE MLP site.
+ *
+ * The operation is the GLM-5.3-Flash MLP site described by the glm5next_mlp
+ * module docs ("GLM-5.3-Flash MLP production surface"), section "The stack
+ * this layer runs":
+ *
+ *   DENSE  (layers 0..first_k_dense_replace): x -> gate_proj/up_proj ->
+ *          clamped SwiGLU -> down_proj                       (dense_ffn_bf16)
+ *   ROUTED (every later layer):
+ *     x -> gate.weight -> fp32 logits -> router_topk -> ids[K], weights[K]
+ *                                                       (moe_router_topk)
+ *     experts[id] (LOCAL ids only): NVFP4 gate/up -> clamped SwiGLU ->
+ *          NVFP4 down           (nvfp4_expert_gemv / nvfp4_grouped_gemm)
+ *     shared expert: BF16 gate/up -> clamped SwiGLU -> BF16 down
+ *     moe_combine -> partial                             (moe_combine)
+ *
+ * and the rules of its section "Traps this module exists to hold": the
+ * SwiGLU clamp is asymmetric (gate bounded above only, up bounded on both
+ * sides) with a limit that is never defaulted; the router's correction bias
+ * steers selection only and each emitted weight is the unbiased sigmoid
+ * score, renormalised over the chosen k and multiplied by
+ * routed_scaling_factor; the shared expert is never scaled; num_experts is
+ * the FULL expert count and the local range is a separate field. The
+ * Constants section's KERNEL_MAX_TOP_K caps k at 16.
+ *
+ * NVFP4 (the experts' format): E2M1 values (OCP MX v1.0), one E4M3 scale per
+ * 16 consecutive elements along K (OCP OFP8), one fp32 scale per tensor;
+ * value = e2m1 * e4m3 * tensor_scale. Canonical layout: row-major [rows, K],
+ * two codes per byte with the even element in the low nibble; scales
+ * row-major [rows, K/16].
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers unless a comment says otherwise,
+ *    16-byte aligned. The caller owns every buffer; the library allocates and
+ *    frees no device memory and keeps no state besides a thread-local error
+ *    message and the thread-local stage-timing events of
+ *    moe_set_stage_events().
+ *  - bf16 tensors are passed as uint16_t bit patterns.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream). Every call is
+ *    stream-ordered and asynchronous; nothing synchronises except
+ *    moe_read_device_status().
+ *  - A call validates its arguments first. On failure it returns a non-zero
+ *    moe_status_t, launches nothing, and moe_last_error() describes why.
+ *  - T = 0 (no tokens) is a no-op that returns MOE_OK.
+ *  - Errors found on the device (an index out of range, a bounded wait that
+ *    ran out) are OR-ed into the status word at the start of the workspace
+ *    and reported by moe_read_device_status(); the affected outputs are then
+ *    unspecified but every access stays in bounds.
+ */
+#ifndef ROUTED_NVFP4_H
+#define ROUTED_NVFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,    /* bad pointer, size, alignment or config field */
+  MOE_ERR_UNSUPPORTED = 2,    /* valid request outside what the kernels cover */
+  MOE_ERR_WORKSPACE = 3,      /* workspace missing or smaller than required */
+  MOE_ERR_CUDA = 4,           /* a CUDA launch or runtime call failed */
+  MOE_ERR_DEVICE_TIMEOUT = 5, /* a bounded device-side wait ran out */
+  MOE_ERR_DEVICE_BOUNDS = 6   /* a device-side index check failed */
+} moe_status_t;
+
+/* Which implementation of the routed experts moe_forward runs. */
+typedef enum {
+  MOE_PATH_DECODE = 0,  /* W4A16 GEMV: bf16 activations x NVFP4 weights */
+  MOE_PATH_PREFILL = 1  /* W4A4 grouped GEMM on tcgen05 block-scaled FP4 */
+} moe_path_t;
+
+/* Projection selector of the expert kernels. */
+typedef enum {
+  MOE_PROJ_GATE_UP = 0, /* gate and up, fused clamped SwiGLU -> h */
+  MOE_PROJ_DOWN = 1     /* down, times the routing weight -> r[t, j] */
+} moe_proj_t;
+
+/*
+ * Site geometry for one rank (Glm5NextMlpConfig: "read from the checkpoint
+ * config -- never defaulted"). Every field is required and validated.
+ *   hidden               H, multiple of 64
+ *   intermediate         I of each routed expert, multiple of 64
+ *   shared_intermediate  Is of the BF16 shared expert, multiple of 64; 0 = none
+ *   num_experts          E, the FULL expert count the router ranks
+ *   local_begin/end      [begin, end) experts this rank computes; ids outside
+ *                        contribute zero (masked-local expert parallelism);
+ *                        [0, E) on one GPU
+ *   top_k                1 .. min(16, E)
+ *   routed_scaling_factor  finite
+ *   swiglu_limit         > 0; +inf allowed (no clamp); NaN rejected
+ */
+typedef struct {
+  int32_t hidden;
+  int32_t intermediate;
+  int32_t shared_intermediate;
+  int32_t num_experts;
+  int32_t local_begin;
+  int32_t local_end;
+  int32_t top_k;
+  float routed_scaling_factor;
+  float swiglu_limit;
+} moe_config_t;
+
+/* One projection of all E experts in canonical NVFP4 layout, contiguous per
+ * expert: codes [E, rows, cols/2], scales [E, rows, cols/16], tensor_scale [E]
+ * (device fp32). gate/up: rows = I, cols = H. down: rows = H, cols = I. */
+typedef struct {
+  const uint8_t* codes;
+  const uint8_t* scales;
+  const float* tensor_scale;
+} nvfp4_bank_t;
+
+/* Weights of one routed site (Glm5NextMoeWeights), already sharded for this
+ * rank. router_w fp32 [E, H] row-major; router_bias fp32 [E]; shared_* bf16
+ * row-major: gate and up [Is, H], down [H, Is] (NULL when Is == 0). */
+typedef struct {
+  const float* router_w;
+  const float* router_bias;
+  nvfp4_bank_t gate;
+  nvfp4_bank_t up;
+  nvfp4_bank_t down;
+  const uint16_t* shared_gate;
+  const uint16_t* shared_up;
+  const uint16_t* shared_down;
+} moe_weights_t;
+
+/*
+ * Routing plan: the A = T*k assignments (a = t*k + j, j = rank slot) grouped
+ * by expert, stably (token order inside each expert). Device int32 arrays:
+ *   counts       [E]    assignments per expert
+ *   offsets      [E+1]  segment starts, offsets[E] = A
+ *   sorted       [A]    assignment at sorted position p
+ *   inv          [A]    sorted position of assignment a
+ *   tile_offsets [E+1]  prefix sum over experts of ceil(counts/128) for LOCAL
+ *                       experts (0 tiles for remote ones)
+ *   active       [E+1]  active[0] = number of LOCAL experts with counts > 0,
+ *                       active[1..] = their ids in ascending order
+ */
+typedef struct {
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* sorted;
+  int32_t* inv;
+  int32_t* tile_offsets;
+  int32_t* active;
+} moe_plan_t;
+
+/* ------------------------------------------------------------------ sizes */
+
+/* Bytes of workspace moe_forward needs for T tokens on `path` (0 on invalid
+ * arguments; moe_last_error() says why). The same workspace also serves every
+ * single-step entry point that takes one. Contents need no initialisation. */
+size_t moe_workspace_size(const moe_config_t* cfg, int32_t T, int32_t path);
+
+/* Bytes of the routing plan arrays for T tokens (one buffer, carved by
+ * moe_plan_carve). */
+size_t moe_plan_size(const moe_config_t* cfg, int32_t T);
+
+/* Carve a plan out of one device buffer of moe_plan_size() bytes. Host-only
+ * pointer arithmetic; launches nothing. */
+moe_status_t moe_plan_carve(const moe_config_t* cfg, int32_t T, void* buf, size_t bytes, moe_plan_t* plan);
+
+/* ------------------------------------------------------------ the steps */
+
+/*
+ * Router (glm5next_mlp, "The stack this layer runs": gate.weight -> fp32
+ * logits -> router_topk; "Traps": the bias steers selection only).
+ *   x       bf16 [T, H]
+ *   logits  out fp32 [T, E]: l[t,e] = sum_i Wr[e,i] * x[t,i], fp32 accumulate
+ *   ids     out int32 [T, k]: top-k of key = fl32(fl32(sigmoid(l)) + bias) in
+ *           rank order; equal keys go to the lower expert index. The sigmoid
+ *           is evaluated in double and rounded once to fp32.
+ *   weights out fp32 [T, k]: rsf * s_j / sum_chosen s with s = fl32 sigmoid
+ *           of the chosen experts' logits (unbiased); 0 if the sum is 0.
+ * All of the FULL expert count are ranked (local range ignored here).
+ */
+moe_status_t moe_router_topk(const moe_config_t* cfg, const uint16_t* x, int32_t T,
+                             const float* router_w, const float* router_bias,
+                             float* logits, int32_t* ids, float* weights, void* stream);
+
+/*
+ * Token sort (the module list's moe_permute family): builds `plan` from ids
+ * int32 [T, k]. ids outside [0, E) set MOE_ERR_DEVICE_BOUNDS in the workspace
+ * status word and are dropped. ws: workspace of at least
+ * moe_workspace_size(cfg, T, MOE_PATH_PREFILL) bytes.
+ */
+moe_status_t moe_permute(const moe_config_t* cfg, const int32_t* ids, int32_t T,
+                         const moe_plan_t* plan, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Decode expert projections (the module list's W4A16 GEMV: "Every
+ * routed-expert projection here is M=1"): bf16 activations times NVFP4
+ * weights, fp32 accumulation, one pass over each touched expert's bytes for
+ * all of that expert's tokens.
+ *   MOE_PROJ_GATE_UP: act = x bf16 [T, H]; out = h bf16 [T*k, I] with
+ *       h[a] = clamped_swiglu(gate_e . x_t, up_e . x_t) for assignment
+ *       a = t*k + j of LOCAL expert e = ids[t, j]; rows of remote
+ *       assignments are not written. `weights` is ignored (may be NULL).
+ *   MOE_PROJ_DOWN: act = h bf16 [T*k, I]; out = r bf16 [T*k, H] with
+ *       r[a] = weights[a] * (down_e . h[a]); rows of remote assignments are
+ *       written as zeros.
+ *   plan: from moe_permute (or moe_forward) for the same ids.
+ */
+moe_status_t nvfp4_expert_gemv(const moe_config_t* cfg, int32_t proj, const uint16_t* act, int32_t T,
+                               const moe_plan_t* plan, const float* weights,
+                               const moe_weights_t* w, uint16_t* out, void* stream);
+
+/*
+ * Clamped SwiGLU (glm5next_mlp "Traps": the clamp is asymmetric):
+ *   h[m, i] = silu(min(g, L)) * min(max(u, -L), L),  silu(z) = z / (1 + e^-z)
+ *   gu fp32 [M, 2*I]: gate in columns [0, I), up in [I, 2I); h bf16 [M, I].
+ */
+moe_status_t clamped_swiglu(const float* gu, int32_t M, int32_t I, float limit, uint16_t* h, void* stream);
+
+/*
+ * moe_combine (glm5next_mlp, "The stack this layer runs" and "Traps"):
+ *   y[t] = bf16( (sum_{j=0}^{k-1} r[t, j]) + shared[t] ), fp32 accumulation in
+ *   that order; the shared row is added unscaled.
+ *   r bf16 [T, k, H]; shared bf16 [T, H] or NULL; y bf16 [T, H].
+ */
+moe_status_t moe_combine(int32_t T, int32_t k, int32_t H, const uint16_t* r, const uint16_t* shared,
+                         uint16_t* y, void* stream);
+
+/*
+ * Dense BF16 FFN (glm5next_mlp, DENSE layers; also the shared expert):
+ *   y = down_proj( clamped_swiglu(gate_proj x, up_proj x) )
+ *   x bf16 [T, H]; wg, wu bf16 [I, H]; wd bf16 [H, I]; y bf16 [T, H].
+ *   fp32 accumulation; h is rounded to bf16 between the two projections.
+ *   H and I multiples of 64. ws: at least dense_ffn_workspace_size(H, I, T).
+ */
+size_t dense_ffn_workspace_size(int32_t H, int32_t I, int32_t T);
+moe_status_t dense_ffn_bf16(int32_t H, int32_t I, float limit, const uint16_t* x, int32_t T,
+                            const uint16_t* wg, const uint16_t* wu, const uint16_t* wd, uint16_t* y,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * NVFP4 dequantisation (debug / bit-exact check of the format):
+ *   out fp32 [rows, K] = e2m1(code) * e4m3(scale) * tensor_scale[0]
+ *   codes [rows, K/2], scales [rows, K/16] canonical; K multiple of 16.
+ *   The fp32 product is exact whenever it is a normal fp32 number.
+ */
+moe_status_t nvfp4_dequant(const uint8_t* codes, const uint8_t* scales, const float* tensor_scale,
+                           int32_t rows, int32_t K, float* out, void* stream);
+
+/* ------------------------------------------------------------ whole site */
+
+/*
+ * One routed site forward: router, top-k, experts (path), shared expert,
+ * combine. x bf16 [T, H] -> y bf16 [T, H]. ws: moe_workspace_size(cfg, T,
+ * path) bytes. The routing plan, logits, ids and weights of the call stay in
+ * the workspace until the next call (see moe_workspace_views).
+ */
+moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const uint16_t* x, int32_t T,
+                         int32_t path, uint16_t* y, void* ws, size_t ws_bytes, void* stream);
+
+/* Device pointers (inside ws) of the intermediates moe_forward leaves behind:
+ * logits fp32 [T,E], ids int32 [T,k], weights fp32 [T,k], the plan, h bf16
+ * [T*k, I], r bf16 [T*k, H], shared bf16 [T, H] (NULL when Is == 0). Host-only
+ * pointer arithmetic. */
+typedef struct {
+  float* logits;
+  int32_t* ids;
+  float* weights;
+  moe_plan_t plan;
+  uint16_t* h;
+  uint16_t* r;
+  uint16_t* shared;
+} moe_views_t;
+moe_status_t moe_workspace_views(const moe_config_t* cfg, int32_t T, int32_t path, void* ws, size_t ws_bytes,
+                                 moe_views_t* views);
+
+/*
+ * Optional stage timing of moe_forward (profiling hook; thread-local state).
+ * `events` holds n cudaEvent_t handles the caller created (timing enabled);
+ * while set, moe_forward records events[s] on its stream before stage s, for
+ * every s < n - 1 up to the last stage, and events[n-1] after the last stage.
+ * Stages are numbered by moe_stage_t whichever path runs; a stage the path
+ * does not have is recorded with zero length; a NULL entry is not recorded.
+ * Under stream capture the records become graph event nodes
+ * (cudaEventRecordExternal). n must be 0 (off, events may be NULL) or
+ * MOE_STAGE_COUNT + 1.
+ */
+typedef enum {
+  MOE_STAGE_ROUTER_LOGITS = 0,
+  MOE_STAGE_TOPK = 1,
+  MOE_STAGE_PERMUTE = 2,
+  MOE_STAGE_ACT_QUANT = 3,
+  MOE_STAGE_EXPERT_GATE_UP = 4,
+  MOE_STAGE_H_QUANT = 5,
+  MOE_STAGE_EXPERT_DOWN = 6,
+  MOE_STAGE_SHARED = 7,
+  MOE_STAGE_COMBINE = 8,
+  MOE_STAGE_COUNT = 9
+} moe_stage_t;
+moe_status_t moe_set_stage_events(void* const* events, int32_t n);
+
+/* Synchronises `stream`, reads the workspace status word, clears it, and
+ * returns MOE_ERR_DEVICE_TIMEOUT / MOE_ERR_DEVICE_BOUNDS / MOE_OK. */
+moe_status_t moe_read_device_status(void* ws, void* stream);
+
+/* Thread-local description of the last failed call on this thread ("" if none). */
+const char* moe_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ROUTED_NVFP4_H */

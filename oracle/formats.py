@@ -130,13 +130,19 @@ def pack_nibbles(codes: np.ndarray) -> np.ndarray:
     return (c[..., 0::2] & 0xF) | ((c[..., 1::2] & 0xF) << 4)
 
 
+# value of every byte of packed codes: [byte, 0] = low nibble, [byte, 1] = high
+_E2M1_PAIR = np.stack([e2m1_value(np.arange(256) & 0xF), e2m1_value(np.arange(256) >> 4)], axis=1)
+_E4M3_ALL = e4m3_value(np.arange(256))
+
+
 def nvfp4_dequant(codes_u8, scales_u8, tensor_scale) -> np.ndarray:
     """NVFP4 [rows, K] -> fp64: e2m1(code) * e4m3(block scale) * tensor_scale.
     Exact in fp64 (2 + 4 + 24 significand bits)."""
-    v = e2m1_value(unpack_nibbles(codes_u8))
-    s = e4m3_value(scales_u8)
-    s = np.repeat(s, 16, axis=-1)
-    return v * s * float(np.float32(tensor_scale))
+    c = np.asarray(codes_u8, dtype=np.uint8)
+    rows, half = c.shape
+    v = _E2M1_PAIR[c].reshape(rows, half * 2 // 16, 16)           # element order, per 16-block
+    s = _E4M3_ALL[np.asarray(scales_u8, dtype=np.uint8)]           # [rows, K/16]
+    return (v * (s * float(np.float32(tensor_scale)))[:, :, None]).reshape(rows, half * 2)
 
 
 def quantize_rows_nvfp4(a_f32):

@@ -1,0 +1,441 @@
+// C ABI of the routed NVFP4 MoE site: argument validation, workspace layout,
+// and the order of launches. Every device step runs in the kernels of this
+// library; nothing here computes on the host.
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+thread_local cudaEvent_t g_stage_ev[MOE_STAGE_COUNT + 1];
+thread_local int g_n_stage_ev = 0;
+
+// Record the stage-timing event before `stage` (or after the last stage when
+// stage == MOE_STAGE_COUNT), if the caller registered events.
+cudaError_t mark(int stage, cudaStream_t st) {
+  if (g_n_stage_ev <= stage || !g_stage_ev[stage]) return cudaSuccess;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(st, &cs);
+  if (e != cudaSuccess) return e;
+  if (cs == cudaStreamCaptureStatusActive) return cudaEventRecordWithFlags(g_stage_ev[stage], st, cudaEventRecordExternal);
+  return cudaEventRecord(g_stage_ev[stage], st);
+}
+
+moe_status_t fail(moe_status_t s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+moe_status_t cuda_fail(cudaError_t e, const char* where) {
+  return fail(MOE_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+#define RNX_CUDA(call, where)                      \
+  do {                                             \
+    cudaError_t e_ = (call);                       \
+    if (e_ != cudaSuccess) return cuda_fail(e_, where); \
+  } while (0)
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+#define RNX_PTR(p, name)                                                              \
+  do {                                                                                \
+    if (!(p)) return fail(MOE_ERR_INVALID_ARG, "%s is NULL", name);                   \
+    if (!aligned16(p)) return fail(MOE_ERR_INVALID_ARG, "%s is not 16-byte aligned", name); \
+  } while (0)
+
+constexpr int kMaxExperts = 1024;
+constexpr int kMaxTopK = 16;            // KERNEL_MAX_TOP_K
+constexpr size_t kAlign = 256;
+
+size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+moe_status_t check_cfg(const moe_config_t* c) {
+  if (!c) return fail(MOE_ERR_INVALID_ARG, "config is NULL");
+  if (c->hidden <= 0 || c->hidden % 64) return fail(MOE_ERR_INVALID_ARG, "hidden=%d must be a positive multiple of 64", c->hidden);
+  if (c->intermediate <= 0 || c->intermediate % 64)
+    return fail(MOE_ERR_INVALID_ARG, "intermediate=%d must be a positive multiple of 64", c->intermediate);
+  if (c->shared_intermediate < 0 || c->shared_intermediate % 64)
+    return fail(MOE_ERR_INVALID_ARG, "shared_intermediate=%d must be 0 or a multiple of 64", c->shared_intermediate);
+  if (c->num_experts <= 0) return fail(MOE_ERR_INVALID_ARG, "num_experts=%d must be positive", c->num_experts);
+  if (c->num_experts > kMaxExperts)
+    return fail(MOE_ERR_UNSUPPORTED, "num_experts=%d above the supported %d", c->num_experts, kMaxExperts);
+  if (c->local_begin < 0 || c->local_begin > c->local_end || c->local_end > c->num_experts)
+    return fail(MOE_ERR_INVALID_ARG, "local range [%d,%d) not inside [0,%d)", c->local_begin, c->local_end, c->num_experts);
+  if (c->top_k < 1 || c->top_k > kMaxTopK || c->top_k > c->num_experts)
+    return fail(MOE_ERR_INVALID_ARG, "top_k=%d must be in 1..min(16, num_experts)", c->top_k);
+  if (!std::isfinite(c->routed_scaling_factor)) return fail(MOE_ERR_INVALID_ARG, "routed_scaling_factor is not finite");
+  if (std::isnan(c->swiglu_limit) || !(c->swiglu_limit > 0.f))
+    return fail(MOE_ERR_INVALID_ARG, "swiglu_limit must be > 0 (inf allowed, NaN rejected)");
+  return MOE_OK;
+}
+
+moe_status_t check_T(int32_t T) {
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d is negative", T);
+  if ((int64_t)T * kMaxTopK > (1LL << 30)) return fail(MOE_ERR_UNSUPPORTED, "T=%d too large", T);
+  return MOE_OK;
+}
+
+moe_status_t check_bank(const nvfp4_bank_t& b, const char* name) {
+  char buf[64];
+  snprintf(buf, sizeof buf, "%s.codes", name);
+  RNX_PTR(b.codes, buf);
+  snprintf(buf, sizeof buf, "%s.scales", name);
+  RNX_PTR(b.scales, buf);
+  snprintf(buf, sizeof buf, "%s.tensor_scale", name);
+  if (!b.tensor_scale) return fail(MOE_ERR_INVALID_ARG, "%s is NULL", buf);
+  return MOE_OK;
+}
+
+// ------------------------------------------------------------ layouts
+
+struct PlanLayout {
+  size_t counts, offsets, sorted, inv, tile_offsets, active, bytes;
+};
+
+PlanLayout plan_layout(int E, int A) {
+  PlanLayout L{};
+  size_t o = 0;
+  L.counts = o; o = up(o + 4 * (size_t)E);
+  L.offsets = o; o = up(o + 4 * (size_t)(E + 1));
+  L.sorted = o; o = up(o + 4 * (size_t)A);
+  L.inv = o; o = up(o + 4 * (size_t)A);
+  L.tile_offsets = o; o = up(o + 4 * (size_t)(E + 1));
+  L.active = o; o = up(o + 4 * (size_t)(E + 1));
+  L.bytes = o;
+  return L;
+}
+
+moe_plan_t plan_at(char* base, const PlanLayout& L) {
+  moe_plan_t p;
+  p.counts = (int32_t*)(base + L.counts);
+  p.offsets = (int32_t*)(base + L.offsets);
+  p.sorted = (int32_t*)(base + L.sorted);
+  p.inv = (int32_t*)(base + L.inv);
+  p.tile_offsets = (int32_t*)(base + L.tile_offsets);
+  p.active = (int32_t*)(base + L.active);
+  return p;
+}
+
+struct WsLayout {
+  size_t status, logits, ids, weights, plan, scratch, h, r, shared_h, shared, bytes;
+  PlanLayout pl;
+};
+
+WsLayout ws_layout(const moe_config_t* c, int T, int /*path*/) {
+  WsLayout L{};
+  const int E = c->num_experts, k = c->top_k, H = c->hidden, I = c->intermediate, Is = c->shared_intermediate;
+  const size_t A = (size_t)T * k;
+  size_t o = 0;
+  L.status = o; o = up(o + 4);
+  L.logits = o; o = up(o + 4 * (size_t)T * E);
+  L.ids = o; o = up(o + 4 * A);
+  L.weights = o; o = up(o + 4 * A);
+  L.pl = plan_layout(E, (int)A);
+  L.plan = o; o = up(o + L.pl.bytes);
+  L.scratch = o; o = up(o + 4 * rnx::permute_scratch_ints((int)A, E));
+  L.h = o; o = up(o + 2 * A * I);
+  L.r = o; o = up(o + 2 * A * H);
+  L.shared_h = o; o = up(o + 2 * (size_t)T * Is);
+  L.shared = o; o = up(o + 2 * (size_t)T * H);
+  L.bytes = o;
+  return L;
+}
+
+moe_status_t check_ws(const moe_config_t* c, int T, int path, void* ws, size_t ws_bytes, WsLayout* L) {
+  *L = ws_layout(c, T, path);
+  if (!ws) return fail(MOE_ERR_WORKSPACE, "workspace is NULL");
+  if (((uintptr_t)ws % kAlign) != 0) return fail(MOE_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (ws_bytes < L->bytes) return fail(MOE_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, L->bytes);
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_last_error(void) { return g_err; }
+
+moe_status_t moe_set_stage_events(void* const* events, int32_t n) {
+  if (n == 0) {
+    g_n_stage_ev = 0;
+    return MOE_OK;
+  }
+  if (n != MOE_STAGE_COUNT + 1 || !events) return fail(MOE_ERR_INVALID_ARG, "need %d stage events", MOE_STAGE_COUNT + 1);
+  for (int i = 0; i < n; ++i) g_stage_ev[i] = (cudaEvent_t)events[i];   // NULL entries are skipped
+  g_n_stage_ev = n;
+  return MOE_OK;
+}
+
+size_t moe_workspace_size(const moe_config_t* cfg, int32_t T, int32_t path) {
+  if (check_cfg(cfg) != MOE_OK || check_T(T) != MOE_OK) return 0;
+  if (path != MOE_PATH_DECODE && path != MOE_PATH_PREFILL) {
+    fail(MOE_ERR_INVALID_ARG, "unknown path %d", path);
+    return 0;
+  }
+  return ws_layout(cfg, T, path).bytes;
+}
+
+size_t moe_plan_size(const moe_config_t* cfg, int32_t T) {
+  if (check_cfg(cfg) != MOE_OK || check_T(T) != MOE_OK) return 0;
+  return plan_layout(cfg->num_experts, T * cfg->top_k).bytes;
+}
+
+moe_status_t moe_plan_carve(const moe_config_t* cfg, int32_t T, void* buf, size_t bytes, moe_plan_t* plan) {
+  moe_status_t s;
+  if ((s = check_cfg(cfg)) != MOE_OK || (s = check_T(T)) != MOE_OK) return s;
+  if (!plan) return fail(MOE_ERR_INVALID_ARG, "plan is NULL");
+  const PlanLayout L = plan_layout(cfg->num_experts, T * cfg->top_k);
+  if (!buf || ((uintptr_t)buf % kAlign)) return fail(MOE_ERR_INVALID_ARG, "plan buffer NULL or not 256-byte aligned");
+  if (bytes < L.bytes) return fail(MOE_ERR_WORKSPACE, "plan buffer has %zu bytes, needs %zu", bytes, L.bytes);
+  *plan = plan_at((char*)buf, L);
+  return MOE_OK;
+}
+
+moe_status_t moe_workspace_views(const moe_config_t* cfg, int32_t T, int32_t path, void* ws, size_t ws_bytes,
+                                 moe_views_t* v) {
+  moe_status_t s;
+  if ((s = check_cfg(cfg)) != MOE_OK || (s = check_T(T)) != MOE_OK) return s;
+  if (!v) return fail(MOE_ERR_INVALID_ARG, "views is NULL");
+  WsLayout L;
+  if ((s = check_ws(cfg, T, path, ws, ws_bytes, &L)) != MOE_OK) return s;
+  char* b = (char*)ws;
+  v->logits = (float*)(b + L.logits);
+  v->ids = (int32_t*)(b + L.ids);
+  v->weights = (float*)(b + L.weights);
+  v->plan = plan_at(b + L.plan, L.pl);
+  v->h = (uint16_t*)(b + L.h);
+  v->r = (uint16_t*)(b + L.r);
+  v->shared = cfg->shared_intermediate > 0 ? (uint16_t*)(b + L.shared) : nullptr;
+  return MOE_OK;
+}
+
+moe_status_t moe_read_device_status(void* ws, void* stream) {
+  if (!ws) return fail(MOE_ERR_WORKSPACE, "workspace is NULL");
+  cudaStream_t st = (cudaStream_t)stream;
+  RNX_CUDA(cudaStreamSynchronize(st), "cudaStreamSynchronize");
+  uint32_t word = 0;
+  RNX_CUDA(cudaMemcpy(&word, ws, sizeof word, cudaMemcpyDeviceToHost), "cudaMemcpy(status)");
+  RNX_CUDA(cudaMemsetAsync(ws, 0, sizeof word, st), "cudaMemsetAsync(status)");
+  RNX_CUDA(cudaStreamSynchronize(st), "cudaStreamSynchronize");
+  if (word & rnx::kDevErrTimeout) return fail(MOE_ERR_DEVICE_TIMEOUT, "a device-side bounded wait ran out (status 0x%x)", word);
+  if (word & rnx::kDevErrBounds) return fail(MOE_ERR_DEVICE_BOUNDS, "a device-side index check failed (status 0x%x)", word);
+  return MOE_OK;
+}
+
+moe_status_t moe_router_topk(const moe_config_t* cfg, const uint16_t* x, int32_t T, const float* router_w,
+                             const float* router_bias, float* logits, int32_t* ids, float* weights, void* stream) {
+  moe_status_t s;
+  if ((s = check_cfg(cfg)) != MOE_OK || (s = check_T(T)) != MOE_OK) return s;
+  if (T == 0) return MOE_OK;
+  RNX_PTR(x, "x");
+  RNX_PTR(router_w, "router_w");
+  RNX_PTR(router_bias, "router_bias");
+  RNX_PTR(logits, "logits");
+  RNX_PTR(ids, "ids");
+  RNX_PTR(weights, "weights");
+  cudaStream_t st = (cudaStream_t)stream;
+  const int E = cfg->num_experts;
+  RNX_CUDA(rnx::launch_router_logits(x, T, cfg->hidden, E, router_w, logits, st), "router logits");
+  RNX_CUDA(rnx::launch_topk(logits, router_bias, T, E, cfg->top_k, cfg->routed_scaling_factor, ids, weights, st),
+           "router top-k");
+  return MOE_OK;
+}
+
+moe_status_t moe_permute(const moe_config_t* cfg, const int32_t* ids, int32_t T, const moe_plan_t* plan, void* ws,
+                         size_t ws_bytes, void* stream) {
+  moe_status_t s;
+  if ((s = check_cfg(cfg)) != MOE_OK || (s = check_T(T)) != MOE_OK) return s;
+  if (T == 0) return MOE_OK;
+  RNX_PTR(ids, "ids");
+  if (!plan) return fail(MOE_ERR_INVALID_ARG, "plan is NULL");
+  RNX_PTR(plan->counts, "plan.counts");
+  RNX_PTR(plan->offsets, "plan.offsets");
+  RNX_PTR(plan->sorted, "plan.sorted");
+  RNX_PTR(plan->inv, "plan.inv");
+  RNX_PTR(plan->tile_offsets, "plan.tile_offsets");
+  RNX_PTR(plan->active, "plan.active");
+  WsLayout L;
+  if ((s = check_ws(cfg, T, MOE_PATH_PREFILL, ws, ws_bytes, &L)) != MOE_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  char* b = (char*)ws;
+  RNX_CUDA(cudaMemsetAsync(b + L.status, 0, 4, st), "clear status");
+  RNX_CUDA(rnx::launch_permute(ids, T * cfg->top_k, cfg->num_experts, cfg->local_begin, cfg->local_end, *plan,
+                               (int32_t*)(b + L.scratch), (uint32_t*)(b + L.status), st),
+           "permute");
+  return MOE_OK;
+}
+
+moe_status_t nvfp4_expert_gemv(const moe_config_t* cfg, int32_t proj, const uint16_t* act, int32_t T,
+                               const moe_plan_t* plan, const float* weights, const moe_weights_t* w, uint16_t* out,
+                               void* stream) {
+  moe_status_t s;
+  if ((s = check_cfg(cfg)) != MOE_OK || (s = check_T(T)) != MOE_OK) return s;
+  if (proj != MOE_PROJ_GATE_UP && proj != MOE_PROJ_DOWN) return fail(MOE_ERR_INVALID_ARG, "unknown proj %d", proj);
+  if (T == 0) return MOE_OK;
+  RNX_PTR(act, "act");
+  RNX_PTR(out, "out");
+  if (!plan || !w) return fail(MOE_ERR_INVALID_ARG, "plan / weights struct is NULL");
+  RNX_PTR(plan->offsets, "plan.offsets");
+  RNX_PTR(plan->sorted, "plan.sorted");
+  RNX_PTR(plan->active, "plan.active");
+  if (proj == MOE_PROJ_GATE_UP) {
+    if ((s = check_bank(w->gate, "gate")) != MOE_OK || (s = check_bank(w->up, "up")) != MOE_OK) return s;
+  } else {
+    if ((s = check_bank(w->down, "down")) != MOE_OK) return s;
+    RNX_PTR(weights, "weights");
+  }
+  rnx::ExpertGemvArgs a{};
+  a.proj = proj;
+  a.T = T; a.H = cfg->hidden; a.I = cfg->intermediate; a.E = cfg->num_experts; a.k = cfg->top_k;
+  a.local_begin = cfg->local_begin; a.local_end = cfg->local_end;
+  a.limit = cfg->swiglu_limit;
+  a.act = act;
+  a.offsets = plan->offsets; a.sorted = plan->sorted; a.active = plan->active;
+  a.weights = weights;
+  a.gate = w->gate; a.up = w->up; a.down = w->down;
+  a.out = out;
+  RNX_CUDA(rnx::launch_nvfp4_gemv(a, (cudaStream_t)stream), "nvfp4_expert_gemv");
+  return MOE_OK;
+}
+
+moe_status_t clamped_swiglu(const float* gu, int32_t M, int32_t I, float limit, uint16_t* h, void* stream) {
+  if (M < 0 || I <= 0 || I % 4) return fail(MOE_ERR_INVALID_ARG, "M=%d, I=%d: need M >= 0, I a positive multiple of 4", M, I);
+  if (std::isnan(limit) || !(limit > 0.f)) return fail(MOE_ERR_INVALID_ARG, "limit must be > 0");
+  if (M == 0) return MOE_OK;
+  RNX_PTR(gu, "gu");
+  RNX_PTR(h, "h");
+  RNX_CUDA(rnx::launch_swiglu(gu, M, I, limit, h, (cudaStream_t)stream), "clamped_swiglu");
+  return MOE_OK;
+}
+
+moe_status_t moe_combine(int32_t T, int32_t k, int32_t H, const uint16_t* r, const uint16_t* shared, uint16_t* y,
+                         void* stream) {
+  if (T < 0 || k < 1 || k > kMaxTopK || H <= 0 || H % 8)
+    return fail(MOE_ERR_INVALID_ARG, "T=%d k=%d H=%d: need T >= 0, 1 <= k <= 16, H a positive multiple of 8", T, k, H);
+  if (T == 0) return MOE_OK;
+  RNX_PTR(r, "r");
+  RNX_PTR(y, "y");
+  if (shared && !aligned16(shared)) return fail(MOE_ERR_INVALID_ARG, "shared is not 16-byte aligned");
+  RNX_CUDA(rnx::launch_combine(T, k, H, r, shared, y, (cudaStream_t)stream), "moe_combine");
+  return MOE_OK;
+}
+
+size_t dense_ffn_workspace_size(int32_t H, int32_t I, int32_t T) {
+  if (H <= 0 || I <= 0 || T < 0) return 0;
+  return up(4) + up(2 * (size_t)T * I);
+}
+
+moe_status_t dense_ffn_bf16(int32_t H, int32_t I, float limit, const uint16_t* x, int32_t T, const uint16_t* wg,
+                            const uint16_t* wu, const uint16_t* wd, uint16_t* y, void* ws, size_t ws_bytes,
+                            void* stream) {
+  if (H <= 0 || H % 64 || I <= 0 || I % 64 || T < 0)
+    return fail(MOE_ERR_INVALID_ARG, "H=%d I=%d T=%d: need H, I positive multiples of 64, T >= 0", H, I, T);
+  if (std::isnan(limit) || !(limit > 0.f)) return fail(MOE_ERR_INVALID_ARG, "limit must be > 0");
+  if (T == 0) return MOE_OK;
+  RNX_PTR(x, "x");
+  RNX_PTR(wg, "wg");
+  RNX_PTR(wu, "wu");
+  RNX_PTR(wd, "wd");
+  RNX_PTR(y, "y");
+  if (!ws || ((uintptr_t)ws % kAlign)) return fail(MOE_ERR_WORKSPACE, "workspace NULL or not 256-byte aligned");
+  if (ws_bytes < dense_ffn_workspace_size(H, I, T))
+    return fail(MOE_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, dense_ffn_workspace_size(H, I, T));
+  uint16_t* hbuf = (uint16_t*)((char*)ws + up(4));
+  RNX_CUDA(rnx::launch_dense_gemv(H, I, limit, x, T, wg, wu, wd, y, hbuf, (cudaStream_t)stream), "dense_ffn_bf16");
+  return MOE_OK;
+}
+
+moe_status_t nvfp4_dequant(const uint8_t* codes, const uint8_t* scales, const float* tensor_scale, int32_t rows,
+                           int32_t K, float* out, void* stream) {
+  if (rows < 0 || K <= 0 || K % 16) return fail(MOE_ERR_INVALID_ARG, "rows=%d K=%d: K must be a positive multiple of 16", rows, K);
+  if (rows == 0) return MOE_OK;
+  if (!codes || ((uintptr_t)codes & 7)) return fail(MOE_ERR_INVALID_ARG, "codes NULL or not 8-byte aligned");
+  if (!scales || !tensor_scale) return fail(MOE_ERR_INVALID_ARG, "scales / tensor_scale is NULL");
+  RNX_PTR(out, "out");
+  RNX_CUDA(rnx::launch_dequant(codes, scales, tensor_scale, rows, K, out, (cudaStream_t)stream), "nvfp4_dequant");
+  return MOE_OK;
+}
+
+moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const uint16_t* x, int32_t T, int32_t path,
+                         uint16_t* y, void* ws, size_t ws_bytes, void* stream) {
+  moe_status_t s;
+  if ((s = check_cfg(cfg)) != MOE_OK || (s = check_T(T)) != MOE_OK) return s;
+  if (path != MOE_PATH_DECODE && path != MOE_PATH_PREFILL) return fail(MOE_ERR_INVALID_ARG, "unknown path %d", path);
+  if (T == 0) return MOE_OK;
+  if (!w) return fail(MOE_ERR_INVALID_ARG, "weights struct is NULL");
+  RNX_PTR(x, "x");
+  RNX_PTR(y, "y");
+  RNX_PTR(w->router_w, "router_w");
+  RNX_PTR(w->router_bias, "router_bias");
+  if ((s = check_bank(w->gate, "gate")) != MOE_OK || (s = check_bank(w->up, "up")) != MOE_OK ||
+      (s = check_bank(w->down, "down")) != MOE_OK)
+    return s;
+  const int Is = cfg->shared_intermediate;
+  if (Is > 0) {
+    RNX_PTR(w->shared_gate, "shared_gate");
+    RNX_PTR(w->shared_up, "shared_up");
+    RNX_PTR(w->shared_down, "shared_down");
+  }
+  if (path == MOE_PATH_PREFILL) return fail(MOE_ERR_UNSUPPORTED, "prefill path not built yet");
+  WsLayout L;
+  if ((s = check_ws(cfg, T, path, ws, ws_bytes, &L)) != MOE_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  char* b = (char*)ws;
+  const int E = cfg->num_experts, k = cfg->top_k, H = cfg->hidden, I = cfg->intermediate;
+  float* logits = (float*)(b + L.logits);
+  int32_t* ids = (int32_t*)(b + L.ids);
+  float* wts = (float*)(b + L.weights);
+  moe_plan_t plan = plan_at(b + L.plan, L.pl);
+  uint16_t* h = (uint16_t*)(b + L.h);
+  uint16_t* r = (uint16_t*)(b + L.r);
+  uint16_t* shared = Is > 0 ? (uint16_t*)(b + L.shared) : nullptr;
+  uint32_t* status = (uint32_t*)(b + L.status);
+
+  RNX_CUDA(cudaMemsetAsync(status, 0, 4, st), "clear status");
+  RNX_CUDA(mark(MOE_STAGE_ROUTER_LOGITS, st), "stage event");
+  RNX_CUDA(rnx::launch_router_logits(x, T, H, E, w->router_w, logits, st), "router logits");
+  RNX_CUDA(mark(MOE_STAGE_TOPK, st), "stage event");
+  RNX_CUDA(rnx::launch_topk(logits, w->router_bias, T, E, k, cfg->routed_scaling_factor, ids, wts, st), "top-k");
+  RNX_CUDA(mark(MOE_STAGE_PERMUTE, st), "stage event");
+  RNX_CUDA(rnx::launch_permute(ids, T * k, E, cfg->local_begin, cfg->local_end, plan, (int32_t*)(b + L.scratch),
+                               status, st),
+           "permute");
+  RNX_CUDA(mark(MOE_STAGE_ACT_QUANT, st), "stage event");
+  rnx::ExpertGemvArgs a{};
+  a.T = T; a.H = H; a.I = I; a.E = E; a.k = k;
+  a.local_begin = cfg->local_begin; a.local_end = cfg->local_end;
+  a.limit = cfg->swiglu_limit;
+  a.offsets = plan.offsets; a.sorted = plan.sorted; a.active = plan.active;
+  a.weights = wts;
+  a.gate = w->gate; a.up = w->up; a.down = w->down;
+  a.status = status;
+  a.proj = MOE_PROJ_GATE_UP; a.act = x; a.out = h;
+  RNX_CUDA(mark(MOE_STAGE_EXPERT_GATE_UP, st), "stage event");
+  RNX_CUDA(rnx::launch_nvfp4_gemv(a, st), "expert gate/up");
+  RNX_CUDA(mark(MOE_STAGE_H_QUANT, st), "stage event");
+  a.proj = MOE_PROJ_DOWN; a.act = h; a.out = r;
+  RNX_CUDA(mark(MOE_STAGE_EXPERT_DOWN, st), "stage event");
+  RNX_CUDA(rnx::launch_nvfp4_gemv(a, st), "expert down");
+  RNX_CUDA(mark(MOE_STAGE_SHARED, st), "stage event");
+  if (Is > 0) {
+    RNX_CUDA(rnx::launch_dense_gemv(H, Is, cfg->swiglu_limit, x, T, w->shared_gate, w->shared_up, w->shared_down,
+                                    shared, (uint16_t*)(b + L.shared_h), st),
+             "shared expert");
+  }
+  RNX_CUDA(mark(MOE_STAGE_COMBINE, st), "stage event");
+  RNX_CUDA(rnx::launch_combine(T, k, H, r, shared, y, st), "combine");
+  RNX_CUDA(mark(MOE_STAGE_COUNT, st), "stage event");
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -104,6 +104,8 @@ def _nibble_table() -> np.ndarray:
 
 
 _NIB = _nibble_table()
+# two random bytes (little-endian uint16) -> one packed byte of two nibbles
+_NIB_PAIR = (_NIB[np.arange(65536) & 0xFF] | (_NIB[np.arange(65536) >> 8] << 4)).astype(np.uint8)
 
 
 def _scale_table() -> np.ndarray:
@@ -130,9 +132,8 @@ def nvfp4_bank(seed: int, proj: str, E: int, rows: int, cols: int, sigma_w: floa
     codes = np.empty((E, rows, cols // 2), np.uint8)
     scales = np.empty((E, rows, cols // 16), np.uint8)
     for e in range(E):
-        raw = np.frombuffer(rc.bytes(rows * cols), dtype=np.uint8).reshape(rows, cols)
-        nib = _NIB[raw]
-        codes[e] = nib[:, 0::2] | (nib[:, 1::2] << 4)
+        raw = np.frombuffer(rc.bytes(rows * cols), dtype="<u2").reshape(rows, cols // 2)
+        codes[e] = _NIB_PAIR[raw]
         rawsc = np.frombuffer(rs.bytes(rows * cols // 16), dtype=np.uint8).reshape(rows, cols // 16)
         scales[e] = _SCALE[rawsc]
     base = sigma_w / _RMS_CODE_TIMES_SCALE
@@ -145,10 +146,10 @@ def bf16_matrix(seed: int, name: str, rows: int, cols: int, sigma: float) -> np.
     return _to_bf16_bits(r.standard_normal((rows, cols), dtype=np.float32) * np.float32(sigma))
 
 
-def make_site(wl: Workload, seed: int = 0, with_dense: bool = False) -> dict:
-    """All inputs of one MoE site forward (and optionally the dense FFN)."""
-    T, H, I, E = wl.T, wl.H, wl.I, wl.E
-    out: dict = {"workload": wl}
+def make_router_and_x(wl: Workload, seed: int = 0) -> dict:
+    """x bf16 [T, H], router_w fp32 [E, H], router_bias fp32 [E] (+ the stress set-up)."""
+    T, H, E = wl.T, wl.H, wl.E
+    out: dict = {}
     rx = _rng(seed, "x")
     x = rx.standard_normal((T, H), dtype=np.float32) * np.float32(wl.x_scale)
     rw = _rng(seed, "router_w")
@@ -170,13 +171,35 @@ def make_site(wl: Workload, seed: int = 0, with_dense: bool = False) -> dict:
     out["x"] = _to_bf16_bits(x)
     out["router_w"] = router_w
     out["router_bias"] = bias
-    for proj, rows, cols in (("gate", I, H), ("up", I, H), ("down", H, I)):
-        c, s, t = nvfp4_bank(seed, proj, E, rows, cols, wl.sigma_w)
+    return out
+
+
+def make_experts(wl: Workload, seed: int = 0) -> dict:
+    """NVFP4 banks: gate/up [E, I, H], down [E, H, I] (codes, scales, tensor scales)."""
+    out: dict = {}
+    for proj, rows, cols in (("gate", wl.I, wl.H), ("up", wl.I, wl.H), ("down", wl.H, wl.I)):
+        c, s, t = nvfp4_bank(seed, proj, wl.E, rows, cols, wl.sigma_w)
         out[f"{proj}_codes"], out[f"{proj}_scales"], out[f"{proj}_ts"] = c, s, t
-    if wl.Is > 0:
-        out["shared_gate"] = bf16_matrix(seed, "shared_gate", wl.Is, H, wl.sigma_w)
-        out["shared_up"] = bf16_matrix(seed, "shared_up", wl.Is, H, wl.sigma_w)
-        out["shared_down"] = bf16_matrix(seed, "shared_down", H, wl.Is, wl.sigma_w)
+    return out
+
+
+def make_shared(wl: Workload, seed: int = 0) -> dict:
+    """BF16 shared expert: gate/up [Is, H], down [H, Is] (empty when Is == 0)."""
+    if wl.Is <= 0:
+        return {}
+    return {
+        "shared_gate": bf16_matrix(seed, "shared_gate", wl.Is, wl.H, wl.sigma_w),
+        "shared_up": bf16_matrix(seed, "shared_up", wl.Is, wl.H, wl.sigma_w),
+        "shared_down": bf16_matrix(seed, "shared_down", wl.H, wl.Is, wl.sigma_w),
+    }
+
+
+def make_site(wl: Workload, seed: int = 0, with_dense: bool = False) -> dict:
+    """All inputs of one MoE site forward (and optionally the dense FFN)."""
+    out: dict = {"workload": wl}
+    out.update(make_router_and_x(wl, seed))
+    out.update(make_experts(wl, seed))
+    out.update(make_shared(wl, seed))
     if with_dense:
         out.update(make_dense(wl, seed))
     return out

@@ -1,0 +1,96 @@
+"""The C-ABI library without a GPU: it loads, exports every function the
+header declares, and rejects bad arguments before touching the device."""
+import ctypes as C
+import math
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+from routed_nvfp4_expert_b200 import capi
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s+\*?([a-z_][a-z0-9_]*)\s*\(", src, re.M):
+                names.add(m.group(1))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = C.CDLL(capi._LIB_PATH)
+    declared = _declared()
+    assert len(declared) >= 15
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert declared == set(capi.EXPORTED)
+
+
+def _cfg(**kw):
+    base = dict(hidden=256, intermediate=128, shared_intermediate=128, num_experts=16, local_begin=0, local_end=16,
+                top_k=4, routed_scaling_factor=2.5, swiglu_limit=7.0)
+    base.update(kw)
+    return capi.SiteConfig(**base)
+
+
+@pytest.mark.parametrize("kw,frag", [
+    (dict(top_k=17), "top_k"), (dict(top_k=0), "top_k"), (dict(num_experts=3, local_end=3), "top_k"),
+    (dict(hidden=100), "hidden"), (dict(intermediate=0), "intermediate"), (dict(shared_intermediate=32), "shared"),
+    (dict(swiglu_limit=math.nan), "swiglu_limit"), (dict(swiglu_limit=-1.0), "swiglu_limit"),
+    (dict(routed_scaling_factor=math.inf), "routed_scaling_factor"), (dict(local_end=17), "local range"),
+    (dict(local_begin=5, local_end=4), "local range"), (dict(num_experts=2000, local_end=2000), "num_experts"),
+])
+def test_config_validation(kw, frag):
+    cfg = _cfg(**kw)
+    lib = capi.lib()
+    assert lib.moe_workspace_size(C.byref(cfg.c()), 4, 0) == 0
+    assert frag in lib.moe_last_error().decode()
+    w = capi.MoeWeights()
+    st = lib.moe_forward(C.byref(cfg.c()), C.byref(w), 16, 4, 0, 16, 256, 1 << 20, None)
+    assert st in (1, 2)
+
+
+def test_swiglu_limit_inf_is_valid():
+    assert capi.lib().moe_workspace_size(C.byref(_cfg(swiglu_limit=math.inf).c()), 4, 0) > 0
+
+
+def test_t_zero_is_a_noop_and_bad_pointers_are_rejected():
+    lib = capi.lib()
+    cfg = _cfg().c()
+    w = capi.MoeWeights()
+    assert lib.moe_forward(C.byref(cfg), C.byref(w), None, 0, 0, None, None, 0, None) == 0
+    # misaligned x
+    st = lib.moe_forward(C.byref(cfg), C.byref(w), 0x1001, 4, 0, 0x2000, 0x3000, 1 << 30, None)
+    assert st == 1 and "x" in lib.moe_last_error().decode()
+    # unknown path
+    assert lib.moe_forward(C.byref(cfg), C.byref(w), 0x1000, 4, 7, 0x2000, 0x3000, 1 << 30, None) == 1
+    # combine: k > 16
+    assert lib.moe_combine(4, 17, 256, 0x1000, None, 0x2000, None) == 1
+    assert lib.moe_combine(0, 4, 256, None, None, None, None) == 0
+
+
+def test_workspace_too_small_is_rejected_before_launch():
+    lib = capi.lib()
+    cfg = _cfg().c()
+    need = lib.moe_workspace_size(C.byref(cfg), 4, 0)
+    assert need > 0
+    ids = 0x10000
+    plan = capi.MoePlan(0x20000, 0x30000, 0x40000, 0x50000, 0x60000, 0x70000)
+    st = lib.moe_permute(C.byref(cfg), ids, 4, C.byref(plan), 0x100000, need - 256, None)
+    assert st == 3 and "workspace" in lib.moe_last_error().decode()
+
+
+def test_plan_carve_is_host_arithmetic():
+    lib = capi.lib()
+    cfg = _cfg().c()
+    n = lib.moe_plan_size(C.byref(cfg), 10)
+    plan = capi.MoePlan()
+    assert lib.moe_plan_carve(C.byref(cfg), 10, 0x100000, n, C.byref(plan)) == 0
+    ptrs = [plan.counts, plan.offsets, plan.sorted, plan.inv, plan.tile_offsets, plan.active]
+    assert ptrs == sorted(ptrs) and all(p % 256 == 0 for p in ptrs) and ptrs[0] == 0x100000
+    assert lib.moe_plan_carve(C.byref(cfg), 10, 0x100000, n - 1, C.byref(plan)) == 3
