@@ -140,6 +140,8 @@ typedef struct {
  *                       experts (0 tiles for remote ones)
  *   active       [E+1]  active[0] = number of LOCAL experts with counts > 0,
  *                       active[1..] = their ids in ascending order
+ *   first        [E]    first[u] = sorted[offsets[active[1+u]]], the first
+ *                       assignment of the u-th active expert
  */
 typedef struct {
   int32_t* counts;
@@ -148,6 +150,7 @@ typedef struct {
   int32_t* inv;
   int32_t* tile_offsets;
   int32_t* active;
+  int32_t* first;
 } moe_plan_t;
 
 /* ------------------------------------------------------------------ sizes */
@@ -205,10 +208,12 @@ moe_status_t moe_permute(const moe_config_t* cfg, const int32_t* ids, int32_t T,
  *       r[a] = weights[a] * (down_e . h[a]); rows of remote assignments are
  *       written as zeros.
  *   plan: from moe_permute (or moe_forward) for the same ids.
+ *   ws:   workspace of at least moe_workspace_size(cfg, T, MOE_PATH_DECODE)
+ *         bytes (status word and per-row activation maxima).
  */
 moe_status_t nvfp4_expert_gemv(const moe_config_t* cfg, int32_t proj, const uint16_t* act, int32_t T,
                                const moe_plan_t* plan, const float* weights,
-                               const moe_weights_t* w, uint16_t* out, void* stream);
+                               const moe_weights_t* w, uint16_t* out, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Clamped SwiGLU (glm5next_mlp "Traps": the clamp is asymmetric):

@@ -57,7 +57,7 @@ class MoeWeights(C.Structure):
 
 class MoePlan(C.Structure):
     _fields_ = [("counts", C.c_void_p), ("offsets", C.c_void_p), ("sorted", C.c_void_p), ("inv", C.c_void_p),
-                ("tile_offsets", C.c_void_p), ("active", C.c_void_p)]
+                ("tile_offsets", C.c_void_p), ("active", C.c_void_p), ("first", C.c_void_p)]
 
 
 class MoeViews(C.Structure):
@@ -78,7 +78,7 @@ def load_library(path: str = _LIB_PATH) -> C.CDLL:
         "moe_plan_carve": (st, [cfgp, i32, vp, sz, C.POINTER(MoePlan)]),
         "moe_router_topk": (st, [cfgp, vp, i32, vp, vp, vp, vp, vp, vp]),
         "moe_permute": (st, [cfgp, vp, i32, C.POINTER(MoePlan), vp, sz, vp]),
-        "nvfp4_expert_gemv": (st, [cfgp, i32, vp, i32, C.POINTER(MoePlan), vp, C.POINTER(MoeWeights), vp, vp]),
+        "nvfp4_expert_gemv": (st, [cfgp, i32, vp, i32, C.POINTER(MoePlan), vp, C.POINTER(MoeWeights), vp, vp, sz, vp]),
         "clamped_swiglu": (st, [vp, i32, i32, C.c_float, vp, vp]),
         "moe_combine": (st, [i32, i32, i32, vp, vp, vp, vp]),
         "dense_ffn_workspace_size": (sz, [i32, i32, i32]),
@@ -220,10 +220,10 @@ def moe_permute(cfg: SiteConfig, ids, plan: MoePlan, ws, stream=None):
 
 
 def nvfp4_expert_gemv(cfg: SiteConfig, proj: int, act, T: int, plan: MoePlan, weights, site: DeviceSite, out,
-                      stream=None):
+                      ws, stream=None):
     w = site.c()
     _check(lib().nvfp4_expert_gemv(C.byref(cfg.c()), proj, _p(act), T, C.byref(plan), _p(weights), C.byref(w),
-                                   _p(out), _stream(stream)))
+                                   _p(out), _p(ws), ws.numel(), _stream(stream)))
 
 
 def clamped_swiglu(gu, limit: float, h, stream=None):

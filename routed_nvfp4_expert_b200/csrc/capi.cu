@@ -99,7 +99,7 @@ moe_status_t check_bank(const nvfp4_bank_t& b, const char* name) {
 // ------------------------------------------------------------ layouts
 
 struct PlanLayout {
-  size_t counts, offsets, sorted, inv, tile_offsets, active, bytes;
+  size_t counts, offsets, sorted, inv, tile_offsets, active, first, bytes;
 };
 
 PlanLayout plan_layout(int E, int A) {
@@ -111,6 +111,7 @@ PlanLayout plan_layout(int E, int A) {
   L.inv = o; o = up(o + 4 * (size_t)A);
   L.tile_offsets = o; o = up(o + 4 * (size_t)(E + 1));
   L.active = o; o = up(o + 4 * (size_t)(E + 1));
+  L.first = o; o = up(o + 4 * (size_t)E);
   L.bytes = o;
   return L;
 }
@@ -123,11 +124,12 @@ moe_plan_t plan_at(char* base, const PlanLayout& L) {
   p.inv = (int32_t*)(base + L.inv);
   p.tile_offsets = (int32_t*)(base + L.tile_offsets);
   p.active = (int32_t*)(base + L.active);
+  p.first = (int32_t*)(base + L.first);
   return p;
 }
 
 struct WsLayout {
-  size_t status, logits, ids, weights, plan, scratch, h, r, shared_h, shared, bytes;
+  size_t status, logits, ids, weights, plan, scratch, h, r, shared_h, shared, xmax, hmax, bytes;
   PlanLayout pl;
 };
 
@@ -147,6 +149,8 @@ WsLayout ws_layout(const moe_config_t* c, int T, int /*path*/) {
   L.r = o; o = up(o + 2 * A * H);
   L.shared_h = o; o = up(o + 2 * (size_t)T * Is);
   L.shared = o; o = up(o + 2 * (size_t)T * H);
+  L.xmax = o; o = up(o + 4 * (size_t)T);
+  L.hmax = o; o = up(o + 4 * A);
   L.bytes = o;
   return L;
 }
@@ -264,6 +268,7 @@ moe_status_t moe_permute(const moe_config_t* cfg, const int32_t* ids, int32_t T,
   RNX_PTR(plan->inv, "plan.inv");
   RNX_PTR(plan->tile_offsets, "plan.tile_offsets");
   RNX_PTR(plan->active, "plan.active");
+  RNX_PTR(plan->first, "plan.first");
   WsLayout L;
   if ((s = check_ws(cfg, T, MOE_PATH_PREFILL, ws, ws_bytes, &L)) != MOE_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
@@ -277,7 +282,7 @@ moe_status_t moe_permute(const moe_config_t* cfg, const int32_t* ids, int32_t T,
 
 moe_status_t nvfp4_expert_gemv(const moe_config_t* cfg, int32_t proj, const uint16_t* act, int32_t T,
                                const moe_plan_t* plan, const float* weights, const moe_weights_t* w, uint16_t* out,
-                               void* stream) {
+                               void* ws, size_t ws_bytes, void* stream) {
   moe_status_t s;
   if ((s = check_cfg(cfg)) != MOE_OK || (s = check_T(T)) != MOE_OK) return s;
   if (proj != MOE_PROJ_GATE_UP && proj != MOE_PROJ_DOWN) return fail(MOE_ERR_INVALID_ARG, "unknown proj %d", proj);
@@ -288,23 +293,35 @@ moe_status_t nvfp4_expert_gemv(const moe_config_t* cfg, int32_t proj, const uint
   RNX_PTR(plan->offsets, "plan.offsets");
   RNX_PTR(plan->sorted, "plan.sorted");
   RNX_PTR(plan->active, "plan.active");
+  RNX_PTR(plan->first, "plan.first");
   if (proj == MOE_PROJ_GATE_UP) {
     if ((s = check_bank(w->gate, "gate")) != MOE_OK || (s = check_bank(w->up, "up")) != MOE_OK) return s;
   } else {
     if ((s = check_bank(w->down, "down")) != MOE_OK) return s;
     RNX_PTR(weights, "weights");
   }
+  WsLayout L;
+  if ((s = check_ws(cfg, T, MOE_PATH_DECODE, ws, ws_bytes, &L)) != MOE_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  char* b = (char*)ws;
+  const int K = proj == MOE_PROJ_GATE_UP ? cfg->hidden : cfg->intermediate;
+  const int R = proj == MOE_PROJ_GATE_UP ? T : T * cfg->top_k;
+  uint32_t* amax = (uint32_t*)(b + (proj == MOE_PROJ_GATE_UP ? L.xmax : L.hmax));
+  RNX_CUDA(cudaMemsetAsync(b + L.status, 0, 4, st), "clear status");
+  RNX_CUDA(rnx::launch_row_absmax(act, R, K, amax, st), "activation row max");
   rnx::ExpertGemvArgs a{};
   a.proj = proj;
   a.T = T; a.H = cfg->hidden; a.I = cfg->intermediate; a.E = cfg->num_experts; a.k = cfg->top_k;
   a.local_begin = cfg->local_begin; a.local_end = cfg->local_end;
   a.limit = cfg->swiglu_limit;
   a.act = act;
-  a.offsets = plan->offsets; a.sorted = plan->sorted; a.active = plan->active;
+  a.offsets = plan->offsets; a.sorted = plan->sorted; a.active = plan->active; a.first = plan->first;
   a.weights = weights;
   a.gate = w->gate; a.up = w->up; a.down = w->down;
   a.out = out;
-  RNX_CUDA(rnx::launch_nvfp4_gemv(a, (cudaStream_t)stream), "nvfp4_expert_gemv");
+  a.status = (uint32_t*)(b + L.status);
+  a.act_max = amax;
+  RNX_CUDA(rnx::launch_nvfp4_gemv(a, st), "nvfp4_expert_gemv");
   return MOE_OK;
 }
 
@@ -403,7 +420,9 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
 
   RNX_CUDA(cudaMemsetAsync(status, 0, 4, st), "clear status");
   RNX_CUDA(mark(MOE_STAGE_ROUTER_LOGITS, st), "stage event");
-  RNX_CUDA(rnx::launch_router_logits(x, T, H, E, w->router_w, logits, st), "router logits");
+  uint32_t* xmax = (uint32_t*)(b + L.xmax);
+  uint32_t* hmax = (uint32_t*)(b + L.hmax);
+  RNX_CUDA(rnx::launch_router_logits(x, T, H, E, w->router_w, logits, st, xmax, hmax, T * k), "router logits");
   RNX_CUDA(mark(MOE_STAGE_TOPK, st), "stage event");
   RNX_CUDA(rnx::launch_topk(logits, w->router_bias, T, E, k, cfg->routed_scaling_factor, ids, wts, st), "top-k");
   RNX_CUDA(mark(MOE_STAGE_PERMUTE, st), "stage event");
@@ -415,15 +434,15 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
   a.T = T; a.H = H; a.I = I; a.E = E; a.k = k;
   a.local_begin = cfg->local_begin; a.local_end = cfg->local_end;
   a.limit = cfg->swiglu_limit;
-  a.offsets = plan.offsets; a.sorted = plan.sorted; a.active = plan.active;
+  a.offsets = plan.offsets; a.sorted = plan.sorted; a.active = plan.active; a.first = plan.first;
   a.weights = wts;
   a.gate = w->gate; a.up = w->up; a.down = w->down;
   a.status = status;
-  a.proj = MOE_PROJ_GATE_UP; a.act = x; a.out = h;
+  a.proj = MOE_PROJ_GATE_UP; a.act = x; a.out = h; a.act_max = xmax; a.out_max = hmax; a.prefetch_down = false;
   RNX_CUDA(mark(MOE_STAGE_EXPERT_GATE_UP, st), "stage event");
   RNX_CUDA(rnx::launch_nvfp4_gemv(a, st), "expert gate/up");
   RNX_CUDA(mark(MOE_STAGE_H_QUANT, st), "stage event");
-  a.proj = MOE_PROJ_DOWN; a.act = h; a.out = r;
+  a.proj = MOE_PROJ_DOWN; a.act = h; a.out = r; a.act_max = hmax; a.out_max = nullptr; a.prefetch_down = false;
   RNX_CUDA(mark(MOE_STAGE_EXPERT_DOWN, st), "stage event");
   RNX_CUDA(rnx::launch_nvfp4_gemv(a, st), "expert down");
   RNX_CUDA(mark(MOE_STAGE_SHARED, st), "stage event");

@@ -3,27 +3,25 @@
 // glm5next_mlp module docs, Constants / W4A16_GEMV_MODULE: at decode every
 // routed-expert projection is M=1, and a tile GEMM measured far below the
 // memory roofline there; the decode weight kernel must stream each touched
-// expert's bytes once at HBM speed. This kernel does exactly that:
+// expert's bytes once at HBM speed. Two forms:
 //
-//  * work item = (active local expert, block of 8*RPW output rows); a
-//    persistent grid loops over items;
-//  * each warp streams RPW weight rows with 128-bit non-allocating loads
-//    (lane l reads the 16-byte chunks l, l+32, ... of a row: 32 E2M1 codes,
-//    two 16-element scale blocks);
-//  * E2M1 pairs become f16x2 with the hardware cvt, and multiply-add into a
-//    per-16-block f16x2 partial against the activations (staged once per
-//    item in shared memory as f16, pre-scaled per row by a power of two so
-//    that |a| < 256: products are exact in f16, an 8-term half-block sum
-//    stays far inside the f16 range); each block partial is widened to fp32
-//    and scaled by its E4M3 block scale into an fp32 accumulator;
-//  * all tokens routed to the expert reuse the same weight registers.
+//  * one token per expert (T = 1, the decode step): the "direct" form below
+//    -- K split across warps, 8 weight rows in flight per warp, activations
+//    pre-scaled from a row max computed upstream;
+//  * several tokens per expert: a work-item loop over (active expert, block
+//    of rows) whose CTA stages the expert's token rows in shared memory once
+//    and applies each weight row to all of them.
 //
+// Both decode E2M1 pairs to f16x2 with the hardware cvt and multiply-add into
+// a per-16-element f16x2 partial against the activations (pre-scaled per row
+// by a power of two so that |a| < 256: products are exact in f16, an 8-term
+// half-block sum stays far inside the f16 range); each block partial is
+// widened to fp32 and scaled by its E4M3 block scale into an fp32 accumulator.
 // GATE_UP fuses the clamped SwiGLU and writes h (bf16) per assignment;
 // DOWN multiplies by the routing weight and writes r[t, j] (bf16).
 
 #include "common.cuh"
 #include "kernels.h"
-#include "tma.cuh"
 
 namespace rnx {
 
@@ -44,6 +42,7 @@ struct GemvParams {
   const int32_t* offsets;     // [E+1]
   const int32_t* sorted;      // [A]
   const int32_t* active;      // [E+1]
+  const int32_t* first;       // [E] first assignment of each active expert
   const float* weights;       // [A] routing weights (DOWN)
   const uint8_t* codes0;      // gate (GATE_UP) or down (DOWN) [E, rows, K/2]
   const uint8_t* scales0;     // [E, rows, K/16]
@@ -52,6 +51,11 @@ struct GemvParams {
   const uint8_t* scales1;
   const float* ts1;
   uint16_t* out;              // GATE_UP: h [A, rows]; DOWN: r [A, rows]
+  const uint32_t* act_max;    // direct form: max |activation row| (fp32 bits), by act row
+  uint32_t* out_max;          // direct GATE_UP: atomicMax of |h| per assignment (nullable)
+  const uint8_t* pf_codes;    // direct GATE_UP: down bank to prefetch into L2 (nullable)
+  const uint8_t* pf_scales;
+  long long pf_codes_per_expert, pf_scales_per_expert;
 };
 
 // Shared-memory activation layout: row m, 16-byte unit index
@@ -248,250 +252,234 @@ nvfp4_gemv_kernel(GemvParams p) {
 }
 
 // ---------------------------------------------------------------------------
-// Streaming form (few tokens per expert, the decode case): a producer warp
-// moves each work item -- S consecutive rows of one expert, which are
-// contiguous in HBM -- into a ring of shared-memory stages with bulk copies on
-// the TMA engine (cp.async.bulk, evict-first L2 policy), completion tracked by
-// mbarriers; 8 consumer warps compute from shared memory. A consumer lane
-// always owns the same 32-element K chunks (c = lane + 32 i), so the token's
-// activations stay in its registers as pre-scaled f16 for the whole kernel and
-// are reloaded only when the item's token set changes.
-constexpr int kStreamConsumers = 8;
-constexpr int kStreamThreads = (kStreamConsumers + 1) * kWarp;
+// Shared pieces of the one-token forms.
 
-struct StreamShape {
-  int S;            // rows per stage (row pairs for GATE_UP)
-  int NS;           // stages in the ring
-  uint32_t stage_bytes;
-};
+// 16 E2M1 code bytes (32 codes) -> 16 f16x2 words.
+RNX_DEVICE void decode_chunk(const uint4& q, uint32_t (&w)[16]) {
+  e2m1x8_to_f16x2x4(q.x, w[0], w[1], w[2], w[3]);
+  e2m1x8_to_f16x2x4(q.y, w[4], w[5], w[6], w[7]);
+  e2m1x8_to_f16x2x4(q.z, w[8], w[9], w[10], w[11]);
+  e2m1x8_to_f16x2x4(q.w, w[12], w[13], w[14], w[15]);
+}
 
-template <int MT, int NI, bool GATE_UP>
-__global__ void __launch_bounds__(kStreamThreads, 1)
-nvfp4_gemv_stream_kernel(GemvParams p, StreamShape sh, uint32_t* status) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ __align__(8) uint64_t full_bar[16];
-  __shared__ __align__(8) uint64_t empty_bar[16];
-  __shared__ volatile int abort_flag;
-  constexpr int NB = GATE_UP ? 2 : 1;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int S = sh.S, NS = sh.NS;
-  const int RW = S / kStreamConsumers;          // rows per consumer warp per stage
-  const int codes_row = p.K / 2, scales_row = p.K / 16;
-  const int nchunks = p.K / 32;
-  const int ipe = p.rows / S;
-  const int n_items = p.active[0] * ipe;
+// acc += s.x * (sum of the first 16 products) + s.y * (sum of the last 16)
+RNX_DEVICE void chunk_fma(const uint32_t (&w)[16], const uint32_t (&x)[16], float2 s, float& acc) {
+  __half2 p0 = __float2half2_rn(0.f), p1 = __float2half2_rn(0.f);
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    p0 = __hfma2(*reinterpret_cast<const __half2*>(&w[j]), *reinterpret_cast<const __half2*>(&x[j]), p0);
+#pragma unroll
+  for (int j = 8; j < 16; ++j)
+    p1 = __hfma2(*reinterpret_cast<const __half2*>(&w[j]), *reinterpret_cast<const __half2*>(&x[j]), p1);
+  const float2 f0 = __half22float2(p0), f1 = __half22float2(p1);
+  acc = fmaf(s.x, f0.x + f0.y, acc);
+  acc = fmaf(s.y, f1.x + f1.y, acc);
+}
 
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < NS; ++i) {
-      mbar_init(&full_bar[i], 1);
-      mbar_init(&empty_bar[i], kStreamConsumers);
-    }
-    abort_flag = 0;
-    fence_barrier_init();
-  }
-  __syncthreads();
+// Power-of-two pre-scale from a row's max |a|: max lands in [128, 256).
+RNX_DEVICE void prescale_from_max(float mx, float& up, float& unscale) {
+  int ex = 0;
+  if (mx > 0.f && mx <= 3.0e38f) frexpf(mx, &ex);
+  up = ldexpf(1.0f, 8 - ex);
+  unscale = ldexpf(1.0f, ex - 8);
+}
 
-  // stage layout: [bank0 codes S rows][bank1 codes][bank0 scales][bank1 scales]
-  auto stage_ptr = [&](int s) { return smem + (size_t)s * sh.stage_bytes; };
-
-  if (warp == kStreamConsumers) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      const uint64_t pol = policy_evict_first();
-      int it = 0;
-      for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it) {
-        const int s = it % NS;
-        const uint32_t ph = (uint32_t)(it / NS) & 1u;
-        if (!mbar_wait(&empty_bar[s], ph ^ 1u) || abort_flag) {
-          set_status(status, kDevErrTimeout);
-          abort_flag = 1;
-          break;
-        }
-        const int u = item / ipe, rb = item - u * ipe;
-        const int e = p.active[1 + u];
-        const size_t row0 = (size_t)e * p.rows + (size_t)rb * S;
-        uint8_t* st = stage_ptr(s);
-        mbar_arrive_expect_tx(&full_bar[s], sh.stage_bytes);
-        bulk_g2s(st, p.codes0 + row0 * codes_row, S * codes_row, &full_bar[s], pol);
-        if (GATE_UP) bulk_g2s(st + S * codes_row, p.codes1 + row0 * codes_row, S * codes_row, &full_bar[s], pol);
-        uint8_t* sc = st + NB * S * codes_row;
-        bulk_g2s(sc, p.scales0 + row0 * scales_row, S * scales_row, &full_bar[s], pol);
-        if (GATE_UP) bulk_g2s(sc + S * scales_row, p.scales1 + row0 * scales_row, S * scales_row, &full_bar[s], pol);
-      }
-      // drain: never leave the CTA with copies still writing its shared memory
-      const int issued = it;
-      for (int j = max(0, issued - NS); j < issued; ++j) {
-        if (!mbar_wait(&full_bar[j % NS], (uint32_t)(j / NS) & 1u)) set_status(status, kDevErrTimeout);
-      }
-    }
-    return;
-  }
-
-  // -------------------------------------------------------------- consumers
-  uint32_t xr[MT][NI][16];        // activations, f16x2, pre-scaled
-  float unscale[MT];
-  int key[MT];
+// This lane's 32-element chunk c of an activation row, pre-scaled, as f16x2.
+RNX_DEVICE void load_act_chunk(const uint16_t* row, int c, bool on, float up, uint32_t (&xr)[16]) {
 #pragma unroll
-  for (int m = 0; m < MT; ++m) key[m] = -1;
-
-  int it = 0;
-  for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it) {
-    const int s = it % NS;
-    const uint32_t ph = (uint32_t)(it / NS) & 1u;
-    const int u = item / ipe, rb = item - u * ipe;
-    const int e = p.active[1 + u];
-    const int seg0 = p.offsets[e];
-    const int nm = min(MT, p.offsets[e + 1] - seg0);
-
-    // (re)load this expert's activation rows into registers while the stage lands
+  for (int q = 0; q < 4; ++q) {
+    const uint4 v = on ? *reinterpret_cast<const uint4*>(row + 32 * c + 8 * q) : make_uint4(0, 0, 0, 0);
+    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      if (m < nm) {
-        const int a = p.sorted[seg0 + m];
-        const int src = GATE_UP ? a / p.k : a;
-        if (src != key[m]) {
-          key[m] = src;
-          const uint16_t* row = p.act + (size_t)src * p.K;
-          uint4 raw[NI][4];
-          float mx = 0.f;
-#pragma unroll
-          for (int i = 0; i < NI; ++i) {
-            const int c = i * 32 + lane;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              raw[i][q] = c < nchunks ? *reinterpret_cast<const uint4*>(row + 32 * c + 8 * q) : make_uint4(0, 0, 0, 0);
-              const uint32_t w4[4] = {raw[i][q].x, raw[i][q].y, raw[i][q].z, raw[i][q].w};
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const float2 f = bf16x2_to_f32x2(w4[j]);
-                mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
-              }
-            }
-          }
-          mx = warp_max(mx);
-          int ex = 0;
-          if (mx > 0.f && mx <= 3.0e38f) frexpf(mx, &ex);
-          const float upv = ldexpf(1.0f, 8 - ex);
-          unscale[m] = ldexpf(1.0f, ex - 8);
-#pragma unroll
-          for (int i = 0; i < NI; ++i)
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint32_t w4[4] = {raw[i][q].x, raw[i][q].y, raw[i][q].z, raw[i][q].w};
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const float2 f = bf16x2_to_f32x2(w4[j]);
-                __half2 h = __floats2half2_rn(f.x * upv, f.y * upv);
-                xr[m][i][4 * q + j] = *reinterpret_cast<uint32_t*>(&h);
-              }
-            }
-        }
-      }
-    }
-
-    if (!mbar_wait(&full_bar[s], ph) || abort_flag) {
-      set_status(status, kDevErrTimeout);
-      abort_flag = 1;
-      break;
-    }
-    const uint8_t* st = stage_ptr(s);
-    const uint8_t* sc = st + NB * S * codes_row;
-    for (int r = 0; r < RW; ++r) {
-      const int lr = warp * RW + r;                       // row within the stage
-      float acc[NB][MT];
-#pragma unroll
-      for (int b = 0; b < NB; ++b)
-#pragma unroll
-        for (int m = 0; m < MT; ++m) acc[b][m] = 0.f;
-#pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        const uint8_t* crow = st + (size_t)(b * S + lr) * codes_row;
-        const uint8_t* srow = sc + (size_t)(b * S + lr) * scales_row;
-#pragma unroll
-        for (int i = 0; i < NI; ++i) {
-          const int c = i * 32 + lane;
-          if (c < nchunks) {
-            const uint4 q = *reinterpret_cast<const uint4*>(crow + 16 * c);
-            const uint16_t sv = *reinterpret_cast<const uint16_t*>(srow + 2 * c);
-            uint32_t w[16];
-            e2m1x8_to_f16x2x4(q.x, w[0], w[1], w[2], w[3]);
-            e2m1x8_to_f16x2x4(q.y, w[4], w[5], w[6], w[7]);
-            e2m1x8_to_f16x2x4(q.z, w[8], w[9], w[10], w[11]);
-            e2m1x8_to_f16x2x4(q.w, w[12], w[13], w[14], w[15]);
-            const float2 scl = e4m3x2_to_f32x2(sv);
-#pragma unroll
-            for (int m = 0; m < MT; ++m) {
-              __half2 p0 = __float2half2_rn(0.f), p1 = __float2half2_rn(0.f);
-#pragma unroll
-              for (int j = 0; j < 8; ++j)
-                p0 = __hfma2(*reinterpret_cast<const __half2*>(&w[j]), *reinterpret_cast<const __half2*>(&xr[m][i][j]), p0);
-#pragma unroll
-              for (int j = 8; j < 16; ++j)
-                p1 = __hfma2(*reinterpret_cast<const __half2*>(&w[j]), *reinterpret_cast<const __half2*>(&xr[m][i][j]), p1);
-              const float2 f0 = __half22float2(p0), f1 = __half22float2(p1);
-              acc[b][m] = fmaf(scl.x, f0.x + f0.y, acc[b][m]);
-              acc[b][m] = fmaf(scl.y, f1.x + f1.y, acc[b][m]);
-            }
-          }
-        }
-      }
-      const int row = rb * S + lr;
-#pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        float tot[NB];
-#pragma unroll
-        for (int b = 0; b < NB; ++b) tot[b] = warp_sum(acc[b][m]);
-        if (lane == 0 && m < nm) {
-          const int a = p.sorted[seg0 + m];
-          if (GATE_UP) {
-            const float g = tot[0] * unscale[m] * p.ts0[e];
-            const float uu = tot[NB - 1] * unscale[m] * p.ts1[e];
-            p.out[(size_t)a * p.rows + row] = f32_to_bf16_bits(clamped_swiglu(g, uu, p.limit));
-          } else {
-            p.out[(size_t)a * p.rows + row] = f32_to_bf16_bits(tot[0] * unscale[m] * p.ts0[e] * p.weights[a]);
-          }
-        }
-      }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty_bar[s]);
-  }
-
-  if (!GATE_UP) {
-    // remote assignments contribute zero rows
-    const int rb0 = p.offsets[p.local_begin], re0 = p.offsets[p.local_end], rend = p.offsets[p.E];
-    const int nremote = rb0 + (rend - re0);
-    const int rows16 = p.rows / 8;
-    const int tid = threadIdx.x;   // consumers only: 256 threads
-    for (long long idx = (long long)blockIdx.x * (kStreamConsumers * kWarp) + tid; idx < (long long)nremote * rows16;
-         idx += (long long)gridDim.x * (kStreamConsumers * kWarp)) {
-      const int rp = (int)(idx / rows16), col = (int)(idx - (long long)rp * rows16);
-      const int pos = rp < rb0 ? rp : re0 + (rp - rb0);
-      const int a = p.sorted[pos];
-      reinterpret_cast<uint4*>(p.out + (size_t)a * p.rows)[col] = make_uint4(0, 0, 0, 0);
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = bf16x2_to_f32x2(w4[j]);
+      __half2 h = __floats2half2_rn(f.x * up, f.y * up);
+      xr[4 * q + j] = *reinterpret_cast<uint32_t*>(&h);
     }
   }
 }
 
-template <int MT, int NI, bool GU>
-cudaError_t launch_stream(const GemvParams& p, int max_items, uint32_t* status, cudaStream_t st) {
-  StreamShape sh;
-  const int codes_row = p.K / 2, scales_row = p.K / 16;
-  const int nb = GU ? 2 : 1;
-  sh.S = GU ? kStreamConsumers : 4 * kStreamConsumers;
-  sh.stage_bytes = (uint32_t)(nb * sh.S * (codes_row + scales_row));
-  const size_t budget = 200 * 1024;
-  sh.NS = (int)std::min<size_t>(16, budget / sh.stage_bytes);
-  const size_t smem = (size_t)sh.NS * sh.stage_bytes;
-  auto kern = nvfp4_gemv_stream_kernel<MT, NI, GU>;
-  static size_t cached = 0;
-  if (cached != smem) {
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
-    cached = smem;
+// Sum N per-lane values over the warp (N a power of two <= 32): afterwards
+// lane l holds the total of value l / (32 / N); lanes that are multiples of
+// 32 / N hold values 0, 1, ..., N-1. log2(N) exchange steps at distances
+// 16, 8, ... each halve the values a lane holds; plain butterflies finish.
+template <int N>
+RNX_DEVICE float warp_reduce_rows(float (&v)[N]) {
+  const int lane = threadIdx.x & 31;
+  int cnt = N;
+#pragma unroll
+  for (int d = 16; d >= 1; d >>= 1) {
+    if (cnt > 1) {
+      const int h = cnt >> 1;
+      const bool hi = lane & d;
+#pragma unroll
+      for (int i = 0; i < (N > 1 ? N / 2 : 1); ++i) {
+        if (i < h) {
+          const float send = hi ? v[i] : v[i + h];
+          const float keep = hi ? v[i + h] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, d);
+        }
+      }
+      cnt = h;
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], d);
+    }
   }
-  const int grid = std::max(1, std::min(max_items, kNumSMs));
-  kern<<<grid, kStreamThreads, smem, st>>>(p, sh, status);
+  return v[0];
+}
+
+// ---------------------------------------------------------------------------
+// Direct form for one token per expert (T = 1 decode). One CTA owns a block
+// of consecutive rows of one expert. K is split across warps: warp w works on
+// chunk group kg = w % NI (lanes own chunks c = 32 kg + lane), so it needs only
+// 16 registers of activations, and keeps 8 weight rows in flight: all of its
+// 128-bit weight loads are issued first, then its activation chunk is fetched
+// and pre-scaled from the row's max |a| (computed upstream: by the router for
+// x, by the gate/up pass for h). Row sums are reduced across each warp
+// together (9 shuffles for 8 rows); the NI partial sums of a row are combined
+// in shared memory in fixed order (deterministic). GATE_UP publishes the max
+// |h| of its assignment (atomicMax on the bit patterns of non-negative floats,
+// exact and order-independent) for the DOWN pass.
+constexpr int kDirectWarps = 8;
+constexpr int kDirectRows = 8;        // weight rows per warp
+
+template <int NI, bool GATE_UP>
+__global__ void __launch_bounds__(kDirectWarps * kWarp, 3)
+nvfp4_gemv_direct_kernel(GemvParams p) {
+  constexpr int RG = kDirectWarps / NI;                  // row groups per CTA
+  constexpr int PAIRS = GATE_UP ? kDirectRows / 2 : 0;   // gate/up pairs per row group
+  constexpr int CTA_ROWS = GATE_UP ? RG * PAIRS : RG * kDirectRows;   // output rows per CTA
+  __shared__ float s_part[NI][RG * kDirectRows];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kg = warp % NI, rg = warp / NI;
+  const int nchunks = p.K / 32;
+  const int codes_row = p.K / 2, scales_row = p.K / 16;
+  const int bpe = (p.rows + CTA_ROWS - 1) / CTA_ROWS;
+  const int u = blockIdx.x / bpe, blk = blockIdx.x - u * bpe;
+  if (u >= p.active[0]) return;
+  // one round trip for the expert and its single assignment, one for the rest
+  const int e = p.active[1 + u];
+  const int a = p.first[u];
+  const int row0 = blk * CTA_ROWS;
+  const float ts0 = p.ts0[e], ts1 = GATE_UP ? p.ts1[e] : 0.f;
+  const float wt = GATE_UP ? 0.f : p.weights[a];
+  const int c = kg * 32 + lane;
+  const bool lane_on = c < nchunks;
+  if (GATE_UP && p.pf_codes && threadIdx.x == 0) {
+    // this CTA's share of the same expert's DOWN weights, pulled into L2 while
+    // the gate/up rows stream (the down pass then reads them from L2)
+    const long long pc = p.pf_codes_per_expert, ps = p.pf_scales_per_expert;
+    const long long c0 = (pc * blk / bpe) & ~15ll, c1 = (pc * (blk + 1) / bpe) & ~15ll;
+    const long long s0 = (ps * blk / bpe) & ~15ll, s1 = (ps * (blk + 1) / bpe) & ~15ll;
+    if (c1 > c0) prefetch_l2(p.pf_codes + (size_t)e * pc + c0, (uint32_t)(c1 - c0));
+    if (s1 > s0) prefetch_l2(p.pf_scales + (size_t)e * ps + s0, (uint32_t)(s1 - s0));
+  }
+
+  // 1. weight loads: 8 rows per warp (GATE_UP: 4 gate rows then 4 up rows)
+  uint4 q[kDirectRows];
+  uint16_t sv[kDirectRows];
+#pragma unroll
+  for (int r = 0; r < kDirectRows; ++r) {
+    int row;
+    const uint8_t *cb, *sb;
+    if (GATE_UP) {
+      row = row0 + rg * PAIRS + (r % PAIRS);
+      cb = r < PAIRS ? p.codes0 : p.codes1;
+      sb = r < PAIRS ? p.scales0 : p.scales1;
+    } else {
+      row = row0 + rg * kDirectRows + r;
+      cb = p.codes0;
+      sb = p.scales0;
+    }
+    const bool on = lane_on && row < p.rows;
+    const size_t gr = (size_t)e * p.rows + row;
+    q[r] = on ? ldg_stream(cb + gr * codes_row + 16 * c) : make_uint4(0, 0, 0, 0);
+    sv[r] = on ? ldg_u16(sb + gr * scales_row + 2 * c) : (uint16_t)0;
+  }
+
+  // 2. this lane's 32-element activation chunk (x token for GATE_UP, h row
+  //    for DOWN) straight from global/L2, pre-scaled by the power of two that
+  //    brings the row's max |a| (supplied) into [128, 256)
+  const uint16_t* arow = p.act + (size_t)(GATE_UP ? a / p.k : a) * p.K;
+  float up, unscale;
+  prescale_from_max(__uint_as_float(p.act_max[GATE_UP ? a / p.k : a]), up, unscale);
+  uint32_t xr[16];
+  load_act_chunk(arow, c, lane_on, up, xr);
+
+  float acc[kDirectRows];
+#pragma unroll
+  for (int r = 0; r < kDirectRows; ++r) {
+    acc[r] = 0.f;
+    uint32_t w[16];
+    decode_chunk(q[r], w);
+    chunk_fma(w, xr, e4m3x2_to_f32x2(sv[r]), acc[r]);
+  }
+  const float tot = warp_reduce_rows<kDirectRows>(acc);   // lane 4r holds row slot r
+  const int r = lane >> 2;
+
+  if (GATE_UP) {
+    if ((lane & 3) == 0) s_part[kg][rg * kDirectRows + r] = tot;
+    __syncthreads();
+    if (threadIdx.x < RG * PAIRS) {
+      const int gq = threadIdx.x / PAIRS, pr = threadIdx.x % PAIRS;
+      const int row = row0 + gq * PAIRS + pr;
+      if (row < p.rows) {
+        float g = 0.f, uu = 0.f;
+#pragma unroll
+        for (int k = 0; k < NI; ++k) {
+          g += s_part[k][gq * kDirectRows + pr];
+          uu += s_part[k][gq * kDirectRows + PAIRS + pr];
+        }
+        g *= unscale * ts0;
+        uu *= unscale * ts1;
+        const uint16_t hb = f32_to_bf16_bits(clamped_swiglu(g, uu, p.limit));
+        p.out[(size_t)a * p.rows + row] = hb;
+        if (p.out_max) atomicMax(p.out_max + a, __float_as_uint(fabsf(bf16_bits_to_f32(hb))));
+      }
+    }
+  } else if (NI == 1) {
+    const int row = row0 + rg * kDirectRows + r;
+    if ((lane & 3) == 0 && row < p.rows)
+      p.out[(size_t)a * p.rows + row] = f32_to_bf16_bits(tot * unscale * ts0 * wt);
+  } else {
+    if ((lane & 3) == 0) s_part[kg][rg * kDirectRows + r] = tot;
+    __syncthreads();
+    if (threadIdx.x < RG * kDirectRows) {
+      const int row = row0 + threadIdx.x;
+      if (row < p.rows) {
+        float o = 0.f;
+#pragma unroll
+        for (int k = 0; k < NI; ++k) o += s_part[k][threadIdx.x];
+        p.out[(size_t)a * p.rows + row] = f32_to_bf16_bits(o * unscale * ts0 * wt);
+      }
+    }
+  }
+}
+
+// remote assignments of the DOWN projection contribute zero rows
+__global__ void __launch_bounds__(256) zero_remote_rows(GemvParams p) {
+  const int rb0 = p.offsets[p.local_begin], re0 = p.offsets[p.local_end], rend = p.offsets[p.E];
+  const int nremote = rb0 + (rend - re0);
+  const int rows16 = p.rows / 8;
+  for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < (long long)nremote * rows16;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const int rp = (int)(idx / rows16), col = (int)(idx - (long long)rp * rows16);
+    const int pos = rp < rb0 ? rp : re0 + (rp - rb0);
+    const int as = p.sorted[pos];
+    reinterpret_cast<uint4*>(p.out + (size_t)as * p.rows)[col] = make_uint4(0, 0, 0, 0);
+  }
+}
+
+template <int NI, bool GU>
+cudaError_t launch_direct(const GemvParams& p, int max_active, bool has_remote, cudaStream_t st) {
+  constexpr int RG = kDirectWarps / NI;
+  constexpr int CTA_ROWS = GU ? RG * (kDirectRows / 2) : RG * kDirectRows;
+  const int bpe = (p.rows + CTA_ROWS - 1) / CTA_ROWS;
+  const int grid = std::max(1, max_active * bpe);
+  nvfp4_gemv_direct_kernel<NI, GU><<<grid, kDirectWarps * kWarp, 0, st>>>(p);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess || GU || !has_remote) return err;
+  zero_remote_rows<<<kNumSMs, 256, 0, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -533,6 +521,7 @@ cudaError_t launch_nvfp4_gemv(const ExpertGemvArgs& a, cudaStream_t st) {
   p.offsets = a.offsets;
   p.sorted = a.sorted;
   p.active = a.active;
+  p.first = a.first;
   p.weights = a.weights;
   if (gu) {
     p.codes0 = a.gate.codes; p.scales0 = a.gate.scales; p.ts0 = a.gate.tensor_scale;
@@ -542,25 +531,23 @@ cudaError_t launch_nvfp4_gemv(const ExpertGemvArgs& a, cudaStream_t st) {
     p.codes1 = nullptr;      p.scales1 = nullptr;       p.ts1 = nullptr;
   }
   p.out = a.out;
+  p.act_max = a.act_max;
+  p.out_max = a.out_max;
+  if (gu && a.prefetch_down && a.down.codes) {
+    p.pf_codes = a.down.codes;
+    p.pf_scales = a.down.scales;
+    p.pf_codes_per_expert = (long long)a.H * a.I / 2;
+    p.pf_scales_per_expert = (long long)a.H * a.I / 16;
+  }
   const int max_active = std::min(a.local_end - a.local_begin, p.A);
   const int max_tok = a.T;   // tokens per expert never exceed T (ids in a row are distinct)
   const int NI = (p.K / 32 + 31) / 32;
-  const int S = gu ? kStreamConsumers : 4 * kStreamConsumers;
-  const bool stream_ok = (p.rows % S) == 0 && (size_t)(gu ? 2 : 1) * S * (p.K / 2 + p.K / 16) * 2 <= 200 * 1024;
-  if (stream_ok && max_tok * NI <= 4) {
-    const int items = std::max(1, max_active * (p.rows / S));
-    if (gu) {
-      if (max_tok == 1 && NI == 4) return launch_stream<1, 4, true>(p, items, a.status, st);
-      if (max_tok == 1 && NI <= 2) return launch_stream<1, 2, true>(p, items, a.status, st);
-      if (max_tok == 1) return launch_stream<1, 1, true>(p, items, a.status, st);
-      if (max_tok == 2 && NI <= 2) return launch_stream<2, 2, true>(p, items, a.status, st);
-    } else {
-      if (NI == 1 && max_tok == 1) return launch_stream<1, 1, false>(p, items, a.status, st);
-      if (NI == 1 && max_tok == 2) return launch_stream<2, 1, false>(p, items, a.status, st);
-      if (NI == 1) return launch_stream<4, 1, false>(p, items, a.status, st);
-      if (NI == 2 && max_tok <= 2) return launch_stream<2, 2, false>(p, items, a.status, st);
-      if (NI <= 4 && max_tok == 1) return launch_stream<1, 4, false>(p, items, a.status, st);
-    }
+  if (max_tok == 1 && a.act_max && p.K <= 8192) {
+    const bool remote = a.local_begin > 0 || a.local_end < a.E;
+    if (NI == 1) return gu ? launch_direct<1, true>(p, max_active, remote, st) : launch_direct<1, false>(p, max_active, remote, st);
+    if (NI == 2) return gu ? launch_direct<2, true>(p, max_active, remote, st) : launch_direct<2, false>(p, max_active, remote, st);
+    if (NI <= 4) return gu ? launch_direct<4, true>(p, max_active, remote, st) : launch_direct<4, false>(p, max_active, remote, st);
+    return gu ? launch_direct<8, true>(p, max_active, remote, st) : launch_direct<8, false>(p, max_active, remote, st);
   }
   if (gu) {
     const int ipe = p.rows / (kGemvWarps * 1);

@@ -19,17 +19,25 @@ struct ExpertGemvArgs {
   const int32_t* offsets;
   const int32_t* sorted;
   const int32_t* active;
+  const int32_t* first;     // plan.first: first assignment of each active expert
   const float* weights;
   nvfp4_bank_t gate, up, down;
   uint16_t* out;
   uint32_t* status;         // device status word (bounded-wait timeouts)
+  const uint32_t* act_max;  // optional: max |activation row| as fp32 bits (x rows by token / h rows by assignment)
+  uint32_t* out_max;        // optional (GATE_UP): receives max |h| per assignment; must start at 0
+  bool prefetch_down;       // GATE_UP (one token per expert): pull the experts' down weights into L2
 };
 
 cudaError_t launch_nvfp4_gemv(const ExpertGemvArgs& a, cudaStream_t st);
 
 // router
+// xmax (nullable): receives max |x_t| per token as fp32 bits; zero (nullable):
+// nzero uint32 words set to 0 (the h-max array of the next expert pass).
 cudaError_t launch_router_logits(const uint16_t* x, int T, int H, int E, const float* wr, float* logits,
-                                 cudaStream_t st);
+                                 cudaStream_t st, uint32_t* xmax = nullptr, uint32_t* zero = nullptr, int nzero = 0);
+// max |row| as fp32 bits for R rows of K bf16 elements
+cudaError_t launch_row_absmax(const uint16_t* rows, int R, int K, uint32_t* out, cudaStream_t st);
 cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, int k, float rsf, int32_t* ids,
                         float* weights, cudaStream_t st);
 

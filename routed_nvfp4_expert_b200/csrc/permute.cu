@@ -76,6 +76,21 @@ RNX_DEVICE void finish_plan(const int* s_cnt, int E, int lb, int le, const moe_p
   }
 }
 
+// first[u] = sorted[offsets[e]] for the u-th active (local, non-empty) expert e.
+// Runs after sorted[] is complete; reads offsets/active/sorted from the plan.
+RNX_DEVICE void write_first(const moe_plan_t& plan, const int* s_off, const int* s_cnt, int E, int lb, int le) {
+  const int n_active = plan.active[0];
+  for (int u = threadIdx.x; u < n_active; u += blockDim.x) {
+    const int e = plan.active[1 + u];
+    plan.first[u] = plan.sorted[plan.offsets[e]];
+  }
+  (void)s_off;
+  (void)s_cnt;
+  (void)E;
+  (void)lb;
+  (void)le;
+}
+
 __global__ void __launch_bounds__(1024) permute_small(const int32_t* __restrict__ ids, int A, int E, int lb, int le,
                                                       moe_plan_t plan, uint32_t* status) {
   __shared__ int s_ids[kSmallMaxA];
@@ -116,6 +131,8 @@ __global__ void __launch_bounds__(1024) permute_small(const int32_t* __restrict_
       }
     }
   }
+  __syncthreads();
+  write_first(plan, s_off, s_cnt, E, lb, le);
 }
 
 // ---- large A
@@ -207,6 +224,14 @@ __global__ void __launch_bounds__(kChunk) permute_scatter(const int32_t* __restr
   plan.inv[a] = pos;
 }
 
+__global__ void __launch_bounds__(256) permute_first(moe_plan_t plan) {
+  const int n_active = plan.active[0];
+  for (int u = blockIdx.x * blockDim.x + threadIdx.x; u < n_active; u += gridDim.x * blockDim.x) {
+    const int e = plan.active[1 + u];
+    plan.first[u] = plan.sorted[plan.offsets[e]];
+  }
+}
+
 }  // namespace
 
 size_t permute_scratch_ints(int A, int E) {
@@ -226,6 +251,7 @@ cudaError_t launch_permute(const int32_t* ids, int A, int E, int lb, int le, con
   permute_hist<<<nb, kChunk, 8 * E * sizeof(int), st>>>(ids, A, E, rank, hist, status);
   permute_scan<<<1, 1024, 0, st>>>(nb, E, lb, le, hist, plan);
   permute_scatter<<<nb, kChunk, 0, st>>>(ids, A, E, rank, hist, plan);
+  permute_first<<<(E + 255) / 256, 256, 0, st>>>(plan);
   return cudaGetLastError();
 }
 

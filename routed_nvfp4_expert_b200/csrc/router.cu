@@ -12,46 +12,82 @@ namespace {
 
 // ---------------------------------------------------------------- logits
 // Small T (decode): the fp32 router matrix (E x H, 4.7 MB at E=288, H=4096)
-// is the only real traffic. Half a CTA (128 threads) owns one expert row and
-// streams it with 128-bit loads; tokens are taken 8 at a time.
+// is the only real traffic. One 128-thread CTA owns one expert row: every
+// thread issues all of its 128-bit weight loads up front (H/512 of them), then
+// multiplies them against the tokens, 8 tokens per pass.
 constexpr int kLogitTokens = 8;
+constexpr int kLogitThreads = 128;
+constexpr int kLogitMaxQ = 16;     // H <= 8192 in this form
 
-__global__ void __launch_bounds__(256) router_logits_gemv(const uint16_t* __restrict__ x, int T, int H, int E,
-                                                          const float* __restrict__ wr, float* __restrict__ logits) {
-  const int half = threadIdx.x >> 7, t128 = threadIdx.x & 127, warp4 = t128 >> 5, lane = threadIdx.x & 31;
-  const int e = blockIdx.x * 2 + half;
-  const bool valid = e < E;
+__global__ void __launch_bounds__(kLogitThreads) router_logits_gemv(const uint16_t* __restrict__ x, int T, int H, int E,
+                                                                   const float* __restrict__ wr,
+                                                                   float* __restrict__ logits, uint32_t* xmax,
+                                                                   uint32_t* zero, int nzero) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int e = blockIdx.x;
   const int nq = H >> 2;
-  __shared__ float red[2][4][kLogitTokens];
-  const float4* wrow = reinterpret_cast<const float4*>(wr + (size_t)(valid ? e : 0) * H);
+  __shared__ float red[4][kLogitTokens];
+  if (e == 0) {
+    // side jobs of CTA 0: max |x_t| per token (fp32 bits; the expert pass
+    // pre-scales with it) and clearing the h-max array the gate/up pass fills
+    for (int i = tid; i < nzero; i += kLogitThreads) zero[i] = 0u;
+    if (xmax) {
+      for (int t = 0; t < T; ++t) {
+        float m = 0.f;
+        for (int g = tid; g < H / 8; g += kLogitThreads) {
+          const uint4 v = reinterpret_cast<const uint4*>(x + (size_t)t * H)[g];
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 f = bf16x2_to_f32x2(w4[j]);
+            m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+          }
+        }
+        m = warp_max(m);
+        if (lane == 0) red[warp][0] = m;
+        __syncthreads();
+        if (tid == 0) xmax[t] = __float_as_uint(fmaxf(fmaxf(red[0][0], red[1][0]), fmaxf(red[2][0], red[3][0])));
+        __syncthreads();
+      }
+    }
+  }
+  const float4* wrow = reinterpret_cast<const float4*>(wr + (size_t)e * H);
+  float4 w[kLogitMaxQ];
+#pragma unroll
+  for (int i = 0; i < kLogitMaxQ; ++i) {
+    const int c = tid + kLogitThreads * i;
+    w[i] = c < nq ? __ldg(wrow + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   for (int t0 = 0; t0 < T; t0 += kLogitTokens) {
     float acc[kLogitTokens];
 #pragma unroll
-    for (int t = 0; t < kLogitTokens; ++t) acc[t] = 0.f;
-#pragma unroll 4
-    for (int c = t128; c < nq; c += 128) {
-      const float4 w = valid ? __ldg(wrow + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int t = 0; t < kLogitTokens; ++t) {
+      acc[t] = 0.f;
+      if (t0 + t < T) {
+        const uint16_t* xr = x + (size_t)(t0 + t) * H;
 #pragma unroll
-      for (int t = 0; t < kLogitTokens; ++t) {
-        if (t0 + t < T) {
-          const uint2 xv = *reinterpret_cast<const uint2*>(x + (size_t)(t0 + t) * H + 4 * c);
-          const float2 a = bf16x2_to_f32x2(xv.x), b = bf16x2_to_f32x2(xv.y);
-          acc[t] = fmaf(w.x, a.x, acc[t]);
-          acc[t] = fmaf(w.y, a.y, acc[t]);
-          acc[t] = fmaf(w.z, b.x, acc[t]);
-          acc[t] = fmaf(w.w, b.y, acc[t]);
+        for (int i = 0; i < kLogitMaxQ; ++i) {
+          const int c = tid + kLogitThreads * i;
+          if (c < nq) {
+            const uint2 xv = *reinterpret_cast<const uint2*>(xr + 4 * c);
+            const float2 a = bf16x2_to_f32x2(xv.x), b = bf16x2_to_f32x2(xv.y);
+            acc[t] = fmaf(w[i].x, a.x, acc[t]);
+            acc[t] = fmaf(w[i].y, a.y, acc[t]);
+            acc[t] = fmaf(w[i].z, b.x, acc[t]);
+            acc[t] = fmaf(w[i].w, b.y, acc[t]);
+          }
         }
       }
     }
 #pragma unroll
     for (int t = 0; t < kLogitTokens; ++t) {
       const float v = warp_sum(acc[t]);
-      if (lane == 0) red[half][warp4][t] = v;
+      if (lane == 0) red[warp][t] = v;
     }
     __syncthreads();
-    if (t128 < kLogitTokens && t0 + t128 < T && valid) {
-      const float v = ((red[half][0][t128] + red[half][1][t128]) + red[half][2][t128]) + red[half][3][t128];
-      logits[(size_t)(t0 + t128) * E + e] = v;
+    if (tid < kLogitTokens && t0 + tid < T) {
+      const float v = ((red[0][tid] + red[1][tid]) + red[2][tid]) + red[3][tid];
+      logits[(size_t)(t0 + tid) * E + e] = v;
     }
     __syncthreads();
   }
@@ -117,26 +153,42 @@ RNX_DEVICE bool better(const Cand& a, const Cand& b) {
   return a.idx < b.idx;
 }
 
+// 8 tokens per CTA. All 256 threads first evaluate the sigmoid scores and
+// selection keys of the CTA's tokens into shared memory; then one warp per
+// token selects its top-k.
+template <int PL>
+__host__ __device__ constexpr int topk_tokens() { return PL > 16 ? 2 : 8; }
+
 template <int PL>
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
                                                    int T, int E, int k, float rsf, int32_t* __restrict__ ids,
                                                    float* __restrict__ weights) {
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (t >= T) return;
+  constexpr int kTopkTokens = topk_tokens<PL>();
+  __shared__ float s_key[kTopkTokens][32 * PL];
+  __shared__ float s_sig[kTopkTokens][32 * PL];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int t0 = blockIdx.x * kTopkTokens;
+  const int ntok = min(kTopkTokens, T - t0);
+  for (int i = threadIdx.x; i < ntok * E; i += blockDim.x) {
+    const int tt = i / E, e = i - tt * E;
+    const float l = logits[(size_t)(t0 + tt) * E + e];
+    // sigmoid in double, rounded once to fp32; then an fp32 add of the bias
+    const float sg = (float)(1.0 / (1.0 + exp(-(double)l)));
+    s_sig[tt][e] = sg;
+    s_key[tt][e] = __fadd_rn(sg, bias[e]);
+  }
+  __syncthreads();
+  if (warp >= ntok) return;
+  const int t = t0 + warp;
   float key[PL], sg[PL];
   int st[PL];
 #pragma unroll
   for (int i = 0; i < PL; ++i) {
     const int e = lane + 32 * i;
     if (e < E) {
-      const float l = logits[(size_t)t * E + e];
-      // sigmoid in double, rounded once to fp32; then an fp32 add of the bias
-      const float s = (float)(1.0 / (1.0 + exp(-(double)l)));
-      const float kk = __fadd_rn(s, bias[e]);
-      sg[i] = s;
-      key[i] = kk;
-      st[i] = isnan(kk) ? 1 : 0;
+      key[i] = s_key[warp][e];
+      sg[i] = s_sig[warp][e];
+      st[i] = isnan(key[i]) ? 1 : 0;
     } else {
       sg[i] = 0.f;
       key[i] = 0.f;
@@ -181,12 +233,36 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
   }
 }
 
+__global__ void __launch_bounds__(256) row_absmax_kernel(const uint16_t* __restrict__ rows, int R, int K,
+                                                         uint32_t* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (r >= R) return;
+  float m = 0.f;
+  for (int g = lane; g < K / 8; g += 32) {
+    const uint4 v = reinterpret_cast<const uint4*>(rows + (size_t)r * K)[g];
+    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = bf16x2_to_f32x2(w4[j]);
+      m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+    }
+  }
+  m = warp_max(m);
+  if (lane == 0) out[r] = __float_as_uint(m);
+}
+
 }  // namespace
 
+cudaError_t launch_row_absmax(const uint16_t* rows, int R, int K, uint32_t* out, cudaStream_t st) {
+  row_absmax_kernel<<<(R + 7) / 8, 256, 0, st>>>(rows, R, K, out);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_router_logits(const uint16_t* x, int T, int H, int E, const float* wr, float* logits,
-                                 cudaStream_t st) {
-  if (T <= 64) {
-    router_logits_gemv<<<(E + 1) / 2, 256, 0, st>>>(x, T, H, E, wr, logits);
+                                 cudaStream_t st, uint32_t* xmax, uint32_t* zero, int nzero) {
+  if (T <= 64 && H <= 4 * kLogitThreads * kLogitMaxQ) {
+    router_logits_gemv<<<E, kLogitThreads, 0, st>>>(x, T, H, E, wr, logits, xmax, zero, nzero);
   } else {
     dim3 grid((E + kSgBN - 1) / kSgBN, (T + kSgBM - 1) / kSgBM);
     router_logits_sgemm<<<grid, 256, 0, st>>>(x, T, H, E, wr, logits);
@@ -196,10 +272,13 @@ cudaError_t launch_router_logits(const uint16_t* x, int T, int H, int E, const f
 
 cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, int k, float rsf, int32_t* ids,
                         float* weights, cudaStream_t st) {
-  const int grid = (T + 7) / 8;
-  if (E <= 32 * 4) topk_kernel<4><<<grid, 256, 0, st>>>(logits, bias, T, E, k, rsf, ids, weights);
-  else if (E <= 32 * 10) topk_kernel<10><<<grid, 256, 0, st>>>(logits, bias, T, E, k, rsf, ids, weights);
-  else topk_kernel<32><<<grid, 256, 0, st>>>(logits, bias, T, E, k, rsf, ids, weights);
+  auto grid = [T](int tpb) { return (T + tpb - 1) / tpb; };
+  if (E <= 32 * 4)
+    topk_kernel<4><<<grid(topk_tokens<4>()), 256, 0, st>>>(logits, bias, T, E, k, rsf, ids, weights);
+  else if (E <= 32 * 10)
+    topk_kernel<10><<<grid(topk_tokens<10>()), 256, 0, st>>>(logits, bias, T, E, k, rsf, ids, weights);
+  else
+    topk_kernel<32><<<grid(topk_tokens<32>()), 256, 0, st>>>(logits, bias, T, E, k, rsf, ids, weights);
   return cudaGetLastError();
 }
 

@@ -48,14 +48,33 @@ RNX_DEVICE bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity to complete.
-// Returns false if it did not complete within kWaitLimitNs.
+// try_wait that lets the hardware suspend the thread for up to hint_ns
+// before returning (no polling loop burning issue slots meanwhile).
+RNX_DEVICE bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity to complete. Polls with a
+// suspend hint; reads %globaltimer only every 1024 polls. Returns false if the
+// phase did not complete within kWaitLimitNs.
 RNX_DEVICE bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer_ns();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+  unsigned long long t0 = 0;
+  for (uint32_t i = 0;; ++i) {
+    if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
+    if ((i & 1023u) == 0) {
+      const unsigned long long t = globaltimer_ns();
+      if (i == 0) t0 = t;
+      else if (t - t0 > kWaitLimitNs) return false;
+    }
   }
 }
 
