@@ -311,6 +311,27 @@ moe_status_t moe_read_device_status(void* ws, void* stream);
 /* Thread-local description of the last failed call on this thread ("" if none). */
 const char* moe_last_error(void);
 
+/*
+ * Decode forward without a caller workspace -- no counterpart in the pages:
+ * it exists for callers that cannot allocate device memory (a memory pool or
+ * custom allocator that forbids cudaMalloc, a framework callback that may not
+ * allocate, a C host program holding only the device pointers of its tensors).
+ * Same computation and arguments as moe_forward(cfg, w, x, T,
+ * MOE_PATH_DECODE, y, ws, ws_bytes, stream), minus the workspace: the scratch
+ * is a library-owned 8 MiB device buffer that every GPU loading the library
+ * keeps until the process exits. Calls needing more than that
+ * (moe_workspace_size(cfg, T, MOE_PATH_DECODE) > 8 MiB) fail with
+ * MOE_ERR_WORKSPACE before touching the device. The first call on each device
+ * looks up the buffer's device address (cudaGetSymbolAddress, with that device
+ * current); make that first call before any stream capture on the device. All
+ * calls on a device share the buffer, which keeps the previous call's
+ * contents; calls whose GPU work overlaps in time (two streams, two host
+ * threads) race on it and must be serialised by the caller. Allocates nothing
+ * (no cudaMalloc / cudaFree). The routing intermediates are not exposed.
+ */
+moe_status_t moe_forward_decode_noalloc(const moe_config_t* cfg, const moe_weights_t* w, const uint16_t* x,
+                                        int32_t T, uint16_t* y, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -27,7 +27,7 @@ EXPORTED = (
     "moe_workspace_size", "moe_plan_size", "moe_plan_carve", "moe_router_topk", "moe_permute",
     "nvfp4_expert_gemv", "clamped_swiglu", "moe_combine", "dense_ffn_workspace_size", "dense_ffn_bf16",
     "nvfp4_dequant", "moe_forward", "moe_workspace_views", "moe_read_device_status", "moe_last_error",
-    "moe_set_stage_events",
+    "moe_set_stage_events", "moe_forward_decode_noalloc",
 )
 STAGES = ("router_logits", "topk", "permute", "act_quant", "expert_gate_up", "h_quant", "expert_down", "shared",
           "combine")
@@ -89,6 +89,7 @@ def load_library(path: str = _LIB_PATH) -> C.CDLL:
         "moe_read_device_status": (st, [vp, vp]),
         "moe_last_error": (C.c_char_p, []),
         "moe_set_stage_events": (st, [C.POINTER(C.c_void_p), i32]),
+        "moe_forward_decode_noalloc": (st, [cfgp, C.POINTER(MoeWeights), vp, i32, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -256,6 +257,14 @@ def moe_forward(cfg: SiteConfig, site: DeviceSite, x, path: int, y, ws, stream=N
     w = w_c if w_c is not None else site.c()
     _check(lib().moe_forward(C.byref(cfg.c()), C.byref(w), _p(x), x.shape[0], path, _p(y), _p(ws), ws.numel(),
                              _stream(stream)))
+
+
+def moe_forward_decode_noalloc(cfg: SiteConfig, site: DeviceSite, x, y, stream=None):
+    """Decode forward on the library's own 8 MiB device scratch buffer (for
+    callers that cannot allocate a workspace); see the C header."""
+    w = site.c()
+    _check(lib().moe_forward_decode_noalloc(C.byref(cfg.c()), C.byref(w), _p(x), x.shape[0], _p(y),
+                                            _stream(stream)))
 
 
 def moe_workspace_views(cfg: SiteConfig, T: int, path: int, ws) -> MoeViews:

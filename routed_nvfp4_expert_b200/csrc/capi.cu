@@ -6,6 +6,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -455,6 +456,62 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
   RNX_CUDA(rnx::launch_combine(T, k, H, r, shared, y, st), "combine");
   RNX_CUDA(mark(MOE_STAGE_COUNT, st), "stage event");
   return MOE_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Decode forward for callers that cannot allocate device memory.
+//
+// Some callers have no way to hand this library a workspace: code running
+// where the CUDA allocator must not be touched (a memory pool or custom
+// allocator owns every byte and forbids cudaMalloc, or a framework callback
+// that may not allocate), or a plain C host program that holds only the device
+// pointers of its tensors. moe_forward_decode_noalloc runs the same decode
+// forward as moe_forward(..., MOE_PATH_DECODE, ...) but takes its scratch from
+// one buffer that lives in this library: g_noalloc_scratch below, 8 MiB, which
+// every GPU that loads the library keeps until the process exits.
+//
+// On the host the array's name denotes a host-side stand-in, not a device
+// address, so the first call on each device asks the runtime for the device
+// address with cudaGetSymbolAddress (that device current) and caches it; that
+// first call should come before any stream capture on the device. All calls
+// on a device share the buffer and it keeps what the last call left in it; the
+// forward clears what must start at zero (the status word, the h-max array)
+// itself. Calls whose GPU work overlaps in time -- on two streams or from two
+// host threads -- race on the buffer: serialise them on one stream.
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[8u << 20];
+
+namespace {
+constexpr size_t kNoAllocBytes = sizeof(g_noalloc_scratch);
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_dev[kNoAllocMaxDevices] = {};
+}  // namespace
+
+moe_status_t moe_forward_decode_noalloc(const moe_config_t* cfg, const moe_weights_t* w, const uint16_t* x,
+                                        int32_t T, uint16_t* y, void* stream) {
+  moe_status_t s;
+  if ((s = check_cfg(cfg)) != MOE_OK || (s = check_T(T)) != MOE_OK) return s;
+  const size_t need = ws_layout(cfg, T, MOE_PATH_DECODE).bytes;
+  if (need > kNoAllocBytes)
+    return fail(MOE_ERR_WORKSPACE, "moe_forward_decode_noalloc: T=%d needs %zu bytes of scratch, the built-in buffer "
+                "holds %zu", T, need, kNoAllocBytes);
+  if (T == 0) return MOE_OK;
+  int dev = 0;
+  RNX_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(MOE_ERR_UNSUPPORTED, "device %d out of range", dev);
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_dev[dev]) {
+      void* p = nullptr;
+      RNX_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress(noalloc scratch)");
+      if (!p) return fail(MOE_ERR_CUDA, "cudaGetSymbolAddress returned NULL");
+      g_noalloc_dev[dev] = p;
+    }
+    scratch = g_noalloc_dev[dev];
+  }
+  return moe_forward(cfg, w, x, T, MOE_PATH_DECODE, y, scratch, kNoAllocBytes, stream);
 }
 
 }  // extern "C"

@@ -94,3 +94,13 @@ def test_plan_carve_is_host_arithmetic():
     ptrs = [plan.counts, plan.offsets, plan.sorted, plan.inv, plan.tile_offsets, plan.active, plan.first]
     assert ptrs == sorted(ptrs) and all(p % 256 == 0 for p in ptrs) and ptrs[0] == 0x100000
     assert lib.moe_plan_carve(C.byref(cfg), 10, 0x100000, n - 1, C.byref(plan)) == 3
+
+
+def test_noalloc_rejects_oversized_requests_before_touching_the_device():
+    lib = capi.lib()
+    cfg = _cfg(hidden=4096, intermediate=1024, shared_intermediate=1024, num_experts=288, local_end=288, top_k=8).c()
+    need = lib.moe_workspace_size(C.byref(cfg), 4096, 0)
+    assert need > 8 << 20
+    w = capi.MoeWeights()
+    st = lib.moe_forward_decode_noalloc(C.byref(cfg), C.byref(w), 0x1000, 4096, 0x2000, None)
+    assert st == 3 and "built-in buffer" in lib.moe_last_error().decode()
