@@ -117,7 +117,10 @@ typedef struct {
 
 /* Weights of one routed site (Glm5NextMoeWeights), already sharded for this
  * rank. router_w fp32 [E, H] row-major; router_bias fp32 [E]; shared_* bf16
- * row-major: gate and up [Is, H], down [H, Is] (NULL when Is == 0). */
+ * row-major: gate and up [Is, H], down [H, Is] (NULL when Is == 0).
+ * prepared: the experts' block scales re-tiled by moe_prepare_weights()
+ * (moe_prepared_size() bytes) for the tensor-core prefill path; NULL is
+ * allowed when only MOE_PATH_DECODE runs. */
 typedef struct {
   const float* router_w;
   const float* router_bias;
@@ -127,6 +130,7 @@ typedef struct {
   const uint16_t* shared_gate;
   const uint16_t* shared_up;
   const uint16_t* shared_down;
+  const uint8_t* prepared;
 } moe_weights_t;
 
 /*
@@ -142,6 +146,12 @@ typedef struct {
  *                       active[1..] = their ids in ascending order
  *   first        [E]    first[u] = sorted[offsets[active[1+u]]], the first
  *                       assignment of the u-th active expert
+ *   tile_rows    [P]    P = moe_padded_rows(cfg, T): the padded tile layout
+ *                       of the prefill, in which every LOCAL expert's rows
+ *                       start on a 128-row tile (tile_offsets); tile_rows[p]
+ *                       is the assignment at padded row p, -1 for padding and
+ *                       for rows past the last tile. Filled by moe_permute
+ *                       and by the prefill path of moe_forward.
  */
 typedef struct {
   int32_t* counts;
@@ -151,6 +161,7 @@ typedef struct {
   int32_t* tile_offsets;
   int32_t* active;
   int32_t* first;
+  int32_t* tile_rows;
 } moe_plan_t;
 
 /* ------------------------------------------------------------------ sizes */
@@ -167,6 +178,30 @@ size_t moe_plan_size(const moe_config_t* cfg, int32_t T);
 /* Carve a plan out of one device buffer of moe_plan_size() bytes. Host-only
  * pointer arithmetic; launches nothing. */
 moe_status_t moe_plan_carve(const moe_config_t* cfg, int32_t T, void* buf, size_t bytes, moe_plan_t* plan);
+
+/* Rows P of the prefill's padded tile layout for T tokens: an upper bound on
+ * sum over local experts of ceil(counts/128) * 128, namely
+ * floor((A + 127 * min(A, E_local)) / 128) * 128 with A = T*k (0 on invalid
+ * arguments). Sizes tile_rows and the quantised activation buffers. */
+int64_t moe_padded_rows(const moe_config_t* cfg, int32_t T);
+
+/* Bytes of the prepared weights (the block scales of gate, up and down
+ * re-tiled into the 512-byte scale atoms of the tensor-core path):
+ * 3 * E * I * H / 16. */
+size_t moe_prepared_size(const moe_config_t* cfg);
+
+/*
+ * Re-tile the experts' block scales for the prefill path. dst (device,
+ * 256-byte aligned, moe_prepared_size() bytes) receives, for gate, then up,
+ * then down, the scales of each expert as atoms [rows/128][K/64][512]: the
+ * scale of row m, 16-element block b of atom (m/128, b/4) sits at byte
+ * (m%32)*16 + ((m%128)/32)*4 + b%4 (32 lanes x 4 columns x 4 blocks, the
+ * layout the 32x128b tensor-memory copy spreads over the four lane
+ * quadrants). Requires I % 128 == 0 and H % 256 == 0. Codes are used in
+ * place. Run once per weight set; stream-ordered.
+ */
+moe_status_t moe_prepare_weights(const moe_config_t* cfg, const moe_weights_t* w, void* dst, size_t dst_bytes,
+                                 void* stream);
 
 /* ------------------------------------------------------------ the steps */
 
@@ -188,9 +223,10 @@ moe_status_t moe_router_topk(const moe_config_t* cfg, const uint16_t* x, int32_t
 
 /*
  * Token sort (the module list's moe_permute family): builds `plan` from ids
- * int32 [T, k]. ids outside [0, E) set MOE_ERR_DEVICE_BOUNDS in the workspace
- * status word and are dropped. ws: workspace of at least
- * moe_workspace_size(cfg, T, MOE_PATH_PREFILL) bytes.
+ * int32 [T, k], including plan.tile_rows. ids outside [0, E) set
+ * MOE_ERR_DEVICE_BOUNDS in the workspace status word and are dropped.
+ * ws: workspace of at least moe_workspace_size(cfg, T, MOE_PATH_DECODE)
+ * bytes (status word and sort scratch).
  */
 moe_status_t moe_permute(const moe_config_t* cfg, const int32_t* ids, int32_t T,
                          const moe_plan_t* plan, void* ws, size_t ws_bytes, void* stream);
@@ -214,6 +250,45 @@ moe_status_t moe_permute(const moe_config_t* cfg, const int32_t* ids, int32_t T,
 moe_status_t nvfp4_expert_gemv(const moe_config_t* cfg, int32_t proj, const uint16_t* act, int32_t T,
                                const moe_plan_t* plan, const float* weights,
                                const moe_weights_t* w, uint16_t* out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * NVFP4 encoding of activation rows for the prefill (the reading of the
+ * glm5next_mlp module docs' forward_prefill_gemm as W4A4 on block-scaled FP4
+ * tensor cores; the pages' own prefill keeps activations in bf16). Every step
+ * in IEEE fp32, per row: r = max|row|, row_scale = r / 2688 (2688 = 6 * 448);
+ * per block of 16: sb = e4m3_rn_satfinite((amax_block / 6) / row_scale),
+ * d = e4m3(sb) * row_scale, code = e2m1_rn_satfinite(v / d). A zero row has
+ * row_scale 0 and all scales and codes 0; a block with d = 0 gets codes 0.
+ *   src       bf16 [rows, K], K a multiple of 64
+ *   codes     out [rows, K/2] (even element in the low nibble)
+ *   sf_atoms  out [ceil(rows/128)][K/64][512] in the atom layout of
+ *             moe_prepare_weights; rows past `rows` in the last tile get 0
+ *   row_scale out fp32 [rows]
+ */
+moe_status_t nvfp4_quantize_rows(const uint16_t* src, int32_t rows, int32_t K, uint8_t* codes, uint8_t* sf_atoms,
+                                 float* row_scale, void* stream);
+
+/*
+ * Prefill expert projections (the glm5next_mlp module docs'
+ * forward_prefill_gemm: the routed experts as one grouped GEMM over the
+ * tokens sorted by expert), here as W4A4 on tcgen05 block-scaled FP4
+ * (kind::mxf4nvf4, E4M3 scale per 16 on both operands, fp32 accumulation).
+ * The A operand is in the padded tile layout of plan.tile_rows, P =
+ * moe_padded_rows(cfg, T) rows: act_codes [P, K/2], act_sf atoms
+ * [P/128][K/64][512], act_scale fp32 [P] (from nvfp4_quantize_rows or the
+ * prefill of moe_forward); padding rows must be zero (codes, scales, scale).
+ *   MOE_PROJ_GATE_UP (K = H): out = h bf16 [P, I], h[p] = clamped_swiglu(
+ *       g, u) of padded row p (0 on padding rows); `weights` unused.
+ *   MOE_PROJ_DOWN (K = I): out = r bf16 [T*k, H], r[a] = weights[a] *
+ *       (down_e . hdeq[p]) for the padded row p of assignment a; rows of
+ *       remote assignments are written as zeros.
+ *   Requires w->prepared, I % 128 == 0, H % 256 == 0.
+ *   ws: at least moe_workspace_size(cfg, T, MOE_PATH_PREFILL) bytes (status).
+ */
+moe_status_t nvfp4_grouped_gemm(const moe_config_t* cfg, int32_t proj, const uint8_t* act_codes,
+                                const uint8_t* act_sf, const float* act_scale, int32_t T, const moe_plan_t* plan,
+                                const float* weights, const moe_weights_t* w, uint16_t* out, void* ws,
+                                size_t ws_bytes, void* stream);
 
 /*
  * Clamped SwiGLU (glm5next_mlp "Traps": the clamp is asymmetric):
@@ -259,14 +334,22 @@ moe_status_t nvfp4_dequant(const uint8_t* codes, const uint8_t* scales, const fl
  * combine. x bf16 [T, H] -> y bf16 [T, H]. ws: moe_workspace_size(cfg, T,
  * path) bytes. The routing plan, logits, ids and weights of the call stay in
  * the workspace until the next call (see moe_workspace_views).
+ *   MOE_PATH_DECODE: W4A16 GEMV experts (nvfp4_expert_gemv).
+ *   MOE_PATH_PREFILL: permute with the padded tile layout, x encoded to
+ *     NVFP4 per assignment row (nvfp4_quantize_rows), grouped GEMM gate/up
+ *     with the clamped SwiGLU, h rounded to bf16 and encoded to NVFP4 per
+ *     row, grouped GEMM down with the routing weight; needs w->prepared,
+ *     I % 128 == 0, H % 256 == 0.
  */
 moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const uint16_t* x, int32_t T,
                          int32_t path, uint16_t* y, void* ws, size_t ws_bytes, void* stream);
 
 /* Device pointers (inside ws) of the intermediates moe_forward leaves behind:
  * logits fp32 [T,E], ids int32 [T,k], weights fp32 [T,k], the plan, h bf16
- * [T*k, I], r bf16 [T*k, H], shared bf16 [T, H] (NULL when Is == 0). Host-only
- * pointer arithmetic. */
+ * ([T*k, I] on the decode path, [P, I] in padded tile rows on the prefill
+ * path), r bf16 [T*k, H], shared bf16 [T, H] (NULL when Is == 0), and on the
+ * prefill path the NVFP4-encoded x and h in padded tile rows (codes, scale
+ * atoms, row scales; NULL on the decode path). Host-only pointer arithmetic. */
 typedef struct {
   float* logits;
   int32_t* ids;
@@ -275,6 +358,12 @@ typedef struct {
   uint16_t* h;
   uint16_t* r;
   uint16_t* shared;
+  uint8_t* xq_codes;
+  uint8_t* xq_sf;
+  float* xq_scale;
+  uint8_t* hq_codes;
+  uint8_t* hq_sf;
+  float* hq_scale;
 } moe_views_t;
 moe_status_t moe_workspace_views(const moe_config_t* cfg, int32_t T, int32_t path, void* ws, size_t ws_bytes,
                                  moe_views_t* views);

@@ -27,7 +27,8 @@ EXPORTED = (
     "moe_workspace_size", "moe_plan_size", "moe_plan_carve", "moe_router_topk", "moe_permute",
     "nvfp4_expert_gemv", "clamped_swiglu", "moe_combine", "dense_ffn_workspace_size", "dense_ffn_bf16",
     "nvfp4_dequant", "moe_forward", "moe_workspace_views", "moe_read_device_status", "moe_last_error",
-    "moe_set_stage_events", "moe_forward_decode_noalloc",
+    "moe_set_stage_events", "moe_forward_decode_noalloc", "moe_padded_rows", "moe_prepared_size",
+    "moe_prepare_weights", "nvfp4_quantize_rows", "nvfp4_grouped_gemm",
 )
 STAGES = ("router_logits", "topk", "permute", "act_quant", "expert_gate_up", "h_quant", "expert_down", "shared",
           "combine")
@@ -52,17 +53,20 @@ class Nvfp4Bank(C.Structure):
 class MoeWeights(C.Structure):
     _fields_ = [("router_w", C.c_void_p), ("router_bias", C.c_void_p), ("gate", Nvfp4Bank), ("up", Nvfp4Bank),
                 ("down", Nvfp4Bank), ("shared_gate", C.c_void_p), ("shared_up", C.c_void_p),
-                ("shared_down", C.c_void_p)]
+                ("shared_down", C.c_void_p), ("prepared", C.c_void_p)]
 
 
 class MoePlan(C.Structure):
     _fields_ = [("counts", C.c_void_p), ("offsets", C.c_void_p), ("sorted", C.c_void_p), ("inv", C.c_void_p),
-                ("tile_offsets", C.c_void_p), ("active", C.c_void_p), ("first", C.c_void_p)]
+                ("tile_offsets", C.c_void_p), ("active", C.c_void_p), ("first", C.c_void_p),
+                ("tile_rows", C.c_void_p)]
 
 
 class MoeViews(C.Structure):
     _fields_ = [("logits", C.c_void_p), ("ids", C.c_void_p), ("weights", C.c_void_p), ("plan", MoePlan),
-                ("h", C.c_void_p), ("r", C.c_void_p), ("shared", C.c_void_p)]
+                ("h", C.c_void_p), ("r", C.c_void_p), ("shared", C.c_void_p), ("xq_codes", C.c_void_p),
+                ("xq_sf", C.c_void_p), ("xq_scale", C.c_void_p), ("hq_codes", C.c_void_p), ("hq_sf", C.c_void_p),
+                ("hq_scale", C.c_void_p)]
 
 
 def load_library(path: str = _LIB_PATH) -> C.CDLL:
@@ -90,6 +94,12 @@ def load_library(path: str = _LIB_PATH) -> C.CDLL:
         "moe_last_error": (C.c_char_p, []),
         "moe_set_stage_events": (st, [C.POINTER(C.c_void_p), i32]),
         "moe_forward_decode_noalloc": (st, [cfgp, C.POINTER(MoeWeights), vp, i32, vp, vp]),
+        "moe_padded_rows": (C.c_int64, [cfgp, i32]),
+        "moe_prepared_size": (sz, [cfgp]),
+        "moe_prepare_weights": (st, [cfgp, C.POINTER(MoeWeights), vp, sz, vp]),
+        "nvfp4_quantize_rows": (st, [vp, i32, i32, vp, vp, vp, vp]),
+        "nvfp4_grouped_gemm": (st, [cfgp, i32, vp, vp, vp, i32, C.POINTER(MoePlan), vp, C.POINTER(MoeWeights), vp,
+                                    vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -155,12 +165,13 @@ class DeviceSite:
     router_bias: torch.Tensor
     banks: dict            # proj -> (codes, scales, ts)
     shared: tuple | None   # (gate, up, down) bf16 or None
+    prepared: torch.Tensor | None = None   # block-scale atoms of moe_prepare_weights (prefill)
 
     def c(self) -> MoeWeights:
         b = {p: Nvfp4Bank(_p(c), _p(s), _p(t)) for p, (c, s, t) in self.banks.items()}
         sh = self.shared or (None, None, None)
         return MoeWeights(_p(self.router_w), _p(self.router_bias), b["gate"], b["up"], b["down"],
-                          _p(sh[0]), _p(sh[1]), _p(sh[2]))
+                          _p(sh[0]), _p(sh[1]), _p(sh[2]), _p(self.prepared))
 
 
 def bf16_tensor(bits, device="cuda") -> torch.Tensor:
@@ -265,6 +276,38 @@ def moe_forward_decode_noalloc(cfg: SiteConfig, site: DeviceSite, x, y, stream=N
     w = site.c()
     _check(lib().moe_forward_decode_noalloc(C.byref(cfg.c()), C.byref(w), _p(x), x.shape[0], _p(y),
                                             _stream(stream)))
+
+
+def moe_padded_rows(cfg: SiteConfig, T: int) -> int:
+    return lib().moe_padded_rows(C.byref(cfg.c()), T)
+
+
+def moe_prepared_size(cfg: SiteConfig) -> int:
+    return lib().moe_prepared_size(C.byref(cfg.c()))
+
+
+def moe_prepare_weights(cfg: SiteConfig, site: DeviceSite, stream=None) -> torch.Tensor:
+    """Allocate and fill the prefill block-scale atoms; also attaches them to
+    ``site.prepared``."""
+    n = moe_prepared_size(cfg)
+    dst = torch.empty(n, dtype=torch.uint8, device=site.router_w.device)
+    w = site.c()
+    _check(lib().moe_prepare_weights(C.byref(cfg.c()), C.byref(w), _p(dst), n, _stream(stream)))
+    site.prepared = dst
+    return dst
+
+
+def nvfp4_quantize_rows(src, codes, sf_atoms, row_scale, stream=None):
+    rows, K = src.shape
+    _check(lib().nvfp4_quantize_rows(_p(src), rows, K, _p(codes), _p(sf_atoms), _p(row_scale), _stream(stream)))
+
+
+def nvfp4_grouped_gemm(cfg: SiteConfig, proj: int, act_codes, act_sf, act_scale, T: int, plan: MoePlan, weights,
+                       site: DeviceSite, out, ws, stream=None):
+    w = site.c()
+    _check(lib().nvfp4_grouped_gemm(C.byref(cfg.c()), proj, _p(act_codes), _p(act_sf), _p(act_scale), T,
+                                    C.byref(plan), _p(weights), C.byref(w), _p(out), _p(ws), ws.numel(),
+                                    _stream(stream)))
 
 
 def moe_workspace_views(cfg: SiteConfig, T: int, path: int, ws) -> MoeViews:

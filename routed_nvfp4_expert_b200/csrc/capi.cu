@@ -100,11 +100,18 @@ moe_status_t check_bank(const nvfp4_bank_t& b, const char* name) {
 // ------------------------------------------------------------ layouts
 
 struct PlanLayout {
-  size_t counts, offsets, sorted, inv, tile_offsets, active, first, bytes;
+  size_t counts, offsets, sorted, inv, tile_offsets, active, first, tile_rows, bytes;
+  int64_t P;   // rows of the padded tile layout
 };
 
-PlanLayout plan_layout(int E, int A) {
+int64_t padded_rows(const moe_config_t* c, int64_t A) {
+  return rnx::padded_rows_bound(A, (int64_t)c->local_end - c->local_begin);
+}
+
+PlanLayout plan_layout(const moe_config_t* c, int A) {
+  const int E = c->num_experts;
   PlanLayout L{};
+  L.P = padded_rows(c, A);
   size_t o = 0;
   L.counts = o; o = up(o + 4 * (size_t)E);
   L.offsets = o; o = up(o + 4 * (size_t)(E + 1));
@@ -113,6 +120,7 @@ PlanLayout plan_layout(int E, int A) {
   L.tile_offsets = o; o = up(o + 4 * (size_t)(E + 1));
   L.active = o; o = up(o + 4 * (size_t)(E + 1));
   L.first = o; o = up(o + 4 * (size_t)E);
+  L.tile_rows = o; o = up(o + 4 * (size_t)L.P);
   L.bytes = o;
   return L;
 }
@@ -126,15 +134,18 @@ moe_plan_t plan_at(char* base, const PlanLayout& L) {
   p.tile_offsets = (int32_t*)(base + L.tile_offsets);
   p.active = (int32_t*)(base + L.active);
   p.first = (int32_t*)(base + L.first);
+  p.tile_rows = (int32_t*)(base + L.tile_rows);
   return p;
 }
 
 struct WsLayout {
-  size_t status, logits, ids, weights, plan, scratch, h, r, shared_h, shared, xmax, hmax, bytes;
+  size_t status, logits, ids, weights, plan, scratch, h, r, shared_h, shared, xmax, hmax;
+  size_t xq, xsf, xts, hq, hsf, hts;   // prefill: NVFP4 x and h in padded tile rows
+  size_t bytes;
   PlanLayout pl;
 };
 
-WsLayout ws_layout(const moe_config_t* c, int T, int /*path*/) {
+WsLayout ws_layout(const moe_config_t* c, int T, int path) {
   WsLayout L{};
   const int E = c->num_experts, k = c->top_k, H = c->hidden, I = c->intermediate, Is = c->shared_intermediate;
   const size_t A = (size_t)T * k;
@@ -143,17 +154,71 @@ WsLayout ws_layout(const moe_config_t* c, int T, int /*path*/) {
   L.logits = o; o = up(o + 4 * (size_t)T * E);
   L.ids = o; o = up(o + 4 * A);
   L.weights = o; o = up(o + 4 * A);
-  L.pl = plan_layout(E, (int)A);
+  L.pl = plan_layout(c, (int)A);
   L.plan = o; o = up(o + L.pl.bytes);
   L.scratch = o; o = up(o + 4 * rnx::permute_scratch_ints((int)A, E));
-  L.h = o; o = up(o + 2 * A * I);
+  const bool pre = path == MOE_PATH_PREFILL;
+  const size_t P = (size_t)L.pl.P;
+  L.h = o; o = up(o + 2 * (pre ? P : A) * I);
   L.r = o; o = up(o + 2 * A * H);
   L.shared_h = o; o = up(o + 2 * (size_t)T * Is);
   L.shared = o; o = up(o + 2 * (size_t)T * H);
   L.xmax = o; o = up(o + 4 * (size_t)T);
   L.hmax = o; o = up(o + 4 * A);
+  if (pre) {
+    L.xq = o; o = up(o + P * H / 2);
+    L.xsf = o; o = up(o + P * H / 16);
+    L.xts = o; o = up(o + 4 * P);
+    L.hq = o; o = up(o + P * I / 2);
+    L.hsf = o; o = up(o + P * I / 16);
+    L.hts = o; o = up(o + 4 * P);
+  }
   L.bytes = o;
   return L;
+}
+
+// Shapes the tensor-core prefill path covers.
+moe_status_t check_prefill_shape(const moe_config_t* c) {
+  if (c->intermediate % 128) return fail(MOE_ERR_UNSUPPORTED, "prefill needs intermediate %% 128 == 0 (got %d)", c->intermediate);
+  if (c->hidden % 256) return fail(MOE_ERR_UNSUPPORTED, "prefill needs hidden %% 256 == 0 (got %d)", c->hidden);
+  return MOE_OK;
+}
+
+struct PreparedLayout {
+  size_t gate, up, down, bytes;
+};
+PreparedLayout prepared_layout(const moe_config_t* c) {
+  const size_t per = (size_t)c->num_experts * c->intermediate * c->hidden / 16;
+  return PreparedLayout{0, per, 2 * per, 3 * per};
+}
+
+rnx::Fp4GemmArgs gemm_args(const moe_config_t* c, int proj, const uint8_t* codes, const uint8_t* sf,
+                           const float* scale, int64_t P, const moe_plan_t& plan, const float* weights,
+                           const moe_weights_t* w, uint16_t* out, uint32_t* status) {
+  const PreparedLayout PL = prepared_layout(c);
+  rnx::Fp4GemmArgs g{};
+  g.gate_up = proj == MOE_PROJ_GATE_UP;
+  g.E = c->num_experts;
+  g.K = g.gate_up ? c->hidden : c->intermediate;
+  g.out_cols = g.gate_up ? c->intermediate : c->hidden;
+  g.bank_rows = g.gate_up ? c->intermediate : c->hidden;
+  g.P_max = P;
+  g.limit = c->swiglu_limit;
+  g.a_codes = codes;
+  g.a_sf = sf;
+  g.row_scale = scale;
+  if (g.gate_up) {
+    g.b0_codes = w->gate.codes; g.b0_sf = w->prepared + PL.gate; g.ts0 = w->gate.tensor_scale;
+    g.b1_codes = w->up.codes;   g.b1_sf = w->prepared + PL.up;   g.ts1 = w->up.tensor_scale;
+  } else {
+    g.b0_codes = w->down.codes; g.b0_sf = w->prepared + PL.down; g.ts0 = w->down.tensor_scale;
+  }
+  g.tile_offsets = plan.tile_offsets;
+  g.tile_rows = plan.tile_rows;
+  g.weights = weights;
+  g.out = out;
+  g.status = status;
+  return g;
 }
 
 moe_status_t check_ws(const moe_config_t* c, int T, int path, void* ws, size_t ws_bytes, WsLayout* L) {
@@ -192,14 +257,14 @@ size_t moe_workspace_size(const moe_config_t* cfg, int32_t T, int32_t path) {
 
 size_t moe_plan_size(const moe_config_t* cfg, int32_t T) {
   if (check_cfg(cfg) != MOE_OK || check_T(T) != MOE_OK) return 0;
-  return plan_layout(cfg->num_experts, T * cfg->top_k).bytes;
+  return plan_layout(cfg, T * cfg->top_k).bytes;
 }
 
 moe_status_t moe_plan_carve(const moe_config_t* cfg, int32_t T, void* buf, size_t bytes, moe_plan_t* plan) {
   moe_status_t s;
   if ((s = check_cfg(cfg)) != MOE_OK || (s = check_T(T)) != MOE_OK) return s;
   if (!plan) return fail(MOE_ERR_INVALID_ARG, "plan is NULL");
-  const PlanLayout L = plan_layout(cfg->num_experts, T * cfg->top_k);
+  const PlanLayout L = plan_layout(cfg, T * cfg->top_k);
   if (!buf || ((uintptr_t)buf % kAlign)) return fail(MOE_ERR_INVALID_ARG, "plan buffer NULL or not 256-byte aligned");
   if (bytes < L.bytes) return fail(MOE_ERR_WORKSPACE, "plan buffer has %zu bytes, needs %zu", bytes, L.bytes);
   *plan = plan_at((char*)buf, L);
@@ -221,6 +286,96 @@ moe_status_t moe_workspace_views(const moe_config_t* cfg, int32_t T, int32_t pat
   v->h = (uint16_t*)(b + L.h);
   v->r = (uint16_t*)(b + L.r);
   v->shared = cfg->shared_intermediate > 0 ? (uint16_t*)(b + L.shared) : nullptr;
+  const bool pre = path == MOE_PATH_PREFILL;
+  v->xq_codes = pre ? (uint8_t*)(b + L.xq) : nullptr;
+  v->xq_sf = pre ? (uint8_t*)(b + L.xsf) : nullptr;
+  v->xq_scale = pre ? (float*)(b + L.xts) : nullptr;
+  v->hq_codes = pre ? (uint8_t*)(b + L.hq) : nullptr;
+  v->hq_sf = pre ? (uint8_t*)(b + L.hsf) : nullptr;
+  v->hq_scale = pre ? (float*)(b + L.hts) : nullptr;
+  return MOE_OK;
+}
+
+int64_t moe_padded_rows(const moe_config_t* cfg, int32_t T) {
+  if (check_cfg(cfg) != MOE_OK || check_T(T) != MOE_OK) return 0;
+  return padded_rows(cfg, (int64_t)T * cfg->top_k);
+}
+
+size_t moe_prepared_size(const moe_config_t* cfg) {
+  if (check_cfg(cfg) != MOE_OK) return 0;
+  return prepared_layout(cfg).bytes;
+}
+
+moe_status_t moe_prepare_weights(const moe_config_t* cfg, const moe_weights_t* w, void* dst, size_t dst_bytes,
+                                 void* stream) {
+  moe_status_t s;
+  if ((s = check_cfg(cfg)) != MOE_OK || (s = check_prefill_shape(cfg)) != MOE_OK) return s;
+  if (!w) return fail(MOE_ERR_INVALID_ARG, "weights struct is NULL");
+  if ((s = check_bank(w->gate, "gate")) != MOE_OK || (s = check_bank(w->up, "up")) != MOE_OK ||
+      (s = check_bank(w->down, "down")) != MOE_OK)
+    return s;
+  const PreparedLayout PL = prepared_layout(cfg);
+  if (!dst || ((uintptr_t)dst % kAlign)) return fail(MOE_ERR_INVALID_ARG, "dst NULL or not 256-byte aligned");
+  if (dst_bytes < PL.bytes) return fail(MOE_ERR_WORKSPACE, "dst has %zu bytes, needs %zu", dst_bytes, PL.bytes);
+  cudaStream_t st = (cudaStream_t)stream;
+  uint8_t* d = (uint8_t*)dst;
+  const int E = cfg->num_experts, H = cfg->hidden, I = cfg->intermediate;
+  RNX_CUDA(rnx::launch_sf_atoms(w->gate.scales, E, I, H, d + PL.gate, st), "prepare gate scales");
+  RNX_CUDA(rnx::launch_sf_atoms(w->up.scales, E, I, H, d + PL.up, st), "prepare up scales");
+  RNX_CUDA(rnx::launch_sf_atoms(w->down.scales, E, H, I, d + PL.down, st), "prepare down scales");
+  return MOE_OK;
+}
+
+moe_status_t nvfp4_quantize_rows(const uint16_t* src, int32_t rows, int32_t K, uint8_t* codes, uint8_t* sf_atoms,
+                                 float* row_scale, void* stream) {
+  if (rows < 0 || K <= 0 || K % 64) return fail(MOE_ERR_INVALID_ARG, "rows=%d K=%d: K must be a positive multiple of 64", rows, K);
+  if (rows == 0) return MOE_OK;
+  RNX_PTR(src, "src");
+  RNX_PTR(codes, "codes");
+  RNX_PTR(sf_atoms, "sf_atoms");
+  RNX_PTR(row_scale, "row_scale");
+  RNX_CUDA(rnx::launch_quant_rows(src, rows, K, nullptr, 0, nullptr, codes, sf_atoms, row_scale, (cudaStream_t)stream),
+           "nvfp4_quantize_rows");
+  return MOE_OK;
+}
+
+moe_status_t nvfp4_grouped_gemm(const moe_config_t* cfg, int32_t proj, const uint8_t* act_codes,
+                                const uint8_t* act_sf, const float* act_scale, int32_t T, const moe_plan_t* plan,
+                                const float* weights, const moe_weights_t* w, uint16_t* out, void* ws,
+                                size_t ws_bytes, void* stream) {
+  moe_status_t s;
+  if ((s = check_cfg(cfg)) != MOE_OK || (s = check_T(T)) != MOE_OK || (s = check_prefill_shape(cfg)) != MOE_OK)
+    return s;
+  if (proj != MOE_PROJ_GATE_UP && proj != MOE_PROJ_DOWN) return fail(MOE_ERR_INVALID_ARG, "unknown proj %d", proj);
+  if (T == 0) return MOE_OK;
+  RNX_PTR(act_codes, "act_codes");
+  RNX_PTR(act_sf, "act_sf");
+  RNX_PTR(act_scale, "act_scale");
+  RNX_PTR(out, "out");
+  if (!plan || !w) return fail(MOE_ERR_INVALID_ARG, "plan / weights struct is NULL");
+  RNX_PTR(plan->tile_offsets, "plan.tile_offsets");
+  RNX_PTR(plan->tile_rows, "plan.tile_rows");
+  RNX_PTR(w->prepared, "prepared");
+  if (proj == MOE_PROJ_GATE_UP) {
+    if ((s = check_bank(w->gate, "gate")) != MOE_OK || (s = check_bank(w->up, "up")) != MOE_OK) return s;
+  } else {
+    if ((s = check_bank(w->down, "down")) != MOE_OK) return s;
+    RNX_PTR(weights, "weights");
+    RNX_PTR(plan->offsets, "plan.offsets");
+    RNX_PTR(plan->sorted, "plan.sorted");
+  }
+  WsLayout L;
+  if ((s = check_ws(cfg, T, MOE_PATH_PREFILL, ws, ws_bytes, &L)) != MOE_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  char* b = (char*)ws;
+  uint32_t* status = (uint32_t*)(b + L.status);
+  RNX_CUDA(cudaMemsetAsync(status, 0, 4, st), "clear status");
+  const rnx::Fp4GemmArgs g = gemm_args(cfg, proj, act_codes, act_sf, act_scale, L.pl.P, *plan, weights, w, out, status);
+  RNX_CUDA(rnx::launch_fp4_grouped_gemm(g, st), "nvfp4_grouped_gemm");
+  if (proj == MOE_PROJ_DOWN)
+    RNX_CUDA(rnx::launch_zero_remote(plan->offsets, plan->sorted, cfg->num_experts, cfg->local_begin, cfg->local_end,
+                                     cfg->hidden, out, st),
+             "zero remote rows");
   return MOE_OK;
 }
 
@@ -270,14 +425,16 @@ moe_status_t moe_permute(const moe_config_t* cfg, const int32_t* ids, int32_t T,
   RNX_PTR(plan->tile_offsets, "plan.tile_offsets");
   RNX_PTR(plan->active, "plan.active");
   RNX_PTR(plan->first, "plan.first");
-  WsLayout L;
-  if ((s = check_ws(cfg, T, MOE_PATH_PREFILL, ws, ws_bytes, &L)) != MOE_OK) return s;
+  RNX_PTR(plan->tile_rows, "plan.tile_rows");
+  WsLayout L;   // status word and sort scratch sit at the same offsets on both paths
+  if ((s = check_ws(cfg, T, MOE_PATH_DECODE, ws, ws_bytes, &L)) != MOE_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
   char* b = (char*)ws;
   RNX_CUDA(cudaMemsetAsync(b + L.status, 0, 4, st), "clear status");
   RNX_CUDA(rnx::launch_permute(ids, T * cfg->top_k, cfg->num_experts, cfg->local_begin, cfg->local_end, *plan,
                                (int32_t*)(b + L.scratch), (uint32_t*)(b + L.status), st),
            "permute");
+  RNX_CUDA(rnx::launch_tile_rows(*plan, cfg->num_experts, L.pl.P, st), "tile rows");
   return MOE_OK;
 }
 
@@ -404,7 +561,10 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
     RNX_PTR(w->shared_up, "shared_up");
     RNX_PTR(w->shared_down, "shared_down");
   }
-  if (path == MOE_PATH_PREFILL) return fail(MOE_ERR_UNSUPPORTED, "prefill path not built yet");
+  if (path == MOE_PATH_PREFILL) {
+    if ((s = check_prefill_shape(cfg)) != MOE_OK) return s;
+    RNX_PTR(w->prepared, "prepared");
+  }
   WsLayout L;
   if ((s = check_ws(cfg, T, path, ws, ws_bytes, &L)) != MOE_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
@@ -431,21 +591,44 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
                                status, st),
            "permute");
   RNX_CUDA(mark(MOE_STAGE_ACT_QUANT, st), "stage event");
-  rnx::ExpertGemvArgs a{};
-  a.T = T; a.H = H; a.I = I; a.E = E; a.k = k;
-  a.local_begin = cfg->local_begin; a.local_end = cfg->local_end;
-  a.limit = cfg->swiglu_limit;
-  a.offsets = plan.offsets; a.sorted = plan.sorted; a.active = plan.active; a.first = plan.first;
-  a.weights = wts;
-  a.gate = w->gate; a.up = w->up; a.down = w->down;
-  a.status = status;
-  a.proj = MOE_PROJ_GATE_UP; a.act = x; a.out = h; a.act_max = xmax; a.out_max = hmax; a.prefetch_down = false;
-  RNX_CUDA(mark(MOE_STAGE_EXPERT_GATE_UP, st), "stage event");
-  RNX_CUDA(rnx::launch_nvfp4_gemv(a, st), "expert gate/up");
-  RNX_CUDA(mark(MOE_STAGE_H_QUANT, st), "stage event");
-  a.proj = MOE_PROJ_DOWN; a.act = h; a.out = r; a.act_max = hmax; a.out_max = nullptr; a.prefetch_down = false;
-  RNX_CUDA(mark(MOE_STAGE_EXPERT_DOWN, st), "stage event");
-  RNX_CUDA(rnx::launch_nvfp4_gemv(a, st), "expert down");
+  if (path == MOE_PATH_PREFILL) {
+    const int64_t P = L.pl.P;
+    uint8_t* xq = (uint8_t*)(b + L.xq);
+    uint8_t* xsf = (uint8_t*)(b + L.xsf);
+    float* xts = (float*)(b + L.xts);
+    uint8_t* hq = (uint8_t*)(b + L.hq);
+    uint8_t* hsf = (uint8_t*)(b + L.hsf);
+    float* hts = (float*)(b + L.hts);
+    const int32_t* used_tiles = plan.tile_offsets + E;
+    RNX_CUDA(rnx::launch_tile_rows(plan, E, P, st), "tile rows");
+    RNX_CUDA(rnx::launch_quant_rows(x, P, H, plan.tile_rows, k, used_tiles, xq, xsf, xts, st), "x quant");
+    RNX_CUDA(mark(MOE_STAGE_EXPERT_GATE_UP, st), "stage event");
+    rnx::Fp4GemmArgs g = gemm_args(cfg, MOE_PROJ_GATE_UP, xq, xsf, xts, P, plan, wts, w, h, status);
+    RNX_CUDA(rnx::launch_fp4_grouped_gemm(g, st), "expert gate/up (tcgen05)");
+    RNX_CUDA(mark(MOE_STAGE_H_QUANT, st), "stage event");
+    RNX_CUDA(rnx::launch_quant_rows(h, P, I, plan.tile_rows, 0, used_tiles, hq, hsf, hts, st), "h quant");
+    RNX_CUDA(mark(MOE_STAGE_EXPERT_DOWN, st), "stage event");
+    g = gemm_args(cfg, MOE_PROJ_DOWN, hq, hsf, hts, P, plan, wts, w, r, status);
+    RNX_CUDA(rnx::launch_fp4_grouped_gemm(g, st), "expert down (tcgen05)");
+    RNX_CUDA(rnx::launch_zero_remote(plan.offsets, plan.sorted, E, cfg->local_begin, cfg->local_end, H, r, st),
+             "zero remote rows");
+  } else {
+    rnx::ExpertGemvArgs a{};
+    a.T = T; a.H = H; a.I = I; a.E = E; a.k = k;
+    a.local_begin = cfg->local_begin; a.local_end = cfg->local_end;
+    a.limit = cfg->swiglu_limit;
+    a.offsets = plan.offsets; a.sorted = plan.sorted; a.active = plan.active; a.first = plan.first;
+    a.weights = wts;
+    a.gate = w->gate; a.up = w->up; a.down = w->down;
+    a.status = status;
+    a.proj = MOE_PROJ_GATE_UP; a.act = x; a.out = h; a.act_max = xmax; a.out_max = hmax; a.prefetch_down = false;
+    RNX_CUDA(mark(MOE_STAGE_EXPERT_GATE_UP, st), "stage event");
+    RNX_CUDA(rnx::launch_nvfp4_gemv(a, st), "expert gate/up");
+    RNX_CUDA(mark(MOE_STAGE_H_QUANT, st), "stage event");
+    a.proj = MOE_PROJ_DOWN; a.act = h; a.out = r; a.act_max = hmax; a.out_max = nullptr; a.prefetch_down = false;
+    RNX_CUDA(mark(MOE_STAGE_EXPERT_DOWN, st), "stage event");
+    RNX_CUDA(rnx::launch_nvfp4_gemv(a, st), "expert down");
+  }
   RNX_CUDA(mark(MOE_STAGE_SHARED, st), "stage event");
   if (Is > 0) {
     RNX_CUDA(rnx::launch_dense_gemv(H, Is, cfg->swiglu_limit, x, T, w->shared_gate, w->shared_up, w->shared_down,

@@ -57,4 +57,52 @@ cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* scales, const fl
 cudaError_t launch_dense_gemv(int H, int I, float limit, const uint16_t* x, int T, const uint16_t* wg,
                               const uint16_t* wu, const uint16_t* wd, uint16_t* y, uint16_t* hbuf, cudaStream_t st);
 
+// ---------------------------------------------------------------- prefill (W4A4, tcgen05)
+
+// Padded tile layout of the prefill: every local expert's rows start on a
+// 128-row tile. tile_rows[p] = assignment at padded row p, -1 for padding.
+// P_max = padded_rows_bound(A, E_local) rows are written (rows past the last
+// used tile get -1 too).
+int64_t padded_rows_bound(int64_t A, int64_t E_local);
+cudaError_t launch_tile_rows(const moe_plan_t& plan, int E, int64_t P_max, cudaStream_t st);
+
+// NVFP4 encoding of bf16 rows (per-row fp32 scale r/2688, E4M3 per 16, E2M1).
+// Output row p reads source row: row_map ? (row_map[p] < 0 ? none : div > 0 ? row_map[p] / div : p) : p
+// ("none" = a zero row).
+// codes [rows, K/2]; sf atoms [ceil(rows/128)][K/64][512]; row_scale [rows].
+// Rows in [rows, ceil128(rows)) get zero scale bytes. used_tiles (nullable,
+// device int): rows at or past used_tiles*128 are left untouched.
+cudaError_t launch_quant_rows(const uint16_t* src, int64_t rows, int K, const int32_t* row_map, int div,
+                              const int32_t* used_tiles, uint8_t* codes, uint8_t* sf, float* row_scale,
+                              cudaStream_t st);
+
+// Canonical block scales [n_experts * rows, K/16] -> atoms [n_experts][rows/128][K/64][512].
+cudaError_t launch_sf_atoms(const uint8_t* scales, int64_t n_experts, int rows, int K, uint8_t* atoms, cudaStream_t st);
+
+// Zero the r rows of assignments routed to experts outside [lb, le).
+cudaError_t launch_zero_remote(const int32_t* offsets, const int32_t* sorted, int E, int lb, int le, int H,
+                               uint16_t* r, cudaStream_t st);
+
+struct Fp4GemmArgs {
+  bool gate_up;
+  int E, K, out_cols, bank_rows;   // bank_rows: rows of one expert in the weight bank (I for gate/up, H for down)
+  int64_t P_max;                   // rows of the A operand buffers
+  float limit;
+  const uint8_t* a_codes;          // [P_max, K/2]
+  const uint8_t* a_sf;             // atoms [P_max/128][K/64][512]
+  const float* row_scale;          // [P_max]
+  const uint8_t* b0_codes;         // gate (or down) codes [E*bank_rows, K/2]
+  const uint8_t* b1_codes;         // up codes (gate_up)
+  const uint8_t* b0_sf;            // atoms [E][bank_rows/128][K/64][512]
+  const uint8_t* b1_sf;
+  const float* ts0;
+  const float* ts1;
+  const int32_t* tile_offsets;     // [E+1]
+  const int32_t* tile_rows;        // [P_max]
+  const float* weights;            // [A] routing weights (down)
+  uint16_t* out;                   // gate_up: h [P_max, out_cols]; down: r [A, out_cols]
+  uint32_t* status;
+};
+cudaError_t launch_fp4_grouped_gemm(const Fp4GemmArgs& a, cudaStream_t st);
+
 }  // namespace rnx

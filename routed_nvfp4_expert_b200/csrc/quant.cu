@@ -1,0 +1,205 @@
+// Prefill data movement around the FP4 grouped GEMM:
+//  - the padded tile layout (tile_rows: assignment of each padded row),
+//  - NVFP4 encoding of bf16 activation rows (x gathered per assignment, or h
+//    in place) with one fp32 scale per row, an E4M3 scale per 16 elements and
+//    E2M1 codes, the scales written straight into the 512-byte atoms the
+//    tensor-core scale copy reads,
+//  - the one-time re-tiling of the weights' block scales into the same atoms,
+//  - zeroing of the rows routed to experts outside the local range.
+//
+// Activation encoding (prefill reading of the glm5next_mlp module docs'
+// forward_prefill_gemm, W4A4 with a per-row second-level scale), every step
+// IEEE fp32 in this order: r = max|row|; ts = r / 2688 (2688 = 6 * 448);
+// per 16-block sb = e4m3_rn_satfinite((amax_blk / 6) / ts); d = e4m3(sb) * ts;
+// code = e2m1_rn_satfinite(v / d). A zero row has ts = 0 and all scales and
+// codes 0; a block with d = 0 gets codes 0.
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace rnx {
+
+namespace {
+
+constexpr int kQuantWarps = 8;
+
+// Byte offset, inside the atoms of a [rows/128][K/64] grid, of the scale of
+// row p, 16-element block b (the 32x4x4 atom: lane p%32, 4-byte column
+// (p%128)/32, byte b%4 within the 64-element K block).
+__host__ __device__ inline long long sf_atom_offset(long long p, int b, int KB) {
+  return ((p >> 7) * KB + (b >> 2)) * 512 + (p & 31) * 16 + ((p & 127) >> 5) * 4 + (b & 3);
+}
+
+RNX_DEVICE void load16(const uint16_t* src, float (&v)[16]) {
+  const uint4 a = *reinterpret_cast<const uint4*>(src);
+  const uint4 c = *reinterpret_cast<const uint4*>(src + 8);
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float2 f = bf16x2_to_f32x2(w[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+
+__global__ void __launch_bounds__(kQuantWarps * 32) quant_rows_kernel(const uint16_t* __restrict__ src, long long rows,
+                                                                      long long rows_pad, int K,
+                                                                      const int32_t* __restrict__ row_map, int div,
+                                                                      const int32_t* __restrict__ used_tiles,
+                                                                      uint8_t* __restrict__ codes,
+                                                                      uint8_t* __restrict__ sf,
+                                                                      float* __restrict__ row_scale) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long p = (long long)blockIdx.x * kQuantWarps + warp;
+  if (p >= rows_pad) return;
+  if (used_tiles && p >= (long long)*used_tiles * kRowsPerTile) return;   // past the last tile in use
+  const int nblk = K / 16, KB = K / 64;
+  long long srow = -1;
+  if (p < rows) {
+    if (row_map) {
+      const int a = row_map[p];
+      srow = a < 0 ? -1 : (div > 0 ? a / div : p);
+    } else {
+      srow = p;
+    }
+  }
+  uint8_t* crow = codes + p * (K / 2);
+  if (srow < 0) {
+    for (int b = lane; b < nblk; b += 32) {
+      if (p < rows) *reinterpret_cast<uint2*>(crow + b * 8) = make_uint2(0, 0);
+      sf[sf_atom_offset(p, b, KB)] = 0;
+    }
+    if (lane == 0 && p < rows) row_scale[p] = 0.f;
+    return;
+  }
+  const uint16_t* x = src + srow * K;
+  float m = 0.f;
+  for (int b = lane; b < nblk; b += 32) {
+    float v[16];
+    load16(x + b * 16, v);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+  }
+  m = warp_max(m);
+  const float ts = m / 2688.0f;
+  for (int b = lane; b < nblk; b += 32) {
+    float v[16];
+    load16(x + b * 16, v);
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    const float q = ts == 0.f ? 0.f : (amax / 6.0f) / ts;
+    const uint8_t sb = f32_to_e4m3_satfinite(q);
+    const float d = e4m3_to_f32(sb) * ts;
+    uint32_t w0 = 0, w1 = 0;
+    if (d != 0.f) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        w0 |= (uint32_t)f32x2_to_e2m1x2_satfinite(v[2 * i] / d, v[2 * i + 1] / d) << (8 * i);
+        w1 |= (uint32_t)f32x2_to_e2m1x2_satfinite(v[8 + 2 * i] / d, v[8 + 2 * i + 1] / d) << (8 * i);
+      }
+    }
+    *reinterpret_cast<uint2*>(crow + b * 8) = make_uint2(w0, w1);
+    sf[sf_atom_offset(p, b, KB)] = sb;
+  }
+  if (lane == 0) row_scale[p] = ts;
+}
+
+// tile_rows[p] for p < P_max.
+__global__ void __launch_bounds__(256) tile_rows_kernel(const int32_t* __restrict__ counts,
+                                                        const int32_t* __restrict__ offsets,
+                                                        const int32_t* __restrict__ sorted,
+                                                        const int32_t* __restrict__ tile_offsets, int E,
+                                                        long long P_max, int32_t* __restrict__ tile_rows) {
+  const int ntiles = tile_offsets[E];
+  for (long long p = (long long)blockIdx.x * blockDim.x + threadIdx.x; p < P_max;
+       p += (long long)gridDim.x * blockDim.x) {
+    const int mt = (int)(p >> 7);
+    int a = -1;
+    if (mt < ntiles) {
+      int lo = 0, hi = E;   // largest e with tile_offsets[e] <= mt
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (tile_offsets[mid] <= mt) lo = mid; else hi = mid;
+      }
+      const int row = (mt - tile_offsets[lo]) * kRowsPerTile + (int)(p & 127);
+      if (row < counts[lo]) a = sorted[offsets[lo] + row];
+    }
+    tile_rows[p] = a;
+  }
+}
+
+__global__ void __launch_bounds__(256) sf_atoms_kernel(const uint8_t* __restrict__ scales, long long total_rows, int K,
+                                                       uint8_t* __restrict__ atoms) {
+  const int KB = K / 64;
+  for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < total_rows * KB;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const long long R = idx / KB;
+    const int kb = (int)(idx - R * KB);
+    const uint32_t w = *reinterpret_cast<const uint32_t*>(scales + R * (K / 16) + kb * 4);
+    *reinterpret_cast<uint32_t*>(atoms + sf_atom_offset(R, kb * 4, KB)) = w;
+  }
+}
+
+__global__ void __launch_bounds__(256) zero_remote_kernel(const int32_t* __restrict__ offsets,
+                                                          const int32_t* __restrict__ sorted, int E, int lb, int le,
+                                                          int H, uint16_t* __restrict__ r) {
+  const int rb0 = offsets[lb], re0 = offsets[le], rend = offsets[E];
+  const long long nremote = rb0 + (rend - re0);
+  const int vec = H / 8;
+  for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < nremote * vec;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const long long rp = idx / vec;
+    const int col = (int)(idx - rp * vec);
+    const long long pos = rp < rb0 ? rp : re0 + (rp - rb0);
+    const int a = sorted[pos];
+    reinterpret_cast<uint4*>(r + (size_t)a * H)[col] = make_uint4(0, 0, 0, 0);
+  }
+}
+
+int grid_for(long long work, int per_block) {
+  const long long g = (work + per_block - 1) / per_block;
+  return (int)std::max(1LL, std::min(g, (long long)kNumSMs * 16));
+}
+
+}  // namespace
+
+int64_t padded_rows_bound(int64_t A, int64_t E_local) {
+  const int64_t n = std::min(A, E_local);
+  return (A + 127 * n) / kRowsPerTile * kRowsPerTile;
+}
+
+cudaError_t launch_tile_rows(const moe_plan_t& plan, int E, int64_t P_max, cudaStream_t st) {
+  if (P_max <= 0) return cudaSuccess;
+  tile_rows_kernel<<<grid_for(P_max, 256), 256, 0, st>>>(plan.counts, plan.offsets, plan.sorted, plan.tile_offsets, E,
+                                                         P_max, plan.tile_rows);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_rows(const uint16_t* src, int64_t rows, int K, const int32_t* row_map, int div,
+                              const int32_t* used_tiles, uint8_t* codes, uint8_t* sf, float* row_scale,
+                              cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  const long long rows_pad = (rows + kRowsPerTile - 1) / kRowsPerTile * kRowsPerTile;
+  const long long grid = (rows_pad + kQuantWarps - 1) / kQuantWarps;
+  quant_rows_kernel<<<(unsigned)grid, kQuantWarps * 32, 0, st>>>(src, rows, rows_pad, K, row_map, div, used_tiles,
+                                                                  codes, sf, row_scale);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sf_atoms(const uint8_t* scales, int64_t n_experts, int rows, int K, uint8_t* atoms,
+                            cudaStream_t st) {
+  const long long total = (long long)n_experts * rows;
+  if (total <= 0) return cudaSuccess;
+  sf_atoms_kernel<<<grid_for(total * (K / 64), 256), 256, 0, st>>>(scales, total, K, atoms);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_zero_remote(const int32_t* offsets, const int32_t* sorted, int E, int lb, int le, int H,
+                               uint16_t* r, cudaStream_t st) {
+  if (lb == 0 && le == E) return cudaSuccess;
+  zero_remote_kernel<<<kNumSMs, 256, 0, st>>>(offsets, sorted, E, lb, le, H, r);
+  return cudaGetLastError();
+}
+
+}  // namespace rnx

@@ -80,7 +80,7 @@ def test_workspace_too_small_is_rejected_before_launch():
     need = lib.moe_workspace_size(C.byref(cfg), 4, 0)
     assert need > 0
     ids = 0x10000
-    plan = capi.MoePlan(0x20000, 0x30000, 0x40000, 0x50000, 0x60000, 0x70000, 0x80000)
+    plan = capi.MoePlan(0x20000, 0x30000, 0x40000, 0x50000, 0x60000, 0x70000, 0x80000, 0x90000)
     st = lib.moe_permute(C.byref(cfg), ids, 4, C.byref(plan), 0x100000, need - 256, None)
     assert st == 3 and "workspace" in lib.moe_last_error().decode()
 
@@ -91,7 +91,8 @@ def test_plan_carve_is_host_arithmetic():
     n = lib.moe_plan_size(C.byref(cfg), 10)
     plan = capi.MoePlan()
     assert lib.moe_plan_carve(C.byref(cfg), 10, 0x100000, n, C.byref(plan)) == 0
-    ptrs = [plan.counts, plan.offsets, plan.sorted, plan.inv, plan.tile_offsets, plan.active, plan.first]
+    ptrs = [plan.counts, plan.offsets, plan.sorted, plan.inv, plan.tile_offsets, plan.active, plan.first,
+            plan.tile_rows]
     assert ptrs == sorted(ptrs) and all(p % 256 == 0 for p in ptrs) and ptrs[0] == 0x100000
     assert lib.moe_plan_carve(C.byref(cfg), 10, 0x100000, n - 1, C.byref(plan)) == 3
 

@@ -1,0 +1,281 @@
+"""GPU parity of the prefill path (W4A4 on tcgen05 block-scaled FP4) against
+the CPU oracle, called through the C ABI: NVFP4 row encoding (bit-exact), the
+re-tiled weight scales (bit-exact), the padded tile layout (bit-exact), the
+grouped GEMM projections (against fp64 dot products of the GPU's own encoded
+operands), and the whole prefill site on the tiny site and the H=4096, E=288
+prefill / stress shapes."""
+import numpy as np
+import pytest
+import torch
+
+from helpers import assert_bf16_close, bf16_np, device_site, oracle_cfg, rel_l2, site_inputs, workload
+from oracle import formats as OF
+from oracle import site as OS
+
+pytestmark = pytest.mark.gpu
+
+capi = pytest.importorskip("routed_nvfp4_expert_b200.capi")
+
+
+# ------------------------------------------------------------------ layout helpers (test side)
+
+def sf_untile(atoms: np.ndarray, rows: int, K: int) -> np.ndarray:
+    """512-byte scale atoms [ceil(rows/128)][K/64][512] -> row-major [rows, K/16]:
+    the scale of row p, block b sits at ((p//128)*K/64 + b//4)*512 +
+    (p%32)*16 + ((p%128)//32)*4 + b%4."""
+    KB = K // 64
+    p = np.arange(rows)[:, None]
+    b = np.arange(K // 16)[None, :]
+    off = ((p // 128) * KB + b // 4) * 512 + (p % 32) * 16 + ((p % 128) // 32) * 4 + b % 4
+    return atoms.reshape(-1)[off]
+
+
+def expected_tile_rows(ref_plan: dict, E: int, P: int, local) -> np.ndarray:
+    lb, le = local
+    out = np.full(P, -1, np.int32)
+    tile = 0
+    for e in range(E):
+        c = int(ref_plan["counts"][e])
+        if not (lb <= e < le) or c == 0:
+            continue
+        o = int(ref_plan["offsets"][e])
+        out[tile * 128: tile * 128 + c] = ref_plan["sorted"][o:o + c]
+        tile += (c + 127) // 128
+    return out
+
+
+def _arr(ptr, n, dtype=torch.int32):
+    return capi.view_tensor(ptr, (n,), dtype).cpu().numpy().copy()
+
+
+# ------------------------------------------------------------------ encoding
+
+@pytest.mark.parametrize("rows,K", [(1, 256), (130, 1024), (300, 4096), (128, 64)])
+def test_quantize_rows_bit_exact(rows, K):
+    rng = np.random.default_rng(rows * 7 + K)
+    x = rng.standard_normal((rows, K)).astype(np.float32) * rng.lognormal(0.0, 2.0, (rows, 1)).astype(np.float32)
+    if rows > 3:
+        x[1] = 0.0                                   # zero row: scale 0, every code and scale 0
+        x[2, : K // 2] = 0.0                         # zero blocks inside a live row
+        x[3] = -np.abs(x[3]) * 1e-3                  # small negatives: codes that round to -0
+        x[3, 5] = -1000.0                            # one outlier sets the row scale
+    bits = OF.f32_to_bf16_bits(x)
+    src = capi.bf16_tensor(bits)
+    tiles = (rows + 127) // 128
+    codes = torch.empty((rows, K // 2), dtype=torch.uint8, device="cuda")
+    sf = torch.full((tiles * 128 * K // 16,), 0xAA, dtype=torch.uint8, device="cuda")
+    scale = torch.empty((rows,), dtype=torch.float32, device="cuda")
+    capi.nvfp4_quantize_rows(src, codes, sf, scale)
+    rc, rs, rt = OF.quantize_rows_nvfp4(OF.bf16_value(bits).astype(np.float32))
+    sfa = sf.cpu().numpy()
+    assert np.array_equal(codes.cpu().numpy(), rc)
+    assert np.array_equal(sf_untile(sfa, rows, K), rs)
+    assert np.array_equal(scale.cpu().numpy().view(np.uint32), rt.view(np.uint32))
+    if rows % 128:                                   # rows past the end of the last tile: zero scales
+        pad = sf_untile(sfa, tiles * 128, K)[rows:]
+        assert not pad.any()
+
+
+def test_prepare_weights_bit_exact():
+    wl = workload("tiny_t4")
+    inp = site_inputs(wl)
+    cfg = capi.config_for(wl)
+    site = device_site(wl, inp)
+    prep = capi.moe_prepare_weights(cfg, site).cpu().numpy()
+    per = wl.E * wl.I * wl.H // 16
+    assert prep.size == 3 * per
+    for i, (p, rows, K) in enumerate((("gate", wl.I, wl.H), ("up", wl.I, wl.H), ("down", wl.H, wl.I))):
+        got = sf_untile(prep[i * per:(i + 1) * per], wl.E * rows, K)
+        assert np.array_equal(got, inp[f"{p}_scales"].reshape(wl.E * rows, K // 16)), p
+
+
+@pytest.mark.parametrize("T,E,k,local", [(4, 16, 4, (0, 16)), (1000, 16, 4, (0, 16)), (300, 32, 4, (8, 20)),
+                                          (4096, 288, 8, (0, 288))])
+def test_tile_rows_bit_exact(T, E, k, local):
+    rng = np.random.default_rng(T * 3 + E)
+    hot = rng.choice(E, min(E, 6), replace=False)
+    ids = np.stack([rng.choice(hot if rng.random() < 0.5 and len(hot) >= k else E, k, replace=False)
+                    for _ in range(T)]).astype(np.int32)
+    cfg = capi.SiteConfig(256, 128, 0, E, local[0], local[1], k, 2.5, 7.0)
+    buf = torch.empty(capi.moe_plan_size(cfg, T), dtype=torch.uint8, device="cuda")
+    plan = capi.moe_plan_carve(cfg, T, buf)
+    ws = capi.alloc_workspace(cfg, T, capi.PATH_DECODE)
+    capi.moe_permute(cfg, torch.from_numpy(ids).cuda(), plan, ws)
+    capi.moe_read_device_status(ws)
+    P = capi.moe_padded_rows(cfg, T)
+    assert P % 128 == 0
+    got = _arr(plan.tile_rows, P)
+    ref = expected_tile_rows(OS.permute(ids, E), E, P, local)
+    assert np.array_equal(got, ref)
+
+
+# ------------------------------------------------------------------ site
+
+def _prefill(wl, inp, local=None, x_bits=None):
+    cfg = capi.config_for(wl, local)
+    site = device_site(wl, inp)
+    capi.moe_prepare_weights(cfg, site)
+    xb = inp["x"] if x_bits is None else x_bits
+    T = xb.shape[0]
+    x = capi.bf16_tensor(xb)
+    y = torch.empty_like(x)
+    ws = capi.alloc_workspace(cfg, T, capi.PATH_PREFILL)
+    capi.moe_forward(cfg, site, x, capi.PATH_PREFILL, y, ws)
+    capi.moe_read_device_status(ws)
+    v = capi.moe_workspace_views(cfg, T, capi.PATH_PREFILL, ws)
+    return cfg, site, y, ws, v
+
+
+def _site_state(wl, cfg, T, v):
+    """Copy the prefill intermediates of the workspace to the host."""
+    E, k, H, I = wl.E, wl.k, wl.H, wl.I
+    P = capi.moe_padded_rows(cfg, T)
+    ntiles = int(_arr(v.plan.tile_offsets, E + 1)[E])
+    Pu = ntiles * 128
+    st = dict(P=P, Pu=Pu, tile_rows=_arr(v.plan.tile_rows, P), tile_offsets=_arr(v.plan.tile_offsets, E + 1),
+              ids=_arr(v.ids, T * k).reshape(T, k), w=_arr(v.weights, T * k, torch.float32))
+    st["xq"] = capi.view_tensor(v.xq_codes, (P, H // 2), torch.uint8).cpu().numpy()[:Pu]
+    st["xsf"] = sf_untile(capi.view_tensor(v.xq_sf, (P * H // 16,), torch.uint8).cpu().numpy(), Pu, H)
+    st["xts"] = capi.view_tensor(v.xq_scale, (P,), torch.float32).cpu().numpy()[:Pu]
+    st["h"] = bf16_np(capi.view_tensor(v.h, (P, I), torch.bfloat16))[:Pu]
+    st["hq"] = capi.view_tensor(v.hq_codes, (P, I // 2), torch.uint8).cpu().numpy()[:Pu]
+    st["hsf"] = sf_untile(capi.view_tensor(v.hq_sf, (P * I // 16,), torch.uint8).cpu().numpy(), Pu, I)
+    st["hts"] = capi.view_tensor(v.hq_scale, (P,), torch.float32).cpu().numpy()[:Pu]
+    st["r"] = bf16_np(capi.view_tensor(v.r, (T, k, H), torch.bfloat16))
+    return st
+
+
+def _expert_of_rows(tile_offsets, Pu):
+    mt = np.arange(Pu) // 128
+    return np.searchsorted(tile_offsets, mt, side="right") - 1
+
+
+@pytest.mark.parametrize("T", [4, 33, 1000])
+def test_prefill_encodings_and_gemms_tiny(T):
+    """Each prefill step against the oracle on the GPU's own inputs: x codes
+    bit-exact, h = clamped SwiGLU of the FP4 gate/up GEMM (fp64 dot products of
+    the encoded operands), h codes bit-exact from the GPU's h, r = weight x the
+    FP4 down GEMM."""
+    wl = workload("tiny_t4", T)
+    inp = site_inputs(wl)
+    cfg, site, y, ws, v = _prefill(wl, inp)
+    st = _site_state(wl, cfg, T, v)
+    Pu, tr = st["Pu"], st["tile_rows"][:st["Pu"]]
+    valid = tr >= 0
+    # x encoded per assignment row (bit-exact), padding rows all zero
+    xsrc = np.zeros((Pu, wl.H), np.float32)
+    xsrc[valid] = OF.bf16_value(inp["x"][tr[valid] // wl.k]).astype(np.float32)
+    rc, rs, rt = OF.quantize_rows_nvfp4(xsrc)
+    assert np.array_equal(st["xq"], rc) and np.array_equal(st["xsf"], rs)
+    assert np.array_equal(st["xts"].view(np.uint32), rt.view(np.uint32))
+    # gate/up GEMM + clamped SwiGLU on the GPU's encoded x
+    xdeq = OF.dequant_rows_nvfp4(st["xq"], st["xsf"], st["xts"])
+    erow = _expert_of_rows(st["tile_offsets"], Pu)
+    cache = OS.ExpertCache(inp)
+    href = np.zeros((Pu, wl.I))
+    for e in np.unique(erow):
+        m = erow == e
+        wg, wu, _ = cache.get(int(e))
+        href[m] = OS.clamped_swiglu(xdeq[m] @ wg.T, xdeq[m] @ wu.T, wl.limit)
+    d = np.abs(st["h"] - href)
+    assert rel_l2(st["h"], href) < 4e-3
+    assert np.all(d <= 2.0 ** -8 * np.abs(href) + 1e-4 * np.abs(href).max()), d.max()
+    assert not st["h"][~valid].any()
+    # h encoded per padded row from the GPU's own bf16 h (bit-exact)
+    hsrc = np.where(valid[:, None], st["h"], 0.0).astype(np.float32)
+    hc, hs, ht = OF.quantize_rows_nvfp4(hsrc)
+    assert np.array_equal(st["hq"], hc) and np.array_equal(st["hsf"], hs)
+    assert np.array_equal(st["hts"].view(np.uint32), ht.view(np.uint32))
+    # down GEMM x routing weight, scattered to r[a]
+    hdeq = OF.dequant_rows_nvfp4(st["hq"], st["hsf"], st["hts"])
+    rref = np.zeros((T * wl.k, wl.H))
+    for e in np.unique(erow):
+        m = (erow == e) & valid
+        _, _, wd = cache.get(int(e))
+        rref[tr[m]] = st["w"][tr[m], None] * (hdeq[m] @ wd.T)
+    r = st["r"].reshape(T * wl.k, wl.H)
+    d = np.abs(r - rref)
+    assert rel_l2(r, rref) < 4e-3
+    assert np.all(d <= 2.0 ** -8 * np.abs(rref) + 1e-4 * np.abs(rref).max()), d.max()
+
+
+def test_grouped_gemm_entry_point_matches_forward():
+    wl = workload("tiny_t4", 300)
+    inp = site_inputs(wl)
+    cfg, site, y, ws, v = _prefill(wl, inp)
+    T, P = wl.T, capi.moe_padded_rows(cfg, wl.T)
+    xq = capi.view_tensor(v.xq_codes, (P, wl.H // 2), torch.uint8)
+    xsf = capi.view_tensor(v.xq_sf, (P * wl.H // 16,), torch.uint8)
+    xts = capi.view_tensor(v.xq_scale, (P,), torch.float32)
+    hq = capi.view_tensor(v.hq_codes, (P, wl.I // 2), torch.uint8)
+    hsf = capi.view_tensor(v.hq_sf, (P * wl.I // 16,), torch.uint8)
+    hts = capi.view_tensor(v.hq_scale, (P,), torch.float32)
+    wts = capi.view_tensor(v.weights, (T * wl.k,), torch.float32)
+    ws2 = capi.alloc_workspace(cfg, T, capi.PATH_PREFILL)
+    h2 = torch.zeros((P, wl.I), dtype=torch.bfloat16, device="cuda")
+    capi.nvfp4_grouped_gemm(cfg, capi.PROJ_GATE_UP, xq, xsf, xts, T, v.plan, wts, site, h2, ws2)
+    r2 = torch.full((T * wl.k, wl.H), 7.0, dtype=torch.bfloat16, device="cuda")
+    capi.nvfp4_grouped_gemm(cfg, capi.PROJ_DOWN, hq, hsf, hts, T, v.plan, wts, site, r2, ws2)
+    capi.moe_read_device_status(ws2)
+    ntiles = int(_arr(v.plan.tile_offsets, wl.E + 1)[wl.E])
+    h = capi.view_tensor(v.h, (P, wl.I), torch.bfloat16)
+    r = capi.view_tensor(v.r, (T * wl.k, wl.H), torch.bfloat16)
+    assert torch.equal(h2[:ntiles * 128], h[:ntiles * 128])
+    assert torch.equal(r2, r)
+
+
+@pytest.mark.parametrize("name,T", [("tiny_t4", None), ("tiny_t4", 33), ("tiny_t4", 1000), ("prefill_t4096", None),
+                                    ("stress_t16384", None)])
+def test_moe_forward_prefill_matches_oracle(name, T):
+    wl = workload(name, T)
+    inp = site_inputs(wl)
+    cfg, site, y, ws, v = _prefill(wl, inp)
+    lg = capi.view_tensor(v.logits, (wl.T, wl.E), torch.float32).cpu().numpy()
+    if wl.T <= 40:
+        tokens = np.arange(wl.T)
+    else:
+        tokens = np.random.default_rng(2).choice(wl.T, 12, replace=False)
+        if wl.stress:                                 # include exactly tied tokens
+            tokens = np.unique(np.concatenate([tokens, inp["tie_tokens"][:4]]))
+    ref = OS.site_forward(inp, oracle_cfg(wl), "prefill", tokens=tokens, gpu_logits=lg[tokens], want_parts=True)
+    ids = capi.view_tensor(v.ids, (wl.T, wl.k), torch.int32).cpu().numpy()
+    assert np.array_equal(ids[tokens], ref["ids"])
+    got = bf16_np(y)[tokens]
+    assert_bf16_close(got, ref["y"], what=f"{wl.name} y")
+    r = capi.view_tensor(v.r, (wl.T, wl.k, wl.H), torch.bfloat16)
+    assert_bf16_close(bf16_np(r)[tokens], ref["r"], what="r")
+
+
+def test_prefill_is_deterministic_and_chunk_invariant():
+    """Per-row encodings keep every token independent of its batch: the routed
+    rows r of a chunked prefill equal those of the whole batch bit for bit."""
+    wl = workload("tiny_t4", 600)
+    inp = site_inputs(wl)
+    _, _, y1, _, v1 = _prefill(wl, inp)
+    r1 = capi.view_tensor(v1.r, (wl.T, wl.k, wl.H), torch.bfloat16).clone()
+    _, _, y2, _, _ = _prefill(wl, inp)
+    assert torch.equal(y1, y2)
+    cut = 217
+    _, _, ya, _, va = _prefill(wl, inp, x_bits=inp["x"][:cut])
+    ra = capi.view_tensor(va.r, (cut, wl.k, wl.H), torch.bfloat16).clone()
+    _, _, yb, _, vb = _prefill(wl, inp, x_bits=inp["x"][cut:])
+    rb = capi.view_tensor(vb.r, (wl.T - cut, wl.k, wl.H), torch.bfloat16).clone()
+    assert torch.equal(torch.cat([ra, rb]), r1)
+    assert_bf16_close(bf16_np(torch.cat([ya, yb])), bf16_np(y1), what="chunked y")
+
+
+@pytest.mark.parametrize("T", [4, 300])
+def test_prefill_local_range_masks_remote_experts(T):
+    wl = workload("tiny_t4", T)
+    inp = site_inputs(wl)
+    local = (5, 11)
+    cfg, site, y, ws, v = _prefill(wl, inp, local=local)
+    lg = capi.view_tensor(v.logits, (wl.T, wl.E), torch.float32).cpu().numpy()
+    tokens = np.arange(min(T, 40))
+    ref = OS.site_forward(inp, oracle_cfg(wl, local), "prefill", tokens=tokens, gpu_logits=lg[tokens],
+                          want_parts=True)
+    assert_bf16_close(bf16_np(y)[tokens], ref["y"], what="local y")
+    ids = capi.view_tensor(v.ids, (wl.T, wl.k), torch.int32).cpu().numpy()
+    r = bf16_np(capi.view_tensor(v.r, (wl.T, wl.k, wl.H), torch.bfloat16))
+    remote = (ids < local[0]) | (ids >= local[1])
+    assert remote.any() and not r[remote].any()
