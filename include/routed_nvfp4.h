@@ -311,7 +311,11 @@ moe_status_t moe_combine(int32_t T, int32_t k, int32_t H, const uint16_t* r, con
  *   y = down_proj( clamped_swiglu(gate_proj x, up_proj x) )
  *   x bf16 [T, H]; wg, wu bf16 [I, H]; wd bf16 [H, I]; y bf16 [T, H].
  *   fp32 accumulation; h is rounded to bf16 between the two projections.
- *   H and I multiples of 64. ws: at least dense_ffn_workspace_size(H, I, T).
+ *   H and I multiples of 64. ws: at least dense_ffn_workspace_size(H, I, T);
+ *   its first 4 bytes are a device status word (moe_read_device_status).
+ *   T >= 128 with I % 128 == 0 and H % 256 == 0 runs as two tcgen05 BF16
+ *   GEMMs (kind::f16), smaller T as a GEMV that streams the weights once per
+ *   group of up to 8 tokens.
  */
 size_t dense_ffn_workspace_size(int32_t H, int32_t I, int32_t T);
 moe_status_t dense_ffn_bf16(int32_t H, int32_t I, float limit, const uint16_t* x, int32_t T,

@@ -526,7 +526,9 @@ moe_status_t dense_ffn_bf16(int32_t H, int32_t I, float limit, const uint16_t* x
   if (ws_bytes < dense_ffn_workspace_size(H, I, T))
     return fail(MOE_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, dense_ffn_workspace_size(H, I, T));
   uint16_t* hbuf = (uint16_t*)((char*)ws + up(4));
-  RNX_CUDA(rnx::launch_dense_gemv(H, I, limit, x, T, wg, wu, wd, y, hbuf, (cudaStream_t)stream), "dense_ffn_bf16");
+  cudaStream_t st = (cudaStream_t)stream;
+  RNX_CUDA(cudaMemsetAsync(ws, 0, 4, st), "clear status");
+  RNX_CUDA(rnx::launch_dense_ffn(H, I, limit, x, T, wg, wu, wd, y, hbuf, (uint32_t*)ws, st), "dense_ffn_bf16");
   return MOE_OK;
 }
 
@@ -631,8 +633,8 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
   }
   RNX_CUDA(mark(MOE_STAGE_SHARED, st), "stage event");
   if (Is > 0) {
-    RNX_CUDA(rnx::launch_dense_gemv(H, Is, cfg->swiglu_limit, x, T, w->shared_gate, w->shared_up, w->shared_down,
-                                    shared, (uint16_t*)(b + L.shared_h), st),
+    RNX_CUDA(rnx::launch_dense_ffn(H, Is, cfg->swiglu_limit, x, T, w->shared_gate, w->shared_up, w->shared_down,
+                                   shared, (uint16_t*)(b + L.shared_h), status, st),
              "shared expert");
   }
   RNX_CUDA(mark(MOE_STAGE_COMBINE, st), "stage event");

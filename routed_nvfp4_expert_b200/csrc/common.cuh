@@ -104,6 +104,15 @@ RNX_DEVICE float clamped_swiglu(float g, float u, float limit) {
   return gc / (1.0f + expf(-gc)) * uc;
 }
 
+// The same with the fast exponential and division intrinsics (__expf,
+// __fdividef): a few fp32 ulps from clamped_swiglu, far inside the bf16
+// rounding that follows; used where the epilogue's issue rate matters.
+RNX_DEVICE float clamped_swiglu_fast(float g, float u, float limit) {
+  const float gc = fminf(g, limit);
+  const float uc = fminf(fmaxf(u, -limit), limit);
+  return __fdividef(gc, 1.0f + __expf(-gc)) * uc;
+}
+
 // Read-only, no-L1-allocate 128-bit global load for streamed weights.
 RNX_DEVICE uint4 ldg_stream(const void* p) {
   uint4 r;

@@ -149,4 +149,15 @@ cudaError_t launch_dense_gemv(int H, int I, float limit, const uint16_t* x, int 
   return launch_mt<false>(I, H, T, 0.f, hbuf, wd, nullptr, y, st);
 }
 
+cudaError_t launch_dense_ffn(int H, int I, float limit, const uint16_t* x, int T, const uint16_t* wg,
+                             const uint16_t* wu, const uint16_t* wd, uint16_t* y, uint16_t* hbuf, uint32_t* status,
+                             cudaStream_t st) {
+  if (T >= kDenseGemmMinT && I % 128 == 0 && H % 256 == 0) {
+    cudaError_t err = launch_bf16_gemm(true, x, T, H, wg, wu, I, limit, hbuf, status, st);
+    if (err != cudaSuccess) return err;
+    return launch_bf16_gemm(false, hbuf, T, I, wd, nullptr, H, 0.f, y, status, st);
+  }
+  return launch_dense_gemv(H, I, limit, x, T, wg, wu, wd, y, hbuf, st);
+}
+
 }  // namespace rnx

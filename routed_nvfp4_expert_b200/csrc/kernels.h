@@ -57,6 +57,20 @@ cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* scales, const fl
 cudaError_t launch_dense_gemv(int H, int I, float limit, const uint16_t* x, int T, const uint16_t* wg,
                               const uint16_t* wu, const uint16_t* wd, uint16_t* y, uint16_t* hbuf, cudaStream_t st);
 
+// BF16 GEMM on tcgen05 (kind::f16): out [M, N] = a [M, K] . b^T with b [N, K].
+// gate_up: b0 = gate rows, b1 = up rows; out = clamped_swiglu(a.b0^T, a.b1^T).
+// N a multiple of 128 (gate_up) or 256, K a multiple of 64. status: device
+// word for bounded-wait timeouts (nullable).
+cudaError_t launch_bf16_gemm(bool gate_up, const uint16_t* a, int M, int K, const uint16_t* b0, const uint16_t* b1,
+                             int N, float limit, uint16_t* out, uint32_t* status, cudaStream_t st);
+
+// Dense BF16 FFN, picking the GEMV form for small T and the tcgen05 GEMM for
+// T >= kDenseGemmMinT (when the shapes allow it).
+constexpr int kDenseGemmMinT = 128;
+cudaError_t launch_dense_ffn(int H, int I, float limit, const uint16_t* x, int T, const uint16_t* wg,
+                             const uint16_t* wu, const uint16_t* wd, uint16_t* y, uint16_t* hbuf, uint32_t* status,
+                             cudaStream_t st);
+
 // ---------------------------------------------------------------- prefill (W4A4, tcgen05)
 
 // Padded tile layout of the prefill: every local expert's rows start on a

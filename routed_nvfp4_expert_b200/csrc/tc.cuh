@@ -87,8 +87,9 @@ RNX_DEVICE void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
-// Each thread of the warp reads 32 consecutive 32-bit columns of its TMEM lane.
-RNX_DEVICE void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+// Each thread of the warp reads 32 consecutive 32-bit columns of its TMEM lane
+// into r[0..31] (r must index registers: constant offsets into local arrays).
+RNX_DEVICE void tmem_ld32(uint32_t taddr, uint32_t* r) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
       "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"

@@ -324,3 +324,23 @@ def test_dense_ffn_decode_matches_oracle(H, I, T):
     ref = OS.dense_ffn(x, d["dense_gate"], d["dense_up"], d["dense_down"], 7.0)
     assert_bf16_close(bf16_np(y), ref, what="dense y")
     assert rel_l2(bf16_np(y), ref) < 5e-3
+
+
+@pytest.mark.parametrize("H,I,T", [(256, 512, 300), (4096, 1024, 4096), (4096, 12288, 640)])
+def test_dense_ffn_tensor_core_matches_oracle(H, I, T):
+    """T >= 128 runs the tcgen05 BF16 GEMMs (ragged last m-tile at T=300);
+    the oracle checks sampled tokens, the last rows included."""
+    from routed_nvfp4_expert_b200 import synthetic as syn
+    wl = syn.Workload("dense", T=T, H=H, I=16, E=1, k=1, Is=0, dense_I=I, sigma_w=0.02 if H == 256 else 0.0064)
+    d = syn.make_dense(wl)
+    x = syn.make_router_and_x(wl)["x"]
+    tb = capi.bf16_tensor
+    y = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(capi.dense_ffn_workspace_size(H, I, T), dtype=torch.uint8, device="cuda")
+    capi.dense_ffn_bf16(7.0, tb(x), tb(d["dense_gate"]), tb(d["dense_up"]), tb(d["dense_down"]), y, ws)
+    capi.moe_read_device_status(ws)
+    tok = np.unique(np.concatenate([np.random.default_rng(T).choice(T, 12, replace=False), [T - 1, T - 2, 0]]))
+    ref = OS.dense_ffn(x[tok], d["dense_gate"], d["dense_up"], d["dense_down"], 7.0)
+    got = bf16_np(y)[tok]
+    assert_bf16_close(got, ref, what="dense y (tensor cores)")
+    assert rel_l2(got, ref) < 5e-3
