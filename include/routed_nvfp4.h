@@ -140,15 +140,15 @@ typedef struct {
  *   offsets      [E+1]  segment starts, offsets[E] = A
  *   sorted       [A]    assignment at sorted position p
  *   inv          [A]    sorted position of assignment a
- *   tile_offsets [E+1]  prefix sum over experts of ceil(counts/128) for LOCAL
- *                       experts (0 tiles for remote ones)
+ *   tile_offsets [E+1]  prefix sum over experts of ceil(counts/256) for LOCAL
+ *                       experts (0 tiles for remote ones): 256-row tiles
  *   active       [E+1]  active[0] = number of LOCAL experts with counts > 0,
  *                       active[1..] = their ids in ascending order
  *   first        [E]    first[u] = sorted[offsets[active[1+u]]], the first
  *                       assignment of the u-th active expert
  *   tile_rows    [P]    P = moe_padded_rows(cfg, T): the padded tile layout
  *                       of the prefill, in which every LOCAL expert's rows
- *                       start on a 128-row tile (tile_offsets); tile_rows[p]
+ *                       start on a 256-row tile (tile_offsets); tile_rows[p]
  *                       is the assignment at padded row p, -1 for padding and
  *                       for rows past the last tile. Filled by moe_permute
  *                       and by the prefill path of moe_forward.
@@ -180,8 +180,8 @@ size_t moe_plan_size(const moe_config_t* cfg, int32_t T);
 moe_status_t moe_plan_carve(const moe_config_t* cfg, int32_t T, void* buf, size_t bytes, moe_plan_t* plan);
 
 /* Rows P of the prefill's padded tile layout for T tokens: an upper bound on
- * sum over local experts of ceil(counts/128) * 128, namely
- * floor((A + 127 * min(A, E_local)) / 128) * 128 with A = T*k (0 on invalid
+ * sum over local experts of ceil(counts/256) * 256, namely
+ * floor((A + 255 * min(A, E_local)) / 256) * 256 with A = T*k (0 on invalid
  * arguments). Sizes tile_rows and the quantised activation buffers. */
 int64_t moe_padded_rows(const moe_config_t* cfg, int32_t T);
 
@@ -284,6 +284,9 @@ moe_status_t nvfp4_quantize_rows(const uint16_t* src, int32_t rows, int32_t K, u
  *       remote assignments are written as zeros.
  *   Requires w->prepared, I % 128 == 0, H % 256 == 0.
  *   ws: at least moe_workspace_size(cfg, T, MOE_PATH_PREFILL) bytes (status).
+ * The kernel runs on clusters of two CTAs (tcgen05.mma.cta_group::2, 256 x
+ * 256 tiles, M split across the pair, each CTA loading half of the weight
+ * tile); no TMA load uses cluster multicast.
  */
 moe_status_t nvfp4_grouped_gemm(const moe_config_t* cfg, int32_t proj, const uint8_t* act_codes,
                                 const uint8_t* act_sf, const float* act_scale, int32_t T, const moe_plan_t* plan,

@@ -14,7 +14,8 @@ namespace rnx {
 
 constexpr int kWarp = 32;
 constexpr int kNumSMs = 148;          // B200
-constexpr int kRowsPerTile = 128;     // M extent of one grouped-GEMM tile
+constexpr int kRowsPerTile = 256;     // expert segments of the padded prefill layout start on these
+                                      // boundaries (M of one CTA-pair tile of the FP4 grouped GEMM)
 
 // Device status word (first 4 bytes of every workspace). Kernels OR error
 // bits in; moe_read_device_status() reads and clears it.

@@ -1,0 +1,270 @@
+// Dense BF16 GEMMs on the 5th-generation tensor cores (tcgen05.mma
+// kind::f16 with bf16 operands, fp32 accumulators in tensor memory): the dense
+// FFN and the shared expert at large T (glm5next_mlp module docs, "The stack
+// this layer runs": DENSE gate_proj/up_proj -> clamped SwiGLU -> down_proj;
+// shared_experts BF16 gate/up -> clamped SwiGLU -> BF16 down).
+//   A = x [M, K] (or h), B = weight rows [N, K], both K-major bf16.
+//   GATE_UP: tile = 128 rows x (128 gate + 128 up weight rows); the epilogue
+//            applies the clamped SwiGLU and stores h bf16 [M, N].
+//   DOWN:    tile = 128 rows x 256 output features, stored bf16 [M, N].
+//
+// One persistent CTA per SM walks the (m-tile, n-tile) list with the m-tiles
+// innermost, so each weight tile is read from HBM once while x stays in L2.
+// Warp roles: warp 0 = TMA producer (4-stage ring of 64-element K slices, 128
+// bytes per row, 128-byte swizzle), warp 1 = MMA issuer (one thread, four
+// M=128 N=256 K=16 MMAs per stage), warp 2 = TMEM allocator (two 256-column
+// accumulators), warps 4-11 = epilogue (warp w reads TMEM lane quadrant w % 4
+// and one half of the accumulator columns, copies them to registers and
+// releases the buffer before the SwiGLU and the stores). Every wait is
+// bounded; a timeout sets the device status word and winds the CTA down
+// (copies and MMAs in flight drained, TMEM freed). No TMA load uses cluster
+// multicast.
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc.cuh"
+#include "tensor_map.h"
+
+namespace rnx {
+
+namespace {
+
+constexpr int kTileM = 128;
+constexpr int kTileN = 256;          // MMA N (GATE_UP: 128 gate + 128 up)
+constexpr int kStepK = 64;           // bf16 elements per stage: 128 bytes per row (one swizzle span)
+constexpr int kStages = 4;
+constexpr int kABytes = kTileM * 128;                // 16 KB
+constexpr int kBBytes = kTileN * 128;                // 32 KB
+constexpr int kStageBytes = kABytes + kBBytes;       // 48 KB
+constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+constexpr int kFirstEpiWarp = 4;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = (kFirstEpiWarp + kEpiWarps) * 32;   // 384
+constexpr uint32_t kTmemCols = 512;                          // two 256-column accumulators
+
+struct GemmParams {
+  CUtensorMap tma_a;       // A [M, K] bf16; box 64 x 128 rows, SW128
+  CUtensorMap tma_b0;      // GATE_UP: gate rows (box 128 rows); DOWN: weight rows (box 256 rows)
+  CUtensorMap tma_b1;      // GATE_UP: up rows
+  uint16_t* out;           // [M, out_cols]
+  uint32_t* status;
+  int M, K, out_cols;
+  float limit;
+};
+
+template <bool GATE_UP>
+__global__ void __launch_bounds__(kThreads, 1) bf16_gemm_kernel(const __grid_constant__ GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
+  __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], mma_done;
+  __shared__ uint32_t s_tmem;
+  __shared__ volatile int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_ksteps = p.K / kStepK;
+  const int n_ntiles = GATE_UP ? p.out_cols / 128 : p.out_cols / kTileN;
+  const int n_mtiles = (p.M + kTileM - 1) / kTileM;
+  const int n_tiles = n_mtiles * n_ntiles;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kEpiWarps);
+    }
+    mbar_init(&mma_done, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(&s_tmem, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int it = 0;
+      for (int tile = blockIdx.x; tile < n_tiles && !abort_flag; tile += gridDim.x) {
+        const int nt = tile / n_mtiles, mt = tile - nt * n_mtiles;   // m-tiles innermost
+        for (int ks = 0; ks < n_ksteps; ++ks, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+          if (!mbar_wait(&empty_bar[s], ph ^ 1u) || abort_flag) {
+            set_status(p.status, kDevErrTimeout);
+            abort_flag = 1;
+            break;
+          }
+          uint8_t* sA = smem + (size_t)s * kStageBytes;
+          uint8_t* sB = sA + kABytes;
+          mbar_arrive_expect_tx(&full_bar[s], (uint32_t)kStageBytes);
+          tma_load_2d(sA, &p.tma_a, ks * kStepK, mt * kTileM, &full_bar[s]);
+          if (GATE_UP) {
+            tma_load_2d(sB, &p.tma_b0, ks * kStepK, nt * 128, &full_bar[s]);
+            tma_load_2d(sB + kBBytes / 2, &p.tma_b1, ks * kStepK, nt * 128, &full_bar[s]);
+          } else {
+            tma_load_2d(sB, &p.tma_b0, ks * kStepK, nt * kTileN, &full_bar[s]);
+          }
+        }
+      }
+      // drain: every copy issued must have landed before the CTA may exit
+      for (int j = max(0, it - kStages); j < it; ++j)
+        if (!mbar_wait(&full_bar[j % kStages], (uint32_t)(j / kStages) & 1u)) set_status(p.status, kDevErrTimeout);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(kTileM, kTileN);
+      int it = 0, tc = 0;
+      for (int tile = blockIdx.x; tile < n_tiles && !abort_flag; tile += gridDim.x, ++tc) {
+        const int b = tc & 1;
+        const uint32_t use = (uint32_t)(tc >> 1);
+        // the epilogue must have drained this accumulator buffer's previous tile
+        if (!mbar_wait(&acc_empty[b], (use & 1u) ^ 1u)) {
+          set_status(p.status, kDevErrTimeout);
+          abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t acc = tmem + 256u * b;
+        for (int ks = 0; ks < n_ksteps; ++ks, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+          if (!mbar_wait(&full_bar[s], ph) || abort_flag) {
+            set_status(p.status, kDevErrTimeout);
+            abort_flag = 1;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t aA = smem_u32(smem + (size_t)s * kStageBytes), aB = aA + kABytes;
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb)   // K = 16 per MMA: 32 bytes of each row
+            mma_bf16(acc, sdesc_k_sw128(aA + 32 * kb), sdesc_k_sw128(aB + 32 * kb), idesc,
+                     (ks > 0 || kb > 0) ? 1u : 0u);
+          mma_commit(&empty_bar[s]);          // the stage is free once these MMAs have read it
+        }
+        if (abort_flag) break;
+        mma_commit(&acc_full[b]);             // the accumulator is final once every MMA is done
+      }
+      mma_commit(&mma_done);
+      if (!mbar_wait(&mma_done, 0)) set_status(p.status, kDevErrTimeout);
+    }
+  } else if (warp >= kFirstEpiWarp) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                          // TMEM lane quadrant this warp may access
+    const int ch = (warp - kFirstEpiWarp) >> 2;     // column half
+    int tc = 0;
+    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++tc) {
+      const int b = tc & 1;
+      const uint32_t use = (uint32_t)(tc >> 1);
+      const int nt = tile / n_mtiles, mt = tile - nt * n_mtiles;
+      const int row = mt * kTileM + q * 32 + lane;   // A row = TMEM lane of this thread
+      const bool valid = row < p.M;
+      if (!mbar_wait(&acc_full[b], use & 1u) || abort_flag) {
+        set_status(p.status, kDevErrTimeout);
+        abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tq = tmem + 256u * b + ((uint32_t)(q * 32) << 16);
+      if (GATE_UP) {
+        uint32_t g[64], u[64];
+        tmem_ld32(tq + 64 * ch, g);
+        tmem_ld32(tq + 64 * ch + 32, g + 32);
+        tmem_ld32(tq + 128 + 64 * ch, u);
+        tmem_ld32(tq + 128 + 64 * ch + 32, u + 32);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[b]);
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(p.out + (size_t)row * p.out_cols + nt * 128 + 64 * ch);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int k0 = 8 * c + 2 * i;
+              w[i] = pack_bf16x2(clamped_swiglu_fast(__uint_as_float(g[k0]), __uint_as_float(u[k0]), p.limit),
+                                 clamped_swiglu_fast(__uint_as_float(g[k0 + 1]), __uint_as_float(u[k0 + 1]), p.limit));
+            }
+            dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      } else {
+        uint32_t v[128];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) tmem_ld32(tq + 128 * ch + 32 * j, v + 32 * j);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[b]);
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(p.out + (size_t)row * p.out_cols + nt * kTileN + 128 * ch);
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              w[i] = pack_bf16x2(__uint_as_float(v[8 * c + 2 * i]), __uint_as_float(v[8 * c + 2 * i + 1]));
+            dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+bool bf16_map(CUtensorMap* m, const uint16_t* base, int K, int rows, uint32_t box_rows) {
+  return make_tensor_map_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)K, (uint64_t)rows, kStepK,
+                            box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+template <bool GU>
+cudaError_t launch(const GemmParams& p, cudaStream_t st) {
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaError_t err = cudaFuncSetAttribute(bf16_gemm_kernel<GU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           kSmemBytes);
+    if (err != cudaSuccess) return err;
+    attr_done = true;
+  }
+  bf16_gemm_kernel<GU><<<kNumSMs, kThreads, kSmemBytes, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bf16_gemm(bool gate_up, const uint16_t* a, int M, int K, const uint16_t* b0, const uint16_t* b1,
+                             int N, float limit, uint16_t* out, uint32_t* status, cudaStream_t st) {
+  if (M <= 0 || K % kStepK || N % (gate_up ? 128 : kTileN)) return cudaErrorInvalidValue;
+  GemmParams p;
+  memset(&p, 0, sizeof p);
+  if (!bf16_map(&p.tma_a, a, K, M, kTileM)) return cudaErrorInvalidValue;
+  if (!bf16_map(&p.tma_b0, b0, K, N, gate_up ? 128 : kTileN)) return cudaErrorInvalidValue;
+  if (gate_up && !bf16_map(&p.tma_b1, b1, K, N, 128)) return cudaErrorInvalidValue;
+  p.out = out;
+  p.status = status;
+  p.M = M;
+  p.K = K;
+  p.out_cols = N;
+  p.limit = limit;
+  return gate_up ? launch<true>(p, st) : launch<false>(p, st);
+}
+
+}  // namespace rnx

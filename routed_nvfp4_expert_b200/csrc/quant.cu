@@ -1,5 +1,6 @@
 // Prefill data movement around the FP4 grouped GEMM:
-//  - the padded tile layout (tile_rows: assignment of each padded row),
+//  - the padded tile layout (tile_rows: assignment of each padded row; every
+//    local expert starts on a kRowsPerTile = 256-row boundary),
 //  - NVFP4 encoding of bf16 activation rows (x gathered per assignment, or h
 //    in place) with one fp32 scale per row, an E4M3 scale per 16 elements and
 //    E2M1 codes, the scales written straight into the 512-byte atoms the
@@ -114,7 +115,7 @@ __global__ void __launch_bounds__(256) tile_rows_kernel(const int32_t* __restric
   const int ntiles = tile_offsets[E];
   for (long long p = (long long)blockIdx.x * blockDim.x + threadIdx.x; p < P_max;
        p += (long long)gridDim.x * blockDim.x) {
-    const int mt = (int)(p >> 7);
+    const int mt = (int)(p / kRowsPerTile);
     int a = -1;
     if (mt < ntiles) {
       int lo = 0, hi = E;   // largest e with tile_offsets[e] <= mt
@@ -122,7 +123,7 @@ __global__ void __launch_bounds__(256) tile_rows_kernel(const int32_t* __restric
         const int mid = (lo + hi) >> 1;
         if (tile_offsets[mid] <= mt) lo = mid; else hi = mid;
       }
-      const int row = (mt - tile_offsets[lo]) * kRowsPerTile + (int)(p & 127);
+      const int row = (mt - tile_offsets[lo]) * kRowsPerTile + (int)(p % kRowsPerTile);
       if (row < counts[lo]) a = sorted[offsets[lo] + row];
     }
     tile_rows[p] = a;
@@ -166,7 +167,7 @@ int grid_for(long long work, int per_block) {
 
 int64_t padded_rows_bound(int64_t A, int64_t E_local) {
   const int64_t n = std::min(A, E_local);
-  return (A + 127 * n) / kRowsPerTile * kRowsPerTile;
+  return (A + (kRowsPerTile - 1) * n) / kRowsPerTile * kRowsPerTile;
 }
 
 cudaError_t launch_tile_rows(const moe_plan_t& plan, int E, int64_t P_max, cudaStream_t st) {
@@ -180,7 +181,7 @@ cudaError_t launch_quant_rows(const uint16_t* src, int64_t rows, int K, const in
                               const int32_t* used_tiles, uint8_t* codes, uint8_t* sf, float* row_scale,
                               cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
-  const long long rows_pad = (rows + kRowsPerTile - 1) / kRowsPerTile * kRowsPerTile;
+  const long long rows_pad = (rows + 127) / 128 * 128;   // whole 128-row scale atoms
   const long long grid = (rows_pad + kQuantWarps - 1) / kQuantWarps;
   quant_rows_kernel<<<(unsigned)grid, kQuantWarps * 32, 0, st>>>(src, rows, rows_pad, K, row_map, div, used_tiles,
                                                                   codes, sf, row_scale);

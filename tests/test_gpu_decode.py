@@ -115,7 +115,7 @@ def _check_plan(got, ids, E, local=(0, None)):
     A = ids.size
     for key in ("counts", "offsets", "sorted", "inv"):
         assert np.array_equal(got[key], ref[key]), key
-    tiles = np.where((np.arange(E) >= lb) & (np.arange(E) < le), (ref["counts"] + 127) // 128, 0)
+    tiles = np.where((np.arange(E) >= lb) & (np.arange(E) < le), (ref["counts"] + 255) // 256, 0)   # 256-row tiles
     assert np.array_equal(got["tile_offsets"], np.concatenate([[0], np.cumsum(tiles)]))
     act = [e for e in range(lb, le) if ref["counts"][e] > 0]
     assert got["active"][0] == len(act) and np.array_equal(got["active"][1:1 + len(act)], act)

@@ -30,6 +30,9 @@ def sf_untile(atoms: np.ndarray, rows: int, K: int) -> np.ndarray:
     return atoms.reshape(-1)[off]
 
 
+TILE = 256   # rows of one padded-layout tile: every local expert starts on a multiple
+
+
 def expected_tile_rows(ref_plan: dict, E: int, P: int, local) -> np.ndarray:
     lb, le = local
     out = np.full(P, -1, np.int32)
@@ -39,8 +42,8 @@ def expected_tile_rows(ref_plan: dict, E: int, P: int, local) -> np.ndarray:
         if not (lb <= e < le) or c == 0:
             continue
         o = int(ref_plan["offsets"][e])
-        out[tile * 128: tile * 128 + c] = ref_plan["sorted"][o:o + c]
-        tile += (c + 127) // 128
+        out[tile * TILE: tile * TILE + c] = ref_plan["sorted"][o:o + c]
+        tile += (c + TILE - 1) // TILE
     return out
 
 
@@ -103,7 +106,7 @@ def test_tile_rows_bit_exact(T, E, k, local):
     capi.moe_permute(cfg, torch.from_numpy(ids).cuda(), plan, ws)
     capi.moe_read_device_status(ws)
     P = capi.moe_padded_rows(cfg, T)
-    assert P % 128 == 0
+    assert P % TILE == 0
     got = _arr(plan.tile_rows, P)
     ref = expected_tile_rows(OS.permute(ids, E), E, P, local)
     assert np.array_equal(got, ref)
@@ -131,7 +134,7 @@ def _site_state(wl, cfg, T, v):
     E, k, H, I = wl.E, wl.k, wl.H, wl.I
     P = capi.moe_padded_rows(cfg, T)
     ntiles = int(_arr(v.plan.tile_offsets, E + 1)[E])
-    Pu = ntiles * 128
+    Pu = ntiles * TILE
     st = dict(P=P, Pu=Pu, tile_rows=_arr(v.plan.tile_rows, P), tile_offsets=_arr(v.plan.tile_offsets, E + 1),
               ids=_arr(v.ids, T * k).reshape(T, k), w=_arr(v.weights, T * k, torch.float32))
     st["xq"] = capi.view_tensor(v.xq_codes, (P, H // 2), torch.uint8).cpu().numpy()[:Pu]
@@ -146,7 +149,7 @@ def _site_state(wl, cfg, T, v):
 
 
 def _expert_of_rows(tile_offsets, Pu):
-    mt = np.arange(Pu) // 128
+    mt = np.arange(Pu) // TILE
     return np.searchsorted(tile_offsets, mt, side="right") - 1
 
 
@@ -220,7 +223,7 @@ def test_grouped_gemm_entry_point_matches_forward():
     ntiles = int(_arr(v.plan.tile_offsets, wl.E + 1)[wl.E])
     h = capi.view_tensor(v.h, (P, wl.I), torch.bfloat16)
     r = capi.view_tensor(v.r, (T * wl.k, wl.H), torch.bfloat16)
-    assert torch.equal(h2[:ntiles * 128], h[:ntiles * 128])
+    assert torch.equal(h2[:ntiles * TILE], h[:ntiles * TILE])
     assert torch.equal(r2, r)
 
 
