@@ -91,18 +91,19 @@ __global__ void __launch_bounds__(kThreads, 1) bf16_gemm_kernel(const __grid_con
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      int it = 0;
-      for (int tile = blockIdx.x; tile < n_tiles && !abort_flag; tile += gridDim.x) {
-        const int nt = tile / n_mtiles, mt = tile - nt * n_mtiles;   // m-tiles innermost
-        for (int ks = 0; ks < n_ksteps; ++ks, ++it) {
-          const int s = it % kStages;
-          const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-          if (!mbar_wait(&empty_bar[s], ph ^ 1u) || abort_flag) {
-            set_status(p.status, kDevErrTimeout);
-            abort_flag = 1;
-            break;
-          }
+    // The whole warp runs the loop (warp-uniform state); one elected lane issues.
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+      const int nt = tile / n_mtiles, mt = tile - nt * n_mtiles;   // m-tiles innermost
+      for (int ks = 0; ks < n_ksteps; ++ks, ++it) {
+        const int s = it % kStages;
+        const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+        if (__any_sync(0xffffffffu, !mbar_wait(&empty_bar[s], ph ^ 1u) || abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (elect_one()) {
           uint8_t* sA = smem + (size_t)s * kStageBytes;
           uint8_t* sB = sA + kABytes;
           mbar_arrive_expect_tx(&full_bar[s], (uint32_t)kStageBytes);
@@ -114,49 +115,64 @@ __global__ void __launch_bounds__(kThreads, 1) bf16_gemm_kernel(const __grid_con
             tma_load_2d(sB, &p.tma_b0, ks * kStepK, nt * kTileN, &full_bar[s]);
           }
         }
+        __syncwarp();
       }
-      // drain: every copy issued must have landed before the CTA may exit
-      for (int j = max(0, it - kStages); j < it; ++j)
-        if (!mbar_wait(&full_bar[j % kStages], (uint32_t)(j / kStages) & 1u)) set_status(p.status, kDevErrTimeout);
     }
+    if (!ok && lane == 0) {
+      set_status(p.status, kDevErrTimeout);
+      abort_flag = 1;
+    }
+    // drain: every copy issued must have landed before the CTA may exit
+    for (int j = max(0, it - kStages); j < it; ++j)
+      if (!mbar_wait(&full_bar[j % kStages], (uint32_t)(j / kStages) & 1u) && lane == 0)
+        set_status(p.status, kDevErrTimeout);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = idesc_bf16(kTileM, kTileN);
-      int it = 0, tc = 0;
-      for (int tile = blockIdx.x; tile < n_tiles && !abort_flag; tile += gridDim.x, ++tc) {
-        const int b = tc & 1;
-        const uint32_t use = (uint32_t)(tc >> 1);
-        // the epilogue must have drained this accumulator buffer's previous tile
-        if (!mbar_wait(&acc_empty[b], (use & 1u) ^ 1u)) {
-          set_status(p.status, kDevErrTimeout);
-          abort_flag = 1;
+    // Whole warp in the loop, one elected lane issues; stage-0 descriptors are
+    // built once and advanced by constant offsets (16-byte units).
+    const uint32_t idesc = idesc_bf16(kTileM, kTileN);
+    const uint32_t s0 = smem_u32(smem);
+    const uint64_t dA0 = sdesc_k_sw128(s0), dB0 = sdesc_k_sw128(s0 + kABytes);
+    int it = 0, tc = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++tc) {
+      const int b = tc & 1;
+      const uint32_t use = (uint32_t)(tc >> 1);
+      // the epilogue must have drained this accumulator buffer's previous tile
+      if (__any_sync(0xffffffffu, !mbar_wait(&acc_empty[b], (use & 1u) ^ 1u))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t acc = tmem + 256u * b;
+      for (int ks = 0; ks < n_ksteps; ++ks, ++it) {
+        const int s = it % kStages;
+        const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+        if (__any_sync(0xffffffffu, !mbar_wait(&full_bar[s], ph) || abort_flag)) {
+          ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t acc = tmem + 256u * b;
-        for (int ks = 0; ks < n_ksteps; ++ks, ++it) {
-          const int s = it % kStages;
-          const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-          if (!mbar_wait(&full_bar[s], ph) || abort_flag) {
-            set_status(p.status, kDevErrTimeout);
-            abort_flag = 1;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t aA = smem_u32(smem + (size_t)s * kStageBytes), aB = aA + kABytes;
+        const uint64_t so = (uint64_t)((s * kStageBytes) >> 4);
+        if (elect_one()) {
 #pragma unroll
           for (int kb = 0; kb < 4; ++kb)   // K = 16 per MMA: 32 bytes of each row
-            mma_bf16(acc, sdesc_k_sw128(aA + 32 * kb), sdesc_k_sw128(aB + 32 * kb), idesc,
-                     (ks > 0 || kb > 0) ? 1u : 0u);
+            mma_bf16(acc, dA0 + so + 2 * kb, dB0 + so + 2 * kb, idesc, (ks > 0 || kb > 0) ? 1u : 0u);
           mma_commit(&empty_bar[s]);          // the stage is free once these MMAs have read it
         }
-        if (abort_flag) break;
-        mma_commit(&acc_full[b]);             // the accumulator is final once every MMA is done
+        __syncwarp();
       }
-      mma_commit(&mma_done);
-      if (!mbar_wait(&mma_done, 0)) set_status(p.status, kDevErrTimeout);
+      if (!ok) break;
+      if (elect_one()) mma_commit(&acc_full[b]);   // the accumulator is final once every MMA is done
+      __syncwarp();
     }
+    if (!ok && lane == 0) {
+      set_status(p.status, kDevErrTimeout);
+      abort_flag = 1;
+    }
+    if (elect_one()) mma_commit(&mma_done);
+    __syncwarp();
+    if (!mbar_wait(&mma_done, 0) && lane == 0) set_status(p.status, kDevErrTimeout);
   } else if (warp >= kFirstEpiWarp) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                          // TMEM lane quadrant this warp may access

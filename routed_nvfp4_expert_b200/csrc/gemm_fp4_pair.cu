@@ -132,20 +132,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
-    if (lane == 0) {
-      int it = 0;
-      for (int tile = pair; tile < n_tiles && !abort_flag; tile += n_pairs) {
-        const int mt = tile / n_ntiles, nt = tile - mt * n_ntiles;
-        const int e = find_expert(s_toff, E, mt);
-        const int arow = mt * kPairM + 128 * (int)rank;   // this CTA's A rows
-        for (int ks = 0; ks < n_ksteps; ++ks, ++it) {
-          const int s = it % kStages;
-          const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-          if (!mbar_wait(&empty_bar[s], ph ^ 1u) || abort_flag) {
-            set_status(p.status, kDevErrTimeout);
-            abort_flag = 1;
-            break;
-          }
+    // The whole warp runs the loop (warp-uniform state); one elected lane issues.
+    int it = 0;
+    bool ok = true;
+    for (int tile = pair; tile < n_tiles && ok; tile += n_pairs) {
+      const int mt = tile / n_ntiles, nt = tile - mt * n_ntiles;
+      const int e = find_expert(s_toff, E, mt);
+      const int arow = mt * kPairM + 128 * (int)rank;   // this CTA's A rows
+      const int rb = e * (p.bank_rows / 128);
+      for (int ks = 0; ks < n_ksteps; ++ks, ++it) {
+        const int s = it % kStages;
+        const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+        if (__any_sync(0xffffffffu, !mbar_wait(&empty_bar[s], ph ^ 1u) || abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (elect_one()) {
           uint8_t* st = smem + (size_t)s * kStageBytes;
           uint8_t* sA = st;
           uint8_t* sB = st + kABytes;
@@ -156,14 +158,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const int kb0 = ks * 4;
           tma_load_2d_pair(sA, &p.tma_a, ks * 128, arow, bar);
           if (GATE_UP) {
-            const int brow = e * p.bank_rows + nt * 128;
-            tma_load_2d_pair(sB, rank == 0 ? &p.tma_b0 : &p.tma_b1, ks * 128, brow, bar);
+            tma_load_2d_pair(sB, rank == 0 ? &p.tma_b0 : &p.tma_b1, ks * 128, e * p.bank_rows + nt * 128, bar);
           } else {
             tma_load_2d_pair(sB, &p.tma_b0, ks * 128, e * p.bank_rows + nt * kTileN + 128 * (int)rank, bar);
           }
           // scale atoms, 256-byte rows: atom j of a [..][KB][512] array spans rows 2j, 2j+1
           tma_load_2d_pair(sSFA, &p.tma_sfa, 0, 2 * ((mt * 2 + (int)rank) * KB + kb0), bar);
-          const int rb = e * (p.bank_rows / 128);
           if (GATE_UP) {
             tma_load_2d_pair(sSFB, &p.tma_sfb0, 0, 2 * ((rb + nt) * KB + kb0), bar);
             tma_load_2d_pair(sSFB + 2048, &p.tma_sfb1, 0, 2 * ((rb + nt) * KB + kb0), bar);
@@ -172,53 +172,85 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tma_load_2d_pair(sSFB + 2048, &p.tma_sfb0, 0, 2 * ((rb + 2 * nt + 1) * KB + kb0), bar);
           }
         }
+        __syncwarp();
       }
-      // drain (even CTA: its full barriers count both CTAs' bytes)
-      if (rank == 0)
-        for (int j = max(0, it - kStages); j < it; ++j)
-          if (!mbar_wait(&full_bar[j % kStages], (uint32_t)(j / kStages) & 1u)) set_status(p.status, kDevErrTimeout);
     }
+    if (!ok && lane == 0) {
+      set_status(p.status, kDevErrTimeout);
+      abort_flag = 1;
+    }
+    // drain (even CTA: its full barriers count both CTAs' bytes)
+    if (rank == 0)
+      for (int j = max(0, it - kStages); j < it; ++j)
+        if (!mbar_wait(&full_bar[j % kStages], (uint32_t)(j / kStages) & 1u) && lane == 0)
+          set_status(p.status, kDevErrTimeout);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (even CTA)
-    if (lane == 0 && rank == 0) {
+    // Whole warp in the loop, one elected lane issues; the descriptors of
+    // stage 0 are built once and advanced by constant offsets (16-byte units).
+    if (rank == 0) {
       const uint32_t idesc = idesc_mxf4nvf4(kPairM, kTileN);
+      const uint32_t s0 = smem_u32(smem);
+      const uint64_t dA0 = sdesc_k_sw128(s0), dB0 = sdesc_k_sw128(s0 + kABytes);
+      const uint64_t dSA0 = sdesc_sf_atom(s0 + kABytes + kBBytes);
+      const uint64_t dSB0 = sdesc_sf_atom(s0 + kABytes + kBBytes + kSfaBytes);
       int it = 0, tc = 0;
-      for (int tile = pair; tile < n_tiles && !abort_flag; tile += n_pairs, ++tc) {
+      bool ok = true;
+      for (int tile = pair; tile < n_tiles && ok; tile += n_pairs, ++tc) {
         // both CTAs' epilogues must have drained the accumulator of the previous tile
-        if (!mbar_wait_cluster(&acc_empty, ((uint32_t)tc & 1u) ^ 1u)) {
-          set_status(p.status, kDevErrTimeout);
-          abort_flag = 1;
+        if (__any_sync(0xffffffffu, !mbar_wait_cluster(&acc_empty, ((uint32_t)tc & 1u) ^ 1u))) {
+          ok = false;
           break;
         }
         tc_fence_after();
         for (int ks = 0; ks < n_ksteps; ++ks, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-          if (!mbar_wait(&full_bar[s], ph) || abort_flag) {
-            set_status(p.status, kDevErrTimeout);
-            abort_flag = 1;
+          if (__any_sync(0xffffffffu, !mbar_wait(&full_bar[s], ph) || abort_flag)) {
+            ok = false;
             break;
           }
           tc_fence_after();
-          uint8_t* st = smem + (size_t)s * kStageBytes;
-          const uint32_t aA = smem_u32(st), aB = aA + kABytes, aSFA = aB + kBBytes, aSFB = aSFA + kSfaBytes;
-          const int nmma = min(4, KB - ks * 4);
+          const uint64_t so = (uint64_t)((s * kStageBytes) >> 4);
           const uint32_t sfa_col = tmem + kColSf + kSfColsPerStage * s, sfb_col = sfa_col + 16;
-          for (int kb = 0; kb < nmma; ++kb) {
-            tmem_cp_sf_pair(sfa_col + 4 * kb, sdesc_sf_atom(aSFA + kb * 512));
-            tmem_cp_sf_pair(sfb_col + 8 * kb, sdesc_sf_atom(aSFB + kb * 512));
-            tmem_cp_sf_pair(sfb_col + 8 * kb + 4, sdesc_sf_atom(aSFB + 2048 + kb * 512));
+          const int nmma = min(4, KB - ks * 4);
+          if (elect_one()) {
+            if (nmma == 4) {
+#pragma unroll
+              for (int kb = 0; kb < 4; ++kb) {
+                tmem_cp_sf_pair(sfa_col + 4 * kb, dSA0 + so + 32 * kb);          // 512-byte atoms
+                tmem_cp_sf_pair(sfb_col + 8 * kb, dSB0 + so + 32 * kb);
+                tmem_cp_sf_pair(sfb_col + 8 * kb + 4, dSB0 + so + 128 + 32 * kb);
+              }
+#pragma unroll
+              for (int kb = 0; kb < 4; ++kb)   // K = 64 per MMA: 32 bytes of each row
+                mma_mxf4nvf4_pair(tmem, dA0 + so + 2 * kb, dB0 + so + 2 * kb, idesc, sfa_col + 4 * kb, sfb_col + 8 * kb,
+                                  (ks > 0 || kb > 0) ? 1u : 0u);
+            } else {
+              for (int kb = 0; kb < nmma; ++kb) {
+                tmem_cp_sf_pair(sfa_col + 4 * kb, dSA0 + so + 32 * kb);
+                tmem_cp_sf_pair(sfb_col + 8 * kb, dSB0 + so + 32 * kb);
+                tmem_cp_sf_pair(sfb_col + 8 * kb + 4, dSB0 + so + 128 + 32 * kb);
+              }
+              for (int kb = 0; kb < nmma; ++kb)
+                mma_mxf4nvf4_pair(tmem, dA0 + so + 2 * kb, dB0 + so + 2 * kb, idesc, sfa_col + 4 * kb, sfb_col + 8 * kb,
+                                  (ks > 0 || kb > 0) ? 1u : 0u);
+            }
+            mma_commit_pair_mc(&empty_bar[s], 0x3);   // frees the stage in both CTAs
           }
-          for (int kb = 0; kb < nmma; ++kb)
-            mma_mxf4nvf4_pair(tmem, sdesc_k_sw128(aA + 32 * kb), sdesc_k_sw128(aB + 32 * kb), idesc, sfa_col + 4 * kb,
-                              sfb_col + 8 * kb, (ks > 0 || kb > 0) ? 1u : 0u);
-          mma_commit_pair_mc(&empty_bar[s], 0x3);   // frees the stage in both CTAs
+          __syncwarp();
         }
-        if (abort_flag) break;
-        mma_commit_pair_mc(&acc_full, 0x3);          // accumulator final in both CTAs
+        if (!ok) break;
+        if (elect_one()) mma_commit_pair_mc(&acc_full, 0x3);   // accumulator final in both CTAs
+        __syncwarp();
       }
-      mma_commit_pair_mc(&mma_done, 0x1);
-      if (!mbar_wait(&mma_done, 0)) set_status(p.status, kDevErrTimeout);
+      if (!ok && lane == 0) {
+        set_status(p.status, kDevErrTimeout);
+        abort_flag = 1;
+      }
+      if (elect_one()) mma_commit_pair_mc(&mma_done, 0x1);
+      __syncwarp();
+      if (!mbar_wait(&mma_done, 0) && lane == 0) set_status(p.status, kDevErrTimeout);
     }
   } else if (warp >= kFirstEpiWarp) {
     // ------------------------------------------------------------ epilogue (both CTAs)

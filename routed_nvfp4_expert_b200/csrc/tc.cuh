@@ -22,6 +22,20 @@ RNX_DEVICE void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
 RNX_DEVICE void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 RNX_DEVICE void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
+// One lane of a converged warp (the others get false). Keeping the whole warp
+// in a role's loop and issuing tcgen05 / TMA instructions from the elected
+// lane keeps the loop state warp-uniform (uniform registers), which is what
+// lets one thread issue MMAs back to back.
+RNX_DEVICE bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .b32 r;\n\t.reg .pred p;\n\t"
+      "elect.sync r|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // ---------------------------------------------------------------- descriptors
 // Shared-memory matrix descriptor, K-major, 128-byte swizzle: rows of 128 B,
 // 8-row groups 1024 B apart (SBO), LBO unused (16 B), descriptor version 1.
