@@ -41,13 +41,17 @@ namespace {
 constexpr int kPairM = 256;          // rows of one pair tile (128 per CTA)
 constexpr int kTileN = 256;          // MMA N
 constexpr int kStepK = 256;          // FP4 elements per stage (128 bytes per row)
-constexpr int kStages = 5;
+constexpr int kStages = 4;
 constexpr int kABytes = 128 * 128;   // this CTA's A rows x 128 bytes
 constexpr int kBBytes = 128 * 128;   // this CTA's half of B
 constexpr int kSfaBytes = 2048;      // 4 atoms: this CTA's 128 rows, 4 K blocks
 constexpr int kSfbBytes = 4096;      // 8 atoms: all 256 B rows, 4 K blocks
 constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;   // 38 KB
-constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+// epilogue staging: each epilogue warp owns 32 rows of up to 256 bytes, row
+// pitch 272 bytes (16-byte rows spread over the banks for the per-row writes)
+constexpr int kStagePitch = 272;
+constexpr int kEpiStageBytes = 32 * kStagePitch;                           // per warp
+constexpr int kSmemBytes = kStages * kStageBytes + 8 * kEpiStageBytes + 1024;
 constexpr uint32_t kTxBytesPair = 2u * kStageBytes;                      // both CTAs' bytes of one stage
 constexpr int kFirstEpiWarp = 4;
 constexpr int kEpiWarps = 8;
@@ -254,10 +258,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kFirstEpiWarp) {
     // ------------------------------------------------------------ epilogue (both CTAs)
+    // Each thread owns one accumulator row (its TMEM lane) and one column half.
+    // The finished bf16 values go to this warp's staging rows in shared
+    // memory; lane 0 then writes each row with one bulk copy (the rows of a
+    // warp are scattered in global memory on the down projection).
     const int q = warp & 3;
     const int ch = (warp - kFirstEpiWarp) >> 2;
     const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
     const uint32_t acc_empty_even = mapa_shared(smem_u32(&acc_empty), 0);
+    uint8_t* stage_rows = smem + (size_t)kStages * kStageBytes + (size_t)(warp - kFirstEpiWarp) * kEpiStageBytes;
+    uint8_t* my_row = stage_rows + lane * kStagePitch;
+    constexpr int kRowOut = GATE_UP ? 128 : 256;     // bytes of this thread's row piece
     int tc = 0;
     for (int tile = pair; tile < n_tiles; tile += n_pairs, ++tc) {
       const int mt = tile / n_ntiles, nt = tile - mt * n_ntiles;
@@ -266,12 +277,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int asg = p.tile_rows[prow];
       const bool valid = asg >= 0;
       const float rs = p.row_scale[prow];
-      if (!mbar_wait(&acc_full, (uint32_t)tc & 1u) || abort_flag) {
-        set_status(p.status, kDevErrTimeout);
-        abort_flag = 1;
+      if (__any_sync(0xffffffffu, !mbar_wait(&acc_full, (uint32_t)tc & 1u) || abort_flag)) {
+        if (lane == 0) {
+          set_status(p.status, kDevErrTimeout);
+          abort_flag = 1;
+        }
         break;
       }
       tc_fence_after();
+      uint16_t* dst;                                 // global row piece of this thread
+      uint4 w4[GATE_UP ? 8 : 16];
       if (GATE_UP) {
         const float sg = rs * p.ts0[e], su = rs * p.ts1[e];
         uint32_t g[64], u[64];
@@ -283,7 +298,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(acc_empty_even);
-        uint4* dst = reinterpret_cast<uint4*>(p.out + (size_t)prow * p.out_cols + nt * 128 + 64 * ch);
+        dst = p.out + (size_t)prow * p.out_cols + nt * 128 + 64 * ch;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           uint32_t w[4];
@@ -294,7 +309,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 clamped_swiglu_fast(__uint_as_float(g[k0]) * sg, __uint_as_float(u[k0]) * su, p.limit),
                 clamped_swiglu_fast(__uint_as_float(g[k0 + 1]) * sg, __uint_as_float(u[k0 + 1]) * su, p.limit));
           }
-          dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+          w4[c] = make_uint4(w[0], w[1], w[2], w[3]);
         }
       } else {
         const int a = valid ? asg : 0;
@@ -306,19 +321,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(acc_empty_even);
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(p.out + (size_t)a * p.out_cols + nt * kTileN + 128 * ch);
+        dst = p.out + (size_t)a * p.out_cols + nt * kTileN + 128 * ch;
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            uint32_t w[4];
+        for (int c = 0; c < 16; ++c) {
+          uint32_t w[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              w[i] = pack_bf16x2(__uint_as_float(v[8 * c + 2 * i]) * sc, __uint_as_float(v[8 * c + 2 * i + 1]) * sc);
-            dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
-          }
+          for (int i = 0; i < 4; ++i)
+            w[i] = pack_bf16x2(__uint_as_float(v[8 * c + 2 * i]) * sc, __uint_as_float(v[8 * c + 2 * i + 1]) * sc);
+          w4[c] = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
+      // the previous tile's bulk copies must have read the staging rows
+      if (lane == 0) bulk_wait_read_all();
+      __syncwarp();
+#pragma unroll
+      for (int c = 0; c < kRowOut / 16; ++c) reinterpret_cast<uint4*>(my_row)[c] = w4[c];
+      fence_proxy_async_smem();        // generic-proxy writes visible to the bulk copies
+      __syncwarp();
+      const bool write = GATE_UP || valid;   // FP4 padding rows of h are written too (as zeros)
+      for (int r = 0; r < 32; ++r) {
+        uint16_t* d = reinterpret_cast<uint16_t*>(__shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(dst), r));
+        const bool wr = __shfl_sync(0xffffffffu, write, r);
+        if (lane == 0 && wr) bulk_s2g(d, stage_rows + r * kStagePitch, kRowOut);
+      }
+      if (lane == 0) bulk_commit_group();
     }
+    if (lane == 0) bulk_wait_all();
   }
 
   // no CTA leaves (or frees TMEM) while the pair's MMAs or copies may still

@@ -95,4 +95,16 @@ RNX_DEVICE void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* b
       : "memory");
 }
 
+// Shared -> global bulk copy (TMA engine), tracked by the issuing thread's
+// bulk async-group. dst, src 16-byte aligned; bytes a multiple of 16.
+RNX_DEVICE void bulk_s2g(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+}
+RNX_DEVICE void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until the source shared memory of every committed group was read.
+RNX_DEVICE void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Wait until every committed group has completed (writes performed).
+RNX_DEVICE void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 }  // namespace rnx
