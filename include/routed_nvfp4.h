@@ -279,9 +279,10 @@ moe_status_t nvfp4_quantize_rows(const uint16_t* src, int32_t rows, int32_t K, u
  * prefill of moe_forward); padding rows must be zero (codes, scales, scale).
  *   MOE_PROJ_GATE_UP (K = H): out = h bf16 [P, I], h[p] = clamped_swiglu(
  *       g, u) of padded row p (0 on padding rows); `weights` unused.
- *   MOE_PROJ_DOWN (K = I): out = r bf16 [T*k, H], r[a] = weights[a] *
- *       (down_e . hdeq[p]) for the padded row p of assignment a; rows of
- *       remote assignments are written as zeros.
+ *   MOE_PROJ_DOWN (K = I): out = rows bf16 [P, H] in the padded tile order,
+ *       rows[p] = weights[a] * (down_e . hdeq[p]) for the assignment a at
+ *       padded row p (0 on padding rows); moe_unpermute /
+ *       moe_unpermute_combine bring them back to token order.
  *   Requires w->prepared, I % 128 == 0, H % 256 == 0.
  *   ws: at least moe_workspace_size(cfg, T, MOE_PATH_PREFILL) bytes (status).
  * The kernel runs on clusters of two CTAs (tcgen05.mma.cta_group::2, 256 x
@@ -292,6 +293,26 @@ moe_status_t nvfp4_grouped_gemm(const moe_config_t* cfg, int32_t proj, const uin
                                 const uint8_t* act_sf, const float* act_scale, int32_t T, const moe_plan_t* plan,
                                 const float* weights, const moe_weights_t* w, uint16_t* out, void* ws,
                                 size_t ws_bytes, void* stream);
+
+/*
+ * Unpermute (the module list's moe_permute family: token sort / permute /
+ * unpermute): rows of the padded tile order back to token order.
+ *   rows bf16 [P, H] (nvfp4_grouped_gemm DOWN); ids int32 [T, k] and plan from
+ *   the same routing; out bf16 [T, k, H]: out[t, j] = rows[p] with p =
+ *   tile_offsets[e] * 256 + inv[a] - offsets[e] for a = t*k + j, e = ids[a]
+ *   local; zeros for remote assignments.
+ */
+moe_status_t moe_unpermute(const moe_config_t* cfg, const uint16_t* rows, int32_t T, const moe_plan_t* plan,
+                           const int32_t* ids, uint16_t* out, void* stream);
+
+/*
+ * Unpermute fused with moe_combine (the prefill's last step): y[t] =
+ * bf16( sum_{j=0}^{k-1} rows[p(t, j)] + shared[t] ), j ascending, then the
+ * unscaled shared row (NULL = none), fp32 accumulation, one rounding; a remote
+ * assignment adds a zero row. Same result as moe_unpermute then moe_combine.
+ */
+moe_status_t moe_unpermute_combine(const moe_config_t* cfg, const uint16_t* rows, int32_t T, const moe_plan_t* plan,
+                                   const int32_t* ids, const uint16_t* shared, uint16_t* y, void* stream);
 
 /*
  * Clamped SwiGLU (glm5next_mlp "Traps": the clamp is asymmetric):
@@ -345,8 +366,8 @@ moe_status_t nvfp4_dequant(const uint8_t* codes, const uint8_t* scales, const fl
  *   MOE_PATH_PREFILL: permute with the padded tile layout, x encoded to
  *     NVFP4 per assignment row (nvfp4_quantize_rows), grouped GEMM gate/up
  *     with the clamped SwiGLU, h rounded to bf16 and encoded to NVFP4 per
- *     row, grouped GEMM down with the routing weight; needs w->prepared,
- *     I % 128 == 0, H % 256 == 0.
+ *     row, grouped GEMM down with the routing weight, unpermute fused with
+ *     the combine; needs w->prepared, I % 128 == 0, H % 256 == 0.
  */
 moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const uint16_t* x, int32_t T,
                          int32_t path, uint16_t* y, void* ws, size_t ws_bytes, void* stream);
@@ -354,7 +375,8 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
 /* Device pointers (inside ws) of the intermediates moe_forward leaves behind:
  * logits fp32 [T,E], ids int32 [T,k], weights fp32 [T,k], the plan, h bf16
  * ([T*k, I] on the decode path, [P, I] in padded tile rows on the prefill
- * path), r bf16 [T*k, H], shared bf16 [T, H] (NULL when Is == 0), and on the
+ * path), r bf16 (decode: [T*k, H] in token order; prefill: [P, H] in the
+ * padded tile order), shared bf16 [T, H] (NULL when Is == 0), and on the
  * prefill path the NVFP4-encoded x and h in padded tile rows (codes, scale
  * atoms, row scales; NULL on the decode path). Host-only pointer arithmetic. */
 typedef struct {

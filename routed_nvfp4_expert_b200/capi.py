@@ -28,7 +28,7 @@ EXPORTED = (
     "nvfp4_expert_gemv", "clamped_swiglu", "moe_combine", "dense_ffn_workspace_size", "dense_ffn_bf16",
     "nvfp4_dequant", "moe_forward", "moe_workspace_views", "moe_read_device_status", "moe_last_error",
     "moe_set_stage_events", "moe_forward_decode_noalloc", "moe_padded_rows", "moe_prepared_size",
-    "moe_prepare_weights", "nvfp4_quantize_rows", "nvfp4_grouped_gemm",
+    "moe_prepare_weights", "nvfp4_quantize_rows", "nvfp4_grouped_gemm", "moe_unpermute", "moe_unpermute_combine",
 )
 STAGES = ("router_logits", "topk", "permute", "act_quant", "expert_gate_up", "h_quant", "expert_down", "shared",
           "combine")
@@ -100,6 +100,8 @@ def load_library(path: str = _LIB_PATH) -> C.CDLL:
         "nvfp4_quantize_rows": (st, [vp, i32, i32, vp, vp, vp, vp]),
         "nvfp4_grouped_gemm": (st, [cfgp, i32, vp, vp, vp, i32, C.POINTER(MoePlan), vp, C.POINTER(MoeWeights), vp,
                                     vp, sz, vp]),
+        "moe_unpermute": (st, [cfgp, vp, i32, C.POINTER(MoePlan), vp, vp, vp]),
+        "moe_unpermute_combine": (st, [cfgp, vp, i32, C.POINTER(MoePlan), vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -308,6 +310,15 @@ def nvfp4_grouped_gemm(cfg: SiteConfig, proj: int, act_codes, act_sf, act_scale,
     _check(lib().nvfp4_grouped_gemm(C.byref(cfg.c()), proj, _p(act_codes), _p(act_sf), _p(act_scale), T,
                                     C.byref(plan), _p(weights), C.byref(w), _p(out), _p(ws), ws.numel(),
                                     _stream(stream)))
+
+
+def moe_unpermute(cfg: SiteConfig, rows, T: int, plan: MoePlan, ids, out, stream=None):
+    _check(lib().moe_unpermute(C.byref(cfg.c()), _p(rows), T, C.byref(plan), _p(ids), _p(out), _stream(stream)))
+
+
+def moe_unpermute_combine(cfg: SiteConfig, rows, T: int, plan: MoePlan, ids, shared, y, stream=None):
+    _check(lib().moe_unpermute_combine(C.byref(cfg.c()), _p(rows), T, C.byref(plan), _p(ids), _p(shared), _p(y),
+                                       _stream(stream)))
 
 
 def moe_workspace_views(cfg: SiteConfig, T: int, path: int, ws) -> MoeViews:

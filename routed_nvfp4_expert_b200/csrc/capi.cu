@@ -160,7 +160,7 @@ WsLayout ws_layout(const moe_config_t* c, int T, int path) {
   const bool pre = path == MOE_PATH_PREFILL;
   const size_t P = (size_t)L.pl.P;
   L.h = o; o = up(o + 2 * (pre ? P : A) * I);
-  L.r = o; o = up(o + 2 * A * H);
+  L.r = o; o = up(o + 2 * (pre ? P : A) * H);   // prefill: down rows in the padded tile order
   L.shared_h = o; o = up(o + 2 * (size_t)T * Is);
   L.shared = o; o = up(o + 2 * (size_t)T * H);
   L.xmax = o; o = up(o + 4 * (size_t)T);
@@ -372,10 +372,43 @@ moe_status_t nvfp4_grouped_gemm(const moe_config_t* cfg, int32_t proj, const uin
   RNX_CUDA(cudaMemsetAsync(status, 0, 4, st), "clear status");
   const rnx::Fp4GemmArgs g = gemm_args(cfg, proj, act_codes, act_sf, act_scale, L.pl.P, *plan, weights, w, out, status);
   RNX_CUDA(rnx::launch_fp4_grouped_gemm(g, st), "nvfp4_grouped_gemm");
-  if (proj == MOE_PROJ_DOWN)
-    RNX_CUDA(rnx::launch_zero_remote(plan->offsets, plan->sorted, cfg->num_experts, cfg->local_begin, cfg->local_end,
-                                     cfg->hidden, out, st),
-             "zero remote rows");
+  return MOE_OK;
+}
+
+moe_status_t moe_unpermute(const moe_config_t* cfg, const uint16_t* rows, int32_t T, const moe_plan_t* plan,
+                           const int32_t* ids, uint16_t* out, void* stream) {
+  moe_status_t s;
+  if ((s = check_cfg(cfg)) != MOE_OK || (s = check_T(T)) != MOE_OK) return s;
+  if (T == 0) return MOE_OK;
+  RNX_PTR(rows, "rows");
+  RNX_PTR(ids, "ids");
+  RNX_PTR(out, "out");
+  if (!plan) return fail(MOE_ERR_INVALID_ARG, "plan is NULL");
+  RNX_PTR(plan->offsets, "plan.offsets");
+  RNX_PTR(plan->inv, "plan.inv");
+  RNX_PTR(plan->tile_offsets, "plan.tile_offsets");
+  const rnx::PaddedIndex q{ids, plan->inv, plan->offsets, plan->tile_offsets, cfg->local_begin, cfg->local_end};
+  RNX_CUDA(rnx::launch_unpermute(q, (long long)T * cfg->top_k, cfg->hidden, rows, out, (cudaStream_t)stream),
+           "moe_unpermute");
+  return MOE_OK;
+}
+
+moe_status_t moe_unpermute_combine(const moe_config_t* cfg, const uint16_t* rows, int32_t T, const moe_plan_t* plan,
+                                   const int32_t* ids, const uint16_t* shared, uint16_t* y, void* stream) {
+  moe_status_t s;
+  if ((s = check_cfg(cfg)) != MOE_OK || (s = check_T(T)) != MOE_OK) return s;
+  if (T == 0) return MOE_OK;
+  RNX_PTR(rows, "rows");
+  RNX_PTR(ids, "ids");
+  RNX_PTR(y, "y");
+  if (shared && !aligned16(shared)) return fail(MOE_ERR_INVALID_ARG, "shared is not 16-byte aligned");
+  if (!plan) return fail(MOE_ERR_INVALID_ARG, "plan is NULL");
+  RNX_PTR(plan->offsets, "plan.offsets");
+  RNX_PTR(plan->inv, "plan.inv");
+  RNX_PTR(plan->tile_offsets, "plan.tile_offsets");
+  const rnx::PaddedIndex q{ids, plan->inv, plan->offsets, plan->tile_offsets, cfg->local_begin, cfg->local_end};
+  RNX_CUDA(rnx::launch_unpermute_combine(q, T, cfg->top_k, cfg->hidden, rows, shared, y, (cudaStream_t)stream),
+           "moe_unpermute_combine");
   return MOE_OK;
 }
 
@@ -612,8 +645,6 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
     RNX_CUDA(mark(MOE_STAGE_EXPERT_DOWN, st), "stage event");
     g = gemm_args(cfg, MOE_PROJ_DOWN, hq, hsf, hts, P, plan, wts, w, r, status);
     RNX_CUDA(rnx::launch_fp4_grouped_gemm(g, st), "expert down (tcgen05)");
-    RNX_CUDA(rnx::launch_zero_remote(plan.offsets, plan.sorted, E, cfg->local_begin, cfg->local_end, H, r, st),
-             "zero remote rows");
   } else {
     rnx::ExpertGemvArgs a{};
     a.T = T; a.H = H; a.I = I; a.E = E; a.k = k;
@@ -638,7 +669,12 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
              "shared expert");
   }
   RNX_CUDA(mark(MOE_STAGE_COMBINE, st), "stage event");
-  RNX_CUDA(rnx::launch_combine(T, k, H, r, shared, y, st), "combine");
+  if (path == MOE_PATH_PREFILL) {
+    const rnx::PaddedIndex q{ids, plan.inv, plan.offsets, plan.tile_offsets, cfg->local_begin, cfg->local_end};
+    RNX_CUDA(rnx::launch_unpermute_combine(q, T, k, H, r, shared, y, st), "unpermute + combine");
+  } else {
+    RNX_CUDA(rnx::launch_combine(T, k, H, r, shared, y, st), "combine");
+  }
   RNX_CUDA(mark(MOE_STAGE_COUNT, st), "stage event");
   return MOE_OK;
 }

@@ -47,6 +47,72 @@ __global__ void __launch_bounds__(256) combine_kernel(int T, int k, int H, const
   }
 }
 
+// Padded-layout row of assignment a (the prefill down projection writes its
+// rows there), -1 when its expert is outside the local range or the id was
+// dropped. tile_offsets are in kRowsPerTile-row tiles.
+RNX_DEVICE long long padded_pos(const PaddedIndex& q, long long a) {
+  const int e = q.ids[a];
+  if (e < q.local_begin || e >= q.local_end) return -1;
+  const int ia = q.inv[a];
+  if (ia < 0) return -1;
+  return (long long)q.tile_offsets[e] * kRowsPerTile + (ia - q.offsets[e]);
+}
+
+RNX_DEVICE void add_bf16x8(float (&acc)[8], uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float2 f = bf16x2_to_f32x2(w[q]);
+    acc[2 * q] += f.x;
+    acc[2 * q + 1] += f.y;
+  }
+}
+
+// Unpermute fused with moe_combine: y[t] = bf16(sum_j rows[pos(t, j)] +
+// shared[t]), j ascending then the shared row, fp32 accumulation; a remote
+// assignment adds a zero row (the same arithmetic as moe_combine over the
+// gathered rows). One CTA per token at a time; positions staged in shared.
+__global__ void __launch_bounds__(256) unpermute_combine_kernel(PaddedIndex q, int T, int k, int H,
+                                                                const uint16_t* __restrict__ rows,
+                                                                const uint16_t* __restrict__ shared,
+                                                                uint16_t* __restrict__ y) {
+  __shared__ long long pos[16];
+  const int per_row = H >> 3;
+  for (int t = blockIdx.x; t < T; t += gridDim.x) {
+    __syncthreads();
+    if (threadIdx.x < k) pos[threadIdx.x] = padded_pos(q, (long long)t * k + threadIdx.x);
+    __syncthreads();
+    for (int c = threadIdx.x; c < per_row; c += blockDim.x) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int j = 0; j < k; ++j) {
+        const long long pr = pos[j];
+        add_bf16x8(acc, pr >= 0 ? reinterpret_cast<const uint4*>(rows + (size_t)pr * H)[c] : make_uint4(0, 0, 0, 0));
+      }
+      if (shared) add_bf16x8(acc, reinterpret_cast<const uint4*>(shared + (size_t)t * H)[c]);
+      uint4 o;
+      o.x = pack_bf16x2(acc[0], acc[1]);
+      o.y = pack_bf16x2(acc[2], acc[3]);
+      o.z = pack_bf16x2(acc[4], acc[5]);
+      o.w = pack_bf16x2(acc[6], acc[7]);
+      reinterpret_cast<uint4*>(y + (size_t)t * H)[c] = o;
+    }
+  }
+}
+
+// Unpermute alone: out[t, j] = rows[pos(t, j)] (zeros for remote assignments).
+__global__ void __launch_bounds__(256) unpermute_kernel(PaddedIndex q, long long A, int H,
+                                                        const uint16_t* __restrict__ rows, uint16_t* __restrict__ out) {
+  const int per_row = H >> 3;
+  const long long n = A * per_row;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const long long a = i / per_row;
+    const int c = (int)(i - a * per_row);
+    const long long pr = padded_pos(q, a);
+    reinterpret_cast<uint4*>(out + (size_t)a * H)[c] =
+        pr >= 0 ? reinterpret_cast<const uint4*>(rows + (size_t)pr * H)[c] : make_uint4(0, 0, 0, 0);
+  }
+}
+
 __global__ void __launch_bounds__(256) swiglu_kernel(const float* __restrict__ gu, int M, int I, float limit,
                                                      uint16_t* __restrict__ h) {
   const int per_row = I >> 2;
@@ -98,6 +164,23 @@ int grid_for(long long n, int threads) {
 cudaError_t launch_combine(int T, int k, int H, const uint16_t* r, const uint16_t* shared, uint16_t* y,
                            cudaStream_t st) {
   combine_kernel<<<grid_for((long long)T * (H / 8), 256), 256, 0, st>>>(T, k, H, r, shared, y);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpermute_combine(const PaddedIndex& q, int T, int k, int H, const uint16_t* rows,
+                                     const uint16_t* shared, uint16_t* y, cudaStream_t st) {
+  if (T <= 0) return cudaSuccess;
+  const int grid = std::min(T, kNumSMs * 8);
+  unpermute_combine_kernel<<<grid, 256, 0, st>>>(q, T, k, H, rows, shared, y);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpermute(const PaddedIndex& q, long long A, int H, const uint16_t* rows, uint16_t* out,
+                             cudaStream_t st) {
+  if (A <= 0) return cudaSuccess;
+  const long long work = A * (H >> 3);
+  const int grid = (int)std::min<long long>((work + 255) / 256, (long long)kNumSMs * 16);
+  unpermute_kernel<<<grid, 256, 0, st>>>(q, A, H, rows, out);
   return cudaGetLastError();
 }
 

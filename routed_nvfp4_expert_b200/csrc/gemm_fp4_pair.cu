@@ -18,7 +18,8 @@
 //            the same 128 intermediate features; the epilogue applies the
 //            scales, the clamped SwiGLU, rounds h to bf16, stores [P, I].
 //   DOWN:    256 output features; the epilogue applies the scales and the
-//            routing weight and writes bf16 rows to r[a] of each assignment.
+//            routing weight and writes bf16 rows [P, H] in the padded tile
+//            order (the unpermute is fused into the combine that follows).
 //
 // Warp roles per CTA: warp 0 = TMA producer (5-stage ring, 38 KB per stage,
 // completions counted on the even CTA's barrier), warp 1 = MMA issuer (even
@@ -47,10 +48,10 @@ constexpr int kBBytes = 128 * 128;   // this CTA's half of B
 constexpr int kSfaBytes = 2048;      // 4 atoms: this CTA's 128 rows, 4 K blocks
 constexpr int kSfbBytes = 4096;      // 8 atoms: all 256 B rows, 4 K blocks
 constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;   // 38 KB
-// epilogue staging: each epilogue warp owns 32 rows of up to 256 bytes, row
-// pitch 272 bytes (16-byte rows spread over the banks for the per-row writes)
-constexpr int kStagePitch = 272;
-constexpr int kEpiStageBytes = 32 * kStagePitch;                           // per warp
+// epilogue staging: each epilogue warp owns two 32-row x 128-byte boxes in
+// the 128-byte swizzled layout of the output tensor map (TMA tensor stores)
+constexpr int kEpiBoxBytes = 32 * 128;
+constexpr int kEpiStageBytes = 2 * kEpiBoxBytes;                           // per warp
 constexpr int kSmemBytes = kStages * kStageBytes + 8 * kEpiStageBytes + 1024;
 constexpr uint32_t kTxBytesPair = 2u * kStageBytes;                      // both CTAs' bytes of one stage
 constexpr int kFirstEpiWarp = 4;
@@ -71,13 +72,13 @@ struct PairParams {
   CUtensorMap tma_sfa;     // A scale atoms viewed as [bytes/256, 256], box 256 x 8 (4 atoms)
   CUtensorMap tma_sfb0;    // gate (or down) scale atoms, same view
   CUtensorMap tma_sfb1;    // up scale atoms
+  CUtensorMap tma_out;     // output [P, out_cols] bf16, box 64 x 32, SW128
   const float* row_scale;  // [P]
   const float* ts0;        // [E]
   const float* ts1;        // [E]
   const int32_t* tile_offsets;   // [E+1], 256-row tiles
   const int32_t* tile_rows;      // [P]
   const float* weights;          // [A]
-  uint16_t* out;
   uint32_t* status;
   int E, K, out_cols, bank_rows;
   float limit;
@@ -259,24 +260,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp >= kFirstEpiWarp) {
     // ------------------------------------------------------------ epilogue (both CTAs)
     // Each thread owns one accumulator row (its TMEM lane) and one column half.
-    // The finished bf16 values go to this warp's staging rows in shared
-    // memory; lane 0 then writes each row with one bulk copy (the rows of a
-    // warp are scattered in global memory on the down projection).
+    // The finished bf16 values go to this warp's swizzled staging boxes; lane
+    // 0 writes each 32-row x 64-column box with one TMA tensor store. Output
+    // rows are in the padded tile order (padding rows hold zeros).
     const int q = warp & 3;
     const int ch = (warp - kFirstEpiWarp) >> 2;
     const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
     const uint32_t acc_empty_even = mapa_shared(smem_u32(&acc_empty), 0);
-    uint8_t* stage_rows = smem + (size_t)kStages * kStageBytes + (size_t)(warp - kFirstEpiWarp) * kEpiStageBytes;
-    uint8_t* my_row = stage_rows + lane * kStagePitch;
-    constexpr int kRowOut = GATE_UP ? 128 : 256;     // bytes of this thread's row piece
+    uint8_t* boxes = smem + (size_t)kStages * kStageBytes + (size_t)(warp - kFirstEpiWarp) * kEpiStageBytes;
+    constexpr int kBoxes = GATE_UP ? 1 : 2;          // 64 bf16 columns per box
     int tc = 0;
     for (int tile = pair; tile < n_tiles; tile += n_pairs, ++tc) {
       const int mt = tile / n_ntiles, nt = tile - mt * n_ntiles;
       const int e = find_expert(s_toff, E, mt);
-      const int prow = mt * kPairM + 128 * (int)rank + q * 32 + lane;   // padded row = TMEM lane
-      const int asg = p.tile_rows[prow];
-      const bool valid = asg >= 0;
-      const float rs = p.row_scale[prow];
+      const int row0 = mt * kPairM + 128 * (int)rank + q * 32;   // first padded row of this warp
+      const int asg = p.tile_rows[row0 + lane];
+      const float rs = p.row_scale[row0 + lane];
       if (__any_sync(0xffffffffu, !mbar_wait(&acc_full, (uint32_t)tc & 1u) || abort_flag)) {
         if (lane == 0) {
           set_status(p.status, kDevErrTimeout);
@@ -285,8 +284,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      uint16_t* dst;                                 // global row piece of this thread
-      uint4 w4[GATE_UP ? 8 : 16];
+      uint4 w4[8 * kBoxes];
+      int col0;                                      // first output column of this warp's boxes
       if (GATE_UP) {
         const float sg = rs * p.ts0[e], su = rs * p.ts1[e];
         uint32_t g[64], u[64];
@@ -298,7 +297,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(acc_empty_even);
-        dst = p.out + (size_t)prow * p.out_cols + nt * 128 + 64 * ch;
+        col0 = nt * 128 + 64 * ch;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           uint32_t w[4];
@@ -312,8 +311,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           w4[c] = make_uint4(w[0], w[1], w[2], w[3]);
         }
       } else {
-        const int a = valid ? asg : 0;
-        const float sc = valid ? rs * p.ts0[e] * p.weights[a] : 0.f;
+        const float sc = asg >= 0 ? rs * p.ts0[e] * p.weights[asg] : 0.f;
         uint32_t v[128];
 #pragma unroll
         for (int j = 0; j < 4; ++j) tmem_ld32(tq + 128 * ch + 32 * j, v + 32 * j);
@@ -321,7 +319,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(acc_empty_even);
-        dst = p.out + (size_t)a * p.out_cols + nt * kTileN + 128 * ch;
+        col0 = nt * kTileN + 128 * ch;
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           uint32_t w[4];
@@ -331,20 +329,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           w4[c] = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
-      // the previous tile's bulk copies must have read the staging rows
+      // the previous tile's stores must have read the staging boxes
       if (lane == 0) bulk_wait_read_all();
       __syncwarp();
 #pragma unroll
-      for (int c = 0; c < kRowOut / 16; ++c) reinterpret_cast<uint4*>(my_row)[c] = w4[c];
-      fence_proxy_async_smem();        // generic-proxy writes visible to the bulk copies
-      __syncwarp();
-      const bool write = GATE_UP || valid;   // FP4 padding rows of h are written too (as zeros)
-      for (int r = 0; r < 32; ++r) {
-        uint16_t* d = reinterpret_cast<uint16_t*>(__shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(dst), r));
-        const bool wr = __shfl_sync(0xffffffffu, write, r);
-        if (lane == 0 && wr) bulk_s2g(d, stage_rows + r * kStagePitch, kRowOut);
+      for (int c = 0; c < 8 * kBoxes; ++c) {       // 16-byte chunk c of this row, 128-byte swizzle
+        const int b = c >> 3, cc = c & 7;
+        *reinterpret_cast<uint4*>(boxes + b * kEpiBoxBytes + lane * 128 + ((cc ^ (lane & 7)) << 4)) = w4[c];
       }
-      if (lane == 0) bulk_commit_group();
+      fence_proxy_async_smem();        // generic-proxy writes visible to the tensor stores
+      __syncwarp();
+      if (lane == 0) {
+#pragma unroll
+        for (int b = 0; b < kBoxes; ++b) tma_store_2d(&p.tma_out, col0 + 64 * b, row0, boxes + b * kEpiBoxBytes);
+        bulk_commit_group();
+      }
+      __syncwarp();
     }
     if (lane == 0) bulk_wait_all();
   }
@@ -386,13 +386,15 @@ cudaError_t launch_fp4_grouped_gemm(const Fp4GemmArgs& a, cudaStream_t st) {
   if (!atom_map(&p.tma_sfa, a.a_sf, a.P_max / 128 * KB)) return cudaErrorInvalidValue;
   if (!atom_map(&p.tma_sfb0, a.b0_sf, brows / 128 * KB)) return cudaErrorInvalidValue;
   if (gu && !atom_map(&p.tma_sfb1, a.b1_sf, brows / 128 * KB)) return cudaErrorInvalidValue;
+  if (!make_tensor_map_2d(&p.tma_out, a.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.out_cols,
+                          (uint64_t)a.P_max, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
   p.row_scale = a.row_scale;
   p.ts0 = a.ts0;
   p.ts1 = a.ts1;
   p.tile_offsets = a.tile_offsets;
   p.tile_rows = a.tile_rows;
   p.weights = a.weights;
-  p.out = a.out;
   p.status = a.status;
   p.E = a.E;
   p.K = a.K;

@@ -47,6 +47,19 @@ cudaError_t launch_permute(const int32_t* ids, int A, int E, int local_begin, in
                            int32_t* scratch, uint32_t* status, cudaStream_t st);
 
 // elementwise
+// Where the prefill down projection left assignment a's row: padded row
+// tile_offsets[e] * kRowsPerTile + inv[a] - offsets[e] for a local expert e = ids[a].
+struct PaddedIndex {
+  const int32_t* ids;
+  const int32_t* inv;
+  const int32_t* offsets;
+  const int32_t* tile_offsets;
+  int local_begin, local_end;
+};
+cudaError_t launch_unpermute_combine(const PaddedIndex& q, int T, int k, int H, const uint16_t* rows,
+                                     const uint16_t* shared, uint16_t* y, cudaStream_t st);
+cudaError_t launch_unpermute(const PaddedIndex& q, long long A, int H, const uint16_t* rows, uint16_t* out,
+                             cudaStream_t st);
 cudaError_t launch_combine(int T, int k, int H, const uint16_t* r, const uint16_t* shared, uint16_t* y,
                            cudaStream_t st);
 cudaError_t launch_swiglu(const float* gu, int M, int I, float limit, uint16_t* h, cudaStream_t st);
@@ -93,10 +106,6 @@ cudaError_t launch_quant_rows(const uint16_t* src, int64_t rows, int K, const in
 // Canonical block scales [n_experts * rows, K/16] -> atoms [n_experts][rows/128][K/64][512].
 cudaError_t launch_sf_atoms(const uint8_t* scales, int64_t n_experts, int rows, int K, uint8_t* atoms, cudaStream_t st);
 
-// Zero the r rows of assignments routed to experts outside [lb, le).
-cudaError_t launch_zero_remote(const int32_t* offsets, const int32_t* sorted, int E, int lb, int le, int H,
-                               uint16_t* r, cudaStream_t st);
-
 struct Fp4GemmArgs {
   bool gate_up;
   int E, K, out_cols, bank_rows;   // bank_rows: rows of one expert in the weight bank (I for gate/up, H for down)
@@ -114,7 +123,7 @@ struct Fp4GemmArgs {
   const int32_t* tile_offsets;     // [E+1]
   const int32_t* tile_rows;        // [P_max]
   const float* weights;            // [A] routing weights (down)
-  uint16_t* out;                   // gate_up: h [P_max, out_cols]; down: r [A, out_cols]
+  uint16_t* out;                   // [P_max, out_cols] in the padded tile order (h, or weighted down rows)
   uint32_t* status;
 };
 cudaError_t launch_fp4_grouped_gemm(const Fp4GemmArgs& a, cudaStream_t st);

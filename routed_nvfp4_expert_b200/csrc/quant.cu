@@ -5,8 +5,7 @@
 //    in place) with one fp32 scale per row, an E4M3 scale per 16 elements and
 //    E2M1 codes, the scales written straight into the 512-byte atoms the
 //    tensor-core scale copy reads,
-//  - the one-time re-tiling of the weights' block scales into the same atoms,
-//  - zeroing of the rows routed to experts outside the local range.
+//  - the one-time re-tiling of the weights' block scales into the same atoms.
 //
 // Activation encoding (prefill reading of the glm5next_mlp module docs'
 // forward_prefill_gemm, W4A4 with a per-row second-level scale), every step
@@ -142,22 +141,6 @@ __global__ void __launch_bounds__(256) sf_atoms_kernel(const uint8_t* __restrict
   }
 }
 
-__global__ void __launch_bounds__(256) zero_remote_kernel(const int32_t* __restrict__ offsets,
-                                                          const int32_t* __restrict__ sorted, int E, int lb, int le,
-                                                          int H, uint16_t* __restrict__ r) {
-  const int rb0 = offsets[lb], re0 = offsets[le], rend = offsets[E];
-  const long long nremote = rb0 + (rend - re0);
-  const int vec = H / 8;
-  for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < nremote * vec;
-       idx += (long long)gridDim.x * blockDim.x) {
-    const long long rp = idx / vec;
-    const int col = (int)(idx - rp * vec);
-    const long long pos = rp < rb0 ? rp : re0 + (rp - rb0);
-    const int a = sorted[pos];
-    reinterpret_cast<uint4*>(r + (size_t)a * H)[col] = make_uint4(0, 0, 0, 0);
-  }
-}
-
 int grid_for(long long work, int per_block) {
   const long long g = (work + per_block - 1) / per_block;
   return (int)std::max(1LL, std::min(g, (long long)kNumSMs * 16));
@@ -193,13 +176,6 @@ cudaError_t launch_sf_atoms(const uint8_t* scales, int64_t n_experts, int rows, 
   const long long total = (long long)n_experts * rows;
   if (total <= 0) return cudaSuccess;
   sf_atoms_kernel<<<grid_for(total * (K / 64), 256), 256, 0, st>>>(scales, total, K, atoms);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_zero_remote(const int32_t* offsets, const int32_t* sorted, int E, int lb, int le, int H,
-                               uint16_t* r, cudaStream_t st) {
-  if (lb == 0 && le == E) return cudaSuccess;
-  zero_remote_kernel<<<kNumSMs, 256, 0, st>>>(offsets, sorted, E, lb, le, H, r);
   return cudaGetLastError();
 }
 

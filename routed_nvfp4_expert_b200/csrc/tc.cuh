@@ -128,6 +128,15 @@ RNX_DEVICE void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uin
       : "memory");
 }
 
+// 2D tiled store of the box at (x, y) from shared memory (the layout the
+// tensor map's swizzle describes), tracked by the thread's bulk async-group.
+// Rows or columns outside the tensor are not written.
+RNX_DEVICE void tma_store_2d(const CUtensorMap* map, int x, int y, const void* src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(map), "r"(x), "r"(y),
+               "r"(smem_u32(src))
+               : "memory");
+}
+
 // Plain 1D bulk copy without an L2 policy.
 RNX_DEVICE void bulk_g2s_plain(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(

@@ -144,8 +144,18 @@ def _site_state(wl, cfg, T, v):
     st["hq"] = capi.view_tensor(v.hq_codes, (P, I // 2), torch.uint8).cpu().numpy()[:Pu]
     st["hsf"] = sf_untile(capi.view_tensor(v.hq_sf, (P * I // 16,), torch.uint8).cpu().numpy(), Pu, I)
     st["hts"] = capi.view_tensor(v.hq_scale, (P,), torch.float32).cpu().numpy()[:Pu]
-    st["r"] = bf16_np(capi.view_tensor(v.r, (T, k, H), torch.bfloat16))
+    st["r_pad"] = bf16_np(capi.view_tensor(v.r, (P, H), torch.bfloat16))[:Pu]
     return st
+
+
+def _token_rows(cfg, wl, T, v):
+    """The routed rows r[t, j] in token order, through moe_unpermute."""
+    P = capi.moe_padded_rows(cfg, T)
+    rows = capi.view_tensor(v.r, (P, wl.H), torch.bfloat16)
+    ids = capi.view_tensor(v.ids, (T, wl.k), torch.int32)
+    out = torch.full((T, wl.k, wl.H), 3.0, dtype=torch.bfloat16, device="cuda")
+    capi.moe_unpermute(cfg, rows, T, v.plan, ids, out)
+    return out
 
 
 def _expert_of_rows(tile_offsets, Pu):
@@ -189,17 +199,21 @@ def test_prefill_encodings_and_gemms_tiny(T):
     hc, hs, ht = OF.quantize_rows_nvfp4(hsrc)
     assert np.array_equal(st["hq"], hc) and np.array_equal(st["hsf"], hs)
     assert np.array_equal(st["hts"].view(np.uint32), ht.view(np.uint32))
-    # down GEMM x routing weight, scattered to r[a]
+    # down GEMM x routing weight, rows in the padded tile order (padding rows zero)
     hdeq = OF.dequant_rows_nvfp4(st["hq"], st["hsf"], st["hts"])
-    rref = np.zeros((T * wl.k, wl.H))
+    rref = np.zeros((Pu, wl.H))
     for e in np.unique(erow):
         m = (erow == e) & valid
         _, _, wd = cache.get(int(e))
-        rref[tr[m]] = st["w"][tr[m], None] * (hdeq[m] @ wd.T)
-    r = st["r"].reshape(T * wl.k, wl.H)
+        rref[m] = st["w"][tr[m], None] * (hdeq[m] @ wd.T)
+    r = st["r_pad"]
     d = np.abs(r - rref)
     assert rel_l2(r, rref) < 4e-3
     assert np.all(d <= 2.0 ** -8 * np.abs(rref) + 1e-4 * np.abs(rref).max()), d.max()
+    assert not r[~valid].any()
+    # unpermute: token order, remote/padding never read
+    rt = bf16_np(_token_rows(cfg, wl, T, v)).reshape(T * wl.k, wl.H)
+    assert np.array_equal(rt[tr[valid]], r[valid])
 
 
 def test_grouped_gemm_entry_point_matches_forward():
@@ -217,14 +231,24 @@ def test_grouped_gemm_entry_point_matches_forward():
     ws2 = capi.alloc_workspace(cfg, T, capi.PATH_PREFILL)
     h2 = torch.zeros((P, wl.I), dtype=torch.bfloat16, device="cuda")
     capi.nvfp4_grouped_gemm(cfg, capi.PROJ_GATE_UP, xq, xsf, xts, T, v.plan, wts, site, h2, ws2)
-    r2 = torch.full((T * wl.k, wl.H), 7.0, dtype=torch.bfloat16, device="cuda")
+    r2 = torch.full((P, wl.H), 7.0, dtype=torch.bfloat16, device="cuda")
     capi.nvfp4_grouped_gemm(cfg, capi.PROJ_DOWN, hq, hsf, hts, T, v.plan, wts, site, r2, ws2)
     capi.moe_read_device_status(ws2)
     ntiles = int(_arr(v.plan.tile_offsets, wl.E + 1)[wl.E])
     h = capi.view_tensor(v.h, (P, wl.I), torch.bfloat16)
-    r = capi.view_tensor(v.r, (T * wl.k, wl.H), torch.bfloat16)
+    r = capi.view_tensor(v.r, (P, wl.H), torch.bfloat16)
     assert torch.equal(h2[:ntiles * TILE], h[:ntiles * TILE])
-    assert torch.equal(r2, r)
+    assert torch.equal(r2[:ntiles * TILE], r[:ntiles * TILE])
+    # the fused unpermute + combine equals unpermute then moe_combine, and y
+    ids = capi.view_tensor(v.ids, (T, wl.k), torch.int32)
+    sh = capi.view_tensor(v.shared, (T, wl.H), torch.bfloat16)
+    y2 = torch.empty_like(y)
+    capi.moe_unpermute_combine(cfg, r, T, v.plan, ids, sh, y2)
+    assert torch.equal(y2, y)
+    rt = _token_rows(cfg, wl, T, v)
+    y3 = torch.empty_like(y)
+    capi.moe_combine(rt, sh, y3)
+    assert torch.equal(y3, y)
 
 
 @pytest.mark.parametrize("name,T", [("tiny_t4", None), ("tiny_t4", 33), ("tiny_t4", 1000), ("prefill_t4096", None),
@@ -245,7 +269,7 @@ def test_moe_forward_prefill_matches_oracle(name, T):
     assert np.array_equal(ids[tokens], ref["ids"])
     got = bf16_np(y)[tokens]
     assert_bf16_close(got, ref["y"], what=f"{wl.name} y")
-    r = capi.view_tensor(v.r, (wl.T, wl.k, wl.H), torch.bfloat16)
+    r = _token_rows(cfg, wl, wl.T, v)
     assert_bf16_close(bf16_np(r)[tokens], ref["r"], what="r")
 
 
@@ -254,15 +278,15 @@ def test_prefill_is_deterministic_and_chunk_invariant():
     rows r of a chunked prefill equal those of the whole batch bit for bit."""
     wl = workload("tiny_t4", 600)
     inp = site_inputs(wl)
-    _, _, y1, _, v1 = _prefill(wl, inp)
-    r1 = capi.view_tensor(v1.r, (wl.T, wl.k, wl.H), torch.bfloat16).clone()
+    cfg1, _, y1, _, v1 = _prefill(wl, inp)
+    r1 = _token_rows(cfg1, wl, wl.T, v1)
     _, _, y2, _, _ = _prefill(wl, inp)
     assert torch.equal(y1, y2)
     cut = 217
-    _, _, ya, _, va = _prefill(wl, inp, x_bits=inp["x"][:cut])
-    ra = capi.view_tensor(va.r, (cut, wl.k, wl.H), torch.bfloat16).clone()
-    _, _, yb, _, vb = _prefill(wl, inp, x_bits=inp["x"][cut:])
-    rb = capi.view_tensor(vb.r, (wl.T - cut, wl.k, wl.H), torch.bfloat16).clone()
+    cfga, _, ya, _, va = _prefill(wl, inp, x_bits=inp["x"][:cut])
+    ra = _token_rows(cfga, wl, cut, va)
+    cfgb, _, yb, _, vb = _prefill(wl, inp, x_bits=inp["x"][cut:])
+    rb = _token_rows(cfgb, wl, wl.T - cut, vb)
     assert torch.equal(torch.cat([ra, rb]), r1)
     assert_bf16_close(bf16_np(torch.cat([ya, yb])), bf16_np(y1), what="chunked y")
 
@@ -279,6 +303,6 @@ def test_prefill_local_range_masks_remote_experts(T):
                           want_parts=True)
     assert_bf16_close(bf16_np(y)[tokens], ref["y"], what="local y")
     ids = capi.view_tensor(v.ids, (wl.T, wl.k), torch.int32).cpu().numpy()
-    r = bf16_np(capi.view_tensor(v.r, (wl.T, wl.k, wl.H), torch.bfloat16))
+    r = bf16_np(_token_rows(cfg, wl, wl.T, v))
     remote = (ids < local[0]) | (ids >= local[1])
     assert remote.any() and not r[remote].any()
