@@ -10,8 +10,10 @@ shared expert, combine) over one batch of synthetic inputs already resident in
 HBM, replayed from a CUDA graph of the public moe_forward call. L2 is flushed
 (a 2x-L2 buffer is read) before every timed step; each step is timed
 with CUDA events on the launching stream; the reported time is the max over
-ranks. The expert-GEMV roofline comes from stage events recorded by the
-library inside the same graph.
+ranks. The roofline of the dominant kernel comes from stage events recorded
+by the library inside the same graph: the expert GEMVs against HBM bandwidth
+on decode workloads (decode_t*), the tcgen05 FP4 grouped GEMMs against the
+dense FP4 tensor peak on prefill workloads (prefill_t4096, stress_t16384).
 
 `e2e` measures the same metric through moe_forward with host buffers: pinned
 host->device copy of x, the forward, device->host copy of y, all inside the
@@ -39,7 +41,8 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-METRIC = "MoE-layer tokens/s (decode) with expert-GEMV HBM GB/s vs roofline"
+METRIC = "MoE-layer tokens/s and achieved HBM GB/s (decode) / FP4 TFLOP/s (prefill) vs roofline"
+FP4_PER_BF16 = 4.0     # nominal dense FP4 / BF16 tensor throughput ratio of B200 (9 / 2.25 PFLOP/s)
 PER_EXPERT_NOTE = "gate+up+down codes, E4M3 scales and tensor scales of each touched expert"
 
 
@@ -61,6 +64,42 @@ def peaks():
 
 
 # ------------------------------------------------------------------ clocks
+
+class NvmlClocks:
+    """SM clock and clock-event reasons read through NVML between timed steps
+    (inside the timed loop, outside the CUDA-event intervals)."""
+    BITS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap"}
+
+    def __init__(self, gpu_index: int):
+        import pynvml
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        self.h = pynvml.nvmlDeviceGetHandleByIndex(gpu_index)
+        self.sm, self.reasons = [], set()
+        self.max = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+
+    def sample(self):
+        nv = self.nv
+        self.sm.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        get = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        bits = get(self.h)
+        for b, name in self.BITS.items():
+            if bits & b:
+                self.reasons.add(name)
+
+    def result(self):
+        if not self.sm:
+            return None
+        return {"sm_mhz": statistics.median(self.sm), "sm_max_mhz": self.max, "reasons": sorted(self.reasons),
+                "samples": len(self.sm), "source": "nvml, sampled after every timed step"}
+
+
+def clock_sampler(gpu_index: int):
+    try:
+        return NvmlClocks(gpu_index)
+    except Exception:          # no NVML: fall back to the nvidia-smi poller
+        return ClockSampler(gpu_index)
+
 
 class ClockSampler:
     """nvidia-smi clock / throttle sampling during the timed region."""
@@ -131,10 +170,13 @@ def run_ours(args, rank, world, local_rank):
     site = capi.site_to_device(inp, dev)
     cfg = capi.config_for(wl)
     path = capi.PATH_DECODE if wl.kind == "decode" else capi.PATH_PREFILL
+    prefill = path == capi.PATH_PREFILL
     T, H = wl.T, wl.H
+    if prefill:
+        capi.moe_prepare_weights(cfg, site)
 
     # rotating activations: a different routing every step (seeded per rank)
-    n_x = 16
+    n_x = 4 if prefill else 16
     x_pool = torch.stack([capi.bf16_tensor(syn.random_x(wl, T, seed=1000 * rank + i), dev) for i in range(n_x)])
     x = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
     y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
@@ -159,6 +201,10 @@ def run_ours(args, rank, world, local_rank):
     stream.synchronize()
     w_c = site.c()
     i_gu, i_sh = capi.STAGES.index("expert_gate_up"), capi.STAGES.index("shared")
+    i_hq, i_dn = capi.STAGES.index("h_quant"), capi.STAGES.index("expert_down")
+    # intervals of the dominant kernels: decode = both expert GEMVs (adjacent);
+    # prefill = the two grouped GEMMs (the h encoding between them excluded)
+    spans = [(i_gu, i_hq), (i_dn, i_sh)] if prefill else [(i_gu, i_sh)]
 
     # warm the kernels once outside capture, then capture the forward into graphs:
     #   timed: stage events only around the expert GEMVs (2 event nodes)
@@ -180,7 +226,8 @@ def run_ours(args, rank, world, local_rank):
         return g
 
     sparse = [None] * nst
-    sparse[i_gu], sparse[i_sh] = ev[i_gu], ev[i_sh]
+    for a_, b_ in spans:
+        sparse[a_], sparse[b_] = ev[a_], ev[b_]
     g_timed = capture(sparse)
     g_plain = capture(None)
     g_stages = capture(ev)
@@ -197,7 +244,7 @@ def run_ours(args, rank, world, local_rank):
         if with_stages == "all":
             return step, [ev[s].elapsed_time(ev[s + 1]) for s in range(nst - 1)]
         if with_stages:
-            return step, ev[i_gu].elapsed_time(ev[i_sh])
+            return step, sum(ev[a_].elapsed_time(ev[b_]) for a_, b_ in spans)
         return step, None
 
     for i in range(args.warmup):
@@ -206,17 +253,20 @@ def run_ours(args, rank, world, local_rank):
 
     dist_barrier(world)
     torch.cuda.synchronize(dev)
-    clocks = ClockSampler(local_rank)
-    clocks.start()
+    clocks = clock_sampler(local_rank)
+    if isinstance(clocks, ClockSampler):
+        clocks.start()
     step_ms, gemv_ms_l, uniq = [], [], []
     for i in range(args.steps):
         ms, gm = one_step(g_timed, args.warmup + i, True)
         step_ms.append(ms)
         gemv_ms_l.append(gm)
+        if isinstance(clocks, NvmlClocks):
+            clocks.sample()
         uniq.append(int(torch.unique(ids_view).numel()))
     torch.cuda.synchronize(dev)
     dist_barrier(world)
-    clk = clocks.stop()
+    clk = clocks.stop() if isinstance(clocks, ClockSampler) else clocks.result()
     capi.moe_read_device_status(ws, stream)
 
     # diagnostics (outside the timed region): no stage events; every stage
@@ -254,10 +304,29 @@ def run_ours(args, rank, world, local_rank):
 
     pk = peaks()
     U = float(np.mean(uniq))
-    algo_bytes = U * expert_bytes(wl)
-    achieved = algo_bytes / (gemv_ms * 1e-3) / 1e9
-    launches_per_step = 8 if T * wl.k <= 1024 else 10
-    traffic = read_traffic_profile()
+    if prefill:
+        flops = 2.0 * T * wl.k * 3 * H * wl.I          # gate + up + down over the T*k assignments
+        fp4_peak = pk["bf16_tflops"] * FP4_PER_BF16
+        achieved = flops / (gemv_ms * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "kernel": "nvfp4_grouped_gemm (tcgen05 mxf4nvf4; gate/up + down launches)",
+                    "achieved": round(achieved, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
+                    "frac": round(achieved / fp4_peak, 4),
+                    "peak_source": f"{pk['source']} bf16 burst x nominal FP4/BF16 ratio {FP4_PER_BF16:g}",
+                    "algorithmic_flops_per_step": flops, "unique_experts_per_step": U,
+                    "traffic": read_traffic_profile(f"nvfp4_grouped_gemm_{wl.name}")}
+        launches_per_step = 14
+        path_name = "prefill grouped GEMM (W4A4, tcgen05 block-scaled FP4)"
+    else:
+        algo_bytes = U * expert_bytes(wl)
+        achieved = algo_bytes / (gemv_ms * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "kernel": "nvfp4_expert_gemv (gate/up + down launches, timed together)",
+                    "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(achieved / pk["hbm_gbs"], 4), "peak_source": pk["source"],
+                    "algorithmic_bytes_per_step": int(algo_bytes), "unique_experts_per_step": U,
+                    "bytes_per_expert": expert_bytes(wl),
+                    "traffic": read_traffic_profile(f"nvfp4_expert_gemv_{wl.name}")}
+        launches_per_step = 8 if T * wl.k <= 1024 else 10
+        path_name = "decode GEMV (W4A16)"
     out = {
         "metric": METRIC,
         "value": round(world * T / (ms_max * 1e-3), 2),
@@ -269,21 +338,18 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "nvfp4 weights x bf16 activations, fp32 accumulate",
+        "dtype": ("nvfp4 weights x nvfp4 activations (tcgen05 mxf4nvf4), fp32 accumulate" if prefill
+                  else "nvfp4 weights x bf16 activations, fp32 accumulate"),
         "data": "synthetic (seeded; NVFP4 experts drawn in the code domain)",
         "config": {"workload": wl.name, "T": T, "hidden": H, "experts": wl.E, "intermediate": wl.I, "top_k": wl.k,
-                   "shared_intermediate": wl.Is, "path": "decode GEMV (W4A16)", "parallelism": f"replicas x{world}",
+                   "shared_intermediate": wl.Is, "path": path_name, "parallelism": f"replicas x{world}",
                    "l2": "flushed before every timed step (read of a 2x L2 buffer)", "graph": "CUDA graph of moe_forward"},
         "diagnostics": {
             "ms_per_step_without_stage_events": round(plain_ms, 5),
             "stages_ms_all_events": {n: round(float(v), 5) for n, v in zip(capi.STAGES, stage_avg)},
-            "note": "timed graph holds 2 stage-event nodes (around the expert GEMVs); stages_ms_all_events "
-                    "comes from a graph with an event node at every stage boundary"},
-        "roofline": {"bound": "hbm", "kernel": "nvfp4_expert_gemv (gate/up + down launches, timed together)",
-                     "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-                     "frac": round(achieved / pk["hbm_gbs"], 4), "peak_source": pk["source"],
-                     "algorithmic_bytes_per_step": int(algo_bytes), "unique_experts_per_step": U,
-                     "bytes_per_expert": expert_bytes(wl), "traffic": traffic},
+            "note": f"timed graph holds {2 * len(spans)} stage-event nodes (around the dominant kernels); "
+                    "stages_ms_all_events comes from a graph with an event node at every stage boundary"},
+        "roofline": roofline,
         "e2e": {"value": round(world * T / (e2e_max * 1e-3), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2,
                 "ms_per_step": round(e2e_max, 5)},
@@ -295,10 +361,10 @@ def run_ours(args, rank, world, local_rank):
     return out
 
 
-def read_traffic_profile():
-    """DRAM bytes per launch of the expert GEMV from the committed ncu summary,
-    if one exists for the current kernels (else null)."""
-    p = os.path.join(ROOT, "profiles", "nvfp4_expert_gemv_decode_t1.traffic.json")
+def read_traffic_profile(stem: str):
+    """DRAM bytes per step of the dominant kernel from the committed ncu
+    summary profiles/<stem>.traffic.json, if one exists (else null)."""
+    p = os.path.join(ROOT, "profiles", f"{stem}.traffic.json")
     if not os.path.exists(p):
         return None
     try:

@@ -185,9 +185,10 @@ moe_status_t moe_plan_carve(const moe_config_t* cfg, int32_t T, void* buf, size_
  * arguments). Sizes tile_rows and the quantised activation buffers. */
 int64_t moe_padded_rows(const moe_config_t* cfg, int32_t T);
 
-/* Bytes of the prepared weights (the block scales of gate, up and down
- * re-tiled into the 512-byte scale atoms of the tensor-core path):
- * 3 * E * I * H / 16. */
+/* Bytes of the prepared weights: the block scales of gate, up and down
+ * re-tiled into the 512-byte scale atoms of the tensor-core path
+ * (3 * E * I * H / 16 bytes), then the router weight split into three bf16
+ * terms (E * 3H * 2 bytes), each part starting on a 256-byte boundary. */
 size_t moe_prepared_size(const moe_config_t* cfg);
 
 /*
@@ -198,7 +199,12 @@ size_t moe_prepared_size(const moe_config_t* cfg);
  * (m%32)*16 + ((m%128)/32)*4 + b%4 (32 lanes x 4 columns x 4 blocks, the
  * layout the 32x128b tensor-memory copy spreads over the four lane
  * quadrants). Requires I % 128 == 0 and H % 256 == 0. Codes are used in
- * place. Run once per weight set; stream-ordered.
+ * place. Then the router weight w fp32 [E, H] as w3 bf16 [E, 3H] = (hi | mid |
+ * lo) per row with w = hi + mid + lo exactly (hi: w with the low 16 bits of
+ * its encoding cleared; mid: the same applied to w - hi; lo = w - hi - mid),
+ * so the prefill's router logits run as one bf16 tensor-core GEMM over K = 3H
+ * whose products are exact in the fp32 accumulator. Run once per weight set;
+ * stream-ordered.
  */
 moe_status_t moe_prepare_weights(const moe_config_t* cfg, const moe_weights_t* w, void* dst, size_t dst_bytes,
                                  void* stream);

@@ -184,12 +184,20 @@ moe_status_t check_prefill_shape(const moe_config_t* c) {
   return MOE_OK;
 }
 
+// Prepared weights: the experts' block scales as 512-byte atoms (gate, up,
+// down), then the router weight split exactly into three bf16 terms [E, 3H].
 struct PreparedLayout {
-  size_t gate, up, down, bytes;
+  size_t gate, up, down, router3, bytes;
 };
 PreparedLayout prepared_layout(const moe_config_t* c) {
   const size_t per = (size_t)c->num_experts * c->intermediate * c->hidden / 16;
-  return PreparedLayout{0, per, 2 * per, 3 * per};
+  const size_t r3 = up(3 * per);
+  return PreparedLayout{0, per, 2 * per, r3, r3 + up((size_t)c->num_experts * 3 * c->hidden * 2)};
+}
+
+// Prefill router on the tensor cores (needs the prepared split and E % 4 == 0).
+bool router_on_tensor_cores(const moe_config_t* c, int T, const moe_weights_t* w) {
+  return w->prepared && T >= rnx::kDenseGemmMinT && c->num_experts % 4 == 0;
 }
 
 rnx::Fp4GemmArgs gemm_args(const moe_config_t* c, int proj, const uint8_t* codes, const uint8_t* sf,
@@ -314,6 +322,7 @@ moe_status_t moe_prepare_weights(const moe_config_t* cfg, const moe_weights_t* w
   if ((s = check_bank(w->gate, "gate")) != MOE_OK || (s = check_bank(w->up, "up")) != MOE_OK ||
       (s = check_bank(w->down, "down")) != MOE_OK)
     return s;
+  RNX_PTR(w->router_w, "router_w");
   const PreparedLayout PL = prepared_layout(cfg);
   if (!dst || ((uintptr_t)dst % kAlign)) return fail(MOE_ERR_INVALID_ARG, "dst NULL or not 256-byte aligned");
   if (dst_bytes < PL.bytes) return fail(MOE_ERR_WORKSPACE, "dst has %zu bytes, needs %zu", dst_bytes, PL.bytes);
@@ -323,6 +332,7 @@ moe_status_t moe_prepare_weights(const moe_config_t* cfg, const moe_weights_t* w
   RNX_CUDA(rnx::launch_sf_atoms(w->gate.scales, E, I, H, d + PL.gate, st), "prepare gate scales");
   RNX_CUDA(rnx::launch_sf_atoms(w->up.scales, E, I, H, d + PL.up, st), "prepare up scales");
   RNX_CUDA(rnx::launch_sf_atoms(w->down.scales, E, H, I, d + PL.down, st), "prepare down scales");
+  RNX_CUDA(rnx::launch_router_split(w->router_w, E, H, (uint16_t*)(d + PL.router3), st), "prepare router split");
   return MOE_OK;
 }
 
@@ -618,7 +628,12 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
   RNX_CUDA(mark(MOE_STAGE_ROUTER_LOGITS, st), "stage event");
   uint32_t* xmax = (uint32_t*)(b + L.xmax);
   uint32_t* hmax = (uint32_t*)(b + L.hmax);
-  RNX_CUDA(rnx::launch_router_logits(x, T, H, E, w->router_w, logits, st, xmax, hmax, T * k), "router logits");
+  if (path == MOE_PATH_PREFILL && router_on_tensor_cores(cfg, T, w)) {
+    const uint16_t* w3 = (const uint16_t*)(w->prepared + prepared_layout(cfg).router3);
+    RNX_CUDA(rnx::launch_router_logits_tc(x, T, H, E, w3, logits, status, st), "router logits (tensor cores)");
+  } else {
+    RNX_CUDA(rnx::launch_router_logits(x, T, H, E, w->router_w, logits, st, xmax, hmax, T * k), "router logits");
+  }
   RNX_CUDA(mark(MOE_STAGE_TOPK, st), "stage event");
   RNX_CUDA(rnx::launch_topk(logits, w->router_bias, T, E, k, cfg->routed_scaling_factor, ids, wts, st), "top-k");
   RNX_CUDA(mark(MOE_STAGE_PERMUTE, st), "stage event");

@@ -7,6 +7,12 @@
 //   GATE_UP: tile = 128 rows x (128 gate + 128 up weight rows); the epilogue
 //            applies the clamped SwiGLU and stores h bf16 [M, N].
 //   DOWN:    tile = 128 rows x 256 output features, stored bf16 [M, N].
+//   LOGITS:  the router logits at large T (the glm5next_mlp stack's
+//            gate.weight -> fp32 logits) as one bf16 GEMM over K = 3H: the fp32
+//            router weight is split exactly into three bf16 terms w = hi + mid
+//            + lo ([E, 3H], built by moe_prepare_weights), x is read three
+//            times along K, products of bf16 are exact in the fp32
+//            accumulator; fp32 logits [M, E] are stored.
 //
 // One persistent CTA per SM walks the (m-tile, n-tile) list with the m-tiles
 // innermost, so each weight tile is read from HBM once while x stays in L2.
@@ -42,18 +48,24 @@ constexpr int kEpiWarps = 8;
 constexpr int kThreads = (kFirstEpiWarp + kEpiWarps) * 32;   // 384
 constexpr uint32_t kTmemCols = 512;                          // two 256-column accumulators
 
+enum { kModeGateUp = 0, kModeDown = 1, kModeLogits = 2 };
+
 struct GemmParams {
-  CUtensorMap tma_a;       // A [M, K] bf16; box 64 x 128 rows, SW128
-  CUtensorMap tma_b0;      // GATE_UP: gate rows (box 128 rows); DOWN: weight rows (box 256 rows)
+  CUtensorMap tma_a;       // A [M, a_period] bf16; box 64 x 128 rows, SW128
+  CUtensorMap tma_b0;      // GATE_UP: gate rows (box 128 rows); DOWN / LOGITS: weight rows (box 256 rows)
   CUtensorMap tma_b1;      // GATE_UP: up rows
-  uint16_t* out;           // [M, out_cols]
+  uint16_t* out;           // GATE_UP / DOWN: bf16 [M, out_cols]
+  float* out_f32;          // LOGITS: fp32 [M, out_cols], columns < out_cols written
   uint32_t* status;
   int M, K, out_cols;
+  int a_period;            // A's K extent; the K loop reads A at k mod a_period (LOGITS: K = 3 a_period)
   float limit;
 };
 
-template <bool GATE_UP>
+template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1) bf16_gemm_kernel(const __grid_constant__ GemmParams p) {
+  constexpr bool GATE_UP = MODE == kModeGateUp;
+  constexpr bool LOGITS = MODE == kModeLogits;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
@@ -63,7 +75,7 @@ __global__ void __launch_bounds__(kThreads, 1) bf16_gemm_kernel(const __grid_con
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_ksteps = p.K / kStepK;
-  const int n_ntiles = GATE_UP ? p.out_cols / 128 : p.out_cols / kTileN;
+  const int n_ntiles = GATE_UP ? p.out_cols / 128 : (p.out_cols + kTileN - 1) / kTileN;
   const int n_mtiles = (p.M + kTileM - 1) / kTileM;
   const int n_tiles = n_mtiles * n_ntiles;
 
@@ -107,7 +119,7 @@ __global__ void __launch_bounds__(kThreads, 1) bf16_gemm_kernel(const __grid_con
           uint8_t* sA = smem + (size_t)s * kStageBytes;
           uint8_t* sB = sA + kABytes;
           mbar_arrive_expect_tx(&full_bar[s], (uint32_t)kStageBytes);
-          tma_load_2d(sA, &p.tma_a, ks * kStepK, mt * kTileM, &full_bar[s]);
+          tma_load_2d(sA, &p.tma_a, LOGITS ? (ks * kStepK) % p.a_period : ks * kStepK, mt * kTileM, &full_bar[s]);
           if (GATE_UP) {
             tma_load_2d(sB, &p.tma_b0, ks * kStepK, nt * 128, &full_bar[s]);
             tma_load_2d(sB + kBBytes / 2, &p.tma_b1, ks * kStepK, nt * 128, &full_bar[s]);
@@ -223,7 +235,18 @@ __global__ void __launch_bounds__(kThreads, 1) bf16_gemm_kernel(const __grid_con
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[b]);
-        if (valid) {
+        if (LOGITS) {
+          if (valid) {
+            float* dst = p.out_f32 + (size_t)row * p.out_cols;
+            const int c0 = nt * kTileN + 128 * ch;
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              if (c0 + 4 * c < p.out_cols)
+                *reinterpret_cast<float4*>(dst + c0 + 4 * c) =
+                    make_float4(__uint_as_float(v[4 * c]), __uint_as_float(v[4 * c + 1]), __uint_as_float(v[4 * c + 2]),
+                                __uint_as_float(v[4 * c + 3]));
+          }
+        } else if (valid) {
           uint4* dst = reinterpret_cast<uint4*>(p.out + (size_t)row * p.out_cols + nt * kTileN + 128 * ch);
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
@@ -251,16 +274,16 @@ bool bf16_map(CUtensorMap* m, const uint16_t* base, int K, int rows, uint32_t bo
                             box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-template <bool GU>
+template <int MODE>
 cudaError_t launch(const GemmParams& p, cudaStream_t st) {
   static bool attr_done = false;
   if (!attr_done) {
-    cudaError_t err = cudaFuncSetAttribute(bf16_gemm_kernel<GU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t err = cudaFuncSetAttribute(bf16_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            kSmemBytes);
     if (err != cudaSuccess) return err;
     attr_done = true;
   }
-  bf16_gemm_kernel<GU><<<kNumSMs, kThreads, kSmemBytes, st>>>(p);
+  bf16_gemm_kernel<MODE><<<kNumSMs, kThreads, kSmemBytes, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -279,8 +302,25 @@ cudaError_t launch_bf16_gemm(bool gate_up, const uint16_t* a, int M, int K, cons
   p.M = M;
   p.K = K;
   p.out_cols = N;
+  p.a_period = K;
   p.limit = limit;
-  return gate_up ? launch<true>(p, st) : launch<false>(p, st);
+  return gate_up ? launch<kModeGateUp>(p, st) : launch<kModeDown>(p, st);
+}
+
+cudaError_t launch_router_logits_tc(const uint16_t* x, int T, int H, int E, const uint16_t* w3, float* logits,
+                                    uint32_t* status, cudaStream_t st) {
+  if (T <= 0 || H % kStepK || E % 4) return cudaErrorInvalidValue;
+  GemmParams p;
+  memset(&p, 0, sizeof p);
+  if (!bf16_map(&p.tma_a, x, H, T, kTileM)) return cudaErrorInvalidValue;
+  if (!bf16_map(&p.tma_b0, w3, 3 * H, E, kTileN)) return cudaErrorInvalidValue;
+  p.out_f32 = logits;
+  p.status = status;
+  p.M = T;
+  p.K = 3 * H;
+  p.out_cols = E;
+  p.a_period = H;
+  return launch<kModeLogits>(p, st);
 }
 
 }  // namespace rnx

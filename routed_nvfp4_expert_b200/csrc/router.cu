@@ -282,4 +282,37 @@ cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, in
   return cudaGetLastError();
 }
 
+namespace {
+
+// Exact three-term bf16 split of an fp32 weight: clearing the low 16 bits of
+// the encoding truncates to the leading 8 significand bits (a bf16 value);
+// each remainder is exact in fp32 and has 16, then 8 significant bits left.
+__global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ w, int E, int H,
+                                                           uint16_t* __restrict__ w3) {
+  const long long n = (long long)E * H;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const long long e = i / H;
+    const int c = (int)(i - e * H);
+    const float v = w[i];
+    const float hi = __uint_as_float(__float_as_uint(v) & 0xFFFF0000u);
+    const float r1 = v - hi;
+    const float mid = __uint_as_float(__float_as_uint(r1) & 0xFFFF0000u);
+    const float lo = r1 - mid;
+    uint16_t* row = w3 + e * 3 * H;
+    row[c] = (uint16_t)(__float_as_uint(hi) >> 16);
+    row[H + c] = (uint16_t)(__float_as_uint(mid) >> 16);
+    row[2 * H + c] = (uint16_t)(__float_as_uint(lo) >> 16);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_router_split(const float* w, int E, int H, uint16_t* w3, cudaStream_t st) {
+  const long long n = (long long)E * H;
+  if (n <= 0) return cudaSuccess;
+  const int grid = (int)std::min<long long>((n + 255) / 256, (long long)kNumSMs * 16);
+  router_split_kernel<<<grid, 256, 0, st>>>(w, E, H, w3);
+  return cudaGetLastError();
+}
+
 }  // namespace rnx

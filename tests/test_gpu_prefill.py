@@ -86,10 +86,16 @@ def test_prepare_weights_bit_exact():
     site = device_site(wl, inp)
     prep = capi.moe_prepare_weights(cfg, site).cpu().numpy()
     per = wl.E * wl.I * wl.H // 16
-    assert prep.size == 3 * per
+    r3 = (3 * per + 255) // 256 * 256
+    assert prep.size == r3 + (wl.E * 3 * wl.H * 2 + 255) // 256 * 256
     for i, (p, rows, K) in enumerate((("gate", wl.I, wl.H), ("up", wl.I, wl.H), ("down", wl.H, wl.I))):
         got = sf_untile(prep[i * per:(i + 1) * per], wl.E * rows, K)
         assert np.array_equal(got, inp[f"{p}_scales"].reshape(wl.E * rows, K // 16)), p
+    # router weight as three bf16 terms whose exact sum is the fp32 weight
+    w3 = prep[r3:r3 + wl.E * 3 * wl.H * 2].view(np.uint16).reshape(wl.E, 3, wl.H)
+    parts = OF.bf16_value(w3)
+    assert np.array_equal(parts[:, 0] + parts[:, 1] + parts[:, 2], inp["router_w"].astype(np.float64))
+    assert np.all(np.abs(parts[:, 1]) <= np.abs(parts[:, 0]) * 2.0 ** -7)
 
 
 @pytest.mark.parametrize("T,E,k,local", [(4, 16, 4, (0, 16)), (1000, 16, 4, (0, 16)), (300, 32, 4, (8, 20)),
@@ -265,6 +271,10 @@ def test_moe_forward_prefill_matches_oracle(name, T):
         if wl.stress:                                 # include exactly tied tokens
             tokens = np.unique(np.concatenate([tokens, inp["tie_tokens"][:4]]))
     ref = OS.site_forward(inp, oracle_cfg(wl), "prefill", tokens=tokens, gpu_logits=lg[tokens], want_parts=True)
+    # logits (tensor-core split-bf16 GEMM at T >= 128): 1e-5 of the token's largest logit
+    rl = ref["logits"]
+    scale = np.maximum(np.abs(rl), np.abs(rl).max(axis=1, keepdims=True))
+    assert np.all(np.abs(lg[tokens] - rl) <= 1e-5 * scale), np.abs(lg[tokens] - rl).max()
     ids = capi.view_tensor(v.ids, (wl.T, wl.k), torch.int32).cpu().numpy()
     assert np.array_equal(ids[tokens], ref["ids"])
     got = bf16_np(y)[tokens]
