@@ -199,8 +199,8 @@ size_t moe_prepared_size(const moe_config_t* cfg);
  * (m%32)*16 + ((m%128)/32)*4 + b%4 (32 lanes x 4 columns x 4 blocks, the
  * layout the 32x128b tensor-memory copy spreads over the four lane
  * quadrants). Requires I % 128 == 0 and H % 256 == 0. Codes are used in
- * place. Then the router weight w fp32 [E, H] as w3 bf16 [E, 3H] = (hi | mid |
- * lo) per row with w = hi + mid + lo exactly (hi: w with the low 16 bits of
+ * place. Then the router weight w fp32 [E, H] as w3 bf16 [E, 3H] = (lo | mid |
+ * hi) per row with w = hi + mid + lo exactly (hi: w with the low 16 bits of
  * its encoding cleared; mid: the same applied to w - hi; lo = w - hi - mid),
  * so the prefill's router logits run as one bf16 tensor-core GEMM over K = 3H
  * whose products are exact in the fp32 accumulator. Run once per weight set;

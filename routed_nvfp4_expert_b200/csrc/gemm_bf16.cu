@@ -9,10 +9,13 @@
 //   DOWN:    tile = 128 rows x 256 output features, stored bf16 [M, N].
 //   LOGITS:  the router logits at large T (the glm5next_mlp stack's
 //            gate.weight -> fp32 logits) as one bf16 GEMM over K = 3H: the fp32
-//            router weight is split exactly into three bf16 terms w = hi + mid
-//            + lo ([E, 3H], built by moe_prepare_weights), x is read three
-//            times along K, products of bf16 are exact in the fp32
-//            accumulator; fp32 logits [M, E] are stored.
+//            router weight is split exactly into three bf16 terms w = lo + mid
+//            + hi ([E, 3H] in that order, built by moe_prepare_weights), x is
+//            read three times along K, products of bf16 are exact in fp32.
+//            The tensor core's accumulation does not round to nearest, so the
+//            small lo and mid terms go first into an empty accumulator and the
+//            hi terms are spread over four accumulators (N = 128 tiles), whose
+//            partial sums the epilogue adds in fp32; fp32 logits [M, E].
 //
 // One persistent CTA per SM walks the (m-tile, n-tile) list with the m-tiles
 // innermost, so each weight tile is read from HBM once while x stays in L2.
@@ -66,6 +69,10 @@ template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1) bf16_gemm_kernel(const __grid_constant__ GemmParams p) {
   constexpr bool GATE_UP = MODE == kModeGateUp;
   constexpr bool LOGITS = MODE == kModeLogits;
+  // LOGITS: N = 128 tiles and four 128-column accumulators in one buffer (the
+  // K segments lo | mid | hi of the split weight go to accumulator 0, the
+  // hi segment's later three quarters to 1..3; partial sums added in fp32)
+  constexpr int kTN = LOGITS ? 128 : kTileN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
@@ -75,7 +82,8 @@ __global__ void __launch_bounds__(kThreads, 1) bf16_gemm_kernel(const __grid_con
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_ksteps = p.K / kStepK;
-  const int n_ntiles = GATE_UP ? p.out_cols / 128 : (p.out_cols + kTileN - 1) / kTileN;
+  const int n_ntiles = GATE_UP ? p.out_cols / 128 : (p.out_cols + kTN - 1) / kTN;
+  const int seg = p.a_period / kStepK, q4 = seg / 4;     // LOGITS: k-steps per segment / per hi quarter
   const int n_mtiles = (p.M + kTileM - 1) / kTileM;
   const int n_tiles = n_mtiles * n_ntiles;
 
@@ -118,13 +126,13 @@ __global__ void __launch_bounds__(kThreads, 1) bf16_gemm_kernel(const __grid_con
         if (elect_one()) {
           uint8_t* sA = smem + (size_t)s * kStageBytes;
           uint8_t* sB = sA + kABytes;
-          mbar_arrive_expect_tx(&full_bar[s], (uint32_t)kStageBytes);
+          mbar_arrive_expect_tx(&full_bar[s], (uint32_t)(kABytes + (LOGITS ? kBBytes / 2 : kBBytes)));
           tma_load_2d(sA, &p.tma_a, LOGITS ? (ks * kStepK) % p.a_period : ks * kStepK, mt * kTileM, &full_bar[s]);
           if (GATE_UP) {
             tma_load_2d(sB, &p.tma_b0, ks * kStepK, nt * 128, &full_bar[s]);
             tma_load_2d(sB + kBBytes / 2, &p.tma_b1, ks * kStepK, nt * 128, &full_bar[s]);
           } else {
-            tma_load_2d(sB, &p.tma_b0, ks * kStepK, nt * kTileN, &full_bar[s]);
+            tma_load_2d(sB, &p.tma_b0, ks * kStepK, nt * kTN, &full_bar[s]);
           }
         }
         __syncwarp();
@@ -142,14 +150,14 @@ __global__ void __launch_bounds__(kThreads, 1) bf16_gemm_kernel(const __grid_con
     // ------------------------------------------------------------ MMA issuer
     // Whole warp in the loop, one elected lane issues; stage-0 descriptors are
     // built once and advanced by constant offsets (16-byte units).
-    const uint32_t idesc = idesc_bf16(kTileM, kTileN);
+    const uint32_t idesc = idesc_bf16(kTileM, kTN);
     const uint32_t s0 = smem_u32(smem);
     const uint64_t dA0 = sdesc_k_sw128(s0), dB0 = sdesc_k_sw128(s0 + kABytes);
     int it = 0, tc = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++tc) {
-      const int b = tc & 1;
-      const uint32_t use = (uint32_t)(tc >> 1);
+      const int b = LOGITS ? 0 : (tc & 1);
+      const uint32_t use = LOGITS ? (uint32_t)tc : (uint32_t)(tc >> 1);
       // the epilogue must have drained this accumulator buffer's previous tile
       if (__any_sync(0xffffffffu, !mbar_wait(&acc_empty[b], (use & 1u) ^ 1u))) {
         ok = false;
@@ -167,9 +175,18 @@ __global__ void __launch_bounds__(kThreads, 1) bf16_gemm_kernel(const __grid_con
         tc_fence_after();
         const uint64_t so = (uint64_t)((s * kStageBytes) >> 4);
         if (elect_one()) {
+          if (LOGITS) {
+            const int ai = ks < 2 * seg + q4 ? 0 : min(3, (ks - 2 * seg) / q4);
+            const int first = ai == 0 ? 0 : 2 * seg + ai * q4;   // first k-step into this accumulator
 #pragma unroll
-          for (int kb = 0; kb < 4; ++kb)   // K = 16 per MMA: 32 bytes of each row
-            mma_bf16(acc, dA0 + so + 2 * kb, dB0 + so + 2 * kb, idesc, (ks > 0 || kb > 0) ? 1u : 0u);
+            for (int kb = 0; kb < 4; ++kb)
+              mma_bf16(acc + 128u * ai, dA0 + so + 2 * kb, dB0 + so + 2 * kb, idesc,
+                       (ks > first || kb > 0) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb)   // K = 16 per MMA: 32 bytes of each row
+              mma_bf16(acc, dA0 + so + 2 * kb, dB0 + so + 2 * kb, idesc, (ks > 0 || kb > 0) ? 1u : 0u);
+          }
           mma_commit(&empty_bar[s]);          // the stage is free once these MMAs have read it
         }
         __syncwarp();
@@ -191,8 +208,8 @@ __global__ void __launch_bounds__(kThreads, 1) bf16_gemm_kernel(const __grid_con
     const int ch = (warp - kFirstEpiWarp) >> 2;     // column half
     int tc = 0;
     for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++tc) {
-      const int b = tc & 1;
-      const uint32_t use = (uint32_t)(tc >> 1);
+      const int b = LOGITS ? 0 : (tc & 1);
+      const uint32_t use = LOGITS ? (uint32_t)tc : (uint32_t)(tc >> 1);
       const int nt = tile / n_mtiles, mt = tile - nt * n_mtiles;
       const int row = mt * kTileM + q * 32 + lane;   // A row = TMEM lane of this thread
       const bool valid = row < p.M;
@@ -227,6 +244,33 @@ __global__ void __launch_bounds__(kThreads, 1) bf16_gemm_kernel(const __grid_con
             dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
+      } else if (LOGITS) {
+        // this warp's 64 columns, 32 at a time: the four accumulators summed in fp32
+#pragma unroll 1
+        for (int sub = 0; sub < 2; ++sub) {
+          const int cl = 64 * ch + 32 * sub;         // column within the tile
+          uint32_t a[4][32];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) tmem_ld32(tq + 128 * i + cl, a[i]);
+          tmem_ld_wait();
+          if (valid) {
+            float* dst = p.out_f32 + (size_t)row * p.out_cols + nt * kTN + cl;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              float o[4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const int x = 4 * c + j;
+                o[j] = ((__uint_as_float(a[0][x]) + __uint_as_float(a[1][x])) + __uint_as_float(a[2][x])) +
+                       __uint_as_float(a[3][x]);
+              }
+              if (nt * kTN + cl + 4 * c < p.out_cols) *reinterpret_cast<float4*>(dst + 4 * c) = make_float4(o[0], o[1], o[2], o[3]);
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[b]);
       } else {
         uint32_t v[128];
 #pragma unroll
@@ -235,18 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1) bf16_gemm_kernel(const __grid_con
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[b]);
-        if (LOGITS) {
-          if (valid) {
-            float* dst = p.out_f32 + (size_t)row * p.out_cols;
-            const int c0 = nt * kTileN + 128 * ch;
-#pragma unroll
-            for (int c = 0; c < 32; ++c)
-              if (c0 + 4 * c < p.out_cols)
-                *reinterpret_cast<float4*>(dst + c0 + 4 * c) =
-                    make_float4(__uint_as_float(v[4 * c]), __uint_as_float(v[4 * c + 1]), __uint_as_float(v[4 * c + 2]),
-                                __uint_as_float(v[4 * c + 3]));
-          }
-        } else if (valid) {
+        if (valid) {
           uint4* dst = reinterpret_cast<uint4*>(p.out + (size_t)row * p.out_cols + nt * kTileN + 128 * ch);
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
@@ -313,7 +346,8 @@ cudaError_t launch_router_logits_tc(const uint16_t* x, int T, int H, int E, cons
   GemmParams p;
   memset(&p, 0, sizeof p);
   if (!bf16_map(&p.tma_a, x, H, T, kTileM)) return cudaErrorInvalidValue;
-  if (!bf16_map(&p.tma_b0, w3, 3 * H, E, kTileN)) return cudaErrorInvalidValue;
+  if (H % 256) return cudaErrorInvalidValue;   // four hi quarters of whole 64-element k-steps
+  if (!bf16_map(&p.tma_b0, w3, 3 * H, E, 128)) return cudaErrorInvalidValue;
   p.out_f32 = logits;
   p.status = status;
   p.M = T;

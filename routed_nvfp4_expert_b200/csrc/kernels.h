@@ -78,11 +78,13 @@ cudaError_t launch_bf16_gemm(bool gate_up, const uint16_t* a, int M, int K, cons
                              int N, float limit, uint16_t* out, uint32_t* status, cudaStream_t st);
 
 // Router logits on the tensor cores: logits [T, E] fp32 = x [T, H] . w^T with
-// w given exactly as w3 [E, 3H] bf16 = (hi | mid | lo) per row. E % 4 == 0.
+// w given exactly as w3 [E, 3H] bf16 = (lo | mid | hi) per row. E % 4 == 0,
+// H % 256 == 0.
 cudaError_t launch_router_logits_tc(const uint16_t* x, int T, int H, int E, const uint16_t* w3, float* logits,
                                     uint32_t* status, cudaStream_t st);
-// w3 [E, 3H] bf16 from the fp32 router weight [E, H]: hi = w with the low 16
-// bits cleared, mid likewise from w - hi, lo = w - hi - mid (all exact).
+// w3 [E, 3H] bf16 (lo | mid | hi) from the fp32 router weight [E, H]: hi = w
+// with the low 16 bits cleared, mid likewise from w - hi, lo = w - hi - mid
+// (all exact).
 cudaError_t launch_router_split(const float* w, int E, int H, uint16_t* w3, cudaStream_t st);
 
 // Dense BF16 FFN, picking the GEMV form for small T and the tcgen05 GEMM for

@@ -298,10 +298,10 @@ __global__ void __launch_bounds__(256) router_split_kernel(const float* __restri
     const float r1 = v - hi;
     const float mid = __uint_as_float(__float_as_uint(r1) & 0xFFFF0000u);
     const float lo = r1 - mid;
-    uint16_t* row = w3 + e * 3 * H;
-    row[c] = (uint16_t)(__float_as_uint(hi) >> 16);
+    uint16_t* row = w3 + e * 3 * H;                  // order lo | mid | hi along K
+    row[c] = (uint16_t)(__float_as_uint(lo) >> 16);
     row[H + c] = (uint16_t)(__float_as_uint(mid) >> 16);
-    row[2 * H + c] = (uint16_t)(__float_as_uint(lo) >> 16);
+    row[2 * H + c] = (uint16_t)(__float_as_uint(hi) >> 16);
   }
 }
 

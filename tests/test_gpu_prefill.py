@@ -95,7 +95,8 @@ def test_prepare_weights_bit_exact():
     w3 = prep[r3:r3 + wl.E * 3 * wl.H * 2].view(np.uint16).reshape(wl.E, 3, wl.H)
     parts = OF.bf16_value(w3)
     assert np.array_equal(parts[:, 0] + parts[:, 1] + parts[:, 2], inp["router_w"].astype(np.float64))
-    assert np.all(np.abs(parts[:, 1]) <= np.abs(parts[:, 0]) * 2.0 ** -7)
+    assert np.all(np.abs(parts[:, 1]) <= np.abs(parts[:, 2]) * 2.0 ** -7)     # order lo | mid | hi
+    assert np.all(np.abs(parts[:, 0]) <= np.abs(parts[:, 1]) * 2.0 ** -7)
 
 
 @pytest.mark.parametrize("T,E,k,local", [(4, 16, 4, (0, 16)), (1000, 16, 4, (0, 16)), (300, 32, 4, (8, 20)),
