@@ -34,8 +34,11 @@
  *  - All tensor pointers are DEVICE pointers unless a comment says otherwise,
  *    16-byte aligned. The caller owns every buffer; the library allocates and
  *    frees no device memory and keeps no state besides a thread-local error
- *    message and the thread-local stage-timing events of
- *    moe_set_stage_events().
+ *    message, the thread-local stage-timing events of moe_set_stage_events()
+ *    and, per host thread and device, the auxiliary stream and event pair on
+ *    which the decode forward runs the shared expert concurrently (created by
+ *    the first decode moe_forward on that thread and device: make it before
+ *    any stream capture).
  *  - bf16 tensors are passed as uint16_t bit patterns.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream). Every call is
  *    stream-ordered and asynchronous; nothing synchronises except

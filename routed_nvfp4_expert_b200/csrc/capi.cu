@@ -14,6 +14,32 @@
 namespace {
 
 thread_local char g_err[512] = "";
+
+// Decode runs the shared expert on an auxiliary stream, concurrently with the
+// router, the routing plan and the routed experts (it only needs x): per host
+// thread and device, one non-blocking stream and a fork / join event pair,
+// created on first use (before any stream capture) and kept for the process.
+struct SideStream {
+  cudaStream_t st = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+constexpr int kMaxDevices = 64;
+thread_local SideStream g_side[kMaxDevices];
+
+cudaError_t side_stream(SideStream** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  SideStream& s = g_side[dev];
+  if (!s.st) {
+    if ((e = cudaStreamCreateWithFlags(&s.st, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming)) != cudaSuccess) return e;
+  }
+  *out = &s;
+  return cudaSuccess;
+}
 thread_local cudaEvent_t g_stage_ev[MOE_STAGE_COUNT + 1];
 thread_local int g_n_stage_ev = 0;
 
@@ -625,6 +651,18 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
   uint32_t* status = (uint32_t*)(b + L.status);
 
   RNX_CUDA(cudaMemsetAsync(status, 0, 4, st), "clear status");
+  // decode: the shared expert forks off to the auxiliary stream right away
+  SideStream* side = nullptr;
+  const bool shared_aside = Is > 0 && path == MOE_PATH_DECODE;
+  if (shared_aside) {
+    RNX_CUDA(side_stream(&side), "auxiliary stream");
+    RNX_CUDA(cudaEventRecord(side->fork, st), "fork event");
+    RNX_CUDA(cudaStreamWaitEvent(side->st, side->fork, 0), "fork wait");
+    RNX_CUDA(rnx::launch_dense_ffn(H, Is, cfg->swiglu_limit, x, T, w->shared_gate, w->shared_up, w->shared_down,
+                                   shared, (uint16_t*)(b + L.shared_h), status, side->st),
+             "shared expert");
+    RNX_CUDA(cudaEventRecord(side->join, side->st), "join event");
+  }
   RNX_CUDA(mark(MOE_STAGE_ROUTER_LOGITS, st), "stage event");
   uint32_t* xmax = (uint32_t*)(b + L.xmax);
   uint32_t* hmax = (uint32_t*)(b + L.hmax);
@@ -678,7 +716,9 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
     RNX_CUDA(rnx::launch_nvfp4_gemv(a, st), "expert down");
   }
   RNX_CUDA(mark(MOE_STAGE_SHARED, st), "stage event");
-  if (Is > 0) {
+  if (shared_aside) {
+    RNX_CUDA(cudaStreamWaitEvent(st, side->join, 0), "join wait");
+  } else if (Is > 0) {
     RNX_CUDA(rnx::launch_dense_ffn(H, Is, cfg->swiglu_limit, x, T, w->shared_gate, w->shared_up, w->shared_down,
                                    shared, (uint16_t*)(b + L.shared_h), status, st),
              "shared expert");

@@ -114,6 +114,17 @@ RNX_DEVICE float clamped_swiglu_fast(float g, float u, float limit) {
   return __fdividef(gc, 1.0f + __expf(-gc)) * uc;
 }
 
+// Programmatic dependent launch. A kernel launched with the programmatic
+// stream-serialization attribute may start before the previous kernel of the
+// stream finished; pdl_wait() blocks until that kernel completed and its
+// writes are visible (a no-op without a programmatic dependency). Every kernel
+// of the chain calls pdl_trigger() only after its own pdl_wait(), so when a
+// kernel starts, the kernel two steps earlier has completed: work before
+// pdl_wait() may read what that one (and anything earlier) wrote, but nothing
+// the immediately preceding kernel writes.
+RNX_DEVICE void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+RNX_DEVICE void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Read-only, no-L1-allocate 128-bit global load for streamed weights.
 RNX_DEVICE uint4 ldg_stream(const void* p) {
   uint4 r;

@@ -13,6 +13,8 @@ namespace {
 // one rounding to bf16. Each thread owns 8 consecutive hidden elements.
 __global__ void __launch_bounds__(256) combine_kernel(int T, int k, int H, const uint16_t* __restrict__ r,
                                                       const uint16_t* __restrict__ shared, uint16_t* __restrict__ y) {
+  pdl_wait();
+  pdl_trigger();
   const int per_row = H >> 3;
   const long long n = (long long)T * per_row;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
@@ -163,7 +165,8 @@ int grid_for(long long n, int threads) {
 
 cudaError_t launch_combine(int T, int k, int H, const uint16_t* r, const uint16_t* shared, uint16_t* y,
                            cudaStream_t st) {
-  combine_kernel<<<grid_for((long long)T * (H / 8), 256), 256, 0, st>>>(T, k, H, r, shared, y);
+  return launch_pdl(combine_kernel, dim3(grid_for((long long)T * (H / 8), 256)), dim3(256), 0, st, T, k, H, r, shared,
+                    y);
   return cudaGetLastError();
 }
 

@@ -356,6 +356,13 @@ nvfp4_gemv_direct_kernel(GemvParams p) {
   const int codes_row = p.K / 2, scales_row = p.K / 16;
   const int bpe = (p.rows + CTA_ROWS - 1) / CTA_ROWS;
   const int u = blockIdx.x / bpe, blk = blockIdx.x - u * bpe;
+  // GATE_UP follows the routing plan's kernel: wait before reading the plan.
+  // DOWN follows GATE_UP: the plan is complete (two kernels back), so the
+  // expert's weight rows stream in before the wait for h.
+  if (GATE_UP) {
+    pdl_wait();
+    pdl_trigger();
+  }
   if (u >= p.active[0]) return;
   // one round trip for the expert and its single assignment, one for the rest
   const int e = p.active[1 + u];
@@ -395,6 +402,11 @@ nvfp4_gemv_direct_kernel(GemvParams p) {
     const size_t gr = (size_t)e * p.rows + row;
     q[r] = on ? ldg_stream(cb + gr * codes_row + 16 * c) : make_uint4(0, 0, 0, 0);
     sv[r] = on ? ldg_u16(sb + gr * scales_row + 2 * c) : (uint16_t)0;
+  }
+
+  if (!GATE_UP) {
+    pdl_wait();
+    pdl_trigger();
   }
 
   // 2. this lane's 32-element activation chunk (x token for GATE_UP, h row
@@ -476,8 +488,7 @@ cudaError_t launch_direct(const GemvParams& p, int max_active, bool has_remote, 
   constexpr int CTA_ROWS = GU ? RG * (kDirectRows / 2) : RG * kDirectRows;
   const int bpe = (p.rows + CTA_ROWS - 1) / CTA_ROWS;
   const int grid = std::max(1, max_active * bpe);
-  nvfp4_gemv_direct_kernel<NI, GU><<<grid, kDirectWarps * kWarp, 0, st>>>(p);
-  cudaError_t err = cudaGetLastError();
+  cudaError_t err = launch_pdl(nvfp4_gemv_direct_kernel<NI, GU>, dim3(grid), dim3(kDirectWarps * kWarp), 0, st, p);
   if (err != cudaSuccess || GU || !has_remote) return err;
   zero_remote_rows<<<kNumSMs, 256, 0, st>>>(p);
   return cudaGetLastError();

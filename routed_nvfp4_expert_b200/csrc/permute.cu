@@ -97,6 +97,8 @@ __global__ void __launch_bounds__(1024) permute_small(const int32_t* __restrict_
   __shared__ int s_cnt[kMaxE];
   __shared__ int s_off[kMaxE];
   __shared__ int s_warp[33];
+  pdl_wait();
+  pdl_trigger();
   for (int e = threadIdx.x; e < E; e += blockDim.x) s_cnt[e] = 0;
   __syncthreads();
   for (int a = threadIdx.x; a < A; a += blockDim.x) {
@@ -242,7 +244,7 @@ size_t permute_scratch_ints(int A, int E) {
 cudaError_t launch_permute(const int32_t* ids, int A, int E, int lb, int le, const moe_plan_t& plan,
                            int32_t* scratch, uint32_t* status, cudaStream_t st) {
   if (A <= kSmallMaxA) {
-    permute_small<<<1, 1024, 0, st>>>(ids, A, E, lb, le, plan, status);
+    return launch_pdl(permute_small, dim3(1), dim3(1024), 0, st, ids, A, E, lb, le, plan, status);
     return cudaGetLastError();
   }
   const int nb = (A + kChunk - 1) / kChunk;

@@ -27,6 +27,16 @@ __global__ void __launch_bounds__(kLogitThreads) router_logits_gemv(const uint16
   const int e = blockIdx.x;
   const int nq = H >> 2;
   __shared__ float red[4][kLogitTokens];
+  // the router weight row does not depend on earlier kernels: load it first
+  const float4* wrow = reinterpret_cast<const float4*>(wr + (size_t)e * H);
+  float4 w[kLogitMaxQ];
+#pragma unroll
+  for (int i = 0; i < kLogitMaxQ; ++i) {
+    const int c = tid + kLogitThreads * i;
+    w[i] = c < nq ? __ldg(wrow + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  pdl_wait();
+  pdl_trigger();
   if (e == 0) {
     // side jobs of CTA 0: max |x_t| per token (fp32 bits; the expert pass
     // pre-scales with it) and clearing the h-max array the gate/up pass fills
@@ -50,13 +60,6 @@ __global__ void __launch_bounds__(kLogitThreads) router_logits_gemv(const uint16
         __syncthreads();
       }
     }
-  }
-  const float4* wrow = reinterpret_cast<const float4*>(wr + (size_t)e * H);
-  float4 w[kLogitMaxQ];
-#pragma unroll
-  for (int i = 0; i < kLogitMaxQ; ++i) {
-    const int c = tid + kLogitThreads * i;
-    w[i] = c < nq ? __ldg(wrow + c) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
   for (int t0 = 0; t0 < T; t0 += kLogitTokens) {
     float acc[kLogitTokens];
@@ -167,6 +170,8 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
   __shared__ float s_key[kTopkTokens][32 * PL];
   __shared__ float s_sig[kTopkTokens][32 * PL];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  pdl_wait();
+  pdl_trigger();
   const int t0 = blockIdx.x * kTopkTokens;
   const int ntok = min(kTopkTokens, T - t0);
   for (int i = threadIdx.x; i < ntok * E; i += blockDim.x) {
@@ -262,7 +267,8 @@ cudaError_t launch_row_absmax(const uint16_t* rows, int R, int K, uint32_t* out,
 cudaError_t launch_router_logits(const uint16_t* x, int T, int H, int E, const float* wr, float* logits,
                                  cudaStream_t st, uint32_t* xmax, uint32_t* zero, int nzero) {
   if (T <= 64 && H <= 4 * kLogitThreads * kLogitMaxQ) {
-    router_logits_gemv<<<E, kLogitThreads, 0, st>>>(x, T, H, E, wr, logits, xmax, zero, nzero);
+    return launch_pdl(router_logits_gemv, dim3(E), dim3(kLogitThreads), 0, st, x, T, H, E, wr, logits, xmax, zero,
+                      nzero);
   } else {
     dim3 grid((E + kSgBN - 1) / kSgBN, (T + kSgBM - 1) / kSgBM);
     router_logits_sgemm<<<grid, 256, 0, st>>>(x, T, H, E, wr, logits);
@@ -274,11 +280,14 @@ cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, in
                         float* weights, cudaStream_t st) {
   auto grid = [T](int tpb) { return (T + tpb - 1) / tpb; };
   if (E <= 32 * 4)
-    topk_kernel<4><<<grid(topk_tokens<4>()), 256, 0, st>>>(logits, bias, T, E, k, rsf, ids, weights);
+    return launch_pdl(topk_kernel<4>, dim3(grid(topk_tokens<4>())), dim3(256), 0, st, logits, bias, T, E, k, rsf, ids,
+                      weights);
   else if (E <= 32 * 10)
-    topk_kernel<10><<<grid(topk_tokens<10>()), 256, 0, st>>>(logits, bias, T, E, k, rsf, ids, weights);
+    return launch_pdl(topk_kernel<10>, dim3(grid(topk_tokens<10>())), dim3(256), 0, st, logits, bias, T, E, k, rsf, ids,
+                      weights);
   else
-    topk_kernel<32><<<grid(topk_tokens<32>()), 256, 0, st>>>(logits, bias, T, E, k, rsf, ids, weights);
+    return launch_pdl(topk_kernel<32>, dim3(grid(topk_tokens<32>())), dim3(256), 0, st, logits, bias, T, E, k, rsf, ids,
+                      weights);
   return cudaGetLastError();
 }
 
