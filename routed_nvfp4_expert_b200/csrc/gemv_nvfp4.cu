@@ -22,10 +22,23 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tma.cuh"
 
 namespace rnx {
 
 namespace {
+
+// Bounded wait (2 s) until *c >= need, acquire at gpu scope.
+RNX_DEVICE bool wait_counter(const int* c, int need) {
+  const unsigned long long t0 = globaltimer_ns();
+  for (;;) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(c) : "memory");
+    if (v >= need) return true;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    __nanosleep(64);
+  }
+}
 
 constexpr int kGemvWarps = 8;
 constexpr int kGemvThreads = kGemvWarps * kWarp;
@@ -53,6 +66,7 @@ struct GemvParams {
   uint16_t* out;              // GATE_UP: h [A, rows]; DOWN: r [A, rows]
   const uint32_t* act_max;    // direct form: max |activation row| (fp32 bits), by act row
   uint32_t* out_max;          // direct GATE_UP: atomicMax of |h| per assignment (nullable)
+  uint32_t* status;           // device status word (bounded waits)
   const uint8_t* pf_codes;    // direct GATE_UP: down bank to prefetch into L2 (nullable)
   const uint8_t* pf_scales;
   long long pf_codes_per_expert, pf_scales_per_expert;
@@ -343,44 +357,27 @@ RNX_DEVICE float warp_reduce_rows(float (&v)[N]) {
 constexpr int kDirectWarps = 8;
 constexpr int kDirectRows = 8;        // weight rows per warp
 
+// One work item of the direct form: CTA_ROWS output rows (row block blk) of
+// expert e for its single assignment a. Shared by the per-projection kernel
+// and the fused gate/up + down kernel. With `ready` non-null (fused DOWN), the
+// weight rows are loaded first and the h row is read only once *ready
+// reaches `need` (the expert's gate/up items are all done); a wait that runs
+// out sets the status word and the item is skipped. Returns false then.
 template <int NI, bool GATE_UP>
-__global__ void __launch_bounds__(kDirectWarps * kWarp, 3)
-nvfp4_gemv_direct_kernel(GemvParams p) {
+RNX_DEVICE bool direct_item(const GemvParams& p, int e, int a, int blk, float* s_part, const int* ready, int need) {
   constexpr int RG = kDirectWarps / NI;                  // row groups per CTA
   constexpr int PAIRS = GATE_UP ? kDirectRows / 2 : 0;   // gate/up pairs per row group
   constexpr int CTA_ROWS = GATE_UP ? RG * PAIRS : RG * kDirectRows;   // output rows per CTA
-  __shared__ float s_part[NI][RG * kDirectRows];
+  __shared__ int s_ok;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kg = warp % NI, rg = warp / NI;
   const int nchunks = p.K / 32;
   const int codes_row = p.K / 2, scales_row = p.K / 16;
-  const int bpe = (p.rows + CTA_ROWS - 1) / CTA_ROWS;
-  const int u = blockIdx.x / bpe, blk = blockIdx.x - u * bpe;
-  // GATE_UP follows the routing plan's kernel: wait before reading the plan.
-  // DOWN follows GATE_UP: the plan is complete (two kernels back), so the
-  // expert's weight rows stream in before the wait for h.
-  if (GATE_UP) {
-    pdl_wait();
-    pdl_trigger();
-  }
-  if (u >= p.active[0]) return;
-  // one round trip for the expert and its single assignment, one for the rest
-  const int e = p.active[1 + u];
-  const int a = p.first[u];
   const int row0 = blk * CTA_ROWS;
   const float ts0 = p.ts0[e], ts1 = GATE_UP ? p.ts1[e] : 0.f;
   const float wt = GATE_UP ? 0.f : p.weights[a];
   const int c = kg * 32 + lane;
   const bool lane_on = c < nchunks;
-  if (GATE_UP && p.pf_codes && threadIdx.x == 0) {
-    // this CTA's share of the same expert's DOWN weights, pulled into L2 while
-    // the gate/up rows stream (the down pass then reads them from L2)
-    const long long pc = p.pf_codes_per_expert, ps = p.pf_scales_per_expert;
-    const long long c0 = (pc * blk / bpe) & ~15ll, c1 = (pc * (blk + 1) / bpe) & ~15ll;
-    const long long s0 = (ps * blk / bpe) & ~15ll, s1 = (ps * (blk + 1) / bpe) & ~15ll;
-    if (c1 > c0) prefetch_l2(p.pf_codes + (size_t)e * pc + c0, (uint32_t)(c1 - c0));
-    if (s1 > s0) prefetch_l2(p.pf_scales + (size_t)e * ps + s0, (uint32_t)(s1 - s0));
-  }
 
   // 1. weight loads: 8 rows per warp (GATE_UP: 4 gate rows then 4 up rows)
   uint4 q[kDirectRows];
@@ -404,14 +401,19 @@ nvfp4_gemv_direct_kernel(GemvParams p) {
     sv[r] = on ? ldg_u16(sb + gr * scales_row + 2 * c) : (uint16_t)0;
   }
 
-  if (!GATE_UP) {
-    pdl_wait();
-    pdl_trigger();
+  if (ready) {
+    if (threadIdx.x == 0) {
+      const bool okw = wait_counter(ready, need);
+      if (!okw) set_status(p.status, kDevErrTimeout);
+      s_ok = okw ? 1 : 0;
+    }
+    __syncthreads();
+    if (!s_ok) return false;
   }
 
   // 2. this lane's 32-element activation chunk (x token for GATE_UP, h row
-  //    for DOWN) straight from global/L2, pre-scaled by the power of two that
-  //    brings the row's max |a| (supplied) into [128, 256)
+  //    for DOWN) pre-scaled by the power of two that brings the row's max |a|
+  //    (supplied) into [128, 256)
   const uint16_t* arow = p.act + (size_t)(GATE_UP ? a / p.k : a) * p.K;
   float up, unscale;
   prescale_from_max(__uint_as_float(p.act_max[GATE_UP ? a / p.k : a]), up, unscale);
@@ -430,7 +432,7 @@ nvfp4_gemv_direct_kernel(GemvParams p) {
   const int r = lane >> 2;
 
   if (GATE_UP) {
-    if ((lane & 3) == 0) s_part[kg][rg * kDirectRows + r] = tot;
+    if ((lane & 3) == 0) s_part[kg * RG * kDirectRows + rg * kDirectRows + r] = tot;
     __syncthreads();
     if (threadIdx.x < RG * PAIRS) {
       const int gq = threadIdx.x / PAIRS, pr = threadIdx.x % PAIRS;
@@ -439,8 +441,8 @@ nvfp4_gemv_direct_kernel(GemvParams p) {
         float g = 0.f, uu = 0.f;
 #pragma unroll
         for (int k = 0; k < NI; ++k) {
-          g += s_part[k][gq * kDirectRows + pr];
-          uu += s_part[k][gq * kDirectRows + PAIRS + pr];
+          g += s_part[k * RG * kDirectRows + gq * kDirectRows + pr];
+          uu += s_part[k * RG * kDirectRows + gq * kDirectRows + PAIRS + pr];
         }
         g *= unscale * ts0;
         uu *= unscale * ts1;
@@ -454,16 +456,75 @@ nvfp4_gemv_direct_kernel(GemvParams p) {
     if ((lane & 3) == 0 && row < p.rows)
       p.out[(size_t)a * p.rows + row] = f32_to_bf16_bits(tot * unscale * ts0 * wt);
   } else {
-    if ((lane & 3) == 0) s_part[kg][rg * kDirectRows + r] = tot;
+    if ((lane & 3) == 0) s_part[kg * RG * kDirectRows + rg * kDirectRows + r] = tot;
     __syncthreads();
     if (threadIdx.x < RG * kDirectRows) {
       const int row = row0 + threadIdx.x;
       if (row < p.rows) {
         float o = 0.f;
 #pragma unroll
-        for (int k = 0; k < NI; ++k) o += s_part[k][threadIdx.x];
+        for (int k = 0; k < NI; ++k) o += s_part[k * RG * kDirectRows + threadIdx.x];
         p.out[(size_t)a * p.rows + row] = f32_to_bf16_bits(o * unscale * ts0 * wt);
       }
+    }
+  }
+  return true;
+}
+
+template <int NI, bool GATE_UP>
+__host__ __device__ constexpr int direct_cta_rows() {
+  return GATE_UP ? (kDirectWarps / NI) * (kDirectRows / 2) : (kDirectWarps / NI) * kDirectRows;
+}
+
+template <int NI, bool GATE_UP>
+__global__ void __launch_bounds__(kDirectWarps * kWarp, 3)
+nvfp4_gemv_direct_kernel(GemvParams p) {
+  __shared__ float s_part[kDirectWarps * kDirectRows];
+  const int bpe = (p.rows + direct_cta_rows<NI, GATE_UP>() - 1) / direct_cta_rows<NI, GATE_UP>();
+  const int u = blockIdx.x / bpe, blk = blockIdx.x - u * bpe;
+  pdl_wait();       // follows the routing plan (GATE_UP) or the h producer (DOWN)
+  pdl_trigger();
+  if (u >= p.active[0]) return;
+  direct_item<NI, GATE_UP>(p, p.active[1 + u], p.first[u], blk, s_part, nullptr, 0);
+}
+
+// Gate/up and down of every active expert in one persistent kernel (one
+// token per expert). Work items are claimed in order from a counter: first
+// the gate/up blocks of every expert, then the down blocks. A down item
+// streams its weight rows, then waits until all gate/up items of its expert
+// have published h (a per-expert counter, release / acquire at gpu scope).
+// Because every gate/up item has a lower number than every down item and
+// gate/up items never wait, each awaited item is already held by a running
+// CTA: the waits end whatever else occupies the GPU. counters: [0] = next
+// item, [1 + u] = finished gate/up items of active expert u; zeroed upstream.
+template <int NIG, int NID>
+__global__ void __launch_bounds__(kDirectWarps * kWarp, 3)
+nvfp4_experts_fused_kernel(GemvParams gu, GemvParams dn, int* counters) {
+  __shared__ float s_part[kDirectWarps * kDirectRows];
+  __shared__ int s_item;
+  constexpr int CR_G = direct_cta_rows<NIG, true>(), CR_D = direct_cta_rows<NID, false>();
+  pdl_wait();       // follows the routing plan
+  pdl_trigger();
+  const int n_act = gu.active[0];
+  const int bpe_g = (gu.rows + CR_G - 1) / CR_G, bpe_d = (dn.rows + CR_D - 1) / CR_D;
+  const int n_g = n_act * bpe_g, n_all = n_g + n_act * bpe_d;
+  for (;;) {
+    __syncthreads();                       // s_item / s_part reuse
+    if (threadIdx.x == 0) s_item = atomicAdd(counters, 1);
+    __syncthreads();
+    const int item = s_item;
+    if (item >= n_all) break;
+    if (item < n_g) {
+      const int u = item / bpe_g, blk = item - u * bpe_g;
+      direct_item<NIG, true>(gu, gu.active[1 + u], gu.first[u], blk, s_part, nullptr, 0);
+      __syncthreads();                     // this item's h rows and maxima are written
+      if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(counters + 1 + u, 1);
+      }
+    } else {
+      const int j = item - n_g, u = j / bpe_d, blk = j - u * bpe_d;
+      direct_item<NID, false>(dn, dn.active[1 + u], dn.first[u], blk, s_part, counters + 1 + u, bpe_g);
     }
   }
 }
@@ -515,11 +576,30 @@ cudaError_t launch_t(const GemvParams& p, int max_items, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-}  // namespace
+template <int NIG, int NID>
+cudaError_t launch_fused(const GemvParams& gu, const GemvParams& dn, int* counters, int max_active, bool has_remote,
+                         cudaStream_t st) {
+  constexpr int CR_G = direct_cta_rows<NIG, true>(), CR_D = direct_cta_rows<NID, false>();
+  const int items = max_active * ((gu.rows + CR_G - 1) / CR_G + (dn.rows + CR_D - 1) / CR_D);
+  const int grid = std::max(1, std::min(items, kNumSMs * 3));
+  cudaError_t err = launch_pdl(nvfp4_experts_fused_kernel<NIG, NID>, dim3(grid), dim3(kDirectWarps * kWarp), 0, st, gu,
+                               dn, counters);
+  if (err != cudaSuccess || !has_remote) return err;
+  zero_remote_rows<<<kNumSMs, 256, 0, st>>>(dn);
+  return cudaGetLastError();
+}
 
-cudaError_t launch_nvfp4_gemv(const ExpertGemvArgs& a, cudaStream_t st) {
+template <int NIG>
+cudaError_t launch_fused_d(int NID, const GemvParams& gu, const GemvParams& dn, int* counters, int max_active,
+                           bool has_remote, cudaStream_t st) {
+  if (NID == 1) return launch_fused<NIG, 1>(gu, dn, counters, max_active, has_remote, st);
+  if (NID == 2) return launch_fused<NIG, 2>(gu, dn, counters, max_active, has_remote, st);
+  if (NID <= 4) return launch_fused<NIG, 4>(gu, dn, counters, max_active, has_remote, st);
+  return launch_fused<NIG, 8>(gu, dn, counters, max_active, has_remote, st);
+}
+
+GemvParams gemv_params(const ExpertGemvArgs& a, bool gu) {
   GemvParams p{};
-  const bool gu = a.proj == MOE_PROJ_GATE_UP;
   p.K = gu ? a.H : a.I;
   p.rows = gu ? a.I : a.H;
   p.k = a.k;
@@ -544,12 +624,37 @@ cudaError_t launch_nvfp4_gemv(const ExpertGemvArgs& a, cudaStream_t st) {
   p.out = a.out;
   p.act_max = a.act_max;
   p.out_max = a.out_max;
+  p.status = a.status;
   if (gu && a.prefetch_down && a.down.codes) {
     p.pf_codes = a.down.codes;
     p.pf_scales = a.down.scales;
     p.pf_codes_per_expert = (long long)a.H * a.I / 2;
     p.pf_scales_per_expert = (long long)a.H * a.I / 16;
   }
+  return p;
+}
+
+}  // namespace
+
+cudaError_t launch_decode_experts(const ExpertGemvArgs& a, uint16_t* h, uint16_t* r, uint32_t* hmax, int* counters,
+                                  cudaStream_t st) {
+  if (a.T != 1 || !a.act_max || !hmax || a.H > 8192 || a.I > 8192) return cudaErrorNotSupported;
+  ExpertGemvArgs g = a, d = a;
+  g.proj = MOE_PROJ_GATE_UP; g.act = a.act; g.out = h; g.out_max = hmax;
+  d.proj = MOE_PROJ_DOWN; d.act = h; d.out = r; d.act_max = hmax; d.out_max = nullptr;
+  const GemvParams pg = gemv_params(g, true), pd = gemv_params(d, false);
+  const int max_active = std::min(a.local_end - a.local_begin, a.T * a.k);
+  const bool remote = a.local_begin > 0 || a.local_end < a.E;
+  const int NIG = (a.H / 32 + 31) / 32, NID = (a.I / 32 + 31) / 32;
+  if (NIG == 1) return launch_fused_d<1>(NID, pg, pd, counters, max_active, remote, st);
+  if (NIG == 2) return launch_fused_d<2>(NID, pg, pd, counters, max_active, remote, st);
+  if (NIG <= 4) return launch_fused_d<4>(NID, pg, pd, counters, max_active, remote, st);
+  return launch_fused_d<8>(NID, pg, pd, counters, max_active, remote, st);
+}
+
+cudaError_t launch_nvfp4_gemv(const ExpertGemvArgs& a, cudaStream_t st) {
+  const bool gu = a.proj == MOE_PROJ_GATE_UP;
+  const GemvParams p = gemv_params(a, gu);
   const int max_active = std::min(a.local_end - a.local_begin, p.A);
   const int max_tok = a.T;   // tokens per expert never exceed T (ids in a row are distinct)
   const int NI = (p.K / 32 + 31) / 32;

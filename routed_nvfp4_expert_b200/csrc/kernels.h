@@ -49,6 +49,13 @@ struct ExpertGemvArgs {
 
 cudaError_t launch_nvfp4_gemv(const ExpertGemvArgs& a, cudaStream_t st);
 
+// One token per expert (T = 1): gate/up and down of every active expert in one
+// persistent kernel. h [k, I] and hmax [k] (zeroed) receive the gate/up
+// output, r [k, H] the down output; counters: 1 + k ints, zeroed upstream.
+// Returns cudaErrorNotSupported when the shape is outside this form.
+cudaError_t launch_decode_experts(const ExpertGemvArgs& a, uint16_t* h, uint16_t* r, uint32_t* hmax, int* counters,
+                                  cudaStream_t st);
+
 // router
 // xmax (nullable): receives max |x_t| per token as fp32 bits; zero (nullable):
 // nzero uint32 words set to 0 (the h-max array of the next expert pass).
