@@ -358,30 +358,33 @@ constexpr int kDirectWarps = 8;
 constexpr int kDirectRows = 8;        // weight rows per warp
 
 // One work item of the direct form: CTA_ROWS output rows (row block blk) of
-// expert e for its single assignment a. Shared by the per-projection kernel
-// and the fused gate/up + down kernel. With `ready` non-null (fused DOWN), the
-// weight rows are loaded first and the h row is read only once *ready
-// reaches `need` (the expert's gate/up items are all done); a wait that runs
-// out sets the status word and the item is skipped. Returns false then.
-template <int NI, bool GATE_UP>
-RNX_DEVICE bool direct_item(const GemvParams& p, int e, int a, int blk, float* s_part, const int* ready, int need) {
-  constexpr int RG = kDirectWarps / NI;                  // row groups per CTA
-  constexpr int PAIRS = GATE_UP ? kDirectRows / 2 : 0;   // gate/up pairs per row group
-  constexpr int CTA_ROWS = GATE_UP ? RG * PAIRS : RG * kDirectRows;   // output rows per CTA
-  __shared__ int s_ok;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kg = warp % NI, rg = warp / NI;
-  const int nchunks = p.K / 32;
-  const int codes_row = p.K / 2, scales_row = p.K / 16;
-  const int row0 = blk * CTA_ROWS;
-  const float ts0 = p.ts0[e], ts1 = GATE_UP ? p.ts1[e] : 0.f;
-  const float wt = GATE_UP ? 0.f : p.weights[a];
-  const int c = kg * 32 + lane;
-  const bool lane_on = c < nchunks;
-
-  // 1. weight loads: 8 rows per warp (GATE_UP: 4 gate rows then 4 up rows)
+// expert e for its single assignment a. An item runs in two phases so that a
+// persistent CTA can issue the next item's weight loads before it finishes
+// the current one: item_loads() issues the 128-bit weight loads (8 rows per
+// warp: GATE_UP 4 gate then 4 up rows) into a register set, item_finish()
+// fetches the activation chunk, multiplies, reduces and stores. With `ready`
+// non-null (fused DOWN), item_finish first waits until *ready reaches `need`
+// (the expert's gate/up items are all done); a wait that runs out sets the
+// status word and the item is skipped.
+struct ItemLoads {
   uint4 q[kDirectRows];
   uint16_t sv[kDirectRows];
+};
+
+template <int NI, bool GATE_UP>
+__host__ __device__ constexpr int direct_cta_rows() {
+  return GATE_UP ? (kDirectWarps / NI) * (kDirectRows / 2) : (kDirectWarps / NI) * kDirectRows;
+}
+
+template <int NI, bool GATE_UP>
+RNX_DEVICE void item_loads(const GemvParams& p, int e, int blk, ItemLoads& L) {
+  constexpr int RG = kDirectWarps / NI;
+  constexpr int PAIRS = GATE_UP ? kDirectRows / 2 : 0;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kg = warp % NI, rg = warp / NI;
+  const int c = kg * 32 + lane;
+  const bool lane_on = c < p.K / 32;
+  const int row0 = blk * direct_cta_rows<NI, GATE_UP>();
 #pragma unroll
   for (int r = 0; r < kDirectRows; ++r) {
     int row;
@@ -397,9 +400,24 @@ RNX_DEVICE bool direct_item(const GemvParams& p, int e, int a, int blk, float* s
     }
     const bool on = lane_on && row < p.rows;
     const size_t gr = (size_t)e * p.rows + row;
-    q[r] = on ? ldg_stream(cb + gr * codes_row + 16 * c) : make_uint4(0, 0, 0, 0);
-    sv[r] = on ? ldg_u16(sb + gr * scales_row + 2 * c) : (uint16_t)0;
+    L.q[r] = on ? ldg_stream(cb + gr * (p.K / 2) + 16 * c) : make_uint4(0, 0, 0, 0);
+    L.sv[r] = on ? ldg_u16(sb + gr * (p.K / 16) + 2 * c) : (uint16_t)0;
   }
+}
+
+template <int NI, bool GATE_UP>
+RNX_DEVICE bool item_finish(const GemvParams& p, int e, int a, int blk, const ItemLoads& L, float* s_part,
+                            const int* ready, int need) {
+  constexpr int RG = kDirectWarps / NI;                  // row groups per CTA
+  constexpr int PAIRS = GATE_UP ? kDirectRows / 2 : 0;   // gate/up pairs per row group
+  __shared__ int s_ok;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kg = warp % NI, rg = warp / NI;
+  const int row0 = blk * direct_cta_rows<NI, GATE_UP>();
+  const int c = kg * 32 + lane;
+  const bool lane_on = c < p.K / 32;
+  const float ts0 = p.ts0[e], ts1 = GATE_UP ? p.ts1[e] : 0.f;
+  const float wt = GATE_UP ? 0.f : p.weights[a];
 
   if (ready) {
     if (threadIdx.x == 0) {
@@ -411,9 +429,9 @@ RNX_DEVICE bool direct_item(const GemvParams& p, int e, int a, int blk, float* s
     if (!s_ok) return false;
   }
 
-  // 2. this lane's 32-element activation chunk (x token for GATE_UP, h row
-  //    for DOWN) pre-scaled by the power of two that brings the row's max |a|
-  //    (supplied) into [128, 256)
+  // this lane's 32-element activation chunk (x token for GATE_UP, h row for
+  // DOWN) pre-scaled by the power of two that brings the row's max |a|
+  // (supplied) into [128, 256)
   const uint16_t* arow = p.act + (size_t)(GATE_UP ? a / p.k : a) * p.K;
   float up, unscale;
   prescale_from_max(__uint_as_float(p.act_max[GATE_UP ? a / p.k : a]), up, unscale);
@@ -425,8 +443,8 @@ RNX_DEVICE bool direct_item(const GemvParams& p, int e, int a, int blk, float* s
   for (int r = 0; r < kDirectRows; ++r) {
     acc[r] = 0.f;
     uint32_t w[16];
-    decode_chunk(q[r], w);
-    chunk_fma(w, xr, e4m3x2_to_f32x2(sv[r]), acc[r]);
+    decode_chunk(L.q[r], w);
+    chunk_fma(w, xr, e4m3x2_to_f32x2(L.sv[r]), acc[r]);
   }
   const float tot = warp_reduce_rows<kDirectRows>(acc);   // lane 4r holds row slot r
   const int r = lane >> 2;
@@ -472,11 +490,6 @@ RNX_DEVICE bool direct_item(const GemvParams& p, int e, int a, int blk, float* s
 }
 
 template <int NI, bool GATE_UP>
-__host__ __device__ constexpr int direct_cta_rows() {
-  return GATE_UP ? (kDirectWarps / NI) * (kDirectRows / 2) : (kDirectWarps / NI) * kDirectRows;
-}
-
-template <int NI, bool GATE_UP>
 __global__ void __launch_bounds__(kDirectWarps * kWarp, 3)
 nvfp4_gemv_direct_kernel(GemvParams p) {
   __shared__ float s_part[kDirectWarps * kDirectRows];
@@ -485,20 +498,26 @@ nvfp4_gemv_direct_kernel(GemvParams p) {
   pdl_wait();       // follows the routing plan (GATE_UP) or the h producer (DOWN)
   pdl_trigger();
   if (u >= p.active[0]) return;
-  direct_item<NI, GATE_UP>(p, p.active[1 + u], p.first[u], blk, s_part, nullptr, 0);
+  const int e = p.active[1 + u];
+  ItemLoads L;
+  item_loads<NI, GATE_UP>(p, e, blk, L);
+  item_finish<NI, GATE_UP>(p, e, p.first[u], blk, L, s_part, nullptr, 0);
 }
 
 // Gate/up and down of every active expert in one persistent kernel (one
 // token per expert). Work items are claimed in order from a counter: first
-// the gate/up blocks of every expert, then the down blocks. A down item
-// streams its weight rows, then waits until all gate/up items of its expert
-// have published h (a per-expert counter, release / acquire at gpu scope).
-// Because every gate/up item has a lower number than every down item and
-// gate/up items never wait, each awaited item is already held by a running
-// CTA: the waits end whatever else occupies the GPU. counters: [0] = next
-// item, [1 + u] = finished gate/up items of active expert u; zeroed upstream.
+// the gate/up blocks of every expert, then the down blocks. Each CTA claims
+// and issues the weight loads of its next item before it finishes the
+// current one (two register sets in flight). A down item waits, after its
+// weight loads, until all gate/up items of its expert have published h (a
+// per-expert counter, release / acquire at gpu scope). Every gate/up item has
+// a lower number than every down item, gate/up items never wait, and a CTA
+// finishes its items in claim order: each awaited item is held by a running
+// CTA that will finish it, whatever else occupies the GPU. counters: [0] =
+// next item, [1 + u] = finished gate/up items of active expert u; zeroed
+// upstream.
 template <int NIG, int NID>
-__global__ void __launch_bounds__(kDirectWarps * kWarp, 3)
+__global__ void __launch_bounds__(kDirectWarps * kWarp, 2)
 nvfp4_experts_fused_kernel(GemvParams gu, GemvParams dn, int* counters) {
   __shared__ float s_part[kDirectWarps * kDirectRows];
   __shared__ int s_item;
@@ -508,15 +527,30 @@ nvfp4_experts_fused_kernel(GemvParams gu, GemvParams dn, int* counters) {
   const int n_act = gu.active[0];
   const int bpe_g = (gu.rows + CR_G - 1) / CR_G, bpe_d = (dn.rows + CR_D - 1) / CR_D;
   const int n_g = n_act * bpe_g, n_all = n_g + n_act * bpe_d;
-  for (;;) {
-    __syncthreads();                       // s_item / s_part reuse
+  auto claim = [&]() {
+    __syncthreads();                       // previous s_item read by every thread
     if (threadIdx.x == 0) s_item = atomicAdd(counters, 1);
     __syncthreads();
-    const int item = s_item;
-    if (item >= n_all) break;
+    return s_item;
+  };
+  auto issue = [&](int item, ItemLoads& L) {
+    if (item < n_g) {
+      const int u = item / bpe_g;
+      item_loads<NIG, true>(gu, gu.active[1 + u], item - u * bpe_g, L);
+    } else if (item < n_all) {
+      const int j = item - n_g, u = j / bpe_d;
+      item_loads<NID, false>(dn, dn.active[1 + u], j - u * bpe_d, L);
+    }
+  };
+  ItemLoads cur, nxt;
+  int item = claim();
+  issue(item, cur);
+  while (item < n_all) {
+    const int next = claim();
+    issue(next, nxt);                      // in flight while this item finishes
     if (item < n_g) {
       const int u = item / bpe_g, blk = item - u * bpe_g;
-      direct_item<NIG, true>(gu, gu.active[1 + u], gu.first[u], blk, s_part, nullptr, 0);
+      item_finish<NIG, true>(gu, gu.active[1 + u], gu.first[u], blk, cur, s_part, nullptr, 0);
       __syncthreads();                     // this item's h rows and maxima are written
       if (threadIdx.x == 0) {
         __threadfence();
@@ -524,8 +558,10 @@ nvfp4_experts_fused_kernel(GemvParams gu, GemvParams dn, int* counters) {
       }
     } else {
       const int j = item - n_g, u = j / bpe_d, blk = j - u * bpe_d;
-      direct_item<NID, false>(dn, dn.active[1 + u], dn.first[u], blk, s_part, counters + 1 + u, bpe_g);
+      item_finish<NID, false>(dn, dn.active[1 + u], dn.first[u], blk, cur, s_part, counters + 1 + u, bpe_g);
     }
+    item = next;
+    cur = nxt;
   }
 }
 
@@ -581,7 +617,7 @@ cudaError_t launch_fused(const GemvParams& gu, const GemvParams& dn, int* counte
                          cudaStream_t st) {
   constexpr int CR_G = direct_cta_rows<NIG, true>(), CR_D = direct_cta_rows<NID, false>();
   const int items = max_active * ((gu.rows + CR_G - 1) / CR_G + (dn.rows + CR_D - 1) / CR_D);
-  const int grid = std::max(1, std::min(items, kNumSMs * 3));
+  const int grid = std::max(1, std::min(items, kNumSMs * 2));
   cudaError_t err = launch_pdl(nvfp4_experts_fused_kernel<NIG, NID>, dim3(grid), dim3(kDirectWarps * kWarp), 0, st, gu,
                                dn, counters);
   if (err != cudaSuccess || !has_remote) return err;
