@@ -505,63 +505,228 @@ nvfp4_gemv_direct_kernel(GemvParams p) {
 }
 
 // Gate/up and down of every active expert in one persistent kernel (one
-// token per expert). Work items are claimed in order from a counter: first
-// the gate/up blocks of every expert, then the down blocks. Each CTA claims
-// and issues the weight loads of its next item before it finishes the
-// current one (two register sets in flight). A down item waits, after its
-// weight loads, until all gate/up items of its expert have published h (a
-// per-expert counter, release / acquire at gpu scope). Every gate/up item has
-// a lower number than every down item, gate/up items never wait, and a CTA
-// finishes its items in claim order: each awaited item is held by a running
-// CTA that will finish it, whatever else occupies the GPU. counters: [0] =
-// next item, [1 + u] = finished gate/up items of active expert u; zeroed
-// upstream.
-template <int NIG, int NID>
-__global__ void __launch_bounds__(kDirectWarps * kWarp, 2)
-nvfp4_experts_fused_kernel(GemvParams gu, GemvParams dn, int* counters) {
-  __shared__ float s_part[kDirectWarps * kDirectRows];
-  __shared__ int s_item;
-  constexpr int CR_G = direct_cta_rows<NIG, true>(), CR_D = direct_cta_rows<NID, false>();
+// token per expert), streaming the weights through shared memory.
+//
+// Work items, in claim order: the gate/up blocks of every active expert (8
+// output features = 8 gate + 8 up rows each), then the down blocks (64 output
+// rows each); one item is 36 KB of codes and scales at H = 4096, I = 1024.
+// One producer warp claims items from a counter and copies each item's rows
+// with bulk copies (TMA engine) into a 5-stage ring, so ~180 KB per SM are in
+// flight whatever the compute warps do; 8 compute warps decode, multiply and
+// reduce from shared memory, release the stage, and write h (with the
+// per-assignment max |h|) or r. A down item waits until every gate/up item of
+// its expert has published h (per-expert counter, release / acquire at gpu
+// scope). Every gate/up item has a lower number than every down item, gate/up
+// items never wait, and each CTA finishes its items in claim order, so every
+// awaited item is held by a running CTA that will finish it. All waits are
+// bounded; a timeout sets the status word and winds the CTA down.
+// counters: [0] = next item, [1 + u] = finished gate/up items of active
+// expert u; zeroed upstream.
+constexpr int kStreamStages = 5;
+constexpr int kStreamItemBytes = 36864;
+constexpr int kStreamCompute = 8;                        // compute warps
+constexpr int kStreamThreads = (kStreamCompute + 1) * 32;
+constexpr int kGuRowsItem = 8;                           // output features per gate/up item
+constexpr int kDnRowsItem = 64;                          // output rows per down item
+constexpr int kStreamMaxH = 4096;
+
+RNX_DEVICE void compute_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kStreamCompute * 32) : "memory"); }
+
+__global__ void __launch_bounds__(kStreamThreads, 1)
+nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn, int* counters) {
+  extern __shared__ __align__(128) uint8_t s_dyn[];
+  uint8_t* stages = s_dyn;                                               // [S][36 KB]
+  uint4* s_x = reinterpret_cast<uint4*>(s_dyn + kStreamStages * kStreamItemBytes);   // x as f16, [4][H/32] units
+  __shared__ __align__(8) uint64_t full_bar[kStreamStages], empty_bar[kStreamStages];
+  __shared__ int s_item[kStreamStages];
+  __shared__ float s_part[kStreamCompute][kDirectRows];
+  __shared__ int s_ok;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int H = gu.K, I = gu.rows;
+  const int nchG = H / 32, nchD = I / 32;
+  const int gu_row_bytes = H / 2, gu_sc_bytes = H / 16, dn_row_bytes = I / 2, dn_sc_bytes = I / 16;
+
+  if (tid == 0) {
+    for (int i = 0; i < kStreamStages; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], kStreamCompute);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
   pdl_wait();       // follows the routing plan
   pdl_trigger();
   const int n_act = gu.active[0];
-  const int bpe_g = (gu.rows + CR_G - 1) / CR_G, bpe_d = (dn.rows + CR_D - 1) / CR_D;
+  const int bpe_g = I / kGuRowsItem, bpe_d = H / kDnRowsItem;
   const int n_g = n_act * bpe_g, n_all = n_g + n_act * bpe_d;
-  auto claim = [&]() {
-    __syncthreads();                       // previous s_item read by every thread
-    if (threadIdx.x == 0) s_item = atomicAdd(counters, 1);
-    __syncthreads();
-    return s_item;
-  };
-  auto issue = [&](int item, ItemLoads& L) {
-    if (item < n_g) {
-      const int u = item / bpe_g;
-      item_loads<NIG, true>(gu, gu.active[1 + u], item - u * bpe_g, L);
-    } else if (item < n_all) {
-      const int j = item - n_g, u = j / bpe_d;
-      item_loads<NID, false>(dn, dn.active[1 + u], j - u * bpe_d, L);
+
+  if (warp == kStreamCompute) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_first();
+      int it = 0;
+      for (;; ++it) {
+        const int s = it % kStreamStages;
+        const uint32_t ph = (uint32_t)(it / kStreamStages) & 1u;
+        const bool free_ok = mbar_wait(&empty_bar[s], ph ^ 1u);
+        const int item = free_ok ? atomicAdd(counters, 1) : -1;
+        if (!free_ok) set_status(gu.status, kDevErrTimeout);
+        if (item < 0 || item >= n_all) {
+          s_item[s] = -1;                  // end of work (or abort) for the compute warps
+          mbar_arrive(&full_bar[s]);
+          break;
+        }
+        s_item[s] = item;
+        uint8_t* st = stages + (size_t)s * kStreamItemBytes;
+        if (item < n_g) {
+          const int u = item / bpe_g, row0 = (item - u * bpe_g) * kGuRowsItem;
+          const size_t gr = (size_t)gu.active[1 + u] * I + row0;
+          const uint32_t cb = kGuRowsItem * gu_row_bytes, sb = kGuRowsItem * gu_sc_bytes;
+          mbar_arrive_expect_tx(&full_bar[s], 2 * (cb + sb));
+          bulk_g2s(st, gu.codes0 + gr * gu_row_bytes, cb, &full_bar[s], pol);
+          bulk_g2s(st + cb, gu.codes1 + gr * gu_row_bytes, cb, &full_bar[s], pol);
+          bulk_g2s(st + 2 * cb, gu.scales0 + gr * gu_sc_bytes, sb, &full_bar[s], pol);
+          bulk_g2s(st + 2 * cb + sb, gu.scales1 + gr * gu_sc_bytes, sb, &full_bar[s], pol);
+        } else {
+          const int j = item - n_g, u = j / bpe_d, row0 = (j - u * bpe_d) * kDnRowsItem;
+          const size_t gr = (size_t)dn.active[1 + u] * H + row0;
+          const uint32_t cb = kDnRowsItem * dn_row_bytes, sb = kDnRowsItem * dn_sc_bytes;
+          mbar_arrive_expect_tx(&full_bar[s], cb + sb);
+          bulk_g2s(st, dn.codes0 + gr * dn_row_bytes, cb, &full_bar[s], pol);
+          bulk_g2s(st + cb, dn.scales0 + gr * dn_sc_bytes, sb, &full_bar[s], pol);
+        }
+      }
+      // copies in flight must land before the CTA may exit
+      for (int j = max(0, it - kStreamStages + 1); j < it; ++j)
+        if (!mbar_wait(&full_bar[j % kStreamStages], (uint32_t)(j / kStreamStages) & 1u))
+          set_status(gu.status, kDevErrTimeout);
     }
-  };
-  ItemLoads cur, nxt;
-  int item = claim();
-  issue(item, cur);
-  while (item < n_all) {
-    const int next = claim();
-    issue(next, nxt);                      // in flight while this item finishes
+    return;
+  }
+
+  // -------------------------------------------------------------- compute warps
+  // the token's x (one token: every gate/up item uses it), pre-scaled to f16
+  float x_up, x_unscale;
+  prescale_from_max(__uint_as_float(gu.act_max[0]), x_up, x_unscale);
+  for (int cq = tid; cq < nchG * 4; cq += kStreamCompute * 32) {
+    const int c = cq >> 2, q = cq & 3;
+    const uint4 v = *reinterpret_cast<const uint4*>(gu.act + 32 * c + 8 * q);
+    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = bf16x2_to_f32x2(w4[j]);
+      __half2 h2 = __floats2half2_rn(f.x * x_up, f.y * x_up);
+      o[j] = *reinterpret_cast<uint32_t*>(&h2);
+    }
+    s_x[q * nchG + c] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  compute_bar();
+
+  for (int it = 0;; ++it) {
+    const int s = it % kStreamStages;
+    const uint32_t ph = (uint32_t)(it / kStreamStages) & 1u;
+    if (__any_sync(0xffffffffu, !mbar_wait(&full_bar[s], ph))) {
+      if (lane == 0) set_status(gu.status, kDevErrTimeout);
+      break;
+    }
+    const int item = s_item[s];
+    if (item < 0) break;
+    const uint8_t* st = stages + (size_t)s * kStreamItemBytes;
     if (item < n_g) {
-      const int u = item / bpe_g, blk = item - u * bpe_g;
-      item_finish<NIG, true>(gu, gu.active[1 + u], gu.first[u], blk, cur, s_part, nullptr, 0);
-      __syncthreads();                     // this item's h rows and maxima are written
-      if (threadIdx.x == 0) {
+      // gate/up: thread t handles chunk c of rows 8 (t >> 7) .. +7 (gate rows
+      // for t < 128, up rows above); partial sums over the warp, then over
+      // the 4 warps of each half in shared memory
+      const int u = item / bpe_g, row0 = (item - u * bpe_g) * kGuRowsItem;
+      const int e = gu.active[1 + u], a = gu.first[u];
+      const int half = tid >> 7;
+      const uint8_t* cb = st + half * kGuRowsItem * gu_row_bytes;
+      const uint8_t* sb = st + 2 * kGuRowsItem * gu_row_bytes + half * kGuRowsItem * gu_sc_bytes;
+      float acc[kDirectRows];
+#pragma unroll
+      for (int r = 0; r < kDirectRows; ++r) acc[r] = 0.f;
+      for (int c = tid & 127; c < nchG; c += 128) {
+        uint32_t xr[16];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 v = s_x[q * nchG + c];
+          xr[4 * q] = v.x; xr[4 * q + 1] = v.y; xr[4 * q + 2] = v.z; xr[4 * q + 3] = v.w;
+        }
+#pragma unroll
+        for (int r = 0; r < kDirectRows; ++r) {
+          const uint4 qv = *reinterpret_cast<const uint4*>(cb + r * gu_row_bytes + 16 * c);
+          const uint16_t sv = *reinterpret_cast<const uint16_t*>(sb + r * gu_sc_bytes + 2 * c);
+          uint32_t w[16];
+          decode_chunk(qv, w);
+          chunk_fma(w, xr, e4m3x2_to_f32x2(sv), acc[r]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[s]);      // this warp is done with the stage
+      const float tot = warp_reduce_rows<kDirectRows>(acc);
+      if ((lane & 3) == 0) s_part[warp][lane >> 2] = tot;
+      compute_bar();
+      if (tid < kGuRowsItem) {
+        float g = 0.f, uu = 0.f;
+#pragma unroll
+        for (int w4 = 0; w4 < 4; ++w4) {
+          g += s_part[w4][tid];
+          uu += s_part[4 + w4][tid];
+        }
+        g *= x_unscale * gu.ts0[e];
+        uu *= x_unscale * gu.ts1[e];
+        const uint16_t hb = f32_to_bf16_bits(clamped_swiglu(g, uu, gu.limit));
+        gu.out[(size_t)a * I + row0 + tid] = hb;
+        atomicMax(gu.out_max + a, __float_as_uint(fabsf(bf16_bits_to_f32(hb))));
+      }
+      compute_bar();                                  // s_part reuse; this item's h written
+      if (tid == 0) {
         __threadfence();
         atomicAdd(counters + 1 + u, 1);
       }
     } else {
-      const int j = item - n_g, u = j / bpe_d, blk = j - u * bpe_d;
-      item_finish<NID, false>(dn, dn.active[1 + u], dn.first[u], blk, cur, s_part, counters + 1 + u, bpe_g);
+      // down: warp w owns rows 8w .. 8w+7 of the item, lane c chunk c
+      const int j = item - n_g, u = j / bpe_d, row0 = (j - u * bpe_d) * kDnRowsItem;
+      const int e = dn.active[1 + u], a = dn.first[u];
+      if (tid == 0) {
+        const bool okw = wait_counter(counters + 1 + u, bpe_g);
+        if (!okw) set_status(gu.status, kDevErrTimeout);
+        s_ok = okw ? 1 : 0;
+      }
+      compute_bar();
+      if (!s_ok) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_bar[s]);
+        continue;
+      }
+      float up, unscale;
+      prescale_from_max(__uint_as_float(dn.act_max[a]), up, unscale);
+      const uint16_t* arow = dn.act + (size_t)a * I;
+      const uint8_t* cb = st + warp * kDirectRows * dn_row_bytes;
+      const uint8_t* sb = st + kDnRowsItem * dn_row_bytes + warp * kDirectRows * dn_sc_bytes;
+      float acc[kDirectRows];
+#pragma unroll
+      for (int r = 0; r < kDirectRows; ++r) acc[r] = 0.f;
+      for (int c = lane; c < nchD; c += 32) {
+        uint32_t xr[16];
+        load_act_chunk(arow, c, true, up, xr);
+#pragma unroll
+        for (int r = 0; r < kDirectRows; ++r) {
+          const uint4 qv = *reinterpret_cast<const uint4*>(cb + r * dn_row_bytes + 16 * c);
+          const uint16_t sv = *reinterpret_cast<const uint16_t*>(sb + r * dn_sc_bytes + 2 * c);
+          uint32_t w[16];
+          decode_chunk(qv, w);
+          chunk_fma(w, xr, e4m3x2_to_f32x2(sv), acc[r]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[s]);
+      const float tot = warp_reduce_rows<kDirectRows>(acc);
+      if ((lane & 3) == 0) {
+        const int row = row0 + warp * kDirectRows + (lane >> 2);
+        dn.out[(size_t)a * H + row] = f32_to_bf16_bits(tot * unscale * dn.ts0[e] * dn.weights[a]);
+      }
     }
-    item = next;
-    cur = nxt;
   }
 }
 
@@ -612,28 +777,6 @@ cudaError_t launch_t(const GemvParams& p, int max_items, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <int NIG, int NID>
-cudaError_t launch_fused(const GemvParams& gu, const GemvParams& dn, int* counters, int max_active, bool has_remote,
-                         cudaStream_t st) {
-  constexpr int CR_G = direct_cta_rows<NIG, true>(), CR_D = direct_cta_rows<NID, false>();
-  const int items = max_active * ((gu.rows + CR_G - 1) / CR_G + (dn.rows + CR_D - 1) / CR_D);
-  const int grid = std::max(1, std::min(items, kNumSMs * 2));
-  cudaError_t err = launch_pdl(nvfp4_experts_fused_kernel<NIG, NID>, dim3(grid), dim3(kDirectWarps * kWarp), 0, st, gu,
-                               dn, counters);
-  if (err != cudaSuccess || !has_remote) return err;
-  zero_remote_rows<<<kNumSMs, 256, 0, st>>>(dn);
-  return cudaGetLastError();
-}
-
-template <int NIG>
-cudaError_t launch_fused_d(int NID, const GemvParams& gu, const GemvParams& dn, int* counters, int max_active,
-                           bool has_remote, cudaStream_t st) {
-  if (NID == 1) return launch_fused<NIG, 1>(gu, dn, counters, max_active, has_remote, st);
-  if (NID == 2) return launch_fused<NIG, 2>(gu, dn, counters, max_active, has_remote, st);
-  if (NID <= 4) return launch_fused<NIG, 4>(gu, dn, counters, max_active, has_remote, st);
-  return launch_fused<NIG, 8>(gu, dn, counters, max_active, has_remote, st);
-}
-
 GemvParams gemv_params(const ExpertGemvArgs& a, bool gu) {
   GemvParams p{};
   p.K = gu ? a.H : a.I;
@@ -674,18 +817,31 @@ GemvParams gemv_params(const ExpertGemvArgs& a, bool gu) {
 
 cudaError_t launch_decode_experts(const ExpertGemvArgs& a, uint16_t* h, uint16_t* r, uint32_t* hmax, int* counters,
                                   cudaStream_t st) {
-  if (a.T != 1 || !a.act_max || !hmax || a.H > 8192 || a.I > 8192) return cudaErrorNotSupported;
+  // one token; an item's rows (16 x H/2 + 16 x H/16 and 64 x I/2 + 64 x I/16
+  // bytes) fit one 36 KB stage
+  if (a.T != 1 || !a.act_max || !hmax || a.H > kStreamMaxH || 36 * a.I > kStreamItemBytes || a.H % kDnRowsItem ||
+      a.I % kGuRowsItem)
+    return cudaErrorNotSupported;
   ExpertGemvArgs g = a, d = a;
   g.proj = MOE_PROJ_GATE_UP; g.act = a.act; g.out = h; g.out_max = hmax;
   d.proj = MOE_PROJ_DOWN; d.act = h; d.out = r; d.act_max = hmax; d.out_max = nullptr;
   const GemvParams pg = gemv_params(g, true), pd = gemv_params(d, false);
   const int max_active = std::min(a.local_end - a.local_begin, a.T * a.k);
   const bool remote = a.local_begin > 0 || a.local_end < a.E;
-  const int NIG = (a.H / 32 + 31) / 32, NID = (a.I / 32 + 31) / 32;
-  if (NIG == 1) return launch_fused_d<1>(NID, pg, pd, counters, max_active, remote, st);
-  if (NIG == 2) return launch_fused_d<2>(NID, pg, pd, counters, max_active, remote, st);
-  if (NIG <= 4) return launch_fused_d<4>(NID, pg, pd, counters, max_active, remote, st);
-  return launch_fused_d<8>(NID, pg, pd, counters, max_active, remote, st);
+  const size_t smem = (size_t)kStreamStages * kStreamItemBytes + (size_t)a.H * 2;
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaError_t err = cudaFuncSetAttribute(nvfp4_experts_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)((size_t)kStreamStages * kStreamItemBytes + kStreamMaxH * 2));
+    if (err != cudaSuccess) return err;
+    attr_done = true;
+  }
+  const int items = max_active * (a.I / kGuRowsItem + a.H / kDnRowsItem);
+  const int grid = std::max(1, std::min(items, kNumSMs));
+  cudaError_t err = launch_pdl(nvfp4_experts_stream_kernel, dim3(grid), dim3(kStreamThreads), smem, st, pg, pd, counters);
+  if (err != cudaSuccess || !remote) return err;
+  zero_remote_rows<<<kNumSMs, 256, 0, st>>>(pd);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_nvfp4_gemv(const ExpertGemvArgs& a, cudaStream_t st) {
