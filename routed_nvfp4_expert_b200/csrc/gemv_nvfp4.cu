@@ -508,25 +508,27 @@ nvfp4_gemv_direct_kernel(GemvParams p) {
 // token per expert), streaming the weights through shared memory.
 //
 // Work items, in claim order: the gate/up blocks of every active expert (8
-// output features = 8 gate + 8 up rows each), then the down blocks (64 output
-// rows each); one item is 36 KB of codes and scales at H = 4096, I = 1024.
-// One producer warp claims items from a counter and copies each item's rows
+// output features = 8 gate + 8 up rows each, one feature per compute warp),
+// then the down blocks (64 output rows each, 8 per warp); one item is 36 KB
+// of codes and scales at H = 4096, I = 1024. Each warp reduces its rows with
+// shuffles only. One producer warp claims items (4 at a time) from a counter
+// and copies each item's rows
 // with bulk copies (TMA engine) into a 5-stage ring, so ~180 KB per SM are in
 // flight whatever the compute warps do; 8 compute warps decode, multiply and
 // reduce from shared memory, release the stage, and write h (with the
 // per-assignment max |h|) or r. A down item waits until every gate/up item of
 // its expert has published h (per-expert counter, release / acquire at gpu
-// scope). Every gate/up item has a lower number than every down item, gate/up
-// items never wait, and each CTA finishes its items in claim order, so every
-// awaited item is held by a running CTA that will finish it. All waits are
-// bounded; a timeout sets the status word and winds the CTA down.
-// counters: [0] = next item, [1 + u] = finished gate/up items of active
-// expert u; zeroed upstream.
+// scope; every warp of a gate/up item counts once). Every gate/up item has a
+// lower number than every down item, gate/up items never wait, and each CTA
+// finishes its items in claim order, so every awaited item is held by a
+// running CTA that will finish it. All waits are bounded; a timeout sets the
+// status word and winds the CTA down. counters: [0] = next item, [1 + u] =
+// finished gate/up warp-rows of active expert u; zeroed upstream.
 constexpr int kStreamStages = 5;
 constexpr int kStreamItemBytes = 36864;
 constexpr int kStreamCompute = 8;                        // compute warps
 constexpr int kStreamThreads = (kStreamCompute + 1) * 32;
-constexpr int kGuRowsItem = 8;                           // output features per gate/up item
+constexpr int kGuRowsItem = kStreamCompute;             // output features per gate/up item (one per warp)
 constexpr int kDnRowsItem = 64;                          // output rows per down item
 constexpr int kStreamMaxH = 4096;
 
@@ -539,8 +541,6 @@ nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn, int* counters) {
   uint4* s_x = reinterpret_cast<uint4*>(s_dyn + kStreamStages * kStreamItemBytes);   // x as f16, [4][H/32] units
   __shared__ __align__(8) uint64_t full_bar[kStreamStages], empty_bar[kStreamStages];
   __shared__ int s_item[kStreamStages];
-  __shared__ float s_part[kStreamCompute][kDirectRows];
-  __shared__ int s_ok;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = gu.K, I = gu.rows;
   const int nchG = H / 32, nchD = I / 32;
@@ -564,12 +564,21 @@ nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn, int* counters) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
+      // items are claimed kClaim at a time, the next batch requested before
+      // the current one is used up (the atomic's round trip overlaps copies)
+      constexpr int kClaim = 4;
+      int batch = atomicAdd(counters, kClaim), next_batch = atomicAdd(counters, kClaim), in_batch = 0;
       int it = 0;
       for (;; ++it) {
         const int s = it % kStreamStages;
         const uint32_t ph = (uint32_t)(it / kStreamStages) & 1u;
         const bool free_ok = mbar_wait(&empty_bar[s], ph ^ 1u);
-        const int item = free_ok ? atomicAdd(counters, 1) : -1;
+        if (in_batch == kClaim) {
+          batch = next_batch;
+          in_batch = 0;
+          if (batch < n_all) next_batch = atomicAdd(counters, kClaim);
+        }
+        const int item = free_ok ? batch + in_batch++ : -1;
         if (!free_ok) set_status(gu.status, kDevErrTimeout);
         if (item < 0 || item >= n_all) {
           s_item[s] = -1;                  // end of work (or abort) for the compute warps
@@ -634,68 +643,52 @@ nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn, int* counters) {
     if (item < 0) break;
     const uint8_t* st = stages + (size_t)s * kStreamItemBytes;
     if (item < n_g) {
-      // gate/up: thread t handles chunk c of rows 8 (t >> 7) .. +7 (gate rows
-      // for t < 128, up rows above); partial sums over the warp, then over
-      // the 4 warps of each half in shared memory
+      // gate/up: warp w owns feature row0 + w (its gate row and its up row)
+      // over the whole K; lanes take chunks w.r.t. lane, lane + 32, ...
       const int u = item / bpe_g, row0 = (item - u * bpe_g) * kGuRowsItem;
       const int e = gu.active[1 + u], a = gu.first[u];
-      const int half = tid >> 7;
-      const uint8_t* cb = st + half * kGuRowsItem * gu_row_bytes;
-      const uint8_t* sb = st + 2 * kGuRowsItem * gu_row_bytes + half * kGuRowsItem * gu_sc_bytes;
-      float acc[kDirectRows];
-#pragma unroll
-      for (int r = 0; r < kDirectRows; ++r) acc[r] = 0.f;
-      for (int c = tid & 127; c < nchG; c += 128) {
+      const uint8_t* cg = st + warp * gu_row_bytes;
+      const uint8_t* cu = st + (kGuRowsItem + warp) * gu_row_bytes;
+      const uint8_t* sg = st + 2 * kGuRowsItem * gu_row_bytes + warp * gu_sc_bytes;
+      const uint8_t* su = st + 2 * kGuRowsItem * gu_row_bytes + (kGuRowsItem + warp) * gu_sc_bytes;
+      float accg = 0.f, accu = 0.f;
+      for (int c = lane; c < nchG; c += 32) {
         uint32_t xr[16];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const uint4 v = s_x[q * nchG + c];
           xr[4 * q] = v.x; xr[4 * q + 1] = v.y; xr[4 * q + 2] = v.z; xr[4 * q + 3] = v.w;
         }
-#pragma unroll
-        for (int r = 0; r < kDirectRows; ++r) {
-          const uint4 qv = *reinterpret_cast<const uint4*>(cb + r * gu_row_bytes + 16 * c);
-          const uint16_t sv = *reinterpret_cast<const uint16_t*>(sb + r * gu_sc_bytes + 2 * c);
-          uint32_t w[16];
-          decode_chunk(qv, w);
-          chunk_fma(w, xr, e4m3x2_to_f32x2(sv), acc[r]);
-        }
+        uint32_t w[16];
+        decode_chunk(*reinterpret_cast<const uint4*>(cg + 16 * c), w);
+        chunk_fma(w, xr, e4m3x2_to_f32x2(*reinterpret_cast<const uint16_t*>(sg + 2 * c)), accg);
+        decode_chunk(*reinterpret_cast<const uint4*>(cu + 16 * c), w);
+        chunk_fma(w, xr, e4m3x2_to_f32x2(*reinterpret_cast<const uint16_t*>(su + 2 * c)), accu);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty_bar[s]);      // this warp is done with the stage
-      const float tot = warp_reduce_rows<kDirectRows>(acc);
-      if ((lane & 3) == 0) s_part[warp][lane >> 2] = tot;
-      compute_bar();
-      if (tid < kGuRowsItem) {
-        float g = 0.f, uu = 0.f;
-#pragma unroll
-        for (int w4 = 0; w4 < 4; ++w4) {
-          g += s_part[w4][tid];
-          uu += s_part[4 + w4][tid];
-        }
-        g *= x_unscale * gu.ts0[e];
-        uu *= x_unscale * gu.ts1[e];
+      accg = warp_sum(accg);
+      accu = warp_sum(accu);
+      if (lane == 0) {
+        const float g = accg * x_unscale * gu.ts0[e], uu = accu * x_unscale * gu.ts1[e];
         const uint16_t hb = f32_to_bf16_bits(clamped_swiglu(g, uu, gu.limit));
-        gu.out[(size_t)a * I + row0 + tid] = hb;
+        gu.out[(size_t)a * I + row0 + warp] = hb;
         atomicMax(gu.out_max + a, __float_as_uint(fabsf(bf16_bits_to_f32(hb))));
-      }
-      compute_bar();                                  // s_part reuse; this item's h written
-      if (tid == 0) {
         __threadfence();
-        atomicAdd(counters + 1 + u, 1);
+        atomicAdd(counters + 1 + u, 1);               // one count per warp: kGuRowsItem per item
       }
     } else {
       // down: warp w owns rows 8w .. 8w+7 of the item, lane c chunk c
       const int j = item - n_g, u = j / bpe_d, row0 = (j - u * bpe_d) * kDnRowsItem;
       const int e = dn.active[1 + u], a = dn.first[u];
-      if (tid == 0) {
-        const bool okw = wait_counter(counters + 1 + u, bpe_g);
+      int okw = 1;
+      if (lane == 0) {
+        okw = wait_counter(counters + 1 + u, bpe_g * kGuRowsItem) ? 1 : 0;
         if (!okw) set_status(gu.status, kDevErrTimeout);
-        s_ok = okw ? 1 : 0;
       }
-      compute_bar();
-      if (!s_ok) {
-        __syncwarp();
+      okw = __shfl_sync(0xffffffffu, okw, 0);
+      __syncwarp();
+      if (!okw) {
         if (lane == 0) mbar_arrive(&empty_bar[s]);
         continue;
       }
