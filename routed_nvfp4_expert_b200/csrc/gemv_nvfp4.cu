@@ -36,7 +36,7 @@ RNX_DEVICE bool wait_counter(const int* c, int need) {
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(c) : "memory");
     if (v >= need) return true;
     if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
-    __nanosleep(64);
+    __nanosleep(256);
   }
 }
 
@@ -511,19 +511,19 @@ nvfp4_gemv_direct_kernel(GemvParams p) {
 // output features = 8 gate + 8 up rows each, one feature per compute warp),
 // then the down blocks (64 output rows each, 8 per warp); one item is 36 KB
 // of codes and scales at H = 4096, I = 1024. Each warp reduces its rows with
-// shuffles only. One producer warp claims items (4 at a time) from a counter
+// shuffles; a gate/up item's CTA counts it done once all 8 rows are written. One producer warp claims items (4 at a time) from a counter
 // and copies each item's rows
 // with bulk copies (TMA engine) into a 5-stage ring, so ~180 KB per SM are in
 // flight whatever the compute warps do; 8 compute warps decode, multiply and
 // reduce from shared memory, release the stage, and write h (with the
 // per-assignment max |h|) or r. A down item waits until every gate/up item of
 // its expert has published h (per-expert counter, release / acquire at gpu
-// scope; every warp of a gate/up item counts once). Every gate/up item has a
+// scope; one count per finished gate/up item). Every gate/up item has a
 // lower number than every down item, gate/up items never wait, and each CTA
 // finishes its items in claim order, so every awaited item is held by a
 // running CTA that will finish it. All waits are bounded; a timeout sets the
 // status word and winds the CTA down. counters: [0] = next item, [1 + u] =
-// finished gate/up warp-rows of active expert u; zeroed upstream.
+// finished gate/up items of active expert u; zeroed upstream.
 constexpr int kStreamStages = 5;
 constexpr int kStreamItemBytes = 36864;
 constexpr int kStreamCompute = 8;                        // compute warps
@@ -531,12 +531,14 @@ constexpr int kStreamThreads = (kStreamCompute + 1) * 32;
 constexpr int kGuRowsItem = kStreamCompute;             // output features per gate/up item (one per warp)
 constexpr int kDnRowsItem = 64;                          // output rows per down item
 constexpr int kStreamMaxH = 4096;
+constexpr int kMaxStreamExperts = 16;                    // one token: at most top_k active experts
 
 RNX_DEVICE void compute_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kStreamCompute * 32) : "memory"); }
 
 __global__ void __launch_bounds__(kStreamThreads, 1)
 nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn, int* counters) {
   extern __shared__ __align__(128) uint8_t s_dyn[];
+  __shared__ int s_ok;
   uint8_t* stages = s_dyn;                                               // [S][36 KB]
   uint4* s_x = reinterpret_cast<uint4*>(s_dyn + kStreamStages * kStreamItemBytes);   // x as f16, [4][H/32] units
   __shared__ __align__(8) uint64_t full_bar[kStreamStages], empty_bar[kStreamStages];
@@ -556,7 +558,16 @@ nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn, int* counters) {
   __syncthreads();
   pdl_wait();       // follows the routing plan
   pdl_trigger();
-  const int n_act = gu.active[0];
+  // the active experts and their assignment (one token: at most top_k of them)
+  __shared__ int s_e[kMaxStreamExperts], s_a[kMaxStreamExperts], s_n;
+  if (tid == 0) s_n = min(gu.active[0], kMaxStreamExperts);
+  __syncthreads();
+  const int n_act = s_n;
+  for (int u = tid; u < n_act; u += blockDim.x) {
+    s_e[u] = gu.active[1 + u];
+    s_a[u] = gu.first[u];
+  }
+  __syncthreads();
   const int bpe_g = I / kGuRowsItem, bpe_d = H / kDnRowsItem;
   const int n_g = n_act * bpe_g, n_all = n_g + n_act * bpe_d;
 
@@ -589,7 +600,7 @@ nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn, int* counters) {
         uint8_t* st = stages + (size_t)s * kStreamItemBytes;
         if (item < n_g) {
           const int u = item / bpe_g, row0 = (item - u * bpe_g) * kGuRowsItem;
-          const size_t gr = (size_t)gu.active[1 + u] * I + row0;
+          const size_t gr = (size_t)s_e[u] * I + row0;
           const uint32_t cb = kGuRowsItem * gu_row_bytes, sb = kGuRowsItem * gu_sc_bytes;
           mbar_arrive_expect_tx(&full_bar[s], 2 * (cb + sb));
           bulk_g2s(st, gu.codes0 + gr * gu_row_bytes, cb, &full_bar[s], pol);
@@ -598,7 +609,7 @@ nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn, int* counters) {
           bulk_g2s(st + 2 * cb + sb, gu.scales1 + gr * gu_sc_bytes, sb, &full_bar[s], pol);
         } else {
           const int j = item - n_g, u = j / bpe_d, row0 = (j - u * bpe_d) * kDnRowsItem;
-          const size_t gr = (size_t)dn.active[1 + u] * H + row0;
+          const size_t gr = (size_t)s_e[u] * H + row0;
           const uint32_t cb = kDnRowsItem * dn_row_bytes, sb = kDnRowsItem * dn_sc_bytes;
           mbar_arrive_expect_tx(&full_bar[s], cb + sb);
           bulk_g2s(st, dn.codes0 + gr * dn_row_bytes, cb, &full_bar[s], pol);
@@ -646,7 +657,7 @@ nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn, int* counters) {
       // gate/up: warp w owns feature row0 + w (its gate row and its up row)
       // over the whole K; lanes take chunks w.r.t. lane, lane + 32, ...
       const int u = item / bpe_g, row0 = (item - u * bpe_g) * kGuRowsItem;
-      const int e = gu.active[1 + u], a = gu.first[u];
+      const int e = s_e[u], a = s_a[u];
       const uint8_t* cg = st + warp * gu_row_bytes;
       const uint8_t* cu = st + (kGuRowsItem + warp) * gu_row_bytes;
       const uint8_t* sg = st + 2 * kGuRowsItem * gu_row_bytes + warp * gu_sc_bytes;
@@ -674,21 +685,24 @@ nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn, int* counters) {
         const uint16_t hb = f32_to_bf16_bits(clamped_swiglu(g, uu, gu.limit));
         gu.out[(size_t)a * I + row0 + warp] = hb;
         atomicMax(gu.out_max + a, __float_as_uint(fabsf(bf16_bits_to_f32(hb))));
+      }
+      compute_bar();                                  // every warp's h row of this item is written
+      if (tid == 0) {
         __threadfence();
-        atomicAdd(counters + 1 + u, 1);               // one count per warp: kGuRowsItem per item
+        atomicAdd(counters + 1 + u, 1);
       }
     } else {
       // down: warp w owns rows 8w .. 8w+7 of the item, lane c chunk c
       const int j = item - n_g, u = j / bpe_d, row0 = (j - u * bpe_d) * kDnRowsItem;
-      const int e = dn.active[1 + u], a = dn.first[u];
-      int okw = 1;
-      if (lane == 0) {
-        okw = wait_counter(counters + 1 + u, bpe_g * kGuRowsItem) ? 1 : 0;
+      const int e = s_e[u], a = s_a[u];
+      if (tid == 0) {
+        const bool okw = wait_counter(counters + 1 + u, bpe_g);
         if (!okw) set_status(gu.status, kDevErrTimeout);
+        s_ok = okw ? 1 : 0;
       }
-      okw = __shfl_sync(0xffffffffu, okw, 0);
-      __syncwarp();
-      if (!okw) {
+      compute_bar();
+      if (!s_ok) {
+        __syncwarp();
         if (lane == 0) mbar_arrive(&empty_bar[s]);
         continue;
       }
