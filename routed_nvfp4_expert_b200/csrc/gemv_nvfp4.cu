@@ -278,14 +278,17 @@ RNX_DEVICE void decode_chunk(const uint4& q, uint32_t (&w)[16]) {
 
 // acc += s.x * (sum of the first 16 products) + s.y * (sum of the last 16)
 RNX_DEVICE void chunk_fma(const uint32_t (&w)[16], const uint32_t (&x)[16], float2 s, float& acc) {
-  __half2 p0 = __float2half2_rn(0.f), p1 = __float2half2_rn(0.f);
+  // two independent 4-step chains per 16-element block (shorter dependency
+  // chains; the f16 partials of a block are added before widening)
+  __half2 p0 = __float2half2_rn(0.f), p1 = __float2half2_rn(0.f), p2 = p0, p3 = p0;
 #pragma unroll
-  for (int j = 0; j < 8; ++j)
+  for (int j = 0; j < 4; ++j) {
     p0 = __hfma2(*reinterpret_cast<const __half2*>(&w[j]), *reinterpret_cast<const __half2*>(&x[j]), p0);
-#pragma unroll
-  for (int j = 8; j < 16; ++j)
-    p1 = __hfma2(*reinterpret_cast<const __half2*>(&w[j]), *reinterpret_cast<const __half2*>(&x[j]), p1);
-  const float2 f0 = __half22float2(p0), f1 = __half22float2(p1);
+    p1 = __hfma2(*reinterpret_cast<const __half2*>(&w[j + 4]), *reinterpret_cast<const __half2*>(&x[j + 4]), p1);
+    p2 = __hfma2(*reinterpret_cast<const __half2*>(&w[j + 8]), *reinterpret_cast<const __half2*>(&x[j + 8]), p2);
+    p3 = __hfma2(*reinterpret_cast<const __half2*>(&w[j + 12]), *reinterpret_cast<const __half2*>(&x[j + 12]), p3);
+  }
+  const float2 f0 = __half22float2(__hadd2(p0, p1)), f1 = __half22float2(__hadd2(p2, p3));
   acc = fmaf(s.x, f0.x + f0.y, acc);
   acc = fmaf(s.y, f1.x + f1.y, acc);
 }
@@ -526,9 +529,10 @@ nvfp4_gemv_direct_kernel(GemvParams p) {
 // finished gate/up items of active expert u; zeroed upstream.
 constexpr int kStreamStages = 5;
 constexpr int kStreamItemBytes = 36864;
-constexpr int kStreamCompute = 8;                        // compute warps
+constexpr int kStreamCompute = 16;                       // compute warps
 constexpr int kStreamThreads = (kStreamCompute + 1) * 32;
-constexpr int kGuRowsItem = kStreamCompute;             // output features per gate/up item (one per warp)
+constexpr int kGuRowsItem = 8;                           // output features per gate/up item
+constexpr int kDnRowsWarp = 4;                           // down rows per compute warp
 constexpr int kDnRowsItem = 64;                          // output rows per down item
 constexpr int kStreamMaxH = 4096;
 constexpr int kMaxStreamExperts = 16;                    // one token: at most top_k active experts
@@ -539,6 +543,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
 nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn, int* counters) {
   extern __shared__ __align__(128) uint8_t s_dyn[];
   __shared__ int s_ok;
+  __shared__ float s_gu[2][2 * kGuRowsItem];                             // gate / up row sums, by item parity
   uint8_t* stages = s_dyn;                                               // [S][36 KB]
   uint4* s_x = reinterpret_cast<uint4*>(s_dyn + kStreamStages * kStreamItemBytes);   // x as f16, [4][H/32] units
   __shared__ __align__(8) uint64_t full_bar[kStreamStages], empty_bar[kStreamStages];
@@ -654,15 +659,14 @@ nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn, int* counters) {
     if (item < 0) break;
     const uint8_t* st = stages + (size_t)s * kStreamItemBytes;
     if (item < n_g) {
-      // gate/up: warp w owns feature row0 + w (its gate row and its up row)
-      // over the whole K; lanes take chunks w.r.t. lane, lane + 32, ...
+      // gate/up: warp w owns one weight row over the whole K (warps 0-7 the
+      // gate rows of the item's 8 features, warps 8-15 their up rows); lanes
+      // take chunks lane, lane + 32, ...
       const int u = item / bpe_g, row0 = (item - u * bpe_g) * kGuRowsItem;
       const int e = s_e[u], a = s_a[u];
-      const uint8_t* cg = st + warp * gu_row_bytes;
-      const uint8_t* cu = st + (kGuRowsItem + warp) * gu_row_bytes;
-      const uint8_t* sg = st + 2 * kGuRowsItem * gu_row_bytes + warp * gu_sc_bytes;
-      const uint8_t* su = st + 2 * kGuRowsItem * gu_row_bytes + (kGuRowsItem + warp) * gu_sc_bytes;
-      float accg = 0.f, accu = 0.f;
+      const uint8_t* cw = st + warp * gu_row_bytes;     // gate rows then up rows, contiguous
+      const uint8_t* sw = st + 2 * kGuRowsItem * gu_row_bytes + warp * gu_sc_bytes;
+      float acc = 0.f;
       for (int c = lane; c < nchG; c += 32) {
         uint32_t xr[16];
 #pragma unroll
@@ -671,22 +675,22 @@ nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn, int* counters) {
           xr[4 * q] = v.x; xr[4 * q + 1] = v.y; xr[4 * q + 2] = v.z; xr[4 * q + 3] = v.w;
         }
         uint32_t w[16];
-        decode_chunk(*reinterpret_cast<const uint4*>(cg + 16 * c), w);
-        chunk_fma(w, xr, e4m3x2_to_f32x2(*reinterpret_cast<const uint16_t*>(sg + 2 * c)), accg);
-        decode_chunk(*reinterpret_cast<const uint4*>(cu + 16 * c), w);
-        chunk_fma(w, xr, e4m3x2_to_f32x2(*reinterpret_cast<const uint16_t*>(su + 2 * c)), accu);
+        decode_chunk(*reinterpret_cast<const uint4*>(cw + 16 * c), w);
+        chunk_fma(w, xr, e4m3x2_to_f32x2(*reinterpret_cast<const uint16_t*>(sw + 2 * c)), acc);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty_bar[s]);      // this warp is done with the stage
-      accg = warp_sum(accg);
-      accu = warp_sum(accu);
-      if (lane == 0) {
-        const float g = accg * x_unscale * gu.ts0[e], uu = accu * x_unscale * gu.ts1[e];
+      acc = warp_sum(acc);
+      if (lane == 0) s_gu[it & 1][warp] = acc;
+      compute_bar();
+      if (tid < kGuRowsItem) {
+        const float g = s_gu[it & 1][tid] * x_unscale * gu.ts0[e];
+        const float uu = s_gu[it & 1][kGuRowsItem + tid] * x_unscale * gu.ts1[e];
         const uint16_t hb = f32_to_bf16_bits(clamped_swiglu(g, uu, gu.limit));
-        gu.out[(size_t)a * I + row0 + warp] = hb;
+        gu.out[(size_t)a * I + row0 + tid] = hb;
         atomicMax(gu.out_max + a, __float_as_uint(fabsf(bf16_bits_to_f32(hb))));
       }
-      compute_bar();                                  // every warp's h row of this item is written
+      compute_bar();                                  // the item's 8 h values are written
       if (tid == 0) {
         __threadfence();
         atomicAdd(counters + 1 + u, 1);
@@ -709,16 +713,16 @@ nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn, int* counters) {
       float up, unscale;
       prescale_from_max(__uint_as_float(dn.act_max[a]), up, unscale);
       const uint16_t* arow = dn.act + (size_t)a * I;
-      const uint8_t* cb = st + warp * kDirectRows * dn_row_bytes;
-      const uint8_t* sb = st + kDnRowsItem * dn_row_bytes + warp * kDirectRows * dn_sc_bytes;
-      float acc[kDirectRows];
+      const uint8_t* cb = st + warp * kDnRowsWarp * dn_row_bytes;
+      const uint8_t* sb = st + kDnRowsItem * dn_row_bytes + warp * kDnRowsWarp * dn_sc_bytes;
+      float acc[kDnRowsWarp];
 #pragma unroll
-      for (int r = 0; r < kDirectRows; ++r) acc[r] = 0.f;
+      for (int r = 0; r < kDnRowsWarp; ++r) acc[r] = 0.f;
       for (int c = lane; c < nchD; c += 32) {
         uint32_t xr[16];
         load_act_chunk(arow, c, true, up, xr);
 #pragma unroll
-        for (int r = 0; r < kDirectRows; ++r) {
+        for (int r = 0; r < kDnRowsWarp; ++r) {
           const uint4 qv = *reinterpret_cast<const uint4*>(cb + r * dn_row_bytes + 16 * c);
           const uint16_t sv = *reinterpret_cast<const uint16_t*>(sb + r * dn_sc_bytes + 2 * c);
           uint32_t w[16];
@@ -728,9 +732,9 @@ nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn, int* counters) {
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty_bar[s]);
-      const float tot = warp_reduce_rows<kDirectRows>(acc);
-      if ((lane & 3) == 0) {
-        const int row = row0 + warp * kDirectRows + (lane >> 2);
+      const float tot = warp_reduce_rows<kDnRowsWarp>(acc);   // lane 8r holds row r
+      if ((lane & 7) == 0) {
+        const int row = row0 + warp * kDnRowsWarp + (lane >> 3);
         dn.out[(size_t)a * H + row] = f32_to_bf16_bits(tot * unscale * dn.ts0[e] * dn.weights[a]);
       }
     }
