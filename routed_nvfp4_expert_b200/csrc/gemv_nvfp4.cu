@@ -514,19 +514,19 @@ nvfp4_gemv_direct_kernel(GemvParams p) {
 // output features = 8 gate + 8 up rows each, one feature per compute warp),
 // then the down blocks (64 output rows each, 8 per warp); one item is 36 KB
 // of codes and scales at H = 4096, I = 1024. Each warp reduces its rows with
-// shuffles; a gate/up item's CTA counts it done once all 8 rows are written. One producer warp claims items (4 at a time) from a counter
+// shuffles; each of a gate/up item's 8 h values is published by its writer. One producer warp claims items (4 at a time) from a counter
 // and copies each item's rows
 // with bulk copies (TMA engine) into a 5-stage ring, so ~180 KB per SM are in
 // flight whatever the compute warps do; 8 compute warps decode, multiply and
 // reduce from shared memory, release the stage, and write h (with the
 // per-assignment max |h|) or r. A down item waits until every gate/up item of
 // its expert has published h (per-expert counter, release / acquire at gpu
-// scope; one count per finished gate/up item). Every gate/up item has a
+// scope; every h value of a gate/up item counts once). Every gate/up item has a
 // lower number than every down item, gate/up items never wait, and each CTA
 // finishes its items in claim order, so every awaited item is held by a
 // running CTA that will finish it. All waits are bounded; a timeout sets the
 // status word and winds the CTA down. counters: [0] = next item, [1 + u] =
-// finished gate/up items of active expert u; zeroed upstream.
+// published h values of active expert u; zeroed upstream.
 constexpr int kStreamStages = 5;
 constexpr int kStreamItemBytes = 36864;
 constexpr int kStreamCompute = 16;                       // compute warps
@@ -563,14 +563,22 @@ nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn, int* counters) {
   __syncthreads();
   pdl_wait();       // follows the routing plan
   pdl_trigger();
-  // the active experts and their assignment (one token: at most top_k of them)
+  // the active experts, their assignment, tensor scales and routing weight
+  // (one token: at most top_k of them)
   __shared__ int s_e[kMaxStreamExperts], s_a[kMaxStreamExperts], s_n;
+  __shared__ float s_tg[kMaxStreamExperts], s_tu[kMaxStreamExperts], s_td[kMaxStreamExperts],
+      s_wt[kMaxStreamExperts];
   if (tid == 0) s_n = min(gu.active[0], kMaxStreamExperts);
   __syncthreads();
   const int n_act = s_n;
   for (int u = tid; u < n_act; u += blockDim.x) {
-    s_e[u] = gu.active[1 + u];
-    s_a[u] = gu.first[u];
+    const int e = gu.active[1 + u], a = gu.first[u];
+    s_e[u] = e;
+    s_a[u] = a;
+    s_tg[u] = gu.ts0[e];
+    s_tu[u] = gu.ts1[e];
+    s_td[u] = dn.ts0[e];
+    s_wt[u] = dn.weights[a];
   }
   __syncthreads();
   const int bpe_g = I / kGuRowsItem, bpe_d = H / kDnRowsItem;
@@ -684,23 +692,21 @@ nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn, int* counters) {
       if (lane == 0) s_gu[it & 1][warp] = acc;
       compute_bar();
       if (tid < kGuRowsItem) {
-        const float g = s_gu[it & 1][tid] * x_unscale * gu.ts0[e];
-        const float uu = s_gu[it & 1][kGuRowsItem + tid] * x_unscale * gu.ts1[e];
+        // each of the 8 writers publishes its own h value: store, max, then a
+        // release add on the expert's counter (8 per item)
+        const float g = s_gu[it & 1][tid] * x_unscale * s_tg[u];
+        const float uu = s_gu[it & 1][kGuRowsItem + tid] * x_unscale * s_tu[u];
         const uint16_t hb = f32_to_bf16_bits(clamped_swiglu(g, uu, gu.limit));
         gu.out[(size_t)a * I + row0 + tid] = hb;
         atomicMax(gu.out_max + a, __float_as_uint(fabsf(bf16_bits_to_f32(hb))));
-      }
-      compute_bar();                                  // the item's 8 h values are written
-      if (tid == 0) {
-        __threadfence();
-        atomicAdd(counters + 1 + u, 1);
+        asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(counters + 1 + u) : "memory");
       }
     } else {
       // down: warp w owns rows 8w .. 8w+7 of the item, lane c chunk c
       const int j = item - n_g, u = j / bpe_d, row0 = (j - u * bpe_d) * kDnRowsItem;
       const int e = s_e[u], a = s_a[u];
       if (tid == 0) {
-        const bool okw = wait_counter(counters + 1 + u, bpe_g);
+        const bool okw = wait_counter(counters + 1 + u, bpe_g * kGuRowsItem);
         if (!okw) set_status(gu.status, kDevErrTimeout);
         s_ok = okw ? 1 : 0;
       }
@@ -735,7 +741,7 @@ nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn, int* counters) {
       const float tot = warp_reduce_rows<kDnRowsWarp>(acc);   // lane 8r holds row r
       if ((lane & 7) == 0) {
         const int row = row0 + warp * kDnRowsWarp + (lane >> 3);
-        dn.out[(size_t)a * H + row] = f32_to_bf16_bits(tot * unscale * dn.ts0[e] * dn.weights[a]);
+        dn.out[(size_t)a * H + row] = f32_to_bf16_bits(tot * unscale * s_td[u] * s_wt[u]);
       }
     }
   }
