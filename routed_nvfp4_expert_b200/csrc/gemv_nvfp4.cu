@@ -511,43 +511,61 @@ nvfp4_gemv_direct_kernel(GemvParams p) {
 // token per expert), streaming the weights through shared memory.
 //
 // Work items, in claim order: the gate/up blocks of every active expert (8
-// output features = 8 gate + 8 up rows each, one feature per compute warp),
-// then the down blocks (64 output rows each, 8 per warp); one item is 36 KB
-// of codes and scales at H = 4096, I = 1024. Each warp reduces its rows with
-// shuffles; each of a gate/up item's 8 h values is published by its writer. One producer warp claims items (4 at a time) from a counter
-// and copies each item's rows
-// with bulk copies (TMA engine) into a 5-stage ring, so ~180 KB per SM are in
-// flight whatever the compute warps do; 8 compute warps decode, multiply and
-// reduce from shared memory, release the stage, and write h (with the
-// per-assignment max |h|) or r. A down item waits until every gate/up item of
-// its expert has published h (per-expert counter, release / acquire at gpu
-// scope; every h value of a gate/up item counts once). Every gate/up item has a
-// lower number than every down item, gate/up items never wait, and each CTA
-// finishes its items in claim order, so every awaited item is held by a
-// running CTA that will finish it. All waits are bounded; a timeout sets the
-// status word and winds the CTA down. counters: [0] = next item, [1 + u] =
-// published h values of active expert u; zeroed upstream.
+// output features = 8 gate + 8 up rows each), then the down blocks (64 output
+// rows each); one item is 36 KB of codes and scales at H = 4096, I = 1024.
+// Warp roles per CTA (one CTA per SM):
+//  * producer (one lane): claims items 4 at a time from a counter and copies
+//    each item's rows with bulk copies (TMA engine) into a 5-stage ring. For a
+//    down item it then waits until every gate/up item of its expert has been
+//    published, and copies the finished h row (and its max |h|) into the same
+//    stage; only then does the stage become full.
+//  * 16 compute warps: decode, multiply and reduce from shared memory (gate/
+//    up: one gate or up row per warp; down: four rows per warp), release the
+//    stage, write h (with the per-assignment max |h|) or r.
+//  * publisher (one lane): after the writers of a gate/up item signal it,
+//    makes their h values visible at gpu scope and counts the item on its
+//    expert's counter -- the fence latency stays off the compute path.
+// Every gate/up item has a lower number than every down item, gate/up items
+// never wait, and each CTA finishes its items in claim order, so every
+// awaited item is held by a running CTA that will finish it. All waits are
+// bounded; a timeout sets the status word and winds the CTA down.
+// counters: [0] = next item, [1 + u] = published gate/up items of active
+// expert u; zeroed upstream.
 constexpr int kStreamStages = 5;
-constexpr int kStreamItemBytes = 36864;
+constexpr int kStreamWeightBytes = 36864;                // codes + scales of one item
+constexpr int kStreamItemBytes = kStreamWeightBytes + 2048 + 16;   // + h row (I <= 1024) + its max
+constexpr int kStreamStageBytes = (kStreamItemBytes + 127) / 128 * 128;
 constexpr int kStreamCompute = 16;                       // compute warps
-constexpr int kStreamThreads = (kStreamCompute + 1) * 32;
+constexpr int kStreamProducer = kStreamCompute, kStreamPublisher = kStreamCompute + 1;
+constexpr int kStreamThreads = (kStreamCompute + 2) * 32;
 constexpr int kGuRowsItem = 8;                           // output features per gate/up item
 constexpr int kDnRowsWarp = 4;                           // down rows per compute warp
 constexpr int kDnRowsItem = 64;                          // output rows per down item
 constexpr int kStreamMaxH = 4096;
+constexpr int kStreamMaxI = 1024;
 constexpr int kMaxStreamExperts = 16;                    // one token: at most top_k active experts
 
 RNX_DEVICE void compute_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kStreamCompute * 32) : "memory"); }
 
+// Hand the n-th gate/up item (expert u, or -1 = end) to the publisher: wait
+// until the publisher has read the slot's previous entry, then write it.
+RNX_DEVICE void pub_slot(int* s_pub, uint64_t* pub_free, int n, int u, uint32_t* status) {
+  if (!mbar_wait(&pub_free[n & 1], ((uint32_t)(n >> 1) & 1u) ^ 1u)) set_status(status, kDevErrTimeout);
+  s_pub[n & 1] = u;
+}
+
 __global__ void __launch_bounds__(kStreamThreads, 1)
 nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn, int* counters) {
   extern __shared__ __align__(128) uint8_t s_dyn[];
-  __shared__ int s_ok;
-  __shared__ float s_gu[2][2 * kGuRowsItem];                             // gate / up row sums, by item parity
-  uint8_t* stages = s_dyn;                                               // [S][36 KB]
-  uint4* s_x = reinterpret_cast<uint4*>(s_dyn + kStreamStages * kStreamItemBytes);   // x as f16, [4][H/32] units
-  __shared__ __align__(8) uint64_t full_bar[kStreamStages], empty_bar[kStreamStages];
+  uint8_t* stages = s_dyn;                                               // [S][stage]
+  uint4* s_x = reinterpret_cast<uint4*>(s_dyn + kStreamStages * kStreamStageBytes);   // x as f16, [4][H/32]
+  __shared__ __align__(8) uint64_t full_bar[kStreamStages], empty_bar[kStreamStages], pub_bar[2], pub_free[2];
   __shared__ int s_item[kStreamStages];
+  __shared__ int s_pub[2];                               // expert of the gate/up item being published, -1 = end
+  __shared__ float s_gu[2][2 * kGuRowsItem];             // gate / up row sums, by item parity
+  __shared__ int s_e[kMaxStreamExperts], s_a[kMaxStreamExperts], s_n;
+  __shared__ float s_tg[kMaxStreamExperts], s_tu[kMaxStreamExperts], s_td[kMaxStreamExperts],
+      s_wt[kMaxStreamExperts];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = gu.K, I = gu.rows;
   const int nchG = H / 32, nchD = I / 32;
@@ -558,16 +576,15 @@ nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn, int* counters) {
       mbar_init(&full_bar[i], 1);
       mbar_init(&empty_bar[i], kStreamCompute);
     }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&pub_bar[b], kGuRowsItem);   // the item's 8 writers
+      mbar_init(&pub_free[b], 1);            // the publisher has read the slot
+    }
     fence_barrier_init();
   }
-  __syncthreads();
   pdl_wait();       // follows the routing plan
   pdl_trigger();
   // the active experts, their assignment, tensor scales and routing weight
-  // (one token: at most top_k of them)
-  __shared__ int s_e[kMaxStreamExperts], s_a[kMaxStreamExperts], s_n;
-  __shared__ float s_tg[kMaxStreamExperts], s_tu[kMaxStreamExperts], s_td[kMaxStreamExperts],
-      s_wt[kMaxStreamExperts];
   if (tid == 0) s_n = min(gu.active[0], kMaxStreamExperts);
   __syncthreads();
   const int n_act = s_n;
@@ -584,12 +601,10 @@ nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn, int* counters) {
   const int bpe_g = I / kGuRowsItem, bpe_d = H / kDnRowsItem;
   const int n_g = n_act * bpe_g, n_all = n_g + n_act * bpe_d;
 
-  if (warp == kStreamCompute) {
+  if (warp == kStreamProducer) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
-      // items are claimed kClaim at a time, the next batch requested before
-      // the current one is used up (the atomic's round trip overlaps copies)
       constexpr int kClaim = 4;
       int batch = atomicAdd(counters, kClaim), next_batch = atomicAdd(counters, kClaim), in_batch = 0;
       int it = 0;
@@ -610,7 +625,7 @@ nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn, int* counters) {
           break;
         }
         s_item[s] = item;
-        uint8_t* st = stages + (size_t)s * kStreamItemBytes;
+        uint8_t* st = stages + (size_t)s * kStreamStageBytes;
         if (item < n_g) {
           const int u = item / bpe_g, row0 = (item - u * bpe_g) * kGuRowsItem;
           const size_t gr = (size_t)s_e[u] * I + row0;
@@ -624,15 +639,40 @@ nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn, int* counters) {
           const int j = item - n_g, u = j / bpe_d, row0 = (j - u * bpe_d) * kDnRowsItem;
           const size_t gr = (size_t)s_e[u] * H + row0;
           const uint32_t cb = kDnRowsItem * dn_row_bytes, sb = kDnRowsItem * dn_sc_bytes;
-          mbar_arrive_expect_tx(&full_bar[s], cb + sb);
           bulk_g2s(st, dn.codes0 + gr * dn_row_bytes, cb, &full_bar[s], pol);
           bulk_g2s(st + cb, dn.scales0 + gr * dn_sc_bytes, sb, &full_bar[s], pol);
+          // the expert's h must be complete before its row is copied
+          const bool ready = wait_counter(counters + 1 + u, bpe_g);
+          if (!ready) set_status(gu.status, kDevErrTimeout);
+          asm volatile("fence.proxy.async.global;" ::: "memory");   // published h -> bulk-copy reads
+          const int a = s_a[u];
+          bulk_g2s(st + kStreamWeightBytes, dn.act + (size_t)a * I, (uint32_t)I * 2, &full_bar[s], pol);
+          bulk_g2s(st + kStreamWeightBytes + 2048, dn.act_max + (a & ~3), 16, &full_bar[s], pol);
+          mbar_arrive_expect_tx(&full_bar[s], cb + sb + (uint32_t)I * 2 + 16);
         }
       }
       // copies in flight must land before the CTA may exit
       for (int j = max(0, it - kStreamStages + 1); j < it; ++j)
         if (!mbar_wait(&full_bar[j % kStreamStages], (uint32_t)(j / kStreamStages) & 1u))
           set_status(gu.status, kDevErrTimeout);
+    }
+    return;
+  }
+
+  if (warp == kStreamPublisher) {
+    // ------------------------------------------------------------ publisher
+    if (lane == 0) {
+      for (int k = 0;; ++k) {
+        if (!mbar_wait(&pub_bar[k & 1], (uint32_t)(k >> 1) & 1u)) {
+          set_status(gu.status, kDevErrTimeout);
+          break;
+        }
+        const int u = s_pub[k & 1];
+        mbar_arrive(&pub_free[k & 1]);
+        if (u < 0) break;
+        __threadfence();                   // the writers' h values, seen through the barrier
+        atomicAdd(counters + 1 + u, 1);
+      }
     }
     return;
   }
@@ -656,6 +696,7 @@ nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn, int* counters) {
   }
   compute_bar();
 
+  int npub = 0;                            // gate/up items handed to the publisher
   for (int it = 0;; ++it) {
     const int s = it % kStreamStages;
     const uint32_t ph = (uint32_t)(it / kStreamStages) & 1u;
@@ -665,13 +706,12 @@ nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn, int* counters) {
     }
     const int item = s_item[s];
     if (item < 0) break;
-    const uint8_t* st = stages + (size_t)s * kStreamItemBytes;
+    const uint8_t* st = stages + (size_t)s * kStreamStageBytes;
     if (item < n_g) {
       // gate/up: warp w owns one weight row over the whole K (warps 0-7 the
-      // gate rows of the item's 8 features, warps 8-15 their up rows); lanes
-      // take chunks lane, lane + 32, ...
+      // gate rows of the item's 8 features, warps 8-15 their up rows)
       const int u = item / bpe_g, row0 = (item - u * bpe_g) * kGuRowsItem;
-      const int e = s_e[u], a = s_a[u];
+      const int a = s_a[u];
       const uint8_t* cw = st + warp * gu_row_bytes;     // gate rows then up rows, contiguous
       const uint8_t* sw = st + 2 * kGuRowsItem * gu_row_bytes + warp * gu_sc_bytes;
       float acc = 0.f;
@@ -692,33 +732,23 @@ nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn, int* counters) {
       if (lane == 0) s_gu[it & 1][warp] = acc;
       compute_bar();
       if (tid < kGuRowsItem) {
-        // each of the 8 writers publishes its own h value: store, max, then a
-        // release add on the expert's counter (8 per item)
         const float g = s_gu[it & 1][tid] * x_unscale * s_tg[u];
         const float uu = s_gu[it & 1][kGuRowsItem + tid] * x_unscale * s_tu[u];
         const uint16_t hb = f32_to_bf16_bits(clamped_swiglu(g, uu, gu.limit));
         gu.out[(size_t)a * I + row0 + tid] = hb;
         atomicMax(gu.out_max + a, __float_as_uint(fabsf(bf16_bits_to_f32(hb))));
-        asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(counters + 1 + u) : "memory");
+        if (tid == 0) pub_slot(s_pub, pub_free, npub, u, gu.status);
+        mbar_arrive(&pub_bar[npub & 1]);
       }
+      ++npub;
     } else {
-      // down: warp w owns rows 8w .. 8w+7 of the item, lane c chunk c
+      // down: warp w owns rows 4w .. 4w+3 of the item, lane c chunk c; the h
+      // row and its max came with the stage
       const int j = item - n_g, u = j / bpe_d, row0 = (j - u * bpe_d) * kDnRowsItem;
-      const int e = s_e[u], a = s_a[u];
-      if (tid == 0) {
-        const bool okw = wait_counter(counters + 1 + u, bpe_g * kGuRowsItem);
-        if (!okw) set_status(gu.status, kDevErrTimeout);
-        s_ok = okw ? 1 : 0;
-      }
-      compute_bar();
-      if (!s_ok) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty_bar[s]);
-        continue;
-      }
+      const int a = s_a[u];
       float up, unscale;
-      prescale_from_max(__uint_as_float(dn.act_max[a]), up, unscale);
-      const uint16_t* arow = dn.act + (size_t)a * I;
+      prescale_from_max(*reinterpret_cast<const float*>(st + kStreamWeightBytes + 2048 + 4 * (a & 3)), up, unscale);
+      const uint16_t* hrow = reinterpret_cast<const uint16_t*>(st + kStreamWeightBytes);
       const uint8_t* cb = st + warp * kDnRowsWarp * dn_row_bytes;
       const uint8_t* sb = st + kDnRowsItem * dn_row_bytes + warp * kDnRowsWarp * dn_sc_bytes;
       float acc[kDnRowsWarp];
@@ -726,7 +756,7 @@ nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn, int* counters) {
       for (int r = 0; r < kDnRowsWarp; ++r) acc[r] = 0.f;
       for (int c = lane; c < nchD; c += 32) {
         uint32_t xr[16];
-        load_act_chunk(arow, c, true, up, xr);
+        load_act_chunk(hrow, c, true, up, xr);
 #pragma unroll
         for (int r = 0; r < kDnRowsWarp; ++r) {
           const uint4 qv = *reinterpret_cast<const uint4*>(cb + r * dn_row_bytes + 16 * c);
@@ -744,6 +774,11 @@ nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn, int* counters) {
         dn.out[(size_t)a * H + row] = f32_to_bf16_bits(tot * unscale * s_td[u] * s_wt[u]);
       }
     }
+  }
+  // end of the publisher's list
+  if (tid < kGuRowsItem) {
+    if (tid == 0) pub_slot(s_pub, pub_free, npub, -1, gu.status);
+    mbar_arrive(&pub_bar[npub & 1]);
   }
 }
 
@@ -836,7 +871,7 @@ cudaError_t launch_decode_experts(const ExpertGemvArgs& a, uint16_t* h, uint16_t
                                   cudaStream_t st) {
   // one token; an item's rows (16 x H/2 + 16 x H/16 and 64 x I/2 + 64 x I/16
   // bytes) fit one 36 KB stage
-  if (a.T != 1 || !a.act_max || !hmax || a.H > kStreamMaxH || 36 * a.I > kStreamItemBytes || a.H % kDnRowsItem ||
+  if (a.T != 1 || !a.act_max || !hmax || a.H > kStreamMaxH || a.I > kStreamMaxI || a.H % kDnRowsItem ||
       a.I % kGuRowsItem)
     return cudaErrorNotSupported;
   ExpertGemvArgs g = a, d = a;
@@ -845,11 +880,11 @@ cudaError_t launch_decode_experts(const ExpertGemvArgs& a, uint16_t* h, uint16_t
   const GemvParams pg = gemv_params(g, true), pd = gemv_params(d, false);
   const int max_active = std::min(a.local_end - a.local_begin, a.T * a.k);
   const bool remote = a.local_begin > 0 || a.local_end < a.E;
-  const size_t smem = (size_t)kStreamStages * kStreamItemBytes + (size_t)a.H * 2;
+  const size_t smem = (size_t)kStreamStages * kStreamStageBytes + (size_t)a.H * 2;
   static bool attr_done = false;
   if (!attr_done) {
     cudaError_t err = cudaFuncSetAttribute(nvfp4_experts_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)((size_t)kStreamStages * kStreamItemBytes + kStreamMaxH * 2));
+                                           (int)((size_t)kStreamStages * kStreamStageBytes + kStreamMaxH * 2));
     if (err != cudaSuccess) return err;
     attr_done = true;
   }
