@@ -190,7 +190,7 @@ WsLayout ws_layout(const moe_config_t* c, int T, int path) {
   L.shared_h = o; o = up(o + 2 * (size_t)T * Is);
   L.shared = o; o = up(o + 2 * (size_t)T * H);
   L.xmax = o; o = up(o + 4 * (size_t)T);
-  L.hmax = o; o = up(o + 4 * (2 * A + 1));   // h maxima [A], then the fused decode kernel's counters [1 + A]
+  L.hmax = o; o = up(o + 4 * (size_t)A);     // h maxima [A]
   if (pre) {
     L.xq = o; o = up(o + P * H / 2);
     L.xsf = o; o = up(o + P * H / 16);
@@ -670,7 +670,11 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
     const uint16_t* w3 = (const uint16_t*)(w->prepared + prepared_layout(cfg).router3);
     RNX_CUDA(rnx::launch_router_logits_tc(x, T, H, E, w3, logits, status, st), "router logits (tensor cores)");
   } else {
-    RNX_CUDA(rnx::launch_router_logits(x, T, H, E, w->router_w, logits, st, xmax, hmax, 2 * T * k + 1),
+    // decode: the h-max array is cleared, and for one token h is set to the
+    // "not yet written" pattern of the fused experts kernel
+    const bool fused = path == MOE_PATH_DECODE && T == 1;
+    RNX_CUDA(rnx::launch_router_logits(x, T, H, E, w->router_w, logits, st, xmax, hmax, T * k,
+                                       fused ? (uint32_t*)h : nullptr, fused ? T * k * I / 2 : 0),
              "router logits");
   }
   RNX_CUDA(mark(MOE_STAGE_TOPK, st), "stage event");
@@ -712,7 +716,7 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
     RNX_CUDA(mark(MOE_STAGE_EXPERT_GATE_UP, st), "stage event");
     // one token: gate/up and down in one persistent kernel (the down stage
     // then has zero length); otherwise one launch per projection
-    cudaError_t fe = rnx::launch_decode_experts(a, h, r, hmax, (int*)(hmax + (size_t)T * k), st);
+    cudaError_t fe = rnx::launch_decode_experts(a, h, r, st);
     if (fe == cudaErrorNotSupported) {
       RNX_CUDA(rnx::launch_nvfp4_gemv(a, st), "expert gate/up");
       RNX_CUDA(mark(MOE_STAGE_H_QUANT, st), "stage event");
