@@ -325,9 +325,9 @@ def run_ours(args, rank, world, local_rank):
                     "algorithmic_bytes_per_step": int(algo_bytes), "unique_experts_per_step": U,
                     "bytes_per_expert": expert_bytes(wl),
                     "traffic": read_traffic_profile(f"nvfp4_expert_gemv_{wl.name}")}
-        # router, top-k, plan, experts (one fused kernel at T = 1, else gate/up + down),
-        # combine, and the shared expert's two GEMVs on the auxiliary stream
-        launches_per_step = (7 if T == 1 else 8) if T * wl.k <= 1024 else 11
+        # router, top-k, plan, expert gate/up, expert down, combine, and the
+        # shared expert's two GEMVs on the auxiliary stream
+        launches_per_step = 8 if T * wl.k <= 1024 else 11
         path_name = "decode GEMV (W4A16)"
     out = {
         "metric": METRIC,

@@ -670,12 +670,7 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
     const uint16_t* w3 = (const uint16_t*)(w->prepared + prepared_layout(cfg).router3);
     RNX_CUDA(rnx::launch_router_logits_tc(x, T, H, E, w3, logits, status, st), "router logits (tensor cores)");
   } else {
-    // decode: the h-max array is cleared, and for one token h is set to the
-    // "not yet written" pattern of the fused experts kernel
-    const bool fused = path == MOE_PATH_DECODE && T == 1;
-    RNX_CUDA(rnx::launch_router_logits(x, T, H, E, w->router_w, logits, st, xmax, hmax, T * k,
-                                       fused ? (uint32_t*)h : nullptr, fused ? T * k * I / 2 : 0),
-             "router logits");
+    RNX_CUDA(rnx::launch_router_logits(x, T, H, E, w->router_w, logits, st, xmax, hmax, T * k), "router logits");
   }
   RNX_CUDA(mark(MOE_STAGE_TOPK, st), "stage event");
   RNX_CUDA(rnx::launch_topk(logits, w->router_bias, T, E, k, cfg->routed_scaling_factor, ids, wts, st), "top-k");
@@ -714,20 +709,11 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
     a.status = status;
     a.proj = MOE_PROJ_GATE_UP; a.act = x; a.out = h; a.act_max = xmax; a.out_max = hmax; a.prefetch_down = false;
     RNX_CUDA(mark(MOE_STAGE_EXPERT_GATE_UP, st), "stage event");
-    // one token: gate/up and down in one persistent kernel (the down stage
-    // then has zero length); otherwise one launch per projection
-    cudaError_t fe = rnx::launch_decode_experts(a, h, r, st);
-    if (fe == cudaErrorNotSupported) {
-      RNX_CUDA(rnx::launch_nvfp4_gemv(a, st), "expert gate/up");
-      RNX_CUDA(mark(MOE_STAGE_H_QUANT, st), "stage event");
-      a.proj = MOE_PROJ_DOWN; a.act = h; a.out = r; a.act_max = hmax; a.out_max = nullptr; a.prefetch_down = false;
-      RNX_CUDA(mark(MOE_STAGE_EXPERT_DOWN, st), "stage event");
-      RNX_CUDA(rnx::launch_nvfp4_gemv(a, st), "expert down");
-    } else {
-      RNX_CUDA(fe, "experts (fused gate/up + down)");
-      RNX_CUDA(mark(MOE_STAGE_H_QUANT, st), "stage event");
-      RNX_CUDA(mark(MOE_STAGE_EXPERT_DOWN, st), "stage event");
-    }
+    RNX_CUDA(rnx::launch_nvfp4_gemv(a, st), "expert gate/up");
+    RNX_CUDA(mark(MOE_STAGE_H_QUANT, st), "stage event");
+    a.proj = MOE_PROJ_DOWN; a.act = h; a.out = r; a.act_max = hmax; a.out_max = nullptr; a.prefetch_down = false;
+    RNX_CUDA(mark(MOE_STAGE_EXPERT_DOWN, st), "stage event");
+    RNX_CUDA(rnx::launch_nvfp4_gemv(a, st), "expert down");
   }
   RNX_CUDA(mark(MOE_STAGE_SHARED, st), "stage event");
   if (shared_aside) {

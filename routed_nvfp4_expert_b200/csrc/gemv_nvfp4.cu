@@ -28,18 +28,6 @@ namespace rnx {
 
 namespace {
 
-// Bounded wait (2 s) until *c >= need, acquire at gpu scope.
-RNX_DEVICE bool wait_counter(const int* c, int need) {
-  const unsigned long long t0 = globaltimer_ns();
-  for (;;) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(c) : "memory");
-    if (v >= need) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
-    __nanosleep(256);
-  }
-}
-
 constexpr int kGemvWarps = 8;
 constexpr int kGemvThreads = kGemvWarps * kWarp;
 
@@ -361,14 +349,10 @@ constexpr int kDirectWarps = 8;
 constexpr int kDirectRows = 8;        // weight rows per warp
 
 // One work item of the direct form: CTA_ROWS output rows (row block blk) of
-// expert e for its single assignment a. An item runs in two phases so that a
-// persistent CTA can issue the next item's weight loads before it finishes
-// the current one: item_loads() issues the 128-bit weight loads (8 rows per
-// warp: GATE_UP 4 gate then 4 up rows) into a register set, item_finish()
-// fetches the activation chunk, multiplies, reduces and stores. With `ready`
-// non-null (fused DOWN), item_finish first waits until *ready reaches `need`
-// (the expert's gate/up items are all done); a wait that runs out sets the
-// status word and the item is skipped.
+// expert e for its single assignment a, in two phases: item_loads() issues
+// the 128-bit weight loads (8 rows per warp: GATE_UP 4 gate then 4 up rows)
+// into a register set, item_finish() fetches the activation chunk,
+// multiplies, reduces and stores.
 struct ItemLoads {
   uint4 q[kDirectRows];
   uint16_t sv[kDirectRows];
@@ -409,11 +393,9 @@ RNX_DEVICE void item_loads(const GemvParams& p, int e, int blk, ItemLoads& L) {
 }
 
 template <int NI, bool GATE_UP>
-RNX_DEVICE bool item_finish(const GemvParams& p, int e, int a, int blk, const ItemLoads& L, float* s_part,
-                            const int* ready, int need) {
+RNX_DEVICE void item_finish(const GemvParams& p, int e, int a, int blk, const ItemLoads& L, float* s_part) {
   constexpr int RG = kDirectWarps / NI;                  // row groups per CTA
   constexpr int PAIRS = GATE_UP ? kDirectRows / 2 : 0;   // gate/up pairs per row group
-  __shared__ int s_ok;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kg = warp % NI, rg = warp / NI;
   const int row0 = blk * direct_cta_rows<NI, GATE_UP>();
@@ -421,16 +403,6 @@ RNX_DEVICE bool item_finish(const GemvParams& p, int e, int a, int blk, const It
   const bool lane_on = c < p.K / 32;
   const float ts0 = p.ts0[e], ts1 = GATE_UP ? p.ts1[e] : 0.f;
   const float wt = GATE_UP ? 0.f : p.weights[a];
-
-  if (ready) {
-    if (threadIdx.x == 0) {
-      const bool okw = wait_counter(ready, need);
-      if (!okw) set_status(p.status, kDevErrTimeout);
-      s_ok = okw ? 1 : 0;
-    }
-    __syncthreads();
-    if (!s_ok) return false;
-  }
 
   // this lane's 32-element activation chunk (x token for GATE_UP, h row for
   // DOWN) pre-scaled by the power of two that brings the row's max |a|
@@ -489,7 +461,6 @@ RNX_DEVICE bool item_finish(const GemvParams& p, int e, int a, int blk, const It
       }
     }
   }
-  return true;
 }
 
 template <int NI, bool GATE_UP>
@@ -504,338 +475,7 @@ nvfp4_gemv_direct_kernel(GemvParams p) {
   const int e = p.active[1 + u];
   ItemLoads L;
   item_loads<NI, GATE_UP>(p, e, blk, L);
-  item_finish<NI, GATE_UP>(p, e, p.first[u], blk, L, s_part, nullptr, 0);
-}
-
-// Gate/up and down of every active expert in one persistent kernel (one
-// token per expert), streaming the weights through shared memory.
-//
-// Work items: the gate/up blocks of each active expert (8 output features =
-// 8 gate + 8 up rows each) and its down blocks (64 output rows each); one
-// item is 36 KB of codes and scales at H = 4096, I = 1024. Items are numbered
-// in the order
-//   gu(0), gu(1), gu(2), gu(3), dn(0), gu(4), dn(1), ..., gu(n-1), dn(n-4), ..., dn(n-1)
-// (the down blocks of expert u follow the gate/up blocks of expert u + 3, so
-// that by the time they are taken their h is usually complete). CTA b owns
-// items b, b + G, b + 2G, ... (G = grid size) and deals them alternately to
-// its two pipelines.
-//
-// A pipeline is a producer warp, a 3-stage ring of shared memory and 8
-// compute warps. Two independent rings per SM keep HBM busier than one deeper
-// ring: a single producer that must wait for its oldest stage before reusing
-// it leaves the memory system idle whenever that stage is the slow one.
-//  * producer (one lane): copies each item's weight rows and block scales
-//    with bulk copies (TMA engine) into its ring.
-//  * compute warps: gate/up -- warp w owns feature w of the item (its gate and
-//    its up row over the whole K) and writes h = clamped SwiGLU itself; down
-//    -- warp w owns rows 8w .. 8w + 7 and writes r. A stage is released as
-//    soon as its bytes have been read.
-// h is the hand-off between the two projections. It is filled with an all-ones
-// pattern (a NaN that the gate/up writers never produce: they store a NaN as
-// the canonical one) before this kernel runs; a down warp reads its lane's
-// 32-element chunk of the assignment's h row from L2 until no element holds
-// the pattern. Every element is stored once, so an element read without the
-// pattern is final: no fence, counter or flag is needed. The warp then takes
-// the row's max |h| over its 32 lanes (the whole row when I <= 1024) for the
-// f16 pre-scale.
-// Every down item has a higher number than every gate/up item of its expert,
-// and each pipeline takes its items in increasing order, so every awaited
-// gate/up item is held by a pipeline that reaches it without waiting on the
-// awaiting one. All waits are bounded; a timeout sets the status word and
-// winds the CTA down.
-constexpr int kRings = 2;
-constexpr int kRingStages = 3;
-constexpr int kDownLag = 3;                              // dn(u) follows gu(u + kDownLag)
-constexpr int kStreamStageBytes = 36864;                 // codes + scales of one item
-constexpr int kStreamGroupWarps = 8;                     // compute warps per pipeline
-constexpr int kStreamCompute = kRings * kStreamGroupWarps;
-constexpr int kStreamProducer = kStreamCompute;          // + ring
-constexpr int kStreamThreads = (kStreamCompute + kRings) * 32;
-constexpr int kStreamSmem = kRings * kRingStages * kStreamStageBytes;   // + x (H f16)
-constexpr int kGuRowsItem = kStreamGroupWarps;           // output features per gate/up item
-constexpr int kDnRowsWarp = 8;                           // down rows per compute warp
-constexpr int kDnRowsItem = kDnRowsWarp * kStreamGroupWarps;   // output rows per down item
-constexpr int kStreamMaxH = 4096;
-constexpr int kStreamMaxI = 1024;
-constexpr int kMaxStreamExperts = 16;                    // one token: at most top_k active experts
-constexpr int kItemEnd = -1;
-constexpr uint32_t kHUnset = 0xFFFFFFFFu;                // two bf16 elements not yet written
-constexpr bool kStreamDisabled = true;
-
-// Item number -> packed (down << 30 | u << 16 | block) in the order above.
-// bpe_g / bpe_d: gate/up and down blocks per expert.
-RNX_DEVICE int stream_item(int item, int n_act, int bpe_g, int bpe_d) {
-  const int lead = min(kDownLag, n_act);                 // gate/up-only steps
-  const int both = n_act - lead;                         // steps with gu(j + lag) then dn(j)
-  if (item < lead * bpe_g) return ((item / bpe_g) << 16) | (item % bpe_g);
-  item -= lead * bpe_g;
-  const int step = bpe_g + bpe_d;
-  if (item < both * step) {
-    const int j = item / step, r = item - j * step;
-    return r < bpe_g ? (((lead + j) << 16) | r) : ((1 << 30) | (j << 16) | (r - bpe_g));
-  }
-  item -= both * step;                                   // trailing down blocks
-  const int j = both + item / bpe_d;
-  return (1 << 30) | (j << 16) | (item % bpe_d);
-}
-
-// The lane's 32-element h chunk (16 bf16 pairs) read from L2; with `wait`, a
-// bounded wait until no element of the warp's chunks is unset (polling with
-// a growing pause, so that waiting warps do not crowd the memory pipeline of
-// the SM). Lanes past the row read nothing.
-RNX_DEVICE bool load_h_chunk(const uint16_t* hrow, int c, bool on, bool wait, uint32_t (&hv)[16]) {
-  const uint4* p = reinterpret_cast<const uint4*>(hrow + 32 * c);
-  const unsigned long long t0 = globaltimer_ns();
-  for (uint32_t pause = 128;; pause = min(2u * pause, 1024u)) {
-    bool ready = true;
-    if (on) {
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint4 v;
-        asm volatile("ld.relaxed.gpu.global.v4.u32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                     : "l"(p + q)
-                     : "memory");
-        hv[4 * q] = v.x; hv[4 * q + 1] = v.y; hv[4 * q + 2] = v.z; hv[4 * q + 3] = v.w;
-      }
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        // an element is unset iff its 16 bits are all ones
-        ready = ready && (hv[j] & 0xFFFFu) != 0xFFFFu && (hv[j] >> 16) != 0xFFFFu;
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < 16; ++j) hv[j] = 0u;
-    }
-    if (!wait || __all_sync(0xffffffffu, ready)) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
-    __nanosleep(pause);
-  }
-}
-
-// Bounded wait (2 s) until the shared int *v >= need (acquire at CTA scope).
-RNX_DEVICE bool wait_shared_at_least(const int* v, int need) {
-  const unsigned long long t0 = globaltimer_ns();
-  for (;;) {
-    int x;
-    asm volatile("ld.acquire.cta.shared.b32 %0, [%1];" : "=r"(x) : "r"(smem_u32(v)) : "memory");
-    if (x >= need) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
-    __nanosleep(32);
-  }
-}
-
-__global__ void __launch_bounds__(kStreamThreads, 1)
-nvfp4_experts_stream_kernel(GemvParams gu, GemvParams dn) {
-  extern __shared__ __align__(128) uint8_t s_dyn[];
-  uint4* s_x = reinterpret_cast<uint4*>(s_dyn + kStreamSmem);            // x as f16, [4][H/32]
-  __shared__ __align__(8) uint64_t full_bar[kRings][kRingStages], empty_bar[kRings][kRingStages];
-  __shared__ int s_item[kRings][kRingStages];            // packed item of each stage, kItemEnd = end
-  __shared__ int s_hseen[kRings];                        // down items whose h row warp 0 found complete
-  __shared__ int s_e[kMaxStreamExperts], s_a[kMaxStreamExperts], s_n;
-  __shared__ float s_tg[kMaxStreamExperts], s_tu[kMaxStreamExperts], s_td[kMaxStreamExperts],
-      s_wt[kMaxStreamExperts];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int H = gu.K, I = gu.rows;
-  const int nchG = H / 32, nchD = I / 32;
-  const int gu_row_bytes = H / 2, gu_sc_bytes = H / 16, dn_row_bytes = I / 2, dn_sc_bytes = I / 16;
-
-  if (tid == 0) {
-    for (int g = 0; g < kRings; ++g) s_hseen[g] = 0;
-    for (int g = 0; g < kRings; ++g)
-      for (int i = 0; i < kRingStages; ++i) {
-        mbar_init(&full_bar[g][i], 1);
-        mbar_init(&empty_bar[g][i], kStreamGroupWarps);    // the compute warps, after reading
-      }
-    fence_barrier_init();
-  }
-  pdl_wait();       // follows the routing plan
-  pdl_trigger();
-  // the active experts, their assignment, tensor scales and routing weight
-  if (tid == 0) s_n = min(gu.active[0], kMaxStreamExperts);
-  __syncthreads();
-  const int n_act = s_n;
-  for (int u = tid; u < n_act; u += blockDim.x) {
-    const int e = gu.active[1 + u], a = gu.first[u];
-    s_e[u] = e;
-    s_a[u] = a;
-    s_tg[u] = gu.ts0[e];
-    s_tu[u] = gu.ts1[e];
-    s_td[u] = dn.ts0[e];
-    s_wt[u] = dn.weights[a];
-  }
-  __syncthreads();
-  const int bpe_g = I / kGuRowsItem, bpe_d = H / kDnRowsItem;
-  const int n_all = n_act * (bpe_g + bpe_d);
-  const uint32_t gcb = kGuRowsItem * gu_row_bytes, gsb = kGuRowsItem * gu_sc_bytes;
-  const uint32_t dcb = kDnRowsItem * dn_row_bytes, dsb = kDnRowsItem * dn_sc_bytes;
-  // this CTA's items for pipeline g: blockIdx.x + (2j + g) * G, j = 0, 1, ...
-  const int item_step = kRings * gridDim.x;
-
-  if (warp >= kStreamProducer) {
-    // ------------------------------------------------------------ producer
-    const int g = warp - kStreamProducer;
-    uint8_t* ring = s_dyn + (size_t)g * kRingStages * kStreamStageBytes;
-    if (lane == 0) {
-      const uint64_t pol = policy_evict_first();
-      int it = 0;
-      for (int item = blockIdx.x + g * gridDim.x;; item += item_step, ++it) {
-        const int s = it % kRingStages;
-        const uint32_t ph = (uint32_t)(it / kRingStages) & 1u;
-        const bool free_ok = mbar_wait(&empty_bar[g][s], ph ^ 1u);
-        if (!free_ok) set_status(gu.status, kDevErrTimeout);
-        if (!free_ok || item >= n_all) {
-          s_item[g][s] = kItemEnd;         // end of work (or abort) for the compute warps
-          mbar_arrive(&full_bar[g][s]);
-          ++it;
-          break;
-        }
-        const int pk = stream_item(item, n_act, bpe_g, bpe_d);
-        const int u = (pk >> 16) & 0x3FFF, blk = pk & 0xFFFF;
-        s_item[g][s] = pk;
-        uint8_t* st = ring + (size_t)s * kStreamStageBytes;
-        if (!(pk >> 30)) {
-          const size_t gr = (size_t)s_e[u] * I + blk * kGuRowsItem;
-          mbar_arrive_expect_tx(&full_bar[g][s], 2 * (gcb + gsb));
-          bulk_g2s(st, gu.codes0 + gr * gu_row_bytes, gcb, &full_bar[g][s], pol);
-          bulk_g2s(st + gcb, gu.codes1 + gr * gu_row_bytes, gcb, &full_bar[g][s], pol);
-          bulk_g2s(st + 2 * gcb, gu.scales0 + gr * gu_sc_bytes, gsb, &full_bar[g][s], pol);
-          bulk_g2s(st + 2 * gcb + gsb, gu.scales1 + gr * gu_sc_bytes, gsb, &full_bar[g][s], pol);
-        } else {
-          const size_t gr = (size_t)s_e[u] * H + blk * kDnRowsItem;
-          mbar_arrive_expect_tx(&full_bar[g][s], dcb + dsb);
-          bulk_g2s(st, dn.codes0 + gr * dn_row_bytes, dcb, &full_bar[g][s], pol);
-          bulk_g2s(st + dcb, dn.scales0 + gr * dn_sc_bytes, dsb, &full_bar[g][s], pol);
-        }
-      }
-      // copies in flight must land before the CTA may exit
-      for (int j = max(0, it - kRingStages); j < it; ++j)
-        if (!mbar_wait(&full_bar[g][j % kRingStages], (uint32_t)(j / kRingStages) & 1u))
-          set_status(gu.status, kDevErrTimeout);
-    }
-    return;
-  }
-
-  // -------------------------------------------------------------- compute warps
-  // the token's x (one token: every gate/up item uses it), pre-scaled to f16
-  float x_up, x_unscale;
-  prescale_from_max(__uint_as_float(gu.act_max[0]), x_up, x_unscale);
-  for (int cq = tid; cq < nchG * 4; cq += kStreamCompute * 32) {
-    const int c = cq >> 2, q = cq & 3;
-    const uint4 v = *reinterpret_cast<const uint4*>(gu.act + 32 * c + 8 * q);
-    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-    uint32_t o[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 f = bf16x2_to_f32x2(w4[j]);
-      __half2 h2 = __floats2half2_rn(f.x * x_up, f.y * x_up);
-      o[j] = *reinterpret_cast<uint32_t*>(&h2);
-    }
-    s_x[q * nchG + c] = make_uint4(o[0], o[1], o[2], o[3]);
-  }
-  asm volatile("bar.sync 1, %0;" ::"n"(kStreamCompute * 32) : "memory");
-
-  const int g = warp / kStreamGroupWarps, gw = warp % kStreamGroupWarps;
-  const uint8_t* ring = s_dyn + (size_t)g * kRingStages * kStreamStageBytes;
-  int ndn = 0;                              // down items taken by this pipeline
-  for (int it = 0;; ++it) {
-    const int s = it % kRingStages;
-    const uint32_t ph = (uint32_t)(it / kRingStages) & 1u;
-    if (__any_sync(0xffffffffu, !mbar_wait(&full_bar[g][s], ph))) {
-      if (lane == 0) set_status(gu.status, kDevErrTimeout);
-      break;
-    }
-    const int pk = s_item[g][s];
-    if (pk == kItemEnd) break;
-    const int u = (pk >> 16) & 0x3FFF, blk = pk & 0xFFFF, a = s_a[u];
-    const uint8_t* st = ring + (size_t)s * kStreamStageBytes;
-    if (!(pk >> 30)) {
-      // gate/up: this warp's feature, gate row gw and up row gw of the item
-      const int f = blk * kGuRowsItem + gw;
-      const uint8_t* cg = st + gw * gu_row_bytes;
-      const uint8_t* cu = st + gcb + gw * gu_row_bytes;
-      const uint8_t* sg = st + 2 * gcb + gw * gu_sc_bytes;
-      const uint8_t* su = sg + gsb;
-      float acc[2] = {0.f, 0.f};
-      for (int c = lane; c < nchG; c += 32) {
-        uint32_t xr[16];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint4 v = s_x[q * nchG + c];
-          xr[4 * q] = v.x; xr[4 * q + 1] = v.y; xr[4 * q + 2] = v.z; xr[4 * q + 3] = v.w;
-        }
-        uint32_t w[16];
-        decode_chunk(*reinterpret_cast<const uint4*>(cg + 16 * c), w);
-        chunk_fma(w, xr, e4m3x2_to_f32x2(*reinterpret_cast<const uint16_t*>(sg + 2 * c)), acc[0]);
-        decode_chunk(*reinterpret_cast<const uint4*>(cu + 16 * c), w);
-        chunk_fma(w, xr, e4m3x2_to_f32x2(*reinterpret_cast<const uint16_t*>(su + 2 * c)), acc[1]);
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty_bar[g][s]);   // stage read
-      const float tot = warp_reduce_rows<2>(acc);      // lanes 0-15: gate, 16-31: up
-      const float upv = __shfl_sync(0xffffffffu, tot, 16);
-      if (lane == 0) {
-        const float gt = tot * x_unscale * s_tg[u], uu = upv * x_unscale * s_tu[u];
-        uint16_t hb = f32_to_bf16_bits(clamped_swiglu(gt, uu, gu.limit));
-        if ((hb & 0x7FFFu) > 0x7F80u) hb = 0x7FC0u;     // any NaN as the canonical one
-        asm volatile("st.relaxed.gpu.global.b16 [%0], %1;" ::"l"(gu.out + (size_t)a * I + f), "h"(hb) : "memory");
-      }
-    } else {
-      // down: rows 8 gw .. 8 gw + 7 of the item, lane c chunk c of h. Warp 0
-      // of the pipeline waits until the row is complete; the others then read
-      // it once (each element is stored once, so what warp 0 saw is final)
-      const int row0 = blk * kDnRowsItem + gw * kDnRowsWarp;
-      uint32_t hv[16];
-      const bool lane_on = lane < nchD;
-      const uint16_t* hrow = dn.act + (size_t)a * I;
-      if (gw == 0) {
-        if (!load_h_chunk(hrow, lane, lane_on, true, hv) && lane == 0) set_status(gu.status, kDevErrTimeout);
-        __syncwarp();
-        if (lane == 0) asm volatile("st.release.cta.shared.b32 [%0], %1;" ::"r"(smem_u32(&s_hseen[g])), "r"(ndn + 1) : "memory");
-      } else {
-        if (lane == 0 && !wait_shared_at_least(&s_hseen[g], ndn + 1)) set_status(gu.status, kDevErrTimeout);
-        __syncwarp();
-        load_h_chunk(hrow, lane, lane_on, false, hv);
-      }
-      ++ndn;
-      float mx = 0.f;
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const float2 f = bf16x2_to_f32x2(hv[j]);
-        mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
-      }
-      mx = warp_max(mx);
-      float up, unscale;
-      prescale_from_max(mx, up, unscale);
-      uint32_t xr[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const float2 f = bf16x2_to_f32x2(hv[j]);
-        __half2 h2 = __floats2half2_rn(f.x * up, f.y * up);
-        xr[j] = *reinterpret_cast<uint32_t*>(&h2);
-      }
-      const uint8_t* cb = st + gw * kDnRowsWarp * dn_row_bytes;
-      const uint8_t* sb = st + dcb + gw * kDnRowsWarp * dn_sc_bytes;
-      float acc[kDnRowsWarp];
-#pragma unroll
-      for (int r = 0; r < kDnRowsWarp; ++r) acc[r] = 0.f;
-      if (lane_on) {
-#pragma unroll
-        for (int r = 0; r < kDnRowsWarp; ++r) {
-          const uint4 qv = *reinterpret_cast<const uint4*>(cb + r * dn_row_bytes + 16 * lane);
-          const uint16_t sv = *reinterpret_cast<const uint16_t*>(sb + r * dn_sc_bytes + 2 * lane);
-          uint32_t w[16];
-          decode_chunk(qv, w);
-          chunk_fma(w, xr, e4m3x2_to_f32x2(sv), acc[r]);
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty_bar[g][s]);   // stage read
-      const float tot = warp_reduce_rows<kDnRowsWarp>(acc);   // lane 4r holds row r
-      if ((lane & 3) == 0)
-        dn.out[(size_t)a * H + row0 + (lane >> 2)] = f32_to_bf16_bits(tot * unscale * s_td[u] * s_wt[u]);
-    }
-  }
+  item_finish<NI, GATE_UP>(p, e, p.first[u], blk, L, s_part);
 }
 
 // remote assignments of the DOWN projection contribute zero rows
@@ -923,35 +563,6 @@ GemvParams gemv_params(const ExpertGemvArgs& a, bool gu) {
 
 }  // namespace
 
-cudaError_t launch_decode_experts(const ExpertGemvArgs& a, uint16_t* h, uint16_t* r, cudaStream_t st) {
-  // one token; an item's rows (16 x H/2 + 16 x H/16 and 64 x I/2 + 64 x I/16
-  // bytes) fit one 36 KB stage, and one warp's lanes cover an h row (I <= 1024)
-  // measured slower than the two direct GEMV launches on B200 (the down
-  // blocks wait several microseconds for h under full HBM load): not taken
-  if (kStreamDisabled || a.T != 1 || !a.act_max || a.H > kStreamMaxH || a.I > kStreamMaxI || a.H % kDnRowsItem ||
-      a.I % kGuRowsItem || a.I % 32)
-    return cudaErrorNotSupported;
-  ExpertGemvArgs g = a, d = a;
-  g.proj = MOE_PROJ_GATE_UP; g.act = a.act; g.out = h; g.out_max = nullptr;
-  d.proj = MOE_PROJ_DOWN; d.act = h; d.out = r; d.act_max = nullptr; d.out_max = nullptr;
-  const GemvParams pg = gemv_params(g, true), pd = gemv_params(d, false);
-  const int max_active = std::min(a.local_end - a.local_begin, a.T * a.k);
-  const bool remote = a.local_begin > 0 || a.local_end < a.E;
-  const size_t smem = (size_t)kStreamSmem + (size_t)a.H * 2;
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaError_t err = cudaFuncSetAttribute(nvfp4_experts_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)((size_t)kStreamSmem + kStreamMaxH * 2));
-    if (err != cudaSuccess) return err;
-    attr_done = true;
-  }
-  const int items = max_active * (a.I / kGuRowsItem + a.H / kDnRowsItem);
-  const int grid = std::max(1, std::min((items + kRings - 1) / kRings, kNumSMs));
-  cudaError_t err = launch_pdl(nvfp4_experts_stream_kernel, dim3(grid), dim3(kStreamThreads), smem, st, pg, pd);
-  if (err != cudaSuccess || !remote) return err;
-  zero_remote_rows<<<kNumSMs, 256, 0, st>>>(pd);
-  return cudaGetLastError();
-}
 
 cudaError_t launch_nvfp4_gemv(const ExpertGemvArgs& a, cudaStream_t st) {
   const bool gu = a.proj == MOE_PROJ_GATE_UP;

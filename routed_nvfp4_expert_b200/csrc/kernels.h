@@ -49,20 +49,12 @@ struct ExpertGemvArgs {
 
 cudaError_t launch_nvfp4_gemv(const ExpertGemvArgs& a, cudaStream_t st);
 
-// One token per expert (T = 1): gate/up and down of every active expert in one
-// persistent kernel. h [k, I] receives the gate/up output and must hold all
-// ones (every bit set) when the kernel starts; r [k, H] receives the down
-// output. Returns cudaErrorNotSupported when the shape is outside this form.
-cudaError_t launch_decode_experts(const ExpertGemvArgs& a, uint16_t* h, uint16_t* r, cudaStream_t st);
-
 // router
 // xmax (nullable): receives max |x_t| per token as fp32 bits; zero (nullable):
-// nzero uint32 words set to 0 (the h-max array of the next expert pass);
-// fill (nullable): nfill uint32 words set to all ones (the h of the one-token
-// experts kernel). The side jobs run only in the GEMV form (T <= 64).
+// nzero uint32 words set to 0 (the h-max array of the next expert pass). The
+// side jobs run only in the GEMV form (T <= 64).
 cudaError_t launch_router_logits(const uint16_t* x, int T, int H, int E, const float* wr, float* logits,
-                                 cudaStream_t st, uint32_t* xmax = nullptr, uint32_t* zero = nullptr, int nzero = 0,
-                                 uint32_t* fill = nullptr, int nfill = 0);
+                                 cudaStream_t st, uint32_t* xmax = nullptr, uint32_t* zero = nullptr, int nzero = 0);
 // max |row| as fp32 bits for R rows of K bf16 elements
 cudaError_t launch_row_absmax(const uint16_t* rows, int R, int K, uint32_t* out, cudaStream_t st);
 cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, int k, float rsf, int32_t* ids,

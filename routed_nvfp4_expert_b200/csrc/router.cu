@@ -22,8 +22,7 @@ constexpr int kLogitMaxQ = 16;     // H <= 8192 in this form
 __global__ void __launch_bounds__(kLogitThreads) router_logits_gemv(const uint16_t* __restrict__ x, int T, int H, int E,
                                                                    const float* __restrict__ wr,
                                                                    float* __restrict__ logits, uint32_t* xmax,
-                                                                   uint32_t* zero, int nzero, uint32_t* fill,
-                                                                   int nfill) {
+                                                                   uint32_t* zero, int nzero) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int e = blockIdx.x;
   const int nq = H >> 2;
@@ -38,9 +37,6 @@ __global__ void __launch_bounds__(kLogitThreads) router_logits_gemv(const uint16
   }
   pdl_wait();
   pdl_trigger();
-  // side job of every CTA: the words to set to all ones (the "not yet
-  // written" pattern of the decode experts kernel's h)
-  for (int i = e * kLogitThreads + tid; i < nfill; i += E * kLogitThreads) fill[i] = 0xFFFFFFFFu;
   if (e == 0) {
     // side jobs of CTA 0: max |x_t| per token (fp32 bits; the expert pass
     // pre-scales with it) and clearing the h-max array the gate/up pass fills
@@ -269,11 +265,10 @@ cudaError_t launch_row_absmax(const uint16_t* rows, int R, int K, uint32_t* out,
 }
 
 cudaError_t launch_router_logits(const uint16_t* x, int T, int H, int E, const float* wr, float* logits,
-                                 cudaStream_t st, uint32_t* xmax, uint32_t* zero, int nzero, uint32_t* fill,
-                                 int nfill) {
+                                 cudaStream_t st, uint32_t* xmax, uint32_t* zero, int nzero) {
   if (T <= 64 && H <= 4 * kLogitThreads * kLogitMaxQ) {
     return launch_pdl(router_logits_gemv, dim3(E), dim3(kLogitThreads), 0, st, x, T, H, E, wr, logits, xmax, zero,
-                      nzero, fill, nfill);
+                      nzero);
   } else {
     dim3 grid((E + kSgBN - 1) / kSgBN, (T + kSgBM - 1) / kSgBM);
     router_logits_sgemm<<<grid, 256, 0, st>>>(x, T, H, E, wr, logits);
