@@ -347,6 +347,10 @@ RNX_DEVICE float warp_reduce_rows(float (&v)[N]) {
 // exact and order-independent) for the DOWN pass.
 constexpr int kDirectWarps = 8;
 constexpr int kDirectRows = 8;        // weight rows per warp
+// 64 registers a thread (no spills): 4 CTAs (32 warps) per SM keep more weight
+// loads in flight, and the down pass (512 CTAs for 8 experts at H = 4096)
+// fits one wave of 4 x 148 CTAs instead of leaving a second, almost empty one
+constexpr int kDirectCtasPerSm = 4;
 
 // One work item of the direct form: CTA_ROWS output rows (row block blk) of
 // expert e for its single assignment a, in two phases: item_loads() issues
@@ -464,7 +468,7 @@ RNX_DEVICE void item_finish(const GemvParams& p, int e, int a, int blk, const It
 }
 
 template <int NI, bool GATE_UP>
-__global__ void __launch_bounds__(kDirectWarps * kWarp, 3)
+__global__ void __launch_bounds__(kDirectWarps * kWarp, kDirectCtasPerSm)
 nvfp4_gemv_direct_kernel(GemvParams p) {
   __shared__ float s_part[kDirectWarps * kDirectRows];
   const int bpe = (p.rows + direct_cta_rows<NI, GATE_UP>() - 1) / direct_cta_rows<NI, GATE_UP>();
