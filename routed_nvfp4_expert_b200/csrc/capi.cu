@@ -673,11 +673,22 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
     RNX_CUDA(rnx::launch_router_logits(x, T, H, E, w->router_w, logits, st, xmax, hmax, T * k), "router logits");
   }
   RNX_CUDA(mark(MOE_STAGE_TOPK, st), "stage event");
-  RNX_CUDA(rnx::launch_topk(logits, w->router_bias, T, E, k, cfg->routed_scaling_factor, ids, wts, st), "top-k");
-  RNX_CUDA(mark(MOE_STAGE_PERMUTE, st), "stage event");
-  RNX_CUDA(rnx::launch_permute(ids, T * k, E, cfg->local_begin, cfg->local_end, plan, (int32_t*)(b + L.scratch),
-                               status, st),
-           "permute");
+  // decode with a handful of tokens: selection and plan in one launch (the
+  // permute stage then has zero length)
+  cudaError_t fp = cudaErrorNotSupported;
+  if (path == MOE_PATH_DECODE)
+    fp = rnx::launch_topk_plan(logits, w->router_bias, T, E, k, cfg->routed_scaling_factor, ids, wts,
+                               cfg->local_begin, cfg->local_end, plan, status, st);
+  if (fp == cudaErrorNotSupported) {
+    RNX_CUDA(rnx::launch_topk(logits, w->router_bias, T, E, k, cfg->routed_scaling_factor, ids, wts, st), "top-k");
+    RNX_CUDA(mark(MOE_STAGE_PERMUTE, st), "stage event");
+    RNX_CUDA(rnx::launch_permute(ids, T * k, E, cfg->local_begin, cfg->local_end, plan, (int32_t*)(b + L.scratch),
+                                 status, st),
+             "permute");
+  } else {
+    RNX_CUDA(fp, "top-k + plan");
+    RNX_CUDA(mark(MOE_STAGE_PERMUTE, st), "stage event");
+  }
   RNX_CUDA(mark(MOE_STAGE_ACT_QUANT, st), "stage event");
   if (path == MOE_PATH_PREFILL) {
     const int64_t P = L.pl.P;

@@ -59,6 +59,11 @@ cudaError_t launch_router_logits(const uint16_t* x, int T, int H, int E, const f
 cudaError_t launch_row_absmax(const uint16_t* rows, int R, int K, uint32_t* out, cudaStream_t st);
 cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, int k, float rsf, int32_t* ids,
                         float* weights, cudaStream_t st);
+// Top-k and the routing plan in one launch when the tokens fit one top-k CTA
+// (T <= 8) and E <= 320, T*k <= 1024; else cudaErrorNotSupported.
+cudaError_t launch_topk_plan(const float* logits, const float* bias, int T, int E, int k, float rsf, int32_t* ids,
+                             float* weights, int lb, int le, const moe_plan_t& plan, uint32_t* status,
+                             cudaStream_t st);
 
 // permutation; scratch is int32 workspace of permute_scratch_ints(T*k, E) entries
 size_t permute_scratch_ints(int A, int E);

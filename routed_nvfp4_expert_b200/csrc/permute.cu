@@ -1,7 +1,7 @@
 // Token sort (glm5next_mlp module docs, MOE_MODULE: the token sort /
 // permute / unpermute family): the A = T*k assignments a = t*k + j are
 // grouped by expert, stably, with counts, offsets, the inverse map, per-expert
-// 128-row tile offsets (local experts only) and the list of active local
+// 256-row tile offsets (local experts only) and the list of active local
 // experts.
 //
 // Small A (decode): one CTA does everything in shared memory.
@@ -10,86 +10,13 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "small_plan.cuh"
 
 namespace rnx {
 
 namespace {
 
-constexpr int kSmallMaxA = 1024;
-constexpr int kMaxE = 1024;
 constexpr int kChunk = 256;   // assignments per histogram block
-
-// Block-wide exclusive scan of up to blockDim.x (multiple of 32, <= 1024)
-// values, one per thread; returns the exclusive prefix, *total gets the sum.
-RNX_DEVICE int block_exclusive_scan(int v, int* s_warp, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  int inc = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int n = __shfl_up_sync(0xffffffffu, inc, o);
-    if (lane >= o) inc += n;
-  }
-  __syncthreads();
-  if (lane == 31) s_warp[warp] = inc;
-  __syncthreads();
-  if (warp == 0) {
-    int w = lane < nw ? s_warp[lane] : 0;
-    int wi = w;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int n = __shfl_up_sync(0xffffffffu, wi, o);
-      if (lane >= o) wi += n;
-    }
-    if (lane < nw) s_warp[lane] = wi - w;
-    if (lane == 31) s_warp[32] = wi;
-  }
-  __syncthreads();
-  const int res = inc - v + s_warp[warp];
-  if (total) *total = s_warp[32];
-  __syncthreads();
-  return res;
-}
-
-// counts -> offsets, tile_offsets, active (one CTA of 1024 threads, E <= 1024)
-RNX_DEVICE void finish_plan(const int* s_cnt, int E, int lb, int le, const moe_plan_t& plan, int* s_warp) {
-  const int e = threadIdx.x;
-  const int c = e < E ? s_cnt[e] : 0;
-  const bool local = e >= lb && e < le;
-  int tot;
-  const int off = block_exclusive_scan(c, s_warp, &tot);
-  const int tiles = (local && e < E) ? (c + kRowsPerTile - 1) / kRowsPerTile : 0;
-  int ttot;
-  const int toff = block_exclusive_scan(tiles, s_warp, &ttot);
-  const int act = (local && e < E && c > 0) ? 1 : 0;
-  int atot;
-  const int aoff = block_exclusive_scan(act, s_warp, &atot);
-  if (e < E) {
-    plan.counts[e] = c;
-    plan.offsets[e] = off;
-    plan.tile_offsets[e] = toff;
-    if (act) plan.active[1 + aoff] = e;
-  }
-  if (e == 0) {
-    plan.offsets[E] = tot;
-    plan.tile_offsets[E] = ttot;
-    plan.active[0] = atot;
-  }
-}
-
-// first[u] = sorted[offsets[e]] for the u-th active (local, non-empty) expert e.
-// Runs after sorted[] is complete; reads offsets/active/sorted from the plan.
-RNX_DEVICE void write_first(const moe_plan_t& plan, const int* s_off, const int* s_cnt, int E, int lb, int le) {
-  const int n_active = plan.active[0];
-  for (int u = threadIdx.x; u < n_active; u += blockDim.x) {
-    const int e = plan.active[1 + u];
-    plan.first[u] = plan.sorted[plan.offsets[e]];
-  }
-  (void)s_off;
-  (void)s_cnt;
-  (void)E;
-  (void)lb;
-  (void)le;
-}
 
 __global__ void __launch_bounds__(1024) permute_small(const int32_t* __restrict__ ids, int A, int E, int lb, int le,
                                                       moe_plan_t plan, uint32_t* status) {
@@ -99,42 +26,7 @@ __global__ void __launch_bounds__(1024) permute_small(const int32_t* __restrict_
   __shared__ int s_warp[33];
   pdl_wait();
   pdl_trigger();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) s_cnt[e] = 0;
-  __syncthreads();
-  for (int a = threadIdx.x; a < A; a += blockDim.x) {
-    int e = ids[a];
-    if (e < 0 || e >= E) {
-      set_status(status, kDevErrBounds);
-      e = -1;
-    } else {
-      atomicAdd(&s_cnt[e], 1);
-    }
-    s_ids[a] = e;
-  }
-  __syncthreads();
-  finish_plan(s_cnt, E, lb, le, plan, s_warp);
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) s_off[e] = plan.offsets[e];
-  __syncthreads();
-  // stable position: offset + number of earlier assignments of the same expert
-  for (int a0 = 0; a0 < A; a0 += blockDim.x) {
-    const int a = a0 + threadIdx.x;
-    const int e = a < A ? s_ids[a] : -1;
-    int rank = 0;
-    const int lim = min(A, a0 + (int)blockDim.x);
-    for (int b = 0; b < lim; ++b) rank += (b < a && s_ids[b] == e) ? 1 : 0;
-    if (a < A) {
-      if (e >= 0) {
-        const int pos = s_off[e] + rank;
-        plan.sorted[pos] = a;
-        plan.inv[a] = pos;
-      } else {
-        plan.inv[a] = -1;
-      }
-    }
-  }
-  __syncthreads();
-  write_first(plan, s_off, s_cnt, E, lb, le);
+  small_plan(ids, A, E, lb, le, plan, status, s_ids, s_cnt, s_off, s_warp);
 }
 
 // ---- large A

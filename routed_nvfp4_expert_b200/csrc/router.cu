@@ -4,6 +4,7 @@
 // "Test Coverage": the gate is fp32).
 
 #include "common.cuh"
+#include "small_plan.cuh"
 #include "kernels.h"
 
 namespace rnx {
@@ -162,18 +163,11 @@ RNX_DEVICE bool better(const Cand& a, const Cand& b) {
 template <int PL>
 __host__ __device__ constexpr int topk_tokens() { return PL > 16 ? 2 : 8; }
 
-template <int PL>
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
-                                                   int T, int E, int k, float rsf, int32_t* __restrict__ ids,
-                                                   float* __restrict__ weights) {
-  constexpr int kTopkTokens = topk_tokens<PL>();
-  __shared__ float s_key[kTopkTokens][32 * PL];
-  __shared__ float s_sig[kTopkTokens][32 * PL];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  pdl_wait();
-  pdl_trigger();
-  const int t0 = blockIdx.x * kTopkTokens;
-  const int ntok = min(kTopkTokens, T - t0);
+// Sigmoid scores and selection keys of ntok tokens (from token t0) into
+// shared memory, by all threads of the CTA.
+template <int PL, int NT>
+RNX_DEVICE void topk_keys(const float* __restrict__ logits, const float* __restrict__ bias, int t0, int ntok, int E,
+                          float (&s_key)[NT][32 * PL], float (&s_sig)[NT][32 * PL]) {
   for (int i = threadIdx.x; i < ntok * E; i += blockDim.x) {
     const int tt = i / E, e = i - tt * E;
     const float l = logits[(size_t)(t0 + tt) * E + e];
@@ -182,17 +176,21 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
     s_sig[tt][e] = sg;
     s_key[tt][e] = __fadd_rn(sg, bias[e]);
   }
-  __syncthreads();
-  if (warp >= ntok) return;
-  const int t = t0 + warp;
+}
+
+// One warp selects token t's top-k from its keys and writes ids / weights.
+template <int PL>
+RNX_DEVICE void topk_warp(const float* s_key_row, const float* s_sig_row, int t, int E, int k, float rsf,
+                          int32_t* __restrict__ ids, float* __restrict__ weights) {
+  const int lane = threadIdx.x & 31;
   float key[PL], sg[PL];
   int st[PL];
 #pragma unroll
   for (int i = 0; i < PL; ++i) {
     const int e = lane + 32 * i;
     if (e < E) {
-      key[i] = s_key[warp][e];
-      sg[i] = s_sig[warp][e];
+      key[i] = s_key_row[e];
+      sg[i] = s_sig_row[e];
       st[i] = isnan(key[i]) ? 1 : 0;
     } else {
       sg[i] = 0.f;
@@ -238,6 +236,48 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
   }
 }
 
+template <int PL>
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
+                                                   int T, int E, int k, float rsf, int32_t* __restrict__ ids,
+                                                   float* __restrict__ weights) {
+  constexpr int kTopkTokens = topk_tokens<PL>();
+  __shared__ float s_key[kTopkTokens][32 * PL];
+  __shared__ float s_sig[kTopkTokens][32 * PL];
+  const int warp = threadIdx.x >> 5;
+  pdl_wait();
+  pdl_trigger();
+  const int t0 = blockIdx.x * kTopkTokens;
+  const int ntok = min(kTopkTokens, T - t0);
+  topk_keys<PL>(logits, bias, t0, ntok, E, s_key, s_sig);
+  __syncthreads();
+  if (warp < ntok) topk_warp<PL>(s_key[warp], s_sig[warp], t0 + warp, E, k, rsf, ids, weights);
+}
+
+// Decode with one top-k CTA's worth of tokens: selection and the routing plan
+// in one launch (1024 threads): the warps of the tokens select, then the whole
+// CTA builds the plan from the ids it has just written.
+template <int PL>
+__global__ void __launch_bounds__(1024) topk_plan_kernel(const float* __restrict__ logits,
+                                                         const float* __restrict__ bias, int T, int E, int k, float rsf,
+                                                         int32_t* ids, float* __restrict__ weights, int lb, int le,
+                                                         moe_plan_t plan, uint32_t* status) {
+  constexpr int kTopkTokens = topk_tokens<PL>();
+  __shared__ float s_key[kTopkTokens][32 * PL];
+  __shared__ float s_sig[kTopkTokens][32 * PL];
+  __shared__ int s_ids[kSmallMaxA];
+  __shared__ int s_cnt[kMaxE];
+  __shared__ int s_off[kMaxE];
+  __shared__ int s_warp[33];
+  const int warp = threadIdx.x >> 5;
+  pdl_wait();
+  pdl_trigger();
+  topk_keys<PL>(logits, bias, 0, T, E, s_key, s_sig);
+  __syncthreads();
+  if (warp < T) topk_warp<PL>(s_key[warp], s_sig[warp], warp, E, k, rsf, ids, weights);
+  __syncthreads();                       // the ids, for every thread of the CTA
+  small_plan(ids, T * k, E, lb, le, plan, status, s_ids, s_cnt, s_off, s_warp);
+}
+
 __global__ void __launch_bounds__(256) row_absmax_kernel(const uint16_t* __restrict__ rows, int R, int K,
                                                          uint32_t* __restrict__ out) {
   const int lane = threadIdx.x & 31;
@@ -274,6 +314,19 @@ cudaError_t launch_router_logits(const uint16_t* x, int T, int H, int E, const f
     router_logits_sgemm<<<grid, 256, 0, st>>>(x, T, H, E, wr, logits);
   }
   return cudaGetLastError();
+}
+
+cudaError_t launch_topk_plan(const float* logits, const float* bias, int T, int E, int k, float rsf, int32_t* ids,
+                             float* weights, int lb, int le, const moe_plan_t& plan, uint32_t* status,
+                             cudaStream_t st) {
+  if (T < 1 || T * k > kSmallMaxA || E > kMaxE) return cudaErrorNotSupported;
+  if (E <= 32 * 4 && T <= topk_tokens<4>())
+    return launch_pdl(topk_plan_kernel<4>, dim3(1), dim3(1024), 0, st, logits, bias, T, E, k, rsf, ids, weights, lb,
+                      le, plan, status);
+  if (E > 32 * 4 && E <= 32 * 10 && T <= topk_tokens<10>())
+    return launch_pdl(topk_plan_kernel<10>, dim3(1), dim3(1024), 0, st, logits, bias, T, E, k, rsf, ids, weights, lb,
+                      le, plan, status);
+  return cudaErrorNotSupported;   // E > 320: the per-lane key arrays outgrow 1024-thread registers
 }
 
 cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, int k, float rsf, int32_t* ids,

@@ -196,6 +196,20 @@ def test_moe_forward_decode_matches_oracle(name, T):
     assert_bf16_close(bf16_np(sh)[tokens], ref["shared"], what="shared")
 
 
+@pytest.mark.parametrize("name,T,local", [("decode_t1", None, None), ("decode_t8", None, None), ("tiny_t4", 1, None),
+                                          ("tiny_t4", None, (3, 11)), ("tiny_t4", 8, (0, 8)), ("decode_t32", None, None)])
+def test_forward_plan_matches_permute(name, T, local):
+    """The decode forward builds the routing plan in the top-k launch when the
+    tokens fit one top-k CTA (else with the permute kernels): either way the
+    plan equals the oracle's permutation of the forward's own ids."""
+    wl = workload(name, T)
+    inp = site_inputs(wl)
+    y, lg, ws, v = _forward(wl, inp, local=local)
+    ids = capi.view_tensor(v.ids, (wl.T, wl.k), torch.int32).cpu().numpy().copy()
+    _check_plan(_read_plan(v.plan, wl.E, wl.T * wl.k), ids, wl.E, local or (0, None))
+    assert np.array_equal(ids, OS.select_experts(lg, inp["router_bias"], wl.k))
+
+
 def test_moe_forward_is_deterministic():
     wl = workload("decode_t64")
     inp = site_inputs(wl)
