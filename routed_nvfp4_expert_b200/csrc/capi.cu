@@ -700,7 +700,9 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
     float* hts = (float*)(b + L.hts);
     const int32_t* used_tiles = plan.tile_offsets + E;
     RNX_CUDA(rnx::launch_tile_rows(plan, E, P, st), "tile rows");
-    RNX_CUDA(rnx::launch_quant_rows(x, P, H, plan.tile_rows, k, used_tiles, xq, xsf, xts, st), "x quant");
+    RNX_CUDA(rnx::launch_quant_tokens(x, T, H, k, ids, plan, cfg->local_begin, cfg->local_end, P, used_tiles, xq, xsf,
+                                      xts, st),
+             "x quant");
     RNX_CUDA(mark(MOE_STAGE_EXPERT_GATE_UP, st), "stage event");
     rnx::Fp4GemmArgs g = gemm_args(cfg, MOE_PROJ_GATE_UP, xq, xsf, xts, P, plan, wts, w, h, status);
     RNX_CUDA(rnx::launch_fp4_grouped_gemm(g, st), "expert gate/up (tcgen05)");

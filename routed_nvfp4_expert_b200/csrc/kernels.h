@@ -136,6 +136,13 @@ cudaError_t launch_tile_rows(const moe_plan_t& plan, int E, int64_t P_max, cudaS
 cudaError_t launch_quant_rows(const uint16_t* src, int64_t rows, int K, const int32_t* row_map, int div,
                               const int32_t* used_tiles, uint8_t* codes, uint8_t* sf, float* row_scale,
                               cudaStream_t st);
+// The prefill's x encoding token-major (each token encoded once, written to
+// the padded rows of its local assignments; padding rows of used tiles
+// zeroed): the same bytes as launch_quant_rows(x, P, K, tile_rows, k, ...).
+// k <= 16, else cudaErrorNotSupported.
+cudaError_t launch_quant_tokens(const uint16_t* x, int T, int K, int k, const int32_t* ids, const moe_plan_t& plan,
+                                int lb, int le, int64_t P, const int32_t* used_tiles, uint8_t* codes, uint8_t* sf,
+                                float* row_scale, cudaStream_t st);
 
 // Canonical block scales [n_experts * rows, K/16] -> atoms [n_experts][rows/128][K/64][512].
 cudaError_t launch_sf_atoms(const uint8_t* scales, int64_t n_experts, int rows, int K, uint8_t* atoms, cudaStream_t st);

@@ -105,6 +105,84 @@ __global__ void __launch_bounds__(kQuantWarps * 32) quant_rows_kernel(const uint
   if (lane == 0) row_scale[p] = ts;
 }
 
+// The prefill's x encoding, token-major: warp t (< T) encodes token t's row
+// once and writes it to the padded row of each of its local assignments
+// (padded row = tile_offsets[e] * 256 + inv[a] - offsets[e], the row whose
+// tile_rows entry is a); warp T + p zeroes padded row p when it is padding
+// inside a tile in use. Same arithmetic, in the same order, as
+// quant_rows_kernel per row; x is read (and divided) once per token instead
+// of once per assignment. k <= 16.
+__global__ void __launch_bounds__(kQuantWarps * 32) quant_tokens_kernel(
+    const uint16_t* __restrict__ x, int T, int K, int k, const int32_t* __restrict__ ids,
+    const int32_t* __restrict__ inv, const int32_t* __restrict__ offsets, const int32_t* __restrict__ tile_offsets,
+    int lb, int le, const int32_t* __restrict__ tile_rows, long long P, const int32_t* __restrict__ used_tiles,
+    uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, float* __restrict__ row_scale) {
+  __shared__ long long s_p[kQuantWarps][16];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long wg = (long long)blockIdx.x * kQuantWarps + warp;
+  const int nblk = K / 16, KB = K / 64;
+  const long long used = min((long long)*used_tiles * kRowsPerTile, P);
+  if (wg >= T) {
+    // a padding row of a tile in use: encoded as zeros
+    const long long p = wg - T;
+    if (p >= used || tile_rows[p] >= 0) return;
+    uint8_t* crow = codes + p * (K / 2);
+    for (int b = lane; b < nblk; b += 32) {
+      *reinterpret_cast<uint2*>(crow + b * 8) = make_uint2(0, 0);
+      sf[sf_atom_offset(p, b, KB)] = 0;
+    }
+    if (lane == 0) row_scale[p] = 0.f;
+    return;
+  }
+  const int t = (int)wg;
+  if (lane < k) {
+    const long long a = (long long)t * k + lane;
+    const int e = ids[a], pos = inv[a];
+    long long p = -1;
+    if (e >= lb && e < le && pos >= 0) p = (long long)tile_offsets[e] * kRowsPerTile + (pos - offsets[e]);
+    s_p[warp][lane] = (p >= 0 && p < used) ? p : -1;
+  }
+  __syncwarp();
+  bool any = false;
+  for (int j = 0; j < k; ++j) any = any || s_p[warp][j] >= 0;
+  if (!any) return;
+  const uint16_t* xr = x + (size_t)t * K;
+  float m = 0.f;
+  for (int b = lane; b < nblk; b += 32) {
+    float v[16];
+    load16(xr + b * 16, v);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+  }
+  m = warp_max(m);
+  const float ts = m / 2688.0f;
+  for (int b = lane; b < nblk; b += 32) {
+    float v[16];
+    load16(xr + b * 16, v);
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    const float q = ts == 0.f ? 0.f : (amax / 6.0f) / ts;
+    const uint8_t sb = f32_to_e4m3_satfinite(q);
+    const float d = e4m3_to_f32(sb) * ts;
+    uint32_t w0 = 0, w1 = 0;
+    if (d != 0.f) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        w0 |= (uint32_t)f32x2_to_e2m1x2_satfinite(v[2 * i] / d, v[2 * i + 1] / d) << (8 * i);
+        w1 |= (uint32_t)f32x2_to_e2m1x2_satfinite(v[8 + 2 * i] / d, v[8 + 2 * i + 1] / d) << (8 * i);
+      }
+    }
+    for (int j = 0; j < k; ++j) {
+      const long long p = s_p[warp][j];
+      if (p < 0) continue;
+      *reinterpret_cast<uint2*>(codes + p * (K / 2) + b * 8) = make_uint2(w0, w1);
+      sf[sf_atom_offset(p, b, KB)] = sb;
+    }
+  }
+  if (lane < k && s_p[warp][lane] >= 0) row_scale[s_p[warp][lane]] = ts;
+}
+
 // tile_rows[p] for p < P_max.
 __global__ void __launch_bounds__(256) tile_rows_kernel(const int32_t* __restrict__ counts,
                                                         const int32_t* __restrict__ offsets,
@@ -168,6 +246,19 @@ cudaError_t launch_quant_rows(const uint16_t* src, int64_t rows, int K, const in
   const long long grid = (rows_pad + kQuantWarps - 1) / kQuantWarps;
   quant_rows_kernel<<<(unsigned)grid, kQuantWarps * 32, 0, st>>>(src, rows, rows_pad, K, row_map, div, used_tiles,
                                                                   codes, sf, row_scale);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_tokens(const uint16_t* x, int T, int K, int k, const int32_t* ids, const moe_plan_t& plan,
+                                int lb, int le, int64_t P, const int32_t* used_tiles, uint8_t* codes, uint8_t* sf,
+                                float* row_scale, cudaStream_t st) {
+  if (k > 16) return cudaErrorNotSupported;
+  const long long warps = (long long)T + P;
+  if (warps <= 0) return cudaSuccess;
+  const long long grid = (warps + kQuantWarps - 1) / kQuantWarps;
+  quant_tokens_kernel<<<(unsigned)grid, kQuantWarps * 32, 0, st>>>(x, T, K, k, ids, plan.inv, plan.offsets,
+                                                                   plan.tile_offsets, lb, le, plan.tile_rows, P,
+                                                                   used_tiles, codes, sf, row_scale);
   return cudaGetLastError();
 }
 
