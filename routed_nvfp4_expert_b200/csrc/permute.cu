@@ -24,9 +24,11 @@ __global__ void __launch_bounds__(1024) permute_small(const int32_t* __restrict_
   __shared__ int s_cnt[kMaxE];
   __shared__ int s_off[kMaxE];
   __shared__ int s_warp[33];
+  __shared__ int s_act[kMaxE + 1];
+  __shared__ int s_sorted[kSmallMaxA];
   pdl_wait();
   pdl_trigger();
-  small_plan(ids, A, E, lb, le, plan, status, s_ids, s_cnt, s_off, s_warp);
+  small_plan(ids, A, E, lb, le, plan, status, s_ids, s_cnt, s_off, s_warp, s_act, s_sorted);
 }
 
 // ---- large A
@@ -71,6 +73,8 @@ __global__ void __launch_bounds__(1024) permute_scan(int nb, int E, int lb, int 
                                                      moe_plan_t plan) {
   __shared__ int s_cnt[kMaxE];
   __shared__ int s_warp[33];
+  __shared__ int s_off[kMaxE];
+  __shared__ int s_act[kMaxE + 1];
   constexpr int kPer = 16;   // 512 blocks per pass
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   for (int e = warp; e < E; e += nw) {
@@ -99,7 +103,7 @@ __global__ void __launch_bounds__(1024) permute_scan(int nb, int E, int lb, int 
     if (lane == 0) s_cnt[e] = carry;
   }
   __syncthreads();
-  finish_plan(s_cnt, E, lb, le, plan, s_warp);
+  finish_plan(s_cnt, E, lb, le, plan, s_warp, s_off, s_act);   // the shared copies go unused here
 }
 
 __global__ void __launch_bounds__(kChunk) permute_scatter(const int32_t* __restrict__ ids, int A, int E,

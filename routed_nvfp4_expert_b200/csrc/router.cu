@@ -144,17 +144,18 @@ __global__ void __launch_bounds__(256) router_logits_sgemm(const uint16_t* __res
 // One warp per token. Lane l holds experts l, l+32, ... Candidate order:
 // unused finite keys first (key descending, then lower index), then NaN keys
 // (lower index first), then used / padding entries.
-struct Cand {
-  int state;   // 0 = live key, 1 = NaN key, 2 = taken or padding
-  float key;
-  int idx;
-  float s;
-};
-
-RNX_DEVICE bool better(const Cand& a, const Cand& b) {
-  if (a.state != b.state) return a.state < b.state;
-  if (a.state == 0 && a.key != b.key) return a.key > b.key;
-  return a.idx < b.idx;
+// That order as one 64-bit integer, larger = better (one warp max per
+// selection round): bits 63..62 the class (live 2, NaN 1, taken / padding 0),
+// bits 61..30 a live key's fp32 bits mapped to unsigned order (a zero key as
+// +0), bits 29..0 the complement of the index (the lower index wins a tie).
+RNX_DEVICE unsigned long long cand_rank(int state, float key, int idx) {
+  uint32_t ok = 0;
+  if (state == 0) {
+    const uint32_t u = key == 0.f ? 0u : __float_as_uint(key);
+    ok = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  }
+  return ((unsigned long long)(2 - state) << 62) | ((unsigned long long)ok << 30) |
+         (unsigned long long)(0x3FFFFFFF - idx);
 }
 
 // 8 tokens per CTA. All 256 threads first evaluate the sigmoid scores and
@@ -201,30 +202,26 @@ RNX_DEVICE void topk_warp(const float* s_key_row, const float* s_sig_row, int t,
   float chosen_s = 0.f;   // lane j keeps the score of rank slot j
   int chosen_id = 0;
   for (int j = 0; j < k; ++j) {
-    Cand best{2, 0.f, 0x7fffffff, 0.f};
+    unsigned long long best = 0ull;
 #pragma unroll
-    for (int i = 0; i < PL; ++i) {
-      Cand c{st[i], key[i], lane + 32 * i, sg[i]};
-      if (better(c, best)) best = c;
-    }
+    for (int i = 0; i < PL; ++i) best = max(best, cand_rank(st[i], key[i], lane + 32 * i));
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      Cand other;
-      other.state = __shfl_xor_sync(0xffffffffu, best.state, o);
-      other.key = __shfl_xor_sync(0xffffffffu, best.key, o);
-      other.idx = __shfl_xor_sync(0xffffffffu, best.idx, o);
-      other.s = __shfl_xor_sync(0xffffffffu, best.s, o);
-      if (better(other, best)) best = other;
-    }
-    // the owner marks its entry taken
-    if ((best.idx & 31) == lane) {
+    for (int o = 16; o > 0; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
+    const int idx = 0x3FFFFFFF - (int)(best & 0x3FFFFFFFull);
+    // the owner marks its entry taken and hands over its score
+    float s_own = 0.f;
+    if ((idx & 31) == lane) {
 #pragma unroll
       for (int i = 0; i < PL; ++i)
-        if (lane + 32 * i == best.idx) st[i] = 2;
+        if (lane + 32 * i == idx) {
+          st[i] = 2;
+          s_own = sg[i];
+        }
     }
+    const float s_best = __shfl_sync(0xffffffffu, s_own, idx & 31);
     if (lane == j) {
-      chosen_s = best.s;
-      chosen_id = best.idx;
+      chosen_s = s_best;
+      chosen_id = idx;
     }
   }
   // renormalise the UNBIASED scores over the chosen k, rank order
@@ -268,6 +265,8 @@ __global__ void __launch_bounds__(1024) topk_plan_kernel(const float* __restrict
   __shared__ int s_cnt[kMaxE];
   __shared__ int s_off[kMaxE];
   __shared__ int s_warp[33];
+  __shared__ int s_act[kMaxE + 1];
+  __shared__ int s_sorted[kSmallMaxA];
   const int warp = threadIdx.x >> 5;
   pdl_wait();
   pdl_trigger();
@@ -275,7 +274,7 @@ __global__ void __launch_bounds__(1024) topk_plan_kernel(const float* __restrict
   __syncthreads();
   if (warp < T) topk_warp<PL>(s_key[warp], s_sig[warp], warp, E, k, rsf, ids, weights);
   __syncthreads();                       // the ids, for every thread of the CTA
-  small_plan(ids, T * k, E, lb, le, plan, status, s_ids, s_cnt, s_off, s_warp);
+  small_plan(ids, T * k, E, lb, le, plan, status, s_ids, s_cnt, s_off, s_warp, s_act, s_sorted);
 }
 
 __global__ void __launch_bounds__(256) row_absmax_kernel(const uint16_t* __restrict__ rows, int R, int K,

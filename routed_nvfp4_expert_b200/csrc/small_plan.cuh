@@ -44,8 +44,11 @@ RNX_DEVICE int block_exclusive_scan(int v, int* s_warp, int* total) {
   return res;
 }
 
-// counts -> offsets, tile_offsets, active (one CTA of 1024 threads, E <= 1024)
-RNX_DEVICE void finish_plan(const int* s_cnt, int E, int lb, int le, const moe_plan_t& plan, int* s_warp) {
+// counts -> offsets, tile_offsets, active (one CTA of 1024 threads, E <= 1024);
+// the offsets and the active list also land in shared memory (s_off[E],
+// s_act[1 + E], count first), so that later steps need no global read-back.
+RNX_DEVICE void finish_plan(const int* s_cnt, int E, int lb, int le, const moe_plan_t& plan, int* s_warp, int* s_off,
+                            int* s_act) {
   const int e = threadIdx.x;
   const int c = e < E ? s_cnt[e] : 0;
   const bool local = e >= lb && e < le;
@@ -61,37 +64,35 @@ RNX_DEVICE void finish_plan(const int* s_cnt, int E, int lb, int le, const moe_p
     plan.counts[e] = c;
     plan.offsets[e] = off;
     plan.tile_offsets[e] = toff;
-    if (act) plan.active[1 + aoff] = e;
+    s_off[e] = off;
+    if (act) {
+      plan.active[1 + aoff] = e;
+      s_act[1 + aoff] = e;
+    }
   }
   if (e == 0) {
     plan.offsets[E] = tot;
     plan.tile_offsets[E] = ttot;
     plan.active[0] = atot;
+    s_act[0] = atot;
   }
 }
 
-// first[u] = sorted[offsets[e]] for the u-th active (local, non-empty) expert e.
-// Runs after sorted[] is complete; reads offsets/active/sorted from the plan.
-RNX_DEVICE void write_first(const moe_plan_t& plan, const int* s_off, const int* s_cnt, int E, int lb, int le) {
-  const int n_active = plan.active[0];
-  for (int u = threadIdx.x; u < n_active; u += blockDim.x) {
-    const int e = plan.active[1 + u];
-    plan.first[u] = plan.sorted[plan.offsets[e]];
-  }
-  (void)s_off;
-  (void)s_cnt;
-  (void)E;
-  (void)lb;
-  (void)le;
+// first[u] = sorted[offsets[e]] for the u-th active (local, non-empty) expert
+// e, from the shared copies of offsets, the active list and sorted.
+RNX_DEVICE void write_first(const moe_plan_t& plan, const int* s_off, const int* s_act, const int* s_sorted) {
+  const int n_active = s_act[0];
+  for (int u = threadIdx.x; u < n_active; u += blockDim.x) plan.first[u] = s_sorted[s_off[s_act[1 + u]]];
 }
 
 
 // ids: A expert ids (global memory; written before this call by any thread of
 // the CTA is fine: the first barrier below orders it). Shared scratch:
-// s_ids[kSmallMaxA], s_cnt[kMaxE], s_off[kMaxE], s_warp[33]. Every thread of
-// the (1024-thread) CTA calls it.
+// s_ids[kSmallMaxA], s_cnt[kMaxE], s_off[kMaxE], s_warp[33], s_act[kMaxE + 1],
+// s_sorted[kSmallMaxA]. Every thread of the (1024-thread) CTA calls it.
 RNX_DEVICE void small_plan(const int32_t* ids, int A, int E, int lb, int le, const moe_plan_t& plan,
-                                  uint32_t* status, int* s_ids, int* s_cnt, int* s_off, int* s_warp) {
+                           uint32_t* status, int* s_ids, int* s_cnt, int* s_off, int* s_warp, int* s_act,
+                           int* s_sorted) {
   for (int e = threadIdx.x; e < E; e += blockDim.x) s_cnt[e] = 0;
   __syncthreads();
   for (int a = threadIdx.x; a < A; a += blockDim.x) {
@@ -105,9 +106,7 @@ RNX_DEVICE void small_plan(const int32_t* ids, int A, int E, int lb, int le, con
     s_ids[a] = e;
   }
   __syncthreads();
-  finish_plan(s_cnt, E, lb, le, plan, s_warp);
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) s_off[e] = plan.offsets[e];
+  finish_plan(s_cnt, E, lb, le, plan, s_warp, s_off, s_act);
   __syncthreads();
   // stable position: offset + number of earlier assignments of the same expert
   for (int a0 = 0; a0 < A; a0 += blockDim.x) {
@@ -120,6 +119,7 @@ RNX_DEVICE void small_plan(const int32_t* ids, int A, int E, int lb, int le, con
       if (e >= 0) {
         const int pos = s_off[e] + rank;
         plan.sorted[pos] = a;
+        s_sorted[pos] = a;
         plan.inv[a] = pos;
       } else {
         plan.inv[a] = -1;
@@ -127,7 +127,7 @@ RNX_DEVICE void small_plan(const int32_t* ids, int A, int E, int lb, int le, con
     }
   }
   __syncthreads();
-  write_first(plan, s_off, s_cnt, E, lb, le);
+  write_first(plan, s_off, s_act, s_sorted);
 }
 
 }  // namespace rnx
