@@ -121,7 +121,7 @@ cudaError_t launch_dense_ffn(int H, int I, float limit, const uint16_t* x, int T
 // ---------------------------------------------------------------- prefill (W4A4, tcgen05)
 
 // Padded tile layout of the prefill: every local expert's rows start on a
-// 128-row tile. tile_rows[p] = assignment at padded row p, -1 for padding.
+// 256-row tile (kRowsPerTile). tile_rows[p] = assignment at padded row p, -1 for padding.
 // P_max = padded_rows_bound(A, E_local) rows are written (rows past the last
 // used tile get -1 too).
 int64_t padded_rows_bound(int64_t A, int64_t E_local);
