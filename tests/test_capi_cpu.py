@@ -105,3 +105,73 @@ def test_noalloc_rejects_oversized_requests_before_touching_the_device():
     w = capi.MoeWeights()
     st = lib.moe_forward_decode_noalloc(C.byref(cfg), C.byref(w), 0x1000, 4096, 0x2000, None)
     assert st == 3 and "built-in buffer" in lib.moe_last_error().decode()
+
+
+def _fake_weights(prepared=None):
+    w = capi.MoeWeights()
+    w.router_w, w.router_bias = 0x10000, 0x11000
+    for i, b in enumerate((w.gate, w.up, w.down)):
+        b.codes, b.scales, b.tensor_scale = 0x100000 * (i + 1), 0x100000 * (i + 1) + 0x80000, 0x12000 + 0x100 * i
+    w.prepared = prepared
+    return w
+
+
+def test_padded_rows_and_prepared_size_are_host_arithmetic():
+    lib = capi.lib()
+    cfg = _cfg()                                   # E = 16, k = 4, H = 256, I = 128
+    for T in (0, 1, 10, 300, 4096):
+        A = T * 4
+        n = min(A, 16)
+        assert lib.moe_padded_rows(C.byref(cfg.c()), T) == (A + 255 * n) // 256 * 256
+    # EP range: only the local experts get tiles
+    assert lib.moe_padded_rows(C.byref(_cfg(local_begin=4, local_end=6).c()), 100) == (400 + 255 * 2) // 256 * 256
+    up = lambda v: (v + 255) // 256 * 256
+    per = 16 * 128 * 256 // 16
+    # gate / up / down scale atoms, then the router weight as three bf16 terms
+    assert lib.moe_prepared_size(C.byref(cfg.c())) == up(3 * per) + up(16 * 3 * 256 * 2)
+
+
+def test_prefill_entry_points_validate_before_launch():
+    lib = capi.lib()
+    cfg = _cfg().c()
+    w = _fake_weights(prepared=0x800000)
+    plan = capi.MoePlan(*[0x900000 + 0x1000 * i for i in range(8)])
+    # shapes the tensor-core prefill does not cover
+    bad = _cfg(hidden=192).c()
+    assert lib.nvfp4_grouped_gemm(C.byref(bad), 0, 0x1000, 0x2000, 0x3000, 4, C.byref(plan), 0x4000, C.byref(w),
+                                  0x5000, 0x6000, 1 << 30, None) == 2
+    assert "hidden" in lib.moe_last_error().decode()
+    assert lib.moe_prepare_weights(C.byref(bad), C.byref(w), 0x700000, 1 << 30, None) == 2
+    # unknown projection, T = 0, missing prepared weights, short workspace
+    assert lib.nvfp4_grouped_gemm(C.byref(cfg), 5, 0x1000, 0x2000, 0x3000, 4, C.byref(plan), 0x4000, C.byref(w),
+                                  0x5000, 0x6000, 1 << 30, None) == 1
+    assert lib.nvfp4_grouped_gemm(C.byref(cfg), 0, None, None, None, 0, None, None, C.byref(w), None, None, 0,
+                                  None) == 0
+    w0 = _fake_weights(prepared=None)
+    assert lib.nvfp4_grouped_gemm(C.byref(cfg), 0, 0x1000, 0x2000, 0x3000, 4, C.byref(plan), 0x4000, C.byref(w0),
+                                  0x5000, 0x6000, 1 << 30, None) == 1
+    assert "prepared" in lib.moe_last_error().decode()
+    assert lib.nvfp4_grouped_gemm(C.byref(cfg), 1, 0x1000, 0x2000, 0x3000, 4, C.byref(plan), 0x4000, C.byref(w),
+                                  0x5000, 0x6000, 256, None) == 3
+    # weight preparation: misaligned or short destination
+    need = lib.moe_prepared_size(C.byref(cfg))
+    assert lib.moe_prepare_weights(C.byref(cfg), C.byref(w), 0x700010, need, None) == 1
+    assert lib.moe_prepare_weights(C.byref(cfg), C.byref(w), 0x700000, need - 1, None) == 3
+    assert lib.moe_prepare_weights(C.byref(cfg), C.byref(capi.MoeWeights()), 0x700000, need, None) == 1
+    # row encoding: K must be a multiple of 64; no rows is a no-op
+    assert lib.nvfp4_quantize_rows(0x1000, 4, 100, 0x2000, 0x3000, 0x4000, None) == 1
+    assert lib.nvfp4_quantize_rows(0x1000, 0, 256, 0x2000, 0x3000, 0x4000, None) == 0
+
+
+def test_unpermute_entry_points_validate_before_launch():
+    lib = capi.lib()
+    cfg = _cfg().c()
+    plan = capi.MoePlan(*[0x900000 + 0x1000 * i for i in range(8)])
+    assert lib.moe_unpermute(C.byref(cfg), None, 0, None, None, None, None) == 0
+    assert lib.moe_unpermute(C.byref(cfg), 0x1000, 4, None, 0x2000, 0x3000, None) == 1
+    assert "plan" in lib.moe_last_error().decode()
+    assert lib.moe_unpermute(C.byref(cfg), 0x1008, 4, C.byref(plan), 0x2000, 0x3000, None) == 1
+    assert "rows" in lib.moe_last_error().decode()
+    assert lib.moe_unpermute_combine(C.byref(cfg), 0x1000, 4, C.byref(plan), 0x2000, 0x3008, 0x4000, None) == 1
+    assert "shared" in lib.moe_last_error().decode()
+    assert lib.moe_unpermute_combine(C.byref(cfg), None, 0, None, None, None, None, None) == 0
