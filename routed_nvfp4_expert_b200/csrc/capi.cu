@@ -720,11 +720,11 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
     a.weights = wts;
     a.gate = w->gate; a.up = w->up; a.down = w->down;
     a.status = status;
-    a.proj = MOE_PROJ_GATE_UP; a.act = x; a.out = h; a.act_max = xmax; a.out_max = hmax; a.prefetch_down = false;
+    a.proj = MOE_PROJ_GATE_UP; a.act = x; a.out = h; a.act_max = xmax; a.out_max = hmax;
     RNX_CUDA(mark(MOE_STAGE_EXPERT_GATE_UP, st), "stage event");
     RNX_CUDA(rnx::launch_nvfp4_gemv(a, st), "expert gate/up");
     RNX_CUDA(mark(MOE_STAGE_H_QUANT, st), "stage event");
-    a.proj = MOE_PROJ_DOWN; a.act = h; a.out = r; a.act_max = hmax; a.out_max = nullptr; a.prefetch_down = false;
+    a.proj = MOE_PROJ_DOWN; a.act = h; a.out = r; a.act_max = hmax; a.out_max = nullptr;
     RNX_CUDA(mark(MOE_STAGE_EXPERT_DOWN, st), "stage event");
     RNX_CUDA(rnx::launch_nvfp4_gemv(a, st), "expert down");
   }

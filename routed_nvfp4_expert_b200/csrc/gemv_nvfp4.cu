@@ -55,9 +55,6 @@ struct GemvParams {
   const uint32_t* act_max;    // direct form: max |activation row| (fp32 bits), by act row
   uint32_t* out_max;          // direct GATE_UP: atomicMax of |h| per assignment (nullable)
   uint32_t* status;           // device status word (bounded waits)
-  const uint8_t* pf_codes;    // direct GATE_UP: down bank to prefetch into L2 (nullable)
-  const uint8_t* pf_scales;
-  long long pf_codes_per_expert, pf_scales_per_expert;
 };
 
 // Shared-memory activation layout: row m, 16-byte unit index
@@ -556,12 +553,6 @@ GemvParams gemv_params(const ExpertGemvArgs& a, bool gu) {
   p.act_max = a.act_max;
   p.out_max = a.out_max;
   p.status = a.status;
-  if (gu && a.prefetch_down && a.down.codes) {
-    p.pf_codes = a.down.codes;
-    p.pf_scales = a.down.scales;
-    p.pf_codes_per_expert = (long long)a.H * a.I / 2;
-    p.pf_scales_per_expert = (long long)a.H * a.I / 16;
-  }
   return p;
 }
 

@@ -44,7 +44,6 @@ struct ExpertGemvArgs {
   uint32_t* status;         // device status word (bounded-wait timeouts)
   const uint32_t* act_max;  // optional: max |activation row| as fp32 bits (x rows by token / h rows by assignment)
   uint32_t* out_max;        // optional (GATE_UP): receives max |h| per assignment; must start at 0
-  bool prefetch_down;       // GATE_UP (one token per expert): pull the experts' down weights into L2
 };
 
 cudaError_t launch_nvfp4_gemv(const ExpertGemvArgs& a, cudaStream_t st);
