@@ -134,12 +134,6 @@ RNX_DEVICE uint4 ldg_stream(const void* p) {
   return r;
 }
 
-// Bulk prefetch of [p, p + bytes) into L2 (TMA engine, no completion tracking).
-// p 16-byte aligned, bytes a multiple of 16.
-RNX_DEVICE void prefetch_l2(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
 RNX_DEVICE uint16_t ldg_u16(const void* p) {
   uint16_t r;
   asm("ld.global.nc.u16 %0, [%1];" : "=h"(r) : "l"(p));

@@ -78,29 +78,6 @@ RNX_DEVICE bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-// L2 policy: streamed once, evict first.
-RNX_DEVICE uint64_t policy_evict_first() {
-  uint64_t pol;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-  return pol;
-}
-
-// Global -> shared bulk copy on the TMA engine, completion counted as bytes on
-// `bar`. dst, src 16-byte aligned; bytes a multiple of 16.
-RNX_DEVICE void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
-          smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
-      : "memory");
-}
-
-// Shared -> global bulk copy (TMA engine), tracked by the issuing thread's
-// bulk async-group. dst, src 16-byte aligned; bytes a multiple of 16.
-RNX_DEVICE void bulk_s2g(void* dst, const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_u32(src)), "r"(bytes)
-               : "memory");
-}
 RNX_DEVICE void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until the source shared memory of every committed group was read.
 RNX_DEVICE void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
