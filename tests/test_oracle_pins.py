@@ -379,3 +379,51 @@ def test_dense_ffn_matches_torch_reference():
     g, u = tb(xb) @ tb(wg).T, tb(xb) @ tb(wu).T
     ref = (torch.nn.functional.silu(torch.clamp(g, max=7.0)) * torch.clamp(u, -7.0, 7.0)) @ tb(wd).T
     assert np.allclose(S.dense_ffn(xb, wg, wu, wd, 7.0), ref.numpy(), rtol=1e-13, atol=1e-16)
+
+
+# ------------------------------------------------------------------ readings 5, 6, 12
+
+def test_zero_score_sum_gives_zero_weights():
+    """Reading 5: no epsilon in the renormalisation; a zero denominator gives
+    zero weights (never NaN). Logits of -1e30 give sigmoid scores of exactly 0."""
+    l64 = np.full((3, 16), -1e30)
+    ids = S.select_experts(l64.astype(np.float32), np.zeros(16, np.float32), 4)
+    assert np.array_equal(ids, np.tile(np.arange(4, dtype=np.int32), (3, 1)))   # all keys equal: lowest indices
+    w = S.routing_weights(l64, ids, 2.5)
+    assert np.all(w == 0.0)
+
+
+def test_nan_keys_rank_last_in_index_order():
+    """Reading 6: a NaN key is chosen only when fewer finite keys than k are
+    left, and NaN keys then go in index order."""
+    E, k = 16, 4
+    logits = np.zeros((2, E), np.float32)
+    bias = np.zeros(E, np.float32)
+    bias[[1, 5, 9]] = np.nan
+    bias[[2, 3]] = 0.25
+    ids = S.select_experts(logits, bias, k)
+    assert ids[0].tolist() == [2, 3, 0, 4]            # finite keys first: 0.75 x2, then 0.5 by index
+    nan_all = np.full(E, np.nan, np.float32)
+    nan_all[7] = 0.0
+    ids2 = S.select_experts(logits, nan_all, k)
+    assert ids2[0].tolist() == [7, 0, 1, 2]          # the one finite key, then NaNs by index
+
+
+def test_prefill_tokens_are_independent_of_their_batch():
+    """Reading 12: the activation encoding's second-level scale is per token
+    row, so a token's prefill output does not depend on the other tokens of
+    the batch (chunked prefill equals whole prefill). A batch-wide scale would
+    break this by far more than the fp64 tolerance."""
+    wl, inp, cfg = _tiny()
+    whole = S.site_forward(inp, cfg, "prefill")["y"]
+    for t in range(wl.T):
+        solo = S.site_forward(inp, cfg, "prefill", tokens=[t])["y"]
+        assert np.allclose(solo[0], whole[t], rtol=1e-12, atol=1e-14)
+    # and scaling one token's x (exactly, by a power of two) leaves the
+    # others' outputs unchanged
+    inp2 = dict(inp)
+    x = np.asarray(inp["x"]).copy()
+    x[0] = syn._to_bf16_bits(F.bf16_value(x[0]) * 4.0)
+    inp2["x"] = x
+    other = S.site_forward(inp2, cfg, "prefill")["y"]
+    assert np.allclose(other[1:], whole[1:], rtol=1e-12, atol=1e-14)
