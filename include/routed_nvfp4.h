@@ -370,12 +370,13 @@ moe_status_t nvfp4_dequant(const uint8_t* codes, const uint8_t* scales, const fl
  * One routed site forward: router, top-k, experts (path), shared expert,
  * combine. x bf16 [T, H] -> y bf16 [T, H]. ws: moe_workspace_size(cfg, T,
  * path) bytes. The routing plan, logits, ids and weights of the call stay in
- * the workspace until the next call (see moe_workspace_views). Every launch
- * after the first is a programmatic dependent launch of its predecessor.
+ * the workspace until the next call (see moe_workspace_views).
  *   MOE_PATH_DECODE: W4A16 GEMV experts (nvfp4_expert_gemv); with up to 8
- *     tokens (E <= 320) top-k and the routing plan are one launch; the shared
- *     expert runs on the library's auxiliary stream of this host thread and
- *     device, forked from and joined back into `stream` with events.
+ *     tokens (E <= 320) top-k and the routing plan are one launch; router,
+ *     top-k, plan, the two expert GEMVs and the combine are chained by
+ *     programmatic dependent launch; the shared expert runs on the library's
+ *     auxiliary stream of this host thread and device, forked from and joined
+ *     back into `stream` with events.
  *   MOE_PATH_PREFILL: permute with the padded tile layout, x encoded to
  *     NVFP4 per token row and written to its assignments' padded rows (the
  *     bytes nvfp4_quantize_rows gives per assignment row), grouped GEMM
