@@ -330,9 +330,11 @@ def run_ours(args, rank, world, local_rank):
                     "algorithmic_bytes_per_step": int(algo_bytes), "unique_experts_per_step": U,
                     "bytes_per_expert": expert_bytes(wl),
                     "traffic": read_traffic_profile(f"nvfp4_expert_gemv_{wl.name}")}
-        # router, top-k, plan, expert gate/up, expert down, combine, and the
+        # router, top-k + plan (one launch up to 8 tokens at E <= 320, else
+        # top-k and the permute), expert gate/up, expert down, combine, and the
         # shared expert's two GEMVs on the auxiliary stream
-        launches_per_step = 8 if T * wl.k <= 1024 else 11
+        fused_plan = T <= 8 and wl.E <= 320 and T * wl.k <= 1024
+        launches_per_step = 7 if fused_plan else (8 if T * wl.k <= 1024 else 11)
         path_name = "decode GEMV (W4A16)"
     out = {
         "metric": METRIC,
