@@ -8,11 +8,13 @@ import torch
 from oracle import site as OS
 from routed_nvfp4_expert_b200 import synthetic as syn
 
-# Output gate for bf16 results: relative L2 <= 1e-2 and
-# max |d| <= 2e-2 + 2^-8 |y_ref| (the added term is half a bf16 ulp).
+# Output gate for bf16 results: relative L2 <= 1e-2 and max |d| <= 2e-2.
+# Where |y_ref| >= 8 the one rounding of the result to bf16 alone can move it
+# by up to 2^-8 |y_ref| > 2e-2, so there the bound is 2e-2 + 2^-8 |y_ref|.
 OUT_REL_L2 = 1e-2
 OUT_ABS = 2e-2
 OUT_REL_ELEM = 2.0 ** -8
+OUT_BIG = 8.0
 LOGIT_REL = 1e-5       # relative to the token's largest |logit|
 WEIGHT_REL = 1e-5
 
@@ -28,7 +30,7 @@ def assert_bf16_close(got, ref, rel=OUT_REL_L2, what="output"):
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
     r = rel_l2(got, ref)
-    bound = OUT_ABS + OUT_REL_ELEM * np.abs(ref)
+    bound = OUT_ABS + np.where(np.abs(ref) >= OUT_BIG, OUT_REL_ELEM * np.abs(ref), 0.0)
     d = np.abs(got - ref)
     bad = d > bound
     assert r <= rel, f"{what}: rel-L2 {r:.3e} > {rel:.1e}"
@@ -37,7 +39,7 @@ def assert_bf16_close(got, ref, rel=OUT_REL_L2, what="output"):
 
 
 def bf16_np(t: torch.Tensor) -> np.ndarray:
-    """torch bf16 (any device) -> fp64 numpy."""
+    """torch bf16 / fp32 (any device) -> fp64 numpy."""
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
@@ -96,3 +98,42 @@ def device_site(wl, inp):
     banks, shared = _device_weights(_geom(wl))
     return capi.DeviceSite(_t.from_numpy(inp["router_w"]).cuda(), _t.from_numpy(inp["router_bias"]).cuda(),
                            banks, shared)
+
+
+def quantised_bank(seed: int, E: int, rows: int, cols: int, sigma: float):
+    """An NVFP4 bank made the way a checkpoint's would be: weights N(0, sigma)
+    (fp32) quantised per expert with tensor scale ts = amax / (6 * 448), block
+    scale = E4M3 round-to-nearest of amax_block / 6 / ts, code = E2M1
+    round-to-nearest of w / (scale * ts). The roundings are ml_dtypes' casts,
+    so this data shares nothing with either side under test. Test data only.
+
+    Returns codes uint8 [E, rows, cols/2], scales uint8 [E, rows, cols/16],
+    ts float32 [E] (the canonical layout)."""
+    import ml_dtypes
+    rng = np.random.default_rng(seed)
+    codes = np.empty((E, rows, cols // 2), np.uint8)
+    scales = np.empty((E, rows, cols // 16), np.uint8)
+    ts = np.empty(E, np.float32)
+    for e in range(E):
+        w = (rng.standard_normal((rows, cols), dtype=np.float32) * np.float32(sigma)).astype(np.float32)
+        t = np.float32(np.abs(w).max() / np.float32(6 * 448))
+        blk = np.abs(w).reshape(rows, cols // 16, 16).max(axis=2)
+        q = np.minimum((blk / np.float32(6)) / t, np.float32(448)).astype(np.float32)
+        sb = q.astype(ml_dtypes.float8_e4m3fn)
+        d = (sb.astype(np.float32) * t).astype(np.float32)
+        ratio = np.where(d[:, :, None] > 0, w.reshape(rows, cols // 16, 16) / d[:, :, None], 0.0)
+        ratio = np.clip(ratio.astype(np.float32), -6, 6)
+        c = ratio.astype(ml_dtypes.float4_e2m1fn).view(np.uint8).reshape(rows, cols) & 0xF
+        codes[e] = (c[:, 0::2] | (c[:, 1::2] << 4)).astype(np.uint8)
+        scales[e] = sb.view(np.uint8)
+        ts[e] = t
+    return codes, scales, ts
+
+
+def with_quantised_banks(wl, inp: dict, seed: int = 3) -> dict:
+    """inp with its three expert banks replaced by quantised_bank() ones."""
+    out = dict(inp)
+    for i, (proj, rows, cols) in enumerate((("gate", wl.I, wl.H), ("up", wl.I, wl.H), ("down", wl.H, wl.I))):
+        c, s, t = quantised_bank(seed * 10 + i, wl.E, rows, cols, wl.sigma_w)
+        out[f"{proj}_codes"], out[f"{proj}_scales"], out[f"{proj}_ts"] = c, s, t
+    return out

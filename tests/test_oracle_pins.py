@@ -124,6 +124,37 @@ def test_act_quant_hand_worked_example():
     assert t.view(np.uint32)[0] == int(golden_comment_field("act_quant_example.txt", "tsx_hex")[0], 16)
 
 
+def test_act_quant_dequant_hand_worked_example():
+    """dequant_rows_nvfp4 on the hand-worked row: every element equals code
+    value x e4m3(scale) x tsx as worked out by hand, sign of zero included."""
+    rows = golden_lines("act_quant_example.txt")
+    a = np.array([[float(r[0]) for r in rows]], np.float32)
+    c, s, t = F.quantize_rows_nvfp4(a)
+    got = F.dequant_rows_nvfp4(c, s, t)[0]
+    want = golden_lines("act_quant_dequant.txt")
+    assert [int(w[0], 16) for w in want] == list(F.unpack_nibbles(c)[0])
+    for g, (_, v) in zip(got, want):
+        assert g == float(v) and math.copysign(1, g) == math.copysign(1, float(v)), (g, v)
+    # per-block scale broadcast: the same codes under swapped block scales
+    # decode block 0 with 0x59 and block 1 with 0x7E
+    got2 = F.dequant_rows_nvfp4(c, s[:, ::-1].copy(), t)[0]
+    assert got2[0] == 6 * 18 * 2.0 ** -9 and got2[16] == 6 * 448 * 2.0 ** -9
+    # the row scale multiplies every element: twice tsx, twice the values
+    got3 = F.dequant_rows_nvfp4(c, s, (t * 2).astype(np.float32))[0]
+    assert np.array_equal(got3, 2 * got)
+
+
+def test_router_logits_hand_worked_example():
+    """l = Wr . x on a non-square router (E = 3, H = 5), worked by hand."""
+    rows = golden_lines("router_logits_example.txt")
+    x = np.array([[float(v) for v in r[1:]] for r in rows if r[0] == "x"], np.float32)
+    w = np.array([[float(v) for v in r[1:]] for r in rows if r[0] == "w"], np.float32)
+    want = np.array([[float(v) for v in r[1:]] for r in rows if r[0] == "logits"])
+    got = S.router_logits(F.f32_to_bf16_bits(x), w)
+    assert got.shape == (2, 3)
+    assert np.array_equal(got, want)
+
+
 def test_act_quant_matches_ml_dtypes_steps():
     """The same steps with the two roundings done by ml_dtypes."""
     rng = np.random.default_rng(7)
@@ -304,6 +335,21 @@ def test_clamp_fires_only_on_tails():
     assert 0 < hot["clamp_fired"] < hot["clamp_total"]
     cfg2.swiglu_limit = math.inf
     assert not np.allclose(S.site_forward(inp2, cfg2, "decode")["y"], hot["y"])
+
+
+def test_stress_recipe_fires_the_clamp_on_about_five_percent():
+    """The stress workload's x8 activations make the clamp fire on ~5% of the
+    gate/up elements (the stress prefill config), while the plain prefill
+    workload's never reach it (the clamp is invisible off the tails)."""
+    from helpers import oracle_cfg, site_inputs, workload
+    for name, lo, hi in (("stress_t16384", 0.03, 0.07), ("prefill_t4096", 0.0, 1e-4)):
+        wl = workload(name)
+        inp = site_inputs(wl)
+        rng = np.random.default_rng(11)
+        tokens = np.setdiff1d(rng.choice(wl.T, 40, replace=False), inp.get("tie_tokens", []))[:24]
+        out = S.site_forward(inp, oracle_cfg(wl), "decode", tokens=tokens)
+        frac = out["clamp_fired"] / out["clamp_total"]
+        assert lo <= frac <= hi, (name, frac)
 
 
 def test_local_range_masks_remote_experts():
