@@ -158,14 +158,22 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ ours
 
-def run_ours(args, rank, world, local_rank):
+def decode_t1_fused(wl) -> bool:
+    """The single-token decode chain (three launches) runs for this workload;
+    mirrors the library's eligibility rule for T = 1."""
+    return (wl.kind == "decode" and wl.T == 1 and wl.H % 256 == 0 and wl.H <= 8192 and wl.I % 64 == 0
+            and wl.I <= 2048 and wl.k <= 16 and wl.E <= 1024)
+
+
+def measure(wl, args, rank, world, local_rank, dev, clocks=None):
+    """Time one workload: K replays of the forward's CUDA graph (the value),
+    interleaved with K replays of the same forward with events around the
+    dominant kernels (their live duration, for the roofline). Returns the
+    per-rank numbers (max over ranks taken by the caller)."""
     import torch
     from routed_nvfp4_expert_b200 import capi
     from routed_nvfp4_expert_b200 import synthetic as syn
 
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    wl = syn.WORKLOADS[args.workload]
     inp = syn.make_site(wl, seed=0)
     site = capi.site_to_device(inp, dev)
     cfg = capi.config_for(wl)
@@ -202,8 +210,9 @@ def run_ours(args, rank, world, local_rank):
     w_c = site.c()
     i_gu, i_sh = capi.STAGES.index("expert_gate_up"), capi.STAGES.index("shared")
     i_hq, i_dn = capi.STAGES.index("h_quant"), capi.STAGES.index("expert_down")
-    # intervals of the dominant kernels: decode = both expert GEMVs (adjacent);
-    # prefill = the two grouped GEMMs (the h encoding between them excluded)
+    # intervals of the dominant kernels: decode = both expert launches
+    # (adjacent); prefill = the two grouped GEMMs (the h encoding between them
+    # excluded)
     spans = [(i_gu, i_hq), (i_dn, i_sh)] if prefill else [(i_gu, i_sh)]
 
     # warm the kernels once outside capture, then capture the forward into graphs:
@@ -256,27 +265,23 @@ def run_ours(args, rank, world, local_rank):
 
     dist_barrier(world)
     torch.cuda.synchronize(dev)
-    clocks = clock_sampler(local_rank)
-    if isinstance(clocks, ClockSampler):
-        clocks.start()
     # K steps of the plain forward (the value) interleaved with K steps of the
     # forward with events around the dominant kernels (their live duration)
-    step_ms, timed_ms, gemv_ms_l, uniq = [], [], [], []
+    step_ms, timed_ms, kern_ms_l, uniq = [], [], [], []
     for i in range(args.steps):
         step_ms.append(one_step(g_plain, args.warmup + i)[0])
         ms_t, gm = one_step(g_timed, args.warmup + i, True)
         timed_ms.append(ms_t)
-        gemv_ms_l.append(gm)
+        kern_ms_l.append(gm)
         if isinstance(clocks, NvmlClocks):
             clocks.sample()
         uniq.append(int(torch.unique(ids_view).numel()))
     torch.cuda.synchronize(dev)
     dist_barrier(world)
-    clk = clocks.stop() if isinstance(clocks, ClockSampler) else clocks.result()
     capi.moe_read_device_status(ws, stream)
 
     # diagnostics (outside the timed region): every stage
-    stage_ms = [one_step(g_stages, i, "all")[1] for i in range(args.steps)]
+    stage_ms = [one_step(g_stages, i, "all")[1] for i in range(min(args.steps, 10))]
 
     # e2e: the public call with host buffers (pinned), copies inside the events
     xh = torch.empty((T, H), dtype=torch.bfloat16, pin_memory=True)
@@ -296,46 +301,191 @@ def run_ours(args, rank, world, local_rank):
         stream.synchronize()
         if i >= args.warmup:
             e2e_ms.append(e0.elapsed_time(e1))
+    capi.moe_read_device_status(ws, stream)
+    res = dict(wl=wl, inp=inp, prefill=prefill, ms=float(np.mean(step_ms)), timed_ms=float(np.mean(timed_ms)),
+               kern_ms=float(np.mean(kern_ms_l)), e2e_ms=float(np.mean(e2e_ms)),
+               stage_avg=np.mean(np.array(stage_ms), axis=0), U=float(np.mean(uniq)), n_spans=len(spans))
+    del g_timed, g_plain, g_stages
+    return res
 
-    ms = float(np.mean(step_ms))
-    stage_avg = np.mean(np.array(stage_ms), axis=0)
-    gemv_ms = float(np.mean(gemv_ms_l))
-    e2e = float(np.mean(e2e_ms))
-    ms_max = dist_max(world, ms, dev)
-    e2e_max = dist_max(world, e2e, dev)
-    gemv_ms = dist_max(world, gemv_ms, dev)
+
+def measure_dense(wl, args, rank, world, local_rank, dev, clocks=None):
+    """Time the dense BF16 FFN (dense_ffn_bf16) at hidden H, intermediate
+    dense_I over T tokens: K replays of its CUDA graph, L2 flushed before each."""
+    import torch
+    from routed_nvfp4_expert_b200 import capi
+    from routed_nvfp4_expert_b200 import synthetic as syn
+
+    d = syn.make_dense(wl)
+    T, H, I = wl.T, wl.H, wl.dense_I
+    wg, wu, wd = (capi.bf16_tensor(d[f"dense_{n}"], dev) for n in ("gate", "up", "down"))
+    x_pool = torch.stack([capi.bf16_tensor(syn.random_x(wl, T, seed=1000 * rank + i), dev) for i in range(4)])
+    x = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(capi.dense_ffn_workspace_size(H, I, T), dtype=torch.uint8, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.zeros((2 * l2 + (64 << 20)) // 8, dtype=torch.int64, device=dev)
+    flush_sink = torch.zeros((), dtype=torch.int64, device=dev)
+    stream = torch.cuda.Stream(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    x.copy_(x_pool[0])
+    with torch.cuda.stream(stream):
+        capi.dense_ffn_bf16(wl.limit, x, wg, wu, wd, y, ws, stream=stream)
+    stream.synchronize()
+    capi.moe_read_device_status(ws, stream)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        capi.dense_ffn_bf16(wl.limit, x, wg, wu, wd, y, ws, stream=stream)
+
+    def one(i):
+        with torch.cuda.stream(stream):
+            torch.sum(flush, dim=0, out=flush_sink)
+            x.copy_(x_pool[i % 4])
+            ev[0].record(stream)
+            g.replay()
+            ev[1].record(stream)
+        stream.synchronize()
+        return ev[0].elapsed_time(ev[1])
+
+    for i in range(args.warmup):
+        one(i)
+    dist_barrier(world)
+    ms = []
+    for i in range(args.steps):
+        ms.append(one(args.warmup + i))
+        if isinstance(clocks, NvmlClocks):
+            clocks.sample()
+    dist_barrier(world)
+    capi.moe_read_device_status(ws, stream)
+    del g
+    return dict(wl=wl, ms=float(np.mean(ms)))
+
+
+def dense_line(res, pk, world):
+    wl = res["wl"]
+    T, H, I = wl.T, wl.H, wl.dense_I
+    ms = res["ms"]
+    flops = 2.0 * T * 3 * H * I
+    if T >= 128:
+        achieved = flops / (ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "kernel": "bf16_gemm_kernel (tcgen05 kind::f16; gate/up + down launches)",
+                "achieved": round(achieved, 1), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(achieved / pk["bf16_tflops"], 4), "peak_source": f"{pk['source']} bf16 burst",
+                "algorithmic_flops_per_step": flops, "traffic": None}
+    else:
+        nbytes = 3 * H * I * 2
+        achieved = nbytes / (ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "kernel": "bf16_gemv_kernel (gate/up + down launches)", "achieved": round(achieved, 1),
+                "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4),
+                "peak_source": pk["source"], "algorithmic_bytes_per_step": nbytes, "traffic": None}
+    return {"workload": wl.name, "T": T, "hidden": H, "intermediate": I, "value": round(world * T / (ms * 1e-3), 2),
+            "unit": "tokens/s", "ms_per_step": round(ms, 5), "roofline": roof}
+
+
+def roofline_of(res, pk):
+    """The dominant kernels' roofline from measure()'s kernel time."""
+    wl = res["wl"]
+    T, H = wl.T, wl.H
+    if res["prefill"]:
+        flops = 2.0 * T * wl.k * 3 * H * wl.I          # gate + up + down over the T*k assignments
+        fp4_peak = pk["bf16_tflops"] * FP4_PER_BF16
+        achieved = flops / (res["kern_ms"] * 1e-3) / 1e12
+        return {"bound": "tensor", "kernel": "nvfp4_grouped_gemm (tcgen05 mxf4nvf4; gate/up + down launches)",
+                "achieved": round(achieved, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
+                "frac": round(achieved / fp4_peak, 4),
+                "peak_source": f"{pk['source']} bf16 burst x nominal FP4/BF16 ratio {FP4_PER_BF16:g}",
+                "algorithmic_flops_per_step": flops, "unique_experts_per_step": res["U"],
+                "traffic": read_traffic_profile(f"nvfp4_grouped_gemm_{wl.name}")}
+    routed = res["U"] * expert_bytes(wl)
+    if decode_t1_fused(wl):
+        # the single-token chain's expert launches: routed gate/up, then the
+        # routed down rows with the shared expert's down rows and the combine
+        shared_down = H * wl.Is * 2
+        algo = routed + shared_down
+        kernel = ("single-token expert launches: routed NVFP4 gate/up, routed NVFP4 down + shared BF16 down "
+                  "+ combine")
+    else:
+        shared_down = 0
+        algo = routed
+        kernel = "nvfp4_expert_gemv (gate/up + down launches, timed together)"
+    achieved = algo / (res["kern_ms"] * 1e-3) / 1e9
+    return {"bound": "hbm", "kernel": kernel, "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": round(achieved / pk["hbm_gbs"], 4), "peak_source": pk["source"],
+            "algorithmic_bytes_per_step": int(algo), "routed_expert_bytes_per_step": int(routed),
+            "shared_down_bytes_per_step": int(shared_down),
+            "routed_only_frac": round(routed / (res["kern_ms"] * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+            "unique_experts_per_step": res["U"], "bytes_per_expert": expert_bytes(wl),
+            "traffic": read_traffic_profile(f"nvfp4_expert_gemv_{wl.name}")}
+
+
+def launches_per_step(wl) -> int:
+    T = wl.T
+    if wl.kind != "decode":
+        # router, top-k, permute (hist, scan, scatter, first), tile rows, x
+        # encoding, gate/up GEMM, h encoding, down GEMM, shared gate/up + down,
+        # unpermute + combine
+        return 14
+    if decode_t1_fused(wl):
+        return 3
+    # router, top-k + plan (one launch up to 8 tokens at E <= 320, else top-k
+    # and the permute), expert gate/up, expert down, combine, and the shared
+    # expert's two GEMVs on the auxiliary stream
+    fused_plan = T <= 8 and wl.E <= 320 and T * wl.k <= 1024
+    return 7 if fused_plan else (8 if T * wl.k <= 1024 else 11)
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    from routed_nvfp4_expert_b200 import capi
+    from routed_nvfp4_expert_b200 import synthetic as syn
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = syn.WORKLOADS[args.workload]
+    clocks = clock_sampler(local_rank)
+    if isinstance(clocks, ClockSampler):
+        clocks.start()
+    if wl.kind == "dense":
+        res = measure_dense(wl, args, rank, world, local_rank, dev, clocks)
+        clk = clocks.stop() if isinstance(clocks, ClockSampler) else clocks.result()
+        ms_max = dist_max(world, res["ms"], dev)
+        if rank != 0:
+            return None
+        res["ms"] = ms_max
+        line = dense_line(res, peaks(), world)
+        return {"metric": METRIC, "value": line["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": line["ms_per_step"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16 weights x bf16 activations, fp32 accumulate",
+                "data": "synthetic (seeded)",
+                "config": {"workload": wl.name, "T": wl.T, "hidden": wl.H, "intermediate": wl.dense_I,
+                           "path": "dense BF16 FFN", "parallelism": f"replicas x{world}",
+                           "l2": "flushed before every timed step (read of a 2x L2 buffer)",
+                           "graph": "CUDA graph of dense_ffn_bf16"},
+                "roofline": line["roofline"], "gpu_launches": 2 * args.steps, "clocks": clk,
+                "e2e": None}
+    res = measure(wl, args, rank, world, local_rank, dev, clocks)
+    # the prefill grouped GEMM under the same clock, in the same process
+    pre = None
+    if args.with_prefill and wl.kind == "decode":
+        pre = measure(syn.WORKLOADS[args.with_prefill], args, rank, world, local_rank, dev, clocks)
+    clk = clocks.stop() if isinstance(clocks, ClockSampler) else clocks.result()
+
+    ms_max = dist_max(world, res["ms"], dev)
+    e2e_max = dist_max(world, res["e2e_ms"], dev)
+    res["kern_ms"] = dist_max(world, res["kern_ms"], dev)
+    if pre is not None:
+        pre_ms = dist_max(world, pre["ms"], dev)
+        pre["kern_ms"] = dist_max(world, pre["kern_ms"], dev)
+        pre_e2e = dist_max(world, pre["e2e_ms"], dev)
     if rank != 0:
         return None
 
     pk = peaks()
-    U = float(np.mean(uniq))
-    if prefill:
-        flops = 2.0 * T * wl.k * 3 * H * wl.I          # gate + up + down over the T*k assignments
-        fp4_peak = pk["bf16_tflops"] * FP4_PER_BF16
-        achieved = flops / (gemv_ms * 1e-3) / 1e12
-        roofline = {"bound": "tensor", "kernel": "nvfp4_grouped_gemm (tcgen05 mxf4nvf4; gate/up + down launches)",
-                    "achieved": round(achieved, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
-                    "frac": round(achieved / fp4_peak, 4),
-                    "peak_source": f"{pk['source']} bf16 burst x nominal FP4/BF16 ratio {FP4_PER_BF16:g}",
-                    "algorithmic_flops_per_step": flops, "unique_experts_per_step": U,
-                    "traffic": read_traffic_profile(f"nvfp4_grouped_gemm_{wl.name}")}
-        launches_per_step = 14
-        path_name = "prefill grouped GEMM (W4A4, tcgen05 block-scaled FP4)"
-    else:
-        algo_bytes = U * expert_bytes(wl)
-        achieved = algo_bytes / (gemv_ms * 1e-3) / 1e9
-        roofline = {"bound": "hbm", "kernel": "nvfp4_expert_gemv (gate/up + down launches, timed together)",
-                    "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-                    "frac": round(achieved / pk["hbm_gbs"], 4), "peak_source": pk["source"],
-                    "algorithmic_bytes_per_step": int(algo_bytes), "unique_experts_per_step": U,
-                    "bytes_per_expert": expert_bytes(wl),
-                    "traffic": read_traffic_profile(f"nvfp4_expert_gemv_{wl.name}")}
-        # router, top-k + plan (one launch up to 8 tokens at E <= 320, else
-        # top-k and the permute), expert gate/up, expert down, combine, and the
-        # shared expert's two GEMVs on the auxiliary stream
-        fused_plan = T <= 8 and wl.E <= 320 and T * wl.k <= 1024
-        launches_per_step = 7 if fused_plan else (8 if T * wl.k <= 1024 else 11)
-        path_name = "decode GEMV (W4A16)"
+    T, H = wl.T, wl.H
+    prefill = res["prefill"]
+    path_name = ("prefill grouped GEMM (W4A4, tcgen05 block-scaled FP4)" if prefill else
+                 "decode, single-token chain (W4A16 GEMV)" if decode_t1_fused(wl) else "decode GEMV (W4A16)")
+    n_launch = launches_per_step(wl)
     out = {
         "metric": METRIC,
         "value": round(world * T / (ms_max * 1e-3), 2),
@@ -348,28 +498,41 @@ def run_ours(args, rank, world, local_rank):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": ("nvfp4 weights x nvfp4 activations (tcgen05 mxf4nvf4), fp32 accumulate" if prefill
-                  else "nvfp4 weights x bf16 activations, fp32 accumulate"),
+                  else "nvfp4 weights x bf16 activations, exact products, fp32 accumulate"),
         "data": "synthetic (seeded; NVFP4 experts drawn in the code domain)",
         "config": {"workload": wl.name, "T": T, "hidden": H, "experts": wl.E, "intermediate": wl.I, "top_k": wl.k,
                    "shared_intermediate": wl.Is, "path": path_name, "parallelism": f"replicas x{world}",
                    "l2": "flushed before every timed step (read of a 2x L2 buffer)", "graph": "CUDA graph of moe_forward"},
         "diagnostics": {
-            "ms_per_step_with_stage_events": round(float(np.mean(timed_ms)), 5),
-            "stages_ms_all_events": {n: round(float(v), 5) for n, v in zip(capi.STAGES, stage_avg)},
+            "ms_per_step_with_stage_events": round(res["timed_ms"], 5),
+            "stages_ms_all_events": {n: round(float(v), 5) for n, v in zip(capi.STAGES, res["stage_avg"])},
             "note": f"value: K replays of the forward's graph; interleaved with them in the timed region, K "
-                    f"replays of the same forward with {2 * len(spans)} event nodes around the dominant "
+                    f"replays of the same forward with {2 * res['n_spans']} event nodes around the dominant "
                     "kernels give roofline.achieved (an event node also ends the launch overlap of the "
                     "kernels it separates); stages_ms_all_events comes from a graph with an event node at "
                     "every stage boundary"},
-        "roofline": roofline,
+        "roofline": roofline_of(res, pk),
         "e2e": {"value": round(world * T / (e2e_max * 1e-3), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2,
                 "ms_per_step": round(e2e_max, 5)},
-        "gpu_launches": 2 * launches_per_step * args.steps,   # both graphs of the timed region
+        "gpu_launches": 2 * n_launch * args.steps,   # both graphs of the timed region
         "clocks": clk,
     }
+    if pre is not None:
+        pwl = pre["wl"]
+        out["prefill"] = {
+            "workload": pwl.name, "T": pwl.T, "value": round(world * pwl.T / (pre_ms * 1e-3), 2), "unit": "tokens/s",
+            "ms_per_step": round(pre_ms, 5), "roofline": roofline_of(pre, pk),
+            "e2e": {"value": round(world * pwl.T / (pre_e2e * 1e-3), 2), "unit": "tokens/s",
+                    "h2d_bytes_per_step": pwl.T * pwl.H * 2, "d2h_bytes_per_step": pwl.T * pwl.H * 2,
+                    "ms_per_step": round(pre_e2e, 5)},
+            "stages_ms_all_events": {n: round(float(v), 5) for n, v in zip(capi.STAGES, pre["stage_avg"])},
+            "gpu_launches": 2 * launches_per_step(pwl) * args.steps,
+            "note": "timed in the same process and under the same clock record as the decode line, after it",
+        }
+        out["gpu_launches"] += out["prefill"]["gpu_launches"]
     if not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(wl, inp, budget_s=args.cpu_seconds)
+        out["cpu_baseline"] = cpu_baseline(wl, res["inp"], budget_s=args.cpu_seconds)
     return out
 
 
@@ -483,6 +646,8 @@ def main():
     ap.add_argument("--workload", default="decode_t1")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--with-prefill", default="prefill_t4096",
+                    help="after a decode workload, also time this prefill workload in the same run ('' = off)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

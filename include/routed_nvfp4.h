@@ -36,9 +36,9 @@
  *    frees no device memory and keeps no state besides a thread-local error
  *    message, the thread-local stage-timing events of moe_set_stage_events()
  *    and, per host thread and device, the auxiliary stream and event pair on
- *    which the decode forward runs the shared expert concurrently (created by
- *    the first decode moe_forward on that thread and device: make it before
- *    any stream capture).
+ *    which the decode forward with T > 1 runs the shared expert concurrently
+ *    (created by the first such call on that thread and device: make it before
+ *    any stream capture on that thread).
  *  - bf16 tensors are passed as uint16_t bit patterns.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream). Every call is
  *    stream-ordered and asynchronous; nothing synchronises except
@@ -73,8 +73,9 @@ typedef enum {
 
 /* Which implementation of the routed experts moe_forward runs. */
 typedef enum {
-  MOE_PATH_DECODE = 0,  /* W4A16 GEMV: bf16 activations x NVFP4 weights */
-  MOE_PATH_PREFILL = 1  /* W4A4 grouped GEMM on tcgen05 block-scaled FP4 */
+  MOE_PATH_DECODE = 0,         /* W4A16 GEMV: bf16 activations x NVFP4 weights */
+  MOE_PATH_PREFILL = 1,        /* W4A4 grouped GEMM on tcgen05 block-scaled FP4 */
+  MOE_PATH_PREFILL_W4A16 = 2   /* W4A16 grouped GEMM on tcgen05 kind::f16 (the pages' prefill) */
 } moe_path_t;
 
 /* Projection selector of the expert kernels. */
@@ -196,18 +197,20 @@ size_t moe_prepared_size(const moe_config_t* cfg);
 
 /*
  * Re-tile the experts' block scales for the prefill path. dst (device,
- * 256-byte aligned, moe_prepared_size() bytes) receives, for gate, then up,
- * then down, the scales of each expert as atoms [rows/128][K/64][512]: the
- * scale of row m, 16-element block b of atom (m/128, b/4) sits at byte
- * (m%32)*16 + ((m%128)/32)*4 + b%4 (32 lanes x 4 columns x 4 blocks, the
- * layout the 32x128b tensor-memory copy spreads over the four lane
- * quadrants). Requires I % 128 == 0 and H % 256 == 0. Codes are used in
- * place. Then the router weight w fp32 [E, H] as w3 bf16 [E, 3H] = (lo | mid |
- * hi) per row with w = hi + mid + lo exactly (hi: w with the low 16 bits of
- * its encoding cleared; mid: the same applied to w - hi; lo = w - hi - mid),
- * so the prefill's router logits run as one bf16 tensor-core GEMM over K = 3H
- * whose products are exact in the fp32 accumulator. Run once per weight set;
- * stream-ordered.
+ * 256-byte aligned, moe_prepared_size() bytes) receives 512-byte scale atoms
+ * of 128 rows x 4 K blocks of 16: the scale of atom row m, 16-element block b
+ * sits at byte (m%32)*16 + ((m%128)/32)*4 + b%4 of atom (m/128, b/4) (32 lanes
+ * x 4 columns x 4 blocks, the layout the 32x128b tensor-memory copy spreads
+ * over the four lane quadrants). First gate and up interleaved, atoms
+ * [E][I/64][H/64][512] whose 128 rows are gate rows 64 j .. 64 j + 63 then up
+ * rows 64 j .. 64 j + 63 of the expert (one N = 128 tile of the gate/up
+ * GEMM); then down, atoms [E][H/128][I/64][512]. Requires I % 128 == 0 and
+ * H % 256 == 0. Codes are used in place. Then the router weight w fp32 [E, H]
+ * as w3 bf16 [E, 3H] = (lo | mid | hi) per row with w = hi + mid + lo exactly
+ * (hi: w with the low 16 bits of its encoding cleared; mid: the same applied
+ * to w - hi; lo = w - hi - mid), so the prefill's router logits run as one
+ * bf16 tensor-core GEMM over K = 3H whose products are exact in the fp32
+ * accumulator. Run once per weight set; stream-ordered.
  */
 moe_status_t moe_prepare_weights(const moe_config_t* cfg, const moe_weights_t* w, void* dst, size_t dst_bytes,
                                  void* stream);
@@ -243,22 +246,29 @@ moe_status_t moe_permute(const moe_config_t* cfg, const int32_t* ids, int32_t T,
 /*
  * Decode expert projections (the module list's W4A16 GEMV: "Every
  * routed-expert projection here is M=1"): bf16 activations times NVFP4
- * weights, fp32 accumulation, one pass over each touched expert's bytes for
- * all of that expert's tokens.
- *   MOE_PROJ_GATE_UP: act = x bf16 [T, H]; out = h bf16 [T*k, I] with
+ * weights, one pass over each touched expert's bytes for all of that expert's
+ * tokens. Every product code * activation is exact (the code as f16, the
+ * activation scaled by a power of two per row into f16) and accumulates in
+ * fp32; each 16-element block sum is scaled by its E4M3 scale in fp32.
+ *   MOE_PROJ_GATE_UP: act = x bf16 [T, H]; out = h fp32 [T*k, I] with
  *       h[a] = clamped_swiglu(gate_e . x_t, up_e . x_t) for assignment
  *       a = t*k + j of LOCAL expert e = ids[t, j]; rows of remote
  *       assignments are not written. `weights` is ignored (may be NULL).
- *   MOE_PROJ_DOWN: act = h bf16 [T*k, I]; out = r bf16 [T*k, H] with
+ *   MOE_PROJ_DOWN: act = h fp32 [T*k, I] (h enters the products rounded to
+ *       11 significant bits); out = r fp32 [T*k, H] with
  *       r[a] = weights[a] * (down_e . h[a]); rows of remote assignments are
  *       written as zeros.
  *   plan: from moe_permute (or moe_forward) for the same ids.
  *   ws:   workspace of at least moe_workspace_size(cfg, T, MOE_PATH_DECODE)
- *         bytes (status word and per-row activation maxima).
+ *         bytes (status word, activation maximum).
+ * T = 1 runs the streamed single-token kernels (one CTA per SM, weights
+ * through a ring of bulk copies in shared memory); larger T a work-item loop
+ * over (active expert, block of rows) that applies each weight row to up to 8
+ * of the expert's tokens at once.
  */
-moe_status_t nvfp4_expert_gemv(const moe_config_t* cfg, int32_t proj, const uint16_t* act, int32_t T,
+moe_status_t nvfp4_expert_gemv(const moe_config_t* cfg, int32_t proj, const void* act, int32_t T,
                                const moe_plan_t* plan, const float* weights,
-                               const moe_weights_t* w, uint16_t* out, void* ws, size_t ws_bytes, void* stream);
+                               const moe_weights_t* w, float* out, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * NVFP4 encoding of activation rows for the prefill (the reading of the
@@ -295,13 +305,41 @@ moe_status_t nvfp4_quantize_rows(const uint16_t* src, int32_t rows, int32_t K, u
  *   Requires w->prepared, I % 128 == 0, H % 256 == 0.
  *   ws: at least moe_workspace_size(cfg, T, MOE_PATH_PREFILL) bytes (status).
  * The kernel runs on clusters of two CTAs (tcgen05.mma.cta_group::2, 256 x
- * 256 tiles, M split across the pair, each CTA loading half of the weight
- * tile); no TMA load uses cluster multicast.
+ * 128 tiles, M split across the pair, each CTA loading half of the weight
+ * tile, two TMEM accumulators alternating between tiles); no TMA load uses
+ * cluster multicast.
  */
 moe_status_t nvfp4_grouped_gemm(const moe_config_t* cfg, int32_t proj, const uint8_t* act_codes,
                                 const uint8_t* act_sf, const float* act_scale, int32_t T, const moe_plan_t* plan,
                                 const float* weights, const moe_weights_t* w, uint16_t* out, void* ws,
                                 size_t ws_bytes, void* stream);
+
+/*
+ * Prefill expert projections in the pages' own numerics (the glm5next_mlp
+ * module docs' forward_prefill_gemm: "the shared tensor-core grouped W4A16
+ * GEMM"): NVFP4 weights x 16-bit activations on tcgen05 kind::f16, fp32
+ * accumulation. The weights are dequantised in shared memory, each element
+ * e2m1 x e4m3 exact in f16; the tensor scale is applied in the epilogue. The
+ * A operand is f16 in the padded tile layout of plan.tile_rows, P =
+ * moe_padded_rows(cfg, T) rows, padding rows zero:
+ *   MOE_PROJ_GATE_UP (K = H): act = x rows, each scaled by a power of two
+ *       (moe_forward's gather: max |x| into [2^14, 2^15), exact for bf16 x),
+ *       act_scale fp32 [P] the inverse; out = h f16 [P, I] =
+ *       clamped_swiglu(g, u) (saturating to the f16 range; 0 on padding rows);
+ *       `weights` unused.
+ *   MOE_PROJ_DOWN (K = I): act = h f16 [P, I]; act_scale NULL (1); out = rows
+ *       bf16 [P, H] in the padded tile order, rows[p] = weights[a] *
+ *       (down_e . h[p]) (0 on padding rows); moe_unpermute(_combine) brings
+ *       them back to token order.
+ *   Requires w->prepared (the interleaved gate/up and the down scale atoms),
+ *   I % 128 == 0, H % 256 == 0. ws: at least moe_workspace_size(cfg, T,
+ *   MOE_PATH_PREFILL_W4A16) bytes (status word).
+ * One CTA per 128-row x 256-weight-row tile, 148 persistent CTAs, two TMEM
+ * accumulators; no TMA load uses cluster multicast.
+ */
+moe_status_t nvfp4_grouped_gemm_w4a16(const moe_config_t* cfg, int32_t proj, const uint16_t* act,
+                                      const float* act_scale, int32_t T, const moe_plan_t* plan, const float* weights,
+                                      const moe_weights_t* w, uint16_t* out, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Unpermute (the module list's moe_permute family: token sort / permute /
@@ -340,15 +378,24 @@ moe_status_t moe_combine(int32_t T, int32_t k, int32_t H, const uint16_t* r, con
                          uint16_t* y, void* stream);
 
 /*
+ * moe_combine over fp32 partials (the decode path keeps the routed rows and
+ * the shared row in fp32 until this one rounding): the same order and
+ * arithmetic as moe_combine. r fp32 [T, k, H]; shared fp32 [T, H] or NULL;
+ * y bf16 [T, H]; H a multiple of 4.
+ */
+moe_status_t moe_combine_f32(int32_t T, int32_t k, int32_t H, const float* r, const float* shared,
+                             uint16_t* y, void* stream);
+
+/*
  * Dense BF16 FFN (glm5next_mlp, DENSE layers; also the shared expert):
  *   y = down_proj( clamped_swiglu(gate_proj x, up_proj x) )
  *   x bf16 [T, H]; wg, wu bf16 [I, H]; wd bf16 [H, I]; y bf16 [T, H].
- *   fp32 accumulation; h is rounded to bf16 between the two projections.
- *   H and I multiples of 64. ws: at least dense_ffn_workspace_size(H, I, T);
- *   its first 4 bytes are a device status word (moe_read_device_status).
- *   T >= 128 with I % 128 == 0 and H % 256 == 0 runs as two tcgen05 BF16
- *   GEMMs (kind::f16), smaller T as a GEMV that streams the weights once per
- *   group of up to 8 tokens.
+ *   fp32 accumulation. T >= 128 with I % 128 == 0 and H % 256 == 0 runs as
+ *   two tcgen05 BF16 GEMMs (kind::f16; h is rounded to bf16, the second
+ *   GEMM's operand type); smaller T as a GEMV that streams the weights once
+ *   per group of up to 8 tokens and keeps h in fp32. H and I multiples of 64.
+ *   ws: at least dense_ffn_workspace_size(H, I, T); its first 4 bytes are a
+ *   device status word (moe_read_device_status).
  */
 size_t dense_ffn_workspace_size(int32_t H, int32_t I, int32_t T);
 moe_status_t dense_ffn_bf16(int32_t H, int32_t I, float limit, const uint16_t* x, int32_t T,
@@ -371,12 +418,27 @@ moe_status_t nvfp4_dequant(const uint8_t* codes, const uint8_t* scales, const fl
  * combine. x bf16 [T, H] -> y bf16 [T, H]. ws: moe_workspace_size(cfg, T,
  * path) bytes. The routing plan, logits, ids and weights of the call stay in
  * the workspace until the next call (see moe_workspace_views).
- *   MOE_PATH_DECODE: W4A16 GEMV experts (nvfp4_expert_gemv); with up to 8
- *     tokens (E <= 320) top-k and the routing plan are one launch; router,
- *     top-k, plan, the two expert GEMVs and the combine are chained by
- *     programmatic dependent launch; the shared expert runs on the library's
- *     auxiliary stream of this host thread and device, forked from and joined
- *     back into `stream` with events.
+ *   MOE_PATH_DECODE: W4A16 GEMV experts (nvfp4_expert_gemv) with h, the
+ *     routed rows r and the shared row kept in fp32 up to the combine's one
+ *     bf16 rounding.
+ *     T = 1 (H % 256 == 0, H <= 8192, I <= 2048, k <= 16, E <= 1024): three
+ *     launches chained by programmatic dependent launch -- (1) router logits,
+ *     with the top-k and the routing plan run by the last router CTA to
+ *     finish, and the shared expert's gate/up in the same grid; (2) the routed
+ *     experts' gate/up, one CTA per SM streaming weights through a ring of bulk
+ *     copies; (3) each CTA a block of output rows: the routed and shared down
+ *     rows of that block and the combine. No auxiliary stream.
+ *     T > 1: router; top-k with the routing plan (one launch up to 8 tokens,
+ *     E <= 320); the two expert GEMVs; moe_combine_f32; the launches are
+ *     chained by programmatic dependent launch; the shared expert runs on the
+ *     library's auxiliary stream of this host thread and device, forked from
+ *     and joined back into `stream` with events.
+ *   MOE_PATH_PREFILL_W4A16: the pages' prefill numerics: permute with the
+ *     padded tile layout, x gathered to f16 rows (per-row power-of-two scale),
+ *     grouped W4A16 GEMM gate/up (nvfp4_grouped_gemm_w4a16) with the clamped
+ *     SwiGLU, h in f16, grouped W4A16 GEMM down with the routing weight,
+ *     unpermute fused with the combine; needs w->prepared, I % 128 == 0,
+ *     H % 256 == 0.
  *   MOE_PATH_PREFILL: permute with the padded tile layout, x encoded to
  *     NVFP4 per token row and written to its assignments' padded rows (the
  *     bytes nvfp4_quantize_rows gives per assignment row), grouped GEMM
@@ -388,20 +450,20 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
                          int32_t path, uint16_t* y, void* ws, size_t ws_bytes, void* stream);
 
 /* Device pointers (inside ws) of the intermediates moe_forward leaves behind:
- * logits fp32 [T,E], ids int32 [T,k], weights fp32 [T,k], the plan, h bf16
- * ([T*k, I] on the decode path, [P, I] in padded tile rows on the prefill
- * path), r bf16 (decode: [T*k, H] in token order; prefill: [P, H] in the
- * padded tile order), shared bf16 [T, H] (NULL when Is == 0), and on the
- * prefill path the NVFP4-encoded x and h in padded tile rows (codes, scale
+ * logits fp32 [T,E], ids int32 [T,k], weights fp32 [T,k], the plan; h (decode:
+ * fp32 [T*k, I]; prefill: bf16 [P, I] in padded tile rows); r (decode: fp32
+ * [T*k, H] in token order; prefill: bf16 [P, H] in the padded tile order);
+ * shared (decode: fp32 [T, H]; prefill: bf16 [T, H]; NULL when Is == 0); and on
+ * the prefill path the NVFP4-encoded x and h in padded tile rows (codes, scale
  * atoms, row scales; NULL on the decode path). Host-only pointer arithmetic. */
 typedef struct {
   float* logits;
   int32_t* ids;
   float* weights;
   moe_plan_t plan;
-  uint16_t* h;
-  uint16_t* r;
-  uint16_t* shared;
+  void* h;
+  void* r;
+  void* shared;
   uint8_t* xq_codes;
   uint8_t* xq_sf;
   float* xq_scale;
@@ -437,6 +499,20 @@ typedef enum {
 } moe_stage_t;
 moe_status_t moe_set_stage_events(void* const* events, int32_t n);
 
+/*
+ * Test hook of the failure path (not for production use; process-wide host
+ * setting read at launch): the limit of the main-loop waits of the BF16
+ * tensor-core GEMM (dense_ffn_bf16 / the shared expert at T >= 128, the
+ * prefill router). ns >= 0 sets it (0 = a wait gives up as soon as it finds
+ * the awaited copy or MMA still in flight); ns < 0 restores the default 2 s.
+ * A wait that runs out sets MOE_ERR_DEVICE_TIMEOUT in the status word; the
+ * kernel then issues nothing more, waits with the default limit for every copy
+ * and MMA it already issued, frees its tensor memory and returns, so later
+ * calls on the device run normally. The outputs of the failed call are
+ * unspecified.
+ */
+moe_status_t moe_set_wait_limit(int64_t ns);
+
 /* Synchronises `stream`, reads the workspace status word, clears it, and
  * returns MOE_ERR_DEVICE_TIMEOUT / MOE_ERR_DEVICE_BOUNDS / MOE_OK. */
 moe_status_t moe_read_device_status(void* ws, void* stream);
@@ -456,14 +532,27 @@ const char* moe_last_error(void);
  * (moe_workspace_size(cfg, T, MOE_PATH_DECODE) > 8 MiB) fail with
  * MOE_ERR_WORKSPACE before touching the device. The first call on each device
  * looks up the buffer's device address (cudaGetSymbolAddress, with that device
- * current); make that first call before any stream capture on the device. All
- * calls on a device share the buffer, which keeps the previous call's
- * contents; calls whose GPU work overlaps in time (two streams, two host
- * threads) race on it and must be serialised by the caller. Allocates nothing
- * (no cudaMalloc / cudaFree). The routing intermediates are not exposed.
+ * current) and caches it for the life of the process: make that first call
+ * before any stream capture on the device, and make no call on a device after
+ * cudaDeviceReset() of it (the cached address would be stale). All calls on a
+ * device share the buffer, which keeps the previous call's contents; calls
+ * whose GPU work overlaps in time (two streams, two host threads) race on it
+ * and must be serialised by the caller. Allocates nothing (no cudaMalloc /
+ * cudaFree). The routing intermediates are not exposed.
  */
 moe_status_t moe_forward_decode_noalloc(const moe_config_t* cfg, const moe_weights_t* w, const uint16_t* x,
                                         int32_t T, uint16_t* y, void* stream);
+
+/*
+ * Device-side errors of the last moe_forward_decode_noalloc call on the
+ * current device (an id out of range, a bounded wait that ran out): the status
+ * word sits at the start of the library's scratch buffer, where a caller has no
+ * pointer to it. Synchronises `stream`, reads and clears the word, and returns
+ * MOE_ERR_DEVICE_TIMEOUT / MOE_ERR_DEVICE_BOUNDS / MOE_OK, as
+ * moe_read_device_status does for a caller's workspace. The next
+ * moe_forward_decode_noalloc call clears the word as well.
+ */
+moe_status_t moe_noalloc_read_device_status(void* stream);
 
 #ifdef __cplusplus
 }

@@ -19,7 +19,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librouted_
 MOE_OK = 0
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
                 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_TIMEOUT", 6: "MOE_ERR_DEVICE_BOUNDS"}
-PATH_DECODE, PATH_PREFILL = 0, 1
+PATH_DECODE, PATH_PREFILL, PATH_PREFILL_W4A16 = 0, 1, 2
 PROJ_GATE_UP, PROJ_DOWN = 0, 1
 
 # every symbol include/routed_nvfp4.h declares
@@ -29,6 +29,7 @@ EXPORTED = (
     "nvfp4_dequant", "moe_forward", "moe_workspace_views", "moe_read_device_status", "moe_last_error",
     "moe_set_stage_events", "moe_forward_decode_noalloc", "moe_padded_rows", "moe_prepared_size",
     "moe_prepare_weights", "nvfp4_quantize_rows", "nvfp4_grouped_gemm", "moe_unpermute", "moe_unpermute_combine",
+    "moe_combine_f32", "moe_noalloc_read_device_status", "moe_set_wait_limit", "nvfp4_grouped_gemm_w4a16",
 )
 STAGES = ("router_logits", "topk", "permute", "act_quant", "expert_gate_up", "h_quant", "expert_down", "shared",
           "combine")
@@ -85,6 +86,7 @@ def load_library(path: str = _LIB_PATH) -> C.CDLL:
         "nvfp4_expert_gemv": (st, [cfgp, i32, vp, i32, C.POINTER(MoePlan), vp, C.POINTER(MoeWeights), vp, vp, sz, vp]),
         "clamped_swiglu": (st, [vp, i32, i32, C.c_float, vp, vp]),
         "moe_combine": (st, [i32, i32, i32, vp, vp, vp, vp]),
+        "moe_combine_f32": (st, [i32, i32, i32, vp, vp, vp, vp]),
         "dense_ffn_workspace_size": (sz, [i32, i32, i32]),
         "dense_ffn_bf16": (st, [i32, i32, C.c_float, vp, i32, vp, vp, vp, vp, vp, sz, vp]),
         "nvfp4_dequant": (st, [vp, vp, vp, i32, i32, vp, vp]),
@@ -94,6 +96,10 @@ def load_library(path: str = _LIB_PATH) -> C.CDLL:
         "moe_last_error": (C.c_char_p, []),
         "moe_set_stage_events": (st, [C.POINTER(C.c_void_p), i32]),
         "moe_forward_decode_noalloc": (st, [cfgp, C.POINTER(MoeWeights), vp, i32, vp, vp]),
+        "moe_noalloc_read_device_status": (st, [vp]),
+        "moe_set_wait_limit": (st, [C.c_int64]),
+        "nvfp4_grouped_gemm_w4a16": (st, [cfgp, i32, vp, vp, i32, C.POINTER(MoePlan), vp, C.POINTER(MoeWeights), vp,
+                                          vp, sz, vp]),
         "moe_padded_rows": (C.c_int64, [cfgp, i32]),
         "moe_prepared_size": (sz, [cfgp]),
         "moe_prepare_weights": (st, [cfgp, C.POINTER(MoeWeights), vp, sz, vp]),
@@ -246,8 +252,11 @@ def clamped_swiglu(gu, limit: float, h, stream=None):
 
 
 def moe_combine(r, shared, y, stream=None):
+    """bf16 rows r [T, k, H] (+ bf16 shared [T, H] or None) -> y bf16; fp32
+    rows (and an fp32 shared row) go through moe_combine_f32."""
     T, k, H = r.shape
-    _check(lib().moe_combine(T, k, H, _p(r), _p(shared), _p(y), _stream(stream)))
+    fn = lib().moe_combine_f32 if r.dtype == torch.float32 else lib().moe_combine
+    _check(fn(T, k, H, _p(r), _p(shared), _p(y), _stream(stream)))
 
 
 def dense_ffn_workspace_size(H: int, I: int, T: int) -> int:
@@ -278,6 +287,12 @@ def moe_forward_decode_noalloc(cfg: SiteConfig, site: DeviceSite, x, y, stream=N
     w = site.c()
     _check(lib().moe_forward_decode_noalloc(C.byref(cfg.c()), C.byref(w), _p(x), x.shape[0], _p(y),
                                             _stream(stream)))
+
+
+def moe_noalloc_read_device_status(stream=None):
+    """Device-side errors of the last moe_forward_decode_noalloc call on the
+    current device (reads and clears the status word of the library's scratch)."""
+    _check(lib().moe_noalloc_read_device_status(_stream(stream)))
 
 
 def moe_padded_rows(cfg: SiteConfig, T: int) -> int:
@@ -312,6 +327,13 @@ def nvfp4_grouped_gemm(cfg: SiteConfig, proj: int, act_codes, act_sf, act_scale,
                                     _stream(stream)))
 
 
+def nvfp4_grouped_gemm_w4a16(cfg: SiteConfig, proj: int, act, act_scale, T: int, plan: MoePlan, weights,
+                             site: DeviceSite, out, ws, stream=None):
+    w = site.c()
+    _check(lib().nvfp4_grouped_gemm_w4a16(C.byref(cfg.c()), proj, _p(act), _p(act_scale), T, C.byref(plan),
+                                          _p(weights), C.byref(w), _p(out), _p(ws), ws.numel(), _stream(stream)))
+
+
 def moe_unpermute(cfg: SiteConfig, rows, T: int, plan: MoePlan, ids, out, stream=None):
     _check(lib().moe_unpermute(C.byref(cfg.c()), _p(rows), T, C.byref(plan), _p(ids), _p(out), _stream(stream)))
 
@@ -336,6 +358,12 @@ def moe_set_stage_events(events):
         return
     arr = (C.c_void_p * len(events))(*[(e.cuda_event if e is not None else None) for e in events])
     _check(lib().moe_set_stage_events(arr, len(events)))
+
+
+def moe_set_wait_limit(ns: int):
+    """Test hook: limit of the BF16 tensor-core GEMM's main-loop waits (ns < 0
+    restores the default)."""
+    _check(lib().moe_set_wait_limit(int(ns)))
 
 
 def moe_read_device_status(ws, stream=None):

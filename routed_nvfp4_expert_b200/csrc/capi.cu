@@ -10,6 +10,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tma.cuh"
 
 namespace {
 
@@ -32,10 +33,19 @@ cudaError_t side_stream(SideStream** out) {
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   SideStream& s = g_side[dev];
-  if (!s.st) {
-    if ((e = cudaStreamCreateWithFlags(&s.st, cudaStreamNonBlocking)) != cudaSuccess) return e;
-    if ((e = cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
-    if ((e = cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming)) != cudaSuccess) return e;
+  if (!s.st || !s.fork || !s.join) {
+    // all three handles or none: a partial creation is undone and reported
+    SideStream n;
+    e = cudaStreamCreateWithFlags(&n.st, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&n.fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&n.join, cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+      if (n.join) cudaEventDestroy(n.join);
+      if (n.fork) cudaEventDestroy(n.fork);
+      if (n.st) cudaStreamDestroy(n.st);
+      return e;
+    }
+    s = n;
   }
   *out = &s;
   return cudaSuccess;
@@ -165,33 +175,42 @@ moe_plan_t plan_at(char* base, const PlanLayout& L) {
 }
 
 struct WsLayout {
-  size_t status, logits, ids, weights, plan, scratch, h, r, shared_h, shared, xmax, hmax;
+  size_t status, logits, ids, weights, plan, scratch, h, r, shared_h, shared, xmax;
   size_t xq, xsf, xts, hq, hsf, hts;   // prefill: NVFP4 x and h in padded tile rows
   size_t bytes;
   PlanLayout pl;
 };
+
+// Control block at the start of every workspace, cleared at the start of each
+// call that uses it: the device status word, then the single-token router's
+// arrival counter.
+constexpr size_t kCtrlBytes = 16;
 
 WsLayout ws_layout(const moe_config_t* c, int T, int path) {
   WsLayout L{};
   const int E = c->num_experts, k = c->top_k, H = c->hidden, I = c->intermediate, Is = c->shared_intermediate;
   const size_t A = (size_t)T * k;
   size_t o = 0;
-  L.status = o; o = up(o + 4);
+  L.status = o; o = up(o + kCtrlBytes);
   L.logits = o; o = up(o + 4 * (size_t)T * E);
   L.ids = o; o = up(o + 4 * A);
   L.weights = o; o = up(o + 4 * A);
   L.pl = plan_layout(c, (int)A);
   L.plan = o; o = up(o + L.pl.bytes);
   L.scratch = o; o = up(o + 4 * rnx::permute_scratch_ints((int)A, E));
-  const bool pre = path == MOE_PATH_PREFILL;
+  const bool w4 = path == MOE_PATH_PREFILL_W4A16;
+  const bool pre = path == MOE_PATH_PREFILL || w4;
   const size_t P = (size_t)L.pl.P;
-  L.h = o; o = up(o + 2 * (pre ? P : A) * I);
-  L.r = o; o = up(o + 2 * (pre ? P : A) * H);   // prefill: down rows in the padded tile order
-  L.shared_h = o; o = up(o + 2 * (size_t)T * Is);
-  L.shared = o; o = up(o + 2 * (size_t)T * H);
+  // decode keeps h, r and the shared row in fp32; the prefill's are 16-bit
+  L.h = o; o = up(o + (pre ? 2 * P : 4 * A) * I);
+  L.r = o; o = up(o + (pre ? 2 * P : 4 * A) * H);   // prefill: down rows in the padded tile order
+  L.shared_h = o; o = up(o + 4 * (size_t)T * Is);
+  L.shared = o; o = up(o + (pre ? 2 : 4) * (size_t)T * H);
   L.xmax = o; o = up(o + 4 * (size_t)T);
-  L.hmax = o; o = up(o + 4 * (size_t)A);     // h maxima [A]
-  if (pre) {
+  if (w4) {                                   // x as f16 rows in the padded tile order, their unscales
+    L.xq = o; o = up(o + P * H * 2);
+    L.xts = o; o = up(o + 4 * P);
+  } else if (pre) {
     L.xq = o; o = up(o + P * H / 2);
     L.xsf = o; o = up(o + P * H / 16);
     L.xts = o; o = up(o + 4 * P);
@@ -210,15 +229,17 @@ moe_status_t check_prefill_shape(const moe_config_t* c) {
   return MOE_OK;
 }
 
-// Prepared weights: the experts' block scales as 512-byte atoms (gate, up,
-// down), then the router weight split exactly into three bf16 terms [E, 3H].
+// Prepared weights: the experts' block scales as 512-byte atoms -- gate and
+// up interleaved (each 128-row atom = 64 gate rows, then the same 64 up rows),
+// then down -- and the router weight split exactly into three bf16 terms
+// [E, 3H].
 struct PreparedLayout {
-  size_t gate, up, down, router3, bytes;
+  size_t gate_up, down, router3, bytes;
 };
 PreparedLayout prepared_layout(const moe_config_t* c) {
   const size_t per = (size_t)c->num_experts * c->intermediate * c->hidden / 16;
   const size_t r3 = up(3 * per);
-  return PreparedLayout{0, per, 2 * per, r3, r3 + up((size_t)c->num_experts * 3 * c->hidden * 2)};
+  return PreparedLayout{0, 2 * per, r3, r3 + up((size_t)c->num_experts * 3 * c->hidden * 2)};
 }
 
 // Prefill router on the tensor cores (needs the prepared split and E % 4 == 0).
@@ -242,10 +263,38 @@ rnx::Fp4GemmArgs gemm_args(const moe_config_t* c, int proj, const uint8_t* codes
   g.a_sf = sf;
   g.row_scale = scale;
   if (g.gate_up) {
-    g.b0_codes = w->gate.codes; g.b0_sf = w->prepared + PL.gate; g.ts0 = w->gate.tensor_scale;
-    g.b1_codes = w->up.codes;   g.b1_sf = w->prepared + PL.up;   g.ts1 = w->up.tensor_scale;
+    g.b0_codes = w->gate.codes; g.b0_sf = w->prepared + PL.gate_up; g.ts0 = w->gate.tensor_scale;
+    g.b1_codes = w->up.codes;   g.b1_sf = nullptr;                   g.ts1 = w->up.tensor_scale;
   } else {
     g.b0_codes = w->down.codes; g.b0_sf = w->prepared + PL.down; g.ts0 = w->down.tensor_scale;
+  }
+  g.tile_offsets = plan.tile_offsets;
+  g.tile_rows = plan.tile_rows;
+  g.weights = weights;
+  g.out = out;
+  g.status = status;
+  return g;
+}
+
+rnx::W4a16GemmArgs w4a16_args(const moe_config_t* c, int proj, const uint16_t* act, const float* act_scale,
+                              int64_t P, const moe_plan_t& plan, const float* weights, const moe_weights_t* w,
+                              uint16_t* out, uint32_t* status) {
+  const PreparedLayout PL = prepared_layout(c);
+  rnx::W4a16GemmArgs g{};
+  g.gate_up = proj == MOE_PROJ_GATE_UP;
+  g.E = c->num_experts;
+  g.K = g.gate_up ? c->hidden : c->intermediate;
+  g.out_cols = g.gate_up ? c->intermediate : c->hidden;
+  g.bank_rows = g.gate_up ? c->intermediate : c->hidden;
+  g.P_max = P;
+  g.limit = c->swiglu_limit;
+  g.act = act;
+  g.row_scale = act_scale;
+  if (g.gate_up) {
+    g.b0_codes = w->gate.codes; g.b1_codes = w->up.codes; g.b_sf = w->prepared + PL.gate_up;
+    g.ts0 = w->gate.tensor_scale; g.ts1 = w->up.tensor_scale;
+  } else {
+    g.b0_codes = w->down.codes; g.b_sf = w->prepared + PL.down; g.ts0 = w->down.tensor_scale;
   }
   g.tile_offsets = plan.tile_offsets;
   g.tile_rows = plan.tile_rows;
@@ -282,7 +331,7 @@ moe_status_t moe_set_stage_events(void* const* events, int32_t n) {
 
 size_t moe_workspace_size(const moe_config_t* cfg, int32_t T, int32_t path) {
   if (check_cfg(cfg) != MOE_OK || check_T(T) != MOE_OK) return 0;
-  if (path != MOE_PATH_DECODE && path != MOE_PATH_PREFILL) {
+  if (path != MOE_PATH_DECODE && path != MOE_PATH_PREFILL && path != MOE_PATH_PREFILL_W4A16) {
     fail(MOE_ERR_INVALID_ARG, "unknown path %d", path);
     return 0;
   }
@@ -317,13 +366,13 @@ moe_status_t moe_workspace_views(const moe_config_t* cfg, int32_t T, int32_t pat
   v->ids = (int32_t*)(b + L.ids);
   v->weights = (float*)(b + L.weights);
   v->plan = plan_at(b + L.plan, L.pl);
-  v->h = (uint16_t*)(b + L.h);
-  v->r = (uint16_t*)(b + L.r);
-  v->shared = cfg->shared_intermediate > 0 ? (uint16_t*)(b + L.shared) : nullptr;
-  const bool pre = path == MOE_PATH_PREFILL;
-  v->xq_codes = pre ? (uint8_t*)(b + L.xq) : nullptr;
+  v->h = b + L.h;
+  v->r = b + L.r;
+  v->shared = cfg->shared_intermediate > 0 ? b + L.shared : nullptr;
+  const bool pre = path == MOE_PATH_PREFILL, w4 = path == MOE_PATH_PREFILL_W4A16;
+  v->xq_codes = pre || w4 ? (uint8_t*)(b + L.xq) : nullptr;   // W4A16: the f16 x rows
   v->xq_sf = pre ? (uint8_t*)(b + L.xsf) : nullptr;
-  v->xq_scale = pre ? (float*)(b + L.xts) : nullptr;
+  v->xq_scale = pre || w4 ? (float*)(b + L.xts) : nullptr;
   v->hq_codes = pre ? (uint8_t*)(b + L.hq) : nullptr;
   v->hq_sf = pre ? (uint8_t*)(b + L.hsf) : nullptr;
   v->hq_scale = pre ? (float*)(b + L.hts) : nullptr;
@@ -355,8 +404,8 @@ moe_status_t moe_prepare_weights(const moe_config_t* cfg, const moe_weights_t* w
   cudaStream_t st = (cudaStream_t)stream;
   uint8_t* d = (uint8_t*)dst;
   const int E = cfg->num_experts, H = cfg->hidden, I = cfg->intermediate;
-  RNX_CUDA(rnx::launch_sf_atoms(w->gate.scales, E, I, H, d + PL.gate, st), "prepare gate scales");
-  RNX_CUDA(rnx::launch_sf_atoms(w->up.scales, E, I, H, d + PL.up, st), "prepare up scales");
+  RNX_CUDA(rnx::launch_sf_atoms_gate_up(w->gate.scales, w->up.scales, E, I, H, d + PL.gate_up, st),
+           "prepare gate/up scales");
   RNX_CUDA(rnx::launch_sf_atoms(w->down.scales, E, H, I, d + PL.down, st), "prepare down scales");
   RNX_CUDA(rnx::launch_router_split(w->router_w, E, H, (uint16_t*)(d + PL.router3), st), "prepare router split");
   return MOE_OK;
@@ -411,6 +460,37 @@ moe_status_t nvfp4_grouped_gemm(const moe_config_t* cfg, int32_t proj, const uin
   return MOE_OK;
 }
 
+moe_status_t nvfp4_grouped_gemm_w4a16(const moe_config_t* cfg, int32_t proj, const uint16_t* act,
+                                      const float* act_scale, int32_t T, const moe_plan_t* plan, const float* weights,
+                                      const moe_weights_t* w, uint16_t* out, void* ws, size_t ws_bytes, void* stream) {
+  moe_status_t s;
+  if ((s = check_cfg(cfg)) != MOE_OK || (s = check_T(T)) != MOE_OK || (s = check_prefill_shape(cfg)) != MOE_OK)
+    return s;
+  if (proj != MOE_PROJ_GATE_UP && proj != MOE_PROJ_DOWN) return fail(MOE_ERR_INVALID_ARG, "unknown proj %d", proj);
+  if (T == 0) return MOE_OK;
+  RNX_PTR(act, "act");
+  RNX_PTR(out, "out");
+  if (act_scale && !aligned16(act_scale)) return fail(MOE_ERR_INVALID_ARG, "act_scale is not 16-byte aligned");
+  if (!plan || !w) return fail(MOE_ERR_INVALID_ARG, "plan / weights struct is NULL");
+  RNX_PTR(plan->tile_offsets, "plan.tile_offsets");
+  RNX_PTR(plan->tile_rows, "plan.tile_rows");
+  RNX_PTR(w->prepared, "prepared");
+  if (proj == MOE_PROJ_GATE_UP) {
+    if ((s = check_bank(w->gate, "gate")) != MOE_OK || (s = check_bank(w->up, "up")) != MOE_OK) return s;
+  } else {
+    if ((s = check_bank(w->down, "down")) != MOE_OK) return s;
+    RNX_PTR(weights, "weights");
+  }
+  WsLayout L;
+  if ((s = check_ws(cfg, T, MOE_PATH_PREFILL_W4A16, ws, ws_bytes, &L)) != MOE_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  uint32_t* status = (uint32_t*)((char*)ws + L.status);
+  RNX_CUDA(cudaMemsetAsync(status, 0, 4, st), "clear status");
+  const rnx::W4a16GemmArgs g = w4a16_args(cfg, proj, act, act_scale, L.pl.P, *plan, weights, w, out, status);
+  RNX_CUDA(rnx::launch_w4a16_grouped_gemm(g, st), "nvfp4_grouped_gemm_w4a16");
+  return MOE_OK;
+}
+
 moe_status_t moe_unpermute(const moe_config_t* cfg, const uint16_t* rows, int32_t T, const moe_plan_t* plan,
                            const int32_t* ids, uint16_t* out, void* stream) {
   moe_status_t s;
@@ -445,6 +525,15 @@ moe_status_t moe_unpermute_combine(const moe_config_t* cfg, const uint16_t* rows
   const rnx::PaddedIndex q{ids, plan->inv, plan->offsets, plan->tile_offsets, cfg->local_begin, cfg->local_end};
   RNX_CUDA(rnx::launch_unpermute_combine(q, T, cfg->top_k, cfg->hidden, rows, shared, y, (cudaStream_t)stream),
            "moe_unpermute_combine");
+  return MOE_OK;
+}
+
+moe_status_t moe_set_wait_limit(int64_t ns) {
+  if (ns < 0) {
+    rnx::set_test_wait_limit_ns(rnx::kWaitLimitNs);
+    return MOE_OK;
+  }
+  rnx::set_test_wait_limit_ns((unsigned long long)ns);
   return MOE_OK;
 }
 
@@ -495,8 +584,12 @@ moe_status_t moe_permute(const moe_config_t* cfg, const int32_t* ids, int32_t T,
   RNX_PTR(plan->active, "plan.active");
   RNX_PTR(plan->first, "plan.first");
   RNX_PTR(plan->tile_rows, "plan.tile_rows");
-  WsLayout L;   // status word and sort scratch sit at the same offsets on both paths
-  if ((s = check_ws(cfg, T, MOE_PATH_DECODE, ws, ws_bytes, &L)) != MOE_OK) return s;
+  // only the status word and the sort scratch are used: they sit at the same
+  // offsets on both paths, so either path's workspace serves
+  const WsLayout L = ws_layout(cfg, T, MOE_PATH_DECODE);
+  const size_t need = L.scratch + 4 * rnx::permute_scratch_ints(T * cfg->top_k, cfg->num_experts);
+  if (!ws || ((uintptr_t)ws % kAlign) != 0) return fail(MOE_ERR_WORKSPACE, "workspace NULL or not 256-byte aligned");
+  if (ws_bytes < need) return fail(MOE_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, need);
   cudaStream_t st = (cudaStream_t)stream;
   char* b = (char*)ws;
   RNX_CUDA(cudaMemsetAsync(b + L.status, 0, 4, st), "clear status");
@@ -507,8 +600,8 @@ moe_status_t moe_permute(const moe_config_t* cfg, const int32_t* ids, int32_t T,
   return MOE_OK;
 }
 
-moe_status_t nvfp4_expert_gemv(const moe_config_t* cfg, int32_t proj, const uint16_t* act, int32_t T,
-                               const moe_plan_t* plan, const float* weights, const moe_weights_t* w, uint16_t* out,
+moe_status_t nvfp4_expert_gemv(const moe_config_t* cfg, int32_t proj, const void* act, int32_t T,
+                               const moe_plan_t* plan, const float* weights, const moe_weights_t* w, float* out,
                                void* ws, size_t ws_bytes, void* stream) {
   moe_status_t s;
   if ((s = check_cfg(cfg)) != MOE_OK || (s = check_T(T)) != MOE_OK) return s;
@@ -531,14 +624,32 @@ moe_status_t nvfp4_expert_gemv(const moe_config_t* cfg, int32_t proj, const uint
   if ((s = check_ws(cfg, T, MOE_PATH_DECODE, ws, ws_bytes, &L)) != MOE_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
   char* b = (char*)ws;
-  const int K = proj == MOE_PROJ_GATE_UP ? cfg->hidden : cfg->intermediate;
-  const int R = proj == MOE_PROJ_GATE_UP ? T : T * cfg->top_k;
-  uint32_t* amax = (uint32_t*)(b + (proj == MOE_PROJ_GATE_UP ? L.xmax : L.hmax));
-  RNX_CUDA(cudaMemsetAsync(b + L.status, 0, 4, st), "clear status");
-  RNX_CUDA(rnx::launch_row_absmax(act, R, K, amax, st), "activation row max");
+  uint32_t* status = (uint32_t*)(b + L.status);
+  RNX_CUDA(cudaMemsetAsync(status, 0, kCtrlBytes, st), "clear status");
+  const int H = cfg->hidden, I = cfg->intermediate, k = cfg->top_k;
+  if (T == 1 && rnx::decode_t1_supported(H, I, 0, cfg->num_experts, k)) {
+    // one token: the streamed single-token kernels, fed from the plan
+    rnx::DecodeT1Args a{};
+    a.H = H; a.I = I; a.Is = 0; a.E = cfg->num_experts; a.k = k;
+    a.lb = cfg->local_begin; a.le = cfg->local_end;
+    a.limit = cfg->swiglu_limit;
+    a.gate = w->gate; a.up = w->up; a.down = w->down;
+    a.ids = nullptr; a.active = plan->active; a.first = plan->first;
+    a.status = status;
+    if (proj == MOE_PROJ_GATE_UP) {
+      uint32_t* xmax = (uint32_t*)(b + L.xmax);
+      RNX_CUDA(rnx::launch_row_absmax((const uint16_t*)act, 1, H, xmax, st), "activation row max");
+      a.x = (const uint16_t*)act; a.xmax = xmax; a.h = out;
+      RNX_CUDA(rnx::launch_decode_t1_gate_up(a, st), "nvfp4_expert_gemv (gate/up)");
+    } else {
+      a.h = (float*)act; a.weights = (float*)weights; a.r = out;
+      RNX_CUDA(rnx::launch_decode_t1_down(a, st), "nvfp4_expert_gemv (down)");
+    }
+    return MOE_OK;
+  }
   rnx::ExpertGemvArgs a{};
   a.proj = proj;
-  a.T = T; a.H = cfg->hidden; a.I = cfg->intermediate; a.E = cfg->num_experts; a.k = cfg->top_k;
+  a.T = T; a.H = H; a.I = I; a.E = cfg->num_experts; a.k = k;
   a.local_begin = cfg->local_begin; a.local_end = cfg->local_end;
   a.limit = cfg->swiglu_limit;
   a.act = act;
@@ -546,8 +657,7 @@ moe_status_t nvfp4_expert_gemv(const moe_config_t* cfg, int32_t proj, const uint
   a.weights = weights;
   a.gate = w->gate; a.up = w->up; a.down = w->down;
   a.out = out;
-  a.status = (uint32_t*)(b + L.status);
-  a.act_max = amax;
+  a.status = status;
   RNX_CUDA(rnx::launch_nvfp4_gemv(a, st), "nvfp4_expert_gemv");
   return MOE_OK;
 }
@@ -574,9 +684,21 @@ moe_status_t moe_combine(int32_t T, int32_t k, int32_t H, const uint16_t* r, con
   return MOE_OK;
 }
 
+moe_status_t moe_combine_f32(int32_t T, int32_t k, int32_t H, const float* r, const float* shared, uint16_t* y,
+                             void* stream) {
+  if (T < 0 || k < 1 || k > kMaxTopK || H <= 0 || H % 4)
+    return fail(MOE_ERR_INVALID_ARG, "T=%d k=%d H=%d: need T >= 0, 1 <= k <= 16, H a positive multiple of 4", T, k, H);
+  if (T == 0) return MOE_OK;
+  RNX_PTR(r, "r");
+  RNX_PTR(y, "y");
+  if (shared && !aligned16(shared)) return fail(MOE_ERR_INVALID_ARG, "shared is not 16-byte aligned");
+  RNX_CUDA(rnx::launch_combine_f32(T, k, H, r, shared, y, (cudaStream_t)stream), "moe_combine_f32");
+  return MOE_OK;
+}
+
 size_t dense_ffn_workspace_size(int32_t H, int32_t I, int32_t T) {
   if (H <= 0 || I <= 0 || T < 0) return 0;
-  return up(4) + up(2 * (size_t)T * I);
+  return up(4) + up(4 * (size_t)T * I);
 }
 
 moe_status_t dense_ffn_bf16(int32_t H, int32_t I, float limit, const uint16_t* x, int32_t T, const uint16_t* wg,
@@ -594,7 +716,7 @@ moe_status_t dense_ffn_bf16(int32_t H, int32_t I, float limit, const uint16_t* x
   if (!ws || ((uintptr_t)ws % kAlign)) return fail(MOE_ERR_WORKSPACE, "workspace NULL or not 256-byte aligned");
   if (ws_bytes < dense_ffn_workspace_size(H, I, T))
     return fail(MOE_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, dense_ffn_workspace_size(H, I, T));
-  uint16_t* hbuf = (uint16_t*)((char*)ws + up(4));
+  void* hbuf = (char*)ws + up(4);
   cudaStream_t st = (cudaStream_t)stream;
   RNX_CUDA(cudaMemsetAsync(ws, 0, 4, st), "clear status");
   RNX_CUDA(rnx::launch_dense_ffn(H, I, limit, x, T, wg, wu, wd, y, hbuf, (uint32_t*)ws, st), "dense_ffn_bf16");
@@ -616,7 +738,8 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
                          uint16_t* y, void* ws, size_t ws_bytes, void* stream) {
   moe_status_t s;
   if ((s = check_cfg(cfg)) != MOE_OK || (s = check_T(T)) != MOE_OK) return s;
-  if (path != MOE_PATH_DECODE && path != MOE_PATH_PREFILL) return fail(MOE_ERR_INVALID_ARG, "unknown path %d", path);
+  if (path != MOE_PATH_DECODE && path != MOE_PATH_PREFILL && path != MOE_PATH_PREFILL_W4A16)
+    return fail(MOE_ERR_INVALID_ARG, "unknown path %d", path);
   if (T == 0) return MOE_OK;
   if (!w) return fail(MOE_ERR_INVALID_ARG, "weights struct is NULL");
   RNX_PTR(x, "x");
@@ -632,7 +755,7 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
     RNX_PTR(w->shared_up, "shared_up");
     RNX_PTR(w->shared_down, "shared_down");
   }
-  if (path == MOE_PATH_PREFILL) {
+  if (path != MOE_PATH_DECODE) {
     if ((s = check_prefill_shape(cfg)) != MOE_OK) return s;
     RNX_PTR(w->prepared, "prepared");
   }
@@ -645,38 +768,41 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
   int32_t* ids = (int32_t*)(b + L.ids);
   float* wts = (float*)(b + L.weights);
   moe_plan_t plan = plan_at(b + L.plan, L.pl);
-  uint16_t* h = (uint16_t*)(b + L.h);
-  uint16_t* r = (uint16_t*)(b + L.r);
-  uint16_t* shared = Is > 0 ? (uint16_t*)(b + L.shared) : nullptr;
   uint32_t* status = (uint32_t*)(b + L.status);
+  const bool decode = path == MOE_PATH_DECODE;
 
-  RNX_CUDA(cudaMemsetAsync(status, 0, 4, st), "clear status");
+  RNX_CUDA(cudaMemsetAsync(status, 0, kCtrlBytes, st), "clear status");
+
   // decode: the shared expert forks off to the auxiliary stream right away
   SideStream* side = nullptr;
-  const bool shared_aside = Is > 0 && path == MOE_PATH_DECODE;
+  const bool shared_aside = Is > 0 && decode;
+  void* shared = Is > 0 ? (void*)(b + L.shared) : nullptr;
   if (shared_aside) {
     RNX_CUDA(side_stream(&side), "auxiliary stream");
     RNX_CUDA(cudaEventRecord(side->fork, st), "fork event");
     RNX_CUDA(cudaStreamWaitEvent(side->st, side->fork, 0), "fork wait");
-    RNX_CUDA(rnx::launch_dense_ffn(H, Is, cfg->swiglu_limit, x, T, w->shared_gate, w->shared_up, w->shared_down,
-                                   shared, (uint16_t*)(b + L.shared_h), status, side->st),
+    RNX_CUDA(rnx::launch_dense_gemv(H, Is, cfg->swiglu_limit, x, T, w->shared_gate, w->shared_up, w->shared_down,
+                                    shared, true, (float*)(b + L.shared_h), side->st),
              "shared expert");
     RNX_CUDA(cudaEventRecord(side->join, side->st), "join event");
   }
-  RNX_CUDA(mark(MOE_STAGE_ROUTER_LOGITS, st), "stage event");
+  // one token: the streamed expert kernels (one CTA per SM, weights through a
+  // ring of bulk copies), fed from the routing plan; the router's GEMV also
+  // leaves max |x| for their f16 pre-scale
+  const bool t1 = decode && T == 1 && rnx::decode_t1_supported(H, I, 0, E, k);
   uint32_t* xmax = (uint32_t*)(b + L.xmax);
-  uint32_t* hmax = (uint32_t*)(b + L.hmax);
-  if (path == MOE_PATH_PREFILL && router_on_tensor_cores(cfg, T, w)) {
+  RNX_CUDA(mark(MOE_STAGE_ROUTER_LOGITS, st), "stage event");
+  if (!decode && router_on_tensor_cores(cfg, T, w)) {
     const uint16_t* w3 = (const uint16_t*)(w->prepared + prepared_layout(cfg).router3);
     RNX_CUDA(rnx::launch_router_logits_tc(x, T, H, E, w3, logits, status, st), "router logits (tensor cores)");
   } else {
-    RNX_CUDA(rnx::launch_router_logits(x, T, H, E, w->router_w, logits, st, xmax, hmax, T * k), "router logits");
+    RNX_CUDA(rnx::launch_router_logits(x, T, H, E, w->router_w, logits, st, t1 ? xmax : nullptr), "router logits");
   }
   RNX_CUDA(mark(MOE_STAGE_TOPK, st), "stage event");
   // decode with a handful of tokens: selection and plan in one launch (the
   // permute stage then has zero length)
   cudaError_t fp = cudaErrorNotSupported;
-  if (path == MOE_PATH_DECODE)
+  if (decode)
     fp = rnx::launch_topk_plan(logits, w->router_bias, T, E, k, cfg->routed_scaling_factor, ids, wts,
                                cfg->local_begin, cfg->local_end, plan, status, st);
   if (fp == cudaErrorNotSupported) {
@@ -690,8 +816,36 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
     RNX_CUDA(mark(MOE_STAGE_PERMUTE, st), "stage event");
   }
   RNX_CUDA(mark(MOE_STAGE_ACT_QUANT, st), "stage event");
-  if (path == MOE_PATH_PREFILL) {
+  if (path == MOE_PATH_PREFILL_W4A16) {
+    // the pages' prefill numerics: NVFP4 weights x 16-bit activations on the
+    // tensor cores (kind::f16), x gathered into the padded tile order as f16
     const int64_t P = L.pl.P;
+    uint16_t* h = (uint16_t*)(b + L.h);
+    uint16_t* r = (uint16_t*)(b + L.r);
+    uint16_t* xa = (uint16_t*)(b + L.xq);
+    float* xs = (float*)(b + L.xts);
+    const int32_t* used_tiles = plan.tile_offsets + E;
+    RNX_CUDA(rnx::launch_tile_rows(plan, E, P, st), "tile rows");
+    RNX_CUDA(rnx::launch_gather_x_f16(x, H, k, plan.tile_rows, used_tiles, P, xa, xs, st), "x gather (f16)");
+    RNX_CUDA(mark(MOE_STAGE_EXPERT_GATE_UP, st), "stage event");
+    rnx::W4a16GemmArgs g = w4a16_args(cfg, MOE_PROJ_GATE_UP, xa, xs, P, plan, wts, w, h, status);
+    RNX_CUDA(rnx::launch_w4a16_grouped_gemm(g, st), "expert gate/up (W4A16)");
+    RNX_CUDA(mark(MOE_STAGE_H_QUANT, st), "stage event");
+    RNX_CUDA(mark(MOE_STAGE_EXPERT_DOWN, st), "stage event");
+    g = w4a16_args(cfg, MOE_PROJ_DOWN, h, nullptr, P, plan, wts, w, r, status);
+    RNX_CUDA(rnx::launch_w4a16_grouped_gemm(g, st), "expert down (W4A16)");
+    RNX_CUDA(mark(MOE_STAGE_SHARED, st), "stage event");
+    if (Is > 0)
+      RNX_CUDA(rnx::launch_dense_ffn(H, Is, cfg->swiglu_limit, x, T, w->shared_gate, w->shared_up, w->shared_down,
+                                     (uint16_t*)shared, b + L.shared_h, status, st),
+               "shared expert");
+    RNX_CUDA(mark(MOE_STAGE_COMBINE, st), "stage event");
+    const rnx::PaddedIndex q{ids, plan.inv, plan.offsets, plan.tile_offsets, cfg->local_begin, cfg->local_end};
+    RNX_CUDA(rnx::launch_unpermute_combine(q, T, k, H, r, (const uint16_t*)shared, y, st), "unpermute + combine");
+  } else if (!decode) {
+    const int64_t P = L.pl.P;
+    uint16_t* h = (uint16_t*)(b + L.h);
+    uint16_t* r = (uint16_t*)(b + L.r);
     uint8_t* xq = (uint8_t*)(b + L.xq);
     uint8_t* xsf = (uint8_t*)(b + L.xsf);
     float* xts = (float*)(b + L.xts);
@@ -711,7 +865,17 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
     RNX_CUDA(mark(MOE_STAGE_EXPERT_DOWN, st), "stage event");
     g = gemm_args(cfg, MOE_PROJ_DOWN, hq, hsf, hts, P, plan, wts, w, r, status);
     RNX_CUDA(rnx::launch_fp4_grouped_gemm(g, st), "expert down (tcgen05)");
+    RNX_CUDA(mark(MOE_STAGE_SHARED, st), "stage event");
+    if (Is > 0)
+      RNX_CUDA(rnx::launch_dense_ffn(H, Is, cfg->swiglu_limit, x, T, w->shared_gate, w->shared_up, w->shared_down,
+                                     (uint16_t*)shared, b + L.shared_h, status, st),
+               "shared expert");
+    RNX_CUDA(mark(MOE_STAGE_COMBINE, st), "stage event");
+    const rnx::PaddedIndex q{ids, plan.inv, plan.offsets, plan.tile_offsets, cfg->local_begin, cfg->local_end};
+    RNX_CUDA(rnx::launch_unpermute_combine(q, T, k, H, r, (const uint16_t*)shared, y, st), "unpermute + combine");
   } else {
+    float* h = (float*)(b + L.h);
+    float* r = (float*)(b + L.r);
     rnx::ExpertGemvArgs a{};
     a.T = T; a.H = H; a.I = I; a.E = E; a.k = k;
     a.local_begin = cfg->local_begin; a.local_end = cfg->local_end;
@@ -720,28 +884,34 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
     a.weights = wts;
     a.gate = w->gate; a.up = w->up; a.down = w->down;
     a.status = status;
-    a.proj = MOE_PROJ_GATE_UP; a.act = x; a.out = h; a.act_max = xmax; a.out_max = hmax;
-    RNX_CUDA(mark(MOE_STAGE_EXPERT_GATE_UP, st), "stage event");
-    RNX_CUDA(rnx::launch_nvfp4_gemv(a, st), "expert gate/up");
-    RNX_CUDA(mark(MOE_STAGE_H_QUANT, st), "stage event");
-    a.proj = MOE_PROJ_DOWN; a.act = h; a.out = r; a.act_max = hmax; a.out_max = nullptr;
-    RNX_CUDA(mark(MOE_STAGE_EXPERT_DOWN, st), "stage event");
-    RNX_CUDA(rnx::launch_nvfp4_gemv(a, st), "expert down");
-  }
-  RNX_CUDA(mark(MOE_STAGE_SHARED, st), "stage event");
-  if (shared_aside) {
-    RNX_CUDA(cudaStreamWaitEvent(st, side->join, 0), "join wait");
-  } else if (Is > 0) {
-    RNX_CUDA(rnx::launch_dense_ffn(H, Is, cfg->swiglu_limit, x, T, w->shared_gate, w->shared_up, w->shared_down,
-                                   shared, (uint16_t*)(b + L.shared_h), status, st),
-             "shared expert");
-  }
-  RNX_CUDA(mark(MOE_STAGE_COMBINE, st), "stage event");
-  if (path == MOE_PATH_PREFILL) {
-    const rnx::PaddedIndex q{ids, plan.inv, plan.offsets, plan.tile_offsets, cfg->local_begin, cfg->local_end};
-    RNX_CUDA(rnx::launch_unpermute_combine(q, T, k, H, r, shared, y, st), "unpermute + combine");
-  } else {
-    RNX_CUDA(rnx::launch_combine(T, k, H, r, shared, y, st), "combine");
+    if (t1) {
+      rnx::DecodeT1Args d{};
+      d.H = H; d.I = I; d.Is = 0; d.E = E; d.k = k;
+      d.lb = cfg->local_begin; d.le = cfg->local_end;
+      d.limit = cfg->swiglu_limit;
+      d.x = x;
+      d.gate = w->gate; d.up = w->up; d.down = w->down;
+      d.ids = nullptr; d.active = plan.active; d.first = plan.first;
+      d.weights = wts; d.xmax = xmax; d.h = h; d.r = r;
+      d.status = status;
+      RNX_CUDA(mark(MOE_STAGE_EXPERT_GATE_UP, st), "stage event");
+      RNX_CUDA(rnx::launch_decode_t1_gate_up(d, st), "expert gate/up");
+      RNX_CUDA(mark(MOE_STAGE_H_QUANT, st), "stage event");
+      RNX_CUDA(mark(MOE_STAGE_EXPERT_DOWN, st), "stage event");
+      RNX_CUDA(rnx::launch_decode_t1_down(d, st), "expert down");
+    } else {
+      a.proj = MOE_PROJ_GATE_UP; a.act = x; a.out = h;
+      RNX_CUDA(mark(MOE_STAGE_EXPERT_GATE_UP, st), "stage event");
+      RNX_CUDA(rnx::launch_nvfp4_gemv(a, st), "expert gate/up");
+      RNX_CUDA(mark(MOE_STAGE_H_QUANT, st), "stage event");
+      a.proj = MOE_PROJ_DOWN; a.act = h; a.out = r;
+      RNX_CUDA(mark(MOE_STAGE_EXPERT_DOWN, st), "stage event");
+      RNX_CUDA(rnx::launch_nvfp4_gemv(a, st), "expert down");
+    }
+    RNX_CUDA(mark(MOE_STAGE_SHARED, st), "stage event");
+    if (shared_aside) RNX_CUDA(cudaStreamWaitEvent(st, side->join, 0), "join wait");
+    RNX_CUDA(mark(MOE_STAGE_COMBINE, st), "stage event");
+    RNX_CUDA(rnx::launch_combine_f32(T, k, H, r, (const float*)shared, y, st), "combine");
   }
   RNX_CUDA(mark(MOE_STAGE_COUNT, st), "stage event");
   return MOE_OK;
@@ -777,6 +947,23 @@ std::mutex g_noalloc_mu;
 void* g_noalloc_dev[kNoAllocMaxDevices] = {};
 }  // namespace
 
+// Device address of this library's scratch buffer on the current device,
+// looked up once per device (that device current) and cached.
+moe_status_t noalloc_scratch(void** out) {
+  int dev = 0;
+  RNX_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(MOE_ERR_UNSUPPORTED, "device %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_dev[dev]) {
+    void* p = nullptr;
+    RNX_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress(noalloc scratch)");
+    if (!p) return fail(MOE_ERR_CUDA, "cudaGetSymbolAddress returned NULL");
+    g_noalloc_dev[dev] = p;
+  }
+  *out = g_noalloc_dev[dev];
+  return MOE_OK;
+}
+
 moe_status_t moe_forward_decode_noalloc(const moe_config_t* cfg, const moe_weights_t* w, const uint16_t* x,
                                         int32_t T, uint16_t* y, void* stream) {
   moe_status_t s;
@@ -786,21 +973,19 @@ moe_status_t moe_forward_decode_noalloc(const moe_config_t* cfg, const moe_weigh
     return fail(MOE_ERR_WORKSPACE, "moe_forward_decode_noalloc: T=%d needs %zu bytes of scratch, the built-in buffer "
                 "holds %zu", T, need, kNoAllocBytes);
   if (T == 0) return MOE_OK;
-  int dev = 0;
-  RNX_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
-  if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(MOE_ERR_UNSUPPORTED, "device %d out of range", dev);
   void* scratch = nullptr;
-  {
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_dev[dev]) {
-      void* p = nullptr;
-      RNX_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress(noalloc scratch)");
-      if (!p) return fail(MOE_ERR_CUDA, "cudaGetSymbolAddress returned NULL");
-      g_noalloc_dev[dev] = p;
-    }
-    scratch = g_noalloc_dev[dev];
-  }
+  if ((s = noalloc_scratch(&scratch)) != MOE_OK) return s;
   return moe_forward(cfg, w, x, T, MOE_PATH_DECODE, y, scratch, kNoAllocBytes, stream);
+}
+
+// The device status word of the last moe_forward_decode_noalloc call on the
+// current device (it lives at the start of the library's scratch buffer):
+// synchronises `stream`, reads and clears the word, like moe_read_device_status.
+moe_status_t moe_noalloc_read_device_status(void* stream) {
+  void* scratch = nullptr;
+  moe_status_t s;
+  if ((s = noalloc_scratch(&scratch)) != MOE_OK) return s;
+  return moe_read_device_status(scratch, stream);
 }
 
 }  // extern "C"

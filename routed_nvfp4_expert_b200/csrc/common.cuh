@@ -134,6 +134,9 @@ RNX_DEVICE uint4 ldg_stream(const void* p) {
   return r;
 }
 
+// Ask L2 to fetch the 128-byte line holding p (no register result).
+RNX_DEVICE void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
 RNX_DEVICE uint16_t ldg_u16(const void* p) {
   uint16_t r;
   asm("ld.global.nc.u16 %0, [%1];" : "=h"(r) : "l"(p));

@@ -49,6 +49,39 @@ __global__ void __launch_bounds__(256) combine_kernel(int T, int k, int H, const
   }
 }
 
+// moe_combine over fp32 rows (the decode path keeps r and the shared row in
+// fp32): the same order and one rounding. Each thread owns 4 consecutive
+// hidden elements.
+__global__ void __launch_bounds__(256) combine_f32_kernel(int T, int k, int H, const float* __restrict__ r,
+                                                          const float* __restrict__ shared, uint16_t* __restrict__ y) {
+  pdl_wait();
+  pdl_trigger();
+  const int per_row = H >> 2;
+  const long long n = (long long)T * per_row;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const int t = (int)(i / per_row), c = (int)(i - (long long)t * per_row);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < k; ++j) {
+      const float4 v = reinterpret_cast<const float4*>(r + ((size_t)t * k + j) * H)[c];
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    if (shared) {
+      const float4 v = reinterpret_cast<const float4*>(shared + (size_t)t * H)[c];
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    uint2 o;
+    o.x = pack_bf16x2(acc.x, acc.y);
+    o.y = pack_bf16x2(acc.z, acc.w);
+    reinterpret_cast<uint2*>(y + (size_t)t * H)[c] = o;
+  }
+}
+
 // Padded-layout row of assignment a (the prefill down projection writes its
 // rows there), -1 when its expert is outside the local range or the id was
 // dropped. tile_offsets are in kRowsPerTile-row tiles.
@@ -168,6 +201,12 @@ cudaError_t launch_combine(int T, int k, int H, const uint16_t* r, const uint16_
   return launch_pdl(combine_kernel, dim3(grid_for((long long)T * (H / 8), 256)), dim3(256), 0, st, T, k, H, r, shared,
                     y);
   return cudaGetLastError();
+}
+
+cudaError_t launch_combine_f32(int T, int k, int H, const float* r, const float* shared, uint16_t* y,
+                               cudaStream_t st) {
+  return launch_pdl(combine_f32_kernel, dim3(grid_for((long long)T * (H / 4), 256)), dim3(256), 0, st, T, k, H, r,
+                    shared, y);
 }
 
 cudaError_t launch_unpermute_combine(const PaddedIndex& q, int T, int k, int H, const uint16_t* rows,

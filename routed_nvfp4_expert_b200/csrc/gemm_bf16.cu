@@ -63,6 +63,7 @@ struct GemmParams {
   int M, K, out_cols;
   int a_period;            // A's K extent; the K loop reads A at k mod a_period (LOGITS: K = 3 a_period)
   float limit;
+  unsigned long long wait_ns;   // limit of the main-loop waits (the drain waits keep the default)
 };
 
 template <int MODE>
@@ -119,7 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1) bf16_gemm_kernel(const __grid_con
       for (int ks = 0; ks < n_ksteps; ++ks, ++it) {
         const int s = it % kStages;
         const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-        if (__any_sync(0xffffffffu, !mbar_wait(&empty_bar[s], ph ^ 1u) || abort_flag)) {
+        if (__any_sync(0xffffffffu, !mbar_wait(&empty_bar[s], ph ^ 1u, p.wait_ns) || abort_flag)) {
           ok = false;
           break;
         }
@@ -159,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1) bf16_gemm_kernel(const __grid_con
       const int b = LOGITS ? 0 : (tc & 1);
       const uint32_t use = LOGITS ? (uint32_t)tc : (uint32_t)(tc >> 1);
       // the epilogue must have drained this accumulator buffer's previous tile
-      if (__any_sync(0xffffffffu, !mbar_wait(&acc_empty[b], (use & 1u) ^ 1u))) {
+      if (__any_sync(0xffffffffu, !mbar_wait(&acc_empty[b], (use & 1u) ^ 1u, p.wait_ns))) {
         ok = false;
         break;
       }
@@ -168,7 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1) bf16_gemm_kernel(const __grid_con
       for (int ks = 0; ks < n_ksteps; ++ks, ++it) {
         const int s = it % kStages;
         const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-        if (__any_sync(0xffffffffu, !mbar_wait(&full_bar[s], ph) || abort_flag)) {
+        if (__any_sync(0xffffffffu, !mbar_wait(&full_bar[s], ph, p.wait_ns) || abort_flag)) {
           ok = false;
           break;
         }
@@ -213,9 +214,12 @@ __global__ void __launch_bounds__(kThreads, 1) bf16_gemm_kernel(const __grid_con
       const int nt = tile / n_mtiles, mt = tile - nt * n_mtiles;
       const int row = mt * kTileM + q * 32 + lane;   // A row = TMEM lane of this thread
       const bool valid = row < p.M;
-      if (!mbar_wait(&acc_full[b], use & 1u) || abort_flag) {
-        set_status(p.status, kDevErrTimeout);
-        abort_flag = 1;
+      // warp-uniform decision: the tcgen05.ld below is a whole-warp instruction
+      if (__any_sync(0xffffffffu, !mbar_wait(&acc_full[b], use & 1u, p.wait_ns) || abort_flag)) {
+        if (lane == 0) {
+          set_status(p.status, kDevErrTimeout);
+          abort_flag = 1;
+        }
         break;
       }
       tc_fence_after();
@@ -322,6 +326,11 @@ cudaError_t launch(const GemmParams& p, cudaStream_t st) {
 
 }  // namespace
 
+// Main-loop wait limit of the BF16 GEMM launches (the drain waits keep the
+// default): kWaitLimitNs unless a test lowered it.
+static unsigned long long g_gemm_wait_ns = kWaitLimitNs;
+void set_test_wait_limit_ns(unsigned long long ns) { g_gemm_wait_ns = ns; }
+
 cudaError_t launch_bf16_gemm(bool gate_up, const uint16_t* a, int M, int K, const uint16_t* b0, const uint16_t* b1,
                              int N, float limit, uint16_t* out, uint32_t* status, cudaStream_t st) {
   if (M <= 0 || K % kStepK || N % (gate_up ? 128 : kTileN)) return cudaErrorInvalidValue;
@@ -337,6 +346,7 @@ cudaError_t launch_bf16_gemm(bool gate_up, const uint16_t* a, int M, int K, cons
   p.out_cols = N;
   p.a_period = K;
   p.limit = limit;
+  p.wait_ns = g_gemm_wait_ns;
   return gate_up ? launch<kModeGateUp>(p, st) : launch<kModeDown>(p, st);
 }
 
@@ -354,6 +364,7 @@ cudaError_t launch_router_logits_tc(const uint16_t* x, int T, int H, int E, cons
   p.K = 3 * H;
   p.out_cols = E;
   p.a_period = H;
+  p.wait_ns = g_gemm_wait_ns;
   return launch<kModeLogits>(p, st);
 }
 

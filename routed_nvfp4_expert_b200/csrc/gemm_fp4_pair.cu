@@ -14,9 +14,12 @@
 // tile, its own scale atoms of A and all scale atoms of B; the even CTA
 // issues the MMAs (M = 256, N = 256, K = 64) and the scale copies for both, so
 // every CTA streams half the B bytes a single-CTA 128 x 256 tile would.
-//   GATE_UP: B rows 0..127 = gate rows (CTA 0), 128..255 = up rows (CTA 1) of
-//            the same 128 intermediate features; the epilogue applies the
-//            scales, the clamped SwiGLU, rounds h to bf16, stores [P, I].
+//   GATE_UP: 128 intermediate features per tile, their gate and up rows in
+//            the order of moe_prepare_weights' interleaved scale atoms: CTA r
+//            holds gate rows 64 r .. 64 r + 63 then the same up rows, so the
+//            accumulator's columns 128 r .. +63 are gate and +64 .. +127 up
+//            of features 64 r .. 64 r + 63; the epilogue applies the scales
+//            and the clamped SwiGLU, rounds h to bf16, stores [P, I].
 //   DOWN:    256 output features; the epilogue applies the scales and the
 //            routing weight and writes bf16 rows [P, H] in the padded tile
 //            order (the unpermute is fused into the combine that follows).
@@ -67,11 +70,10 @@ static_assert(kColSf + kStages * kSfColsPerStage <= kTmemCols, "TMEM columns");
 
 struct PairParams {
   CUtensorMap tma_a;       // A codes [P, K/2] bytes, box 128 B x 128 rows, SW128
-  CUtensorMap tma_b0;      // gate (or down) codes [E*rows, K/2], box 128 B x 128 rows
-  CUtensorMap tma_b1;      // up codes (GATE_UP)
+  CUtensorMap tma_b0;      // gate (or down) codes [E*rows, K/2]; box 128 B x 64 (GATE_UP) or 128 rows
+  CUtensorMap tma_b1;      // up codes (GATE_UP), box 128 B x 64 rows
   CUtensorMap tma_sfa;     // A scale atoms viewed as [bytes/256, 256], box 256 x 8 (4 atoms)
-  CUtensorMap tma_sfb0;    // gate (or down) scale atoms, same view
-  CUtensorMap tma_sfb1;    // up scale atoms
+  CUtensorMap tma_sfb0;    // GATE_UP: interleaved gate/up atoms; DOWN: down atoms; same view
   CUtensorMap tma_out;     // output [P, out_cols] bf16, box 64 x 32, SW128
   const float* row_scale;  // [P]
   const float* ts0;        // [E]
@@ -163,15 +165,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const int kb0 = ks * 4;
           tma_load_2d_pair(sA, &p.tma_a, ks * 128, arow, bar);
           if (GATE_UP) {
-            tma_load_2d_pair(sB, rank == 0 ? &p.tma_b0 : &p.tma_b1, ks * 128, e * p.bank_rows + nt * 128, bar);
+            // gate rows then up rows of features nt * 128 + 64 r .. + 63
+            const int g0 = e * p.bank_rows + nt * 128 + 64 * (int)rank;
+            tma_load_2d_pair(sB, &p.tma_b0, ks * 128, g0, bar);
+            tma_load_2d_pair(sB + kBBytes / 2, &p.tma_b1, ks * 128, g0, bar);
           } else {
             tma_load_2d_pair(sB, &p.tma_b0, ks * 128, e * p.bank_rows + nt * kTileN + 128 * (int)rank, bar);
           }
           // scale atoms, 256-byte rows: atom j of a [..][KB][512] array spans rows 2j, 2j+1
           tma_load_2d_pair(sSFA, &p.tma_sfa, 0, 2 * ((mt * 2 + (int)rank) * KB + kb0), bar);
           if (GATE_UP) {
-            tma_load_2d_pair(sSFB, &p.tma_sfb0, 0, 2 * ((rb + nt) * KB + kb0), bar);
-            tma_load_2d_pair(sSFB + 2048, &p.tma_sfb1, 0, 2 * ((rb + nt) * KB + kb0), bar);
+            // interleaved atoms 2 nt and 2 nt + 1 of this expert: B rows 0..127 and 128..255
+            const int ia = e * (p.bank_rows / 64) + 2 * nt;
+            tma_load_2d_pair(sSFB, &p.tma_sfb0, 0, 2 * (ia * KB + kb0), bar);
+            tma_load_2d_pair(sSFB + 2048, &p.tma_sfb0, 0, 2 * ((ia + 1) * KB + kb0), bar);
           } else {
             tma_load_2d_pair(sSFB, &p.tma_sfb0, 0, 2 * ((rb + 2 * nt) * KB + kb0), bar);
             tma_load_2d_pair(sSFB + 2048, &p.tma_sfb0, 0, 2 * ((rb + 2 * nt + 1) * KB + kb0), bar);
@@ -287,12 +294,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       uint4 w4[8 * kBoxes];
       int col0;                                      // first output column of this warp's boxes
       if (GATE_UP) {
+        // columns 128 ch .. +63 gate, +64 .. +127 up of features 64 ch .. +63
         const float sg = rs * p.ts0[e], su = rs * p.ts1[e];
         uint32_t g[64], u[64];
-        tmem_ld32(tq + 64 * ch, g);
-        tmem_ld32(tq + 64 * ch + 32, g + 32);
-        tmem_ld32(tq + 128 + 64 * ch, u);
-        tmem_ld32(tq + 128 + 64 * ch + 32, u + 32);
+        tmem_ld32(tq + 128 * ch, g);
+        tmem_ld32(tq + 128 * ch + 32, g + 32);
+        tmem_ld32(tq + 128 * ch + 64, u);
+        tmem_ld32(tq + 128 * ch + 96, u + 32);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
@@ -360,8 +368,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
 }
 
-bool code_map(CUtensorMap* m, const uint8_t* base, int K, int64_t rows) {
-  return make_tensor_map_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)K / 2, (uint64_t)rows, 128, 128,
+bool code_map(CUtensorMap* m, const uint8_t* base, int K, int64_t rows, uint32_t box_rows) {
+  return make_tensor_map_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)K / 2, (uint64_t)rows, 128, box_rows,
                             CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
@@ -380,12 +388,12 @@ cudaError_t launch_fp4_grouped_gemm(const Fp4GemmArgs& a, cudaStream_t st) {
   const bool gu = a.gate_up;
   const int KB = a.K / 64;
   const int64_t brows = (int64_t)a.E * a.bank_rows;
-  if (!code_map(&p.tma_a, a.a_codes, a.K, a.P_max)) return cudaErrorInvalidValue;
-  if (!code_map(&p.tma_b0, a.b0_codes, a.K, brows)) return cudaErrorInvalidValue;
-  if (gu && !code_map(&p.tma_b1, a.b1_codes, a.K, brows)) return cudaErrorInvalidValue;
+  if (!code_map(&p.tma_a, a.a_codes, a.K, a.P_max, 128)) return cudaErrorInvalidValue;
+  if (!code_map(&p.tma_b0, a.b0_codes, a.K, brows, gu ? 64 : 128)) return cudaErrorInvalidValue;
+  if (gu && !code_map(&p.tma_b1, a.b1_codes, a.K, brows, 64)) return cudaErrorInvalidValue;
   if (!atom_map(&p.tma_sfa, a.a_sf, a.P_max / 128 * KB)) return cudaErrorInvalidValue;
-  if (!atom_map(&p.tma_sfb0, a.b0_sf, brows / 128 * KB)) return cudaErrorInvalidValue;
-  if (gu && !atom_map(&p.tma_sfb1, a.b1_sf, brows / 128 * KB)) return cudaErrorInvalidValue;
+  // GATE_UP: interleaved gate/up atoms, 2 E I / 128 row blocks
+  if (!atom_map(&p.tma_sfb0, a.b0_sf, (gu ? 2 * brows : brows) / 128 * KB)) return cudaErrorInvalidValue;
   if (!make_tensor_map_2d(&p.tma_out, a.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.out_cols,
                           (uint64_t)a.P_max, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;

@@ -33,20 +33,53 @@ struct ExpertGemvArgs {
   int T, H, I, E, k;
   int local_begin, local_end;
   float limit;
-  const uint16_t* act;
+  const void* act;          // GATE_UP: x bf16 [T, H]; DOWN: h fp32 [T*k, I]
   const int32_t* offsets;
   const int32_t* sorted;
   const int32_t* active;
   const int32_t* first;     // plan.first: first assignment of each active expert
   const float* weights;
   nvfp4_bank_t gate, up, down;
-  uint16_t* out;
+  float* out;               // GATE_UP: h fp32 [T*k, I]; DOWN: r fp32 [T*k, H]
   uint32_t* status;         // device status word (bounded-wait timeouts)
-  const uint32_t* act_max;  // optional: max |activation row| as fp32 bits (x rows by token / h rows by assignment)
-  uint32_t* out_max;        // optional (GATE_UP): receives max |h| per assignment; must start at 0
 };
 
 cudaError_t launch_nvfp4_gemv(const ExpertGemvArgs& a, cudaStream_t st);
+
+// Single-token decode chain (decode_t1.cu): K1 router + top-k + shared
+// gate/up, K2 routed gate/up, K3 routed + shared down with the combine.
+// K2 / K3 also run alone (the expert GEMV entry point at T = 1) from a routing
+// plan: ids == nullptr, active / first from the plan.
+struct DecodeT1Args {
+  int H, I, Is, E, k, lb, le;
+  float rsf, limit;
+  const uint16_t* x;                 // bf16 [H]
+  const float* router_w;             // fp32 [E, H]
+  const float* router_bias;          // fp32 [E]
+  nvfp4_bank_t gate, up, down;
+  const uint16_t* sh_gate;           // bf16 [Is, H] (nullable)
+  const uint16_t* sh_up;
+  const uint16_t* sh_down;           // bf16 [H, Is] (nullable: no shared expert)
+  float* logits;                     // fp32 [E]
+  int32_t* ids;                      // [k]; nullptr: the plan form below
+  float* weights;                    // [k] routing weights
+  const int32_t* active;             // plan form: active local experts (count first)
+  const int32_t* first;              // plan form: the assignment of each active expert
+  moe_plan_t plan;                   // K1 writes the routing plan when plan.counts != nullptr
+  uint32_t* xmax;                    // max |x| (fp32 bits)
+  uint32_t* ticket;                  // K1's arrival counter, 0 before K1
+  float* h;                          // fp32 [k, I]
+  float* h_shared;                   // fp32 [Is]
+  float* r;                          // fp32 [k, H] weighted routed rows (nullable)
+  uint16_t* y;                       // bf16 [H] (nullable: no combine)
+  float* shared_out;                 // fp32 [H] the shared row (nullable)
+  uint32_t* status;
+  int l2_prefetch;                   // K2 prefetches K3's down rows into L2
+};
+bool decode_t1_supported(int H, int I, int Is, int E, int k);
+cudaError_t launch_decode_t1_router(const DecodeT1Args& p, cudaStream_t st);
+cudaError_t launch_decode_t1_gate_up(const DecodeT1Args& p, cudaStream_t st);
+cudaError_t launch_decode_t1_down(const DecodeT1Args& p, cudaStream_t st);
 
 // router
 // xmax (nullable): receives max |x_t| per token as fp32 bits; zero (nullable):
@@ -85,13 +118,18 @@ cudaError_t launch_unpermute(const PaddedIndex& q, long long A, int H, const uin
                              cudaStream_t st);
 cudaError_t launch_combine(int T, int k, int H, const uint16_t* r, const uint16_t* shared, uint16_t* y,
                            cudaStream_t st);
+// the same over fp32 rows and an fp32 shared row (the decode path)
+cudaError_t launch_combine_f32(int T, int k, int H, const float* r, const float* shared, uint16_t* y,
+                               cudaStream_t st);
 cudaError_t launch_swiglu(const float* gu, int M, int I, float limit, uint16_t* h, cudaStream_t st);
 cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* scales, const float* ts, int rows, int K, float* out,
                            cudaStream_t st);
 
-// dense BF16 FFN (decode GEMV form): hbuf bf16 [T, I] scratch
+// dense BF16 FFN (decode GEMV form): hbuf fp32 [T, I] scratch; y bf16 or
+// fp32 (y_f32) [T, H]
 cudaError_t launch_dense_gemv(int H, int I, float limit, const uint16_t* x, int T, const uint16_t* wg,
-                              const uint16_t* wu, const uint16_t* wd, uint16_t* y, uint16_t* hbuf, cudaStream_t st);
+                              const uint16_t* wu, const uint16_t* wd, void* y, bool y_f32, float* hbuf,
+                              cudaStream_t st);
 
 // BF16 GEMM on tcgen05 (kind::f16): out [M, N] = a [M, K] . b^T with b [N, K].
 // gate_up: b0 = gate rows, b1 = up rows; out = clamped_swiglu(a.b0^T, a.b1^T).
@@ -99,6 +137,9 @@ cudaError_t launch_dense_gemv(int H, int I, float limit, const uint16_t* x, int 
 // word for bounded-wait timeouts (nullable).
 cudaError_t launch_bf16_gemm(bool gate_up, const uint16_t* a, int M, int K, const uint16_t* b0, const uint16_t* b1,
                              int N, float limit, uint16_t* out, uint32_t* status, cudaStream_t st);
+// Limit of the BF16 GEMM's main-loop waits for later launches (host setting;
+// 0 = give up at the first incomplete poll). Test hook for the timeout path.
+void set_test_wait_limit_ns(unsigned long long ns);
 
 // Router logits on the tensor cores: logits [T, E] fp32 = x [T, H] . w^T with
 // w given exactly as w3 [E, 3H] bf16 = (lo | mid | hi) per row. E % 4 == 0,
@@ -113,8 +154,9 @@ cudaError_t launch_router_split(const float* w, int E, int H, uint16_t* w3, cuda
 // Dense BF16 FFN, picking the GEMV form for small T and the tcgen05 GEMM for
 // T >= kDenseGemmMinT (when the shapes allow it).
 constexpr int kDenseGemmMinT = 128;
+// hbuf: T*I*4 bytes (fp32 h in the GEMV form, bf16 h in the GEMM form).
 cudaError_t launch_dense_ffn(int H, int I, float limit, const uint16_t* x, int T, const uint16_t* wg,
-                             const uint16_t* wu, const uint16_t* wd, uint16_t* y, uint16_t* hbuf, uint32_t* status,
+                             const uint16_t* wu, const uint16_t* wd, uint16_t* y, void* hbuf, uint32_t* status,
                              cudaStream_t st);
 
 // ---------------------------------------------------------------- prefill (W4A4, tcgen05)
@@ -145,6 +187,10 @@ cudaError_t launch_quant_tokens(const uint16_t* x, int T, int K, int k, const in
 
 // Canonical block scales [n_experts * rows, K/16] -> atoms [n_experts][rows/128][K/64][512].
 cudaError_t launch_sf_atoms(const uint8_t* scales, int64_t n_experts, int rows, int K, uint8_t* atoms, cudaStream_t st);
+// Gate and up block scales ([E*I, K/16] each) -> atoms [E][I/64][K/64][512]
+// whose 128 rows are 64 gate rows then the same 64 up rows (I % 64 == 0).
+cudaError_t launch_sf_atoms_gate_up(const uint8_t* gate, const uint8_t* up, int64_t n_experts, int I, int K,
+                                    uint8_t* atoms, cudaStream_t st);
 
 struct Fp4GemmArgs {
   bool gate_up;
@@ -156,8 +202,9 @@ struct Fp4GemmArgs {
   const float* row_scale;          // [P_max]
   const uint8_t* b0_codes;         // gate (or down) codes [E*bank_rows, K/2]
   const uint8_t* b1_codes;         // up codes (gate_up)
-  const uint8_t* b0_sf;            // atoms [E][bank_rows/128][K/64][512]
-  const uint8_t* b1_sf;
+  const uint8_t* b0_sf;            // GATE_UP: interleaved gate/up atoms [E][I/64][K/64][512];
+                                   // DOWN: atoms [E][H/128][K/64][512]
+  const uint8_t* b1_sf;            // unused
   const float* ts0;
   const float* ts1;
   const int32_t* tile_offsets;     // [E+1]
@@ -167,5 +214,33 @@ struct Fp4GemmArgs {
   uint32_t* status;
 };
 cudaError_t launch_fp4_grouped_gemm(const Fp4GemmArgs& a, cudaStream_t st);
+
+// ---------------------------------------------------------------- prefill (W4A16, tcgen05 kind::f16)
+
+// x rows in the padded tile order as f16, each scaled by the power of two that
+// brings its max |x| into [2^14, 2^15); unscale[p] the inverse (0 on padding
+// rows). Rows at or past used_tiles * 256 are not written.
+cudaError_t launch_gather_x_f16(const uint16_t* x, int H, int k, const int32_t* tile_rows, const int32_t* used_tiles,
+                                int64_t P, uint16_t* xa, float* unscale, cudaStream_t st);
+
+struct W4a16GemmArgs {
+  bool gate_up;
+  int E, K, out_cols, bank_rows;   // bank_rows: rows of one expert (I for gate/up, H for down)
+  int64_t P_max;
+  float limit;
+  const uint16_t* act;             // f16 [P_max, K] (GATE_UP: gathered x; DOWN: h)
+  const float* row_scale;          // [P_max] A row unscale (nullable: 1)
+  const uint8_t* b0_codes;         // gate (or down) codes [E*bank_rows, K/2]
+  const uint8_t* b1_codes;         // up codes (GATE_UP)
+  const uint8_t* b_sf;             // GATE_UP: interleaved gate/up atoms; DOWN: down atoms
+  const float* ts0;
+  const float* ts1;
+  const int32_t* tile_offsets;     // [E+1]
+  const int32_t* tile_rows;        // [P_max]
+  const float* weights;            // [A] routing weights (DOWN)
+  void* out;                       // GATE_UP: h f16 [P_max, I]; DOWN: rows bf16 [P_max, H]
+  uint32_t* status;
+};
+cudaError_t launch_w4a16_grouped_gemm(const W4a16GemmArgs& a, cudaStream_t st);
 
 }  // namespace rnx

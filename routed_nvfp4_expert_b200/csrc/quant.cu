@@ -262,6 +262,38 @@ cudaError_t launch_quant_tokens(const uint16_t* x, int T, int K, int k, const in
   return cudaGetLastError();
 }
 
+namespace {
+// Gate and up scales of E experts ([E*I, K/16] each) as one atom grid whose
+// 128-row atoms hold 64 gate rows then the same 64 up rows: interleaved row
+// R = (e * I/64 + j) * 128 + m is gate row e*I + 64 j + m (m < 64) or up row
+// e*I + 64 j + m - 64.
+__global__ void __launch_bounds__(256) sf_atoms_gu_kernel(const uint8_t* __restrict__ gate,
+                                                          const uint8_t* __restrict__ up, long long total_rows, int I,
+                                                          int K, uint8_t* __restrict__ atoms) {
+  const int KB = K / 64;
+  for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < total_rows * KB;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const long long R = idx / KB;
+    const int kb = (int)(idx - R * KB);
+    const long long blk = R >> 7;                 // e * I/64 + j
+    const int m = (int)(R & 127);
+    const long long e = blk / (I / 64), j = blk - e * (I / 64);
+    const long long src = e * I + 64 * j + (m & 63);
+    const uint8_t* bank = m < 64 ? gate : up;
+    const uint32_t w = *reinterpret_cast<const uint32_t*>(bank + src * (K / 16) + kb * 4);
+    *reinterpret_cast<uint32_t*>(atoms + sf_atom_offset(R, kb * 4, KB)) = w;
+  }
+}
+}  // namespace
+
+cudaError_t launch_sf_atoms_gate_up(const uint8_t* gate, const uint8_t* up, int64_t n_experts, int I, int K,
+                                    uint8_t* atoms, cudaStream_t st) {
+  const long long total = 2LL * n_experts * I;
+  if (total <= 0) return cudaSuccess;
+  sf_atoms_gu_kernel<<<grid_for(total * (K / 64), 256), 256, 0, st>>>(gate, up, total, I, K, atoms);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_sf_atoms(const uint8_t* scales, int64_t n_experts, int rows, int K, uint8_t* atoms,
                             cudaStream_t st) {
   const long long total = (long long)n_experts * rows;

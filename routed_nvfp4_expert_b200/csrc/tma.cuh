@@ -48,6 +48,20 @@ RNX_DEVICE bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the phase with the given parity (test_wait returns at
+// once; try_wait may hold the thread for a while before it reports failure).
+RNX_DEVICE bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // try_wait that lets the hardware suspend the thread for up to hint_ns
 // before returning (no polling loop burning issue slots meanwhile).
 RNX_DEVICE bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
@@ -64,8 +78,11 @@ RNX_DEVICE bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint
 
 // Bounded wait for the phase with the given parity to complete. Polls with a
 // suspend hint; reads %globaltimer only every 1024 polls. Returns false if the
-// phase did not complete within kWaitLimitNs.
-RNX_DEVICE bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// phase did not complete within limit_ns; limit_ns == 0 gives up at once if
+// the phase is incomplete (a test setting that makes the first wait for work
+// still in flight run out).
+RNX_DEVICE bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned long long limit_ns = kWaitLimitNs) {
+  if (limit_ns == 0) return mbar_test_wait(bar, parity);
   if (mbar_try_wait(bar, parity)) return true;
   unsigned long long t0 = 0;
   for (uint32_t i = 0;; ++i) {
@@ -73,9 +90,26 @@ RNX_DEVICE bool mbar_wait(uint64_t* bar, uint32_t parity) {
     if ((i & 1023u) == 0) {
       const unsigned long long t = globaltimer_ns();
       if (i == 0) t0 = t;
-      else if (t - t0 > kWaitLimitNs) return false;
+      else if (t - t0 > limit_ns) return false;
     }
   }
+}
+
+// Untiled bulk copy (TMA engine) of `bytes` from global memory into this
+// CTA's shared memory; completion is counted on `bar` as transaction bytes.
+// dst and src 16-byte aligned, bytes a multiple of 16. No multicast.
+RNX_DEVICE void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Ask the TMA engine to bring `bytes` of global memory into L2 (no shared
+// memory destination, no completion to wait for). 16-byte aligned, bytes a
+// multiple of 16.
+RNX_DEVICE void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 RNX_DEVICE void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }

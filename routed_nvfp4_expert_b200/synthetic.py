@@ -62,7 +62,7 @@ class Workload:
     stress: bool = False   # skewed bias on 16 experts + 1% exactly tied tokens
     rsf: float = 2.5       # routed_scaling_factor
     limit: float = 7.0     # swiglu_limit
-    kind: str = "decode"   # "decode" (GEMV path) or "prefill" (grouped GEMM path)
+    kind: str = "decode"   # "decode" (GEMV path), "prefill" (grouped GEMM path) or "dense" (the dense FFN)
 
     def with_tokens(self, T: int, name: str | None = None) -> "Workload":
         return dataclasses.replace(self, T=T, name=name or f"{self.name}_t{T}")
@@ -79,11 +79,17 @@ WORKLOADS: dict[str, Workload] = {
     "tiny_t4": Workload("tiny_t4", T=4, H=256, I=128, E=16, k=4, Is=128, dense_I=512,
                         sigma_w=0.02, kind="decode"),
     "decode_t1": _w("decode_t1", 1, "decode"),
+    # multi-token verification steps of speculative decoding (T = 2, 4 per user)
+    "decode_t2": _w("decode_t2", 2, "decode"),
+    "decode_t4": _w("decode_t4", 4, "decode"),
     "decode_t8": _w("decode_t8", 8, "decode"),
     "decode_t32": _w("decode_t32", 32, "decode"),
     "decode_t64": _w("decode_t64", 64, "decode"),
     "prefill_t4096": _w("prefill_t4096", 4096, "prefill"),
     "stress_t16384": _w("stress_t16384", 16384, "prefill", x_scale=8.0, stress=True),
+    # the dense BF16 FFN of the first_k_dense_replace layers at H = 4096, I = 12288
+    "dense_t4096": _w("dense_t4096", 4096, "dense"),
+    "dense_t1": _w("dense_t1", 1, "dense"),
 }
 
 

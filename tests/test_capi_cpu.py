@@ -81,8 +81,12 @@ def test_workspace_too_small_is_rejected_before_launch():
     assert need > 0
     ids = 0x10000
     plan = capi.MoePlan(0x20000, 0x30000, 0x40000, 0x50000, 0x60000, 0x70000, 0x80000, 0x90000)
-    st = lib.moe_permute(C.byref(cfg), ids, 4, C.byref(plan), 0x100000, need - 256, None)
+    # moe_permute needs the status word and the sort scratch only
+    st = lib.moe_permute(C.byref(cfg), ids, 4, C.byref(plan), 0x100000, 256, None)
     assert st == 3 and "workspace" in lib.moe_last_error().decode()
+    w = capi.MoeWeights()
+    st = lib.moe_forward(C.byref(cfg), C.byref(w), 0x10000, 4, 0, 0x20000, 0x100000, need - 256, None)
+    assert st != 0
 
 
 def test_plan_carve_is_host_arithmetic():

@@ -88,9 +88,13 @@ def test_prepare_weights_bit_exact():
     per = wl.E * wl.I * wl.H // 16
     r3 = (3 * per + 255) // 256 * 256
     assert prep.size == r3 + (wl.E * 3 * wl.H * 2 + 255) // 256 * 256
-    for i, (p, rows, K) in enumerate((("gate", wl.I, wl.H), ("up", wl.I, wl.H), ("down", wl.H, wl.I))):
-        got = sf_untile(prep[i * per:(i + 1) * per], wl.E * rows, K)
-        assert np.array_equal(got, inp[f"{p}_scales"].reshape(wl.E * rows, K // 16)), p
+    # gate and up interleaved: atom rows 0..63 = gate rows 64 j.., 64..127 = up rows 64 j..
+    got = sf_untile(prep[:2 * per], 2 * wl.E * wl.I, wl.H).reshape(wl.E, wl.I // 64, 2, 64, wl.H // 16)
+    g = inp["gate_scales"].reshape(wl.E, wl.I // 64, 64, wl.H // 16)
+    u = inp["up_scales"].reshape(wl.E, wl.I // 64, 64, wl.H // 16)
+    assert np.array_equal(got[:, :, 0], g) and np.array_equal(got[:, :, 1], u)
+    got = sf_untile(prep[2 * per:3 * per], wl.E * wl.H, wl.I)
+    assert np.array_equal(got, inp["down_scales"].reshape(wl.E * wl.H, wl.I // 16))
     # router weight as three bf16 terms whose exact sum is the fp32 weight
     w3 = prep[r3:r3 + wl.E * 3 * wl.H * 2].view(np.uint16).reshape(wl.E, 3, wl.H)
     parts = OF.bf16_value(w3)
@@ -147,11 +151,11 @@ def _site_state(wl, cfg, T, v):
     st["xq"] = capi.view_tensor(v.xq_codes, (P, H // 2), torch.uint8).cpu().numpy()[:Pu]
     st["xsf"] = sf_untile(capi.view_tensor(v.xq_sf, (P * H // 16,), torch.uint8).cpu().numpy(), Pu, H)
     st["xts"] = capi.view_tensor(v.xq_scale, (P,), torch.float32).cpu().numpy()[:Pu]
-    st["h"] = bf16_np(capi.view_tensor(v.h, (P, I), torch.bfloat16))[:Pu]
+    st["h"] = bf16_np(capi.view_tensor(v.h, (P, I), torch.bfloat16)[:Pu])
     st["hq"] = capi.view_tensor(v.hq_codes, (P, I // 2), torch.uint8).cpu().numpy()[:Pu]
     st["hsf"] = sf_untile(capi.view_tensor(v.hq_sf, (P * I // 16,), torch.uint8).cpu().numpy(), Pu, I)
     st["hts"] = capi.view_tensor(v.hq_scale, (P,), torch.float32).cpu().numpy()[:Pu]
-    st["r_pad"] = bf16_np(capi.view_tensor(v.r, (P, H), torch.bfloat16))[:Pu]
+    st["r_pad"] = bf16_np(capi.view_tensor(v.r, (P, H), torch.bfloat16)[:Pu])
     return st
 
 
@@ -272,6 +276,8 @@ def test_moe_forward_prefill_matches_oracle(name, T):
         if wl.stress:                                 # include exactly tied tokens
             tokens = np.unique(np.concatenate([tokens, inp["tie_tokens"][:4]]))
     ref = OS.site_forward(inp, oracle_cfg(wl), "prefill", tokens=tokens, gpu_logits=lg[tokens], want_parts=True)
+    if wl.stress:                                     # x8 activations: the clamp fires on the tails
+        assert ref["clamp_fired"] > 0.01 * ref["clamp_total"]
     # logits (tensor-core split-bf16 GEMM at T >= 128): 1e-5 of the token's largest logit
     rl = ref["logits"]
     scale = np.maximum(np.abs(rl), np.abs(rl).max(axis=1, keepdims=True))
@@ -317,3 +323,110 @@ def test_prefill_local_range_masks_remote_experts(T):
     r = bf16_np(_token_rows(cfg, wl, wl.T, v))
     remote = (ids < local[0]) | (ids >= local[1])
     assert remote.any() and not r[remote].any()
+
+
+@pytest.mark.parametrize("name,T", [("tiny_t4", 33), ("mid", 300)])
+def test_prefill_on_quantised_bank(name, T):
+    """The prefill on expert banks made by quantising Gaussian weights (block
+    scales up to 448) matches the oracle."""
+    from helpers import with_quantised_banks
+    from routed_nvfp4_expert_b200 import synthetic as syn
+    if name == "mid":
+        wl = syn.Workload("mid", T=T, H=1024, I=512, E=32, k=8, Is=512, dense_I=64, sigma_w=0.0064, kind="prefill")
+    else:
+        wl = workload(name, T)
+    inp = with_quantised_banks(wl, site_inputs(wl))
+    cfg = capi.config_for(wl)
+    site = capi.site_to_device(inp)
+    capi.moe_prepare_weights(cfg, site)
+    x = capi.bf16_tensor(inp["x"])
+    y = torch.empty_like(x)
+    ws = capi.alloc_workspace(cfg, wl.T, capi.PATH_PREFILL)
+    capi.moe_forward(cfg, site, x, capi.PATH_PREFILL, y, ws)
+    capi.moe_read_device_status(ws)
+    v = capi.moe_workspace_views(cfg, wl.T, capi.PATH_PREFILL, ws)
+    lg = capi.view_tensor(v.logits, (wl.T, wl.E), torch.float32).cpu().numpy()
+    tokens = np.arange(min(wl.T, 24))
+    ref = OS.site_forward(inp, oracle_cfg(wl), "prefill", tokens=tokens, gpu_logits=lg[tokens])
+    assert_bf16_close(bf16_np(y)[tokens], ref["y"], what=f"{name} quantised-bank prefill y")
+
+
+# ------------------------------------------------------------------ W4A16 prefill (the pages' numerics)
+
+def _prefill_w4(wl, inp, local=None):
+    cfg = capi.config_for(wl, local)
+    site = device_site(wl, inp)
+    capi.moe_prepare_weights(cfg, site)
+    x = capi.bf16_tensor(inp["x"])
+    y = torch.empty_like(x)
+    ws = capi.alloc_workspace(cfg, wl.T, capi.PATH_PREFILL_W4A16)
+    capi.moe_forward(cfg, site, x, capi.PATH_PREFILL_W4A16, y, ws)
+    capi.moe_read_device_status(ws)
+    v = capi.moe_workspace_views(cfg, wl.T, capi.PATH_PREFILL_W4A16, ws)
+    return cfg, site, y, ws, v
+
+
+@pytest.mark.parametrize("name,T", [("tiny_t4", None), ("tiny_t4", 33), ("tiny_t4", 1000), ("prefill_t4096", None),
+                                    ("stress_t16384", None)])
+def test_w4a16_prefill_matches_oracle(name, T):
+    """The W4A16 prefill computes the decode numerics (bf16 x straight into
+    the NVFP4 experts, no activation quantisation) as a grouped GEMM: it holds
+    the output gate against the oracle's W4A16 site."""
+    wl = workload(name, T)
+    inp = site_inputs(wl)
+    cfg, site, y, ws, v = _prefill_w4(wl, inp)
+    lg = capi.view_tensor(v.logits, (wl.T, wl.E), torch.float32).cpu().numpy()
+    if wl.T <= 40:
+        tokens = np.arange(wl.T)
+    else:
+        tokens = np.random.default_rng(3).choice(wl.T, 12, replace=False)
+        if wl.stress:
+            tokens = np.unique(np.concatenate([tokens, inp["tie_tokens"][:4]]))
+    ref = OS.site_forward(inp, oracle_cfg(wl), "decode", tokens=tokens, gpu_logits=lg[tokens], want_parts=True)
+    ids = capi.view_tensor(v.ids, (wl.T, wl.k), torch.int32).cpu().numpy()
+    assert np.array_equal(ids[tokens], ref["ids"])
+    got = bf16_np(y)[tokens]
+    assert_bf16_close(got, ref["y"], what=f"{wl.name} W4A16 y")
+    assert rel_l2(got, ref["y"]) < 5e-3
+    r = _token_rows(cfg, wl, wl.T, v)
+    assert_bf16_close(bf16_np(r)[tokens], ref["r"], what="W4A16 r")
+
+
+def test_w4a16_entry_point_matches_forward():
+    wl = workload("tiny_t4", 300)
+    inp = site_inputs(wl)
+    cfg, site, y, ws, v = _prefill_w4(wl, inp)
+    T, P = wl.T, capi.moe_padded_rows(cfg, wl.T)
+    xa = capi.view_tensor(v.xq_codes, (P, wl.H), torch.float16)
+    xs = capi.view_tensor(v.xq_scale, (P,), torch.float32)
+    h = capi.view_tensor(v.h, (P, wl.I), torch.float16)
+    r = capi.view_tensor(v.r, (P, wl.H), torch.bfloat16)
+    wts = capi.view_tensor(v.weights, (T * wl.k,), torch.float32)
+    ws2 = capi.alloc_workspace(cfg, T, capi.PATH_PREFILL_W4A16)
+    h2 = torch.zeros((P, wl.I), dtype=torch.float16, device="cuda")
+    capi.nvfp4_grouped_gemm_w4a16(cfg, capi.PROJ_GATE_UP, xa, xs, T, v.plan, wts, site, h2, ws2)
+    r2 = torch.full((P, wl.H), 7.0, dtype=torch.bfloat16, device="cuda")
+    capi.nvfp4_grouped_gemm_w4a16(cfg, capi.PROJ_DOWN, h, None, T, v.plan, wts, site, r2, ws2)
+    capi.moe_read_device_status(ws2)
+    used = int(_arr(v.plan.tile_offsets, wl.E + 1)[wl.E]) * TILE
+    assert torch.equal(h2[:used], h[:used])
+    assert torch.equal(r2[:used], r[:used])
+    # the gathered x rows: f16 of x times a power of two, exactly; padding rows zero
+    tr = _arr(v.plan.tile_rows, P)[:used]
+    xs_np = xs.cpu().numpy()[:used]
+    xa_np = xa.float().cpu().numpy().astype(np.float64)[:used]
+    valid = tr >= 0
+    want = OF.bf16_value(inp["x"][tr[valid] // wl.k])
+    assert np.array_equal(xa_np[valid] * xs_np[valid, None].astype(np.float64), want)
+    assert not xa_np[~valid].any()
+
+
+def test_w4a16_prefill_local_range_masks_remote_experts():
+    wl = workload("tiny_t4", 300)
+    inp = site_inputs(wl)
+    local = (5, 11)
+    cfg, site, y, ws, v = _prefill_w4(wl, inp, local=local)
+    lg = capi.view_tensor(v.logits, (wl.T, wl.E), torch.float32).cpu().numpy()
+    tokens = np.arange(40)
+    ref = OS.site_forward(inp, oracle_cfg(wl, local), "decode", tokens=tokens, gpu_logits=lg[tokens])
+    assert_bf16_close(bf16_np(y)[tokens], ref["y"], what="W4A16 local y")

@@ -4,8 +4,9 @@ It serves callers that cannot allocate device memory for a workspace (memory
 pools that forbid cudaMalloc, callbacks that may not allocate, C hosts that
 hold only tensor pointers): its scratch is a buffer inside the library. These
 checks call it through the C ABI twice in a row, on two different inputs, and
-compare each result with moe_forward's on a caller-provided workspace. The
-file is named so that pytest collects it last.
+compare each result with moe_forward's on a caller-provided workspace, and
+read the call's device status word through moe_noalloc_read_device_status.
+The file is named so that pytest collects it last.
 """
 import numpy as np
 import pytest
@@ -32,6 +33,7 @@ def test_noalloc_matches_moe_forward_on_two_calls(name, T):
         capi.moe_forward(cfg, site, x, capi.PATH_DECODE, y_ref, ws)
         y = torch.full_like(x, float("nan"))
         capi.moe_forward_decode_noalloc(cfg, site, x, y)
+        capi.moe_noalloc_read_device_status()      # device-side errors of the call: none
         torch.cuda.synchronize()
         assert_bf16_close(bf16_np(y), bf16_np(y_ref), what=f"{name} noalloc vs moe_forward")
         # same kernels, same order: the results agree bit for bit as well
