@@ -36,7 +36,7 @@
  *    frees no device memory and keeps no state besides a thread-local error
  *    message, the thread-local stage-timing events of moe_set_stage_events()
  *    and, per host thread and device, the auxiliary stream and event pair on
- *    which the decode forward with T > 1 runs the shared expert concurrently
+ *    which the decode forward runs the shared expert concurrently
  *    (created by the first such call on that thread and device: make it before
  *    any stream capture on that thread).
  *  - bf16 tensors are passed as uint16_t bit patterns.
@@ -298,20 +298,20 @@ moe_status_t nvfp4_quantize_rows(const uint16_t* src, int32_t rows, int32_t K, u
  * prefill of moe_forward); padding rows must be zero (codes, scales, scale).
  *   MOE_PROJ_GATE_UP (K = H): out = h bf16 [P, I], h[p] = clamped_swiglu(
  *       g, u) of padded row p (0 on padding rows); `weights` unused.
- *   MOE_PROJ_DOWN (K = I): out = rows bf16 [P, H] in the padded tile order,
+ *   MOE_PROJ_DOWN (K = I): out = rows fp32 [P, H] in the padded tile order,
  *       rows[p] = weights[a] * (down_e . hdeq[p]) for the assignment a at
  *       padded row p (0 on padding rows); moe_unpermute /
  *       moe_unpermute_combine bring them back to token order.
  *   Requires w->prepared, I % 128 == 0, H % 256 == 0.
  *   ws: at least moe_workspace_size(cfg, T, MOE_PATH_PREFILL) bytes (status).
- * The kernel runs on clusters of two CTAs (tcgen05.mma.cta_group::2, 256 x
- * 128 tiles, M split across the pair, each CTA loading half of the weight
- * tile, two TMEM accumulators alternating between tiles); no TMA load uses
- * cluster multicast.
+ * The kernel runs on clusters of two CTAs (tcgen05.mma.cta_group::2, tiles of
+ * 256 rows x 256 weight rows, M split across the pair, each CTA loading half
+ * of the weight tile, one TMEM accumulator); no TMA load uses cluster
+ * multicast.
  */
 moe_status_t nvfp4_grouped_gemm(const moe_config_t* cfg, int32_t proj, const uint8_t* act_codes,
                                 const uint8_t* act_sf, const float* act_scale, int32_t T, const moe_plan_t* plan,
-                                const float* weights, const moe_weights_t* w, uint16_t* out, void* ws,
+                                const float* weights, const moe_weights_t* w, void* out, void* ws,
                                 size_t ws_bytes, void* stream);
 
 /*
@@ -328,7 +328,7 @@ moe_status_t nvfp4_grouped_gemm(const moe_config_t* cfg, int32_t proj, const uin
  *       clamped_swiglu(g, u) (saturating to the f16 range; 0 on padding rows);
  *       `weights` unused.
  *   MOE_PROJ_DOWN (K = I): act = h f16 [P, I]; act_scale NULL (1); out = rows
- *       bf16 [P, H] in the padded tile order, rows[p] = weights[a] *
+ *       fp32 [P, H] in the padded tile order, rows[p] = weights[a] *
  *       (down_e . h[p]) (0 on padding rows); moe_unpermute(_combine) brings
  *       them back to token order.
  *   Requires w->prepared (the interleaved gate/up and the down scale atoms),
@@ -339,27 +339,28 @@ moe_status_t nvfp4_grouped_gemm(const moe_config_t* cfg, int32_t proj, const uin
  */
 moe_status_t nvfp4_grouped_gemm_w4a16(const moe_config_t* cfg, int32_t proj, const uint16_t* act,
                                       const float* act_scale, int32_t T, const moe_plan_t* plan, const float* weights,
-                                      const moe_weights_t* w, uint16_t* out, void* ws, size_t ws_bytes, void* stream);
+                                      const moe_weights_t* w, void* out, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Unpermute (the module list's moe_permute family: token sort / permute /
  * unpermute): rows of the padded tile order back to token order.
- *   rows bf16 [P, H] (nvfp4_grouped_gemm DOWN); ids int32 [T, k] and plan from
- *   the same routing; out bf16 [T, k, H]: out[t, j] = rows[p] with p =
+ *   rows fp32 [P, H] (nvfp4_grouped_gemm DOWN); ids int32 [T, k] and plan from
+ *   the same routing; out fp32 [T, k, H]: out[t, j] = rows[p] with p =
  *   tile_offsets[e] * 256 + inv[a] - offsets[e] for a = t*k + j, e = ids[a]
  *   local; zeros for remote assignments.
  */
-moe_status_t moe_unpermute(const moe_config_t* cfg, const uint16_t* rows, int32_t T, const moe_plan_t* plan,
-                           const int32_t* ids, uint16_t* out, void* stream);
+moe_status_t moe_unpermute(const moe_config_t* cfg, const float* rows, int32_t T, const moe_plan_t* plan,
+                           const int32_t* ids, float* out, void* stream);
 
 /*
  * Unpermute fused with moe_combine (the prefill's last step): y[t] =
  * bf16( sum_{j=0}^{k-1} rows[p(t, j)] + shared[t] ), j ascending, then the
- * unscaled shared row (NULL = none), fp32 accumulation, one rounding; a remote
- * assignment adds a zero row. Same result as moe_unpermute then moe_combine.
+ * unscaled shared row (fp32 [T, H], NULL = none), fp32 accumulation, one
+ * rounding; rows fp32 [P, H]; a remote assignment adds a zero row. Same
+ * result as moe_unpermute then moe_combine_f32.
  */
-moe_status_t moe_unpermute_combine(const moe_config_t* cfg, const uint16_t* rows, int32_t T, const moe_plan_t* plan,
-                                   const int32_t* ids, const uint16_t* shared, uint16_t* y, void* stream);
+moe_status_t moe_unpermute_combine(const moe_config_t* cfg, const float* rows, int32_t T, const moe_plan_t* plan,
+                                   const int32_t* ids, const float* shared, uint16_t* y, void* stream);
 
 /*
  * Clamped SwiGLU (glm5next_mlp "Traps": the clamp is asymmetric):
@@ -421,18 +422,18 @@ moe_status_t nvfp4_dequant(const uint8_t* codes, const uint8_t* scales, const fl
  *   MOE_PATH_DECODE: W4A16 GEMV experts (nvfp4_expert_gemv) with h, the
  *     routed rows r and the shared row kept in fp32 up to the combine's one
  *     bf16 rounding.
- *     T = 1 (H % 256 == 0, H <= 8192, I <= 2048, k <= 16, E <= 1024): three
- *     launches chained by programmatic dependent launch -- (1) router logits,
- *     with the top-k and the routing plan run by the last router CTA to
- *     finish, and the shared expert's gate/up in the same grid; (2) the routed
- *     experts' gate/up, one CTA per SM streaming weights through a ring of bulk
- *     copies; (3) each CTA a block of output rows: the routed and shared down
- *     rows of that block and the combine. No auxiliary stream.
- *     T > 1: router; top-k with the routing plan (one launch up to 8 tokens,
- *     E <= 320); the two expert GEMVs; moe_combine_f32; the launches are
- *     chained by programmatic dependent launch; the shared expert runs on the
+ *     Launches, chained by programmatic dependent launch: router logits
+ *     (with max |x| per token); top-k with the routing plan (one launch up to
+ *     8 tokens, E <= 320, else top-k and the permute); the routed experts'
+ *     gate/up and down; moe_combine_f32. The shared expert runs on the
  *     library's auxiliary stream of this host thread and device, forked from
  *     and joined back into `stream` with events.
+ *     T = 1 with H % 512 == 0, H <= 8192, I % 256 == 0, I <= 2048, k <= 16,
+ *     E <= 1024: the expert projections run on the tensor cores, one CTA per
+ *     SM streaming 16-row weight tiles through a TMA ring into mma.sync
+ *     (each E2M1 code times its E4M3 scale exact in f16, x or h scaled by a
+ *     power of two into f16, fp32 accumulation). Otherwise the GEMV kernels
+ *     of nvfp4_expert_gemv.
  *   MOE_PATH_PREFILL_W4A16: the pages' prefill numerics: permute with the
  *     padded tile layout, x gathered to f16 rows (per-row power-of-two scale),
  *     grouped W4A16 GEMM gate/up (nvfp4_grouped_gemm_w4a16) with the clamped
@@ -451,11 +452,12 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
 
 /* Device pointers (inside ws) of the intermediates moe_forward leaves behind:
  * logits fp32 [T,E], ids int32 [T,k], weights fp32 [T,k], the plan; h (decode:
- * fp32 [T*k, I]; prefill: bf16 [P, I] in padded tile rows); r (decode: fp32
- * [T*k, H] in token order; prefill: bf16 [P, H] in the padded tile order);
- * shared (decode: fp32 [T, H]; prefill: bf16 [T, H]; NULL when Is == 0); and on
- * the prefill path the NVFP4-encoded x and h in padded tile rows (codes, scale
- * atoms, row scales; NULL on the decode path). Host-only pointer arithmetic. */
+ * fp32 [T*k, I]; prefill: [P, I] in padded tile rows, bf16 on MOE_PATH_PREFILL,
+ * f16 on MOE_PATH_PREFILL_W4A16); r (fp32; decode: [T*k, H] in token order;
+ * prefill: [P, H] in the padded tile order); shared (fp32 [T, H]; NULL when
+ * Is == 0); and on MOE_PATH_PREFILL the NVFP4-encoded x and h in padded tile
+ * rows (codes, scale atoms, row scales; NULL otherwise). Host-only pointer
+ * arithmetic. */
 typedef struct {
   float* logits;
   int32_t* ids;

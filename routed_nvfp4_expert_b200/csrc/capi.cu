@@ -201,11 +201,13 @@ WsLayout ws_layout(const moe_config_t* c, int T, int path) {
   const bool w4 = path == MOE_PATH_PREFILL_W4A16;
   const bool pre = path == MOE_PATH_PREFILL || w4;
   const size_t P = (size_t)L.pl.P;
-  // decode keeps h, r and the shared row in fp32; the prefill's are 16-bit
+  // the routed rows r and the shared row are fp32 on every path (the combine
+  // sums them in fp32 and rounds y once); h is fp32 at decode, 16-bit in the
+  // prefill's padded tile rows
   L.h = o; o = up(o + (pre ? 2 * P : 4 * A) * I);
-  L.r = o; o = up(o + (pre ? 2 * P : 4 * A) * H);   // prefill: down rows in the padded tile order
+  L.r = o; o = up(o + 4 * (pre ? P : A) * H);   // prefill: down rows in the padded tile order
   L.shared_h = o; o = up(o + 4 * (size_t)T * Is);
-  L.shared = o; o = up(o + (pre ? 2 : 4) * (size_t)T * H);
+  L.shared = o; o = up(o + 4 * (size_t)T * H);
   L.xmax = o; o = up(o + 4 * (size_t)T);
   if (w4) {                                   // x as f16 rows in the padded tile order, their unscales
     L.xq = o; o = up(o + P * H * 2);
@@ -249,7 +251,7 @@ bool router_on_tensor_cores(const moe_config_t* c, int T, const moe_weights_t* w
 
 rnx::Fp4GemmArgs gemm_args(const moe_config_t* c, int proj, const uint8_t* codes, const uint8_t* sf,
                            const float* scale, int64_t P, const moe_plan_t& plan, const float* weights,
-                           const moe_weights_t* w, uint16_t* out, uint32_t* status) {
+                           const moe_weights_t* w, void* out, uint32_t* status) {
   const PreparedLayout PL = prepared_layout(c);
   rnx::Fp4GemmArgs g{};
   g.gate_up = proj == MOE_PROJ_GATE_UP;
@@ -278,7 +280,7 @@ rnx::Fp4GemmArgs gemm_args(const moe_config_t* c, int proj, const uint8_t* codes
 
 rnx::W4a16GemmArgs w4a16_args(const moe_config_t* c, int proj, const uint16_t* act, const float* act_scale,
                               int64_t P, const moe_plan_t& plan, const float* weights, const moe_weights_t* w,
-                              uint16_t* out, uint32_t* status) {
+                              void* out, uint32_t* status) {
   const PreparedLayout PL = prepared_layout(c);
   rnx::W4a16GemmArgs g{};
   g.gate_up = proj == MOE_PROJ_GATE_UP;
@@ -426,7 +428,7 @@ moe_status_t nvfp4_quantize_rows(const uint16_t* src, int32_t rows, int32_t K, u
 
 moe_status_t nvfp4_grouped_gemm(const moe_config_t* cfg, int32_t proj, const uint8_t* act_codes,
                                 const uint8_t* act_sf, const float* act_scale, int32_t T, const moe_plan_t* plan,
-                                const float* weights, const moe_weights_t* w, uint16_t* out, void* ws,
+                                const float* weights, const moe_weights_t* w, void* out, void* ws,
                                 size_t ws_bytes, void* stream) {
   moe_status_t s;
   if ((s = check_cfg(cfg)) != MOE_OK || (s = check_T(T)) != MOE_OK || (s = check_prefill_shape(cfg)) != MOE_OK)
@@ -462,7 +464,7 @@ moe_status_t nvfp4_grouped_gemm(const moe_config_t* cfg, int32_t proj, const uin
 
 moe_status_t nvfp4_grouped_gemm_w4a16(const moe_config_t* cfg, int32_t proj, const uint16_t* act,
                                       const float* act_scale, int32_t T, const moe_plan_t* plan, const float* weights,
-                                      const moe_weights_t* w, uint16_t* out, void* ws, size_t ws_bytes, void* stream) {
+                                      const moe_weights_t* w, void* out, void* ws, size_t ws_bytes, void* stream) {
   moe_status_t s;
   if ((s = check_cfg(cfg)) != MOE_OK || (s = check_T(T)) != MOE_OK || (s = check_prefill_shape(cfg)) != MOE_OK)
     return s;
@@ -491,8 +493,8 @@ moe_status_t nvfp4_grouped_gemm_w4a16(const moe_config_t* cfg, int32_t proj, con
   return MOE_OK;
 }
 
-moe_status_t moe_unpermute(const moe_config_t* cfg, const uint16_t* rows, int32_t T, const moe_plan_t* plan,
-                           const int32_t* ids, uint16_t* out, void* stream) {
+moe_status_t moe_unpermute(const moe_config_t* cfg, const float* rows, int32_t T, const moe_plan_t* plan,
+                           const int32_t* ids, float* out, void* stream) {
   moe_status_t s;
   if ((s = check_cfg(cfg)) != MOE_OK || (s = check_T(T)) != MOE_OK) return s;
   if (T == 0) return MOE_OK;
@@ -509,8 +511,8 @@ moe_status_t moe_unpermute(const moe_config_t* cfg, const uint16_t* rows, int32_
   return MOE_OK;
 }
 
-moe_status_t moe_unpermute_combine(const moe_config_t* cfg, const uint16_t* rows, int32_t T, const moe_plan_t* plan,
-                                   const int32_t* ids, const uint16_t* shared, uint16_t* y, void* stream) {
+moe_status_t moe_unpermute_combine(const moe_config_t* cfg, const float* rows, int32_t T, const moe_plan_t* plan,
+                                   const int32_t* ids, const float* shared, uint16_t* y, void* stream) {
   moe_status_t s;
   if ((s = check_cfg(cfg)) != MOE_OK || (s = check_T(T)) != MOE_OK) return s;
   if (T == 0) return MOE_OK;
@@ -627,14 +629,14 @@ moe_status_t nvfp4_expert_gemv(const moe_config_t* cfg, int32_t proj, const void
   uint32_t* status = (uint32_t*)(b + L.status);
   RNX_CUDA(cudaMemsetAsync(status, 0, kCtrlBytes, st), "clear status");
   const int H = cfg->hidden, I = cfg->intermediate, k = cfg->top_k;
-  if (T == 1 && rnx::decode_t1_supported(H, I, 0, cfg->num_experts, k)) {
-    // one token: the streamed single-token kernels, fed from the plan
+  if (T == 1 && rnx::decode_t1_supported(H, I, cfg->num_experts, k)) {
+    // one token: the tensor-core single-token kernels, fed from the plan
     rnx::DecodeT1Args a{};
-    a.H = H; a.I = I; a.Is = 0; a.E = cfg->num_experts; a.k = k;
+    a.H = H; a.I = I; a.E = cfg->num_experts; a.k = k;
     a.lb = cfg->local_begin; a.le = cfg->local_end;
     a.limit = cfg->swiglu_limit;
     a.gate = w->gate; a.up = w->up; a.down = w->down;
-    a.ids = nullptr; a.active = plan->active; a.first = plan->first;
+    a.active = plan->active; a.first = plan->first;
     a.status = status;
     if (proj == MOE_PROJ_GATE_UP) {
       uint32_t* xmax = (uint32_t*)(b + L.xmax);
@@ -642,7 +644,7 @@ moe_status_t nvfp4_expert_gemv(const moe_config_t* cfg, int32_t proj, const void
       a.x = (const uint16_t*)act; a.xmax = xmax; a.h = out;
       RNX_CUDA(rnx::launch_decode_t1_gate_up(a, st), "nvfp4_expert_gemv (gate/up)");
     } else {
-      a.h = (float*)act; a.weights = (float*)weights; a.r = out;
+      a.h = (float*)act; a.weights = weights; a.r = out;
       RNX_CUDA(rnx::launch_decode_t1_down(a, st), "nvfp4_expert_gemv (down)");
     }
     return MOE_OK;
@@ -719,7 +721,7 @@ moe_status_t dense_ffn_bf16(int32_t H, int32_t I, float limit, const uint16_t* x
   void* hbuf = (char*)ws + up(4);
   cudaStream_t st = (cudaStream_t)stream;
   RNX_CUDA(cudaMemsetAsync(ws, 0, 4, st), "clear status");
-  RNX_CUDA(rnx::launch_dense_ffn(H, I, limit, x, T, wg, wu, wd, y, hbuf, (uint32_t*)ws, st), "dense_ffn_bf16");
+  RNX_CUDA(rnx::launch_dense_ffn(H, I, limit, x, T, wg, wu, wd, y, false, hbuf, (uint32_t*)ws, st), "dense_ffn_bf16");
   return MOE_OK;
 }
 
@@ -786,10 +788,10 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
              "shared expert");
     RNX_CUDA(cudaEventRecord(side->join, side->st), "join event");
   }
-  // one token: the streamed expert kernels (one CTA per SM, weights through a
-  // ring of bulk copies), fed from the routing plan; the router's GEMV also
+  // one token: the tensor-core expert kernels (one CTA per SM, weight tiles
+  // through a TMA ring), fed from the routing plan; the router's GEMV also
   // leaves max |x| for their f16 pre-scale
-  const bool t1 = decode && T == 1 && rnx::decode_t1_supported(H, I, 0, E, k);
+  const bool t1 = decode && T == 1 && rnx::decode_t1_supported(H, I, E, k);
   uint32_t* xmax = (uint32_t*)(b + L.xmax);
   RNX_CUDA(mark(MOE_STAGE_ROUTER_LOGITS, st), "stage event");
   if (!decode && router_on_tensor_cores(cfg, T, w)) {
@@ -821,7 +823,7 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
     // tensor cores (kind::f16), x gathered into the padded tile order as f16
     const int64_t P = L.pl.P;
     uint16_t* h = (uint16_t*)(b + L.h);
-    uint16_t* r = (uint16_t*)(b + L.r);
+    float* r = (float*)(b + L.r);
     uint16_t* xa = (uint16_t*)(b + L.xq);
     float* xs = (float*)(b + L.xts);
     const int32_t* used_tiles = plan.tile_offsets + E;
@@ -837,15 +839,15 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
     RNX_CUDA(mark(MOE_STAGE_SHARED, st), "stage event");
     if (Is > 0)
       RNX_CUDA(rnx::launch_dense_ffn(H, Is, cfg->swiglu_limit, x, T, w->shared_gate, w->shared_up, w->shared_down,
-                                     (uint16_t*)shared, b + L.shared_h, status, st),
+                                     shared, true, b + L.shared_h, status, st),
                "shared expert");
     RNX_CUDA(mark(MOE_STAGE_COMBINE, st), "stage event");
     const rnx::PaddedIndex q{ids, plan.inv, plan.offsets, plan.tile_offsets, cfg->local_begin, cfg->local_end};
-    RNX_CUDA(rnx::launch_unpermute_combine(q, T, k, H, r, (const uint16_t*)shared, y, st), "unpermute + combine");
+    RNX_CUDA(rnx::launch_unpermute_combine(q, T, k, H, r, (const float*)shared, y, st), "unpermute + combine");
   } else if (!decode) {
     const int64_t P = L.pl.P;
     uint16_t* h = (uint16_t*)(b + L.h);
-    uint16_t* r = (uint16_t*)(b + L.r);
+    float* r = (float*)(b + L.r);
     uint8_t* xq = (uint8_t*)(b + L.xq);
     uint8_t* xsf = (uint8_t*)(b + L.xsf);
     float* xts = (float*)(b + L.xts);
@@ -868,11 +870,11 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
     RNX_CUDA(mark(MOE_STAGE_SHARED, st), "stage event");
     if (Is > 0)
       RNX_CUDA(rnx::launch_dense_ffn(H, Is, cfg->swiglu_limit, x, T, w->shared_gate, w->shared_up, w->shared_down,
-                                     (uint16_t*)shared, b + L.shared_h, status, st),
+                                     shared, true, b + L.shared_h, status, st),
                "shared expert");
     RNX_CUDA(mark(MOE_STAGE_COMBINE, st), "stage event");
     const rnx::PaddedIndex q{ids, plan.inv, plan.offsets, plan.tile_offsets, cfg->local_begin, cfg->local_end};
-    RNX_CUDA(rnx::launch_unpermute_combine(q, T, k, H, r, (const uint16_t*)shared, y, st), "unpermute + combine");
+    RNX_CUDA(rnx::launch_unpermute_combine(q, T, k, H, r, (const float*)shared, y, st), "unpermute + combine");
   } else {
     float* h = (float*)(b + L.h);
     float* r = (float*)(b + L.r);
@@ -886,12 +888,12 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
     a.status = status;
     if (t1) {
       rnx::DecodeT1Args d{};
-      d.H = H; d.I = I; d.Is = 0; d.E = E; d.k = k;
+      d.H = H; d.I = I; d.E = E; d.k = k;
       d.lb = cfg->local_begin; d.le = cfg->local_end;
       d.limit = cfg->swiglu_limit;
       d.x = x;
       d.gate = w->gate; d.up = w->up; d.down = w->down;
-      d.ids = nullptr; d.active = plan.active; d.first = plan.first;
+      d.active = plan.active; d.first = plan.first;
       d.weights = wts; d.xmax = xmax; d.h = h; d.r = r;
       d.status = status;
       RNX_CUDA(mark(MOE_STAGE_EXPERT_GATE_UP, st), "stage event");

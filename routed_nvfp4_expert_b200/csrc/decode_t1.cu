@@ -1,686 +1,561 @@
-// Single-token decode of the routed MoE site in three launches chained by
-// programmatic dependent launch (glm5next_mlp module docs, "The stack this
-// layer runs"; Constants / W4A16_GEMV_MODULE: at decode every routed-expert
-// projection is M = 1, so the step is a stream over the touched experts'
-// bytes):
+// Single-token decode of the routed experts on the tensor cores
+// (glm5next_mlp module docs, Constants / W4A16_GEMV_MODULE: at decode every
+// routed-expert projection is M = 1, so the step is a stream over the touched
+// experts' bytes). Two launches chained by programmatic dependent launch:
 //
-//   K1  router logits (fp32 gate.weight . x) + sigmoid top-k by the last
-//       router CTA to finish, and, in the same grid, the BF16 shared expert's
-//       gate/up with its clamped SwiGLU (h_shared, fp32);
-//   K2  the routed experts' NVFP4 gate/up with the clamped SwiGLU (h, fp32),
-//       streamed through a ring of bulk copies (TMA engine) in shared memory
-//       by one producer warp per CTA, one CTA per SM; the producer warp
-//       finally asks L2 for the slice of down weights that K3's CTA of the
-//       same index will read;
-//   K3  each CTA owns a block of output rows: the routed NVFP4 down rows of
-//       every chosen expert and the shared expert's BF16 down rows for that
-//       block, all loaded at once by bulk copies issued before it waits for
-//       K2, then moe_combine on the spot: y = bf16(sum_j w_j o_j + shared),
-//       j in rank order, fp32 throughout (the combine happens before any
-//       reduce: section "Why one all-reduce covers BOTH EP and TP").
+//   gate/up  the live experts' NVFP4 gate and up rows against x, with the
+//            clamped SwiGLU (h, fp32 [k, I]);
+//   down     the live experts' NVFP4 down rows against h, times the routing
+//            weight (r, fp32 [k, H]; rows of assignments that are not live are
+//            zero). moe_combine then sums r and the shared row.
 //
-// Arithmetic: NVFP4 codes are decoded to f16 with the hardware cvt; the
-// activation (x, or h) is scaled by a power of two per row into f16 (a bf16
-// x is exact there, an fp32 h keeps 11 significant bits); every
-// product code * activation is exact and accumulated in fp32 by the
-// mixed-precision fma (f16 inputs, fp32 accumulator); each 16-element block
-// sum is scaled by its E4M3 scale in fp32.
+// Both kernels run one CTA per SM: a producer warp streams 16-row tiles of
+// codes and E4M3 scales into a ring of shared-memory stages with TMA (128-byte
+// swizzle for the codes), sixteen consumer warps multiply them on the tensor
+// cores with mma.sync m16n8k16 (f16 operands, fp32 accumulators).
+//
+// Arithmetic. A 16-row weight tile is the A operand: each E2M1 code is decoded
+// to f16 by the hardware cvt and multiplied (f16) by its block's E4M3 scale;
+// the product has at most 6 significant bits and lies in [2^-10, 2688], so it
+// is exact in f16. The activation (x, or h) times a per-row power of two
+// (max |a| in [2^14, 2^15)) in f16 is the B operand, column 0 (the other seven
+// columns are zero). Every product is exact in the tensor core's fp32
+// accumulation, so only the fp32 sums round; the power of two and the tensor
+// scale are applied to the fp32 totals.
+//
+// K order. The 16 k-slots of one mma hold, in the A fragment of lane (g, t),
+// four consecutive codes of the 32 that lane loaded (one 16-byte word of its
+// row); B holds the activation at the same positions. A dot product does not
+// depend on the order of its terms, so this is the plain row . activation.
 
 #include "common.cuh"
-#include "kernels.h"
 #include "gemv_common.cuh"
+#include "kernels.h"
+#include "tc.cuh"
+#include "tensor_map.h"
 #include "tma.cuh"
-#include "topk.cuh"
 
 namespace rnx {
 
 namespace {
 
-// Self-checks of the data-dependent accesses (built with -DRNX_DEVICE_CHECKS):
-// a failed check ORs the bounds bit and the check's id (bits 8..15) into the
-// status word and skips the access.
-#ifdef RNX_DEVICE_CHECKS
-#define RNX_DCHECK(cond, id, status) (((cond)) ? true : (set_status((status), kDevErrBounds | ((uint32_t)(id) << 8)), false))
-#else
-#define RNX_DCHECK(cond, id, status) true
-#endif
-RNX_DEVICE bool al16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+constexpr int kMaxLive = 16;               // top-k <= 16
+// Consumer warps per CTA. A gate/up consumer holds its ring stage while it
+// computes, so the ring keeps NS - kGuConsumers stages of copies in flight;
+// the down kernel has its whole share of tiles in flight before it starts.
+constexpr int kGuConsumers = 8;
+constexpr int kDnConsumers = 16;
+constexpr int kGuThreads = (kGuConsumers + 1) * kWarp;
+constexpr int kDnThreads = (kDnConsumers + 1) * kWarp;
+// Status bits 8..13 name the bounded wait that ran out.
+enum : uint32_t {
+  kWaitGuEmpty = 1u << 8,
+  kWaitGuFull = 1u << 9,
+  kWaitGuDrain = 1u << 10,
+  kWaitDnEmpty = 1u << 11,
+  kWaitDnFull = 1u << 12,
+  kWaitDnDrain = 1u << 13,
+};
+constexpr int kSmemBudget = 200 * 1024;
+constexpr int kBox = 2048;                 // one code box: 16 rows x 128 bytes (256 codes)
+constexpr int kGuCodes = 512;              // codes per row in one gate/up stage
+constexpr int kGuStage = 4 * kBox + 2 * 16 * (kGuCodes / 16);   // gate, up boxes + their scales: 9216
+constexpr int kMaxStages = 24;
 
 RNX_DEVICE void named_bar_sync(int id, int nthreads) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory"); }
 
-// The token's live assignments (expert inside the local range, id valid), in
-// assignment order: from ids[0..k) (slot j = assignment j), or from a routing
-// plan's active list (expert order; first[u] = the assignment). One thread.
-// s_live[0] = count, s_live[1 + u] = expert, s_live[1 + kMaxK + u] = assignment.
-constexpr int kMaxK = 16;
-RNX_DEVICE void build_live(const int32_t* ids, const int32_t* active, const int32_t* first, int k, int E, int lb,
-                           int le, uint32_t* status, bool report, int* s_live) {
-  int n = 0;
-  if (ids) {
-    for (int j = 0; j < k; ++j) {
-      const int e = ids[j];
-      if (e < 0 || e >= E) {
-        if (report) set_status(status, kDevErrBounds);
-        continue;
+// mma tile row of fragment row g (0..7): rows g and g + 1 (the two row
+// groups one shared-memory wavefront serves) sit 4 apart in the tile, so their
+// swizzled 16-byte words fall in opposite halves of the 128-byte line.
+RNX_DEVICE int tile_row(int g) { return ((g & 1) << 2) | (g >> 1); }
+
+RNX_DEVICE uint32_t e4m3x2_to_f16x2(uint16_t s) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(s));
+  return h;
+}
+RNX_DEVICE uint32_t hmul2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+RNX_DEVICE uint32_t lo_lo(uint32_t v) { return __byte_perm(v, 0u, 0x1010); }
+RNX_DEVICE uint32_t hi_hi(uint32_t v) { return __byte_perm(v, 0u, 0x3232); }
+
+RNX_DEVICE void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                          uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// One warp's share of a stage: NM matrices (mat_stride bytes apart; scales
+// sf_stride apart, sp bytes per scale row) of 16 rows x (2 npair) chunks of
+// 128 codes, against the B fragments bf of those chunks (8 per chunk, one
+// uint2 per lane t). Codes sit in boxes of 16 rows x 128 bytes written by TMA
+// with the 128-byte swizzle (16-byte word w of row r at w ^ (r & 7)).
+// acc[m][c & 1] accumulates chunk c (two chains per matrix).
+template <int NM>
+RNX_DEVICE void stage_mma(const uint8_t* st, int mat_stride, const uint8_t* sf, int sf_stride, int sp, int npair,
+                          const uint2* bf, bool b_on, int g, int t, float (&acc)[NM][2][4]) {
+  const int r0 = tile_row(g);
+  for (int cp = 0; cp < npair; ++cp) {
+#pragma unroll
+    for (int hc = 0; hc < 2; ++hc) {
+      const int c = 2 * cp + hc;
+      const int o0 = cp * kBox + r0 * 128 + ((((hc << 2) | t) ^ r0) << 4);   // row r0 + 8: o0 + 1024
+      uint2 b[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) b[i] = b_on ? bf[(c * 8 + i) * 4 + t] : make_uint2(0u, 0u);
+#pragma unroll
+      for (int m = 0; m < NM; ++m) {
+        const uint8_t* cm = st + m * mat_stride;
+        const uint4 q0 = *reinterpret_cast<const uint4*>(cm + o0);
+        const uint4 q1 = *reinterpret_cast<const uint4*>(cm + o0 + 1024);
+        const uint8_t* sm = sf + m * sf_stride + 8 * c + 2 * t;
+        const uint32_t s0 = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(sm + r0 * sp));
+        const uint32_t s1 = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(sm + (r0 + 8) * sp));
+        uint32_t w0[16], w1[16];
+        e2m1x8_to_f16x2x4(q0.x, w0[0], w0[1], w0[2], w0[3]);
+        e2m1x8_to_f16x2x4(q0.y, w0[4], w0[5], w0[6], w0[7]);
+        e2m1x8_to_f16x2x4(q0.z, w0[8], w0[9], w0[10], w0[11]);
+        e2m1x8_to_f16x2x4(q0.w, w0[12], w0[13], w0[14], w0[15]);
+        e2m1x8_to_f16x2x4(q1.x, w1[0], w1[1], w1[2], w1[3]);
+        e2m1x8_to_f16x2x4(q1.y, w1[4], w1[5], w1[6], w1[7]);
+        e2m1x8_to_f16x2x4(q1.z, w1[8], w1[9], w1[10], w1[11]);
+        e2m1x8_to_f16x2x4(q1.w, w1[12], w1[13], w1[14], w1[15]);
+        // the lane's 32 codes are two 16-code blocks: words 0..7, 8..15
+        const uint32_t s0a = lo_lo(s0), s0b = hi_hi(s0), s1a = lo_lo(s1), s1b = hi_hi(s1);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t sc0 = i < 4 ? s0a : s0b, sc1 = i < 4 ? s1a : s1b;
+          mma_16816(acc[m][hc], hmul2(w0[2 * i], sc0), hmul2(w1[2 * i], sc1), hmul2(w0[2 * i + 1], sc0),
+                    hmul2(w1[2 * i + 1], sc1), b[i].x, b[i].y);
+        }
       }
-      if (e < lb || e >= le) continue;
-      s_live[1 + n] = e;
-      s_live[1 + kMaxK + n] = j;
+    }
+  }
+}
+
+// The token's live experts from the routing plan (active list, expert order;
+// first[u] = the assignment), kept only when the id and assignment are in
+// range: s_live[0] = count, s_live[1 + u] = expert, s_live[1 + kMaxLive + u] =
+// assignment, s_ts[u] / s_ts[kMaxLive + u] = the two tensor scales asked for
+// (bank0, bank1; bank1 may be null). All threads call it (two barriers).
+RNX_DEVICE void load_live(const DecodeT1Args& p, const float* ts0, const float* ts1, int* s_tmp, int* s_live,
+                          float* s_ts) {
+  const int u = threadIdx.x;
+  if (u < kMaxLive) {
+    // one round for the count, the ids and the assignments (entries past the
+    // count are read but not used; the arrays hold at least E entries), one
+    // for the tensor scales
+    const int n = min(p.active[0], kMaxLive);
+    int e = -1, a = -1;
+    if (u < p.E) {
+      e = p.active[1 + u];
+      a = p.first[u];
+    }
+    const bool ok = u < n && e >= 0 && e < p.E && e >= p.lb && e < p.le && a >= 0 && a < p.k;
+    if (u < n && !ok && blockIdx.x == 0) set_status(p.status, kDevErrBounds);
+    float t0 = 0.f, t1 = 0.f;
+    if (ok) {
+      t0 = ts0[e];
+      if (ts1) t1 = ts1[e];
+    }
+    s_tmp[u] = ok ? e : -1;
+    s_tmp[kMaxLive + u] = a;
+    reinterpret_cast<float*>(s_tmp)[2 * kMaxLive + u] = t0;
+    reinterpret_cast<float*>(s_tmp)[3 * kMaxLive + u] = t1;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int n = 0;
+    for (int v = 0; v < kMaxLive; ++v) {
+      if (s_tmp[v] < 0) continue;
+      s_live[1 + n] = s_tmp[v];
+      s_live[1 + kMaxLive + n] = s_tmp[kMaxLive + v];
+      s_ts[n] = reinterpret_cast<float*>(s_tmp)[2 * kMaxLive + v];
+      s_ts[kMaxLive + n] = reinterpret_cast<float*>(s_tmp)[3 * kMaxLive + v];
       ++n;
     }
-  } else {
-    n = min(active[0], kMaxK);
-    for (int u = 0; u < n; ++u) {
-      s_live[1 + u] = active[1 + u];
-      s_live[1 + kMaxK + u] = first[u];
-    }
+    s_live[0] = n;
   }
-  s_live[0] = n;
-}
-
-// Balanced split of H output rows over G CTAs: CTA c owns [row_begin(c), row_begin(c + 1)).
-RNX_DEVICE __host__ int row_begin(int c, int H, int G) { return (int)(((long long)c * H) / G); }
-
-// ============================================================== K1
-constexpr int kK1Threads = 256;
-constexpr int kK1MaxQ = 16;        // router: H / 512 float4 per thread (H <= 8192)
-constexpr int kK1SharedRound = 8;  // shared gate/up: uint4 of each row per lane per round
-
-template <int PL>
-__global__ void __launch_bounds__(kK1Threads, 2) k1_router_topk_shared(DecodeT1Args p) {
-  __shared__ float red[8];
-  __shared__ int s_last;
-  __shared__ float s_key[1][32 * PL];
-  __shared__ float s_sig[1][32 * PL];
-  __shared__ __align__(16) uint16_t s_x[8192];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n_router = (p.E + 1) / 2;
-  const int H = p.H;
-
-  if ((int)blockIdx.x < n_router) {
-    // ---------------------------------------------------------- router
-    const int half = warp >> 2, th = tid & 127;
-    const int e = 2 * blockIdx.x + half;
-    const bool e_on = e < p.E;
-    const int nq = H >> 2;
-    const float4* wrow = reinterpret_cast<const float4*>(p.router_w + (size_t)(e_on ? e : 0) * H);
-    float4 w[kK1MaxQ];
-#pragma unroll
-    for (int i = 0; i < kK1MaxQ; ++i) {
-      const int c = th + 128 * i;
-      w[i] = (e_on && c < nq) ? __ldg(wrow + c) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    pdl_wait();
-    pdl_trigger();
-    float acc = 0.f;
-#pragma unroll
-    for (int i = 0; i < kK1MaxQ; ++i) {
-      const int c = th + 128 * i;
-      if (c < nq) {
-        const uint2 xv = *reinterpret_cast<const uint2*>(p.x + 4 * c);
-        const float2 a = bf16x2_to_f32x2(xv.x), b = bf16x2_to_f32x2(xv.y);
-        acc = fmaf(w[i].x, a.x, acc);
-        acc = fmaf(w[i].y, a.y, acc);
-        acc = fmaf(w[i].z, b.x, acc);
-        acc = fmaf(w[i].w, b.y, acc);
-      }
-    }
-    acc = warp_sum(acc);
-    if (lane == 0) red[warp] = acc;
-    if (blockIdx.x == 0) {
-      // max |x| for the gate/up pass's f16 pre-scale
-      float m = 0.f;
-      for (int g = tid; g < H / 8; g += kK1Threads) {
-        const uint4 v = reinterpret_cast<const uint4*>(p.x)[g];
-        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float2 f = bf16x2_to_f32x2(w4[j]);
-          m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
-        }
-      }
-      m = warp_max(m);
-      __syncthreads();
-      if (lane == 0) s_key[0][warp] = m;
-      __syncthreads();
-      if (tid == 0) {
-        float mm = 0.f;
-        for (int i = 0; i < 8; ++i) mm = fmaxf(mm, s_key[0][i]);
-        *p.xmax = __float_as_uint(mm);
-      }
-    }
-    __syncthreads();
-    if (tid < 2 && 2 * (int)blockIdx.x + tid < p.E) {
-      const float v = ((red[4 * tid] + red[4 * tid + 1]) + red[4 * tid + 2]) + red[4 * tid + 3];
-      p.logits[2 * blockIdx.x + tid] = v;
-    }
-    // the last router CTA to finish runs the selection
-    __syncthreads();
-    if (tid == 0) {
-      __threadfence();
-      const unsigned prev = atomicAdd(p.ticket, 1u);
-      s_last = prev == (unsigned)(n_router - 1);
-    }
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    // selection keys from the (now complete) logits, then one warp selects
-    for (int i = tid; i < p.E; i += kK1Threads) {
-      const float l = __ldcg(p.logits + i);
-      const float sg = (float)(1.0 / (1.0 + exp(-(double)l)));
-      s_sig[0][i] = sg;
-      s_key[0][i] = __fadd_rn(sg, p.router_bias[i]);
-    }
-    __syncthreads();
-    if (warp == 0) topk_warp<PL>(s_key[0], s_sig[0], 0, p.E, p.k, p.rsf, p.ids, p.weights);
-    __syncthreads();                       // ids visible to the whole CTA
-    if (p.plan.counts) {
-      // the routing plan of one token (counts, offsets, sorted, inv, tile
-      // offsets, active list, first): k distinct ids, O(E k) per CTA
-      int id[kMaxK];
-      bool valid[kMaxK];
-#pragma unroll
-      for (int j = 0; j < kMaxK; ++j) {
-        id[j] = j < p.k ? p.ids[j] : -1;
-        valid[j] = j < p.k && id[j] >= 0 && id[j] < p.E;
-      }
-      for (int e = tid; e <= p.E; e += kK1Threads) {
-        int cnt = 0, off = 0, toff = 0;
-#pragma unroll
-        for (int j = 0; j < kMaxK; ++j) {
-          if (!valid[j]) continue;
-          cnt += id[j] == e;
-          off += id[j] < e;
-          toff += (id[j] < e && id[j] >= p.lb && id[j] < p.le);
-        }
-        if (e < p.E) p.plan.counts[e] = cnt;
-        p.plan.offsets[e] = off;
-        p.plan.tile_offsets[e] = toff;
-      }
-      if (tid < p.k) {
-        const int j = tid;
-        if (valid[j]) {
-          int pos = 0, lpos = 0;
-#pragma unroll
-          for (int i = 0; i < kMaxK; ++i) {
-            pos += valid[i] && id[i] < id[j];
-            lpos += valid[i] && id[i] < id[j] && id[i] >= p.lb && id[i] < p.le;
-          }
-          p.plan.sorted[pos] = j;
-          p.plan.inv[j] = pos;
-          if (id[j] >= p.lb && id[j] < p.le) {
-            p.plan.active[1 + lpos] = id[j];
-            p.plan.first[lpos] = j;
-          }
-        } else {
-          p.plan.inv[j] = -1;
-          set_status(p.status, kDevErrBounds);
-        }
-      }
-      if (tid == 0) {
-        int nl = 0;
-#pragma unroll
-        for (int j = 0; j < kMaxK; ++j) nl += valid[j] && id[j] >= p.lb && id[j] < p.le;
-        p.plan.active[0] = nl;
-      }
-    }
-    return;
-  }
-
-  // ------------------------------------------------------------ shared gate/up
-  // one row pair (gate row, up row) per warp; weights stream in rounds of
-  // 8 uint4 per row per lane, the first round issued before the wait
-  const int row = ((int)blockIdx.x - n_router) * 8 + warp;
-  const bool row_on = row < p.Is;
-  const int nu4 = H >> 3;                       // uint4 per row
-  const uint4* grow = reinterpret_cast<const uint4*>(p.sh_gate + (size_t)(row_on ? row : 0) * H);
-  const uint4* urow = reinterpret_cast<const uint4*>(p.sh_up + (size_t)(row_on ? row : 0) * H);
-  uint4 wg[kK1SharedRound], wu[kK1SharedRound];
-#pragma unroll
-  for (int i = 0; i < kK1SharedRound; ++i) {
-    const int c = lane + 32 * i;
-    wg[i] = (row_on && c < nu4) ? ldg_stream(grow + c) : make_uint4(0, 0, 0, 0);
-    wu[i] = (row_on && c < nu4) ? ldg_stream(urow + c) : make_uint4(0, 0, 0, 0);
-  }
-  pdl_wait();
-  pdl_trigger();
-  for (int g = tid; g < nu4; g += kK1Threads) reinterpret_cast<uint4*>(s_x)[g] = reinterpret_cast<const uint4*>(p.x)[g];
   __syncthreads();
-  float ag = 0.f, au = 0.f;
-  const int rounds = (nu4 + 32 * kK1SharedRound - 1) / (32 * kK1SharedRound);
-  for (int rd = 0; rd < rounds; ++rd) {
-    if (rd > 0) {
-#pragma unroll
-      for (int i = 0; i < kK1SharedRound; ++i) {
-        const int c = rd * 32 * kK1SharedRound + lane + 32 * i;
-        wg[i] = (row_on && c < nu4) ? ldg_stream(grow + c) : make_uint4(0, 0, 0, 0);
-        wu[i] = (row_on && c < nu4) ? ldg_stream(urow + c) : make_uint4(0, 0, 0, 0);
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < kK1SharedRound; ++i) {
-      const int c = rd * 32 * kK1SharedRound + lane + 32 * i;
-      if (c < nu4) {
-        const uint4 xv = reinterpret_cast<const uint4*>(s_x)[c];
-        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-        const uint32_t gw[4] = {wg[i].x, wg[i].y, wg[i].z, wg[i].w};
-        const uint32_t uw[4] = {wu[i].x, wu[i].y, wu[i].z, wu[i].w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 xf = bf16x2_to_f32x2(xw[q]);
-          const float2 gf = bf16x2_to_f32x2(gw[q]);
-          const float2 uf = bf16x2_to_f32x2(uw[q]);
-          ag = fmaf(gf.x, xf.x, ag);
-          ag = fmaf(gf.y, xf.y, ag);
-          au = fmaf(uf.x, xf.x, au);
-          au = fmaf(uf.y, xf.y, au);
-        }
-      }
-    }
-  }
-  ag = warp_sum(ag);
-  au = warp_sum(au);
-  if (lane == 0 && row_on) {
-    const float hv = clamped_swiglu(ag, au, p.limit);
-    p.h_shared[row] = hv;
-  }
 }
 
-// ============================================================== K2
-constexpr int kGuR = 4;                 // row pairs (gate row + up row) per stage
-constexpr int kGuKS = 4;                // K slices
-constexpr int kGuRG = 2;                // row groups (kGuR / kGuRG row pairs each)
-constexpr int kGuConsumers = kGuKS * kGuRG;
-constexpr int kGuThreads = (kGuConsumers + 1) * kWarp;
-constexpr int kGuMaxStages = 16;
-constexpr int kGuSmemBudget = 200 * 1024;
+// ============================================================== gate/up
 
-__host__ __device__ inline int gu_stage_bytes(int K) { return kGuR * K + kGuR * K / 8; }
-
-struct GuSmem {
-  int stage_bytes, nstages, bar_off, red_off, live_off, ts_off, flag_off, total;
+struct GuParams {
+  CUtensorMap gc, uc;      // gate / up codes [E I, H/2] bytes, box 128 B x 16 rows, SW128
+  CUtensorMap gs, us;      // gate / up scales [E I, H/16] bytes, box 32 B x 16 rows
+  DecodeT1Args a;
 };
-__host__ __device__ inline GuSmem gu_smem(int K) {
-  GuSmem s;
-  s.stage_bytes = gu_stage_bytes(K);
-  s.nstages = kGuSmemBudget / s.stage_bytes;
-  if (s.nstages > kGuMaxStages) s.nstages = kGuMaxStages;
-  s.bar_off = s.nstages * s.stage_bytes;
-  s.red_off = s.bar_off + 2 * s.nstages * 8;
-  s.live_off = s.red_off + 2 * kGuKS * 2 * kGuR * 4;
-  s.ts_off = s.live_off + (1 + 2 * kMaxK) * 4;
-  s.flag_off = s.ts_off + 2 * kMaxK * 4;
-  s.total = s.flag_off + 16;
-  return s;
+
+// Shared memory of one gate/up CTA (offsets from the 1024-aligned base):
+// NS ring stages, x as B fragments (H f16), NB item slots of P partial tiles
+// (gate 16 + up 16 fp32 each) with their arrival counters, barriers, the live
+// list.
+struct GuLayout {
+  int P, NS, NB, xs, part, cnt, bar, live, tmp, ts, flag, total;
+};
+__host__ __device__ inline GuLayout gu_layout(int H) {
+  GuLayout L{};
+  L.P = H / kGuCodes;
+  for (int ns = kMaxStages; ns >= 2; --ns) {
+    L.NS = ns;
+    // an item slot is reused kGuConsumers + ns stages later at the earliest:
+    // by then the warp that summed the item has released its next stage
+    L.NB = 1 + (ns + kGuConsumers - 1 + L.P - 1) / L.P;
+    L.xs = ns * kGuStage;
+    L.part = L.xs + H * 2;
+    L.cnt = L.part + L.NB * L.P * 32 * 4;
+    L.bar = (L.cnt + L.NB * 4 + 7) / 8 * 8;
+    L.live = L.bar + 2 * ns * 8;
+    L.tmp = L.live + (1 + 2 * kMaxLive) * 4;
+    L.ts = L.tmp + 4 * kMaxLive * 4;
+    L.flag = L.ts + 2 * kMaxLive * 4;
+    L.total = L.flag + 16 + 1024;     // + alignment slack of the dynamic base
+    if (L.total <= kSmemBudget) break;
+  }
+  return L;
 }
 
-template <int CPL>
-__global__ void __launch_bounds__(kGuThreads, 1) k2_gate_up(DecodeT1Args p) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  const GuSmem L = gu_smem(p.H);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar_off);
-  uint64_t* empty = full + L.nstages;
-  float* red = reinterpret_cast<float*>(smem + L.red_off);          // [2][KS][2R]
-  int* s_live = reinterpret_cast<int*>(smem + L.live_off);
-  float* s_ts = reinterpret_cast<float*>(smem + L.ts_off);           // [2][kMaxK] gate, up tensor scales
-  // iteration at which the consumers stop (set by a consumer whose wait ran
-  // out before it reaches that iteration's barrier; read after the barrier,
-  // so every consumer breaks at the same iteration)
-  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + L.flag_off);
+__global__ void __launch_bounds__(kGuThreads, 1) t1_gate_up_kernel(const __grid_constant__ GuParams prm) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const DecodeT1Args& p = prm.a;
+  const int H = p.H, I = p.I;
+  const GuLayout L = gu_layout(H);
+  const int P = L.P, NS = L.NS, NB = L.NB;
+  uint2* xs = reinterpret_cast<uint2*>(smem + L.xs);
+  float* part = reinterpret_cast<float*>(smem + L.part);
+  int* cnt = reinterpret_cast<int*>(smem + L.cnt);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar);
+  uint64_t* empty = full + NS;
+  int* s_live = reinterpret_cast<int*>(smem + L.live);
+  float* s_ts = reinterpret_cast<float*>(smem + L.ts);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + L.flag);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int K = p.H, I = p.I, NS = L.nstages;
+
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kGuConsumers);
+      mbar_init(&empty[s], 1);
     }
+    for (int b = 0; b < NB; ++b) cnt[b] = 0;
+    *s_abort = 0;
     fence_barrier_init();
-    *s_abort = 0x7fffffff;
   }
-  pdl_wait();              // ids (or the plan) and the x max come from earlier launches
+  pdl_wait();              // the plan and max |x| come from earlier launches
   pdl_trigger();
-  if (threadIdx.x == 0)
-    build_live(p.ids, p.active, p.first, p.k, p.E, p.lb, p.le, p.status, blockIdx.x == 0, s_live);
-  __syncthreads();
+  load_live(p, p.gate.tensor_scale, p.up.tensor_scale, reinterpret_cast<int*>(smem + L.tmp), s_live, s_ts);
   const int n_live = s_live[0];
-  // the live experts' tensor scales, read once (the per-item epilogue would
-  // otherwise wait on a global load every item)
-  if (threadIdx.x < n_live) {
-    s_ts[threadIdx.x] = p.gate.tensor_scale[s_live[1 + threadIdx.x]];
-    s_ts[kMaxK + threadIdx.x] = p.up.tensor_scale[s_live[1 + threadIdx.x]];
-  }
-  __syncthreads();
-  const int NB = I / kGuR;
-  const int N = n_live * NB;
-  const int G = gridDim.x, c0 = blockIdx.x;
-  const int n_mine = c0 < N ? (N - 1 - c0) / G + 1 : 0;
-  const int half_codes = kGuR * K / 2, scales_bytes = kGuR * K / 16;
+  const int TPE = I / 16;                    // 16-row tiles per expert
+  const int N = n_live * TPE, G = gridDim.x, c0 = blockIdx.x;
+  const int n_items = c0 < N ? (N - 1 - c0) / G + 1 : 0;
+  const int n_stages = n_items * P;
 
   if (warp == kGuConsumers) {
     // ---------------------------------------------------------- producer
     if (lane == 0) {
-      for (int m = 0; m < n_mine; ++m) {
-        const int i = c0 + m * G;
-        const int u = i / NB, rb = i - u * NB;
-        const int e = s_live[1 + u];
+      int issued = 0;
+      for (int m = 0; m < n_stages; ++m) {
+        if (*s_abort) break;
         const int s = m % NS;
         if (m >= NS && !mbar_wait(&empty[s], ((uint32_t)(m / NS) & 1u) ^ 1u)) {
-          set_status(p.status, kDevErrTimeout);   // consumers then run out on the stage it never fills
+          set_status(p.status, kDevErrTimeout | kWaitGuEmpty);
+          *s_abort = 1;
           break;
         }
-        uint8_t* st = smem + (size_t)s * L.stage_bytes;
-        const size_t row0 = (size_t)e * I + (size_t)rb * kGuR;
-        if (!RNX_DCHECK(e >= 0 && e < p.E && row0 + kGuR <= (size_t)p.E * I, 10, p.status)) break;
-        if (!RNX_DCHECK(al16(st) && al16(p.gate.codes + row0 * (K / 2)) && al16(p.gate.scales + row0 * (K / 16)) &&
-                            half_codes % 16 == 0 && scales_bytes % 16 == 0 &&
-                            (size_t)(s + 1) * L.stage_bytes <= (size_t)L.bar_off,
-                        11, p.status))
-          break;
-        mbar_arrive_expect_tx(&full[s], (uint32_t)L.stage_bytes);
-        bulk_g2s(st, p.gate.codes + row0 * (K / 2), half_codes, &full[s]);
-        bulk_g2s(st + half_codes, p.up.codes + row0 * (K / 2), half_codes, &full[s]);
-        bulk_g2s(st + 2 * half_codes, p.gate.scales + row0 * (K / 16), scales_bytes, &full[s]);
-        bulk_g2s(st + 2 * half_codes + scales_bytes, p.up.scales + row0 * (K / 16), scales_bytes, &full[s]);
+        const int j = m / P, pt = m - j * P;
+        const int i = c0 + j * G, u = i / TPE, tile = i - u * TPE;
+        const int row0 = s_live[1 + u] * I + tile * 16;
+        uint8_t* st = smem + (size_t)s * kGuStage;
+        const int x0 = pt * (kGuCodes / 2);
+        mbar_arrive_expect_tx(&full[s], (uint32_t)kGuStage);
+        tma_load_2d(st, &prm.gc, x0, row0, &full[s]);
+        tma_load_2d(st + kBox, &prm.gc, x0 + 128, row0, &full[s]);
+        tma_load_2d(st + 2 * kBox, &prm.uc, x0, row0, &full[s]);
+        tma_load_2d(st + 3 * kBox, &prm.uc, x0 + 128, row0, &full[s]);
+        tma_load_2d(st + 4 * kBox, &prm.gs, pt * (kGuCodes / 16), row0, &full[s]);
+        tma_load_2d(st + 4 * kBox + 512, &prm.us, pt * (kGuCodes / 16), row0, &full[s]);
+        issued = m + 1;
       }
+      // no copy may still be landing when the CTA exits
+      for (int m = max(0, issued - NS); m < issued; ++m)
+        if (!mbar_wait(&full[m % NS], (uint32_t)(m / NS) & 1u)) set_status(p.status, kDevErrTimeout | kWaitGuDrain);
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------ consumers
+  float up, unscale;
+  prescale15(__uint_as_float(*p.xmax), up, unscale);
+  // x as B fragments: entry (chunk cg, step i, lane t) = x[128 cg + 32 t + 4 i + 0..3]
+  for (int f = threadIdx.x; f < H / 4; f += kGuConsumers * kWarp) {
+    const int t = f & 3, i = (f >> 2) & 7, cg = f >> 5;
+    const uint2 v = *reinterpret_cast<const uint2*>(p.x + 128 * cg + 32 * t + 4 * i);
+    const float2 a = bf16x2_to_f32x2(v.x), b = bf16x2_to_f32x2(v.y);
+    __half2 h0 = __floats2half2_rn(a.x * up, a.y * up), h1 = __floats2half2_rn(b.x * up, b.y * up);
+    xs[f] = make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
+  }
+  named_bar_sync(1, kGuConsumers * kWarp);
+
+  const int g = lane >> 2, t = lane & 3;
+  for (int m = warp; m < n_stages; m += kGuConsumers) {
+    if (*s_abort) break;
+    const int s = m % NS;
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (uint32_t)(m / NS) & 1u));
+    if (!ok) {
+      if (lane == 0) {
+        set_status(p.status, kDevErrTimeout | kWaitGuFull);
+        *s_abort = 1;
+      }
+      break;
+    }
+    const int j = m / P, pt = m - j * P;
+    const int i = c0 + j * G, u = i / TPE, tile = i - u * TPE;
+    float acc[2][2][4];
+#pragma unroll
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+      for (int b = 0; b < 2; ++b)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[a][b][q] = 0.f;
+    const uint8_t* st = smem + (size_t)s * kGuStage;
+    stage_mma<2>(st, 2 * kBox, st + 4 * kBox, 512, kGuCodes / 16, kGuCodes / 256, xs + pt * (kGuCodes / 128) * 32,
+                 lane < 4, g, t, acc);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    // column 0 of the tile lives in lanes t == 0: rows tile_row(g), + 8
+    const int slot = j % NB;
+    float* pb = part + (slot * P + pt) * 32;
+    if (t == 0) {
+      const int r0 = tile_row(g);
+      pb[r0] = acc[0][0][0] + acc[0][1][0];
+      pb[r0 + 8] = acc[0][0][2] + acc[0][1][2];
+      pb[16 + r0] = acc[1][0][0] + acc[1][1][0];
+      pb[16 + r0 + 8] = acc[1][0][2] + acc[1][1][2];
     }
     __syncwarp();
-    // the down pass's CTA of this index reads these rows next: the producer
-    // warp asks L2 for them (plain prefetches, one per 128-byte line) while
-    // the consumers compute the last stages
-    if (p.l2_prefetch) {
-      const int n0 = row_begin(c0, p.H, G), n1 = row_begin(c0 + 1, p.H, G);
-      const size_t cb = (size_t)(n1 - n0) * (I / 2), sb = (size_t)(n1 - n0) * (I / 16);
-      for (int u = 0; u < n_live; ++u) {
-        const size_t e = (size_t)s_live[1 + u];
-        const uint8_t* c = p.down.codes + (e * p.H + n0) * (I / 2);
-        const uint8_t* sc = p.down.scales + (e * p.H + n0) * (I / 16);
-        for (size_t o = 128 * (size_t)lane; o < cb; o += 128 * 32) prefetch_l2(c + o);
-        for (size_t o = 128 * (size_t)lane; o < sb; o += 128 * 32) prefetch_l2(sc + o);
+    int last = 0;
+    if (lane == 0) {
+      __threadfence_block();
+      last = atomicAdd(&cnt[slot], 1) == P - 1;
+    }
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (last) {
+      // the tile's P partial sums in part order, then the SwiGLU
+      __threadfence_block();
+      if (lane < 16) {
+        const float* pj = part + slot * P * 32;
+        float gs = 0.f, us = 0.f;
+        for (int q = 0; q < P; ++q) {
+          gs += pj[q * 32 + lane];
+          us += pj[q * 32 + 16 + lane];
+        }
+        gs *= unscale * s_ts[u];
+        us *= unscale * s_ts[kMaxLive + u];
+        const int a = s_live[1 + kMaxLive + u];
+        p.h[(size_t)a * I + tile * 16 + lane] = clamped_swiglu(gs, us, p.limit);
       }
-      if (p.sh_down) {
-        const uint8_t* sd = reinterpret_cast<const uint8_t*>(p.sh_down + (size_t)n0 * p.Is);
-        const size_t db = (size_t)(n1 - n0) * p.Is * 2;
-        for (size_t o = 128 * (size_t)lane; o < db; o += 128 * 32) prefetch_l2(sd + o);
+      __syncwarp();
+      if (lane == 0) cnt[slot] = 0;
+    }
+  }
+}
+
+// ============================================================== down
+
+struct DnParams {
+  CUtensorMap dc;          // down codes [E H, I/2] bytes, box 128 B x 16 rows, SW128
+  CUtensorMap ds;          // down scales [E H, I/16] bytes, box I/16 B x 16 rows
+  DecodeT1Args a;
+};
+
+struct DnLayout {
+  int stage, NS, hs, hsc, hmax, bar, live, tmp, ts, flag, total;
+};
+constexpr int kHq = 16;          // float4 of h per consumer thread: k I / 4 <= kHq * 512 (k <= 16, I <= 2048)
+__host__ __device__ inline int dn_stage_bytes(int I) { return (9 * I + 1023) / 1024 * 1024; }
+__host__ __device__ inline DnLayout dn_layout(int I, int k) {
+  DnLayout L{};
+  L.stage = dn_stage_bytes(I);
+  for (int ns = kMaxStages; ns >= 1; --ns) {
+    L.NS = ns;
+    L.hs = ns * L.stage;
+    L.hsc = L.hs + k * I * 2;
+    L.hmax = L.hsc + kMaxLive * 4;
+    L.bar = (L.hmax + kMaxLive * 4 + 7) / 8 * 8;
+    L.live = L.bar + 2 * ns * 8;
+    L.tmp = L.live + (1 + 2 * kMaxLive) * 4;
+    L.ts = L.tmp + 4 * kMaxLive * 4;
+    L.flag = L.ts + 2 * kMaxLive * 4;
+    L.total = L.flag + 16 + 1024;
+    if (L.total <= kSmemBudget) break;
+  }
+  return L;
+}
+
+__global__ void __launch_bounds__(kDnThreads, 1) t1_down_kernel(const __grid_constant__ DnParams prm) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const DecodeT1Args& p = prm.a;
+  const int H = p.H, I = p.I, k = p.k;
+  const DnLayout L = dn_layout(I, k);
+  const int NS = L.NS;
+  // Each consumer warp owns D ring slots and consumes their phases in order
+  // (item m: warp m % WE, its (m / WE)-th item), so no wait can target a
+  // phase two ahead of its barrier.
+  const int WE = min(kDnConsumers, NS), D = NS / WE;
+  uint2* hs = reinterpret_cast<uint2*>(smem + L.hs);
+  float* hsc = reinterpret_cast<float*>(smem + L.hsc);
+  uint32_t* hmax = reinterpret_cast<uint32_t*>(smem + L.hmax);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar);
+  uint64_t* empty = full + NS;
+  int* s_live = reinterpret_cast<int*>(smem + L.live);
+  float* s_ts = reinterpret_cast<float*>(smem + L.ts);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + L.flag);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    *s_abort = 0;
+    fence_barrier_init();
+  }
+  // The plan comes from two launches back, complete when this grid starts:
+  // the weight stream starts before the wait for h.
+  load_live(p, p.down.tensor_scale, nullptr, reinterpret_cast<int*>(smem + L.tmp), s_live, s_ts);
+  const int n_live = s_live[0];
+  const int TPE = H / 16;
+  const int N = n_live * TPE, G = gridDim.x, c0 = blockIdx.x;
+  const int n_items = c0 < N ? (N - 1 - c0) / G + 1 : 0;
+  const int nbox = I / 256;
+
+  if (warp == kDnConsumers) {
+    // ---------------------------------------------------------- producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int m = 0; m < n_items; ++m) {
+        if (*s_abort) break;
+        const int w = m % WE, l = m / WE, s = w * D + l % D;
+        if (l >= D && !mbar_wait(&empty[s], ((uint32_t)(l / D) & 1u) ^ 1u)) {
+          set_status(p.status, kDevErrTimeout | kWaitDnEmpty);
+          *s_abort = 1;
+          break;
+        }
+        const int i = c0 + m * G, u = i / TPE, tile = i - u * TPE;
+        const int row0 = s_live[1 + u] * H + tile * 16;
+        uint8_t* st = smem + (size_t)s * L.stage;
+        mbar_arrive_expect_tx(&full[s], (uint32_t)(9 * I));
+        for (int b = 0; b < nbox; ++b) tma_load_2d(st + b * kBox, &prm.dc, b * 128, row0, &full[s]);
+        tma_load_2d(st + 8 * I, &prm.ds, 0, row0, &full[s]);
+        issued = m + 1;
+      }
+      for (int m = max(0, issued - WE * D); m < issued; ++m) {
+        const int w = m % WE, l = m / WE;
+        if (!mbar_wait(&full[w * D + l % D], (uint32_t)(l / D) & 1u)) set_status(p.status, kDevErrTimeout | kWaitDnDrain);
       }
     }
     return;
   }
 
   // ------------------------------------------------------------ consumers
-  const int ks = warp % kGuKS, rg = warp / kGuKS;
-  const int CS = (K / 32) / kGuKS;         // chunks per K slice
-  float up, unscale;
-  prescale15(__uint_as_float(*p.xmax), up, unscale);
-  uint32_t xr[CPL][16];
-#pragma unroll
-  for (int i = 0; i < CPL; ++i) act_chunk_bf16(p.x, ks * CS + lane + 32 * i, lane + 32 * i < CS, up, xr[i]);
-  constexpr int RPW = kGuR / kGuRG;        // row pairs per warp
-
-  for (int m = 0; m < n_mine; ++m) {
-    const int i = c0 + m * G;
-    const int u = i / NB, rb = i - u * NB;
-    const int s = m % NS;
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (uint32_t)(m / NS) & 1u));
-    float acc[2 * RPW];
-#pragma unroll
-    for (int r = 0; r < 2 * RPW; ++r) acc[r] = 0.f;
-    if (ok) {
-      const uint8_t* st = smem + (size_t)s * L.stage_bytes;
-#pragma unroll
-      for (int ci = 0; ci < CPL; ++ci) {
-        const int cl = lane + 32 * ci;
-        if (cl < CS) {
-          const int c = ks * CS + cl;
-#pragma unroll
-          for (int r = 0; r < 2 * RPW; ++r) {
-            const int bank = r / RPW, rr = rg * RPW + (r % RPW);
-            const uint4 q = *reinterpret_cast<const uint4*>(st + bank * half_codes + rr * (K / 2) + 16 * c);
-            const uint16_t sc =
-                *reinterpret_cast<const uint16_t*>(st + 2 * half_codes + bank * scales_bytes + rr * (K / 16) + 2 * c);
-            acc[r] = chunk_dot_f32(q, sc, xr[ci], acc[r]);
-          }
-        }
-      }
-    } else if (lane == 0) {
-      set_status(p.status, kDevErrTimeout);
-      atomicMin(const_cast<int*>(s_abort), m);
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
-    const float tot = warp_reduce_rows<2 * RPW>(acc);       // lane 8 r holds slot r
-    float* rb_red = red + (m & 1) * (kGuKS * 2 * kGuR);
-    if ((lane & (32 / (2 * RPW) - 1)) == 0) {
-      const int r = lane / (32 / (2 * RPW));
-      const int bank = r / RPW, rr = rg * RPW + (r % RPW);
-      rb_red[ks * 2 * kGuR + bank * kGuR + rr] = tot;
-    }
-    named_bar_sync(1, kGuConsumers * kWarp);
-    if (*s_abort <= m) break;
-    if (threadIdx.x < kGuR) {
-      const int rr = threadIdx.x;
-      const int e = s_live[1 + u], a = s_live[1 + kMaxK + u];
-      float g = 0.f, uu = 0.f;
-#pragma unroll
-      for (int k2 = 0; k2 < kGuKS; ++k2) {
-        g += rb_red[k2 * 2 * kGuR + rr];
-        uu += rb_red[k2 * 2 * kGuR + kGuR + rr];
-      }
-      g *= unscale * s_ts[u];
-      uu *= unscale * s_ts[kMaxK + u];
-      const float hv = clamped_swiglu(g, uu, p.limit);
-      if (RNX_DCHECK(a >= 0 && a < p.k && rb * kGuR + rr < I && e >= 0 && e < p.E, 13, p.status))
-        p.h[(size_t)a * I + rb * kGuR + rr] = hv;
-    }
-  }
-}
-
-// ============================================================== K3
-constexpr int kDnWarps = 16;
-constexpr int kDnThreads = kDnWarps * kWarp;
-constexpr int kDnRowBatch = 8;
-
-struct DnSmem {
-  int nr, seg_codes, seg_scales, codes_off, scales_off, shared_off, bar_off, rs_off, sh_off, live_off, flag_off, total;
-};
-// Shared-memory plan of one K3 CTA: nr rows of k routed segments (codes,
-// scales) and of the shared expert's down rows, one mbarrier per segment.
-__host__ __device__ inline DnSmem dn_smem(int H, int I, int Is, int k, int G) {
-  DnSmem s;
-  s.nr = (H + G - 1) / G;
-  s.seg_codes = (s.nr * (I / 2) + 15) / 16 * 16;
-  s.seg_scales = (s.nr * (I / 16) + 15) / 16 * 16;
-  s.codes_off = 0;
-  s.scales_off = s.codes_off + k * s.seg_codes;
-  s.shared_off = s.scales_off + k * s.seg_scales;
-  s.bar_off = (s.shared_off + s.nr * Is * 2 + 15) / 16 * 16;
-  s.rs_off = s.bar_off + (k + 1) * 8;
-  s.sh_off = s.rs_off + k * s.nr * 4;
-  s.live_off = s.sh_off + s.nr * 4;
-  s.flag_off = s.live_off + (1 + 2 * kMaxK) * 4;
-  s.total = s.flag_off + 16;
-  return s;
-}
-
-template <int CPL>
-__global__ void __launch_bounds__(kDnThreads, 1) k3_down_combine(DecodeT1Args p) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  const int G = gridDim.x, c0 = blockIdx.x;
-  const int H = p.H, I = p.I, k = p.k;
-  const bool with_shared = p.sh_down != nullptr;
-  const int Is = with_shared ? p.Is : 0;
-  const DnSmem L = dn_smem(H, I, Is, k, G);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L.bar_off);
-  float* rs = reinterpret_cast<float*>(smem + L.rs_off);         // [k][nr] weighted routed rows
-  float* sh = reinterpret_cast<float*>(smem + L.sh_off);         // [nr] shared rows
-  int* s_live = reinterpret_cast<int*>(smem + L.live_off);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = row_begin(c0, H, G), n1 = row_begin(c0 + 1, H, G), nrows = n1 - n0;
-
-  // The ids come from two launches back, complete when this grid starts: the
-  // weight loads go out before the wait for h. Codes and the shared rows by
-  // bulk copies (one mbarrier per segment); the E4M3 scales (a ninth of the
-  // bytes, rows of I/16 bytes that need not be 16-byte aligned) by plain
-  // 4-byte loads of all threads.
-  if (threadIdx.x == 0) {
-    build_live(p.ids, p.active, p.first, k, p.E, p.lb, p.le, p.status, false, s_live);
-    for (int s = 0; s <= k; ++s) mbar_init(&bar[s], 1);
-    fence_barrier_init();
-    const int n_live = s_live[0];
-    if (nrows > 0) {
-      for (int u = 0; u < n_live; ++u) {
-        const size_t e = (size_t)s_live[1 + u];
-        const uint32_t cb = (uint32_t)(nrows * (I / 2));
-        if (!RNX_DCHECK(e < (size_t)p.E && nrows <= L.nr && cb <= (uint32_t)L.seg_codes && cb % 16 == 0 &&
-                            al16(smem + L.codes_off + u * L.seg_codes) && al16(p.down.codes + (e * H + n0) * (I / 2)),
-                        20, p.status))
-          continue;
-        mbar_arrive_expect_tx(&bar[u], cb);
-        bulk_g2s(smem + L.codes_off + u * L.seg_codes, p.down.codes + (e * H + n0) * (I / 2), cb, &bar[u]);
-      }
-      if (with_shared && RNX_DCHECK(al16(smem + L.shared_off) && al16(p.sh_down + (size_t)n0 * Is) &&
-                                        (L.shared_off + nrows * Is * 2) <= L.bar_off,
-                                    21, p.status)) {
-        const uint32_t b = (uint32_t)(nrows * Is * 2);
-        mbar_arrive_expect_tx(&bar[k], b);
-        bulk_g2s(smem + L.shared_off, p.sh_down + (size_t)n0 * Is, b, &bar[k]);
-      }
-    }
-  }
-  for (int i = threadIdx.x; i < k * L.nr; i += kDnThreads) rs[i] = 0.f;
-  __syncthreads();
-  {
-    const int n_live = s_live[0];
-    const int words = nrows * (I / 16) / 4;          // 4-byte words of one segment's scales
-    for (int i = threadIdx.x; i < n_live * words; i += kDnThreads) {
-      const int u = i / words, wd = i - u * words;
-      const size_t e = (size_t)s_live[1 + u];
-      const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(p.down.scales + (e * H + n0) * (I / 16)) + wd);
-      reinterpret_cast<uint32_t*>(smem + L.scales_off + u * L.seg_scales)[wd] = v;
-    }
-  }
-  __syncthreads();
   pdl_wait();                // h comes from the previous launch
   pdl_trigger();
-  const int n_live = s_live[0];
+  // h rows of the live experts as B fragments (f16, a power of two per row
+  // from the row's max |h|), and each row's output factor. All consumer
+  // threads: one round of loads (kHq float4 per thread, issued together), the
+  // row maxima through shared memory, then the conversion.
+  {
+    const int tid = threadIdx.x, nq = n_live * (I / 4);
+    float4 v[kHq];
+#pragma unroll
+    for (int q = 0; q < kHq; ++q) {
+      const int f = tid + q * kDnConsumers * kWarp;
+      if (f < nq) {
+        const int u = f / (I / 4), c = f - u * (I / 4);
+        v[q] = *reinterpret_cast<const float4*>(p.h + (size_t)s_live[1 + kMaxLive + u] * I + 4 * c);
+      } else {
+        v[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    if (tid < kMaxLive) hmax[tid] = 0u;
+    named_bar_sync(1, kDnConsumers * kWarp);
+#pragma unroll
+    for (int q = 0; q < kHq; ++q) {
+      const int f = tid + q * kDnConsumers * kWarp;
+      if (f < nq) {
+        const float m = fmaxf(fmaxf(fabsf(v[q].x), fabsf(v[q].y)), fmaxf(fabsf(v[q].z), fabsf(v[q].w)));
+        atomicMax(&hmax[f / (I / 4)], __float_as_uint(m));       // non-negative floats order as integers
+      }
+    }
+    named_bar_sync(1, kDnConsumers * kWarp);
+#pragma unroll
+    for (int q = 0; q < kHq; ++q) {
+      const int f = tid + q * kDnConsumers * kWarp;
+      if (f < nq) {
+        const int u = f / (I / 4), c = f - u * (I / 4), pos = 4 * c;
+        float upx, unscale;
+        prescale15(__uint_as_float(hmax[u]), upx, unscale);
+        __half2 h0 = __floats2half2_rn(v[q].x * upx, v[q].y * upx);
+        __half2 h1 = __floats2half2_rn(v[q].z * upx, v[q].w * upx);
+        hs[(size_t)u * (I / 4) + ((pos >> 7) * 8 + ((pos >> 2) & 7)) * 4 + ((pos >> 5) & 3)] =
+            make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
+      }
+    }
+    if (tid < n_live) {
+      float upx, unscale;
+      prescale15(__uint_as_float(hmax[tid]), upx, unscale);
+      hsc[tid] = unscale * s_ts[tid] * p.weights[s_live[1 + kMaxLive + tid]];
+    }
+  }
+  named_bar_sync(1, kDnConsumers * kWarp);
 
-  // routed rows: task t = (live assignment u, part of the row block); the
-  // parts split each assignment's rows so that every warp has a task
-  const int parts = n_live > 0 ? max(1, kDnWarps / n_live) : 1;
-  for (int task = warp; task < n_live * parts; task += kDnWarps) {
-    const int u = task / parts, part = task - u * parts;
-    const int ra = part * nrows / parts, rz = (part + 1) * nrows / parts;
-    const bool ok = nrows == 0 || __all_sync(0xffffffffu, mbar_wait(&bar[u], 0));
+  const int g = lane >> 2, t = lane & 3;
+  for (int m = warp; m < n_items && warp < WE; m += WE) {
+    if (*s_abort) break;
+    const int l = m / WE, s = warp * D + l % D;
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (uint32_t)(l / D) & 1u));
     if (!ok) {
-      if (lane == 0) set_status(p.status, kDevErrTimeout);
-      continue;
+      if (lane == 0) {
+        set_status(p.status, kDevErrTimeout | kWaitDnFull);
+        *s_abort = 1;
+      }
+      break;
     }
-    const int e = s_live[1 + u], a = s_live[1 + kMaxK + u];
-    if (!RNX_DCHECK(e >= 0 && e < p.E && a >= 0 && a < k && rz <= L.nr, 22, p.status)) continue;
-    // the warp holds the whole h row (chunk lane + 32 i per lane): its max
-    // |h| sets the f16 pre-scale
-    const float* hrow = p.h + (size_t)a * I;
-    float mx = 0.f;
+    const int i = c0 + m * G, u = i / TPE, tile = i - u * TPE;
+    float acc[1][2][4];
 #pragma unroll
-    for (int i = 0; i < CPL; ++i) {
-      const int c = lane + 32 * i;
-      if (c < I / 32) {
+    for (int b = 0; b < 2; ++b)
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float4 v = *reinterpret_cast<const float4*>(hrow + 32 * c + 4 * q);
-          mx = fmaxf(mx, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
-        }
-      }
-    }
-    mx = warp_max(mx);
-    float upx, unscale;
-    prescale15(mx, upx, unscale);
-    uint32_t xr[CPL][16];
-#pragma unroll
-    for (int i = 0; i < CPL; ++i) act_chunk_f32(hrow, lane + 32 * i, lane + 32 * i < I / 32, upx, xr[i]);
-    const float scale = unscale * p.down.tensor_scale[e] * p.weights[a];
-    const uint8_t* codes = smem + L.codes_off + u * L.seg_codes;
-    const uint8_t* scales = smem + L.scales_off + u * L.seg_scales;
-    for (int r0 = ra; r0 < rz; r0 += kDnRowBatch) {
-      float acc[kDnRowBatch];
-#pragma unroll
-      for (int rr = 0; rr < kDnRowBatch; ++rr) {
-        acc[rr] = 0.f;
-        const int r = r0 + rr;
-        if (r < rz) {
-#pragma unroll
-          for (int i = 0; i < CPL; ++i) {
-            const int c = lane + 32 * i;
-            if (c < I / 32) {
-              const uint4 q = *reinterpret_cast<const uint4*>(codes + r * (I / 2) + 16 * c);
-              const uint16_t sc = *reinterpret_cast<const uint16_t*>(scales + r * (I / 16) + 2 * c);
-              acc[rr] = chunk_dot_f32(q, sc, xr[i], acc[rr]);
-            }
-          }
-        }
-      }
-      const float tot = warp_reduce_rows<kDnRowBatch>(acc);   // lane 4 r holds row r0 + r
-      const int r = r0 + (lane >> 2);
-      if ((lane & 3) == 0 && r < rz) {
-        const float v = tot * scale;
-        rs[a * L.nr + r] = v;
-        if (p.r) p.r[(size_t)a * H + n0 + r] = v;
-      }
+      for (int q = 0; q < 4; ++q) acc[0][b][q] = 0.f;
+    const uint8_t* st = smem + (size_t)s * L.stage;
+    stage_mma<1>(st, 0, st + 8 * I, 0, I / 16, I / 256, hs + (size_t)u * (I / 4), lane < 4, g, t, acc);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    if (t == 0) {
+      const int a = s_live[1 + kMaxLive + u];
+      const float sc = hsc[u];
+      const int r0 = tile_row(g);
+      float* rr = p.r + (size_t)a * H + tile * 16;
+      rr[r0] = (acc[0][0][0] + acc[0][1][0]) * sc;
+      rr[r0 + 8] = (acc[0][0][2] + acc[0][1][2]) * sc;
     }
   }
 
-  // shared expert's down rows: fp32 FMAs of the bf16 weights and h_shared
-  if (with_shared && nrows > 0) {
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar[k], 0));
-    if (!ok) {
-      if (lane == 0) set_status(p.status, kDevErrTimeout);
-    } else {
-      const int nu4 = Is / 8;
-      for (int r = warp; r < nrows; r += kDnWarps) {
-        const uint4* wrow = reinterpret_cast<const uint4*>(smem + L.shared_off + (size_t)r * Is * 2);
-        float acc = 0.f;
-        for (int c = lane; c < nu4; c += 32) {
-          const uint4 wv = wrow[c];
-          const float4 h0 = *reinterpret_cast<const float4*>(p.h_shared + 8 * c);
-          const float4 h1 = *reinterpret_cast<const float4*>(p.h_shared + 8 * c + 4);
-          const float2 w0 = bf16x2_to_f32x2(wv.x), w1 = bf16x2_to_f32x2(wv.y);
-          const float2 w2 = bf16x2_to_f32x2(wv.z), w3 = bf16x2_to_f32x2(wv.w);
-          acc = fmaf(w0.x, h0.x, acc);
-          acc = fmaf(w0.y, h0.y, acc);
-          acc = fmaf(w1.x, h0.z, acc);
-          acc = fmaf(w1.y, h0.w, acc);
-          acc = fmaf(w2.x, h1.x, acc);
-          acc = fmaf(w2.y, h1.y, acc);
-          acc = fmaf(w3.x, h1.z, acc);
-          acc = fmaf(w3.y, h1.w, acc);
-        }
-        acc = warp_sum(acc);
-        if (lane == 0) sh[r] = acc;
-      }
-    }
-  }
-  __syncthreads();
-
-  // rows of assignments that are not live (remote experts, dropped ids) are zero
-  if (p.r) {
-    for (int a = 0; a < k; ++a) {
-      bool live = false;
-      for (int u = 0; u < n_live; ++u) live |= s_live[1 + kMaxK + u] == a;
-      if (!live)
-        for (int r = threadIdx.x; r < nrows; r += kDnThreads) p.r[(size_t)a * H + n0 + r] = 0.f;
-    }
-  }
-  // moe_combine: the k routed rows in rank order, then the shared row, fp32,
-  // one rounding to bf16
-  if (p.y) {
-    for (int r = threadIdx.x; r < nrows; r += kDnThreads) {
-      float acc = 0.f;
-      for (int j = 0; j < k; ++j) acc += rs[j * L.nr + r];
-      if (with_shared) {
-        acc += sh[r];
-        if (p.shared_out) p.shared_out[n0 + r] = sh[r];
-      }
-      p.y[n0 + r] = f32_to_bf16_bits(acc);
-    }
+  // rows of assignments that are not live (remote experts, dropped ids) are
+  // zero: this CTA's slice of each
+  const int n0 = (int)((long long)c0 * H / G), n1 = (int)((long long)(c0 + 1) * H / G);
+  for (int a = 0; a < k; ++a) {
+    bool live = false;
+    for (int u = 0; u < n_live; ++u) live |= s_live[1 + kMaxLive + u] == a;
+    if (!live)
+      for (int r = n0 + (int)threadIdx.x; r < n1; r += kDnConsumers * kWarp) p.r[(size_t)a * H + r] = 0.f;
   }
 }
 
@@ -696,47 +571,60 @@ int sm_count() {
   return cached[dev];
 }
 
-template <typename Kern>
-cudaError_t set_smem(Kern kern, int bytes) {
-  return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-}
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 }  // namespace
 
-bool decode_t1_supported(int H, int I, int Is, int E, int k) {
-  const int G = sm_count();
-  if (H % 256 || H > 8192 || I % 64 || I > 2048 || k < 1 || k > kMaxK || E < 1 || E > 1024) return false;
-  if (Is < 0 || Is % 8 || Is > 8192) return false;
-  if (I % kGuR) return false;
-  if (gu_smem(H).nstages < 2 || gu_smem(H).total > 227 * 1024) return false;
-  if (dn_smem(H, I, Is, k, G).total > 227 * 1024) return false;
+bool decode_t1_supported(int H, int I, int E, int k) {
+  if (H % kGuCodes || H > 8192 || I % 256 || I > 2048 || k < 1 || k > kMaxLive || E < 1 || E > 1024) return false;
+  if ((long long)E * (H > I ? H : I) >= (1ll << 31)) return false;
+  const GuLayout g = gu_layout(H);
+  if (g.total > kSmemBudget || g.NS < 2) return false;
+  const DnLayout d = dn_layout(I, k);
+  if (d.total > kSmemBudget || d.NS < 2) return false;
   return true;
 }
 
-cudaError_t launch_decode_t1_gate_up(const DecodeT1Args& p, cudaStream_t st) {
-  const GuSmem L = gu_smem(p.H);
-  const int CPL = ((p.H / 32) / kGuKS + 31) / 32;
-  auto kern = CPL <= 1 ? k2_gate_up<1> : k2_gate_up<2>;
-  cudaError_t e = set_smem(kern, L.total);
+cudaError_t launch_decode_t1_gate_up(const DecodeT1Args& a, cudaStream_t st) {
+  if (!decode_t1_supported(a.H, a.I, a.E, a.k)) return cudaErrorInvalidValue;
+  if (!aligned16(a.gate.codes) || !aligned16(a.up.codes) || !aligned16(a.gate.scales) || !aligned16(a.up.scales) ||
+      ((uintptr_t)a.x & 7u))
+    return cudaErrorInvalidValue;
+  GuParams p;
+  memset(&p, 0, sizeof p);
+  const uint64_t rows = (uint64_t)a.E * a.I;
+  if (!make_tensor_map_2d(&p.gc, a.gate.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.H / 2, rows, 128, 16,
+                          CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tensor_map_2d(&p.uc, a.up.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.H / 2, rows, 128, 16,
+                          CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tensor_map_2d(&p.gs, a.gate.scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.H / 16, rows, kGuCodes / 16, 16,
+                          CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tensor_map_2d(&p.us, a.up.scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.H / 16, rows, kGuCodes / 16, 16,
+                          CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  p.a = a;
+  const GuLayout L = gu_layout(a.H);
+  cudaError_t e = cudaFuncSetAttribute(t1_gate_up_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
   if (e != cudaSuccess) return e;
-  return launch_pdl(kern, dim3(sm_count()), dim3(kGuThreads), (size_t)L.total, st, p);
+  return launch_pdl(t1_gate_up_kernel, dim3(sm_count()), dim3(kGuThreads), (size_t)L.total, st, p);
 }
 
-cudaError_t launch_decode_t1_down(const DecodeT1Args& p, cudaStream_t st) {
-  const int G = sm_count();
-  const DnSmem L = dn_smem(p.H, p.I, p.sh_down ? p.Is : 0, p.k, G);
-  const int CPL = (p.I / 32 + 31) / 32;
-  auto kern = CPL <= 1 ? k3_down_combine<1> : k3_down_combine<2>;
-  cudaError_t e = set_smem(kern, L.total);
+cudaError_t launch_decode_t1_down(const DecodeT1Args& a, cudaStream_t st) {
+  if (!decode_t1_supported(a.H, a.I, a.E, a.k)) return cudaErrorInvalidValue;
+  if (!aligned16(a.down.codes) || !aligned16(a.down.scales) || !aligned16(a.h)) return cudaErrorInvalidValue;
+  DnParams p;
+  memset(&p, 0, sizeof p);
+  const uint64_t rows = (uint64_t)a.E * a.H;
+  if (!make_tensor_map_2d(&p.dc, a.down.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.I / 2, rows, 128, 16,
+                          CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tensor_map_2d(&p.ds, a.down.scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.I / 16, rows, a.I / 16, 16,
+                          CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  p.a = a;
+  const DnLayout L = dn_layout(a.I, a.k);
+  cudaError_t e = cudaFuncSetAttribute(t1_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
   if (e != cudaSuccess) return e;
-  return launch_pdl(kern, dim3(G), dim3(kDnThreads), (size_t)L.total, st, p);
-}
-
-cudaError_t launch_decode_t1_router(const DecodeT1Args& p, cudaStream_t st) {
-  const int grid = (p.E + 1) / 2 + (p.Is + 7) / 8;
-  if (p.E <= 32 * 4) return launch_pdl(k1_router_topk_shared<4>, dim3(grid), dim3(kK1Threads), 0, st, p);
-  if (p.E <= 32 * 10) return launch_pdl(k1_router_topk_shared<10>, dim3(grid), dim3(kK1Threads), 0, st, p);
-  return launch_pdl(k1_router_topk_shared<32>, dim3(grid), dim3(kK1Threads), 0, st, p);
+  return launch_pdl(t1_down_kernel, dim3(sm_count()), dim3(kDnThreads), (size_t)L.total, st, p);
 }
 
 }  // namespace rnx

@@ -176,15 +176,19 @@ cudaError_t launch_dense_gemv(int H, int I, float limit, const uint16_t* x, int 
 }
 
 cudaError_t launch_dense_ffn(int H, int I, float limit, const uint16_t* x, int T, const uint16_t* wg,
-                             const uint16_t* wu, const uint16_t* wd, uint16_t* y, void* hbuf, uint32_t* status,
-                             cudaStream_t st) {
+                             const uint16_t* wu, const uint16_t* wd, void* y, bool y_f32, void* hbuf,
+                             uint32_t* status, cudaStream_t st) {
   if (T >= kDenseGemmMinT && I % 128 == 0 && H % 256 == 0) {
+    // the fp32 output (the site's shared row) carries h as two bf16 terms;
+    // the bf16 output (the dense FFN entry point) rounds h to bf16
     uint16_t* hb = reinterpret_cast<uint16_t*>(hbuf);
-    cudaError_t err = launch_bf16_gemm(true, x, T, H, wg, wu, I, limit, hb, status, st);
+    cudaError_t err = launch_bf16_gemm(true, x, T, H, wg, wu, I, limit, hb, status, st, nullptr, y_f32);
     if (err != cudaSuccess) return err;
-    return launch_bf16_gemm(false, hb, T, I, wd, nullptr, H, 0.f, y, status, st);
+    return launch_bf16_gemm(false, hb, T, y_f32 ? 2 * I : I, wd, nullptr, H, 0.f,
+                            y_f32 ? nullptr : static_cast<uint16_t*>(y), status, st,
+                            y_f32 ? static_cast<float*>(y) : nullptr, y_f32);
   }
-  return launch_dense_gemv(H, I, limit, x, T, wg, wu, wd, y, false, reinterpret_cast<float*>(hbuf), st);
+  return launch_dense_gemv(H, I, limit, x, T, wg, wu, wd, y, y_f32, reinterpret_cast<float*>(hbuf), st);
 }
 
 }  // namespace rnx

@@ -108,43 +108,49 @@ RNX_DEVICE void add_bf16x8(float (&acc)[8], uint4 v) {
 // assignment adds a zero row (the same arithmetic as moe_combine over the
 // gathered rows). One CTA per token at a time; positions staged in shared.
 __global__ void __launch_bounds__(256) unpermute_combine_kernel(PaddedIndex q, int T, int k, int H,
-                                                                const uint16_t* __restrict__ rows,
-                                                                const uint16_t* __restrict__ shared,
+                                                                const float* __restrict__ rows,
+                                                                const float* __restrict__ shared,
                                                                 uint16_t* __restrict__ y) {
   __shared__ long long pos[16];
-  const int per_row = H >> 3;
+  const int per_row = H >> 2;
   for (int t = blockIdx.x; t < T; t += gridDim.x) {
     __syncthreads();
     if (threadIdx.x < k) pos[threadIdx.x] = padded_pos(q, (long long)t * k + threadIdx.x);
     __syncthreads();
     for (int c = threadIdx.x; c < per_row; c += blockDim.x) {
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int j = 0; j < k; ++j) {
         const long long pr = pos[j];
-        add_bf16x8(acc, pr >= 0 ? reinterpret_cast<const uint4*>(rows + (size_t)pr * H)[c] : make_uint4(0, 0, 0, 0));
+        const float4 v =
+            pr >= 0 ? reinterpret_cast<const float4*>(rows + (size_t)pr * H)[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
       }
-      if (shared) add_bf16x8(acc, reinterpret_cast<const uint4*>(shared + (size_t)t * H)[c]);
-      uint4 o;
-      o.x = pack_bf16x2(acc[0], acc[1]);
-      o.y = pack_bf16x2(acc[2], acc[3]);
-      o.z = pack_bf16x2(acc[4], acc[5]);
-      o.w = pack_bf16x2(acc[6], acc[7]);
-      reinterpret_cast<uint4*>(y + (size_t)t * H)[c] = o;
+      if (shared) {
+        const float4 v = reinterpret_cast<const float4*>(shared + (size_t)t * H)[c];
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+      reinterpret_cast<uint2*>(y + (size_t)t * H)[c] = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
     }
   }
 }
 
 // Unpermute alone: out[t, j] = rows[pos(t, j)] (zeros for remote assignments).
 __global__ void __launch_bounds__(256) unpermute_kernel(PaddedIndex q, long long A, int H,
-                                                        const uint16_t* __restrict__ rows, uint16_t* __restrict__ out) {
-  const int per_row = H >> 3;
+                                                        const float* __restrict__ rows, float* __restrict__ out) {
+  const int per_row = H >> 2;
   const long long n = A * per_row;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
     const long long a = i / per_row;
     const int c = (int)(i - a * per_row);
     const long long pr = padded_pos(q, a);
-    reinterpret_cast<uint4*>(out + (size_t)a * H)[c] =
-        pr >= 0 ? reinterpret_cast<const uint4*>(rows + (size_t)pr * H)[c] : make_uint4(0, 0, 0, 0);
+    reinterpret_cast<float4*>(out + (size_t)a * H)[c] =
+        pr >= 0 ? reinterpret_cast<const float4*>(rows + (size_t)pr * H)[c] : make_float4(0.f, 0.f, 0.f, 0.f);
   }
 }
 
@@ -209,18 +215,18 @@ cudaError_t launch_combine_f32(int T, int k, int H, const float* r, const float*
                     shared, y);
 }
 
-cudaError_t launch_unpermute_combine(const PaddedIndex& q, int T, int k, int H, const uint16_t* rows,
-                                     const uint16_t* shared, uint16_t* y, cudaStream_t st) {
+cudaError_t launch_unpermute_combine(const PaddedIndex& q, int T, int k, int H, const float* rows,
+                                     const float* shared, uint16_t* y, cudaStream_t st) {
   if (T <= 0) return cudaSuccess;
   const int grid = std::min(T, kNumSMs * 8);
   unpermute_combine_kernel<<<grid, 256, 0, st>>>(q, T, k, H, rows, shared, y);
   return cudaGetLastError();
 }
 
-cudaError_t launch_unpermute(const PaddedIndex& q, long long A, int H, const uint16_t* rows, uint16_t* out,
+cudaError_t launch_unpermute(const PaddedIndex& q, long long A, int H, const float* rows, float* out,
                              cudaStream_t st) {
   if (A <= 0) return cudaSuccess;
-  const long long work = A * (H >> 3);
+  const long long work = A * (H >> 2);
   const int grid = (int)std::min<long long>((work + 255) / 256, (long long)kNumSMs * 16);
   unpermute_kernel<<<grid, 256, 0, st>>>(q, A, H, rows, out);
   return cudaGetLastError();

@@ -58,10 +58,14 @@ struct GemmParams {
   CUtensorMap tma_b0;      // GATE_UP: gate rows (box 128 rows); DOWN / LOGITS: weight rows (box 256 rows)
   CUtensorMap tma_b1;      // GATE_UP: up rows
   uint16_t* out;           // GATE_UP / DOWN: bf16 [M, out_cols]
-  float* out_f32;          // LOGITS: fp32 [M, out_cols], columns < out_cols written
+  float* out_f32;          // LOGITS, and DOWN when set: fp32 [M, out_cols], columns < out_cols written
   uint32_t* status;
   int M, K, out_cols;
   int a_period;            // A's K extent; the K loop reads A at k mod a_period (LOGITS: K = 3 a_period)
+  int b_period;            // DOWN: B's K extent; the K loop reads B at k mod b_period (0: K). With
+                           // A = [h_hi | h_lo] and b_period = K / 2 the product is (h_hi + h_lo) . b
+  int split_h;             // GATE_UP: h written as two bf16 terms per element, h_hi at column c and
+                           // h_lo = bf16(h - h_hi) at column out_cols + c (row pitch 2 out_cols)
   float limit;
   unsigned long long wait_ns;   // limit of the main-loop waits (the drain waits keep the default)
 };
@@ -133,7 +137,8 @@ __global__ void __launch_bounds__(kThreads, 1) bf16_gemm_kernel(const __grid_con
             tma_load_2d(sB, &p.tma_b0, ks * kStepK, nt * 128, &full_bar[s]);
             tma_load_2d(sB + kBBytes / 2, &p.tma_b1, ks * kStepK, nt * 128, &full_bar[s]);
           } else {
-            tma_load_2d(sB, &p.tma_b0, ks * kStepK, nt * kTN, &full_bar[s]);
+            tma_load_2d(sB, &p.tma_b0, p.b_period ? (ks * kStepK) % p.b_period : ks * kStepK, nt * kTN,
+                        &full_bar[s]);
           }
         }
         __syncwarp();
@@ -235,17 +240,22 @@ __global__ void __launch_bounds__(kThreads, 1) bf16_gemm_kernel(const __grid_con
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[b]);
         if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(p.out + (size_t)row * p.out_cols + nt * 128 + 64 * ch);
+          const size_t pitch = p.split_h ? 2 * (size_t)p.out_cols : (size_t)p.out_cols;
+          uint4* dst = reinterpret_cast<uint4*>(p.out + (size_t)row * pitch + nt * 128 + 64 * ch);
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            uint32_t w[4];
+            uint32_t w[4], wl[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int k0 = 8 * c + 2 * i;
-              w[i] = pack_bf16x2(clamped_swiglu_fast(__uint_as_float(g[k0]), __uint_as_float(u[k0]), p.limit),
-                                 clamped_swiglu_fast(__uint_as_float(g[k0 + 1]), __uint_as_float(u[k0 + 1]), p.limit));
+              const float h0 = clamped_swiglu_fast(__uint_as_float(g[k0]), __uint_as_float(u[k0]), p.limit);
+              const float h1 = clamped_swiglu_fast(__uint_as_float(g[k0 + 1]), __uint_as_float(u[k0 + 1]), p.limit);
+              w[i] = pack_bf16x2(h0, h1);
+              // the rounding error of the bf16 term, itself in bf16 (exact difference in fp32)
+              wl[i] = pack_bf16x2(h0 - __uint_as_float(w[i] << 16), h1 - __uint_as_float(w[i] & 0xFFFF0000u));
             }
             dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+            if (p.split_h) dst[c + p.out_cols / 8] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
           }
         }
       } else if (LOGITS) {
@@ -283,7 +293,14 @@ __global__ void __launch_bounds__(kThreads, 1) bf16_gemm_kernel(const __grid_con
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[b]);
-        if (valid) {
+        if (valid && p.out_f32) {
+          // fp32 rows (the site's shared expert, summed in fp32 by the combine)
+          float4* dst = reinterpret_cast<float4*>(p.out_f32 + (size_t)row * p.out_cols + nt * kTileN + 128 * ch);
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            dst[c] = make_float4(__uint_as_float(v[4 * c]), __uint_as_float(v[4 * c + 1]),
+                                 __uint_as_float(v[4 * c + 2]), __uint_as_float(v[4 * c + 3]));
+        } else if (valid) {
           uint4* dst = reinterpret_cast<uint4*>(p.out + (size_t)row * p.out_cols + nt * kTileN + 128 * ch);
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
@@ -332,14 +349,20 @@ static unsigned long long g_gemm_wait_ns = kWaitLimitNs;
 void set_test_wait_limit_ns(unsigned long long ns) { g_gemm_wait_ns = ns; }
 
 cudaError_t launch_bf16_gemm(bool gate_up, const uint16_t* a, int M, int K, const uint16_t* b0, const uint16_t* b1,
-                             int N, float limit, uint16_t* out, uint32_t* status, cudaStream_t st) {
+                             int N, float limit, uint16_t* out, uint32_t* status, cudaStream_t st, float* out_f32,
+                             bool split) {
   if (M <= 0 || K % kStepK || N % (gate_up ? 128 : kTileN)) return cudaErrorInvalidValue;
+  const bool split_down = split && !gate_up;
+  if (split_down && (K / 2) % kStepK) return cudaErrorInvalidValue;
   GemmParams p;
   memset(&p, 0, sizeof p);
   if (!bf16_map(&p.tma_a, a, K, M, kTileM)) return cudaErrorInvalidValue;
-  if (!bf16_map(&p.tma_b0, b0, K, N, gate_up ? 128 : kTileN)) return cudaErrorInvalidValue;
+  if (!bf16_map(&p.tma_b0, b0, split_down ? K / 2 : K, N, gate_up ? 128 : kTileN)) return cudaErrorInvalidValue;
+  p.b_period = split_down ? K / 2 : 0;
+  p.split_h = split && gate_up;
   if (gate_up && !bf16_map(&p.tma_b1, b1, K, N, 128)) return cudaErrorInvalidValue;
   p.out = out;
+  p.out_f32 = gate_up ? nullptr : out_f32;
   p.status = status;
   p.M = M;
   p.K = K;

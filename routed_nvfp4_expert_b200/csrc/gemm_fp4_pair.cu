@@ -21,8 +21,9 @@
 //            of features 64 r .. 64 r + 63; the epilogue applies the scales
 //            and the clamped SwiGLU, rounds h to bf16, stores [P, I].
 //   DOWN:    256 output features; the epilogue applies the scales and the
-//            routing weight and writes bf16 rows [P, H] in the padded tile
-//            order (the unpermute is fused into the combine that follows).
+//            routing weight and writes fp32 rows [P, H] in the padded tile
+//            order (the unpermute is fused into the combine that follows,
+//            which sums them in fp32).
 //
 // Warp roles per CTA: warp 0 = TMA producer (5-stage ring, 38 KB per stage,
 // completions counted on the even CTA's barrier), warp 1 = MMA issuer (even
@@ -74,7 +75,7 @@ struct PairParams {
   CUtensorMap tma_b1;      // up codes (GATE_UP), box 128 B x 64 rows
   CUtensorMap tma_sfa;     // A scale atoms viewed as [bytes/256, 256], box 256 x 8 (4 atoms)
   CUtensorMap tma_sfb0;    // GATE_UP: interleaved gate/up atoms; DOWN: down atoms; same view
-  CUtensorMap tma_out;     // output [P, out_cols] bf16, box 64 x 32, SW128
+  CUtensorMap tma_out;     // output [P, out_cols]: GATE_UP bf16, box 64 x 32; DOWN fp32, box 32 x 32; SW128
   const float* row_scale;  // [P]
   const float* ts0;        // [E]
   const float* ts1;        // [E]
@@ -267,15 +268,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp >= kFirstEpiWarp) {
     // ------------------------------------------------------------ epilogue (both CTAs)
     // Each thread owns one accumulator row (its TMEM lane) and one column half.
-    // The finished bf16 values go to this warp's swizzled staging boxes; lane
-    // 0 writes each 32-row x 64-column box with one TMA tensor store. Output
-    // rows are in the padded tile order (padding rows hold zeros).
+    // The finished values go to this warp's swizzled staging boxes (GATE_UP:
+    // one 32-row x 64-column bf16 box; DOWN: fp32, two passes of two 32-row x
+    // 32-column boxes); lane 0 writes each box with one TMA tensor store.
+    // Output rows are in the padded tile order (padding rows hold zeros).
     const int q = warp & 3;
     const int ch = (warp - kFirstEpiWarp) >> 2;
     const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
     const uint32_t acc_empty_even = mapa_shared(smem_u32(&acc_empty), 0);
     uint8_t* boxes = smem + (size_t)kStages * kStageBytes + (size_t)(warp - kFirstEpiWarp) * kEpiStageBytes;
-    constexpr int kBoxes = GATE_UP ? 1 : 2;          // 64 bf16 columns per box
     int tc = 0;
     for (int tile = pair; tile < n_tiles; tile += n_pairs, ++tc) {
       const int mt = tile / n_ntiles, nt = tile - mt * n_ntiles;
@@ -291,8 +292,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      uint4 w4[8 * kBoxes];
-      int col0;                                      // first output column of this warp's boxes
       if (GATE_UP) {
         // columns 128 ch .. +63 gate, +64 .. +127 up of features 64 ch .. +63
         const float sg = rs * p.ts0[e], su = rs * p.ts1[e];
@@ -305,7 +304,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(acc_empty_even);
-        col0 = nt * 128 + 64 * ch;
+        const int col0 = nt * 128 + 64 * ch;         // first output column of this warp's box
+        uint4 w4[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           uint32_t w[4];
@@ -318,7 +318,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           w4[c] = make_uint4(w[0], w[1], w[2], w[3]);
         }
+        // the previous tile's stores must have read the staging box
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
+#pragma unroll
+        for (int c = 0; c < 8; ++c)                  // 16-byte chunk c of this row, 128-byte swizzle
+          *reinterpret_cast<uint4*>(boxes + lane * 128 + ((c ^ (lane & 7)) << 4)) = w4[c];
+        fence_proxy_async_smem();                    // generic-proxy writes visible to the tensor store
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&p.tma_out, col0, row0, boxes);
+          bulk_commit_group();
+        }
+        __syncwarp();
       } else {
+        // fp32 rows: 128 columns per thread, two passes of two 32-column boxes
         const float sc = asg >= 0 ? rs * p.ts0[e] * p.weights[asg] : 0.f;
         uint32_t v[128];
 #pragma unroll
@@ -327,32 +341,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(acc_empty_even);
-        col0 = nt * kTileN + 128 * ch;
+        const int col0 = nt * kTileN + 128 * ch;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          uint32_t w[4];
+        for (int pass = 0; pass < 2; ++pass) {
+          if (lane == 0) bulk_wait_read_all();      // the boxes' previous stores have read them
+          __syncwarp();
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            w[i] = pack_bf16x2(__uint_as_float(v[8 * c + 2 * i]) * sc, __uint_as_float(v[8 * c + 2 * i + 1]) * sc);
-          w4[c] = make_uint4(w[0], w[1], w[2], w[3]);
+          for (int b = 0; b < 2; ++b)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const int x = 64 * pass + 32 * b + 4 * c;
+              *reinterpret_cast<float4*>(boxes + b * kEpiBoxBytes + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                  make_float4(__uint_as_float(v[x]) * sc, __uint_as_float(v[x + 1]) * sc,
+                              __uint_as_float(v[x + 2]) * sc, __uint_as_float(v[x + 3]) * sc);
+            }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+#pragma unroll
+            for (int b = 0; b < 2; ++b) tma_store_2d(&p.tma_out, col0 + 64 * pass + 32 * b, row0, boxes + b * kEpiBoxBytes);
+            bulk_commit_group();
+          }
+          __syncwarp();
         }
       }
-      // the previous tile's stores must have read the staging boxes
-      if (lane == 0) bulk_wait_read_all();
-      __syncwarp();
-#pragma unroll
-      for (int c = 0; c < 8 * kBoxes; ++c) {       // 16-byte chunk c of this row, 128-byte swizzle
-        const int b = c >> 3, cc = c & 7;
-        *reinterpret_cast<uint4*>(boxes + b * kEpiBoxBytes + lane * 128 + ((cc ^ (lane & 7)) << 4)) = w4[c];
-      }
-      fence_proxy_async_smem();        // generic-proxy writes visible to the tensor stores
-      __syncwarp();
-      if (lane == 0) {
-#pragma unroll
-        for (int b = 0; b < kBoxes; ++b) tma_store_2d(&p.tma_out, col0 + 64 * b, row0, boxes + b * kEpiBoxBytes);
-        bulk_commit_group();
-      }
-      __syncwarp();
     }
     if (lane == 0) bulk_wait_all();
   }
@@ -394,9 +406,13 @@ cudaError_t launch_fp4_grouped_gemm(const Fp4GemmArgs& a, cudaStream_t st) {
   if (!atom_map(&p.tma_sfa, a.a_sf, a.P_max / 128 * KB)) return cudaErrorInvalidValue;
   // GATE_UP: interleaved gate/up atoms, 2 E I / 128 row blocks
   if (!atom_map(&p.tma_sfb0, a.b0_sf, (gu ? 2 * brows : brows) / 128 * KB)) return cudaErrorInvalidValue;
-  if (!make_tensor_map_2d(&p.tma_out, a.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.out_cols,
-                          (uint64_t)a.P_max, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
+  // output boxes: GATE_UP bf16 h, 64 columns x 32 rows; DOWN fp32 rows, 32 x 32
+  const bool out_ok =
+      gu ? make_tensor_map_2d(&p.tma_out, a.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.out_cols,
+                              (uint64_t)a.P_max, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B)
+         : make_tensor_map_2d(&p.tma_out, a.out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)a.out_cols,
+                              (uint64_t)a.P_max, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!out_ok) return cudaErrorInvalidValue;
   p.row_scale = a.row_scale;
   p.ts0 = a.ts0;
   p.ts1 = a.ts1;

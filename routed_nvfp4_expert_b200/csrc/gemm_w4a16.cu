@@ -63,7 +63,7 @@ struct W4Params {
   CUtensorMap tma_c0;      // gate (or down) codes [E*rows, K/2] bytes; box 32 B x 128 rows
   CUtensorMap tma_c1;      // up codes (GATE_UP)
   CUtensorMap tma_sf;      // scale atoms as [2 n_atoms, 256]; box 256 x 4 (2 atoms)
-  void* out;               // GATE_UP: h f16 [P, I]; DOWN: rows bf16 [P, H]
+  void* out;               // GATE_UP: h f16 [P, I]; DOWN: rows fp32 [P, H]
   const float* row_scale;  // [P] A row unscale (nullable: 1)
   const float* ts0;        // [E]
   const float* ts1;        // [E]
@@ -360,8 +360,8 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
       } else {
         const int asg = p.tile_rows[row];
         const float sc = asg >= 0 ? rs * p.ts0[e] * p.weights[asg] : 0.f;
-        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) + (size_t)row * p.out_cols +
-                                              nt * kTileN + 128 * ch);
+        float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + (size_t)row * p.out_cols +
+                                                nt * kTileN + 128 * ch);
 #pragma unroll 1
         for (int hh = 0; hh < 2; ++hh) {
           uint32_t v[64];
@@ -369,13 +369,9 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
           tmem_ld32(tq + 128 * ch + 64 * hh + 32, v + 32);
           tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            uint32_t w[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              w[i] = pack_bf16x2(__uint_as_float(v[8 * c + 2 * i]) * sc, __uint_as_float(v[8 * c + 2 * i + 1]) * sc);
-            dst[8 * hh + c] = make_uint4(w[0], w[1], w[2], w[3]);
-          }
+          for (int c = 0; c < 16; ++c)
+            dst[16 * hh + c] = make_float4(__uint_as_float(v[4 * c]) * sc, __uint_as_float(v[4 * c + 1]) * sc,
+                                           __uint_as_float(v[4 * c + 2]) * sc, __uint_as_float(v[4 * c + 3]) * sc);
         }
       }
       tc_fence_before();

@@ -46,38 +46,25 @@ struct ExpertGemvArgs {
 
 cudaError_t launch_nvfp4_gemv(const ExpertGemvArgs& a, cudaStream_t st);
 
-// Single-token decode chain (decode_t1.cu): K1 router + top-k + shared
-// gate/up, K2 routed gate/up, K3 routed + shared down with the combine.
-// K2 / K3 also run alone (the expert GEMV entry point at T = 1) from a routing
-// plan: ids == nullptr, active / first from the plan.
+// Single-token expert projections on the tensor cores (decode_t1.cu): the
+// live experts' gate/up with the clamped SwiGLU (h), then their down rows
+// times the routing weights (r), both from the routing plan.
 struct DecodeT1Args {
-  int H, I, Is, E, k, lb, le;
-  float rsf, limit;
+  int H, I, E, k, lb, le;
+  float limit;
   const uint16_t* x;                 // bf16 [H]
-  const float* router_w;             // fp32 [E, H]
-  const float* router_bias;          // fp32 [E]
   nvfp4_bank_t gate, up, down;
-  const uint16_t* sh_gate;           // bf16 [Is, H] (nullable)
-  const uint16_t* sh_up;
-  const uint16_t* sh_down;           // bf16 [H, Is] (nullable: no shared expert)
-  float* logits;                     // fp32 [E]
-  int32_t* ids;                      // [k]; nullptr: the plan form below
-  float* weights;                    // [k] routing weights
-  const int32_t* active;             // plan form: active local experts (count first)
-  const int32_t* first;              // plan form: the assignment of each active expert
-  moe_plan_t plan;                   // K1 writes the routing plan when plan.counts != nullptr
-  uint32_t* xmax;                    // max |x| (fp32 bits)
-  uint32_t* ticket;                  // K1's arrival counter, 0 before K1
+  const int32_t* active;             // routing plan: active local experts (count first)
+  const int32_t* first;              // routing plan: the assignment of each active expert
+  const float* weights;              // [k] routing weights
+  const uint32_t* xmax;              // max |x| (fp32 bits)
   float* h;                          // fp32 [k, I]
-  float* h_shared;                   // fp32 [Is]
-  float* r;                          // fp32 [k, H] weighted routed rows (nullable)
-  uint16_t* y;                       // bf16 [H] (nullable: no combine)
-  float* shared_out;                 // fp32 [H] the shared row (nullable)
+  float* r;                          // fp32 [k, H] weighted routed rows
   uint32_t* status;
-  int l2_prefetch;                   // K2 prefetches K3's down rows into L2
 };
-bool decode_t1_supported(int H, int I, int Is, int E, int k);
-cudaError_t launch_decode_t1_router(const DecodeT1Args& p, cudaStream_t st);
+// H a multiple of 512 up to 8192, I a multiple of 256 up to 2048, k <= 16,
+// E <= 1024 (the shared-memory plans fit).
+bool decode_t1_supported(int H, int I, int E, int k);
 cudaError_t launch_decode_t1_gate_up(const DecodeT1Args& p, cudaStream_t st);
 cudaError_t launch_decode_t1_down(const DecodeT1Args& p, cudaStream_t st);
 
@@ -112,9 +99,11 @@ struct PaddedIndex {
   const int32_t* tile_offsets;
   int local_begin, local_end;
 };
-cudaError_t launch_unpermute_combine(const PaddedIndex& q, int T, int k, int H, const uint16_t* rows,
-                                     const uint16_t* shared, uint16_t* y, cudaStream_t st);
-cudaError_t launch_unpermute(const PaddedIndex& q, long long A, int H, const uint16_t* rows, uint16_t* out,
+// rows: fp32 [P, H] weighted down rows in the padded tile order; shared:
+// fp32 [T, H] (nullable).
+cudaError_t launch_unpermute_combine(const PaddedIndex& q, int T, int k, int H, const float* rows,
+                                     const float* shared, uint16_t* y, cudaStream_t st);
+cudaError_t launch_unpermute(const PaddedIndex& q, long long A, int H, const float* rows, float* out,
                              cudaStream_t st);
 cudaError_t launch_combine(int T, int k, int H, const uint16_t* r, const uint16_t* shared, uint16_t* y,
                            cudaStream_t st);
@@ -134,9 +123,14 @@ cudaError_t launch_dense_gemv(int H, int I, float limit, const uint16_t* x, int 
 // BF16 GEMM on tcgen05 (kind::f16): out [M, N] = a [M, K] . b^T with b [N, K].
 // gate_up: b0 = gate rows, b1 = up rows; out = clamped_swiglu(a.b0^T, a.b1^T).
 // N a multiple of 128 (gate_up) or 256, K a multiple of 64. status: device
-// word for bounded-wait timeouts (nullable).
+// word for bounded-wait timeouts (nullable). out_f32 (not gate_up): fp32
+// output [M, N] in place of out. split: gate_up writes h as two bf16 terms
+// (hi at column c, lo = bf16(h - hi) at N + c; out [M, 2N]); the down
+// product then takes a = [hi | lo] with K = 2 x the weight's K, reading b0
+// twice, so h enters with 16 significant bits.
 cudaError_t launch_bf16_gemm(bool gate_up, const uint16_t* a, int M, int K, const uint16_t* b0, const uint16_t* b1,
-                             int N, float limit, uint16_t* out, uint32_t* status, cudaStream_t st);
+                             int N, float limit, uint16_t* out, uint32_t* status, cudaStream_t st,
+                             float* out_f32 = nullptr, bool split = false);
 // Limit of the BF16 GEMM's main-loop waits for later launches (host setting;
 // 0 = give up at the first incomplete poll). Test hook for the timeout path.
 void set_test_wait_limit_ns(unsigned long long ns);
@@ -154,10 +148,12 @@ cudaError_t launch_router_split(const float* w, int E, int H, uint16_t* w3, cuda
 // Dense BF16 FFN, picking the GEMV form for small T and the tcgen05 GEMM for
 // T >= kDenseGemmMinT (when the shapes allow it).
 constexpr int kDenseGemmMinT = 128;
-// hbuf: T*I*4 bytes (fp32 h in the GEMV form, bf16 h in the GEMM form).
+// hbuf: T*I*4 bytes (fp32 h in the GEMV form; in the GEMM form bf16 h, or,
+// when y_f32, h as two bf16 terms hi + lo).
+// y: bf16 [T, H], or fp32 when y_f32.
 cudaError_t launch_dense_ffn(int H, int I, float limit, const uint16_t* x, int T, const uint16_t* wg,
-                             const uint16_t* wu, const uint16_t* wd, uint16_t* y, void* hbuf, uint32_t* status,
-                             cudaStream_t st);
+                             const uint16_t* wu, const uint16_t* wd, void* y, bool y_f32, void* hbuf,
+                             uint32_t* status, cudaStream_t st);
 
 // ---------------------------------------------------------------- prefill (W4A4, tcgen05)
 
@@ -210,7 +206,8 @@ struct Fp4GemmArgs {
   const int32_t* tile_offsets;     // [E+1]
   const int32_t* tile_rows;        // [P_max]
   const float* weights;            // [A] routing weights (down)
-  uint16_t* out;                   // [P_max, out_cols] in the padded tile order (h, or weighted down rows)
+  void* out;                       // [P_max, out_cols] in the padded tile order: GATE_UP h bf16,
+                                   // DOWN weighted rows fp32
   uint32_t* status;
 };
 cudaError_t launch_fp4_grouped_gemm(const Fp4GemmArgs& a, cudaStream_t st);
@@ -238,7 +235,7 @@ struct W4a16GemmArgs {
   const int32_t* tile_offsets;     // [E+1]
   const int32_t* tile_rows;        // [P_max]
   const float* weights;            // [A] routing weights (DOWN)
-  void* out;                       // GATE_UP: h f16 [P_max, I]; DOWN: rows bf16 [P_max, H]
+  void* out;                       // GATE_UP: h f16 [P_max, I]; DOWN: rows fp32 [P_max, H]
   uint32_t* status;
 };
 cudaError_t launch_w4a16_grouped_gemm(const W4a16GemmArgs& a, cudaStream_t st);

@@ -376,3 +376,93 @@ def test_decode_on_quantised_bank(name, T):
     ref = OS.site_forward(inp, oracle_cfg(wl), "decode", gpu_logits=lg)
     assert_bf16_close(bf16_np(y), ref["y"], what=f"{name} quantised-bank y")
     assert rel_l2(bf16_np(y), ref["y"]) < 5e-3
+
+
+# ------------------------------------------------------------------ single-token tensor-core kernels
+#
+# One token with H a multiple of 512 and I a multiple of 256 runs the routed
+# experts on the tensor cores (16-row weight tiles streamed by TMA, mma.sync);
+# these shapes cover one and several 512-code parts per gate/up tile, 1 to 16
+# live experts, items that do not divide evenly over the SMs, the largest
+# supported H and I, and sites without a shared expert.
+
+def _t1(H, I, E, k, Is, **kw):
+    from routed_nvfp4_expert_b200 import synthetic as syn
+    return syn.Workload(f"t1_H{H}_I{I}_E{E}_k{k}", T=1, H=H, I=I, E=E, k=k, Is=Is, dense_I=64,
+                        sigma_w=kw.pop("sigma_w", 0.0064 if H >= 2048 else 0.02), **kw)
+
+
+T1_SHAPES = [(512, 256, 32, 4, 256), (1536, 768, 24, 6, 256), (1024, 512, 40, 16, 0), (8192, 2048, 12, 8, 512)]
+
+
+@pytest.mark.parametrize("H,I,E,k,Is", T1_SHAPES)
+def test_t1_tensor_core_forward_matches_oracle(H, I, E, k, Is):
+    wl = _t1(H, I, E, k, Is)
+    inp = site_inputs(wl)
+    y, lg, ws, v = _forward(wl, inp)
+    ref = OS.site_forward(inp, oracle_cfg(wl), "decode", gpu_logits=lg, want_parts=True)
+    got = bf16_np(y)
+    assert_bf16_close(got, ref["y"], what=f"{wl.name} y")
+    assert rel_l2(got, ref["y"]) < 5e-3
+    r = capi.view_tensor(v.r, (1, k, H), torch.float32)
+    assert_bf16_close(bf16_np(r), ref["r"], what="r")
+    # h: the SwiGLU rows of the live assignments (fp32)
+    h = capi.view_tensor(v.h, (k, I), torch.float32).cpu().numpy().astype(np.float64)
+    ids = ref["ids"][0]
+    cache = OS.ExpertCache(inp)
+    a64 = OF.bf16_value(inp["x"])
+    for j in range(k):
+        wg, wu, _ = cache.get(int(ids[j]))
+        assert_bf16_close(h[j], OS.clamped_swiglu(wg @ a64[0], wu @ a64[0], wl.limit), what=f"h[{j}]")
+    # the same input twice: bit-identical (every sum in a fixed order)
+    y2, _, _, _ = _forward(wl, inp)
+    assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
+
+
+@pytest.mark.parametrize("local", [(0, 16), (16, 32), (7, 7), (5, 21)])
+def test_t1_tensor_core_local_range(local):
+    wl = _t1(512, 256, 32, 8, 256)
+    inp = site_inputs(wl)
+    y, lg, _, v = _forward(wl, inp, local=local)
+    ref = OS.site_forward(inp, oracle_cfg(wl, local), "decode", gpu_logits=lg, want_parts=True)
+    assert_bf16_close(bf16_np(y), ref["y"], what=f"local {local}")
+    r = capi.view_tensor(v.r, (1, wl.k, wl.H), torch.float32).cpu().numpy()
+    remote = ~((ref["ids"][0] >= local[0]) & (ref["ids"][0] < local[1]))
+    assert (r[0][remote] == 0).all()
+
+
+def test_t1_tensor_core_clamp_fires_and_matches_oracle():
+    wl = _t1(512, 256, 32, 8, 256, x_scale=64.0)
+    inp = site_inputs(wl)
+    y, lg, _, _ = _forward(wl, inp)
+    ref = OS.site_forward(inp, oracle_cfg(wl), "decode", gpu_logits=lg)
+    assert 0.05 * ref["clamp_total"] < ref["clamp_fired"] < ref["clamp_total"]
+    assert_bf16_close(bf16_np(y), ref["y"], what="clamped y")
+
+
+def test_t1_tensor_core_standalone_gemv():
+    """The expert GEMV entry point at T = 1 runs the same kernels: its h and r
+    match the oracle and moe_combine of r gives the routed part of y."""
+    wl = _t1(1536, 768, 24, 6, 0)
+    inp = site_inputs(wl)
+    cfg = capi.config_for(wl)
+    site = device_site(wl, inp)
+    k = wl.k
+    logits = torch.empty((1, wl.E), dtype=torch.float32, device="cuda")
+    ids = torch.empty((1, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((1, k), dtype=torch.float32, device="cuda")
+    capi.moe_router_topk(cfg, _x(inp), site.router_w, site.router_bias, logits, ids, w)
+    buf, plan = _plan_tensors(cfg, 1)
+    wsp = capi.alloc_workspace(cfg, 1, capi.PATH_PREFILL)
+    capi.moe_permute(cfg, ids, plan, wsp)
+    h = torch.full((k, wl.I), 3.0, dtype=torch.float32, device="cuda")
+    r = torch.full((1, k, wl.H), 5.0, dtype=torch.float32, device="cuda")
+    wsd = capi.alloc_workspace(cfg, 1, capi.PATH_DECODE)
+    capi.nvfp4_expert_gemv(cfg, capi.PROJ_GATE_UP, _x(inp), 1, plan, None, site, h, wsd)
+    capi.nvfp4_expert_gemv(cfg, capi.PROJ_DOWN, h, 1, plan, w, site, r, wsd)
+    capi.moe_read_device_status(wsd)
+    y = torch.empty((1, wl.H), dtype=torch.bfloat16, device="cuda")
+    capi.moe_combine(r, None, y)
+    ref = OS.site_forward(inp, oracle_cfg(wl), "decode", gpu_logits=logits.cpu().numpy(), want_parts=True)
+    assert_bf16_close(bf16_np(r), ref["r"], what="r rows")
+    assert_bf16_close(bf16_np(y), ref["y"], what="routed y")

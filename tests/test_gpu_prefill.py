@@ -155,16 +155,16 @@ def _site_state(wl, cfg, T, v):
     st["hq"] = capi.view_tensor(v.hq_codes, (P, I // 2), torch.uint8).cpu().numpy()[:Pu]
     st["hsf"] = sf_untile(capi.view_tensor(v.hq_sf, (P * I // 16,), torch.uint8).cpu().numpy(), Pu, I)
     st["hts"] = capi.view_tensor(v.hq_scale, (P,), torch.float32).cpu().numpy()[:Pu]
-    st["r_pad"] = bf16_np(capi.view_tensor(v.r, (P, H), torch.bfloat16)[:Pu])
+    st["r_pad"] = bf16_np(capi.view_tensor(v.r, (P, H), torch.float32)[:Pu])
     return st
 
 
 def _token_rows(cfg, wl, T, v):
     """The routed rows r[t, j] in token order, through moe_unpermute."""
     P = capi.moe_padded_rows(cfg, T)
-    rows = capi.view_tensor(v.r, (P, wl.H), torch.bfloat16)
+    rows = capi.view_tensor(v.r, (P, wl.H), torch.float32)
     ids = capi.view_tensor(v.ids, (T, wl.k), torch.int32)
-    out = torch.full((T, wl.k, wl.H), 3.0, dtype=torch.bfloat16, device="cuda")
+    out = torch.full((T, wl.k, wl.H), 3.0, dtype=torch.float32, device="cuda")
     capi.moe_unpermute(cfg, rows, T, v.plan, ids, out)
     return out
 
@@ -242,17 +242,17 @@ def test_grouped_gemm_entry_point_matches_forward():
     ws2 = capi.alloc_workspace(cfg, T, capi.PATH_PREFILL)
     h2 = torch.zeros((P, wl.I), dtype=torch.bfloat16, device="cuda")
     capi.nvfp4_grouped_gemm(cfg, capi.PROJ_GATE_UP, xq, xsf, xts, T, v.plan, wts, site, h2, ws2)
-    r2 = torch.full((P, wl.H), 7.0, dtype=torch.bfloat16, device="cuda")
+    r2 = torch.full((P, wl.H), 7.0, dtype=torch.float32, device="cuda")
     capi.nvfp4_grouped_gemm(cfg, capi.PROJ_DOWN, hq, hsf, hts, T, v.plan, wts, site, r2, ws2)
     capi.moe_read_device_status(ws2)
     ntiles = int(_arr(v.plan.tile_offsets, wl.E + 1)[wl.E])
     h = capi.view_tensor(v.h, (P, wl.I), torch.bfloat16)
-    r = capi.view_tensor(v.r, (P, wl.H), torch.bfloat16)
+    r = capi.view_tensor(v.r, (P, wl.H), torch.float32)
     assert torch.equal(h2[:ntiles * TILE], h[:ntiles * TILE])
     assert torch.equal(r2[:ntiles * TILE], r[:ntiles * TILE])
     # the fused unpermute + combine equals unpermute then moe_combine, and y
     ids = capi.view_tensor(v.ids, (T, wl.k), torch.int32)
-    sh = capi.view_tensor(v.shared, (T, wl.H), torch.bfloat16)
+    sh = capi.view_tensor(v.shared, (T, wl.H), torch.float32)
     y2 = torch.empty_like(y)
     capi.moe_unpermute_combine(cfg, r, T, v.plan, ids, sh, y2)
     assert torch.equal(y2, y)
@@ -285,9 +285,68 @@ def test_moe_forward_prefill_matches_oracle(name, T):
     ids = capi.view_tensor(v.ids, (wl.T, wl.k), torch.int32).cpu().numpy()
     assert np.array_equal(ids[tokens], ref["ids"])
     got = bf16_np(y)[tokens]
-    assert_bf16_close(got, ref["y"], what=f"{wl.name} y")
-    r = _token_rows(cfg, wl, wl.T, v)
-    assert_bf16_close(bf16_np(r)[tokens], ref["r"], what="r")
+    if not wl.stress:
+        assert_bf16_close(got, ref["y"], what=f"{wl.name} y")
+        r = _token_rows(cfg, wl, wl.T, v)
+        assert_bf16_close(bf16_np(r)[tokens], ref["r"], what="r")
+        return
+    # x8 activations put many h values next to an NVFP4 code boundary. The h
+    # encoding is a decision on the GPU's bf16 h, whose GEMM sum rounds in
+    # another order than the oracle's fp64 h, so the two sides may pick
+    # neighbouring codes there. The GPU's h is held to the GEMM tolerance
+    # against the oracle; y to the elementwise gate against the oracle's down
+    # projection and combine of the GPU's own h encoding, and to the relative
+    # L2 bound against the independent oracle.
+    prow, pids = _assignment_rows(cfg, wl, v, tokens)
+    live = prow >= 0
+    P = capi.moe_padded_rows(cfg, wl.T)
+    sel = np.where(live, prow, 0).reshape(-1)
+    hg = bf16_np(capi.view_tensor(v.h, (P, wl.I), torch.bfloat16)[torch.from_numpy(sel).cuda().long()])
+    cache = OS.ExpertCache(inp)
+    xdeq = OS.prefill_activation(inp["x"][tokens])
+    for ti, j in zip(*np.nonzero(live)):
+        wg, wu, _ = cache.get(int(pids[ti, j]))
+        href = OS.clamped_swiglu(wg @ xdeq[ti], wu @ xdeq[ti], wl.limit)
+        hrow = hg[ti * wl.k + j]
+        d = np.abs(hrow - href)
+        assert np.all(d <= 2.0 ** -8 * np.abs(href) + 1e-4 * np.abs(href).max()), (ti, j, d.max())
+    yh = _y_from_gpu_h(wl, cfg, v, inp, tokens, prow, pids, ref)
+    assert_bf16_close(got, yh, what=f"{wl.name} y (oracle down on the GPU's h codes)")
+    assert rel_l2(got, ref["y"]) < 5e-3
+
+
+def _assignment_rows(cfg, wl, v, tokens):
+    """Padded-layout row of each assignment (t, j) of the given tokens (-1 for
+    a remote expert), and the ids: expert e's segment starts at tile
+    tile_offsets[e], in the stable sorted order of the plan."""
+    E, k, T = wl.E, wl.k, wl.T
+    ids = _arr(v.ids, T * k).reshape(T, k)[tokens]
+    inv = _arr(v.plan.inv, T * k).reshape(T, k)[tokens]
+    offs = _arr(v.plan.offsets, E + 1)
+    toffs = _arr(v.plan.tile_offsets, E + 1)
+    local = (ids >= cfg.local_begin) & (ids < cfg.local_end)
+    rows = toffs[ids] * TILE + (inv - offs[ids])
+    return np.where(local, rows, -1), ids
+
+
+def _y_from_gpu_h(wl, cfg, v, inp, tokens, prow, ids, ref):
+    """The oracle's down projection, routing weights and combine applied to the
+    GPU's NVFP4 encoding of h for the given tokens."""
+    P = capi.moe_padded_rows(cfg, wl.T)
+    sel = np.where(prow >= 0, prow, 0).reshape(-1)
+    codes = capi.view_tensor(v.hq_codes, (P, wl.I // 2), torch.uint8)[torch.from_numpy(sel).cuda().long()]
+    atoms = capi.view_tensor(v.hq_sf, (P * wl.I // 16,), torch.uint8).cpu().numpy()
+    KB = wl.I // 64
+    pp, b = sel[:, None], np.arange(wl.I // 16)[None, :]
+    sf = atoms[((pp // 128) * KB + b // 4) * 512 + (pp % 32) * 16 + ((pp % 128) // 32) * 4 + b % 4]
+    ts = capi.view_tensor(v.hq_scale, (P,), torch.float32).cpu().numpy()[sel]
+    hdeq = OF.dequant_rows_nvfp4(codes.cpu().numpy(), sf, ts).reshape(len(tokens), wl.k, wl.I)
+    cache = OS.ExpertCache(inp)
+    r = np.zeros((len(tokens), wl.k, wl.H))
+    for ti, j in zip(*np.nonzero(prow >= 0)):
+        _, _, wd = cache.get(int(ids[ti, j]))
+        r[ti, j] = ref["weights"][ti, j] * (wd @ hdeq[ti, j])
+    return OS.combine(r, ref["shared"])
 
 
 def test_prefill_is_deterministic_and_chunk_invariant():
@@ -400,12 +459,12 @@ def test_w4a16_entry_point_matches_forward():
     xa = capi.view_tensor(v.xq_codes, (P, wl.H), torch.float16)
     xs = capi.view_tensor(v.xq_scale, (P,), torch.float32)
     h = capi.view_tensor(v.h, (P, wl.I), torch.float16)
-    r = capi.view_tensor(v.r, (P, wl.H), torch.bfloat16)
+    r = capi.view_tensor(v.r, (P, wl.H), torch.float32)
     wts = capi.view_tensor(v.weights, (T * wl.k,), torch.float32)
     ws2 = capi.alloc_workspace(cfg, T, capi.PATH_PREFILL_W4A16)
     h2 = torch.zeros((P, wl.I), dtype=torch.float16, device="cuda")
     capi.nvfp4_grouped_gemm_w4a16(cfg, capi.PROJ_GATE_UP, xa, xs, T, v.plan, wts, site, h2, ws2)
-    r2 = torch.full((P, wl.H), 7.0, dtype=torch.bfloat16, device="cuda")
+    r2 = torch.full((P, wl.H), 7.0, dtype=torch.float32, device="cuda")
     capi.nvfp4_grouped_gemm_w4a16(cfg, capi.PROJ_DOWN, h, None, T, v.plan, wts, site, r2, ws2)
     capi.moe_read_device_status(ws2)
     used = int(_arr(v.plan.tile_offsets, wl.E + 1)[wl.E]) * TILE
