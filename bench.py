@@ -161,7 +161,7 @@ class ClockSampler:
 def decode_t1_fused(wl) -> bool:
     """The single-token tensor-core expert kernels run for this workload;
     mirrors the library's eligibility rule for T = 1."""
-    return (wl.kind == "decode" and wl.T == 1 and wl.H % 512 == 0 and wl.H <= 8192 and wl.I % 256 == 0
+    return (wl.kind == "decode" and wl.T == 1 and wl.H % 1024 == 0 and wl.H <= 8192 and wl.I % 128 == 0
             and wl.I <= 2048 and wl.k <= 16 and wl.E <= 1024)
 
 

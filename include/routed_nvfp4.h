@@ -428,11 +428,12 @@ moe_status_t nvfp4_dequant(const uint8_t* codes, const uint8_t* scales, const fl
  *     gate/up and down; moe_combine_f32. The shared expert runs on the
  *     library's auxiliary stream of this host thread and device, forked from
  *     and joined back into `stream` with events.
- *     T = 1 with H % 512 == 0, H <= 8192, I % 256 == 0, I <= 2048, k <= 16,
- *     E <= 1024: the expert projections run on the tensor cores, one CTA per
- *     SM streaming 16-row weight tiles through a TMA ring into mma.sync
- *     (each E2M1 code times its E4M3 scale exact in f16, x or h scaled by a
- *     power of two into f16, fp32 accumulation). Otherwise the GEMV kernels
+ *     T = 1 with H % 1024 == 0, H <= 8192, I % 128 == 0, I <= 2048, k <= 16,
+ *     E <= 1024: the expert projections run on the tensor cores, each warp
+ *     loading its weight rows straight into registers with 128-bit loads and
+ *     multiplying them with mma.sync (each E2M1 code times its E4M3 scale
+ *     exact in f16, x or h scaled by a power of two into f16, fp32
+ *     accumulation). Otherwise the GEMV kernels
  *     of nvfp4_expert_gemv.
  *   MOE_PATH_PREFILL_W4A16: the pages' prefill numerics: permute with the
  *     padded tile layout, x gathered to f16 rows (per-row power-of-two scale),

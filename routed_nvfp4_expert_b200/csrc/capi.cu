@@ -895,6 +895,7 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
       d.gate = w->gate; d.up = w->up; d.down = w->down;
       d.active = plan.active; d.first = plan.first;
       d.weights = wts; d.xmax = xmax; d.h = h; d.r = r;
+      d.l2_down = 1;
       d.status = status;
       RNX_CUDA(mark(MOE_STAGE_EXPERT_GATE_UP, st), "stage event");
       RNX_CUDA(rnx::launch_decode_t1_gate_up(d, st), "expert gate/up");

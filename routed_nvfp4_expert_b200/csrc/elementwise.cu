@@ -6,6 +6,8 @@
 
 namespace rnx {
 
+constexpr int kMaxTopKRows = 16;   // k <= 16 (the pages' KERNEL_MAX_TOP_K)
+
 namespace {
 
 // moe_combine (glm5next_mlp, "The stack this layer runs" / "Traps"): the k
@@ -51,8 +53,8 @@ __global__ void __launch_bounds__(256) combine_kernel(int T, int k, int H, const
 
 // moe_combine over fp32 rows (the decode path keeps r and the shared row in
 // fp32): the same order and one rounding. Each thread owns 4 consecutive
-// hidden elements.
-__global__ void __launch_bounds__(256) combine_f32_kernel(int T, int k, int H, const float* __restrict__ r,
+// hidden elements; its k + 1 loads go out together before the sum.
+__global__ void __launch_bounds__(128) combine_f32_kernel(int T, int k, int H, const float* __restrict__ r,
                                                           const float* __restrict__ shared, uint16_t* __restrict__ y) {
   pdl_wait();
   pdl_trigger();
@@ -60,20 +62,26 @@ __global__ void __launch_bounds__(256) combine_f32_kernel(int T, int k, int H, c
   const long long n = (long long)T * per_row;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
     const int t = (int)(i / per_row), c = (int)(i - (long long)t * per_row);
+    float4 v[kMaxTopKRows];
+#pragma unroll
+    for (int j = 0; j < kMaxTopKRows; ++j)
+      v[j] = j < k ? reinterpret_cast<const float4*>(r + ((size_t)t * k + j) * H)[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 sv = shared ? reinterpret_cast<const float4*>(shared + (size_t)t * H)[c] : make_float4(0.f, 0.f, 0.f, 0.f);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < k; ++j) {
-      const float4 v = reinterpret_cast<const float4*>(r + ((size_t)t * k + j) * H)[c];
-      acc.x += v.x;
-      acc.y += v.y;
-      acc.z += v.z;
-      acc.w += v.w;
+#pragma unroll
+    for (int j = 0; j < kMaxTopKRows; ++j) {
+      if (j < k) {
+        acc.x += v[j].x;
+        acc.y += v[j].y;
+        acc.z += v[j].z;
+        acc.w += v[j].w;
+      }
     }
     if (shared) {
-      const float4 v = reinterpret_cast<const float4*>(shared + (size_t)t * H)[c];
-      acc.x += v.x;
-      acc.y += v.y;
-      acc.z += v.z;
-      acc.w += v.w;
+      acc.x += sv.x;
+      acc.y += sv.y;
+      acc.z += sv.z;
+      acc.w += sv.w;
     }
     uint2 o;
     o.x = pack_bf16x2(acc.x, acc.y);
@@ -211,7 +219,8 @@ cudaError_t launch_combine(int T, int k, int H, const uint16_t* r, const uint16_
 
 cudaError_t launch_combine_f32(int T, int k, int H, const float* r, const float* shared, uint16_t* y,
                                cudaStream_t st) {
-  return launch_pdl(combine_f32_kernel, dim3(grid_for((long long)T * (H / 4), 256)), dim3(256), 0, st, T, k, H, r,
+  if (k > kMaxTopKRows) return cudaErrorInvalidValue;
+  return launch_pdl(combine_f32_kernel, dim3(grid_for((long long)T * (H / 4), 128)), dim3(128), 0, st, T, k, H, r,
                     shared, y);
 }
 

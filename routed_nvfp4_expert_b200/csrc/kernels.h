@@ -46,9 +46,10 @@ struct ExpertGemvArgs {
 
 cudaError_t launch_nvfp4_gemv(const ExpertGemvArgs& a, cudaStream_t st);
 
-// Single-token expert projections on the tensor cores (decode_t1.cu): the
-// live experts' gate/up with the clamped SwiGLU (h), then their down rows
-// times the routing weights (r), both from the routing plan.
+// Single-token expert projections on the tensor cores (decode_t1.cu), from
+// the routing plan: gate/up writes h (clamped SwiGLU of the live experts'
+// gate and up projections; zero rows for the other assignments), down writes
+// the weighted rows r.
 struct DecodeT1Args {
   int H, I, E, k, lb, le;
   float limit;
@@ -61,9 +62,10 @@ struct DecodeT1Args {
   float* h;                          // fp32 [k, I]
   float* r;                          // fp32 [k, H] weighted routed rows
   uint32_t* status;
+  int l2_down;                       // gate/up also asks L2 for the down tiles the down kernel reads next
 };
-// H a multiple of 512 up to 8192, I a multiple of 256 up to 2048, k <= 16,
-// E <= 1024 (the shared-memory plans fit).
+// H a multiple of 1024 up to 8192, I a multiple of 128 up to 2048, k <= 16,
+// E <= 1024.
 bool decode_t1_supported(int H, int I, int E, int k);
 cudaError_t launch_decode_t1_gate_up(const DecodeT1Args& p, cudaStream_t st);
 cudaError_t launch_decode_t1_down(const DecodeT1Args& p, cudaStream_t st);
@@ -111,6 +113,7 @@ cudaError_t launch_combine(int T, int k, int H, const uint16_t* r, const uint16_
 cudaError_t launch_combine_f32(int T, int k, int H, const float* r, const float* shared, uint16_t* y,
                                cudaStream_t st);
 cudaError_t launch_swiglu(const float* gu, int M, int I, float limit, uint16_t* h, cudaStream_t st);
+
 cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* scales, const float* ts, int rows, int K, float* out,
                            cudaStream_t st);
 

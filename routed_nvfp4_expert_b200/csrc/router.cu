@@ -12,6 +12,9 @@ namespace rnx {
 
 namespace {
 
+constexpr int kMaxTopK = 16;   // the pages' KERNEL_MAX_TOP_K
+
+
 // ---------------------------------------------------------------- logits
 // Small T (decode): the fp32 router matrix (E x H, 4.7 MB at E=288, H=4096)
 // is the only real traffic. One 128-thread CTA owns one expert row: every
@@ -185,6 +188,77 @@ __global__ void __launch_bounds__(1024) topk_plan_kernel(const float* __restrict
   small_plan(ids, T * k, E, lb, le, plan, status, s_ids, s_cnt, s_off, s_warp, s_act, s_sorted);
 }
 
+// One token: selection and its routing plan in one CTA without block-wide
+// scans: with k distinct ids every plan entry is a count over the k ids.
+// counts[e] = [e chosen], offsets[e] = #chosen ids < e, tile_offsets[e] =
+// #chosen local ids < e (one 256-row tile per chosen local expert), sorted /
+// inv by expert order, the active list of the chosen local experts in
+// expert order with first[u] = its assignment. All threads load and score the
+// logits (one round of loads), warp 0 selects, all threads write the plan.
+constexpr int kT1PlanThreads = 256;
+template <int PL>
+__global__ void __launch_bounds__(kT1PlanThreads) topk_plan_t1_kernel(const float* __restrict__ logits,
+                                                                      const float* __restrict__ bias, int E, int k,
+                                                                      float rsf, int32_t* ids,
+                                                                      float* __restrict__ weights, int lb, int le,
+                                                                      moe_plan_t plan, uint32_t* status) {
+  __shared__ float s_key[1][32 * PL];
+  __shared__ float s_sig[1][32 * PL];
+  __shared__ int s_ids[kMaxTopK];
+  pdl_wait();
+  pdl_trigger();
+  topk_keys<PL>(logits, bias, 0, 1, E, s_key, s_sig);
+  __syncthreads();
+  if (threadIdx.x < 32) topk_warp<PL>(s_key[0], s_sig[0], 0, E, k, rsf, ids, weights, s_ids);
+  __syncthreads();
+  int id[kMaxTopK];
+  bool valid[kMaxTopK];
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j) {
+    id[j] = j < k ? s_ids[j] : -1;
+    valid[j] = j < k && id[j] >= 0 && id[j] < E;
+  }
+  for (int e = threadIdx.x; e <= E; e += kT1PlanThreads) {
+    int cnt = 0, off = 0, toff = 0;
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      if (!valid[j]) continue;
+      cnt += id[j] == e;
+      off += id[j] < e;
+      toff += id[j] < e && id[j] >= lb && id[j] < le;
+    }
+    if (e < E) plan.counts[e] = cnt;
+    plan.offsets[e] = off;
+    plan.tile_offsets[e] = toff;
+  }
+  if (threadIdx.x < k) {
+    const int j = threadIdx.x;
+    if (valid[j]) {
+      int pos = 0, lpos = 0;
+#pragma unroll
+      for (int i = 0; i < kMaxTopK; ++i) {
+        pos += valid[i] && id[i] < id[j];
+        lpos += valid[i] && id[i] < id[j] && id[i] >= lb && id[i] < le;
+      }
+      plan.sorted[pos] = j;
+      plan.inv[j] = pos;
+      if (id[j] >= lb && id[j] < le) {
+        plan.active[1 + lpos] = id[j];
+        plan.first[lpos] = j;
+      }
+    } else {
+      plan.inv[j] = -1;
+      set_status(status, kDevErrBounds);
+    }
+  }
+  if (threadIdx.x == 0) {
+    int nl = 0;
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) nl += valid[j] && id[j] >= lb && id[j] < le;
+    plan.active[0] = nl;
+  }
+}
+
 __global__ void __launch_bounds__(256) row_absmax_kernel(const uint16_t* __restrict__ rows, int R, int K,
                                                          uint32_t* __restrict__ out) {
   const int lane = threadIdx.x & 31;
@@ -227,6 +301,16 @@ cudaError_t launch_topk_plan(const float* logits, const float* bias, int T, int 
                              float* weights, int lb, int le, const moe_plan_t& plan, uint32_t* status,
                              cudaStream_t st) {
   if (T < 1 || T * k > kSmallMaxA || E > kMaxE) return cudaErrorNotSupported;
+  if (T == 1 && k <= kMaxTopK) {
+    if (E <= 32 * 4)
+      return launch_pdl(topk_plan_t1_kernel<4>, dim3(1), dim3(kT1PlanThreads), 0, st, logits, bias, E, k, rsf, ids, weights, lb, le,
+                        plan, status);
+    if (E <= 32 * 10)
+      return launch_pdl(topk_plan_t1_kernel<10>, dim3(1), dim3(kT1PlanThreads), 0, st, logits, bias, E, k, rsf, ids, weights, lb,
+                        le, plan, status);
+    return launch_pdl(topk_plan_t1_kernel<32>, dim3(1), dim3(kT1PlanThreads), 0, st, logits, bias, E, k, rsf, ids, weights, lb, le,
+                      plan, status);
+  }
   if (E <= 32 * 4 && T <= topk_tokens<4>())
     return launch_pdl(topk_plan_kernel<4>, dim3(1), dim3(1024), 0, st, logits, bias, T, E, k, rsf, ids, weights, lb,
                       le, plan, status);

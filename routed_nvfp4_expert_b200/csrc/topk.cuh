@@ -48,10 +48,11 @@ RNX_DEVICE void topk_keys(const float* __restrict__ logits, const float* __restr
   }
 }
 
-// One warp selects token t's top-k from its keys and writes ids / weights.
+// One warp selects token t's top-k from its keys and writes ids / weights
+// (and the ids to s_ids[0..k) as well when given).
 template <int PL>
 RNX_DEVICE void topk_warp(const float* s_key_row, const float* s_sig_row, int t, int E, int k, float rsf,
-                          int32_t* __restrict__ ids, float* __restrict__ weights) {
+                          int32_t* __restrict__ ids, float* __restrict__ weights, int* s_ids = nullptr) {
   const int lane = threadIdx.x & 31;
   float key[PL], sg[PL];
   int st[PL];
@@ -97,6 +98,7 @@ RNX_DEVICE void topk_warp(const float* s_key_row, const float* s_sig_row, int t,
   float sum = 0.f;
   for (int j = 0; j < k; ++j) sum += __shfl_sync(0xffffffffu, chosen_s, j);
   if (lane < k) {
+    if (s_ids) s_ids[lane] = chosen_id;
     ids[(size_t)t * k + lane] = chosen_id;
     weights[(size_t)t * k + lane] = sum > 0.f ? rsf * (chosen_s / sum) : 0.f;
   }

@@ -380,10 +380,11 @@ def test_decode_on_quantised_bank(name, T):
 
 # ------------------------------------------------------------------ single-token tensor-core kernels
 #
-# One token with H a multiple of 512 and I a multiple of 256 runs the routed
-# experts on the tensor cores (16-row weight tiles streamed by TMA, mma.sync);
-# these shapes cover one and several 512-code parts per gate/up tile, 1 to 16
-# live experts, items that do not divide evenly over the SMs, the largest
+# One token with H a multiple of 1024 and I a multiple of 128 runs the routed
+# experts on the tensor cores (weights loaded straight into registers,
+# mma.sync); these shapes cover one to eight 128-code steps per K octant of a
+# gate/up row pair, one and two register batches of a down tile, 1 to 16 live
+# experts, items that do not divide evenly over the SMs' warps, the largest
 # supported H and I, and sites without a shared expert.
 
 def _t1(H, I, E, k, Is, **kw):
@@ -392,7 +393,7 @@ def _t1(H, I, E, k, Is, **kw):
                         sigma_w=kw.pop("sigma_w", 0.0064 if H >= 2048 else 0.02), **kw)
 
 
-T1_SHAPES = [(512, 256, 32, 4, 256), (1536, 768, 24, 6, 256), (1024, 512, 40, 16, 0), (8192, 2048, 12, 8, 512)]
+T1_SHAPES = [(1024, 128, 32, 4, 256), (3072, 768, 24, 6, 256), (1024, 512, 40, 16, 0), (8192, 2048, 12, 8, 512)]
 
 
 @pytest.mark.parametrize("H,I,E,k,Is", T1_SHAPES)
@@ -421,7 +422,7 @@ def test_t1_tensor_core_forward_matches_oracle(H, I, E, k, Is):
 
 @pytest.mark.parametrize("local", [(0, 16), (16, 32), (7, 7), (5, 21)])
 def test_t1_tensor_core_local_range(local):
-    wl = _t1(512, 256, 32, 8, 256)
+    wl = _t1(1024, 256, 32, 8, 256)
     inp = site_inputs(wl)
     y, lg, _, v = _forward(wl, inp, local=local)
     ref = OS.site_forward(inp, oracle_cfg(wl, local), "decode", gpu_logits=lg, want_parts=True)
@@ -432,7 +433,7 @@ def test_t1_tensor_core_local_range(local):
 
 
 def test_t1_tensor_core_clamp_fires_and_matches_oracle():
-    wl = _t1(512, 256, 32, 8, 256, x_scale=64.0)
+    wl = _t1(1024, 256, 32, 8, 256, x_scale=64.0)
     inp = site_inputs(wl)
     y, lg, _, _ = _forward(wl, inp)
     ref = OS.site_forward(inp, oracle_cfg(wl), "decode", gpu_logits=lg)
@@ -443,7 +444,7 @@ def test_t1_tensor_core_clamp_fires_and_matches_oracle():
 def test_t1_tensor_core_standalone_gemv():
     """The expert GEMV entry point at T = 1 runs the same kernels: its h and r
     match the oracle and moe_combine of r gives the routed part of y."""
-    wl = _t1(1536, 768, 24, 6, 0)
+    wl = _t1(3072, 768, 24, 6, 0)
     inp = site_inputs(wl)
     cfg = capi.config_for(wl)
     site = device_site(wl, inp)
