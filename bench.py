@@ -177,8 +177,11 @@ def measure(wl, args, rank, world, local_rank, dev, clocks=None):
     inp = syn.make_site(wl, seed=0)
     site = capi.site_to_device(inp, dev)
     cfg = capi.config_for(wl)
-    path = capi.PATH_DECODE if wl.kind == "decode" else capi.PATH_PREFILL
-    prefill = path == capi.PATH_PREFILL
+    if wl.kind == "decode":
+        path = capi.PATH_DECODE
+    else:
+        path = capi.PATH_PREFILL_W4A16 if getattr(args, "prefill_path", "w4a4") == "w4a16" else capi.PATH_PREFILL
+    prefill = path != capi.PATH_DECODE
     T, H = wl.T, wl.H
     if prefill:
         capi.moe_prepare_weights(cfg, site)
@@ -302,7 +305,7 @@ def measure(wl, args, rank, world, local_rank, dev, clocks=None):
         if i >= args.warmup:
             e2e_ms.append(e0.elapsed_time(e1))
     capi.moe_read_device_status(ws, stream)
-    res = dict(wl=wl, inp=inp, prefill=prefill, ms=float(np.mean(step_ms)), timed_ms=float(np.mean(timed_ms)),
+    res = dict(wl=wl, inp=inp, prefill=prefill, w4a16=path == capi.PATH_PREFILL_W4A16, ms=float(np.mean(step_ms)), timed_ms=float(np.mean(timed_ms)),
                kern_ms=float(np.mean(kern_ms_l)), e2e_ms=float(np.mean(e2e_ms)),
                stage_avg=np.mean(np.array(stage_ms), axis=0), U=float(np.mean(uniq)), n_spans=len(spans))
     del g_timed, g_plain, g_stages
@@ -388,17 +391,22 @@ def roofline_of(res, pk):
     T, H = wl.T, wl.H
     if res["prefill"]:
         flops = 2.0 * T * wl.k * 3 * H * wl.I          # gate + up + down over the T*k assignments
-        fp4_peak = pk["bf16_tflops"] * FP4_PER_BF16
         achieved = flops / (res["kern_ms"] * 1e-3) / 1e12
-        return {"bound": "tensor", "kernel": "nvfp4_grouped_gemm (tcgen05 mxf4nvf4; gate/up + down launches)",
-                "achieved": round(achieved, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
-                "frac": round(achieved / fp4_peak, 4),
-                "peak_source": f"{pk['source']} bf16 burst x nominal FP4/BF16 ratio {FP4_PER_BF16:g}",
+        if res.get("w4a16"):
+            # kind::f16 tensor math (f16 operands): the measured bf16 peak is the roof
+            peak, src = pk["bf16_tflops"], f"{pk['source']} bf16 burst (f16 operands, same rate)"
+            kernel, stem = "w4a16_gemm_kernel (tcgen05 kind::f16; gate/up + down launches)", "w4a16_grouped_gemm"
+        else:
+            peak = pk["bf16_tflops"] * FP4_PER_BF16
+            src = f"{pk['source']} bf16 burst x nominal FP4/BF16 ratio {FP4_PER_BF16:g}"
+            kernel, stem = "nvfp4_grouped_gemm (tcgen05 mxf4nvf4; gate/up + down launches)", "nvfp4_grouped_gemm"
+        return {"bound": "tensor", "kernel": kernel, "achieved": round(achieved, 1), "peak": round(peak, 1),
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "peak_source": src,
                 "algorithmic_flops_per_step": flops, "unique_experts_per_step": res["U"],
-                "traffic": read_traffic_profile(f"nvfp4_grouped_gemm_{wl.name}")}
+                "traffic": read_traffic_profile(f"{stem}_{wl.name}")}
     routed = res["U"] * expert_bytes(wl)
     if decode_t1_fused(wl):
-        kernel = "t1_gate_up_kernel + t1_down_kernel (mma.sync m16n8k16 on TMA-fed tiles; timed together)"
+        kernel = "t1_gate_up_kernel + t1_down_kernel (128-bit weight loads, mma.sync m16n8k16; timed together)"
     else:
         kernel = "nvfp4_expert_gemv (gate/up + down launches, timed together)"
     achieved = routed / (res["kern_ms"] * 1e-3) / 1e9
@@ -409,13 +417,13 @@ def roofline_of(res, pk):
             "traffic": read_traffic_profile(f"decode_experts_{wl.name}")}
 
 
-def launches_per_step(wl) -> int:
+def launches_per_step(wl, w4a16=False) -> int:
     T = wl.T
     if wl.kind != "decode":
         # router, top-k, permute (hist, scan, scatter, first), tile rows, x
-        # encoding, gate/up GEMM, h encoding, down GEMM, shared gate/up + down,
-        # unpermute + combine
-        return 14
+        # encoding (W4A16: x gather), gate/up GEMM, h encoding (W4A4 only),
+        # down GEMM, shared gate/up + down, unpermute + combine
+        return 13 if w4a16 else 14
     # router, top-k + plan (one launch up to 8 tokens at E <= 320, else top-k
     # and the permute), expert gate/up, expert down, combine, and the shared
     # expert's two GEMVs on the auxiliary stream
@@ -472,9 +480,10 @@ def run_ours(args, rank, world, local_rank):
     pk = peaks()
     T, H = wl.T, wl.H
     prefill = res["prefill"]
-    path_name = ("prefill grouped GEMM (W4A4, tcgen05 block-scaled FP4)" if prefill else
+    path_name = (("prefill grouped GEMM (W4A16, tcgen05 kind::f16)" if res["w4a16"] else
+                  "prefill grouped GEMM (W4A4, tcgen05 block-scaled FP4)") if prefill else
                  "decode, single-token tensor-core expert kernels (W4A16)" if decode_t1_fused(wl) else "decode GEMV (W4A16)")
-    n_launch = launches_per_step(wl)
+    n_launch = launches_per_step(wl, res["w4a16"])
     out = {
         "metric": METRIC,
         "value": round(world * T / (ms_max * 1e-3), 2),
@@ -486,7 +495,8 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": ("nvfp4 weights x nvfp4 activations (tcgen05 mxf4nvf4), fp32 accumulate" if prefill
+        "dtype": (("nvfp4 weights x f16 activations (tcgen05 kind::f16), fp32 accumulate" if res["w4a16"] else
+                   "nvfp4 weights x nvfp4 activations (tcgen05 mxf4nvf4), fp32 accumulate") if prefill
                   else "nvfp4 weights x bf16 activations, exact products, fp32 accumulate"),
         "data": "synthetic (seeded; NVFP4 experts drawn in the code domain)",
         "config": {"workload": wl.name, "T": T, "hidden": H, "experts": wl.E, "intermediate": wl.I, "top_k": wl.k,
@@ -516,7 +526,7 @@ def run_ours(args, rank, world, local_rank):
                     "h2d_bytes_per_step": pwl.T * pwl.H * 2, "d2h_bytes_per_step": pwl.T * pwl.H * 2,
                     "ms_per_step": round(pre_e2e, 5)},
             "stages_ms_all_events": {n: round(float(v), 5) for n, v in zip(capi.STAGES, pre["stage_avg"])},
-            "gpu_launches": 2 * launches_per_step(pwl) * args.steps,
+            "gpu_launches": 2 * launches_per_step(pwl, pre["w4a16"]) * args.steps,
             "note": "timed in the same process and under the same clock record as the decode line, after it",
         }
         out["gpu_launches"] += out["prefill"]["gpu_launches"]
@@ -635,6 +645,9 @@ def main():
     ap.add_argument("--workload", default="decode_t1")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--prefill-path", default="w4a4", choices=["w4a4", "w4a16"],
+                    help="prefill expert numerics: NVFP4 activations on the block-scaled FP4 tensor cores (w4a4) "
+                         "or 16-bit activations on kind::f16 (w4a16)")
     ap.add_argument("--with-prefill", default="prefill_t4096",
                     help="after a decode workload, also time this prefill workload in the same run ('' = off)")
     args = ap.parse_args()

@@ -11,10 +11,11 @@
 //            r and the shared row.
 //
 // One CTA of 16 warps per SM. Each warp streams its weight rows straight into
-// registers with coalesced 128-bit loads (about 9 KB per warp in flight, 144
-// KB per SM), no shared-memory staging of weights, and multiplies them on the
-// tensor cores with mma.sync m16n8k16 (f16 operands, fp32 accumulators). The
-// down kernel issues the loads of its first tile before it waits for h.
+// registers with coalesced 128-bit loads (a warp reads 512 contiguous bytes of
+// a row per load; about 8 KB per warp in flight), no shared-memory staging of
+// weights, and multiplies them on the tensor cores with mma.sync m16n8k16
+// (f16 operands, fp32 accumulators). Gate/up also asks L2 for the down
+// kernel's tiles; the down kernel loads its first tile before it waits for h.
 //
 // Arithmetic. Weights are the A operand: each E2M1 code is decoded to f16 by
 // the hardware cvt and multiplied (f16) by its block's E4M3 scale; the product
@@ -24,18 +25,17 @@
 // core's fp32 accumulation, so only the fp32 sums round; the power of two and
 // the tensor scale are applied to the fp32 totals.
 //
-// Layouts. A dot product does not depend on the order of its terms; the
-// kernels only choose which weights meet which activations in one mma.
-//   gate/up: an mma's 16 A rows are (row 0 of the pair, K octant g) and
-//     (row 1, octant g) for g = 0..7, and B column n holds x's octant n, so
-//     the diagonal D[g][g] (and D[g + 8][g]) is octant g's partial dot
-//     product of each row; a warp sum over the eight octants finishes it. Lane
-//     (g, t) reads 16 contiguous bytes of each row per step.
-//   down: an mma's 16 A rows are 16 consecutive weight rows over the same 16
-//     k positions and B column 0 holds h (the other columns are zero); lane
-//     (g, t) holds rows g and g + 8.
-// In both, the 16 k-slots of lane (g, t) hold four consecutive codes of the
-// 32 it loaded, and B holds the activation at the same positions.
+// Layout. A dot product does not depend on the order of its terms; the
+// kernels only choose which weights meet which activations in one mma. Both
+// work on pairs of weight rows: an mma's 16 A rows are (row 0 of the pair,
+// octant g) and (row 1, octant g) for g = 0..7, where octant g of a row is
+// its 128-code chunks g, g + 8, g + 16, ...; B column n holds the activation's
+// octant n. The diagonal D[g][g] (and D[g + 8][g]) is then octant g's partial
+// dot product of each row, and the sum over the eight octants finishes it.
+// Lane (g, t) holds, per step, the 16 bytes of chunk 8 c + g at 16 t of each
+// row, so a warp load covers 512 contiguous bytes; its 16 k-slots per mma
+// hold four consecutive codes of those 32, and B holds the activation at the
+// same positions.
 
 #include "common.cuh"
 #include "gemv_common.cuh"
@@ -48,7 +48,6 @@ namespace {
 constexpr int kMaxLive = 16;               // top-k <= 16
 constexpr int kWarps = 16;                 // warps per CTA, one CTA per SM
 constexpr int kThreads = kWarps * kWarp;
-constexpr int kDnBatch = 8;                // down: 128-code chunks held in registers at a time
 
 RNX_DEVICE uint32_t e4m3x2_to_f16x2(uint16_t s) {
   uint32_t h;
@@ -147,14 +146,84 @@ RNX_DEVICE void load_live(const DecodeT1Args& p, const float* ts0, const float* 
   __syncthreads();
 }
 
+// Row-pair loads and products (both kernels). Rows r and r + 1 of a bank
+// with K codes per row; octant g of a row = its 128-code chunks g, g + 8,
+// g + 16, ...; step c covers chunks 8 c .. 8 c + 7, so lane (g, t) reads the
+// 16 bytes at 64 (8 c + g) + 16 t and a warp reads 512 contiguous bytes of a
+// row per step (its scales: 64 contiguous bytes). Chunks past K / 128 read
+// as zero.
+RNX_DEVICE void pair_load(const nvfp4_bank_t& bk, size_t r, int K, int c, int g, int t, uint4 (&q)[2], uint32_t& sc) {
+  const bool on = 8 * c + g < K / 128;
+  const uint8_t* cp = bk.codes + r * (K / 2) + 64 * (8 * c + g) + 16 * t;
+  q[0] = on ? ldg_stream(cp) : make_uint4(0u, 0u, 0u, 0u);
+  q[1] = on ? ldg_stream(cp + K / 2) : make_uint4(0u, 0u, 0u, 0u);
+  const uint8_t* sp = bk.scales + r * (K / 16) + 8 * (8 * c + g) + 2 * t;
+  sc = on ? (uint32_t)ldg_u16(sp) | ((uint32_t)ldg_u16(sp + K / 16) << 16) : 0u;
+}
+
+// The 8 mma of one step: A rows g = (row 0, octant g), g + 8 = (row 1,
+// octant g); bj = the step's B fragments at this lane (entry 32 i).
+RNX_DEVICE void pair_mma(const uint4 (&q)[2], uint32_t sc, const uint2* bj, float (&acc)[2][4]) {
+  const uint32_t s0 = e4m3x2_to_f16x2((uint16_t)(sc & 0xFFFFu)), s1 = e4m3x2_to_f16x2((uint16_t)(sc >> 16));
+  const uint32_t s0a = lo_lo(s0), s0b = hi_hi(s0), s1a = lo_lo(s1), s1b = hi_hi(s1);
+#define RNX_PAIR_STEP(II) \
+  mma_step<II>(acc[(II) & 1], q[0], q[1], (II) < 4 ? s0a : s0b, (II) < 4 ? s1a : s1b, bj[(II) * 32]);
+  RNX_PAIR_STEP(0) RNX_PAIR_STEP(1) RNX_PAIR_STEP(2) RNX_PAIR_STEP(3)
+  RNX_PAIR_STEP(4) RNX_PAIR_STEP(5) RNX_PAIR_STEP(6) RNX_PAIR_STEP(7)
+#undef RNX_PAIR_STEP
+}
+
+// The same with one accumulation chain.
+RNX_DEVICE void pair_mma1(const uint4 (&q)[2], uint32_t sc, const uint2* bj, float (&acc)[4]) {
+  const uint32_t s0 = e4m3x2_to_f16x2((uint16_t)(sc & 0xFFFFu)), s1 = e4m3x2_to_f16x2((uint16_t)(sc >> 16));
+  const uint32_t s0a = lo_lo(s0), s0b = hi_hi(s0), s1a = lo_lo(s1), s1b = hi_hi(s1);
+#define RNX_PAIR_STEP(II) mma_step<II>(acc, q[0], q[1], (II) < 4 ? s0a : s0b, (II) < 4 ? s1a : s1b, bj[(II) * 32]);
+  RNX_PAIR_STEP(0) RNX_PAIR_STEP(1) RNX_PAIR_STEP(2) RNX_PAIR_STEP(3)
+  RNX_PAIR_STEP(4) RNX_PAIR_STEP(5) RNX_PAIR_STEP(6) RNX_PAIR_STEP(7)
+#undef RNX_PAIR_STEP
+}
+RNX_DEVICE void pair_diag1(const float (&acc)[4], int g, int t, float* red) {
+  if (t == (g >> 1)) {
+    red[g] = (g & 1) ? acc[1] : acc[0];
+    red[8 + g] = (g & 1) ? acc[3] : acc[2];
+  }
+}
+
+// The diagonal of a pair's accumulator: octant g of row 0 is D[g][g], of row
+// 1 D[g + 8][g], in lane (g, g / 2), element g % 2. Writes them to red[0..8)
+// (row 0) and red[8..16) (row 1), indexed by octant.
+RNX_DEVICE void pair_diag(const float (&acc)[2][4], int g, int t, float* red) {
+  if (t == (g >> 1)) {
+    red[g] = (g & 1) ? acc[0][1] + acc[1][1] : acc[0][0] + acc[1][0];
+    red[8 + g] = (g & 1) ? acc[0][3] + acc[1][3] : acc[0][2] + acc[1][2];
+  }
+}
+RNX_DEVICE float octant_sum(const float* v) {
+  return ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
+}
+
+// B fragments of a K-element activation row a (scaled by up, rounded to f16)
+// in the order of pair_mma: entry (c * 8 + i) * 32 + lane =
+// a[128 (8 c + n) + 32 t + 4 i + 0..3] with n = lane / 4, t = lane % 4 (zeros
+// past K).
+RNX_DEVICE uint2 b_frag_f16(float4 v, float up) {
+  __half2 h0 = __floats2half2_rn(v.x * up, v.y * up), h1 = __floats2half2_rn(v.z * up, v.w * up);
+  return make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
+}
+RNX_DEVICE int b_frag_pos(int f) {    // element index of entry f (4 consecutive elements)
+  const int ln = f & 31, i = (f >> 5) & 7, c = f >> 8;
+  return 128 * (8 * c + (ln >> 2)) + 32 * (ln & 3) + 4 * i;
+}
+
 // ============================================================== gate/up
 //
 // Item = a pair of rows (2 rp, 2 rp + 1) of one live expert's gate and up
-// matrices, full K; one warp per item at a time. NCH = H / 1024 steps of
-// 128 codes per octant, taken 4 at a time into registers.
+// matrices, full K; one warp per item at a time. NCH = H / 1024 steps, taken
+// 4 at a time into registers.
 
 __global__ void __launch_bounds__(kThreads, 1) t1_gate_up_kernel(const DecodeT1Args p) {
   __shared__ __align__(16) uint2 xs[8192 / 4];      // x as B fragments, H <= 8192
+  __shared__ float s_red[kWarps][2][16];
   __shared__ int s_live[1 + 2 * kMaxLive];
   __shared__ int s_tmp[4 * kMaxLive];
   __shared__ float s_ts[2 * kMaxLive];
@@ -167,31 +236,52 @@ __global__ void __launch_bounds__(kThreads, 1) t1_gate_up_kernel(const DecodeT1A
   const int n_live = s_live[0];
   const int N = n_live * (I / 2), GW = gridDim.x * kWarps;
   const int first = blockIdx.x * kWarps + warp;
-  auto rows = [&](int i, int& u, size_t& r0) {
+  auto rows = [&](int i, int& u) {
     u = i / (I / 2);
-    r0 = (size_t)s_live[1 + u] * I + 2 * (size_t)(i - u * (I / 2));
+    return (size_t)s_live[1 + u] * I + 2 * (size_t)(i - u * (I / 2));
   };
-  // x as B fragments: entry ((c * 8 + i) * 32 + lane') = x[n H/8 + 128 c + 32 t' + 4 i + 0..3],
-  // n = lane' / 4 (octant), t' = lane' % 4
+  if (first < N) {            // the first item into L2 while x is staged
+    int u;
+    const size_t r0 = rows(first, u);
+    for (int o = lane * 128; o < H; o += 32 * 128) {
+      prefetch_l2(p.gate.codes + r0 * (H / 2) + o);
+      prefetch_l2(p.up.codes + r0 * (H / 2) + o);
+    }
+    if (lane * 128 < H / 8) {
+      prefetch_l2(p.gate.scales + r0 * (H / 16) + lane * 128);
+      prefetch_l2(p.up.scales + r0 * (H / 16) + lane * 128);
+    }
+  }
   float up, unscale;
   prescale15(__uint_as_float(*p.xmax), up, unscale);
   for (int f = threadIdx.x; f < H / 4; f += kThreads) {
-    const int ln = f & 31, i = (f >> 5) & 7, c = f >> 8;
-    const uint2 v = *reinterpret_cast<const uint2*>(p.x + (ln >> 2) * (H / 8) + 128 * c + 32 * (ln & 3) + 4 * i);
+    const uint2 v = *reinterpret_cast<const uint2*>(p.x + b_frag_pos(f));
     const float2 a = bf16x2_to_f32x2(v.x), b = bf16x2_to_f32x2(v.y);
-    __half2 h0 = __floats2half2_rn(a.x * up, a.y * up), h1 = __floats2half2_rn(b.x * up, b.y * up);
-    xs[f] = make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
+    xs[f] = b_frag_f16(make_float4(a.x, a.y, b.x, b.y), up);
   }
   __syncthreads();
 
-  // Ask L2 for every weight byte this CTA's warps will read, then for a share
-  // of the down kernel's tiles (all of the step's expert bytes fit in L2): the
-  // memory system streams from DRAM without gaps while the warps compute from
-  // L2. x was staged first so that its loads did not queue behind these.
-  for (int i = first; i < N; i += GW) {
+  uint4 qg[4][2], qu[4][2];  // [step][row] of the gate and up rows
+  uint32_t sg[4], su[4];
+  auto load4 = [&](size_t r0, int c0) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (c0 + j < NCH) {
+        pair_load(p.gate, r0, H, c0 + j, g, t, qg[j], sg[j]);
+        pair_load(p.up, r0, H, c0 + j, g, t, qu[j], su[j]);
+      }
+    }
+  };
+  if (first < N) {
     int u;
-    size_t r0;
-    rows(i, u, r0);
+    load4(rows(first, u), 0);
+  }
+  // Ask L2 for this warp's later items and for a share of the down kernel's
+  // tiles (all of the step's expert bytes fit in L2), after the first item's
+  // own loads went out.
+  for (int i = first + GW; i < N; i += GW) {
+    int u;
+    const size_t r0 = rows(i, u);
     for (int o = lane * 128; o < H; o += 32 * 128) {          // 2 rows x H/2 code bytes per matrix
       prefetch_l2(p.gate.codes + r0 * (H / 2) + o);
       prefetch_l2(p.up.codes + r0 * (H / 2) + o);
@@ -213,81 +303,38 @@ __global__ void __launch_bounds__(kThreads, 1) t1_gate_up_kernel(const DecodeT1A
 
   for (int i = first; i < N; i += GW) {
     int u;
-    size_t r0;
-    rows(i, u, r0);
-    float acc[2][2][4];      // [matrix][chain][fragment]
+    const size_t r0 = rows(i, u);
+    float ag[2][4], au[2][4];
 #pragma unroll
-    for (int m = 0; m < 2; ++m)
+    for (int j = 0; j < 2; ++j)
 #pragma unroll
-      for (int j = 0; j < 2; ++j)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[m][j][q] = 0.f;
+      for (int q = 0; q < 4; ++q) ag[j][q] = au[j][q] = 0.f;
     for (int c0 = 0; c0 < NCH; c0 += 4) {
-      // this lane's 16 bytes of each row at octant g, steps c0 .. c0 + 3
-      uint4 q[2][2][4];        // [matrix][row][step]
-      uint32_t sc[2][4];       // [matrix][step]: row 0's scale pair, row 1's in the high half
-#pragma unroll
-      for (int m = 0; m < 2; ++m) {
-        const nvfp4_bank_t& bk = m ? p.up : p.gate;
-        const uint8_t* sp = bk.scales + r0 * (H / 16) + g * (H / 128) + 2 * t;
-#pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {
-          const uint8_t* cp = bk.codes + (r0 + rr) * (H / 2) + g * (H / 16) + 16 * t;
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            q[m][rr][j] = c0 + j < NCH ? ldg_stream(cp + 64 * (c0 + j)) : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          sc[m][j] = c0 + j < NCH ? (uint32_t)ldg_u16(sp + 8 * (c0 + j)) |
-                                        ((uint32_t)ldg_u16(sp + H / 16 + 8 * (c0 + j)) << 16)
-                                  : 0u;
-      }
+      if (c0 > 0) load4(r0, c0);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         if (c0 + j < NCH) {
-          uint32_t z[2][4];      // per matrix: row 0 block 2t, 2t + 1, row 1 block 2t, 2t + 1 (f16x2 broadcast)
-#pragma unroll
-          for (int m = 0; m < 2; ++m) {
-            const uint32_t s0 = e4m3x2_to_f16x2((uint16_t)(sc[m][j] & 0xFFFFu)),
-                           s1 = e4m3x2_to_f16x2((uint16_t)(sc[m][j] >> 16));
-            z[m][0] = lo_lo(s0);
-            z[m][1] = hi_hi(s0);
-            z[m][2] = lo_lo(s1);
-            z[m][3] = hi_hi(s1);
-          }
-          const uint2* bj = xs + (c0 + j) * 8 * 32 + lane;
-#define RNX_GU_STEP(II)                                                                                    \
-  {                                                                                                         \
-    const uint2 b = bj[(II) * 32];                                                                          \
-    mma_step<II>(acc[0][(II) & 1], q[0][0][j], q[0][1][j], z[0][(II) < 4 ? 0 : 1], z[0][(II) < 4 ? 2 : 3], b); \
-    mma_step<II>(acc[1][(II) & 1], q[1][0][j], q[1][1][j], z[1][(II) < 4 ? 0 : 1], z[1][(II) < 4 ? 2 : 3], b); \
-  }
-          RNX_GU_STEP(0) RNX_GU_STEP(1) RNX_GU_STEP(2) RNX_GU_STEP(3)
-          RNX_GU_STEP(4) RNX_GU_STEP(5) RNX_GU_STEP(6) RNX_GU_STEP(7)
-#undef RNX_GU_STEP
+          const uint2* bj = xs + (c0 + j) * 256 + lane;
+          pair_mma(qg[j], sg[j], bj, ag);
+          pair_mma(qu[j], su[j], bj, au);
         }
       }
     }
-    // the diagonal: octant g of row 0 is D[g][g], of row 1 D[g + 8][g], in
-    // lane (g, g / 2), element g % 2; then the sum over the eight octants
-    float v[2][2];
-#pragma unroll
-    for (int m = 0; m < 2; ++m) {
-      float d[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) d[q] = acc[m][0][q] + acc[m][1][q];
-      const bool mine = t == (g >> 1);
-      v[m][0] = warp_sum(mine ? ((g & 1) ? d[1] : d[0]) : 0.f);
-      v[m][1] = warp_sum(mine ? ((g & 1) ? d[3] : d[2]) : 0.f);
+    if (i + GW < N) {
+      int u2;
+      load4(rows(i + GW, u2), 0);        // the next item's first steps (L2) while this one finishes
     }
-    if (lane == 0) {
-      const float sg = unscale * s_ts[u], su = unscale * s_ts[kMaxLive + u];
-      const float2 hv = make_float2(clamped_swiglu(v[0][0] * sg, v[1][0] * su, p.limit),
-                                    clamped_swiglu(v[0][1] * sg, v[1][1] * su, p.limit));
+    float* red = &s_red[warp][0][0];
+    pair_diag(ag, g, t, red);
+    pair_diag(au, g, t, red + 16);
+    __syncwarp();
+    if (lane < 2) {
+      const float gs = octant_sum(red + 8 * lane) * unscale * s_ts[u];
+      const float us = octant_sum(red + 16 + 8 * lane) * unscale * s_ts[kMaxLive + u];
       const size_t a = (size_t)s_live[1 + kMaxLive + u];
-      *reinterpret_cast<float2*>(p.h + a * I + (r0 - (size_t)s_live[1 + u] * I)) = hv;
+      p.h[a * I + (r0 - (size_t)s_live[1 + u] * I) + lane] = clamped_swiglu(gs, us, p.limit);
     }
+    __syncwarp();
   }
 
   // h rows of assignments that are not live (remote experts, dropped ids)
@@ -303,111 +350,78 @@ __global__ void __launch_bounds__(kThreads, 1) t1_gate_up_kernel(const DecodeT1A
 
 // ============================================================== down
 //
-// Item = a 16-row tile of one live expert's down matrix, full K (I / 128
-// chunks, kDnBatch at a time in registers); one warp per item at a time.
+// Item = a 16-row tile (8 row pairs) of one live expert's down matrix, full
+// K = I in NCD = ceil(I / 1024) steps, one step of all 8 pairs in
+// registers at a time; one warp per item at a time.
 
-struct DnTile {
-  uint4 q[2][kDnBatch];      // rows g and g + 8, chunk c0 + j, this lane's 16 bytes
-  uint32_t sc[kDnBatch];     // their E4M3 scale pairs: row g's, row g + 8's in the high half
-};
+constexpr int kHq = 4;           // B-fragment entries of h per thread held in registers while staging
 
-RNX_DEVICE void dn_load(const DecodeT1Args& p, size_t row0, int c0, int nch, int g, int t, DnTile& T) {
-  const int I = p.I;
-#pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
-    const uint8_t* cp = p.down.codes + (row0 + g + 8 * rr) * (I / 2) + 16 * t;
-#pragma unroll
-    for (int j = 0; j < kDnBatch; ++j) T.q[rr][j] = c0 + j < nch ? ldg_stream(cp + 64 * (c0 + j)) : make_uint4(0u, 0u, 0u, 0u);
-  }
-  const uint8_t* sp = p.down.scales + (row0 + g) * (I / 16) + 2 * t;
-#pragma unroll
-  for (int j = 0; j < kDnBatch; ++j)
-    T.sc[j] = c0 + j < nch ? (uint32_t)ldg_u16(sp + 8 * (c0 + j)) | ((uint32_t)ldg_u16(sp + 8 * (I / 16) + 8 * (c0 + j)) << 16)
-                           : 0u;
-}
-
-RNX_DEVICE void dn_mma(const DnTile& T, int c0, int nch, const uint2* bf, bool b_on, int t, float (&acc)[4][4]) {
-#pragma unroll
-  for (int j = 0; j < kDnBatch; ++j) {
-    if (c0 + j < nch) {
-      const uint32_t s0 = e4m3x2_to_f16x2((uint16_t)(T.sc[j] & 0xFFFFu)), s1 = e4m3x2_to_f16x2((uint16_t)(T.sc[j] >> 16));
-      const uint32_t s0a = lo_lo(s0), s0b = hi_hi(s0), s1a = lo_lo(s1), s1b = hi_hi(s1);
-      const uint2* bj = bf + (c0 + j) * 8 * 4 + t;
-#define RNX_DN_STEP(II)                                                                                        \
-  mma_step<II>(acc[(II) & 3], T.q[0][j], T.q[1][j], (II) < 4 ? s0a : s0b, (II) < 4 ? s1a : s1b,                \
-               b_on ? bj[(II) * 4] : make_uint2(0u, 0u));
-      RNX_DN_STEP(0) RNX_DN_STEP(1) RNX_DN_STEP(2) RNX_DN_STEP(3)
-      RNX_DN_STEP(4) RNX_DN_STEP(5) RNX_DN_STEP(6) RNX_DN_STEP(7)
-#undef RNX_DN_STEP
-    }
-  }
-}
-
-constexpr int kHq = 8;           // float4 of h per thread held in registers while staging
-
+// ONE_STEP: I <= 1024, every pair's K in one step (its diagonal taken right
+// after its 8 mma); else I = 2048, two steps, the tile in two halves of four
+// pairs.
+template <bool ONE_STEP>
 __global__ void __launch_bounds__(kThreads, 1) t1_down_kernel(const DecodeT1Args p) {
-  extern __shared__ __align__(16) uint2 hs[];               // h as B fragments: k x I f16
+  extern __shared__ __align__(16) uint2 hs[];               // h as B fragments: k x NCD x 256
+  __shared__ float s_red[kWarps][8][16];
   __shared__ float s_up[kMaxLive], s_sc[kMaxLive];
   __shared__ uint32_t s_max[kMaxLive];
   __shared__ int s_live[1 + 2 * kMaxLive];
   __shared__ int s_tmp[4 * kMaxLive];
   __shared__ float s_ts[2 * kMaxLive];
-  const int H = p.H, I = p.I, k = p.k, NCH = I / 128;
+  const int H = p.H, I = p.I, k = p.k, NCD = (I + 1023) / 1024, FPE = NCD * 256;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
 
-  // The plan comes from two launches back, complete when this grid starts:
-  // the first tile's weights are loaded before the wait for h.
+  // The plan comes from two launches back, complete when this grid starts.
+  // The weights were requested into L2 by the gate/up launch: h is staged
+  // first (its loads would otherwise queue behind the weight loads).
   load_live(p, p.down.tensor_scale, nullptr, s_tmp, s_live, s_ts);
   const int n_live = s_live[0];
   const int TPE = H / 16, N = n_live * TPE, GW = gridDim.x * kWarps;
   int i = blockIdx.x * kWarps + warp;
-  DnTile T;
+  uint4 q[8][2];
+  uint32_t sc[8];
   auto row_of = [&](int it, int& u) {
     u = it / TPE;
     return (size_t)s_live[1 + u] * H + 16 * (size_t)(it - u * TPE);
   };
-  if (i < N) {
-    int u;
-    dn_load(p, row_of(i, u), 0, NCH, g, t, T);
-  }
   if (threadIdx.x < kMaxLive) s_max[threadIdx.x] = 0u;
   pdl_wait();                // h comes from the previous launch
   pdl_trigger();
 
-  // h rows of the live experts as B fragments: entry ((c * 8 + i) * 4 + t) =
-  // h[128 c + 32 t + 4 i + 0..3] times the row's power of two. The row maxima
-  // first (one shared atomic per warp and row: a warp's 32 consecutive float4
-  // lie in one row), then the conversion.
+  // h rows of the live experts as B fragments (b_frag_pos order) times the
+  // row's power of two: the row maxima first (one shared atomic per warp: a
+  // warp's 32 consecutive entries lie in one row), then the conversion.
   {
-    const int nq = n_live * (I / 4);
+    const int nq = n_live * FPE;
     const bool in_regs = nq <= kHq * kThreads;
     float4 v[kHq];
     auto load_h = [&](int f) {
-      const int u = f / (I / 4);
-      return *reinterpret_cast<const float4*>(p.h + (size_t)s_live[1 + kMaxLive + u] * I + 4 * (f - u * (I / 4)));
+      const int u = f / FPE, pos = b_frag_pos(f - u * FPE);
+      if (pos >= I) return make_float4(0.f, 0.f, 0.f, 0.f);
+      return *reinterpret_cast<const float4*>(p.h + (size_t)s_live[1 + kMaxLive + u] * I + pos);
     };
     auto amax4 = [](float4 a) { return fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))); };
     __syncthreads();
     if (in_regs) {
 #pragma unroll
-      for (int q = 0; q < kHq; ++q) {
-        const int f = threadIdx.x + q * kThreads;
-        v[q] = f < nq ? load_h(f) : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int qq = 0; qq < kHq; ++qq) {
+        const int f = threadIdx.x + qq * kThreads;
+        v[qq] = f < nq ? load_h(f) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
-    for (int q = 0; q * kThreads < nq; ++q) {
-      const int f = threadIdx.x + q * kThreads;             // warp-uniform: f < nq for all lanes or none
+    for (int qn = 0; qn * kThreads < nq; ++qn) {
+      const int f = threadIdx.x + qn * kThreads;            // warp-uniform: f < nq for all lanes or none
       if (f - lane < nq) {
         float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
         if (in_regs) {
 #pragma unroll
           for (int qq = 0; qq < kHq; ++qq)
-            if (qq == q) a = v[qq];
+            if (qq == qn) a = v[qq];
         } else {
           a = load_h(f);
         }
         const float m = warp_max(amax4(a));
-        if (lane == 0) atomicMax(&s_max[f / (I / 4)], __float_as_uint(m));   // non-negative floats order as integers
+        if (lane == 0) atomicMax(&s_max[f / FPE], __float_as_uint(m));   // non-negative floats order as integers
       }
     }
     __syncthreads();
@@ -418,51 +432,76 @@ __global__ void __launch_bounds__(kThreads, 1) t1_down_kernel(const DecodeT1Args
       s_sc[threadIdx.x] = us * s_ts[threadIdx.x] * p.weights[s_live[1 + kMaxLive + threadIdx.x]];
     }
     __syncthreads();
-    for (int q = 0; q * kThreads < nq; ++q) {
-      const int f = threadIdx.x + q * kThreads;
+    for (int qn = 0; qn * kThreads < nq; ++qn) {
+      const int f = threadIdx.x + qn * kThreads;
       if (f < nq) {
         float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
         if (in_regs) {
 #pragma unroll
           for (int qq = 0; qq < kHq; ++qq)
-            if (qq == q) a = v[qq];
+            if (qq == qn) a = v[qq];
         } else {
           a = load_h(f);
         }
-        const int u = f / (I / 4), pos = 4 * (f - u * (I / 4));
-        const float upx = s_up[u];
-        __half2 h0 = __floats2half2_rn(a.x * upx, a.y * upx), h1 = __floats2half2_rn(a.z * upx, a.w * upx);
-        hs[(size_t)u * (I / 4) + ((pos >> 7) * 8 + ((pos >> 2) & 7)) * 4 + ((pos >> 5) & 3)] =
-            make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
+        hs[f] = b_frag_f16(a, s_up[f / FPE]);
       }
     }
     __syncthreads();
   }
 
+  if (i < N) {
+    int u;
+    const size_t r0 = row_of(i, u);
+#pragma unroll
+    for (int pr = 0; pr < (ONE_STEP ? 8 : 4); ++pr) pair_load(p.down, r0 + 2 * pr, I, 0, g, t, q[pr], sc[pr]);
+  }
   for (; i < N; i += GW) {
     int u;
     const size_t row0 = row_of(i, u);
-    float acc[4][4];
+    const uint2* bf = hs + (size_t)u * FPE + lane;
+    float* red = &s_red[warp][0][0];
+    if (ONE_STEP) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+      for (int pr = 0; pr < 8; ++pr) {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        pair_mma1(q[pr], sc[pr], bf, acc);
+        pair_diag1(acc, g, t, red + 16 * pr);
+      }
+    } else {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) acc[j][q] = 0.f;
-    const uint2* bf = hs + (size_t)u * (I / 4);
-    for (int c0 = 0; c0 < NCH; c0 += kDnBatch) {
-      if (c0 > 0) dn_load(p, row0, c0, NCH, g, t, T);
-      dn_mma(T, c0, NCH, bf, lane < 4, t, acc);
-    }
-    if (t == 0) {
-      const float sc = s_sc[u];
-      const size_t a = (size_t)s_live[1 + kMaxLive + u];
-      float* rr = p.r + a * H + (row0 - (size_t)s_live[1 + u] * H);
-      rr[g] = ((acc[0][0] + acc[1][0]) + (acc[2][0] + acc[3][0])) * sc;
-      rr[g + 8] = ((acc[0][2] + acc[1][2]) + (acc[2][2] + acc[3][2])) * sc;
+      for (int half = 0; half < 2; ++half) {
+        float acc[4][4];
+#pragma unroll
+        for (int pr = 0; pr < 4; ++pr)
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq) acc[pr][qq] = 0.f;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          if (half > 0 || c > 0) {
+#pragma unroll
+            for (int pr = 0; pr < 4; ++pr) pair_load(p.down, row0 + 2 * (4 * half + pr), I, c, g, t, q[pr], sc[pr]);
+          }
+#pragma unroll
+          for (int pr = 0; pr < 4; ++pr) pair_mma1(q[pr], sc[pr], bf + c * 256, acc[pr]);
+        }
+#pragma unroll
+        for (int pr = 0; pr < 4; ++pr) pair_diag1(acc[pr], g, t, red + 16 * (4 * half + pr));
+      }
     }
     if (i + GW < N) {
       int u2;
-      dn_load(p, row_of(i + GW, u2), 0, NCH, g, t, T);
+      const size_t rn = row_of(i + GW, u2);
+#pragma unroll
+      for (int pr = 0; pr < (ONE_STEP ? 8 : 4); ++pr) pair_load(p.down, rn + 2 * pr, I, 0, g, t, q[pr], sc[pr]);
     }
+    __syncwarp();
+    if (lane < 16) {
+      // lane = 2 pair + row: output row row0 + lane; rows 0, 1 of pair pr at red[16 pr + 8 row]
+      const int pr = lane >> 1, rr = lane & 1;
+      const size_t a = (size_t)s_live[1 + kMaxLive + u];
+      p.r[a * H + (row0 - (size_t)s_live[1 + u] * H) + lane] = octant_sum(red + 16 * pr + 8 * rr) * s_sc[u];
+    }
+    __syncwarp();
   }
 
   // rows of assignments that are not live (remote experts, dropped ids) are
@@ -508,10 +547,11 @@ cudaError_t launch_decode_t1_gate_up(const DecodeT1Args& a, cudaStream_t st) {
 cudaError_t launch_decode_t1_down(const DecodeT1Args& a, cudaStream_t st) {
   if (!decode_t1_supported(a.H, a.I, a.E, a.k)) return cudaErrorInvalidValue;
   if (!aligned16(a.down.codes) || ((uintptr_t)a.down.scales & 1u) || !aligned16(a.h)) return cudaErrorInvalidValue;
-  const int smem = a.k * a.I * 2;
-  cudaError_t e = cudaFuncSetAttribute(t1_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const int smem = a.k * ((a.I + 1023) / 1024) * 256 * 8;
+  auto kern = a.I <= 1024 ? t1_down_kernel<true> : t1_down_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(t1_down_kernel, dim3(sm_count()), dim3(kThreads), (size_t)smem, st, a);
+  return launch_pdl(kern, dim3(sm_count()), dim3(kThreads), (size_t)smem, st, a);
 }
 
 }  // namespace rnx

@@ -393,7 +393,8 @@ def _t1(H, I, E, k, Is, **kw):
                         sigma_w=kw.pop("sigma_w", 0.0064 if H >= 2048 else 0.02), **kw)
 
 
-T1_SHAPES = [(1024, 128, 32, 4, 256), (3072, 768, 24, 6, 256), (1024, 512, 40, 16, 0), (8192, 2048, 12, 8, 512)]
+T1_SHAPES = [(1024, 128, 32, 4, 256), (3072, 768, 24, 6, 256), (1024, 512, 40, 16, 0), (2048, 1536, 20, 5, 128),
+             (8192, 2048, 12, 8, 512)]
 
 
 @pytest.mark.parametrize("H,I,E,k,Is", T1_SHAPES)
