@@ -158,11 +158,18 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ ours
 
-def decode_t1_fused(wl) -> bool:
-    """The single-token tensor-core expert kernels run for this workload;
-    mirrors the library's eligibility rule for T = 1."""
-    return (wl.kind == "decode" and wl.T == 1 and wl.H % 1024 == 0 and wl.H <= 8192 and wl.I % 128 == 0
-            and wl.I <= 2048 and wl.k <= 16 and wl.E <= 1024)
+def decode_mma(wl) -> bool:
+    """The tensor-core decode expert kernels run for this workload; mirrors
+    the library's eligibility rule (a handful of tokens, shapes that stage in
+    shared memory)."""
+    if wl.kind != "decode" or not (1 <= wl.T <= 8):
+        return False
+    if wl.H % 1024 or wl.H > 8192 or wl.I % 128 or wl.I > 2048 or wl.k > 16 or wl.E > 1024 or wl.T * wl.k > 128:
+        return False
+    budget = 200 * 1024
+    gu = ((wl.T * (wl.H + 8) * 2 + 15) // 16) * 16 + 2 * 4 * 4 * 256 * 4
+    dn = wl.T * wl.k * (wl.I + 8) * 2
+    return gu <= budget and dn <= budget
 
 
 def measure(wl, args, rank, world, local_rank, dev, clocks=None):
@@ -405,8 +412,8 @@ def roofline_of(res, pk):
                 "algorithmic_flops_per_step": flops, "unique_experts_per_step": res["U"],
                 "traffic": read_traffic_profile(f"{stem}_{wl.name}")}
     routed = res["U"] * expert_bytes(wl)
-    if decode_t1_fused(wl):
-        kernel = "t1_gate_up_kernel + t1_down_kernel (128-bit weight loads, mma.sync m16n8k16; timed together)"
+    if decode_mma(wl):
+        kernel = "mma_gate_up_kernel + mma_down_kernel (128-bit weight loads, mma.sync m16n8k16; timed together)"
     else:
         kernel = "nvfp4_expert_gemv (gate/up + down launches, timed together)"
     achieved = routed / (res["kern_ms"] * 1e-3) / 1e9
@@ -482,7 +489,7 @@ def run_ours(args, rank, world, local_rank):
     prefill = res["prefill"]
     path_name = (("prefill grouped GEMM (W4A16, tcgen05 kind::f16)" if res["w4a16"] else
                   "prefill grouped GEMM (W4A4, tcgen05 block-scaled FP4)") if prefill else
-                 "decode, single-token tensor-core expert kernels (W4A16)" if decode_t1_fused(wl) else "decode GEMV (W4A16)")
+                 "decode, tensor-core expert kernels (W4A16)" if decode_mma(wl) else "decode GEMV (W4A16)")
     n_launch = launches_per_step(wl, res["w4a16"])
     out = {
         "metric": METRIC,

@@ -629,23 +629,24 @@ moe_status_t nvfp4_expert_gemv(const moe_config_t* cfg, int32_t proj, const void
   uint32_t* status = (uint32_t*)(b + L.status);
   RNX_CUDA(cudaMemsetAsync(status, 0, kCtrlBytes, st), "clear status");
   const int H = cfg->hidden, I = cfg->intermediate, k = cfg->top_k;
-  if (T == 1 && rnx::decode_t1_supported(H, I, cfg->num_experts, k)) {
-    // one token: the tensor-core single-token kernels, fed from the plan
-    rnx::DecodeT1Args a{};
-    a.H = H; a.I = I; a.E = cfg->num_experts; a.k = k;
+  if (rnx::decode_mma_supported(T, H, I, cfg->num_experts, k) && aligned16(act)) {
+    // a handful of tokens: the tensor-core decode kernels, fed from the plan
+    RNX_PTR(plan->counts, "plan.counts");
+    rnx::DecodeMmaArgs a{};
+    a.T = T; a.H = H; a.I = I; a.E = cfg->num_experts; a.k = k;
     a.lb = cfg->local_begin; a.le = cfg->local_end;
     a.limit = cfg->swiglu_limit;
     a.gate = w->gate; a.up = w->up; a.down = w->down;
-    a.active = plan->active; a.first = plan->first;
+    a.active = plan->active; a.counts = plan->counts; a.offsets = plan->offsets; a.sorted = plan->sorted;
     a.status = status;
     if (proj == MOE_PROJ_GATE_UP) {
       uint32_t* xmax = (uint32_t*)(b + L.xmax);
-      RNX_CUDA(rnx::launch_row_absmax((const uint16_t*)act, 1, H, xmax, st), "activation row max");
+      RNX_CUDA(rnx::launch_row_absmax((const uint16_t*)act, T, H, xmax, st), "activation row max");
       a.x = (const uint16_t*)act; a.xmax = xmax; a.h = out;
-      RNX_CUDA(rnx::launch_decode_t1_gate_up(a, st), "nvfp4_expert_gemv (gate/up)");
+      RNX_CUDA(rnx::launch_decode_mma_gate_up(a, st), "nvfp4_expert_gemv (gate/up)");
     } else {
       a.h = (float*)act; a.weights = weights; a.r = out;
-      RNX_CUDA(rnx::launch_decode_t1_down(a, st), "nvfp4_expert_gemv (down)");
+      RNX_CUDA(rnx::launch_decode_mma_down(a, st), "nvfp4_expert_gemv (down)");
     }
     return MOE_OK;
   }
@@ -788,10 +789,10 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
              "shared expert");
     RNX_CUDA(cudaEventRecord(side->join, side->st), "join event");
   }
-  // one token: the tensor-core expert kernels (one CTA per SM, weight tiles
-  // through a TMA ring), fed from the routing plan; the router's GEMV also
-  // leaves max |x| for their f16 pre-scale
-  const bool t1 = decode && T == 1 && rnx::decode_t1_supported(H, I, E, k);
+  // a handful of tokens: the tensor-core expert kernels (one CTA per SM,
+  // weight rows streamed into registers), fed from the routing plan; the
+  // router's GEMV also leaves max |x_t| for their f16 pre-scale
+  const bool t1 = decode && rnx::decode_mma_supported(T, H, I, E, k) && aligned16(x);
   uint32_t* xmax = (uint32_t*)(b + L.xmax);
   RNX_CUDA(mark(MOE_STAGE_ROUTER_LOGITS, st), "stage event");
   if (!decode && router_on_tensor_cores(cfg, T, w)) {
@@ -887,21 +888,20 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
     a.gate = w->gate; a.up = w->up; a.down = w->down;
     a.status = status;
     if (t1) {
-      rnx::DecodeT1Args d{};
-      d.H = H; d.I = I; d.E = E; d.k = k;
+      rnx::DecodeMmaArgs d{};
+      d.T = T; d.H = H; d.I = I; d.E = E; d.k = k;
       d.lb = cfg->local_begin; d.le = cfg->local_end;
       d.limit = cfg->swiglu_limit;
       d.x = x;
       d.gate = w->gate; d.up = w->up; d.down = w->down;
-      d.active = plan.active; d.first = plan.first;
+      d.active = plan.active; d.counts = plan.counts; d.offsets = plan.offsets; d.sorted = plan.sorted;
       d.weights = wts; d.xmax = xmax; d.h = h; d.r = r;
-      d.l2_down = 1;
       d.status = status;
       RNX_CUDA(mark(MOE_STAGE_EXPERT_GATE_UP, st), "stage event");
-      RNX_CUDA(rnx::launch_decode_t1_gate_up(d, st), "expert gate/up");
+      RNX_CUDA(rnx::launch_decode_mma_gate_up(d, st), "expert gate/up");
       RNX_CUDA(mark(MOE_STAGE_H_QUANT, st), "stage event");
       RNX_CUDA(mark(MOE_STAGE_EXPERT_DOWN, st), "stage event");
-      RNX_CUDA(rnx::launch_decode_t1_down(d, st), "expert down");
+      RNX_CUDA(rnx::launch_decode_mma_down(d, st), "expert down");
     } else {
       a.proj = MOE_PROJ_GATE_UP; a.act = x; a.out = h;
       RNX_CUDA(mark(MOE_STAGE_EXPERT_GATE_UP, st), "stage event");

@@ -46,29 +46,31 @@ struct ExpertGemvArgs {
 
 cudaError_t launch_nvfp4_gemv(const ExpertGemvArgs& a, cudaStream_t st);
 
-// Single-token expert projections on the tensor cores (decode_t1.cu), from
-// the routing plan: gate/up writes h (clamped SwiGLU of the live experts'
-// gate and up projections; zero rows for the other assignments), down writes
-// the weighted rows r.
-struct DecodeT1Args {
-  int H, I, E, k, lb, le;
+// Decode expert projections for a handful of tokens on the tensor cores
+// (decode_mma.cu), from the routing plan: gate/up writes h (clamped SwiGLU of
+// the live experts' gate and up projections; zero rows for the other
+// assignments), down writes the weighted rows r (zero rows likewise).
+struct DecodeMmaArgs {
+  int T, H, I, E, k, lb, le;
   float limit;
-  const uint16_t* x;                 // bf16 [H]
+  const uint16_t* x;                 // bf16 [T, H], 16-byte aligned
   nvfp4_bank_t gate, up, down;
   const int32_t* active;             // routing plan: active local experts (count first)
-  const int32_t* first;              // routing plan: the assignment of each active expert
-  const float* weights;              // [k] routing weights
-  const uint32_t* xmax;              // max |x| (fp32 bits)
-  float* h;                          // fp32 [k, I]
-  float* r;                          // fp32 [k, H] weighted routed rows
+  const int32_t* counts;             // routing plan: assignments per expert
+  const int32_t* offsets;            // routing plan: first entry of each expert in sorted
+  const int32_t* sorted;             // routing plan: assignments grouped by expert
+  const float* weights;              // [T*k] routing weights
+  const uint32_t* xmax;              // [T] max |x_t| (fp32 bits)
+  float* h;                          // fp32 [T*k, I]
+  float* r;                          // fp32 [T*k, H] weighted routed rows
   uint32_t* status;
-  int l2_down;                       // gate/up also asks L2 for the down tiles the down kernel reads next
 };
-// H a multiple of 1024 up to 8192, I a multiple of 128 up to 2048, k <= 16,
-// E <= 1024.
-bool decode_t1_supported(int H, int I, int E, int k);
-cudaError_t launch_decode_t1_gate_up(const DecodeT1Args& p, cudaStream_t st);
-cudaError_t launch_decode_t1_down(const DecodeT1Args& p, cudaStream_t st);
+// 1 <= T <= 8, H a multiple of 1024 up to 8192, I a multiple of 128 up to
+// 2048, k <= 16, T*k <= 128, E <= 1024, and the staged activations fit in
+// shared memory (T*(H+8)*2 and T*k*(I+8)*2 bytes, 200 KB each).
+bool decode_mma_supported(int T, int H, int I, int E, int k);
+cudaError_t launch_decode_mma_gate_up(const DecodeMmaArgs& p, cudaStream_t st);
+cudaError_t launch_decode_mma_down(const DecodeMmaArgs& p, cudaStream_t st);
 
 // router
 // xmax (nullable): receives max |x_t| per token as fp32 bits; zero (nullable):

@@ -378,44 +378,46 @@ def test_decode_on_quantised_bank(name, T):
     assert rel_l2(bf16_np(y), ref["y"]) < 5e-3
 
 
-# ------------------------------------------------------------------ single-token tensor-core kernels
+# ------------------------------------------------------------------ tensor-core decode kernels
 #
-# One token with H a multiple of 1024 and I a multiple of 128 runs the routed
-# experts on the tensor cores (weights loaded straight into registers,
-# mma.sync); these shapes cover one to eight 128-code steps per K octant of a
-# gate/up row pair, one and two register batches of a down tile, 1 to 16 live
-# experts, items that do not divide evenly over the SMs' warps, the largest
-# supported H and I, and sites without a shared expert.
+# Up to 8 tokens with H a multiple of 1024 and I a multiple of 128 run the
+# routed experts on the tensor cores (weights streamed straight into
+# registers, mma.sync, one B column per token of an expert); these shapes
+# cover one to sixteen 128-code steps per K quarter of a gate/up tile, one to
+# sixteen steps of a down tile, 1 to 64 live experts, experts shared by
+# several tokens (up to 8 columns), tiles that do not divide evenly over the
+# SMs, the largest supported H and I, and sites without a shared expert.
 
-def _t1(H, I, E, k, Is, **kw):
+def _t1(H, I, E, k, Is, T=1, **kw):
     from routed_nvfp4_expert_b200 import synthetic as syn
-    return syn.Workload(f"t1_H{H}_I{I}_E{E}_k{k}", T=1, H=H, I=I, E=E, k=k, Is=Is, dense_I=64,
+    return syn.Workload(f"mma_T{T}_H{H}_I{I}_E{E}_k{k}", T=T, H=H, I=I, E=E, k=k, Is=Is, dense_I=64,
                         sigma_w=kw.pop("sigma_w", 0.0064 if H >= 2048 else 0.02), **kw)
 
 
-T1_SHAPES = [(1024, 128, 32, 4, 256), (3072, 768, 24, 6, 256), (1024, 512, 40, 16, 0), (2048, 1536, 20, 5, 128),
-             (8192, 2048, 12, 8, 512)]
+T1_SHAPES = [(1, 1024, 128, 32, 4, 256), (1, 3072, 768, 24, 6, 256), (1, 1024, 512, 40, 16, 0),
+             (1, 2048, 1536, 20, 5, 128), (1, 8192, 2048, 12, 8, 512), (3, 1024, 256, 16, 4, 128),
+             (8, 2048, 512, 24, 8, 256), (5, 4096, 1024, 40, 8, 0), (8, 1024, 128, 8, 8, 64)]
 
 
-@pytest.mark.parametrize("H,I,E,k,Is", T1_SHAPES)
-def test_t1_tensor_core_forward_matches_oracle(H, I, E, k, Is):
-    wl = _t1(H, I, E, k, Is)
+@pytest.mark.parametrize("T,H,I,E,k,Is", T1_SHAPES)
+def test_t1_tensor_core_forward_matches_oracle(T, H, I, E, k, Is):
+    wl = _t1(H, I, E, k, Is, T=T)
     inp = site_inputs(wl)
     y, lg, ws, v = _forward(wl, inp)
     ref = OS.site_forward(inp, oracle_cfg(wl), "decode", gpu_logits=lg, want_parts=True)
     got = bf16_np(y)
     assert_bf16_close(got, ref["y"], what=f"{wl.name} y")
     assert rel_l2(got, ref["y"]) < 5e-3
-    r = capi.view_tensor(v.r, (1, k, H), torch.float32)
+    r = capi.view_tensor(v.r, (T, k, H), torch.float32)
     assert_bf16_close(bf16_np(r), ref["r"], what="r")
     # h: the SwiGLU rows of the live assignments (fp32)
-    h = capi.view_tensor(v.h, (k, I), torch.float32).cpu().numpy().astype(np.float64)
-    ids = ref["ids"][0]
+    h = capi.view_tensor(v.h, (T, k, I), torch.float32).cpu().numpy().astype(np.float64)
     cache = OS.ExpertCache(inp)
     a64 = OF.bf16_value(inp["x"])
-    for j in range(k):
-        wg, wu, _ = cache.get(int(ids[j]))
-        assert_bf16_close(h[j], OS.clamped_swiglu(wg @ a64[0], wu @ a64[0], wl.limit), what=f"h[{j}]")
+    for t in range(T):
+        for j in range(k):
+            wg, wu, _ = cache.get(int(ref["ids"][t][j]))
+            assert_bf16_close(h[t, j], OS.clamped_swiglu(wg @ a64[t], wu @ a64[t], wl.limit), what=f"h[{t},{j}]")
     # the same input twice: bit-identical (every sum in a fixed order)
     y2, _, _, _ = _forward(wl, inp)
     assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
