@@ -37,6 +37,9 @@
 // consecutive codes of those 32 (k-slots 2t, 2t+1, 2t+8, 2t+9), and B holds
 // each token's activations at the same four positions.
 
+#include <algorithm>
+#include <cmath>
+
 #include "common.cuh"
 #include "gemv_common.cuh"
 #include "kernels.h"
@@ -50,8 +53,6 @@ constexpr int kThreads = kWarps * kWarp;
 constexpr int kMaxCols = 8;                // tokens per expert (mma N)
 constexpr int kMaxAsg = 128;               // T * k
 constexpr int kMaxLive = 128;              // live experts <= T * k
-constexpr int kSeg = 4;                    // gate/up: K split across the warps of a tile
-constexpr int kSlots = kWarps / kSeg;      // gate/up: tiles per CTA round
 constexpr int kDepthGU = 4;                // gate/up steps in flight per warp
 constexpr int kDepthD = 6;                 // down steps in flight per warp
 constexpr int kPad = 8;                    // f16 elements of padding per staged activation row
@@ -85,6 +86,32 @@ RNX_DEVICE void e2m1_pair(uint32_t w, uint32_t& a, uint32_t& b) {
         : "r"(w));
 }
 RNX_DEVICE uint32_t word_of(const uint4& q, int i) { return i == 0 ? q.x : i == 1 ? q.y : i == 2 ? q.z : q.w; }
+
+// Loads that the compiler keeps in program order with each other: the
+// activation loads of a launch's prologue go out ahead of its first weight
+// loads (the weight ring: streaming, no L1 allocation).
+RNX_DEVICE uint4 ldg_ordered(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+RNX_DEVICE uint4 ldg_ring(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+RNX_DEVICE uint32_t ldg_ring_u16(const void* p) {
+  uint16_t r;
+  asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(r) : "l"(p));
+  return r;
+}
+RNX_DEVICE float4 ldg_f4_ordered(const float* p) {
+  float4 r;
+  asm volatile("ld.global.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w) : "l"(p));
+  return r;
+}
 
 RNX_DEVICE void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
                           uint32_t b1) {
@@ -120,7 +147,8 @@ RNX_DEVICE void step_mma(float (&acc)[4], const uint4& q0, const uint4& q1, uint
 // The routing plan's live experts in shared memory: e[u], the expert of live
 // slot u (expert order), n[u] its token count (0 when its plan entry is out of
 // range: its tiles then read expert 0's bytes and write nothing), off[u] its
-// first entry in sorted[]; tsa / tsb the tensor scales asked for.
+// first entry in sorted[]; tsa / tsb the tensor scales asked for (filled by
+// load_scales, after the plan).
 struct PlanS {
   int n_live;
   int e[kMaxLive], n[kMaxLive], off[kMaxLive];
@@ -128,10 +156,20 @@ struct PlanS {
   uint8_t live_asg[kMaxAsg];
   float tsa[kMaxLive], tsb[kMaxLive];
 };
+constexpr int kMaxE = 1024;
 
-RNX_DEVICE void load_plan(const DecodeMmaArgs& p, const float* ts0, const float* ts1, PlanS& S) {
-  const int TK = p.T * p.k, i = threadIdx.x;
-  const int n_raw = min(min(max(p.active[0], 0), p.E), kMaxLive);   // active holds E + 1 entries
+// One round of global loads (the active list, every expert's count and
+// offset, the sorted assignments), then the live slots from shared memory.
+// All threads call it (three barriers).
+RNX_DEVICE void load_plan(const DecodeMmaArgs& p, PlanS& S, int* s_cnt, int* s_off) {
+  const int TK = p.T * p.k, E = p.E, i = threadIdx.x;
+  const int n_raw = min(min(max(p.active[0], 0), E), kMaxLive);   // active holds E + 1 entries
+  for (int e = i; e < E; e += kThreads) {
+    s_cnt[e] = p.counts[e];
+    s_off[e] = p.offsets[e];
+  }
+  int act = 0;
+  if (i < min(E, kMaxLive)) act = p.active[1 + i];
   if (i < kMaxAsg) {
     int v = 0;
     if (i < TK) {
@@ -144,13 +182,14 @@ RNX_DEVICE void load_plan(const DecodeMmaArgs& p, const float* ts0, const float*
     S.sorted[i] = v;
     S.live_asg[i] = 0;
   }
+  if (i == 0) S.n_live = n_raw;
+  __syncthreads();
   if (i < n_raw) {
-    int e = p.active[1 + i];
-    int off = 0, cnt = 0;
-    bool ok = e >= 0 && e < p.E && e >= p.lb && e < p.le;
+    int e = act, off = 0, cnt = 0;
+    bool ok = e >= 0 && e < E && e >= p.lb && e < p.le;
     if (ok) {
-      off = p.offsets[e];
-      cnt = p.counts[e];
+      off = s_off[e];
+      cnt = s_cnt[e];
       ok = off >= 0 && cnt >= 1 && cnt <= min(p.T, kMaxCols) && off + cnt <= TK;
     }
     if (!ok) {
@@ -162,14 +201,21 @@ RNX_DEVICE void load_plan(const DecodeMmaArgs& p, const float* ts0, const float*
     S.e[i] = e;
     S.n[i] = cnt;
     S.off[i] = off;
-    S.tsa[i] = ok ? ts0[e] : 0.f;
-    S.tsb[i] = (ok && ts1) ? ts1[e] : 0.f;
   }
-  if (i == 0) S.n_live = n_raw;
   __syncthreads();
   if (i < n_raw)
     for (int c = 0; c < S.n[i]; ++c) S.live_asg[S.sorted[S.off[i] + c]] = 1;
   __syncthreads();
+}
+
+// The live experts' tensor scales (visible after the caller's next barrier).
+RNX_DEVICE void load_scales(const PlanS& S, const float* ts0, const float* ts1, PlanS& W) {
+  const int i = threadIdx.x;
+  if (i < S.n_live) {
+    const bool ok = S.n[i] > 0;
+    W.tsa[i] = ok ? ts0[S.e[i]] : 0.f;
+    W.tsb[i] = (ok && ts1) ? ts1[S.e[i]] : 0.f;
+  }
 }
 
 // Zero rows (of `width` floats) of the assignments that are not live: this
@@ -182,24 +228,32 @@ RNX_DEVICE void zero_dead_rows(const PlanS& S, int TK, int width, float* out) {
       for (int c = n0 + (int)threadIdx.x; c < n1; c += kThreads) out[(size_t)a * width + c] = 0.f;
 }
 
-RNX_DEVICE void bar_named(int id, int count) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory"); }
 
 // ============================================================== gate/up
 //
-// Item = (tile, segment): tile = 16 rows (gate and up) of one live expert,
-// segment = a quarter of K = H; the 4 warps of a CTA tile slot take the 4
-// segments of one tile and meet at a named barrier, after which the slot sums
-// the quarters in a fixed order and applies the SwiGLU. A CTA takes tiles
-// blockIdx + G (4 rho + slot) in rounds rho. NS = H / 512 steps of 128 codes.
+// Work unit = two 8-row blocks of the live experts' gate and up matrices
+// (mma rows g and g + 8), full K = H split over the 4 warps of a CTA slot
+// (NS = H / 512 steps of 128 codes each); the slot's warps meet at a named
+// barrier and the slot sums the quarters in a fixed order and applies the
+// SwiGLU. Blocks go round-robin over the CTAs (block b to CTA b mod G), so
+// every SM streams the same bytes to within one 8-row block; with one token
+// any two of a CTA's blocks form a unit, with several tokens a unit is the
+// two halves of one 16-row tile (one expert: one set of token columns).
 
 struct GuRegs {
   uint4 g0, g1, u0, u1;
   uint32_t sg, su;
 };
 
+constexpr int kSeg = 4;                    // K split across the warps of a slot
+constexpr int kSlots = kWarps / kSeg;      // units per CTA round
+
+RNX_DEVICE void bar_named(int id, int count) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory"); }
+
 __global__ void __launch_bounds__(kThreads, 1) mma_gate_up_kernel(const DecodeMmaArgs p) {
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ PlanS S;
+  __shared__ int s_cnt[kMaxE], s_off[kMaxE];
   __shared__ float s_unscale[kMaxCols];
   const int H = p.H, I = p.I, T = p.T, k = p.k, TK = T * k;
   const int XR = H + kPad;                                   // staged row length (f16)
@@ -211,82 +265,125 @@ __global__ void __launch_bounds__(kThreads, 1) mma_gate_up_kernel(const DecodeMm
 
   pdl_wait();              // the plan and max |x| come from earlier launches
   pdl_trigger();
-  load_plan(p, p.gate.tensor_scale, p.up.tensor_scale, S);
-  const int TPE = I / 16, NT = S.n_live * TPE, G = gridDim.x;
-  // this slot's rounds: tiles blockIdx + G (kSlots rho + slot) below NT
-  const int tile0 = blockIdx.x + G * slot;
-  const int R = tile0 < NT ? (NT - 1 - tile0) / (G * kSlots) + 1 : 0;
+  load_plan(p, S, s_cnt, s_off);
+  const int BPE = I / 8, NB = S.n_live * BPE, G = gridDim.x;
+  // this CTA's blocks: blockIdx + G j for j < nb; unit i = blocks (2i, 2i + 1)
+  // of that list (one token), or tile blockIdx + G i = blocks (2 tile, 2 tile
+  // + 1) (several tokens)
+  const bool one = T == 1;
+  const int c = blockIdx.x;
+  const int nb = c < NB ? (NB - 1 - c) / G + 1 : 0;
+  const int NTl = NB / 2, ntl = c < NTl ? (NTl - 1 - c) / G + 1 : 0;
+  const int NU = one ? (nb + 1) / 2 : ntl;
+  // this slot's units: slot + kSlots rho
+  const int R = slot < NU ? (NU - 1 - slot) / kSlots + 1 : 0;
   const int Q = R * NS;
-
-  // load cursor: round lr, step ls, lane byte offsets of the tile's rows
-  int lr = 0, ls = 0;
-  size_t oc = 0, os = 0;
-  auto tile_offsets = [&](int rho) {
-    const int tau = tile0 + G * kSlots * rho;
-    const int u = tau / TPE, rb = tau - u * TPE;
-    const size_t row = (size_t)S.e[u] * I + 16 * rb + g;
-    oc = row * (H / 2) + seg * (H / 8) + 16 * t;
-    os = row * (H / 16) + seg * (H / 64) + 2 * t;
-  };
-  auto load = [&](GuRegs& r) {
-    const size_t c = oc + 64 * ls, sofs = os + 8 * ls;
-    r.g0 = ldg_stream(p.gate.codes + c);
-    r.g1 = ldg_stream(p.gate.codes + c + 4 * (size_t)H);
-    r.u0 = ldg_stream(p.up.codes + c);
-    r.u1 = ldg_stream(p.up.codes + c + 4 * (size_t)H);
-    r.sg = (uint32_t)ldg_u16(p.gate.scales + sofs) | ((uint32_t)ldg_u16(p.gate.scales + sofs + H / 2) << 16);
-    r.su = (uint32_t)ldg_u16(p.up.scales + sofs) | ((uint32_t)ldg_u16(p.up.scales + sofs + H / 2) << 16);
-    if (++ls == NS) {
-      ls = 0;
-      if (++lr < R) tile_offsets(lr);
+  auto unit_blocks = [&](int rho, int& ba, int& bb) {
+    const int i = slot + kSlots * rho;
+    if (one) {
+      ba = c + G * (2 * i);
+      bb = 2 * i + 1 < nb ? c + G * (2 * i + 1) : -1;
+    } else {
+      ba = 2 * (c + G * i);
+      bb = ba + 1;
     }
   };
 
+  // x first (the tokens as B columns: f16 of x times the token's power of
+  // two, in passes of kXq 16-byte chunks per thread), then the weight ring.
+  // Load cursor: round lr, step ls, lane byte offsets of its two rows
+  // (32-bit: a bank's codes are below 4 GB).
+  int lr = 0, ls = 0;
+  uint32_t oca = 0, ocb = 0, osa = 0, osb = 0;
+  auto unit_offsets = [&](int rho) {
+    int ba, bb;
+    unit_blocks(rho, ba, bb);
+    if (bb < 0) bb = ba;                   // a lone block: its twin rows read again, not written
+    const int ua = ba / BPE, ub = bb / BPE;
+    const uint32_t ra = (uint32_t)S.e[ua] * (uint32_t)I + 8 * (ba - ua * BPE) + g;
+    const uint32_t rb = (uint32_t)S.e[ub] * (uint32_t)I + 8 * (bb - ub * BPE) + g;
+    oca = ra * (uint32_t)(H / 2) + seg * (H / 8) + 16 * t;
+    ocb = rb * (uint32_t)(H / 2) + seg * (H / 8) + 16 * t;
+    osa = ra * (uint32_t)(H / 16) + seg * (H / 64) + 2 * t;
+    osb = rb * (uint32_t)(H / 16) + seg * (H / 64) + 2 * t;
+  };
+  auto load = [&](GuRegs& r) {
+    const uint32_t d = 64 * ls, e8 = 8 * ls;
+    r.g0 = ldg_ring(p.gate.codes + (oca + d));
+    r.g1 = ldg_ring(p.gate.codes + (ocb + d));
+    r.u0 = ldg_ring(p.up.codes + (oca + d));
+    r.u1 = ldg_ring(p.up.codes + (ocb + d));
+    r.sg = ldg_ring_u16(p.gate.scales + (osa + e8)) | (ldg_ring_u16(p.gate.scales + (osb + e8)) << 16);
+    r.su = ldg_ring_u16(p.up.scales + (osa + e8)) | (ldg_ring_u16(p.up.scales + (osb + e8)) << 16);
+    if (++ls == NS) {
+      ls = 0;
+      if (++lr < R) unit_offsets(lr);
+    }
+  };
   GuRegs ring[kDepthGU];
-  if (R > 0) tile_offsets(0);
+
+  constexpr int kXq = 4;
+  const int NXC = T * (H / 8);
+  float xup[kMaxCols];
+#pragma unroll
+  for (int tk = 0; tk < kMaxCols; ++tk) {
+    float un = 1.f;
+    xup[tk] = 1.f;
+    if (tk < T) prescale15(__uint_as_float(p.xmax[tk]), xup[tk], un);
+    if (threadIdx.x == 0 && tk < T) s_unscale[tk] = un;
+  }
+  for (int c0 = 0; c0 < NXC; c0 += kThreads * kXq) {
+    uint4 xv[kXq];
+#pragma unroll
+    for (int j = 0; j < kXq; ++j) {
+      const int cc = c0 + threadIdx.x + kThreads * j;
+      if (cc < NXC) xv[j] = ldg_ordered(p.x + (size_t)(cc / (H / 8)) * H + 8 * (cc % (H / 8)));
+    }
+    if (c0 == 0) load_scales(S, p.gate.tensor_scale, p.up.tensor_scale, S);
+#pragma unroll
+    for (int j = 0; j < kXq; ++j) {
+      const int cc = c0 + threadIdx.x + kThreads * j;
+      if (cc < NXC) {
+        const int tk = cc / (H / 8), q = cc - tk * (H / 8);
+        float up = xup[0];
+#pragma unroll
+        for (int z = 1; z < kMaxCols; ++z)
+          if (z == tk) up = xup[z];
+        const uint32_t w4[4] = {xv[j].x, xv[j].y, xv[j].z, xv[j].w};
+        uint32_t o[4];
+#pragma unroll
+        for (int z = 0; z < 4; ++z) {
+          const float2 f = bf16x2_to_f32x2(w4[z]);
+          __half2 h2 = __floats2half2_rn(f.x * up, f.y * up);
+          o[z] = *reinterpret_cast<uint32_t*>(&h2);
+        }
+        *reinterpret_cast<uint4*>(xs + (size_t)tk * XR + 8 * q) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+    }
+  }
+  // the weight ring goes out once x is converted: issued earlier, its
+  // requests would hold up the conversion's own loads in the memory queues
+  if (R > 0) unit_offsets(0);
 #pragma unroll
   for (int j = 0; j < kDepthGU; ++j)
     if (j < Q) load(ring[j]);
-
-  // the tokens as B columns: f16 of x times the token's power of two
-  if (threadIdx.x < T) {
-    float up, unscale;
-    prescale15(__uint_as_float(p.xmax[threadIdx.x]), up, unscale);
-    s_unscale[threadIdx.x] = unscale;
-  }
-  for (int c = threadIdx.x; c < T * (H / 8); c += kThreads) {
-    const int tk = c / (H / 8), q = c - tk * (H / 8);
-    float up, unscale;
-    prescale15(__uint_as_float(p.xmax[tk]), up, unscale);
-    const uint4 v = *reinterpret_cast<const uint4*>(p.x + (size_t)tk * H + 8 * q);
-    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-    uint32_t o[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 f = bf16x2_to_f32x2(w4[j]);
-      __half2 h2 = __floats2half2_rn(f.x * up, f.y * up);
-      o[j] = *reinterpret_cast<uint32_t*>(&h2);
-    }
-    *reinterpret_cast<uint4*>(xs + (size_t)tk * XR + 8 * q) = make_uint4(o[0], o[1], o[2], o[3]);
-  }
   __syncthreads();
 
-  // compute cursor
-  int cr = 0, cs = 0, cu = 0, crb = 0;
+  // compute cursor: round cr, step cs
+  int cr = 0, cs = 0, cba = 0, cbb = -1;
   const uint16_t* brow = xs;
-  auto tile_setup = [&](int rho) {
-    const int tau = tile0 + G * kSlots * rho;
-    cu = tau / TPE;
-    crb = tau - cu * TPE;
-    const int n = max(S.n[cu], 1), col = g < n ? g : 0;
-    const int tok = S.sorted[S.off[cu] + col] / k;
+  auto unit_setup = [&](int rho) {
+    unit_blocks(rho, cba, cbb);
+    const int u = cba / BPE;                // several tokens: both blocks belong to expert u
+    const int n = max(S.n[u], 1), col = g < n ? g : 0;
+    const int tok = S.sorted[S.off[u] + col] / k;
     brow = xs + (size_t)tok * XR + seg * (H / 4) + 32 * t;
   };
-  if (R > 0) tile_setup(0);
+  if (R > 0) unit_setup(0);
   float ag[4] = {0.f, 0.f, 0.f, 0.f}, au[4] = {0.f, 0.f, 0.f, 0.f};
   int buf = 0;
 
-  auto finish_item = [&]() {
+  auto finish_unit = [&]() {
     // the slot's partial sums: red[buf][slot][seg][gate/up][16 rows][8 cols]
     float* rs = red + ((size_t)(buf * kSlots + slot) * kSeg + seg) * 256;
     *reinterpret_cast<float2*>(rs + 8 * g + 2 * t) = make_float2(ag[0], ag[1]);
@@ -294,18 +391,23 @@ __global__ void __launch_bounds__(kThreads, 1) mma_gate_up_kernel(const DecodeMm
     *reinterpret_cast<float2*>(rs + 128 + 8 * g + 2 * t) = make_float2(au[0], au[1]);
     *reinterpret_cast<float2*>(rs + 128 + 8 * (g + 8) + 2 * t) = make_float2(au[2], au[3]);
     bar_named(1 + slot, kSeg * kWarp);
-    const int i = seg * kWarp + lane, row = i >> 3, col = i & 7;
-    if (col < S.n[cu]) {
-      const float* r0 = red + (size_t)(buf * kSlots + slot) * kSeg * 256;
-      float gs = 0.f, us = 0.f;
+    const int i = seg * kWarp + lane, row = i >> 3, col = i & 7;     // 16 rows x 8 columns
+    const int blk = row < 8 ? cba : cbb;
+    if (blk >= 0) {
+      const int u = blk / BPE;
+      if (col < S.n[u]) {
+        const float* r0 = red + (size_t)(buf * kSlots + slot) * kSeg * 256;
+        float gs = 0.f, us = 0.f;
 #pragma unroll
-      for (int q = 0; q < kSeg; ++q) {
-        gs += r0[q * 256 + 8 * row + col];
-        us += r0[q * 256 + 128 + 8 * row + col];
+        for (int q = 0; q < kSeg; ++q) {
+          gs += r0[q * 256 + 8 * row + col];
+          us += r0[q * 256 + 128 + 8 * row + col];
+        }
+        const int a = S.sorted[S.off[u] + col];
+        const float un = s_unscale[a / k];
+        p.h[(size_t)a * I + 8 * (blk - u * BPE) + (row & 7)] =
+            clamped_swiglu(gs * un * S.tsa[u], us * un * S.tsb[u], p.limit);
       }
-      const int a = S.sorted[S.off[cu] + col];
-      const float un = s_unscale[a / k];
-      p.h[(size_t)a * I + 16 * crb + row] = clamped_swiglu(gs * un * S.tsa[cu], us * un * S.tsb[cu], p.limit);
     }
     buf ^= 1;
 #pragma unroll
@@ -323,8 +425,8 @@ __global__ void __launch_bounds__(kThreads, 1) mma_gate_up_kernel(const DecodeMm
         if (q0 + j + kDepthGU < Q) load(ring[j]);
         if (++cs == NS) {
           cs = 0;
-          finish_item();
-          if (++cr < R) tile_setup(cr);
+          finish_unit();
+          if (++cr < R) unit_setup(cr);
         }
       }
     }
@@ -347,6 +449,7 @@ struct DnRegs {
 __global__ void __launch_bounds__(kThreads, 1) mma_down_kernel(const DecodeMmaArgs p) {
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ PlanS S;
+  __shared__ int s_cnt[kMaxE], s_off[kMaxE];
   __shared__ float s_sc[kMaxAsg], s_up[kMaxAsg];
   __shared__ uint32_t s_max[kMaxAsg];
   const int H = p.H, I = p.I, T = p.T, k = p.k, TK = T * k;
@@ -355,76 +458,107 @@ __global__ void __launch_bounds__(kThreads, 1) mma_down_kernel(const DecodeMmaAr
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int NSD = I / 128;
 
-  // The plan comes from two launches back, complete when this grid starts;
-  // the weight loads need only the plan, so they go out before the wait for h.
-  load_plan(p, p.down.tensor_scale, nullptr, S);
+  // The plan and the routing weights come from two launches back, complete
+  // when this grid starts: the plan and the tensor scales before the wait for
+  // h; after it h is staged, then the weight ring goes out (issued earlier,
+  // its requests would hold up the staging's own loads in the memory queues).
+  load_plan(p, S, s_cnt, s_off);
+  load_scales(S, p.down.tensor_scale, nullptr, S);
   const int TPE = H / 16, NT = S.n_live * TPE, G = gridDim.x, GW = G * kWarps;
   const int tile0 = blockIdx.x + G * warp;
   const int R = tile0 < NT ? (NT - 1 - tile0) / GW + 1 : 0;
   const int Q = R * NSD;
+  float wa = 0.f;
+  if (threadIdx.x < TK) wa = p.weights[threadIdx.x];
+  if (threadIdx.x < kMaxAsg) s_max[threadIdx.x] = 0u;
+  const bool fixed = p.h_up > 0.f;
+  if (fixed && threadIdx.x < TK) {
+    s_up[threadIdx.x] = p.h_up;
+    s_sc[threadIdx.x] = p.h_unscale * wa;
+  }
 
   int lr = 0, ls = 0;
-  size_t oc = 0, os = 0;
+  uint32_t oc = 0, os = 0;
   auto tile_offsets = [&](int rho) {
     const int tau = tile0 + GW * rho;
     const int u = tau / TPE, rb = tau - u * TPE;
-    const size_t row = (size_t)S.e[u] * H + 16 * rb + g;
-    oc = row * (I / 2) + 16 * t;
-    os = row * (I / 16) + 2 * t;
+    const uint32_t row = (uint32_t)S.e[u] * (uint32_t)H + 16 * rb + g;
+    oc = row * (uint32_t)(I / 2) + 16 * t;
+    os = row * (uint32_t)(I / 16) + 2 * t;
   };
   auto load = [&](DnRegs& r) {
-    const size_t c = oc + 64 * ls, sofs = os + 8 * ls;
-    r.c0 = ldg_stream(p.down.codes + c);
-    r.c1 = ldg_stream(p.down.codes + c + 4 * (size_t)I);
-    r.sc = (uint32_t)ldg_u16(p.down.scales + sofs) | ((uint32_t)ldg_u16(p.down.scales + sofs + I / 2) << 16);
+    const uint32_t c = oc + 64 * ls, sofs = os + 8 * ls;
+    r.c0 = ldg_ring(p.down.codes + c);
+    r.c1 = ldg_ring(p.down.codes + (c + 4 * I));
+    r.sc = ldg_ring_u16(p.down.scales + sofs) | (ldg_ring_u16(p.down.scales + (sofs + I / 2)) << 16);
     if (++ls == NSD) {
       ls = 0;
       if (++lr < R) tile_offsets(lr);
     }
   };
   DnRegs ring[kDepthD];
+  pdl_wait();                // h comes from the previous launch
+  pdl_trigger();
+
+  // h rows of the live assignments as B columns, f16 of h times the row's
+  // power of two: a fixed one from the clamp's bound on |h| when the limit is
+  // finite, else from each row's maximum (a first pass; one shared atomic
+  // per warp and row: with I a multiple of 128 a warp's 32 float4 lie in one
+  // row). Loads go out kHq at a time per thread.
+  constexpr int kHq = 4;
+  const int Q4 = I / 4, NH = TK * Q4;                      // NH % 32 == 0: warp-uniform bounds
+  __syncthreads();
+  if (!fixed) {
+    for (int c0 = 0; c0 < NH; c0 += kThreads * kHq) {
+      float4 v[kHq];
+#pragma unroll
+      for (int j = 0; j < kHq; ++j) {
+        const int c = c0 + threadIdx.x + kThreads * j, a = c / Q4;
+        v[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (c < NH && S.live_asg[a]) v[j] = ldg_f4_ordered(p.h + (size_t)a * I + 4 * (c - a * Q4));
+      }
+#pragma unroll
+      for (int j = 0; j < kHq; ++j) {
+        const int c = c0 + threadIdx.x + kThreads * j;
+        if (c < NH) {
+          const float m = warp_max(fmaxf(fmaxf(fabsf(v[j].x), fabsf(v[j].y)), fmaxf(fabsf(v[j].z), fabsf(v[j].w))));
+          if (lane == 0) atomicMax(&s_max[c / Q4], __float_as_uint(m));   // non-negative floats order as integers
+        }
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x < TK) {
+      float upx, us;
+      prescale15(__uint_as_float(s_max[threadIdx.x]), upx, us);
+      s_up[threadIdx.x] = upx;
+      s_sc[threadIdx.x] = us * wa;
+    }
+    __syncthreads();
+  }
+  for (int c0 = 0; c0 < NH; c0 += kThreads * kHq) {
+    float4 v[kHq];
+#pragma unroll
+    for (int j = 0; j < kHq; ++j) {
+      const int c = c0 + threadIdx.x + kThreads * j, a = c / Q4;
+      v[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (c < NH && S.live_asg[a]) v[j] = ldg_f4_ordered(p.h + (size_t)a * I + 4 * (c - a * Q4));
+    }
+#pragma unroll
+    for (int j = 0; j < kHq; ++j) {
+      const int c = c0 + threadIdx.x + kThreads * j;
+      if (c < NH) {
+        const int a = c / Q4, q = c - a * Q4;
+        const float upx = s_up[a];
+        __half2 h0 = __floats2half2_rn(v[j].x * upx, v[j].y * upx), h1 = __floats2half2_rn(v[j].z * upx, v[j].w * upx);
+        *reinterpret_cast<uint2*>(hs + (size_t)a * HR + 4 * q) =
+            make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
+      }
+    }
+  }
   if (R > 0) tile_offsets(0);
 #pragma unroll
   for (int j = 0; j < kDepthD; ++j)
     if (j < Q) load(ring[j]);
-  if (threadIdx.x < kMaxAsg) s_max[threadIdx.x] = 0u;
-
-  pdl_wait();                // h comes from the previous launch
-  pdl_trigger();
-
-  // h rows of the live assignments as B columns: the row maxima first (one
-  // shared atomic per warp: with I a multiple of 128 a warp's 32 float4 lie
-  // in one row), then the f16 conversion times the row's power of two.
-  const int Q4 = I / 4;
-  __syncthreads();
-  for (int c = threadIdx.x; c < TK * Q4; c += kThreads) {   // warp-uniform bound: TK * Q4 % 32 == 0
-    const int a = c / Q4;
-    float m = 0.f;
-    if (S.live_asg[a]) {
-      const float4 v = *reinterpret_cast<const float4*>(p.h + (size_t)a * I + 4 * (c - a * Q4));
-      m = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
-    }
-    m = warp_max(m);
-    if (lane == 0) atomicMax(&s_max[a], __float_as_uint(m));   // non-negative floats order as integers
-  }
-  __syncthreads();
-  if (threadIdx.x < TK) {
-    const int a = threadIdx.x;
-    float upx, us;
-    prescale15(__uint_as_float(s_max[a]), upx, us);
-    s_up[a] = upx;
-    s_sc[a] = us * p.weights[a];
-  }
-  __syncthreads();
-  for (int c = threadIdx.x; c < TK * Q4; c += kThreads) {
-    const int a = c / Q4, q = c - a * Q4;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (S.live_asg[a]) v = *reinterpret_cast<const float4*>(p.h + (size_t)a * I + 4 * q);
-    const float upx = s_up[a];
-    __half2 h0 = __floats2half2_rn(v.x * upx, v.y * upx), h1 = __floats2half2_rn(v.z * upx, v.w * upx);
-    *reinterpret_cast<uint2*>(hs + (size_t)a * HR + 4 * q) =
-        make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
-  }
   __syncthreads();
 
   int cr = 0, cs = 0, cu = 0, crb = 0;
@@ -499,12 +633,13 @@ constexpr size_t kSmemBudget = 200 * 1024;
 
 }  // namespace
 
+
 bool decode_mma_supported(int T, int H, int I, int E, int k) {
   if (T < 1 || T > kMaxCols || H % 1024 || H > 8192 || I % 128 || I > 2048 || k < 1 || k > 16 || E < 1 ||
-      E > 1024 || T * k > kMaxAsg)
+      E > kMaxE || T * k > kMaxAsg)
     return false;
   if (gate_up_smem(T, H) > kSmemBudget || down_smem(T, k, I) > kSmemBudget) return false;
-  return (long long)E * (H > I ? H : I) < (1ll << 31);
+  return (long long)E * H * I / 2 < (1ll << 32);               // 32-bit byte offsets into a bank
 }
 
 cudaError_t launch_decode_mma_gate_up(const DecodeMmaArgs& a, cudaStream_t st) {
@@ -525,7 +660,20 @@ cudaError_t launch_decode_mma_down(const DecodeMmaArgs& a, cudaStream_t st) {
   const size_t smem = down_smem(a.T, a.k, a.I);
   cudaError_t e = cudaFuncSetAttribute(mma_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(mma_down_kernel, dim3(sm_count()), dim3(kThreads), smem, st, a);
+  // |h| = |silu(min(g, L))| |clamp(u, -L, L)| <= max(L, 0.28) L (silu(z) <= z
+  // for z >= 0 and |silu(z)| < 0.279 for z < 0): with a finite limit one power
+  // of two puts every h row under 2^15 in f16
+  DecodeMmaArgs b = a;
+  b.h_up = 0.f;
+  b.h_unscale = 0.f;
+  const double bound = std::max((double)a.limit, 0.28) * (double)a.limit;
+  if (std::isfinite(bound) && bound > 0.0 && bound < 1e30) {
+    int ex = 0;
+    std::frexp(bound, &ex);
+    b.h_up = (float)std::ldexp(1.0, 15 - ex);
+    b.h_unscale = (float)std::ldexp(1.0, ex - 15);
+  }
+  return launch_pdl(mma_down_kernel, dim3(sm_count()), dim3(kThreads), smem, st, b);
 }
 
 }  // namespace rnx

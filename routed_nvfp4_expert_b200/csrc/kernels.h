@@ -64,10 +64,12 @@ struct DecodeMmaArgs {
   float* h;                          // fp32 [T*k, I]
   float* r;                          // fp32 [T*k, H] weighted routed rows
   uint32_t* status;
+  float h_up, h_unscale;             // set by the down launcher: fixed power of two for h (0: per-row maxima)
 };
 // 1 <= T <= 8, H a multiple of 1024 up to 8192, I a multiple of 128 up to
-// 2048, k <= 16, T*k <= 128, E <= 1024, and the staged activations fit in
-// shared memory (T*(H+8)*2 and T*k*(I+8)*2 bytes, 200 KB each).
+// 2048, k <= 16, T*k <= 128, E <= 1024, a bank below 4 GB, and the staged
+// activations fit in shared memory (T*(H+8)*2 and T*k*(I+8)*2 bytes, 200 KB
+// each).
 bool decode_mma_supported(int T, int H, int I, int E, int k);
 cudaError_t launch_decode_mma_gate_up(const DecodeMmaArgs& p, cudaStream_t st);
 cudaError_t launch_decode_mma_down(const DecodeMmaArgs& p, cudaStream_t st);

@@ -211,39 +211,36 @@ __global__ void __launch_bounds__(kT1PlanThreads) topk_plan_t1_kernel(const floa
   __syncthreads();
   if (threadIdx.x < 32) topk_warp<PL>(s_key[0], s_sig[0], 0, E, k, rsf, ids, weights, s_ids);
   __syncthreads();
-  int id[kMaxTopK];
-  bool valid[kMaxTopK];
-#pragma unroll
-  for (int j = 0; j < kMaxTopK; ++j) {
-    id[j] = j < k ? s_ids[j] : -1;
-    valid[j] = j < k && id[j] >= 0 && id[j] < E;
-  }
+  // every plan entry is a count over the k chosen ids (read from shared
+  // memory: a per-thread copy indexed by the thread would live in local memory)
+  auto id_at = [&](int j) { return s_ids[j]; };
+  auto valid_at = [&](int j) { const int v = s_ids[j]; return j < k && v >= 0 && v < E; };
   for (int e = threadIdx.x; e <= E; e += kT1PlanThreads) {
     int cnt = 0, off = 0, toff = 0;
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) {
-      if (!valid[j]) continue;
-      cnt += id[j] == e;
-      off += id[j] < e;
-      toff += id[j] < e && id[j] >= lb && id[j] < le;
+    for (int j = 0; j < k; ++j) {
+      const int v = id_at(j);
+      if (!valid_at(j)) continue;
+      cnt += v == e;
+      off += v < e;
+      toff += v < e && v >= lb && v < le;
     }
     if (e < E) plan.counts[e] = cnt;
     plan.offsets[e] = off;
     plan.tile_offsets[e] = toff;
   }
   if (threadIdx.x < k) {
-    const int j = threadIdx.x;
-    if (valid[j]) {
+    const int j = threadIdx.x, idj = id_at(j);
+    if (valid_at(j)) {
       int pos = 0, lpos = 0;
-#pragma unroll
-      for (int i = 0; i < kMaxTopK; ++i) {
-        pos += valid[i] && id[i] < id[j];
-        lpos += valid[i] && id[i] < id[j] && id[i] >= lb && id[i] < le;
+      for (int i = 0; i < k; ++i) {
+        const int v = id_at(i);
+        pos += valid_at(i) && v < idj;
+        lpos += valid_at(i) && v < idj && v >= lb && v < le;
       }
       plan.sorted[pos] = j;
       plan.inv[j] = pos;
-      if (id[j] >= lb && id[j] < le) {
-        plan.active[1 + lpos] = id[j];
+      if (idj >= lb && idj < le) {
+        plan.active[1 + lpos] = idj;
         plan.first[lpos] = j;
       }
     } else {
@@ -253,8 +250,7 @@ __global__ void __launch_bounds__(kT1PlanThreads) topk_plan_t1_kernel(const floa
   }
   if (threadIdx.x == 0) {
     int nl = 0;
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) nl += valid[j] && id[j] >= lb && id[j] < le;
+    for (int j = 0; j < k; ++j) nl += valid_at(j) && id_at(j) >= lb && id_at(j) < le;
     plan.active[0] = nl;
   }
 }

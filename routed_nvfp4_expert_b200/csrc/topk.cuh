@@ -10,22 +10,9 @@
 
 namespace rnx {
 
-// One warp per token. Lane l holds experts l, l+32, ... Candidate order:
-// unused finite keys first (key descending, then lower index), then NaN keys
-// (lower index first), then used / padding entries.
-// That order as one 64-bit integer, larger = better (one warp max per
-// selection round): bits 63..62 the class (live 2, NaN 1, taken / padding 0),
-// bits 61..30 a live key's fp32 bits mapped to unsigned order (a zero key as
-// +0), bits 29..0 the complement of the index (the lower index wins a tie).
-RNX_DEVICE unsigned long long cand_rank(int state, float key, int idx) {
-  uint32_t ok = 0;
-  if (state == 0) {
-    const uint32_t u = key == 0.f ? 0u : __float_as_uint(key);
-    ok = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-  }
-  return ((unsigned long long)(2 - state) << 62) | ((unsigned long long)ok << 30) |
-         (unsigned long long)(0x3FFFFFFF - idx);
-}
+// Candidate order of a selection (one warp per token, lane l holds experts
+// l, l + 32, ...): unused non-NaN keys first (key descending, then lower
+// index), then NaN keys (lower index first), then used / padding entries.
 
 // 8 tokens per CTA. All 256 threads first evaluate the sigmoid scores and
 // selection keys of the CTA's tokens into shared memory; then one warp per
@@ -49,44 +36,49 @@ RNX_DEVICE void topk_keys(const float* __restrict__ logits, const float* __restr
 }
 
 // One warp selects token t's top-k from its keys and writes ids / weights
-// (and the ids to s_ids[0..k) as well when given).
+// (and the ids to s_ids[0..k) as well when given). Each candidate's 32-bit
+// rank key is formed once: live keys (finite or infinite) in fp32 order
+// mapped to unsigned order, all above 1; NaN keys 1; taken / padding 0. A
+// selection round is one warp max of the rank keys (redux), then one warp min
+// of the indices that hold it (the lower index wins a tie), and the owner
+// clears the chosen key.
+RNX_DEVICE uint32_t rank_key(float key) {
+  if (isnan(key)) return 1u;
+  const uint32_t u = key == 0.f ? 0u : __float_as_uint(key);   // -0 as +0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);         // >= 0x007FFFFF for every non-NaN key
+}
+
 template <int PL>
 RNX_DEVICE void topk_warp(const float* s_key_row, const float* s_sig_row, int t, int E, int k, float rsf,
                           int32_t* __restrict__ ids, float* __restrict__ weights, int* s_ids = nullptr) {
   const int lane = threadIdx.x & 31;
-  float key[PL], sg[PL];
-  int st[PL];
+  uint32_t rk[PL];
+  float sg[PL];
 #pragma unroll
   for (int i = 0; i < PL; ++i) {
     const int e = lane + 32 * i;
-    if (e < E) {
-      key[i] = s_key_row[e];
-      sg[i] = s_sig_row[e];
-      st[i] = isnan(key[i]) ? 1 : 0;
-    } else {
-      sg[i] = 0.f;
-      key[i] = 0.f;
-      st[i] = 2;
-    }
+    rk[i] = e < E ? rank_key(s_key_row[e]) : 0u;
+    sg[i] = e < E ? s_sig_row[e] : 0.f;
   }
   float chosen_s = 0.f;   // lane j keeps the score of rank slot j
   int chosen_id = 0;
   for (int j = 0; j < k; ++j) {
-    unsigned long long best = 0ull;
+    uint32_t m = rk[0];
 #pragma unroll
-    for (int i = 0; i < PL; ++i) best = max(best, cand_rank(st[i], key[i], lane + 32 * i));
+    for (int i = 1; i < PL; ++i) m = max(m, rk[i]);
+    const uint32_t best = __reduce_max_sync(0xffffffffu, m);
+    // the lowest index holding the best key: this lane's first, then the warp's
+    uint32_t mine = 0xFFFFFFFFu;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
-    const int idx = 0x3FFFFFFF - (int)(best & 0x3FFFFFFFull);
-    // the owner marks its entry taken and hands over its score
+    for (int i = PL - 1; i >= 0; --i) mine = rk[i] == best ? (uint32_t)(lane + 32 * i) : mine;
+    const int idx = (int)__reduce_min_sync(0xffffffffu, mine);
+    // the owner clears the chosen key and hands over its score
     float s_own = 0.f;
-    if ((idx & 31) == lane) {
 #pragma unroll
-      for (int i = 0; i < PL; ++i)
-        if (lane + 32 * i == idx) {
-          st[i] = 2;
-          s_own = sg[i];
-        }
+    for (int i = 0; i < PL; ++i) {
+      const bool hit = lane + 32 * i == idx;
+      s_own = hit ? sg[i] : s_own;
+      rk[i] = hit ? 0u : rk[i];
     }
     const float s_best = __shfl_sync(0xffffffffu, s_own, idx & 31);
     if (lane == j) {
