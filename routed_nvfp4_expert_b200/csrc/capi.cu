@@ -776,7 +776,9 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
 
   RNX_CUDA(cudaMemsetAsync(status, 0, kCtrlBytes, st), "clear status");
 
-  // decode: the shared expert forks off to the auxiliary stream right away
+  // decode: the shared expert forks off to the auxiliary stream right away;
+  // its launches follow the router's (the router then does not wait behind
+  // them to start)
   SideStream* side = nullptr;
   const bool shared_aside = Is > 0 && decode;
   void* shared = Is > 0 ? (void*)(b + L.shared) : nullptr;
@@ -784,10 +786,6 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
     RNX_CUDA(side_stream(&side), "auxiliary stream");
     RNX_CUDA(cudaEventRecord(side->fork, st), "fork event");
     RNX_CUDA(cudaStreamWaitEvent(side->st, side->fork, 0), "fork wait");
-    RNX_CUDA(rnx::launch_dense_gemv(H, Is, cfg->swiglu_limit, x, T, w->shared_gate, w->shared_up, w->shared_down,
-                                    shared, true, (float*)(b + L.shared_h), side->st),
-             "shared expert");
-    RNX_CUDA(cudaEventRecord(side->join, side->st), "join event");
   }
   // a handful of tokens: the tensor-core expert kernels (one CTA per SM,
   // weight rows streamed into registers), fed from the routing plan; the
@@ -800,6 +798,12 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
     RNX_CUDA(rnx::launch_router_logits_tc(x, T, H, E, w3, logits, status, st), "router logits (tensor cores)");
   } else {
     RNX_CUDA(rnx::launch_router_logits(x, T, H, E, w->router_w, logits, st, t1 ? xmax : nullptr), "router logits");
+  }
+  if (shared_aside) {
+    RNX_CUDA(rnx::launch_dense_gemv(H, Is, cfg->swiglu_limit, x, T, w->shared_gate, w->shared_up, w->shared_down,
+                                    shared, true, (float*)(b + L.shared_h), side->st),
+             "shared expert");
+    RNX_CUDA(cudaEventRecord(side->join, side->st), "join event");
   }
   RNX_CUDA(mark(MOE_STAGE_TOPK, st), "stage event");
   // decode with a handful of tokens: selection and plan in one launch (the

@@ -43,6 +43,7 @@
 #include "common.cuh"
 #include "gemv_common.cuh"
 #include "kernels.h"
+#include "tma.cuh"
 
 namespace rnx {
 
@@ -361,13 +362,15 @@ __global__ void __launch_bounds__(kThreads, 1) mma_gate_up_kernel(const DecodeMm
       }
     }
   }
-  // the weight ring goes out once x is converted: issued earlier, its
-  // requests would hold up the conversion's own loads in the memory queues
+  // the weight ring goes out once x is staged (issued earlier, its requests
+  // would hold up the staging's own loads in the memory queues), and after
+  // the barrier: a warp whose ring loads stall on a full memory queue holds
+  // up no other warp
+  __syncthreads();
   if (R > 0) unit_offsets(0);
 #pragma unroll
   for (int j = 0; j < kDepthGU; ++j)
     if (j < Q) load(ring[j]);
-  __syncthreads();
 
   // compute cursor: round cr, step cs
   int cr = 0, cs = 0, cba = 0, cbb = -1;
@@ -432,6 +435,67 @@ __global__ void __launch_bounds__(kThreads, 1) mma_gate_up_kernel(const DecodeMm
     }
   }
   zero_dead_rows(S, TK, I, p.h);
+}
+
+// h rows of the live assignments as B columns, f16 of h times the row's
+// power of two: a fixed one from the clamp's bound on |h| when the limit is
+// finite (s_up / s_sc set by the caller), else from each row's maximum (a
+// first pass; one shared atomic per warp and row: with I a multiple of 128 a
+// warp's 32 float4 lie in one row). Loads go out kHq at a time per thread.
+// All threads call it; a barrier of the caller's then publishes hs.
+RNX_DEVICE void stage_h(const DecodeMmaArgs& p, const PlanS& S, uint16_t* hs, uint32_t* s_max, float* s_up,
+                        float* s_sc, float wa, bool fixed) {
+  const int I = p.I, TK = p.T * p.k, HR = I + kPad, lane = threadIdx.x & 31;
+  constexpr int kHq = 4;
+  const int Q4 = I / 4, NH = TK * Q4;                      // NH % 32 == 0: warp-uniform bounds
+  __syncthreads();
+  if (!fixed) {
+    for (int c0 = 0; c0 < NH; c0 += kThreads * kHq) {
+      float4 v[kHq];
+#pragma unroll
+      for (int j = 0; j < kHq; ++j) {
+        const int c = c0 + threadIdx.x + kThreads * j, a = c / Q4;
+        v[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (c < NH && S.live_asg[a]) v[j] = ldg_f4_ordered(p.h + (size_t)a * I + 4 * (c - a * Q4));
+      }
+#pragma unroll
+      for (int j = 0; j < kHq; ++j) {
+        const int c = c0 + threadIdx.x + kThreads * j;
+        if (c < NH) {
+          const float m = warp_max(fmaxf(fmaxf(fabsf(v[j].x), fabsf(v[j].y)), fmaxf(fabsf(v[j].z), fabsf(v[j].w))));
+          if (lane == 0) atomicMax(&s_max[c / Q4], __float_as_uint(m));   // non-negative floats order as integers
+        }
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x < TK) {
+      float upx, us;
+      prescale15(__uint_as_float(s_max[threadIdx.x]), upx, us);
+      s_up[threadIdx.x] = upx;
+      s_sc[threadIdx.x] = us * wa;
+    }
+    __syncthreads();
+  }
+  for (int c0 = 0; c0 < NH; c0 += kThreads * kHq) {
+    float4 v[kHq];
+#pragma unroll
+    for (int j = 0; j < kHq; ++j) {
+      const int c = c0 + threadIdx.x + kThreads * j, a = c / Q4;
+      v[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (c < NH && S.live_asg[a]) v[j] = ldg_f4_ordered(p.h + (size_t)a * I + 4 * (c - a * Q4));
+    }
+#pragma unroll
+    for (int j = 0; j < kHq; ++j) {
+      const int c = c0 + threadIdx.x + kThreads * j;
+      if (c < NH) {
+        const int a = c / Q4, q = c - a * Q4;
+        const float upx = s_up[a];
+        __half2 h0 = __floats2half2_rn(v[j].x * upx, v[j].y * upx), h1 = __floats2half2_rn(v[j].z * upx, v[j].w * upx);
+        *reinterpret_cast<uint2*>(hs + (size_t)a * HR + 4 * q) =
+            make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
+      }
+    }
+  }
 }
 
 // ============================================================== down
@@ -500,66 +564,12 @@ __global__ void __launch_bounds__(kThreads, 1) mma_down_kernel(const DecodeMmaAr
   pdl_wait();                // h comes from the previous launch
   pdl_trigger();
 
-  // h rows of the live assignments as B columns, f16 of h times the row's
-  // power of two: a fixed one from the clamp's bound on |h| when the limit is
-  // finite, else from each row's maximum (a first pass; one shared atomic
-  // per warp and row: with I a multiple of 128 a warp's 32 float4 lie in one
-  // row). Loads go out kHq at a time per thread.
-  constexpr int kHq = 4;
-  const int Q4 = I / 4, NH = TK * Q4;                      // NH % 32 == 0: warp-uniform bounds
+  stage_h(p, S, hs, s_max, s_up, s_sc, wa, fixed);
   __syncthreads();
-  if (!fixed) {
-    for (int c0 = 0; c0 < NH; c0 += kThreads * kHq) {
-      float4 v[kHq];
-#pragma unroll
-      for (int j = 0; j < kHq; ++j) {
-        const int c = c0 + threadIdx.x + kThreads * j, a = c / Q4;
-        v[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (c < NH && S.live_asg[a]) v[j] = ldg_f4_ordered(p.h + (size_t)a * I + 4 * (c - a * Q4));
-      }
-#pragma unroll
-      for (int j = 0; j < kHq; ++j) {
-        const int c = c0 + threadIdx.x + kThreads * j;
-        if (c < NH) {
-          const float m = warp_max(fmaxf(fmaxf(fabsf(v[j].x), fabsf(v[j].y)), fmaxf(fabsf(v[j].z), fabsf(v[j].w))));
-          if (lane == 0) atomicMax(&s_max[c / Q4], __float_as_uint(m));   // non-negative floats order as integers
-        }
-      }
-    }
-    __syncthreads();
-    if (threadIdx.x < TK) {
-      float upx, us;
-      prescale15(__uint_as_float(s_max[threadIdx.x]), upx, us);
-      s_up[threadIdx.x] = upx;
-      s_sc[threadIdx.x] = us * wa;
-    }
-    __syncthreads();
-  }
-  for (int c0 = 0; c0 < NH; c0 += kThreads * kHq) {
-    float4 v[kHq];
-#pragma unroll
-    for (int j = 0; j < kHq; ++j) {
-      const int c = c0 + threadIdx.x + kThreads * j, a = c / Q4;
-      v[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (c < NH && S.live_asg[a]) v[j] = ldg_f4_ordered(p.h + (size_t)a * I + 4 * (c - a * Q4));
-    }
-#pragma unroll
-    for (int j = 0; j < kHq; ++j) {
-      const int c = c0 + threadIdx.x + kThreads * j;
-      if (c < NH) {
-        const int a = c / Q4, q = c - a * Q4;
-        const float upx = s_up[a];
-        __half2 h0 = __floats2half2_rn(v[j].x * upx, v[j].y * upx), h1 = __floats2half2_rn(v[j].z * upx, v[j].w * upx);
-        *reinterpret_cast<uint2*>(hs + (size_t)a * HR + 4 * q) =
-            make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
-      }
-    }
-  }
   if (R > 0) tile_offsets(0);
 #pragma unroll
   for (int j = 0; j < kDepthD; ++j)
     if (j < Q) load(ring[j]);
-  __syncthreads();
 
   int cr = 0, cs = 0, cu = 0, crb = 0;
   const uint16_t* brow = hs;
@@ -610,6 +620,114 @@ __global__ void __launch_bounds__(kThreads, 1) mma_down_kernel(const DecodeMmaAr
   zero_dead_rows(S, TK, H, p.r);
 }
 
+// Down with bulk copies (one token's worth of assignments, I up to 1024):
+// a tile's 16 rows of codes are contiguous in the bank (8 I bytes), and so
+// are their scales (I bytes), so each warp pulls its tile into its own
+// shared-memory stage with two bulk copies (the TMA engine, no load slots of
+// the SM held) issued before the wait for h, and multiplies from there.
+// Every wait on a copy is bounded: when it runs out the status word gets the
+// timeout bit and the warp waits (bounded again) for the copy before it
+// leaves.
+
+__global__ void __launch_bounds__(kThreads, 1) mma_down_bulk_kernel(const DecodeMmaArgs p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ PlanS S;
+  __shared__ int s_cnt[kMaxE], s_off[kMaxE];
+  __shared__ float s_sc[kMaxAsg], s_up[kMaxAsg];
+  __shared__ uint32_t s_max[kMaxAsg];
+  __shared__ __align__(8) uint64_t s_bar[kWarps];
+  const int H = p.H, I = p.I, T = p.T, k = p.k, TK = T * k;
+  const int HR = I + kPad;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int NSD = I / 128;
+  const uint32_t SB = 9u * (uint32_t)I;                       // stage bytes: 8 I of codes, I of scales
+  uint8_t* stage = smem + (size_t)warp * SB;
+  uint16_t* hs = reinterpret_cast<uint16_t*>(smem + (size_t)kWarps * SB);   // [TK][HR] f16 bits
+  uint64_t* bar = &s_bar[warp];
+  if (lane == 0) {
+    mbar_init(bar, 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+
+  // The plan and the routing weights come from two launches back, complete
+  // when this grid starts: the plan, the tensor scales and this warp's first
+  // tile before the wait for h.
+  load_plan(p, S, s_cnt, s_off);
+  load_scales(S, p.down.tensor_scale, nullptr, S);
+  const int TPE = H / 16, NT = S.n_live * TPE, G = gridDim.x, GW = G * kWarps;
+  const int tile0 = blockIdx.x + G * warp;
+  const int R = tile0 < NT ? (NT - 1 - tile0) / GW + 1 : 0;
+  auto issue = [&](int rho) {                 // lane 0: tile rho of this warp into the stage
+    const int tau = tile0 + GW * rho;
+    const int u = tau / TPE, rb = tau - u * TPE;
+    const size_t row0 = (size_t)S.e[u] * H + 16 * rb;
+    mbar_arrive_expect_tx(bar, SB);
+    bulk_g2s(stage, p.down.codes + row0 * (I / 2), 8u * (uint32_t)I, bar);
+    bulk_g2s(stage + 8 * I, p.down.scales + row0 * (I / 16), (uint32_t)I, bar);
+  };
+  if (R > 0 && lane == 0) issue(0);
+  float wa = 0.f;
+  if (threadIdx.x < TK) wa = p.weights[threadIdx.x];
+  if (threadIdx.x < kMaxAsg) s_max[threadIdx.x] = 0u;
+  const bool fixed = p.h_up > 0.f;
+  if (fixed && threadIdx.x < TK) {
+    s_up[threadIdx.x] = p.h_up;
+    s_sc[threadIdx.x] = p.h_unscale * wa;
+  }
+
+  pdl_wait();                // h comes from the previous launch
+  pdl_trigger();
+  __syncthreads();
+  stage_h(p, S, hs, s_max, s_up, s_sc, wa, fixed);
+  __syncthreads();
+
+  for (int rho = 0; rho < R; ++rho) {
+    if (!mbar_wait(bar, (uint32_t)(rho & 1), p.wait_limit_ns)) {
+      if (lane == 0) set_status(p.status, kDevErrTimeout);
+      mbar_wait(bar, (uint32_t)(rho & 1), p.wait_limit_ns);   // the copy's own end, bounded again
+      break;
+    }
+    const int tau = tile0 + GW * rho;
+    const int cu = tau / TPE, crb = tau - cu * TPE;
+    const int n = S.n[cu], col0 = g < max(n, 1) ? g : 0;
+    const uint16_t* brow = hs + (size_t)S.sorted[S.off[cu] + col0] * HR + 32 * t;
+    const uint8_t* r0 = stage + g * (I / 2) + 16 * t;
+    const uint8_t* r1 = r0 + 8 * (I / 2);
+    const uint8_t* s0 = stage + 8 * I + g * (I / 16) + 2 * t;
+    const uint8_t* s1 = s0 + 8 * (I / 16);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int st = 0; st < NSD; ++st) {
+      const uint4 q0 = *reinterpret_cast<const uint4*>(r0 + 64 * st);
+      const uint4 q1 = *reinterpret_cast<const uint4*>(r1 + 64 * st);
+      const uint32_t sc = (uint32_t)*reinterpret_cast<const uint16_t*>(s0 + 8 * st) |
+                          ((uint32_t)*reinterpret_cast<const uint16_t*>(s1 + 8 * st) << 16);
+      const uint4* bp = reinterpret_cast<const uint4*>(brow + 128 * st);
+      const uint4 b[4] = {bp[0], bp[1], bp[2], bp[3]};
+      step_mma(acc, q0, q1, sc, b);
+    }
+    // lane (g, t) holds columns 2t, 2t + 1 of rows g, g + 8
+    const size_t row = 16 * (size_t)crb;
+    const float ts = S.tsa[cu];
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      const int col = 2 * t + h2;
+      if (col < n) {
+        const int a = S.sorted[S.off[cu] + col];
+        const float sc = s_sc[a] * ts;
+        p.r[(size_t)a * H + row + g] = acc[h2] * sc;
+        p.r[(size_t)a * H + row + g + 8] = acc[2 + h2] * sc;
+      }
+    }
+    if (rho + 1 < R) {
+      __syncwarp();                          // every lane done with the stage
+      fence_proxy_async_smem();
+      if (lane == 0) issue(rho + 1);
+    }
+  }
+  zero_dead_rows(S, TK, H, p.r);
+}
+
 int sm_count() {
   static int cached[64] = {0};
   int dev = 0;
@@ -628,6 +746,8 @@ size_t gate_up_smem(int T, int H) {
   return (((size_t)T * (H + kPad) * 2 + 15) & ~(size_t)15) + (size_t)2 * kSlots * kSeg * 256 * sizeof(float);
 }
 size_t down_smem(int T, int k, int I) { return (size_t)T * k * (I + kPad) * 2; }
+size_t down_bulk_smem(int T, int k, int I) { return (size_t)kWarps * 9 * I + down_smem(T, k, I); }
+constexpr size_t kBulkSmemBudget = 200 * 1024;   // with the static shared memory, under 227 KB
 
 constexpr size_t kSmemBudget = 200 * 1024;
 
@@ -672,6 +792,13 @@ cudaError_t launch_decode_mma_down(const DecodeMmaArgs& a, cudaStream_t st) {
     std::frexp(bound, &ex);
     b.h_up = (float)std::ldexp(1.0, 15 - ex);
     b.h_unscale = (float)std::ldexp(1.0, ex - 15);
+  }
+  b.wait_limit_ns = b.wait_limit_ns ? b.wait_limit_ns : kWaitLimitNs;
+  if (down_bulk_smem(a.T, a.k, a.I) <= kBulkSmemBudget && aligned16(a.down.scales)) {
+    const size_t bs = down_bulk_smem(a.T, a.k, a.I);
+    e = cudaFuncSetAttribute(mma_down_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bs);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(mma_down_bulk_kernel, dim3(sm_count()), dim3(kThreads), bs, st, b);
   }
   return launch_pdl(mma_down_kernel, dim3(sm_count()), dim3(kThreads), smem, st, b);
 }

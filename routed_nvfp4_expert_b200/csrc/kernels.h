@@ -65,6 +65,7 @@ struct DecodeMmaArgs {
   float* r;                          // fp32 [T*k, H] weighted routed rows
   uint32_t* status;
   float h_up, h_unscale;             // set by the down launcher: fixed power of two for h (0: per-row maxima)
+  unsigned long long wait_limit_ns;  // bound on each wait for a bulk copy (0: the library default)
 };
 // 1 <= T <= 8, H a multiple of 1024 up to 8192, I a multiple of 128 up to
 // 2048, k <= 16, T*k <= 128, E <= 1024, a bank below 4 GB, and the staged
