@@ -773,19 +773,31 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
   moe_plan_t plan = plan_at(b + L.plan, L.pl);
   uint32_t* status = (uint32_t*)(b + L.status);
   const bool decode = path == MOE_PATH_DECODE;
+  // the control block starts at zero: cleared by the router's GEMV (its first
+  // CTA, before any later kernel of the call can set a bit; no memset node
+  // in front of the router), else by a memset
+  const bool router_clears = decode && rnx::router_gemv_form(T, H);
+  if (!router_clears) RNX_CUDA(cudaMemsetAsync(status, 0, kCtrlBytes, st), "clear status");
 
-  RNX_CUDA(cudaMemsetAsync(status, 0, kCtrlBytes, st), "clear status");
-
-  // decode: the shared expert forks off to the auxiliary stream right away;
-  // its launches follow the router's (the router then does not wait behind
-  // them to start)
+  // decode: the shared expert forks off to the auxiliary stream right away.
+  // With one token its launches follow the router's (the router then does
+  // not wait behind them to start); with several tokens its two GEMVs are
+  // longer and run ahead of the router, clear of the top-k that follows it.
   SideStream* side = nullptr;
   const bool shared_aside = Is > 0 && decode;
   void* shared = Is > 0 ? (void*)(b + L.shared) : nullptr;
+  auto launch_shared = [&]() -> moe_status_t {
+    RNX_CUDA(rnx::launch_dense_gemv(H, Is, cfg->swiglu_limit, x, T, w->shared_gate, w->shared_up, w->shared_down,
+                                    shared, true, (float*)(b + L.shared_h), side->st),
+             "shared expert");
+    RNX_CUDA(cudaEventRecord(side->join, side->st), "join event");
+    return MOE_OK;
+  };
   if (shared_aside) {
     RNX_CUDA(side_stream(&side), "auxiliary stream");
     RNX_CUDA(cudaEventRecord(side->fork, st), "fork event");
     RNX_CUDA(cudaStreamWaitEvent(side->st, side->fork, 0), "fork wait");
+    if (T > 1 && (s = launch_shared()) != MOE_OK) return s;
   }
   // a handful of tokens: the tensor-core expert kernels (one CTA per SM,
   // weight rows streamed into registers), fed from the routing plan; the
@@ -797,14 +809,11 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
     const uint16_t* w3 = (const uint16_t*)(w->prepared + prepared_layout(cfg).router3);
     RNX_CUDA(rnx::launch_router_logits_tc(x, T, H, E, w3, logits, status, st), "router logits (tensor cores)");
   } else {
-    RNX_CUDA(rnx::launch_router_logits(x, T, H, E, w->router_w, logits, st, t1 ? xmax : nullptr), "router logits");
+    RNX_CUDA(rnx::launch_router_logits(x, T, H, E, w->router_w, logits, st, t1 ? xmax : nullptr,
+                                       router_clears ? status : nullptr, router_clears ? (int)(kCtrlBytes / 4) : 0),
+             "router logits");
   }
-  if (shared_aside) {
-    RNX_CUDA(rnx::launch_dense_gemv(H, Is, cfg->swiglu_limit, x, T, w->shared_gate, w->shared_up, w->shared_down,
-                                    shared, true, (float*)(b + L.shared_h), side->st),
-             "shared expert");
-    RNX_CUDA(cudaEventRecord(side->join, side->st), "join event");
-  }
+  if (shared_aside && T == 1 && (s = launch_shared()) != MOE_OK) return s;
   RNX_CUDA(mark(MOE_STAGE_TOPK, st), "stage event");
   // decode with a handful of tokens: selection and plan in one launch (the
   // permute stage then has zero length)

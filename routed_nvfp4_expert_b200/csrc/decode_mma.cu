@@ -165,7 +165,7 @@ constexpr int kMaxE = 1024;
 RNX_DEVICE void load_plan(const DecodeMmaArgs& p, PlanS& S, int* s_cnt, int* s_off) {
   const int TK = p.T * p.k, E = p.E, i = threadIdx.x;
   const int n_raw = min(min(max(p.active[0], 0), E), kMaxLive);   // active holds E + 1 entries
-  for (int e = i; e < E; e += kThreads) {
+  for (int e = i; e < E; e += blockDim.x) {
     s_cnt[e] = p.counts[e];
     s_off[e] = p.offsets[e];
   }
@@ -226,7 +226,7 @@ RNX_DEVICE void zero_dead_rows(const PlanS& S, int TK, int width, float* out) {
   const int n1 = (int)((long long)(blockIdx.x + 1) * width / gridDim.x);
   for (int a = 0; a < TK; ++a)
     if (!S.live_asg[a])
-      for (int c = n0 + (int)threadIdx.x; c < n1; c += kThreads) out[(size_t)a * width + c] = 0.f;
+      for (int c = n0 + (int)threadIdx.x; c < n1; c += blockDim.x) out[(size_t)a * width + c] = 0.f;
 }
 
 

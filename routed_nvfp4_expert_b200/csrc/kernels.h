@@ -81,6 +81,8 @@ cudaError_t launch_decode_mma_down(const DecodeMmaArgs& p, cudaStream_t st);
 // side jobs run only in the GEMV form (T <= 64).
 cudaError_t launch_router_logits(const uint16_t* x, int T, int H, int E, const float* wr, float* logits,
                                  cudaStream_t st, uint32_t* xmax = nullptr, uint32_t* zero = nullptr, int nzero = 0);
+// The GEMV form (the one with the side jobs above) serves these shapes.
+bool router_gemv_form(int T, int H);
 // max |row| as fp32 bits for R rows of K bf16 elements
 cudaError_t launch_row_absmax(const uint16_t* rows, int R, int K, uint32_t* out, cudaStream_t st);
 cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, int k, float rsf, int32_t* ids,

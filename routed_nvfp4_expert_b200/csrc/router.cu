@@ -44,7 +44,8 @@ __global__ void __launch_bounds__(kLogitThreads) router_logits_gemv(const uint16
   pdl_trigger();
   if (e == 0) {
     // side jobs of CTA 0: max |x_t| per token (fp32 bits; the expert pass
-    // pre-scales with it) and clearing the h-max array the gate/up pass fills
+    // pre-scales with it) and clearing the words asked for (the call's
+    // control block)
     for (int i = tid; i < nzero; i += kLogitThreads) zero[i] = 0u;
     if (xmax) {
       for (int t = 0; t < T; ++t) {
@@ -205,9 +206,26 @@ __global__ void __launch_bounds__(kT1PlanThreads) topk_plan_t1_kernel(const floa
   __shared__ float s_key[1][32 * PL];
   __shared__ float s_sig[1][32 * PL];
   __shared__ int s_ids[kMaxTopK];
+  // the correction bias is a weight: loaded before the wait for the logits
+  constexpr int kBq = (32 * PL + kT1PlanThreads - 1) / kT1PlanThreads;
+  float bq[kBq];
+#pragma unroll
+  for (int j = 0; j < kBq; ++j) {
+    const int e = threadIdx.x + kT1PlanThreads * j;
+    bq[j] = e < E ? bias[e] : 0.f;
+  }
   pdl_wait();
   pdl_trigger();
-  topk_keys<PL>(logits, bias, 0, 1, E, s_key, s_sig);
+#pragma unroll
+  for (int j = 0; j < kBq; ++j) {
+    const int e = threadIdx.x + kT1PlanThreads * j;
+    if (e < E) {
+      // sigmoid in double, rounded once to fp32; then an fp32 add of the bias
+      const float sg = (float)(1.0 / (1.0 + exp(-(double)logits[e])));
+      s_sig[0][e] = sg;
+      s_key[0][e] = __fadd_rn(sg, bq[j]);
+    }
+  }
   __syncthreads();
   if (threadIdx.x < 32) topk_warp<PL>(s_key[0], s_sig[0], 0, E, k, rsf, ids, weights, s_ids);
   __syncthreads();
@@ -281,9 +299,11 @@ cudaError_t launch_row_absmax(const uint16_t* rows, int R, int K, uint32_t* out,
   return cudaGetLastError();
 }
 
+bool router_gemv_form(int T, int H) { return T <= 64 && H <= 4 * kLogitThreads * kLogitMaxQ; }
+
 cudaError_t launch_router_logits(const uint16_t* x, int T, int H, int E, const float* wr, float* logits,
                                  cudaStream_t st, uint32_t* xmax, uint32_t* zero, int nzero) {
-  if (T <= 64 && H <= 4 * kLogitThreads * kLogitMaxQ) {
+  if (router_gemv_form(T, H)) {
     return launch_pdl(router_logits_gemv, dim3(E), dim3(kLogitThreads), 0, st, x, T, H, E, wr, logits, xmax, zero,
                       nzero);
   } else {
