@@ -788,7 +788,7 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
   void* shared = Is > 0 ? (void*)(b + L.shared) : nullptr;
   auto launch_shared = [&]() -> moe_status_t {
     RNX_CUDA(rnx::launch_dense_gemv(H, Is, cfg->swiglu_limit, x, T, w->shared_gate, w->shared_up, w->shared_down,
-                                    shared, true, (float*)(b + L.shared_h), side->st),
+                                    shared, true, (float*)(b + L.shared_h), side->st, true),
              "shared expert");
     RNX_CUDA(cudaEventRecord(side->join, side->st), "join event");
     return MOE_OK;

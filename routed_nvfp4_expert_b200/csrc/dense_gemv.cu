@@ -135,7 +135,7 @@ bf16_gemv_kernel(int K, int rows, int T, float limit, const void* __restrict__ a
 
 template <int MT, bool GU, bool OF>
 cudaError_t launch_t(int K, int rows, int T, float limit, const void* act, const uint16_t* w0,
-                     const uint16_t* w1, void* out, cudaStream_t st) {
+                     const uint16_t* w1, void* out, cudaStream_t st, bool bg) {
   const size_t smem = (size_t)MT * K * (GU ? 2 : 4);
   auto kern = bf16_gemv_kernel<MT, GU, OF>;
   static size_t cached_smem = 0;
@@ -150,29 +150,32 @@ cudaError_t launch_t(int K, int rows, int T, float limit, const void* act, const
   const int rows_per_item = kDgWarps * (GU ? 1 : 2);
   const int items = rows / rows_per_item;
   const int grid = std::max(1, std::min(items, kNumSMs * std::max(per_sm, 1)));
+  if (bg)
+    return launch_ex(kern, dim3(grid), dim3(kDgThreads), smem, st, GU, launch_priority_low(), K, rows, T, limit, act,
+                     w0, w1, out);
   return launch_pdl(kern, dim3(grid), dim3(kDgThreads), smem, st, K, rows, T, limit, act, w0, w1, out);
 }
 
 template <bool GU, bool OF>
 cudaError_t launch_mt(int K, int rows, int T, float limit, const void* act, const uint16_t* w0,
-                      const uint16_t* w1, void* out, cudaStream_t st) {
+                      const uint16_t* w1, void* out, cudaStream_t st, bool bg = false) {
   const size_t budget = 96 * 1024;
   const size_t es = GU ? 2 : 4;
-  if (T >= 8 && (size_t)8 * K * es <= budget) return launch_t<8, GU, OF>(K, rows, T, limit, act, w0, w1, out, st);
-  if (T >= 4 && (size_t)4 * K * es <= budget) return launch_t<4, GU, OF>(K, rows, T, limit, act, w0, w1, out, st);
-  if (T >= 2 && (size_t)2 * K * es <= budget) return launch_t<2, GU, OF>(K, rows, T, limit, act, w0, w1, out, st);
-  return launch_t<1, GU, OF>(K, rows, T, limit, act, w0, w1, out, st);
+  if (T >= 8 && (size_t)8 * K * es <= budget) return launch_t<8, GU, OF>(K, rows, T, limit, act, w0, w1, out, st, bg);
+  if (T >= 4 && (size_t)4 * K * es <= budget) return launch_t<4, GU, OF>(K, rows, T, limit, act, w0, w1, out, st, bg);
+  if (T >= 2 && (size_t)2 * K * es <= budget) return launch_t<2, GU, OF>(K, rows, T, limit, act, w0, w1, out, st, bg);
+  return launch_t<1, GU, OF>(K, rows, T, limit, act, w0, w1, out, st, bg);
 }
 
 }  // namespace
 
 cudaError_t launch_dense_gemv(int H, int I, float limit, const uint16_t* x, int T, const uint16_t* wg,
                               const uint16_t* wu, const uint16_t* wd, void* y, bool y_f32, float* hbuf,
-                              cudaStream_t st) {
-  cudaError_t err = launch_mt<true, true>(H, I, T, limit, x, wg, wu, hbuf, st);
+                              cudaStream_t st, bool background) {
+  cudaError_t err = launch_mt<true, true>(H, I, T, limit, x, wg, wu, hbuf, st, background);
   if (err != cudaSuccess) return err;
-  return y_f32 ? launch_mt<false, true>(I, H, T, 0.f, hbuf, wd, nullptr, y, st)
-               : launch_mt<false, false>(I, H, T, 0.f, hbuf, wd, nullptr, y, st);
+  return y_f32 ? launch_mt<false, true>(I, H, T, 0.f, hbuf, wd, nullptr, y, st, background)
+               : launch_mt<false, false>(I, H, T, 0.f, hbuf, wd, nullptr, y, st, background);
 }
 
 cudaError_t launch_dense_ffn(int H, int I, float limit, const uint16_t* x, int T, const uint16_t* wg,

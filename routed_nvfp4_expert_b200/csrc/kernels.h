@@ -11,21 +11,56 @@
 
 namespace rnx {
 
-// Launch with programmatic stream serialization (see pdl_wait / pdl_trigger).
+// Launch priorities (cudaLaunchAttributePriority): the library's kernels go
+// at the device's greatest priority, except the decode shared expert's on the
+// auxiliary stream, which runs at the least one, so that when SMs free up the
+// routed chain's CTAs are placed first.
+inline int launch_priority_high() {
+  static int prio = 1;                       // 1: not asked yet
+  if (prio == 1) {
+    int least = 0, greatest = 0;
+    prio = cudaDeviceGetStreamPriorityRange(&least, &greatest) == cudaSuccess ? greatest : 0;
+  }
+  return prio;
+}
+inline int launch_priority_low() {
+  static int prio = 1;
+  if (prio == 1) {
+    int least = 0, greatest = 0;
+    prio = cudaDeviceGetStreamPriorityRange(&least, &greatest) == cudaSuccess ? least : 0;
+  }
+  return prio;
+}
+
+// Launch with a priority and, when pdl is set, programmatic stream
+// serialization (see pdl_wait / pdl_trigger).
 template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-                       Args&&... args) {
+cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                      int prio, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  attr[n].id = cudaLaunchAttributePriority;
+  attr[n].val.priority = prio;
+  ++n;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = n;
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  return launch_ex(kern, grid, block, smem, st, true, launch_priority_high(), std::forward<Args>(args)...);
 }
 
 struct ExpertGemvArgs {
@@ -126,9 +161,12 @@ cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* scales, const fl
 
 // dense BF16 FFN (decode GEMV form): hbuf fp32 [T, I] scratch; y bf16 or
 // fp32 (y_f32) [T, H]
+// background: the decode site's shared expert on its auxiliary stream (least
+// priority; the down GEMV launched only once the gate/up one is done, so that
+// it holds no SM while it waits).
 cudaError_t launch_dense_gemv(int H, int I, float limit, const uint16_t* x, int T, const uint16_t* wg,
                               const uint16_t* wu, const uint16_t* wd, void* y, bool y_f32, float* hbuf,
-                              cudaStream_t st);
+                              cudaStream_t st, bool background = false);
 
 // BF16 GEMM on tcgen05 (kind::f16): out [M, N] = a [M, K] . b^T with b [N, K].
 // gate_up: b0 = gate rows, b1 = up rows; out = clamped_swiglu(a.b0^T, a.b1^T).
