@@ -413,7 +413,7 @@ def roofline_of(res, pk):
                 "traffic": read_traffic_profile(f"{stem}_{wl.name}")}
     routed = res["U"] * expert_bytes(wl)
     if decode_mma(wl):
-        kernel = "mma_gate_up_kernel + mma_down_kernel (128-bit weight loads, mma.sync m16n8k16; timed together)"
+        kernel = "mma_gate_up_kernel + mma_down_bulk_kernel (register-ring and bulk-copy weight streams, mma.sync m16n8k16; timed together)"
     else:
         kernel = "nvfp4_expert_gemv (gate/up + down launches, timed together)"
     achieved = routed / (res["kern_ms"] * 1e-3) / 1e9
