@@ -22,11 +22,12 @@
 //            and the clamped SwiGLU, rounds h to bf16, stores [P, I].
 //   DOWN:    256 output features; the epilogue applies the scales and the
 //            routing weight and writes fp32 rows [P, H] in the padded tile
-//            order (the unpermute is fused into the combine that follows,
-//            which sums them in fp32).
+//            order with plain coalesced stores after a transpose through
+//            shared memory (the unpermute is fused into the combine that
+//            follows, which sums them in fp32).
 //
-// Warp roles per CTA: warp 0 = TMA producer (5-stage ring, 38 KB per stage,
-// completions counted on the even CTA's barrier), warp 1 = MMA issuer (even
+// Warp roles per CTA: warp 0 = TMA producer (ring of 38 KB stages, 5 deep for
+// GATE_UP and 4 for DOWN; completions counted on the even CTA's barrier), warp 1 = MMA issuer (even
 // CTA only, one thread), warp 2 = TMEM allocator (both CTAs), warps 4-11 =
 // epilogue (warp w reads TMEM lane quadrant w % 4 and one half of the 256
 // accumulator columns, copies them to registers and releases the accumulator
@@ -46,17 +47,24 @@ namespace {
 constexpr int kPairM = 256;          // rows of one pair tile (128 per CTA)
 constexpr int kTileN = 256;          // MMA N
 constexpr int kStepK = 256;          // FP4 elements per stage (128 bytes per row)
-constexpr int kStages = 4;
+constexpr int kStages = 5;           // GATE_UP ring depth (DOWN: 4, its larger staging takes the fifth)
 constexpr int kABytes = 128 * 128;   // this CTA's A rows x 128 bytes
 constexpr int kBBytes = 128 * 128;   // this CTA's half of B
 constexpr int kSfaBytes = 2048;      // 4 atoms: this CTA's 128 rows, 4 K blocks
 constexpr int kSfbBytes = 4096;      // 8 atoms: all 256 B rows, 4 K blocks
 constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;   // 38 KB
-// epilogue staging: each epilogue warp owns two 32-row x 128-byte boxes in
-// the 128-byte swizzled layout of the output tensor map (TMA tensor stores)
+// epilogue staging per epilogue warp: GATE_UP, one 32-row x 128-byte box in
+// the 128-byte swizzled layout of the output tensor map (TMA tensor stores);
+// DOWN, 32 rows x 256 bytes through which its fp32 rows are transposed
 constexpr int kEpiBoxBytes = 32 * 128;
-constexpr int kEpiStageBytes = 2 * kEpiBoxBytes;                           // per warp
-constexpr int kSmemBytes = kStages * kStageBytes + 8 * kEpiStageBytes + 1024;
+template <bool GATE_UP>
+__host__ __device__ constexpr int stages_of() { return GATE_UP ? kStages : kStages - 1; }
+template <bool GATE_UP>
+__host__ __device__ constexpr int epi_stage_bytes_of() { return GATE_UP ? kEpiBoxBytes : 2 * kEpiBoxBytes; }
+template <bool GATE_UP>
+__host__ __device__ constexpr int smem_bytes_of() {
+  return stages_of<GATE_UP>() * kStageBytes + 8 * epi_stage_bytes_of<GATE_UP>() + 1024;
+}
 constexpr uint32_t kTxBytesPair = 2u * kStageBytes;                      // both CTAs' bytes of one stage
 constexpr int kFirstEpiWarp = 4;
 constexpr int kEpiWarps = 8;
@@ -75,7 +83,8 @@ struct PairParams {
   CUtensorMap tma_b1;      // up codes (GATE_UP), box 128 B x 64 rows
   CUtensorMap tma_sfa;     // A scale atoms viewed as [bytes/256, 256], box 256 x 8 (4 atoms)
   CUtensorMap tma_sfb0;    // GATE_UP: interleaved gate/up atoms; DOWN: down atoms; same view
-  CUtensorMap tma_out;     // output [P, out_cols]: GATE_UP bf16, box 64 x 32; DOWN fp32, box 32 x 32; SW128
+  CUtensorMap tma_out;     // GATE_UP output h [P, out_cols] bf16, box 64 x 32, SW128
+  float* out_f32;          // DOWN output [P, out_cols] fp32
   const float* row_scale;  // [P]
   const float* ts0;        // [E]
   const float* ts1;        // [E]
@@ -87,25 +96,51 @@ struct PairParams {
   float limit;
 };
 
-RNX_DEVICE int find_expert(const int32_t* s_toff, int E, int mt) {
-  int lo = 0, hi = E;                 // largest e with s_toff[e] <= mt
+// largest e with tile_offsets[e] <= mt (read through the read-only cache:
+// the table stays out of shared memory, which the ring and staging fill)
+RNX_DEVICE int find_expert(const int32_t* __restrict__ toff, int E, int mt) {
+  int lo = 0, hi = E;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (s_toff[mid] <= mt) lo = mid; else hi = mid;
+    if (__ldg(toff + mid) <= mt) lo = mid; else hi = mid;
   }
   return lo;
+}
+
+// DOWN epilogue transpose: lane r writes its row's 64 scaled fp32 values
+// into row r of a 32-row x 256-byte area (16-byte chunk c at position
+// c ^ (r & 15)) ...
+__device__ __forceinline__ void stage_rows_256(uint8_t* area, const uint32_t (&v)[64], float sc, int lane) {
+#pragma unroll
+  for (int c = 0; c < 16; ++c)
+    *reinterpret_cast<float4*>(area + lane * 256 + ((c ^ (lane & 15)) << 4)) =
+        make_float4(__uint_as_float(v[4 * c]) * sc, __uint_as_float(v[4 * c + 1]) * sc,
+                    __uint_as_float(v[4 * c + 2]) * sc, __uint_as_float(v[4 * c + 3]) * sc);
+  __syncwarp();
+}
+// ... and the warp stores the area row by row, 16 lanes per 256-byte row
+// segment (row r at dst + r * ld floats).
+__device__ __forceinline__ void store_rows_256(const uint8_t* area, float* dst, int ld, int c16, int rsub) {
+#pragma unroll 4
+  for (int i = 0; i < 16; ++i) {
+    const int r = 2 * i + rsub;
+    const float4 x4 = *reinterpret_cast<const float4*>(area + r * 256 + ((c16 ^ (r & 15)) << 4));
+    *reinterpret_cast<float4*>(dst + (size_t)r * ld) = x4;
+  }
+  __syncwarp();
 }
 
 template <bool GATE_UP>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     fp4_pair_gemm_kernel(const __grid_constant__ PairParams p) {
+  constexpr int kS = stages_of<GATE_UP>();
+  constexpr int kEpiStage = epi_stage_bytes_of<GATE_UP>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
+  __shared__ __align__(8) uint64_t full_bar[kS], empty_bar[kS];
   __shared__ __align__(8) uint64_t acc_full, acc_empty, mma_done;
   __shared__ uint32_t s_tmem;
   __shared__ volatile int abort_flag;
-  __shared__ int s_toff[kMaxExperts + 1];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();          // 0 = even CTA (issues the MMAs)
@@ -115,9 +150,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int n_ntiles = GATE_UP ? p.out_cols / 128 : p.out_cols / kTileN;
   const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
 
-  for (int i = threadIdx.x; i <= E; i += blockDim.x) s_toff[i] = p.tile_offsets[i];
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kS; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
@@ -135,7 +169,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   cluster_sync_all();          // barriers of both CTAs initialised, TMEM allocated in both
   tc_fence_after();
   const uint32_t tmem = s_tmem;
-  const int n_mtiles = s_toff[E];
+  const int n_mtiles = __ldg(p.tile_offsets + E);
   const int n_tiles = n_mtiles * n_ntiles;
 
   if (warp == 0) {
@@ -145,13 +179,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int tile = pair; tile < n_tiles && ok; tile += n_pairs) {
       const int mt = tile / n_ntiles, nt = tile - mt * n_ntiles;
-      const int e = find_expert(s_toff, E, mt);
+      const int e = find_expert(p.tile_offsets, E, mt);
       const int arow = mt * kPairM + 128 * (int)rank;   // this CTA's A rows
       const int rb = e * (p.bank_rows / 128);
       for (int ks = 0; ks < n_ksteps; ++ks, ++it) {
-        const int s = it % kStages;
-        const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-        if (__any_sync(0xffffffffu, !mbar_wait(&empty_bar[s], ph ^ 1u) || abort_flag)) {
+        const int s = it % kS;
+        const uint32_t ph = (uint32_t)(it / kS) & 1u;
+        if (__any_sync(0xffffffffu, !mbar_wait_poll(&empty_bar[s], ph ^ 1u) || abort_flag)) {
           ok = false;
           break;
         }
@@ -194,8 +228,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     // drain (even CTA: its full barriers count both CTAs' bytes)
     if (rank == 0)
-      for (int j = max(0, it - kStages); j < it; ++j)
-        if (!mbar_wait(&full_bar[j % kStages], (uint32_t)(j / kStages) & 1u) && lane == 0)
+      for (int j = max(0, it - kS); j < it; ++j)
+        if (!mbar_wait(&full_bar[j % kS], (uint32_t)(j / kS) & 1u) && lane == 0)
           set_status(p.status, kDevErrTimeout);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (even CTA)
@@ -217,9 +251,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         for (int ks = 0; ks < n_ksteps; ++ks, ++it) {
-          const int s = it % kStages;
-          const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-          if (__any_sync(0xffffffffu, !mbar_wait(&full_bar[s], ph) || abort_flag)) {
+          const int s = it % kS;
+          const uint32_t ph = (uint32_t)(it / kS) & 1u;
+          if (__any_sync(0xffffffffu, !mbar_wait_poll(&full_bar[s], ph) || abort_flag)) {
             ok = false;
             break;
           }
@@ -268,23 +302,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp >= kFirstEpiWarp) {
     // ------------------------------------------------------------ epilogue (both CTAs)
     // Each thread owns one accumulator row (its TMEM lane) and one column half.
-    // The finished values go to this warp's swizzled staging boxes (GATE_UP:
-    // one 32-row x 64-column bf16 box; DOWN: fp32, two passes of two 32-row x
-    // 32-column boxes); lane 0 writes each box with one TMA tensor store.
+    // The finished values go through this warp's swizzled staging box
+    // (GATE_UP: one 32-row x 64-column bf16 box, written by lane 0 with one
+    // TMA tensor store; DOWN: two 32-row x 64-column fp32 halves, read back
+    // row-contiguous and stored by all lanes).
     // Output rows are in the padded tile order (padding rows hold zeros).
     const int q = warp & 3;
     const int ch = (warp - kFirstEpiWarp) >> 2;
     const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
     const uint32_t acc_empty_even = mapa_shared(smem_u32(&acc_empty), 0);
-    uint8_t* boxes = smem + (size_t)kStages * kStageBytes + (size_t)(warp - kFirstEpiWarp) * kEpiStageBytes;
+    uint8_t* boxes = smem + (size_t)kS * kStageBytes + (size_t)(warp - kFirstEpiWarp) * kEpiStage;
+    // This lane's row metadata is read ahead so that no global load latency
+    // sits between an accumulator's completion and its release: two tiles
+    // ahead the expert, the row's assignment, its A unscale and the expert's
+    // tensor scales; one tile ahead the routing weight of that assignment.
+    struct RowMeta {
+      int asg;
+      float rs, t0, t1;
+    };
+    auto meta_of = [&](int tile) {
+      RowMeta m{-1, 0.f, 0.f, 0.f};
+      if (tile < n_tiles) {
+        const int mt = tile / n_ntiles;
+        const int e = find_expert(p.tile_offsets, E, mt);
+        const int row = mt * kPairM + 128 * (int)rank + q * 32 + lane;
+        m.asg = __ldg(p.tile_rows + row);
+        m.rs = __ldg(p.row_scale + row);
+        m.t0 = __ldg(p.ts0 + e);
+        if (GATE_UP) m.t1 = __ldg(p.ts1 + e);
+      }
+      return m;
+    };
+    auto weight_of = [&](const RowMeta& m) { return !GATE_UP && m.asg >= 0 ? __ldg(p.weights + m.asg) : 0.f; };
+    RowMeta m_cur = meta_of(pair), m_next = meta_of(pair + n_pairs);
+    float w_cur = weight_of(m_cur);
     int tc = 0;
     for (int tile = pair; tile < n_tiles; tile += n_pairs, ++tc) {
       const int mt = tile / n_ntiles, nt = tile - mt * n_ntiles;
-      const int e = find_expert(s_toff, E, mt);
       const int row0 = mt * kPairM + 128 * (int)rank + q * 32;   // first padded row of this warp
-      const int asg = p.tile_rows[row0 + lane];
-      const float rs = p.row_scale[row0 + lane];
-      if (__any_sync(0xffffffffu, !mbar_wait(&acc_full, (uint32_t)tc & 1u) || abort_flag)) {
+      const RowMeta m = m_cur;
+      const float w = w_cur;
+      m_cur = m_next;
+      w_cur = weight_of(m_next);
+      m_next = meta_of(tile + 2 * n_pairs);
+      if (__any_sync(0xffffffffu, !mbar_wait_poll(&acc_full, (uint32_t)tc & 1u) || abort_flag)) {
         if (lane == 0) {
           set_status(p.status, kDevErrTimeout);
           abort_flag = 1;
@@ -294,7 +355,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_after();
       if (GATE_UP) {
         // columns 128 ch .. +63 gate, +64 .. +127 up of features 64 ch .. +63
-        const float sg = rs * p.ts0[e], su = rs * p.ts1[e];
+        const float sg = m.rs * m.t0, su = m.rs * m.t1;
         uint32_t g[64], u[64];
         tmem_ld32(tq + 128 * ch, g);
         tmem_ld32(tq + 128 * ch + 32, g + 32);
@@ -332,38 +393,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
       } else {
-        // fp32 rows: 128 columns per thread, two passes of two 32-column boxes
-        const float sc = asg >= 0 ? rs * p.ts0[e] * p.weights[asg] : 0.f;
-        uint32_t v[128];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) tmem_ld32(tq + 128 * ch + 32 * j, v + 32 * j);
+        // fp32 rows: 128 columns per thread in two halves of 64, transposed
+        // through the warp's staging area (32 rows x 256 B, 16-byte chunks
+        // XOR-swizzled by the row, so both the row-per-lane writes and the
+        // row-contiguous reads take the minimum 4 wavefronts) and stored with
+        // plain 16-byte stores, 16 lanes per 256-byte row segment: each store
+        // instruction writes four whole 128-byte lines. The first half goes
+        // to shared memory and the second to registers before the
+        // accumulator is released, so no global store precedes the release.
+        const float sc = m.asg >= 0 ? m.rs * m.t0 * w : 0.f;
+        const int c16 = lane & 15, rsub = lane >> 4;
+        float* out_base = p.out_f32 + (size_t)row0 * p.out_cols + nt * kTileN + 128 * ch + 4 * c16;
+        uint32_t v[64];
+        tmem_ld32(tq + 128 * ch, v);
+        tmem_ld32(tq + 128 * ch + 32, v + 32);
+        tmem_ld_wait();
+        __syncwarp();                                  // the previous tile's reads of the area are done
+        stage_rows_256(boxes, v, sc, lane);
+        tmem_ld32(tq + 128 * ch + 64, v);
+        tmem_ld32(tq + 128 * ch + 96, v + 32);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(acc_empty_even);
-        const int col0 = nt * kTileN + 128 * ch;
-#pragma unroll
-        for (int pass = 0; pass < 2; ++pass) {
-          if (lane == 0) bulk_wait_read_all();      // the boxes' previous stores have read them
-          __syncwarp();
-#pragma unroll
-          for (int b = 0; b < 2; ++b)
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const int x = 64 * pass + 32 * b + 4 * c;
-              *reinterpret_cast<float4*>(boxes + b * kEpiBoxBytes + lane * 128 + ((c ^ (lane & 7)) << 4)) =
-                  make_float4(__uint_as_float(v[x]) * sc, __uint_as_float(v[x + 1]) * sc,
-                              __uint_as_float(v[x + 2]) * sc, __uint_as_float(v[x + 3]) * sc);
-            }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-#pragma unroll
-            for (int b = 0; b < 2; ++b) tma_store_2d(&p.tma_out, col0 + 64 * pass + 32 * b, row0, boxes + b * kEpiBoxBytes);
-            bulk_commit_group();
-          }
-          __syncwarp();
-        }
+        store_rows_256(boxes, out_base, p.out_cols, c16, rsub);
+        stage_rows_256(boxes, v, sc, lane);
+        store_rows_256(boxes, out_base + 64, p.out_cols, c16, rsub);
       }
     }
     if (lane == 0) bulk_wait_all();
@@ -406,13 +461,14 @@ cudaError_t launch_fp4_grouped_gemm(const Fp4GemmArgs& a, cudaStream_t st) {
   if (!atom_map(&p.tma_sfa, a.a_sf, a.P_max / 128 * KB)) return cudaErrorInvalidValue;
   // GATE_UP: interleaved gate/up atoms, 2 E I / 128 row blocks
   if (!atom_map(&p.tma_sfb0, a.b0_sf, (gu ? 2 * brows : brows) / 128 * KB)) return cudaErrorInvalidValue;
-  // output boxes: GATE_UP bf16 h, 64 columns x 32 rows; DOWN fp32 rows, 32 x 32
-  const bool out_ok =
-      gu ? make_tensor_map_2d(&p.tma_out, a.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.out_cols,
-                              (uint64_t)a.P_max, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B)
-         : make_tensor_map_2d(&p.tma_out, a.out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)a.out_cols,
-                              (uint64_t)a.P_max, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (!out_ok) return cudaErrorInvalidValue;
+  // output boxes (GATE_UP only): bf16 h, 64 columns x 32 rows
+  if (gu && !make_tensor_map_2d(&p.tma_out, a.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.out_cols,
+                                (uint64_t)a.P_max, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  // DOWN rows are stored 16 bytes at a time (whole 128-byte lines when the
+  // output is 256-byte aligned, as the workspace is)
+  if (!gu && (reinterpret_cast<uintptr_t>(a.out) % 16 || a.out_cols % kTileN)) return cudaErrorInvalidValue;
+  p.out_f32 = gu ? nullptr : static_cast<float*>(a.out);
   p.row_scale = a.row_scale;
   p.ts0 = a.ts0;
   p.ts1 = a.ts1;
@@ -426,13 +482,14 @@ cudaError_t launch_fp4_grouped_gemm(const Fp4GemmArgs& a, cudaStream_t st) {
   p.bank_rows = a.bank_rows;
   p.limit = a.limit;
   auto kern = gu ? fp4_pair_gemm_kernel<true> : fp4_pair_gemm_kernel<false>;
+  const int smem_bytes = gu ? smem_bytes_of<true>() : smem_bytes_of<false>();
   static bool attr_done[2] = {false, false};
   if (!attr_done[gu]) {
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
     if (err != cudaSuccess) return err;
     attr_done[gu] = true;
   }
-  kern<<<kNumSMs, kThreads, kSmemBytes, st>>>(p);   // 74 clusters of 2 (compile-time cluster shape)
+  kern<<<kNumSMs, kThreads, smem_bytes, st>>>(p);   // 74 clusters of 2 (compile-time cluster shape)
   return cudaGetLastError();
 }
 

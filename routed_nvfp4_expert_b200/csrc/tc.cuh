@@ -144,8 +144,14 @@ RNX_DEVICE uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
   return r;
 }
 
+// Arrive on a barrier of this or the peer CTA (a shared::cluster address)
+// with CTA-scope release. Used for "accumulator drained" signals, which order
+// only this thread's completed tcgen05.ld (tcgen05.wait::ld, then
+// tcgen05.fence::before_thread_sync) before the peer's MMAs; no data passes
+// through memory. A cluster-scope release would first wait for every global
+// load and store this thread has in flight, about 1-4 us under load.
 RNX_DEVICE void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 RNX_DEVICE bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {

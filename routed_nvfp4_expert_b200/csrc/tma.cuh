@@ -95,6 +95,18 @@ RNX_DEVICE bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned long long lim
   }
 }
 
+// Bounded wait as mbar_wait, polling try_wait without a suspend hint: for
+// waits on a critical path, where a suspended thread may resume late.
+RNX_DEVICE bool mbar_wait_poll(uint64_t* bar, uint32_t parity, unsigned long long limit_ns = kWaitLimitNs) {
+  if (limit_ns == 0) return mbar_test_wait(bar, parity);
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255u) == 0 && globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
 // Untiled bulk copy (TMA engine) of `bytes` from global memory into this
 // CTA's shared memory; completion is counted on `bar` as transaction bytes.
 // dst and src 16-byte aligned, bytes a multiple of 16. No multicast.
