@@ -96,13 +96,15 @@ struct PairParams {
   float limit;
 };
 
-// largest e with tile_offsets[e] <= mt (read through the read-only cache:
-// the table stays out of shared memory, which the ring and staging fill)
+// largest e with tile_offsets[e] <= mt. SMEM: the table was copied to shared
+// memory (DOWN); else it is read through the read-only cache (GATE_UP, whose
+// 5-stage ring and staging leave no room for it).
+template <bool SMEM>
 RNX_DEVICE int find_expert(const int32_t* __restrict__ toff, int E, int mt) {
   int lo = 0, hi = E;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (__ldg(toff + mid) <= mt) lo = mid; else hi = mid;
+    if ((SMEM ? toff[mid] : __ldg(toff + mid)) <= mt) lo = mid; else hi = mid;
   }
   return lo;
 }
@@ -141,6 +143,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t acc_full, acc_empty, mma_done;
   __shared__ uint32_t s_tmem;
   __shared__ volatile int abort_flag;
+  __shared__ int s_toff[GATE_UP ? 1 : kMaxExperts + 1];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();          // 0 = even CTA (issues the MMAs)
@@ -150,6 +153,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int n_ntiles = GATE_UP ? p.out_cols / 128 : p.out_cols / kTileN;
   const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
 
+  if (!GATE_UP)   // published by the cluster barrier below
+    for (int i = threadIdx.x; i <= E; i += blockDim.x) s_toff[i] = p.tile_offsets[i];
   if (threadIdx.x == 0) {
     for (int s = 0; s < kS; ++s) {
       mbar_init(&full_bar[s], 1);
@@ -170,6 +175,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = s_tmem;
   const int n_mtiles = __ldg(p.tile_offsets + E);
+  const int32_t* toff = GATE_UP ? p.tile_offsets : s_toff;
   const int n_tiles = n_mtiles * n_ntiles;
 
   if (warp == 0) {
@@ -179,7 +185,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int tile = pair; tile < n_tiles && ok; tile += n_pairs) {
       const int mt = tile / n_ntiles, nt = tile - mt * n_ntiles;
-      const int e = find_expert(p.tile_offsets, E, mt);
+      const int e = find_expert<!GATE_UP>(toff, E, mt);
       const int arow = mt * kPairM + 128 * (int)rank;   // this CTA's A rows
       const int rb = e * (p.bank_rows / 128);
       for (int ks = 0; ks < n_ksteps; ++ks, ++it) {
@@ -324,7 +330,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       RowMeta m{-1, 0.f, 0.f, 0.f};
       if (tile < n_tiles) {
         const int mt = tile / n_ntiles;
-        const int e = find_expert(p.tile_offsets, E, mt);
+        const int e = find_expert<!GATE_UP>(toff, E, mt);
         const int row = mt * kPairM + 128 * (int)rank + q * 32 + lane;
         m.asg = __ldg(p.tile_rows + row);
         m.rs = __ldg(p.row_scale + row);
@@ -342,9 +348,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int row0 = mt * kPairM + 128 * (int)rank + q * 32;   // first padded row of this warp
       const RowMeta m = m_cur;
       const float w = w_cur;
-      m_cur = m_next;
-      w_cur = weight_of(m_next);
-      m_next = meta_of(tile + 2 * n_pairs);
+      // issued right after the release, ahead of this tile's stores, so that
+      // they do not queue behind them
+      auto advance_meta = [&]() {
+        m_cur = m_next;
+        w_cur = weight_of(m_next);
+        m_next = meta_of(tile + 2 * n_pairs);
+      };
       if (__any_sync(0xffffffffu, !mbar_wait_poll(&acc_full, (uint32_t)tc & 1u) || abort_flag)) {
         if (lane == 0) {
           set_status(p.status, kDevErrTimeout);
@@ -365,6 +375,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(acc_empty_even);
+        advance_meta();
         const int col0 = nt * 128 + 64 * ch;         // first output column of this warp's box
         uint4 w4[8];
 #pragma unroll
@@ -416,6 +427,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(acc_empty_even);
+        advance_meta();
         store_rows_256(boxes, out_base, p.out_cols, c16, rsub);
         stage_rows_256(boxes, v, sc, lane);
         store_rows_256(boxes, out_base + 64, p.out_cols, c16, rsub);
