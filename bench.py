@@ -190,8 +190,9 @@ def measure(wl, args, rank, world, local_rank, dev, clocks=None):
         path = capi.PATH_PREFILL_W4A16 if getattr(args, "prefill_path", "w4a4") == "w4a16" else capi.PATH_PREFILL
     prefill = path != capi.PATH_DECODE
     T, H = wl.T, wl.H
-    if prefill:
-        capi.moe_prepare_weights(cfg, site)
+    # the block-scale atoms of the grouped GEMMs (prefill, and decode batches
+    # of 9 or more tokens): weight preparation, once, outside the timed region
+    capi.moe_prepare_weights(cfg, site)
 
     # rotating activations: a different routing every step (seeded per rank)
     n_x = 4 if prefill else 16
@@ -392,6 +393,13 @@ def dense_line(res, pk, world):
             "unit": "tokens/s", "ms_per_step": round(ms, 5), "roofline": roof}
 
 
+def decode_grouped(wl) -> bool:
+    """Decode batches of 9 or more tokens run their experts on the grouped
+    W4A16 GEMM (the weights' scale atoms are prepared); mirrors the library's
+    rule."""
+    return wl.kind == "decode" and wl.T >= 9 and wl.I % 128 == 0 and wl.H % 256 == 0
+
+
 def roofline_of(res, pk):
     """The dominant kernels' roofline from measure()'s kernel time."""
     wl = res["wl"]
@@ -414,6 +422,9 @@ def roofline_of(res, pk):
     routed = res["U"] * expert_bytes(wl)
     if decode_mma(wl):
         kernel = "mma_gate_up_kernel + mma_down_bulk_kernel (register-ring and bulk-copy weight streams, mma.sync m16n8k16; timed together)"
+    elif decode_grouped(wl):
+        kernel = ("w4a16_gemm_kernel (grouped W4A16 GEMM, tcgen05 kind::f16, padding halves skipped; "
+                  "gate/up + down launches, timed together)")
     else:
         kernel = "nvfp4_expert_gemv (gate/up + down launches, timed together)"
     achieved = routed / (res["kern_ms"] * 1e-3) / 1e9
@@ -434,8 +445,10 @@ def launches_per_step(wl, w4a16=False) -> int:
     # router, top-k + plan (one launch up to 8 tokens at E <= 320, else top-k
     # and the permute), expert gate/up, expert down, combine, and the shared
     # expert's two GEMVs on the auxiliary stream
+    # (grouped W4A16 GEMM: also the tile rows and the x gather)
     fused_plan = T <= 8 and wl.E <= 320 and T * wl.k <= 1024
-    return 7 if fused_plan else (8 if T * wl.k <= 1024 else 11)
+    n = 7 if fused_plan else (8 if T * wl.k <= 1024 else 11)
+    return n + (2 if decode_grouped(wl) else 0)
 
 
 def run_ours(args, rank, world, local_rank):
@@ -489,7 +502,8 @@ def run_ours(args, rank, world, local_rank):
     prefill = res["prefill"]
     path_name = (("prefill grouped GEMM (W4A16, tcgen05 kind::f16)" if res["w4a16"] else
                   "prefill grouped GEMM (W4A4, tcgen05 block-scaled FP4)") if prefill else
-                 "decode, tensor-core expert kernels (W4A16)" if decode_mma(wl) else "decode GEMV (W4A16)")
+                 "decode, tensor-core expert kernels (W4A16)" if decode_mma(wl) else
+                 "decode, grouped W4A16 GEMM (tcgen05 kind::f16)" if decode_grouped(wl) else "decode GEMV (W4A16)")
     n_launch = launches_per_step(wl, res["w4a16"])
     out = {
         "metric": METRIC,

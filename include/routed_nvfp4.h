@@ -428,13 +428,18 @@ moe_status_t nvfp4_dequant(const uint8_t* codes, const uint8_t* scales, const fl
  *     gate/up and down; moe_combine_f32. The shared expert runs on the
  *     library's auxiliary stream of this host thread and device, forked from
  *     and joined back into `stream` with events.
- *     T = 1 with H % 1024 == 0, H <= 8192, I % 128 == 0, I <= 2048, k <= 16,
+ *     T <= 8 with H % 1024 == 0, H <= 8192, I % 128 == 0, I <= 2048, k <= 16,
  *     E <= 1024: the expert projections run on the tensor cores, each warp
  *     loading its weight rows straight into registers with 128-bit loads and
  *     multiplying them with mma.sync (each E2M1 code times its E4M3 scale
  *     exact in f16, x or h scaled by a power of two into f16, fp32
- *     accumulation). Otherwise the GEMV kernels
- *     of nvfp4_expert_gemv.
+ *     accumulation). T >= 9 with I % 128 == 0, H % 256 == 0, w->prepared set
+ *     and ws of at least moe_workspace_size(cfg, T, MOE_PATH_DECODE) bytes:
+ *     the grouped W4A16 GEMM of MOE_PATH_PREFILL_W4A16 (x gathered to f16
+ *     rows, h in f16, the same exact-product numerics), skipping the 128-row
+ *     halves of the padded tile layout that hold only padding, with the down
+ *     GEMM writing r in assignment order. Otherwise the GEMV kernels of
+ *     nvfp4_expert_gemv.
  *   MOE_PATH_PREFILL_W4A16: the pages' prefill numerics: permute with the
  *     padded tile layout, x gathered to f16 rows (per-row power-of-two scale),
  *     grouped W4A16 GEMM gate/up (nvfp4_grouped_gemm_w4a16) with the clamped
@@ -453,8 +458,9 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
 
 /* Device pointers (inside ws) of the intermediates moe_forward leaves behind:
  * logits fp32 [T,E], ids int32 [T,k], weights fp32 [T,k], the plan; h (decode:
- * fp32 [T*k, I]; prefill: [P, I] in padded tile rows, bf16 on MOE_PATH_PREFILL,
- * f16 on MOE_PATH_PREFILL_W4A16); r (fp32; decode: [T*k, H] in token order;
+ * fp32 [T*k, I], or f16 [P, I] in padded tile rows when the decode ran on the
+ * grouped W4A16 GEMM; prefill: [P, I] in padded tile rows, bf16 on
+ * MOE_PATH_PREFILL, f16 on MOE_PATH_PREFILL_W4A16); r (fp32; decode: [T*k, H] in token order;
  * prefill: [P, H] in the padded tile order); shared (fp32 [T, H]; NULL when
  * Is == 0); and on MOE_PATH_PREFILL the NVFP4-encoded x and h in padded tile
  * rows (codes, scale atoms, row scales; NULL otherwise). Host-only pointer

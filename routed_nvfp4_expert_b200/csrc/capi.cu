@@ -2,6 +2,7 @@
 // and the order of launches. Every device step runs in the kernels of this
 // library; nothing here computes on the host.
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -179,6 +180,7 @@ struct WsLayout {
   size_t xq, xsf, xts, hq, hsf, hts;   // prefill: NVFP4 x and h in padded tile rows
   size_t bytes;
   PlanLayout pl;
+  bool grouped;   // decode layout with the grouped W4A16 GEMM's buffers
 };
 
 // Control block at the start of every workspace, cleared at the start of each
@@ -186,7 +188,18 @@ struct WsLayout {
 // arrival counter.
 constexpr size_t kCtrlBytes = 16;
 
-WsLayout ws_layout(const moe_config_t* c, int T, int path) {
+// Decode batches of more tokens than the tensor-core GEMV takes run their
+// experts on the grouped W4A16 GEMM (same numerics: 16-bit activations, each
+// weight exact in f16, fp32 accumulation) when the shapes fit it, the
+// prepared scale atoms exist and the workspace holds its buffers.
+constexpr int kDecodeGroupedMinT = 9;
+bool decode_grouped_shape(const moe_config_t* c, int T) {
+  return T >= kDecodeGroupedMinT && c->intermediate % 128 == 0 && c->hidden % 256 == 0;
+}
+
+// grouped: decode layout with the grouped GEMM's buffers (-1: whenever the
+// shapes allow it, as moe_workspace_size sizes it)
+WsLayout ws_layout(const moe_config_t* c, int T, int path, int grouped = -1) {
   WsLayout L{};
   const int E = c->num_experts, k = c->top_k, H = c->hidden, I = c->intermediate, Is = c->shared_intermediate;
   const size_t A = (size_t)T * k;
@@ -200,16 +213,19 @@ WsLayout ws_layout(const moe_config_t* c, int T, int path) {
   L.scratch = o; o = up(o + 4 * rnx::permute_scratch_ints((int)A, E));
   const bool w4 = path == MOE_PATH_PREFILL_W4A16;
   const bool pre = path == MOE_PATH_PREFILL || w4;
+  const bool grp = path == MOE_PATH_DECODE && (grouped < 0 ? decode_grouped_shape(c, T) : grouped != 0);
   const size_t P = (size_t)L.pl.P;
+  L.grouped = grp;
   // the routed rows r and the shared row are fp32 on every path (the combine
   // sums them in fp32 and rounds y once); h is fp32 at decode, 16-bit in the
-  // prefill's padded tile rows
-  L.h = o; o = up(o + (pre ? 2 * P : 4 * A) * I);
+  // prefill's padded tile rows (and in the decode's, on the grouped GEMM,
+  // whose down GEMM writes r in assignment order)
+  L.h = o; o = up(o + (pre ? 2 * P : grp ? std::max(2 * P, 4 * A) : 4 * A) * I);
   L.r = o; o = up(o + 4 * (pre ? P : A) * H);   // prefill: down rows in the padded tile order
   L.shared_h = o; o = up(o + 4 * (size_t)T * Is);
   L.shared = o; o = up(o + 4 * (size_t)T * H);
   L.xmax = o; o = up(o + 4 * (size_t)T);
-  if (w4) {                                   // x as f16 rows in the padded tile order, their unscales
+  if (w4 || grp) {                            // x as f16 rows in the padded tile order, their unscales
     L.xq = o; o = up(o + P * H * 2);
     L.xts = o; o = up(o + 4 * P);
   } else if (pre) {
@@ -306,8 +322,12 @@ rnx::W4a16GemmArgs w4a16_args(const moe_config_t* c, int proj, const uint16_t* a
   return g;
 }
 
+// The layout a call uses: the decode's grouped-GEMM layout whenever the
+// shapes allow it and the workspace holds it (moe_forward and
+// moe_workspace_views apply the same rule), else the plain one.
 moe_status_t check_ws(const moe_config_t* c, int T, int path, void* ws, size_t ws_bytes, WsLayout* L) {
-  *L = ws_layout(c, T, path);
+  const bool grp = path == MOE_PATH_DECODE && decode_grouped_shape(c, T) && ws_bytes >= ws_layout(c, T, path, 1).bytes;
+  *L = ws_layout(c, T, path, grp ? 1 : 0);
   if (!ws) return fail(MOE_ERR_WORKSPACE, "workspace is NULL");
   if (((uintptr_t)ws % kAlign) != 0) return fail(MOE_ERR_WORKSPACE, "workspace must be 256-byte aligned");
   if (ws_bytes < L->bytes) return fail(MOE_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, L->bytes);
@@ -803,6 +823,7 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
   // weight rows streamed into registers), fed from the routing plan; the
   // router's GEMV also leaves max |x_t| for their f16 pre-scale
   const bool t1 = decode && rnx::decode_mma_supported(T, H, I, E, k) && aligned16(x);
+  const bool grouped = decode && !t1 && L.grouped && w->prepared;
   uint32_t* xmax = (uint32_t*)(b + L.xmax);
   RNX_CUDA(mark(MOE_STAGE_ROUTER_LOGITS, st), "stage event");
   if (!decode && router_on_tensor_cores(cfg, T, w)) {
@@ -900,7 +921,30 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
     a.weights = wts;
     a.gate = w->gate; a.up = w->up; a.down = w->down;
     a.status = status;
-    if (t1) {
+    if (grouped) {
+      // a decode batch on the grouped W4A16 GEMM: x gathered to f16 rows of
+      // the padded tile order, 128-row halves of padding skipped; the down
+      // GEMM writes r [T*k, H] in assignment order (rows of assignments
+      // outside the local range are zeroed first, as no tile writes them)
+      const int64_t P = L.pl.P;
+      uint16_t* hh = (uint16_t*)(b + L.h);
+      uint16_t* xa = (uint16_t*)(b + L.xq);
+      float* xs = (float*)(b + L.xts);
+      const int32_t* used_tiles = plan.tile_offsets + E;
+      RNX_CUDA(rnx::launch_tile_rows(plan, E, P, st), "tile rows");
+      RNX_CUDA(rnx::launch_gather_x_f16(x, H, k, plan.tile_rows, used_tiles, P, xa, xs, st, true), "x gather (f16)");
+      if (cfg->local_begin > 0 || cfg->local_end < E)
+        RNX_CUDA(cudaMemsetAsync(r, 0, sizeof(float) * (size_t)T * k * H, st), "clear remote rows");
+      RNX_CUDA(mark(MOE_STAGE_EXPERT_GATE_UP, st), "stage event");
+      rnx::W4a16GemmArgs g = w4a16_args(cfg, MOE_PROJ_GATE_UP, xa, xs, P, plan, wts, w, hh, status);
+      g.sparse = true;
+      RNX_CUDA(rnx::launch_w4a16_grouped_gemm(g, st), "expert gate/up (grouped W4A16)");
+      RNX_CUDA(mark(MOE_STAGE_H_QUANT, st), "stage event");
+      RNX_CUDA(mark(MOE_STAGE_EXPERT_DOWN, st), "stage event");
+      g = w4a16_args(cfg, MOE_PROJ_DOWN, hh, nullptr, P, plan, wts, w, r, status);
+      g.sparse = true;
+      RNX_CUDA(rnx::launch_w4a16_grouped_gemm(g, st), "expert down (grouped W4A16)");
+    } else if (t1) {
       rnx::DecodeMmaArgs d{};
       d.T = T; d.H = H; d.I = I; d.E = E; d.k = k;
       d.lb = cfg->local_begin; d.le = cfg->local_end;
@@ -984,7 +1028,7 @@ moe_status_t moe_forward_decode_noalloc(const moe_config_t* cfg, const moe_weigh
                                         int32_t T, uint16_t* y, void* stream) {
   moe_status_t s;
   if ((s = check_cfg(cfg)) != MOE_OK || (s = check_T(T)) != MOE_OK) return s;
-  const size_t need = ws_layout(cfg, T, MOE_PATH_DECODE).bytes;
+  const size_t need = ws_layout(cfg, T, MOE_PATH_DECODE, 0).bytes;
   if (need > kNoAllocBytes)
     return fail(MOE_ERR_WORKSPACE, "moe_forward_decode_noalloc: T=%d needs %zu bytes of scratch, the built-in buffer "
                 "holds %zu", T, need, kNoAllocBytes);

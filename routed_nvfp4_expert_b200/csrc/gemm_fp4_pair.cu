@@ -462,6 +462,7 @@ bool atom_map(CUtensorMap* m, const uint8_t* base, int64_t n_atoms) {
 
 cudaError_t launch_fp4_grouped_gemm(const Fp4GemmArgs& a, cudaStream_t st) {
   if (a.E > kMaxExperts || a.P_max % kPairM) return cudaErrorInvalidValue;
+  if (a.P_max == 0) return cudaSuccess;   // no local expert: no rows, no tiles
   PairParams p;
   memset(&p, 0, sizeof p);
   const bool gu = a.gate_up;

@@ -73,7 +73,16 @@ struct W4Params {
   uint32_t* status;
   int E, K, out_cols, bank_rows;
   float limit;
+  int sparse;                    // see W4a16GemmArgs::sparse
 };
+
+// Sparse mode (a decode batch: a few tokens per expert): a 128-row half tile
+// whose first row is padding holds nothing but padding, since an expert's
+// real rows come first in its 256-row tiles. Every role skips such tiles
+// alike, before touching any ring or accumulator counter.
+RNX_DEVICE bool skip_half(const W4Params& p, int mt) {
+  return p.sparse && __ldg(p.tile_rows + (size_t)mt * kTileM) < 0;
+}
 
 RNX_DEVICE int find_expert(const int32_t* s_toff, int E, int t256) {
   int lo = 0, hi = E;                 // largest e with s_toff[e] <= t256
@@ -152,6 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
     bool ok = true;
     for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
       const int mt = tile / n_ntiles, nt = tile - mt * n_ntiles;   // n-tiles innermost
+      if (skip_half(p, mt)) continue;
       const int e = find_expert(s_toff, E, mt >> 1);
       // the tile's scale atoms: GATE_UP interleaved atoms 2 nt, 2 nt + 1 (64
       // gate + 64 up rows each); DOWN atoms 2 nt, 2 nt + 1 of 128 rows
@@ -214,6 +224,10 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
     int it = 0, tc = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++tc) {
+      if (skip_half(p, tile / n_ntiles)) {
+        --tc;   // skipped tiles take no accumulator turn
+        continue;
+      }
       const int b = tc & 1;
       const uint32_t use = (uint32_t)(tc >> 1);
       if (__any_sync(0xffffffffu, !mbar_wait(&acc_empty[b], (use & 1u) ^ 1u))) {
@@ -257,6 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
     int it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+      if (skip_half(p, tile / n_ntiles)) continue;
       for (int ks = 0; ks < n_ksteps; ++ks, ++it) {
         const int s = it % kStages, rs = it % kRawStages;
         const uint32_t ph = (uint32_t)(it / kStages) & 1u, rph = (uint32_t)(it / kRawStages) & 1u;
@@ -317,6 +332,10 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
     const int ch = (warp - kFirstEpiWarp) >> 2;
     int tc = 0;
     for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++tc) {
+      if (skip_half(p, tile / n_ntiles)) {
+        --tc;
+        continue;
+      }
       const int b = tc & 1;
       const uint32_t use = (uint32_t)(tc >> 1);
       const int mt = tile / n_ntiles, nt = tile - mt * n_ntiles;
@@ -360,7 +379,11 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
       } else {
         const int asg = p.tile_rows[row];
         const float sc = asg >= 0 ? rs * p.ts0[e] * p.weights[asg] : 0.f;
-        float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + (size_t)row * p.out_cols +
+        // sparse: row p goes to assignment row tile_rows[p]; padding rows are
+        // not written
+        const bool keep = !p.sparse || asg >= 0;
+        float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) +
+                                                (size_t)(p.sparse ? max(asg, 0) : row) * p.out_cols +
                                                 nt * kTileN + 128 * ch);
 #pragma unroll 1
         for (int hh = 0; hh < 2; ++hh) {
@@ -368,10 +391,12 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
           tmem_ld32(tq + 128 * ch + 64 * hh, v);
           tmem_ld32(tq + 128 * ch + 64 * hh + 32, v + 32);
           tmem_ld_wait();
+          if (keep) {
 #pragma unroll
-          for (int c = 0; c < 16; ++c)
-            dst[16 * hh + c] = make_float4(__uint_as_float(v[4 * c]) * sc, __uint_as_float(v[4 * c + 1]) * sc,
-                                           __uint_as_float(v[4 * c + 2]) * sc, __uint_as_float(v[4 * c + 3]) * sc);
+            for (int c = 0; c < 16; ++c)
+              dst[16 * hh + c] = make_float4(__uint_as_float(v[4 * c]) * sc, __uint_as_float(v[4 * c + 1]) * sc,
+                                             __uint_as_float(v[4 * c + 2]) * sc, __uint_as_float(v[4 * c + 3]) * sc);
+          }
         }
       }
       tc_fence_before();
@@ -394,13 +419,16 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
 __global__ void __launch_bounds__(256) gather_x_f16_kernel(const uint16_t* __restrict__ x, int H, int k,
                                                            const int32_t* __restrict__ tile_rows,
                                                            const int32_t* __restrict__ used_tiles, long long P,
-                                                           uint16_t* __restrict__ xa, float* __restrict__ unscale) {
+                                                           uint16_t* __restrict__ xa, float* __restrict__ unscale,
+                                                           int sparse) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long row = (long long)blockIdx.x * 8 + warp;
   if (row >= P) return;
   if (row >= (long long)*used_tiles * kRowsPerTile) return;   // past the last tile in use: never read
   const int a = tile_rows[row];
   uint4* dst = reinterpret_cast<uint4*>(xa + row * H);
+  // sparse: halves holding only padding are skipped by the GEMMs, never read
+  if (a < 0 && sparse && tile_rows[row & ~(long long)(kTileM - 1)] < 0) return;
   if (a < 0) {
     for (int g = lane; g < H / 8; g += 32) dst[g] = make_uint4(0, 0, 0, 0);
     if (lane == 0) unscale[row] = 0.f;
@@ -454,14 +482,16 @@ bool atom_map2(CUtensorMap* m, const uint8_t* base, int64_t n_atoms) {
 }  // namespace
 
 cudaError_t launch_gather_x_f16(const uint16_t* x, int H, int k, const int32_t* tile_rows, const int32_t* used_tiles,
-                                int64_t P, uint16_t* xa, float* unscale, cudaStream_t st) {
+                                int64_t P, uint16_t* xa, float* unscale, cudaStream_t st, bool sparse) {
   if (P <= 0) return cudaSuccess;
-  gather_x_f16_kernel<<<(unsigned)((P + 7) / 8), 256, 0, st>>>(x, H, k, tile_rows, used_tiles, P, xa, unscale);
+  gather_x_f16_kernel<<<(unsigned)((P + 7) / 8), 256, 0, st>>>(x, H, k, tile_rows, used_tiles, P, xa, unscale,
+                                                               sparse ? 1 : 0);
   return cudaGetLastError();
 }
 
 cudaError_t launch_w4a16_grouped_gemm(const W4a16GemmArgs& a, cudaStream_t st) {
   if (a.E > kMaxExperts || a.P_max % kRowsPerTile || a.K % kStepK) return cudaErrorInvalidValue;
+  if (a.P_max == 0) return cudaSuccess;   // no local expert: no rows, no tiles
   if (a.gate_up ? (a.out_cols % 128) : (a.out_cols % kTileN)) return cudaErrorInvalidValue;
   W4Params p;
   memset(&p, 0, sizeof p);
@@ -485,6 +515,7 @@ cudaError_t launch_w4a16_grouped_gemm(const W4a16GemmArgs& a, cudaStream_t st) {
   p.out_cols = a.out_cols;
   p.bank_rows = a.bank_rows;
   p.limit = a.limit;
+  p.sparse = a.sparse ? 1 : 0;
   auto kern = gu ? w4a16_gemm_kernel<true> : w4a16_gemm_kernel<false>;
   static bool attr_done[2] = {false, false};
   if (!attr_done[gu]) {

@@ -264,9 +264,10 @@ cudaError_t launch_fp4_grouped_gemm(const Fp4GemmArgs& a, cudaStream_t st);
 
 // x rows in the padded tile order as f16, each scaled by the power of two that
 // brings its max |x| into [2^14, 2^15); unscale[p] the inverse (0 on padding
-// rows). Rows at or past used_tiles * 256 are not written.
+// rows). Rows at or past used_tiles * 256 are not written, nor (sparse) the
+// rows of 128-row halves that hold only padding.
 cudaError_t launch_gather_x_f16(const uint16_t* x, int H, int k, const int32_t* tile_rows, const int32_t* used_tiles,
-                                int64_t P, uint16_t* xa, float* unscale, cudaStream_t st);
+                                int64_t P, uint16_t* xa, float* unscale, cudaStream_t st, bool sparse = false);
 
 struct W4a16GemmArgs {
   bool gate_up;
@@ -285,6 +286,9 @@ struct W4a16GemmArgs {
   const float* weights;            // [A] routing weights (DOWN)
   void* out;                       // GATE_UP: h f16 [P_max, I]; DOWN: rows fp32 [P_max, H]
   uint32_t* status;
+  bool sparse = false;             // decode batches: 128-row halves holding only padding are skipped, and
+                                   // DOWN writes row p to out row tile_rows[p] (rows fp32 [A, H] in
+                                   // assignment order; padding rows not written)
 };
 cudaError_t launch_w4a16_grouped_gemm(const W4a16GemmArgs& a, cudaStream_t st);
 

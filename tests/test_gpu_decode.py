@@ -161,13 +161,17 @@ def test_permute_out_of_range_id_sets_bounds_status():
 
 # ------------------------------------------------------------------ site
 
-def _forward(wl, inp, local=None, rsf=None, limit=None):
+def _forward(wl, inp, local=None, rsf=None, limit=None, prepared=True):
+    """One decode forward. With the prepared scale atoms, batches of 9 or more
+    tokens run on the grouped W4A16 GEMM; without them, on the GEMV kernels."""
     cfg = capi.config_for(wl, local)
     if rsf is not None:
         cfg.routed_scaling_factor = rsf
     if limit is not None:
         cfg.swiglu_limit = limit
     site = device_site(wl, inp)
+    if prepared:
+        capi.moe_prepare_weights(cfg, site)
     x = _x(inp)
     y = torch.empty_like(x)
     ws = capi.alloc_workspace(cfg, wl.T, capi.PATH_DECODE)
@@ -178,12 +182,14 @@ def _forward(wl, inp, local=None, rsf=None, limit=None):
     return y, logits, ws, v
 
 
-@pytest.mark.parametrize("name,T", [("tiny_t4", None), ("tiny_t4", 33), ("decode_t1", None), ("decode_t8", None),
-                                    ("decode_t32", None), ("decode_t64", None)])
-def test_moe_forward_decode_matches_oracle(name, T):
+@pytest.mark.parametrize("name,T,prepared", [("tiny_t4", None, True), ("tiny_t4", 33, True), ("tiny_t4", 33, False),
+                                             ("decode_t1", None, True), ("decode_t8", None, True),
+                                             ("decode_t32", None, True), ("decode_t32", None, False),
+                                             ("decode_t64", None, True)])
+def test_moe_forward_decode_matches_oracle(name, T, prepared):
     wl = workload(name, T)
     inp = site_inputs(wl)
-    y, lg, ws, v = _forward(wl, inp)
+    y, lg, ws, v = _forward(wl, inp, prepared=prepared)
     tokens = np.arange(wl.T) if wl.T <= 16 else np.random.default_rng(1).choice(wl.T, 16, replace=False)
     ref = OS.site_forward(inp, oracle_cfg(wl), "decode", tokens=tokens, gpu_logits=lg[tokens], want_parts=True)
     got = bf16_np(y)[tokens]
