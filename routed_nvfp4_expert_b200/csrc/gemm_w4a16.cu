@@ -24,6 +24,8 @@
 // is bounded; a timeout sets the device status word and winds the CTA down.
 // No TMA load uses cluster multicast.
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -416,15 +418,10 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
 // Padded tile rows of x as f16: row p holds token tile_rows[p] / k scaled by
 // the power of two that brings its max |x| into [2^14, 2^15) (exact for bf16),
 // unscale[p] the inverse; padding rows (and rows past the used tiles) zero.
-__global__ void __launch_bounds__(256) gather_x_f16_kernel(const uint16_t* __restrict__ x, int H, int k,
-                                                           const int32_t* __restrict__ tile_rows,
-                                                           const int32_t* __restrict__ used_tiles, long long P,
-                                                           uint16_t* __restrict__ xa, float* __restrict__ unscale,
-                                                           int sparse) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long row = (long long)blockIdx.x * 8 + warp;
-  if (row >= P) return;
-  if (row >= (long long)*used_tiles * kRowsPerTile) return;   // past the last tile in use: never read
+RNX_DEVICE void gather_row_f16(long long row, const uint16_t* __restrict__ x, int H, int k,
+                               const int32_t* __restrict__ tile_rows, uint16_t* __restrict__ xa,
+                               float* __restrict__ unscale, int sparse) {
+  const int lane = threadIdx.x & 31;
   const int a = tile_rows[row];
   uint4* dst = reinterpret_cast<uint4*>(xa + row * H);
   // sparse: halves holding only padding are skipped by the GEMMs, never read
@@ -464,6 +461,19 @@ __global__ void __launch_bounds__(256) gather_x_f16_kernel(const uint16_t* __res
   if (lane == 0) unscale[row] = ldexpf(1.0f, ex - 15);
 }
 
+// Warps stride over the rows of the tiles in use (rows past them are never
+// read); the grid is bounded by the SM count, as the row bound P covers the
+// worst routing.
+__global__ void __launch_bounds__(256) gather_x_f16_kernel(const uint16_t* __restrict__ x, int H, int k,
+                                                           const int32_t* __restrict__ tile_rows,
+                                                           const int32_t* __restrict__ used_tiles, long long P,
+                                                           uint16_t* __restrict__ xa, float* __restrict__ unscale,
+                                                           int sparse) {
+  const long long lim = min(P, (long long)*used_tiles * kRowsPerTile);
+  for (long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5); row < lim; row += (long long)gridDim.x * 8)
+    gather_row_f16(row, x, H, k, tile_rows, xa, unscale, sparse);
+}
+
 bool f16_map(CUtensorMap* m, const void* base, int K, int64_t rows) {
   return make_tensor_map_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)rows, kStepK, kTileM,
                             CU_TENSOR_MAP_SWIZZLE_128B);
@@ -484,8 +494,8 @@ bool atom_map2(CUtensorMap* m, const uint8_t* base, int64_t n_atoms) {
 cudaError_t launch_gather_x_f16(const uint16_t* x, int H, int k, const int32_t* tile_rows, const int32_t* used_tiles,
                                 int64_t P, uint16_t* xa, float* unscale, cudaStream_t st, bool sparse) {
   if (P <= 0) return cudaSuccess;
-  gather_x_f16_kernel<<<(unsigned)((P + 7) / 8), 256, 0, st>>>(x, H, k, tile_rows, used_tiles, P, xa, unscale,
-                                                               sparse ? 1 : 0);
+  const unsigned grid = (unsigned)std::min<int64_t>((P + 7) / 8, 8 * kNumSMs);
+  gather_x_f16_kernel<<<grid, 256, 0, st>>>(x, H, k, tile_rows, used_tiles, P, xa, unscale, sparse ? 1 : 0);
   return cudaGetLastError();
 }
 
