@@ -102,6 +102,81 @@ __global__ void __launch_bounds__(kLogitThreads) router_logits_gemv(const uint16
   }
 }
 
+// 9 to 64 tokens: read from L2 by every CTA, the token rows cost more than
+// the router matrix once T passes a few tokens. A 256-thread CTA owns four
+// expert rows (H <= 4096, in registers), so each token row is read once per
+// four experts; 8 tokens per pass, one warp sum per (expert, token), the
+// warps' partials added in a fixed order.
+constexpr int kRbExperts = 4, kRbThreads = 256, kRbQ = 4, kRbTokens = 8;
+
+__global__ void __launch_bounds__(kRbThreads) router_logits_gemv4(const uint16_t* __restrict__ x, int T, int H, int E,
+                                                                  const float* __restrict__ wr,
+                                                                  float* __restrict__ logits, uint32_t* zero,
+                                                                  int nzero) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int e0 = blockIdx.x * kRbExperts;
+  const int nq = H >> 2;
+  __shared__ float red[kRbThreads / 32][kRbExperts * kRbTokens];
+  float4 w[kRbExperts][kRbQ];
+#pragma unroll
+  for (int j = 0; j < kRbExperts; ++j)
+#pragma unroll
+    for (int i = 0; i < kRbQ; ++i) {
+      const int c = tid + kRbThreads * i;
+      w[j][i] = (c < nq && e0 + j < E) ? __ldg(reinterpret_cast<const float4*>(wr + (size_t)(e0 + j) * H) + c)
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  pdl_wait();
+  pdl_trigger();
+  if (blockIdx.x == 0)
+    for (int i = tid; i < nzero; i += kRbThreads) zero[i] = 0u;   // the call's control block
+  for (int t0 = 0; t0 < T; t0 += kRbTokens) {
+    float acc[kRbExperts][kRbTokens];
+#pragma unroll
+    for (int t = 0; t < kRbTokens; ++t) {
+      float2 xa[kRbQ], xb[kRbQ];
+#pragma unroll
+      for (int i = 0; i < kRbQ; ++i) {
+        const int c = tid + kRbThreads * i;
+        uint2 xv = make_uint2(0u, 0u);
+        if (t0 + t < T && c < nq) xv = *reinterpret_cast<const uint2*>(x + (size_t)(t0 + t) * H + 4 * c);
+        xa[i] = bf16x2_to_f32x2(xv.x);
+        xb[i] = bf16x2_to_f32x2(xv.y);
+      }
+#pragma unroll
+      for (int j = 0; j < kRbExperts; ++j) {
+        float a = 0.f;
+#pragma unroll
+        for (int i = 0; i < kRbQ; ++i) {
+          a = fmaf(w[j][i].x, xa[i].x, a);
+          a = fmaf(w[j][i].y, xa[i].y, a);
+          a = fmaf(w[j][i].z, xb[i].x, a);
+          a = fmaf(w[j][i].w, xb[i].y, a);
+        }
+        acc[j][t] = a;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kRbExperts; ++j)
+#pragma unroll
+      for (int t = 0; t < kRbTokens; ++t) {
+        const float v = warp_sum(acc[j][t]);
+        if (lane == 0) red[warp][j * kRbTokens + t] = v;
+      }
+    __syncthreads();
+    if (tid < kRbExperts * kRbTokens) {
+      const int j = tid / kRbTokens, t = tid % kRbTokens;
+      if (t0 + t < T && e0 + j < E) {
+        float v = red[0][tid];
+#pragma unroll
+        for (int q = 1; q < kRbThreads / 32; ++q) v += red[q][tid];
+        logits[(size_t)(t0 + t) * E + e0 + j] = v;
+      }
+    }
+    __syncthreads();
+  }
+}
+
 // Large T (prefill): a plain tiled fp32 GEMM on CUDA cores,
 // logits[T, E] = x[T, H] * Wr[E, H]^T. 64x64 output tile, 256 threads, 4x4 each.
 constexpr int kSgBM = 64, kSgBN = 64, kSgBK = 16;
@@ -303,7 +378,10 @@ bool router_gemv_form(int T, int H) { return T <= 64 && H <= 4 * kLogitThreads *
 
 cudaError_t launch_router_logits(const uint16_t* x, int T, int H, int E, const float* wr, float* logits,
                                  cudaStream_t st, uint32_t* xmax, uint32_t* zero, int nzero) {
-  if (router_gemv_form(T, H)) {
+  if (router_gemv_form(T, H) && T > kLogitTokens && !xmax && H <= kRbThreads * kRbQ * 4) {
+    return launch_pdl(router_logits_gemv4, dim3((E + kRbExperts - 1) / kRbExperts), dim3(kRbThreads), 0, st, x, T, H,
+                      E, wr, logits, zero, nzero);
+  } else if (router_gemv_form(T, H)) {
     return launch_pdl(router_logits_gemv, dim3(E), dim3(kLogitThreads), 0, st, x, T, H, E, wr, logits, xmax, zero,
                       nzero);
   } else {
