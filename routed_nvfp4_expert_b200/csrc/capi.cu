@@ -793,23 +793,38 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
   moe_plan_t plan = plan_at(b + L.plan, L.pl);
   uint32_t* status = (uint32_t*)(b + L.status);
   const bool decode = path == MOE_PATH_DECODE;
+  const bool t1 = decode && rnx::decode_mma_supported(T, H, I, E, k) && aligned16(x);
+  const bool grouped = decode && !t1 && L.grouped && w->prepared;
   // the control block starts at zero: cleared by the router's GEMV (its first
   // CTA, before any later kernel of the call can set a bit; no memset node
-  // in front of the router), else by a memset
-  const bool router_clears = decode && rnx::router_gemv_form(T, H);
+  // in front of the router), else by a memset (also when the shared expert's
+  // GEMMs, which can set a bit, run beside the router)
+  const bool router_clears = decode && rnx::router_gemv_form(T, H) && !grouped;
   if (!router_clears) RNX_CUDA(cudaMemsetAsync(status, 0, kCtrlBytes, st), "clear status");
 
   // decode: the shared expert forks off to the auxiliary stream right away.
   // With one token its launches follow the router's (the router then does
-  // not wait behind them to start); with several tokens its two GEMVs are
-  // longer and run ahead of the router, clear of the top-k that follows it.
+  // not wait behind them to start); with several tokens they are longer and
+  // run ahead of the router, clear of the top-k that follows it. Up to 8
+  // tokens the routed experts run on the tensor-core expert kernels (one CTA
+  // per SM, weight rows streamed into registers, fed from the routing plan;
+  // the router's GEMV also leaves max |x_t| for their f16 pre-scale). A
+  // larger batch takes the grouped W4A16 GEMM, and its shared expert the
+  // tcgen05 GEMMs (the GEMV form would stream the weights once per 8
+  // tokens), done beside the router, top-k and permute, before the grouped
+  // GEMM's persistent CTAs take every SM.
   SideStream* side = nullptr;
   const bool shared_aside = Is > 0 && decode;
   void* shared = Is > 0 ? (void*)(b + L.shared) : nullptr;
   auto launch_shared = [&]() -> moe_status_t {
-    RNX_CUDA(rnx::launch_dense_gemv(H, Is, cfg->swiglu_limit, x, T, w->shared_gate, w->shared_up, w->shared_down,
-                                    shared, true, (float*)(b + L.shared_h), side->st, true),
-             "shared expert");
+    if (grouped)
+      RNX_CUDA(rnx::launch_dense_ffn(H, Is, cfg->swiglu_limit, x, T, w->shared_gate, w->shared_up, w->shared_down,
+                                     shared, true, b + L.shared_h, status, side->st, 1),
+               "shared expert");
+    else
+      RNX_CUDA(rnx::launch_dense_gemv(H, Is, cfg->swiglu_limit, x, T, w->shared_gate, w->shared_up, w->shared_down,
+                                      shared, true, (float*)(b + L.shared_h), side->st, true),
+               "shared expert");
     RNX_CUDA(cudaEventRecord(side->join, side->st), "join event");
     return MOE_OK;
   };
@@ -819,11 +834,6 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* w, const 
     RNX_CUDA(cudaStreamWaitEvent(side->st, side->fork, 0), "fork wait");
     if (T > 1 && (s = launch_shared()) != MOE_OK) return s;
   }
-  // a handful of tokens: the tensor-core expert kernels (one CTA per SM,
-  // weight rows streamed into registers), fed from the routing plan; the
-  // router's GEMV also leaves max |x_t| for their f16 pre-scale
-  const bool t1 = decode && rnx::decode_mma_supported(T, H, I, E, k) && aligned16(x);
-  const bool grouped = decode && !t1 && L.grouped && w->prepared;
   uint32_t* xmax = (uint32_t*)(b + L.xmax);
   RNX_CUDA(mark(MOE_STAGE_ROUTER_LOGITS, st), "stage event");
   if (!decode && router_on_tensor_cores(cfg, T, w)) {

@@ -180,8 +180,8 @@ cudaError_t launch_dense_gemv(int H, int I, float limit, const uint16_t* x, int 
 
 cudaError_t launch_dense_ffn(int H, int I, float limit, const uint16_t* x, int T, const uint16_t* wg,
                              const uint16_t* wu, const uint16_t* wd, void* y, bool y_f32, void* hbuf,
-                             uint32_t* status, cudaStream_t st) {
-  if (T >= kDenseGemmMinT && I % 128 == 0 && H % 256 == 0) {
+                             uint32_t* status, cudaStream_t st, int min_t) {
+  if (T >= min_t && I % 128 == 0 && H % 256 == 0) {
     // the fp32 output (the site's shared row) carries h as two bf16 terms;
     // the bf16 output (the dense FFN entry point) rounds h to bf16
     uint16_t* hb = reinterpret_cast<uint16_t*>(hbuf);

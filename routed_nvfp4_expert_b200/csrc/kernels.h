@@ -194,14 +194,14 @@ cudaError_t launch_router_logits_tc(const uint16_t* x, int T, int H, int E, cons
 cudaError_t launch_router_split(const float* w, int E, int H, uint16_t* w3, cudaStream_t st);
 
 // Dense BF16 FFN, picking the GEMV form for small T and the tcgen05 GEMM for
-// T >= kDenseGemmMinT (when the shapes allow it).
+// T >= min_t (default kDenseGemmMinT; when the shapes allow it).
 constexpr int kDenseGemmMinT = 128;
 // hbuf: T*I*4 bytes (fp32 h in the GEMV form; in the GEMM form bf16 h, or,
 // when y_f32, h as two bf16 terms hi + lo).
 // y: bf16 [T, H], or fp32 when y_f32.
 cudaError_t launch_dense_ffn(int H, int I, float limit, const uint16_t* x, int T, const uint16_t* wg,
                              const uint16_t* wu, const uint16_t* wd, void* y, bool y_f32, void* hbuf,
-                             uint32_t* status, cudaStream_t st);
+                             uint32_t* status, cudaStream_t st, int min_t = kDenseGemmMinT);
 
 // ---------------------------------------------------------------- prefill (W4A4, tcgen05)
 
