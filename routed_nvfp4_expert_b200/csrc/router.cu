@@ -102,17 +102,18 @@ __global__ void __launch_bounds__(kLogitThreads) router_logits_gemv(const uint16
   }
 }
 
-// 9 to 64 tokens: read from L2 by every CTA, the token rows cost more than
-// the router matrix once T passes a few tokens. A 256-thread CTA owns four
-// expert rows (H <= 4096, in registers), so each token row is read once per
-// four experts; 8 tokens per pass, one warp sum per (expert, token), the
-// warps' partials added in a fixed order.
+// 2 to 64 tokens: read from L2 by every CTA, the token rows cost more than
+// the router matrix once T passes a token. A 256-thread CTA owns four expert
+// rows (H <= 4096, in registers), so each token row is read once per four
+// experts; 8 tokens per pass, one warp sum per (expert, token), the warps'
+// partials added in a fixed order. CTA t < T also leaves max |x_t| (fp32
+// bits) when asked.
 constexpr int kRbExperts = 4, kRbThreads = 256, kRbQ = 4, kRbTokens = 8;
 
 __global__ void __launch_bounds__(kRbThreads) router_logits_gemv4(const uint16_t* __restrict__ x, int T, int H, int E,
                                                                   const float* __restrict__ wr,
-                                                                  float* __restrict__ logits, uint32_t* zero,
-                                                                  int nzero) {
+                                                                  float* __restrict__ logits, uint32_t* xmax,
+                                                                  uint32_t* zero, int nzero) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int e0 = blockIdx.x * kRbExperts;
   const int nq = H >> 2;
@@ -130,6 +131,29 @@ __global__ void __launch_bounds__(kRbThreads) router_logits_gemv4(const uint16_t
   pdl_trigger();
   if (blockIdx.x == 0)
     for (int i = tid; i < nzero; i += kRbThreads) zero[i] = 0u;   // the call's control block
+  if (xmax && (int)blockIdx.x < T) {
+    const int t = blockIdx.x;
+    float m = 0.f;
+    for (int g = tid; g < H / 8; g += kRbThreads) {
+      const uint4 v = reinterpret_cast<const uint4*>(x + (size_t)t * H)[g];
+      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = bf16x2_to_f32x2(w4[j]);
+        m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+      }
+    }
+    m = warp_max(m);
+    if (lane == 0) red[warp][0] = m;
+    __syncthreads();
+    if (tid == 0) {
+      float a = red[0][0];
+#pragma unroll
+      for (int q = 1; q < kRbThreads / 32; ++q) a = fmaxf(a, red[q][0]);
+      xmax[t] = __float_as_uint(a);
+    }
+    __syncthreads();
+  }
   for (int t0 = 0; t0 < T; t0 += kRbTokens) {
     float acc[kRbExperts][kRbTokens];
 #pragma unroll
@@ -378,9 +402,10 @@ bool router_gemv_form(int T, int H) { return T <= 64 && H <= 4 * kLogitThreads *
 
 cudaError_t launch_router_logits(const uint16_t* x, int T, int H, int E, const float* wr, float* logits,
                                  cudaStream_t st, uint32_t* xmax, uint32_t* zero, int nzero) {
-  if (router_gemv_form(T, H) && T > kLogitTokens && !xmax && H <= kRbThreads * kRbQ * 4) {
-    return launch_pdl(router_logits_gemv4, dim3((E + kRbExperts - 1) / kRbExperts), dim3(kRbThreads), 0, st, x, T, H,
-                      E, wr, logits, zero, nzero);
+  const int rb_ctas = (E + kRbExperts - 1) / kRbExperts;
+  if (router_gemv_form(T, H) && T > 1 && H <= kRbThreads * kRbQ * 4 && (!xmax || T <= rb_ctas)) {
+    return launch_pdl(router_logits_gemv4, dim3(rb_ctas), dim3(kRbThreads), 0, st, x, T, H, E, wr, logits, xmax,
+                      zero, nzero);
   } else if (router_gemv_form(T, H)) {
     return launch_pdl(router_logits_gemv, dim3(E), dim3(kLogitThreads), 0, st, x, T, H, E, wr, logits, xmax, zero,
                       nzero);

@@ -32,8 +32,7 @@ def main():
     site = capi.site_to_device(inp)
     cfg = capi.config_for(wl)
     path = capi.PATH_DECODE if wl.kind == "decode" else capi.PATH_PREFILL
-    if path == capi.PATH_PREFILL:
-        capi.moe_prepare_weights(cfg, site)
+    capi.moe_prepare_weights(cfg, site)   # the grouped GEMMs' scale atoms (prefill, decode batches >= 9)
     x = capi.bf16_tensor(inp["x"])
     y = torch.empty_like(x)
     ws = capi.alloc_workspace(cfg, wl.T, path)
