@@ -264,9 +264,54 @@ __global__ void __launch_bounds__(kThreads, 1) mma_gate_up_kernel(const DecodeMm
   const int slot = warp / kSeg, seg = warp % kSeg;
   const int NS = H / 512;
 
-  pdl_wait();              // the plan and max |x| come from earlier launches
+  // x first (the tokens as B columns: f16 of x times the token's power of
+  // two, in passes of kXq 16-byte chunks per thread), before the wait: x is
+  // the call's input, and max |x_t| comes from the launch two back (the
+  // router), which had completed when the previous launch passed its own
+  // wait, before this one could start. The plan, from the previous launch,
+  // is read after the wait.
+  constexpr int kXq = 4;
+  const int NXC = T * (H / 8);
+  float xup[kMaxCols];
+#pragma unroll
+  for (int tk = 0; tk < kMaxCols; ++tk) {
+    float un = 1.f;
+    xup[tk] = 1.f;
+    if (tk < T) prescale15(__uint_as_float(p.xmax[tk]), xup[tk], un);
+    if (threadIdx.x == 0 && tk < T) s_unscale[tk] = un;
+  }
+  for (int c0 = 0; c0 < NXC; c0 += kThreads * kXq) {
+    uint4 xv[kXq];
+#pragma unroll
+    for (int j = 0; j < kXq; ++j) {
+      const int cc = c0 + threadIdx.x + kThreads * j;
+      if (cc < NXC) xv[j] = ldg_ordered(p.x + (size_t)(cc / (H / 8)) * H + 8 * (cc % (H / 8)));
+    }
+#pragma unroll
+    for (int j = 0; j < kXq; ++j) {
+      const int cc = c0 + threadIdx.x + kThreads * j;
+      if (cc < NXC) {
+        const int tk = cc / (H / 8), q = cc - tk * (H / 8);
+        float up = xup[0];
+#pragma unroll
+        for (int z = 1; z < kMaxCols; ++z)
+          if (z == tk) up = xup[z];
+        const uint32_t w4[4] = {xv[j].x, xv[j].y, xv[j].z, xv[j].w};
+        uint32_t o[4];
+#pragma unroll
+        for (int z = 0; z < 4; ++z) {
+          const float2 f = bf16x2_to_f32x2(w4[z]);
+          __half2 h2 = __floats2half2_rn(f.x * up, f.y * up);
+          o[z] = *reinterpret_cast<uint32_t*>(&h2);
+        }
+        *reinterpret_cast<uint4*>(xs + (size_t)tk * XR + 8 * q) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+    }
+  }
+  pdl_wait();
   pdl_trigger();
   load_plan(p, S, s_cnt, s_off);
+  load_scales(S, p.gate.tensor_scale, p.up.tensor_scale, S);
   const int BPE = I / 8, NB = S.n_live * BPE, G = gridDim.x;
   // this CTA's blocks: blockIdx + G j for j < nb; unit i = blocks (2i, 2i + 1)
   // of that list (one token), or tile blockIdx + G i = blocks (2 tile, 2 tile
@@ -290,9 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1) mma_gate_up_kernel(const DecodeMm
     }
   };
 
-  // x first (the tokens as B columns: f16 of x times the token's power of
-  // two, in passes of kXq 16-byte chunks per thread), then the weight ring.
-  // Load cursor: round lr, step ls, lane byte offsets of its two rows
+  // Weight ring load cursor: round lr, step ls, lane byte offsets of its two rows
   // (32-bit: a bank's codes are below 4 GB).
   int lr = 0, ls = 0;
   uint32_t oca = 0, ocb = 0, osa = 0, osb = 0;
@@ -323,45 +366,6 @@ __global__ void __launch_bounds__(kThreads, 1) mma_gate_up_kernel(const DecodeMm
   };
   GuRegs ring[kDepthGU];
 
-  constexpr int kXq = 4;
-  const int NXC = T * (H / 8);
-  float xup[kMaxCols];
-#pragma unroll
-  for (int tk = 0; tk < kMaxCols; ++tk) {
-    float un = 1.f;
-    xup[tk] = 1.f;
-    if (tk < T) prescale15(__uint_as_float(p.xmax[tk]), xup[tk], un);
-    if (threadIdx.x == 0 && tk < T) s_unscale[tk] = un;
-  }
-  for (int c0 = 0; c0 < NXC; c0 += kThreads * kXq) {
-    uint4 xv[kXq];
-#pragma unroll
-    for (int j = 0; j < kXq; ++j) {
-      const int cc = c0 + threadIdx.x + kThreads * j;
-      if (cc < NXC) xv[j] = ldg_ordered(p.x + (size_t)(cc / (H / 8)) * H + 8 * (cc % (H / 8)));
-    }
-    if (c0 == 0) load_scales(S, p.gate.tensor_scale, p.up.tensor_scale, S);
-#pragma unroll
-    for (int j = 0; j < kXq; ++j) {
-      const int cc = c0 + threadIdx.x + kThreads * j;
-      if (cc < NXC) {
-        const int tk = cc / (H / 8), q = cc - tk * (H / 8);
-        float up = xup[0];
-#pragma unroll
-        for (int z = 1; z < kMaxCols; ++z)
-          if (z == tk) up = xup[z];
-        const uint32_t w4[4] = {xv[j].x, xv[j].y, xv[j].z, xv[j].w};
-        uint32_t o[4];
-#pragma unroll
-        for (int z = 0; z < 4; ++z) {
-          const float2 f = bf16x2_to_f32x2(w4[z]);
-          __half2 h2 = __floats2half2_rn(f.x * up, f.y * up);
-          o[z] = *reinterpret_cast<uint32_t*>(&h2);
-        }
-        *reinterpret_cast<uint4*>(xs + (size_t)tk * XR + 8 * q) = make_uint4(o[0], o[1], o[2], o[3]);
-      }
-    }
-  }
   // the weight ring goes out once x is staged (issued earlier, its requests
   // would hold up the staging's own loads in the memory queues), and after
   // the barrier: a warp whose ring loads stall on a full memory queue holds
