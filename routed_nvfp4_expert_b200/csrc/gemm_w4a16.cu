@@ -20,7 +20,8 @@
 // the (m-tile, n-tile) list with the n-tiles innermost, two 256-column
 // accumulators alternating between tiles.
 // Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer, warp 2 = TMEM
-// allocator, warps 4-11 = epilogue, warps 12-15 = dequantisation. Every wait
+// allocator, warps 4-7 = epilogue (one per TMEM lane quadrant), warps 8-15 =
+// dequantisation (the part that bounds a tile's time). Every wait
 // is bounded; a timeout sets the device status word and winds the CTA down.
 // No TMA load uses cluster multicast.
 
@@ -48,9 +49,9 @@ constexpr int kRawSfBytes = 1024;               // 2 scale atoms (256 rows x 4 b
 constexpr int kRawBytes = kRawCodeBytes + kRawSfBytes;
 constexpr int kSmemBytes = kStages * kStageBytes + kRawStages * kRawBytes + 1024;
 constexpr int kFirstEpiWarp = 4;
-constexpr int kEpiWarps = 8;
-constexpr int kFirstDqWarp = 12;
-constexpr int kDqWarps = 4;
+constexpr int kEpiWarps = 4;                    // one per TMEM lane quadrant, both column halves
+constexpr int kFirstDqWarp = 8;
+constexpr int kDqWarps = 8;                     // the dequantisation bounds the launch: most warps go there
 constexpr int kThreads = (kFirstDqWarp + kDqWarps) * 32;   // 512
 constexpr uint32_t kTmemCols = 512;                        // two 256-column accumulators
 constexpr int kMaxExperts = 1024;
@@ -268,7 +269,8 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
     if (!mbar_wait(&mma_done, 0) && lane == 0) set_status(p.status, kDevErrTimeout);
   } else if (warp >= kFirstDqWarp) {
     // ------------------------------------------------------------ dequantisation
-    // Thread t of the four warps owns B rows t and t + 128 of every stage.
+    // Thread t of the dequantisation warps owns B rows t, t + 32 kDqWarps, ...
+    // of every stage.
     const int t = threadIdx.x - kFirstDqWarp * 32;
     int it = 0;
     bool ok = true;
@@ -285,8 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
         const uint8_t* r = raw + (size_t)rs * kRawBytes;
         uint8_t* sB = smem + (size_t)s * kStageBytes + kABytes;
 #pragma unroll
-        for (int hsel = 0; hsel < 2; ++hsel) {
-          const int row = t + 128 * hsel;
+        for (int row = t; row < kTileN; row += kDqWarps * 32) {
           // scale atom of this B row (see the producer): GATE_UP rows 0..127
           // gate, 128..255 up, 64 of each per interleaved atom
           int j, m;
@@ -331,7 +332,6 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
   } else if (warp >= kFirstEpiWarp) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
-    const int ch = (warp - kFirstEpiWarp) >> 2;
     int tc = 0;
     for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++tc) {
       if (skip_half(p, tile / n_ntiles)) {
@@ -353,51 +353,55 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
       }
       tc_fence_after();
       const uint32_t tq = tmem + 256u * b + ((uint32_t)(q * 32) << 16);
-      // the accumulator in two halves (fewer live registers); the buffer is
-      // released after both, the MMAs meanwhile fill the other one
-      if (GATE_UP) {
-        const float sg = rs * p.ts0[e], su = rs * p.ts1[e];
-        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) + (size_t)row * p.out_cols +
-                                              nt * 128 + 64 * ch);
+      // the accumulator in column halves ch and, within each, two passes
+      // (fewer live registers); the buffer is released after all of them,
+      // the MMAs meanwhile fill the other one
 #pragma unroll 1
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t g[32], u[32];
-          tmem_ld32(tq + 64 * ch + 32 * hh, g);
-          tmem_ld32(tq + 128 + 64 * ch + 32 * hh, u);
-          tmem_ld_wait();
+      for (int ch = 0; ch < 2; ++ch) {
+        if (GATE_UP) {
+          const float sg = rs * p.ts0[e], su = rs * p.ts1[e];
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) + (size_t)row * p.out_cols +
+                                                nt * 128 + 64 * ch);
+#pragma unroll 1
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t g[32], u[32];
+            tmem_ld32(tq + 64 * ch + 32 * hh, g);
+            tmem_ld32(tq + 128 + 64 * ch + 32 * hh, u);
+            tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t w[4];
+            for (int c = 0; c < 4; ++c) {
+              uint32_t w[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int k0 = 8 * c + 2 * i;
-              w[i] = pack_f16x2_sat(
-                  clamped_swiglu_fast(__uint_as_float(g[k0]) * sg, __uint_as_float(u[k0]) * su, p.limit),
-                  clamped_swiglu_fast(__uint_as_float(g[k0 + 1]) * sg, __uint_as_float(u[k0 + 1]) * su, p.limit));
+              for (int i = 0; i < 4; ++i) {
+                const int k0 = 8 * c + 2 * i;
+                w[i] = pack_f16x2_sat(
+                    clamped_swiglu_fast(__uint_as_float(g[k0]) * sg, __uint_as_float(u[k0]) * su, p.limit),
+                    clamped_swiglu_fast(__uint_as_float(g[k0 + 1]) * sg, __uint_as_float(u[k0 + 1]) * su, p.limit));
+              }
+              dst[4 * hh + c] = make_uint4(w[0], w[1], w[2], w[3]);
             }
-            dst[4 * hh + c] = make_uint4(w[0], w[1], w[2], w[3]);
           }
-        }
-      } else {
-        const int asg = p.tile_rows[row];
-        const float sc = asg >= 0 ? rs * p.ts0[e] * p.weights[asg] : 0.f;
-        // sparse: row p goes to assignment row tile_rows[p]; padding rows are
-        // not written
-        const bool keep = !p.sparse || asg >= 0;
-        float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) +
-                                                (size_t)(p.sparse ? max(asg, 0) : row) * p.out_cols +
-                                                nt * kTileN + 128 * ch);
+        } else {
+          const int asg = p.tile_rows[row];
+          const float sc = asg >= 0 ? rs * p.ts0[e] * p.weights[asg] : 0.f;
+          // sparse: row p goes to assignment row tile_rows[p]; padding rows are
+          // not written
+          const bool keep = !p.sparse || asg >= 0;
+          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) +
+                                                  (size_t)(p.sparse ? max(asg, 0) : row) * p.out_cols +
+                                                  nt * kTileN + 128 * ch);
 #pragma unroll 1
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t v[64];
-          tmem_ld32(tq + 128 * ch + 64 * hh, v);
-          tmem_ld32(tq + 128 * ch + 64 * hh + 32, v + 32);
-          tmem_ld_wait();
-          if (keep) {
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t v[64];
+            tmem_ld32(tq + 128 * ch + 64 * hh, v);
+            tmem_ld32(tq + 128 * ch + 64 * hh + 32, v + 32);
+            tmem_ld_wait();
+            if (keep) {
 #pragma unroll
-            for (int c = 0; c < 16; ++c)
-              dst[16 * hh + c] = make_float4(__uint_as_float(v[4 * c]) * sc, __uint_as_float(v[4 * c + 1]) * sc,
-                                             __uint_as_float(v[4 * c + 2]) * sc, __uint_as_float(v[4 * c + 3]) * sc);
+              for (int c = 0; c < 16; ++c)
+                dst[16 * hh + c] = make_float4(__uint_as_float(v[4 * c]) * sc, __uint_as_float(v[4 * c + 1]) * sc,
+                                               __uint_as_float(v[4 * c + 2]) * sc, __uint_as_float(v[4 * c + 3]) * sc);
+            }
           }
         }
       }
