@@ -172,7 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
       const int KB = p.K / 64;
       for (int ks = 0; ks < n_ksteps; ++ks) {
         const int rs = it_r % kRawStages;
-        if (__any_sync(0xffffffffu, !mbar_wait(&raw_empty[rs], ((uint32_t)(it_r / kRawStages) & 1u) ^ 1u) ||
+        if (__any_sync(0xffffffffu, !mbar_wait_poll(&raw_empty[rs], ((uint32_t)(it_r / kRawStages) & 1u) ^ 1u) ||
                                         abort_flag)) {
           ok = false;
           break;
@@ -194,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
         __syncwarp();
         ++it_r;
         const int s = it_a % kStages;
-        if (__any_sync(0xffffffffu, !mbar_wait(&empty_bar[s], ((uint32_t)(it_a / kStages) & 1u) ^ 1u) ||
+        if (__any_sync(0xffffffffu, !mbar_wait_poll(&empty_bar[s], ((uint32_t)(it_a / kStages) & 1u) ^ 1u) ||
                                         abort_flag)) {
           ok = false;
           break;
@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
       }
       const int b = tc & 1;
       const uint32_t use = (uint32_t)(tc >> 1);
-      if (__any_sync(0xffffffffu, !mbar_wait(&acc_empty[b], (use & 1u) ^ 1u))) {
+      if (__any_sync(0xffffffffu, !mbar_wait_poll(&acc_empty[b], (use & 1u) ^ 1u))) {
         ok = false;
         break;
       }
@@ -242,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
       for (int ks = 0; ks < n_ksteps; ++ks, ++it) {
         const int s = it % kStages;
         const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-        if (__any_sync(0xffffffffu, !mbar_wait(&a_full[s], ph) || !mbar_wait(&b_full[s], ph) || abort_flag)) {
+        if (__any_sync(0xffffffffu, !mbar_wait_poll(&a_full[s], ph) || !mbar_wait_poll(&b_full[s], ph) || abort_flag)) {
           ok = false;
           break;
         }
@@ -279,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
       for (int ks = 0; ks < n_ksteps; ++ks, ++it) {
         const int s = it % kStages, rs = it % kRawStages;
         const uint32_t ph = (uint32_t)(it / kStages) & 1u, rph = (uint32_t)(it / kRawStages) & 1u;
-        if (__any_sync(0xffffffffu, !mbar_wait(&raw_full[rs], rph) || !mbar_wait(&empty_bar[s], ph ^ 1u) ||
+        if (__any_sync(0xffffffffu, !mbar_wait_poll(&raw_full[rs], rph) || !mbar_wait_poll(&empty_bar[s], ph ^ 1u) ||
                                         abort_flag)) {
           ok = false;
           break;
@@ -344,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
       const int e = find_expert(s_toff, E, mt >> 1);
       const int row = mt * kTileM + q * 32 + lane;
       const float rs = p.row_scale ? p.row_scale[row] : 1.f;
-      if (__any_sync(0xffffffffu, !mbar_wait(&acc_full[b], use & 1u) || abort_flag)) {
+      if (__any_sync(0xffffffffu, !mbar_wait_poll(&acc_full[b], use & 1u) || abort_flag)) {
         if (lane == 0) {
           set_status(p.status, kDevErrTimeout);
           abort_flag = 1;
