@@ -179,3 +179,29 @@ def test_unpermute_entry_points_validate_before_launch():
     assert lib.moe_unpermute_combine(C.byref(cfg), 0x1000, 4, C.byref(plan), 0x2000, 0x3008, 0x4000, None) == 1
     assert "shared" in lib.moe_last_error().decode()
     assert lib.moe_unpermute_combine(C.byref(cfg), None, 0, None, None, None, None, None) == 0
+
+
+def test_decode_workspace_holds_the_grouped_gemm_buffers_from_nine_tokens():
+    """Decode batches of 9 or more tokens run on the grouped W4A16 GEMM when
+    the workspace holds its buffers: moe_workspace_size sizes them (x as f16
+    rows of the padded tile layout, h as f16 padded rows), and a workspace of
+    that size lays them out behind the decode's own (host arithmetic only)."""
+    lib = capi.lib()
+    cfg = _cfg()                                   # E = 16, k = 4, H = 256, I = 128
+    c = cfg.c()
+    w8 = lib.moe_workspace_size(C.byref(c), 8, 0)
+    w9 = lib.moe_workspace_size(C.byref(c), 9, 0)
+    P9 = lib.moe_padded_rows(C.byref(c), 9)
+    assert P9 % 256 == 0 and P9 >= 9 * 4
+    # the gathered f16 x rows alone take P * H * 2 bytes
+    assert w9 > w8 + P9 * 256 * 2
+    # a shape the grouped GEMM does not take keeps the plain layout
+    odd = _cfg(intermediate=96, shared_intermediate=96).c()
+    assert lib.moe_workspace_size(C.byref(odd), 9, 0) < lib.moe_workspace_size(C.byref(c), 9, 0)
+    base = 0x1000000
+    v = capi.MoeViews()
+    assert lib.moe_workspace_views(C.byref(c), 9, 0, base, w9, C.byref(v)) == 0
+    # h (f16 padded rows, at least 4 bytes per assignment element) ends before r
+    assert v.r - v.h >= max(2 * P9, 4 * 36) * 128
+    # r stays [T*k, H] fp32 in assignment order on both forms
+    assert v.shared - v.r >= 4 * 36 * 256
