@@ -89,6 +89,7 @@ __global__ void __launch_bounds__(1024) permute_scan(int nb, int E, int lb, int 
       }
 #pragma unroll
       for (int i = 0; i < kPer; ++i) {
+        if (b0 + 32 * i >= nb) break;   // warp-uniform: the rest of the pass is past the blocks
         int inc = v[i];
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {

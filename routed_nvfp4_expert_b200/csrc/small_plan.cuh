@@ -6,12 +6,17 @@
 // top-k + plan kernel of the decode path.
 #pragma once
 
+#include <climits>
+
 #include "common.cuh"
 
 namespace rnx {
 
-constexpr int kSmallMaxA = 1024;
+constexpr int kSmallMaxA = 1024;   // a power of two (the bitonic sort below)
 constexpr int kMaxE = 1024;
+// up to this many assignments the stable rank is a count over the earlier
+// ones (A steps per thread); above, a bitonic sort (log2^2 kSmallMaxA / 2 steps)
+constexpr int kSmallRankA = 256;
 
 // Block-wide exclusive scan of up to blockDim.x (multiple of 32, <= 1024)
 // values, one per thread; returns the exclusive prefix, *total gets the sum.
@@ -108,6 +113,45 @@ RNX_DEVICE void small_plan(const int32_t* ids, int A, int E, int lb, int le, con
   __syncthreads();
   finish_plan(s_cnt, E, lb, le, plan, s_warp, s_off, s_act);
   __syncthreads();
+  if (A > kSmallRankA) {
+    // stable order by expert: a bitonic sort of the keys e * kSmallMaxA + a
+    // (ids out of range and the slots past A sort last), one key per thread
+    // (the CTA has kSmallMaxA threads); the k-th key is the assignment at
+    // position k, offset + rank
+    for (int i = threadIdx.x; i < kSmallMaxA; i += blockDim.x) {
+      const int e = i < A ? s_ids[i] : -1;
+      s_sorted[i] = e >= 0 ? e * kSmallMaxA + i : INT_MAX;
+    }
+    for (int kk = 2; kk <= kSmallMaxA; kk <<= 1)
+      for (int j = kk >> 1; j > 0; j >>= 1) {
+        __syncthreads();
+        for (int i = threadIdx.x; i < kSmallMaxA; i += blockDim.x) {
+          const int ixj = i ^ j;
+          if (ixj > i) {
+            const int x = s_sorted[i], y = s_sorted[ixj];
+            if ((x > y) == ((i & kk) == 0)) {
+              s_sorted[i] = y;
+              s_sorted[ixj] = x;
+            }
+          }
+        }
+      }
+    __syncthreads();
+    for (int pos = threadIdx.x; pos < A; pos += blockDim.x) {
+      const int key = s_sorted[pos];
+      if (key != INT_MAX) {
+        const int a = key & (kSmallMaxA - 1);
+        plan.sorted[pos] = a;
+        plan.inv[a] = pos;
+        s_sorted[pos] = a;
+      }
+    }
+    for (int a = threadIdx.x; a < A; a += blockDim.x)
+      if (s_ids[a] < 0) plan.inv[a] = -1;
+    __syncthreads();
+    write_first(plan, s_off, s_act, s_sorted);
+    return;
+  }
   // stable position: offset + number of earlier assignments of the same expert
   for (int a0 = 0; a0 < A; a0 += blockDim.x) {
     const int a = a0 + threadIdx.x;
