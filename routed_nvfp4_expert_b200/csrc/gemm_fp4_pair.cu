@@ -26,12 +26,13 @@
 //            shared memory (the unpermute is fused into the combine that
 //            follows, which sums them in fp32).
 //
-// Warp roles per CTA: warp 0 = TMA producer (ring of 38 KB stages, 5 deep for
-// GATE_UP and 4 for DOWN; completions counted on the even CTA's barrier), warp 1 = MMA issuer (even
-// CTA only, one thread), warp 2 = TMEM allocator (both CTAs), warps 4-11 =
-// epilogue (warp w reads TMEM lane quadrant w % 4 and one half of the 256
-// accumulator columns, copies them to registers and releases the accumulator
-// before the SwiGLU / scaling and the stores). Every wait is bounded; a
+// Warp roles per CTA: warp 0 = TMA producer (ring of 38 KB stages, 5 deep
+// for GATE_UP and 4 for DOWN; completions counted on the even CTA's
+// barrier), warp 1 = MMA issuer (even CTA only, one thread), warp 2 = TMEM
+// allocator (both CTAs), warps 4-11 = epilogue (warp w reads TMEM lane
+// quadrant w % 4 and one half of the 256 accumulator columns, copies them to
+// registers and releases the accumulator with a CTA-scope arrive before the
+// SwiGLU / scaling and the stores). Every wait is bounded; a
 // timeout sets the device status word and winds the pair down. No TMA load
 // uses cluster multicast (only the MMA completion commit is multicast).
 
