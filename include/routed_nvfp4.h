@@ -172,7 +172,13 @@ typedef struct {
 
 /* Bytes of workspace moe_forward needs for T tokens on `path` (0 on invalid
  * arguments; moe_last_error() says why). The same workspace also serves every
- * single-step entry point that takes one. Contents need no initialisation. */
+ * single-step entry point that takes one. Contents need no initialisation.
+ * MOE_PATH_DECODE with T >= 9 (I % 128 == 0, H % 256 == 0) includes the
+ * grouped W4A16 GEMM's buffers in the padded tile layout (x as f16 [P, H],
+ * h as f16 [P, I], P = moe_padded_rows(cfg, T)): about 0.68 GB at T = 32 and
+ * 0.77 GB at T = 64 for H = 4096, I = 1024, E = 288, k = 8. A decode
+ * workspace smaller than that but large enough for the plain decode layout
+ * is accepted, and the forward then runs the GEMV form (nvfp4_expert_gemv). */
 size_t moe_workspace_size(const moe_config_t* cfg, int32_t T, int32_t path);
 
 /* Bytes of the routing plan arrays for T tokens (one buffer, carved by
